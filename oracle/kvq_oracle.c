@@ -1,0 +1,426 @@
+/*
+ * kvq_oracle.c -- plain, slow CPU oracle for layer-wise mixed-precision KV-cache
+ * quantization and single-token decode attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the package smoke check and the
+ * CPU-baseline leg of the benchmark may load this library.  It shares no code,
+ * header, table or helper with the CUDA library; the only thing both sides agree
+ * on is the storage format, which is written out as a specification below and
+ * implemented here independently.
+ *
+ * Sources (web pages on the subject; cited by page title and section):
+ *  [KVT]  "KVTuner: Sensitivity-Aware Layer-Wise Mixed-Precision KV Cache
+ *          Quantization ..." (atlas.scime.ai summary) -- Approach; Measured effects
+ *          table; Limitations (KIVI kernel, HF transformers).
+ *  [MIX]  "Mixed-precision KV-cache quantization per-layer sensitivity"
+ *          (llms-explorer) -- Facts: per-layer K/V precision pairs, per-channel
+ *          asymmetric keys vs per-token asymmetric.
+ *  [TRI]  "TriAxialKV per-role mixed-precision KV quantization for agentic
+ *          prefills" (llms-explorer) -- Facts: asymmetric groupwise quantizer with
+ *          group size 32; INT2 per-channel keys, per-token values; leftover INT2
+ *          keys routed through the INT4 per-token path; INT2/INT4 page pools;
+ *          bitwidth-homogeneous flash-decoding splits merged by log-sum-exp.
+ *
+ * Precision: every quantizer step is one correctly rounded IEEE binary32
+ * operation (x86-64 SSE arithmetic, built with -ffp-contract=off, no fast-math);
+ * dequantisation and attention are binary64.
+ *
+ * ---------------------------------------------------------------------------
+ * Q1  Group quantizer ([TRI] Facts: asymmetric, groupwise, g = 32; [MIX] Facts:
+ *     asymmetric keys per channel, values per token).  For 32 inputs x_i and
+ *     bits b in {2,4,8}:
+ *        mn = min x_i, mx = max x_i
+ *        s32 = (mx - mn) / (2^b - 1)            binary32 subtract, then divide
+ *        s16 = fp16_rne(s32), z16 = fp16_rne(mn) stored scale and zero
+ *        s = float(s16), z = float(z16)
+ *        code_i = 0 if s == 0, else clamp(rne((x_i - z) / s), 0, 2^b - 1)
+ *        dequant  x^_i = code_i * s + z          (binary64 here)
+ *     Reading: the divisor in the code formula is the stored fp16 scale (the
+ *     value the decoder multiplies by), and the zero is the fp16 group minimum.
+ *
+ * Q2  Grouping axes.  Keys in per-channel mode: 32 consecutive tokens of one
+ *     channel; the L mod 32 newest tokens are not quantized and stay in a bf16
+ *     residual.  Values, and keys in per-token mode: 32 consecutive channels of
+ *     one token.
+ *
+ * Q3  Storage format (version 1).  The pages fix no layout; this one is chosen so
+ *     that a decoder thread's tensor-core operand fragments are contiguous.
+ *     Per (batch b, kv head h) the cache is a sequence of 32-token block records.
+ *     Record of block beta (tokens 32*beta .. 32*beta+31), D = head_dim, nj = D/32:
+ *        [K codes: 4*D*bk bytes][K s/z: 4*D bytes][V codes: 4*D*bv][V s/z: 4*D]
+ *     s/z entries are (scale fp16, zero fp16) pairs, 4 bytes:
+ *        per-channel K: entry d (channel) at 4*d
+ *        per-token K and V: entry (u, j) at 4*(u*nj + j), u = token in block,
+ *                           j = channel group d/32
+ *     Code areas are two 16-token halves of 2*D*b bytes each.  Token u of the
+ *     block lies in half eta = u/16.  Inside a half, every code belongs to one of
+ *     32 "lanes" and one half-word "slot" of that lane:
+ *        K (role: key operand), token u, channel d:
+ *           i = (u%16)/8, gk = u%8, k = d/16, e = d%16,
+ *           t = (e%8)/2, r = e/8, hb = e%2,
+ *           lane = 4*gk + t, slot = (2*k + i)*2 + r
+ *        V (role: value operand), token u, channel d:
+ *           e = u%16, t = (e%8)/2, ch = e/8, hb = e%2,
+ *           m = d/16, rho = d%16, g = rho%8, rh = rho/8,
+ *           lane = 4*g + t, slot = 4*m + 2*ch + rh
+ *     Each lane owns Wh = D*b/64 little-endian 32-bit words per half, holding
+ *     F = 32/b fields of b bits, LSB first.  A word carries P = F/2 slots: slot
+ *     p of the word uses field p for hb = 0 and field p + P for hb = 1.  So a
+ *     code sits in lane word w = slot / P at field (slot % P) + hb*P, bit
+ *     offset field*b.  Lane words are stored in chunks of c = min(4, Wh) words:
+ *        word index in half = ((w / c)*32 + lane)*c + (w % c).
+ *     Residual (per-channel K): 32 tokens x D bf16, entry (u, d) at 2*(u*D + d).
+ *     Canonical image of a (b, h) unit holding L tokens: records 0..ceil(L/32)-1,
+ *     then (per-channel K only) the residual; every byte that holds no token of
+ *     0..L-1 is zero (the unfilled part of the last block and of the residual).
+ *
+ * Q4  Attention (fp64): O[hq] = sum_t softmax_t(q . k^_t / sqrt(D)) v^_t over all L
+ *     cached tokens, quantized ones and residual alike, no mask; GQA: the kv head
+ *     of query head hq is hq / G.
+ * ---------------------------------------------------------------------------
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_PER_CHANNEL 0
+#define ORC_PER_TOKEN 1
+
+/* ---------------- number formats (IEEE 754 definitions) ---------------- */
+
+/* bf16 bit pattern -> binary32: the bf16 pattern is the top half of a binary32. */
+static float orc_bf16_to_f32(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* binary16 bit pattern -> binary64, from the encoding definition. */
+static double orc_f16_to_f64(uint16_t h) {
+    int s = h >> 15, e = (h >> 10) & 31, m = h & 1023;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);                 /* subnormal: m * 2^-24 */
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + m), e - 25);     /* (1 + m/1024) * 2^(e-15) */
+    return s ? -v : v;
+}
+
+/* binary32 -> binary16, round to nearest, ties to even. */
+static uint16_t orc_f32_to_f16(float f) {
+    if (isnan(f)) return 0x7E00;
+    uint16_t sign = signbit(f) ? 0x8000 : 0;
+    double v = fabs((double)f);
+    if (v >= 65520.0) return sign | 0x7C00;        /* halfway above 65504 rounds to inf */
+    if (v < ldexp(1.0, -14)) {                     /* result grid: multiples of 2^-24 */
+        double n = rint(ldexp(v, 24));             /* exact scaling; rint is RNE */
+        return sign | (uint16_t)n;                 /* n == 1024 encodes the min normal */
+    }
+    int ex;
+    frexp(v, &ex);                                  /* v = f * 2^ex, f in [0.5, 1) */
+    int E = ex - 1;                                 /* 2^E <= v < 2^(E+1) */
+    double n = rint(ldexp(v, 10 - E));              /* significand * 1024, in [1024, 2048] */
+    if (n == 2048.0) { n = 1024.0; E += 1; }
+    if (E > 15) return sign | 0x7C00;
+    return sign | (uint16_t)(((E + 15) << 10) | ((int)n - 1024));
+}
+
+/* ---------------- Q1: group quantizer ---------------- */
+
+/* Quantize n values x[i*xs] (binary32) with b bits; writes scale/zero (fp16 bits)
+ * and codes[i*cs]. */
+static void orc_quant(const float *x, int n, int xs, int bits, uint16_t *s16, uint16_t *z16,
+                      uint8_t *codes, int cs) {
+    float mn = x[0], mx = x[0];
+    for (int i = 1; i < n; i++) {
+        float v = x[i * xs];
+        if (v < mn) mn = v;
+        if (v > mx) mx = v;
+    }
+    float qmax = (float)((1 << bits) - 1);
+    float range = mx - mn;                          /* binary32, correctly rounded */
+    float s32 = range / qmax;                       /* binary32 IEEE division */
+    *s16 = orc_f32_to_f16(s32);
+    *z16 = orc_f32_to_f16(mn);
+    float s = (float)orc_f16_to_f64(*s16);
+    float z = (float)orc_f16_to_f64(*z16);
+    for (int i = 0; i < n; i++) {
+        uint8_t c = 0;
+        if (s != 0.0f) {
+            float diff = x[i * xs] - z;
+            float qv = diff / s;
+            float r = rintf(qv);                    /* default rounding mode: ties to even */
+            if (r < 0.0f) r = 0.0f;
+            if (r > qmax) r = qmax;
+            c = (uint8_t)r;
+        }
+        codes[i * cs] = c;
+    }
+}
+
+/* ---------------- Q3: storage format ---------------- */
+
+long orc_record_bytes(int D, int bk, int bv) { return 4L * D * (bk + bv) + 8L * D; }
+
+long orc_unit_image_bytes(int L, int D, int bk, int bv, int kmode) {
+    long nblk = (L + 31) / 32;
+    long r = nblk * orc_record_bytes(D, bk, bv);
+    if (kmode == ORC_PER_CHANNEL) r += 64L * D;    /* residual: 32 tokens x D bf16 */
+    return r;
+}
+
+/* Byte offset (inside a code area of one block) and bit offset of the code of
+ * token u (0..31), channel d, for role 0 = key operand, 1 = value operand. */
+static void orc_code_pos(int role, int u, int d, int D, int bits, long *byte_off, int *bit_off) {
+    int eta = u / 16, lane, slot, hb;
+    if (role == 0) {
+        int i = (u % 16) / 8, gk = u % 8, k = d / 16, e = d % 16;
+        int t = (e % 8) / 2, r = e / 8;
+        hb = e % 2;
+        lane = 4 * gk + t;
+        slot = (2 * k + i) * 2 + r;
+    } else {
+        int e = u % 16, t = (e % 8) / 2, ch = e / 8;
+        int m = d / 16, rho = d % 16, g = rho % 8, rh = rho / 8;
+        hb = e % 2;
+        lane = 4 * g + t;
+        slot = 4 * m + 2 * ch + rh;
+    }
+    int F = 32 / bits, P = F / 2;
+    int Wh = D * bits / 64;
+    int c = Wh < 4 ? Wh : 4;
+    int w = slot / P;
+    int field = slot % P + hb * P;
+    long word = ((long)(w / c) * 32 + lane) * c + (w % c);
+    *byte_off = (long)eta * (2L * D * bits) + 4 * word;
+    *bit_off = field * bits;
+}
+
+static void orc_put_code(uint8_t *area, int role, int u, int d, int D, int bits, unsigned code) {
+    long bo;
+    int bit;
+    orc_code_pos(role, u, d, D, bits, &bo, &bit);
+    uint32_t w;
+    memcpy(&w, area + bo, 4);
+    uint32_t mask = ((1u << bits) - 1u) << bit;
+    w = (w & ~mask) | ((code << bit) & mask);
+    memcpy(area + bo, &w, 4);
+}
+
+/* Position of the code of (u, d) inside a code area (exported for tests). */
+void orc_code_position(int role, int u, int d, int D, int bits, long *byte_off, int *bit_off) {
+    orc_code_pos(role, u, d, D, bits, byte_off, bit_off);
+}
+
+/* Read back the code of (u, d) from a code area (used by tests to decode images). */
+unsigned orc_get_code(const uint8_t *area, int role, int u, int d, int D, int bits) {
+    long bo;
+    int bit;
+    orc_code_pos(role, u, d, D, bits, &bo, &bit);
+    uint32_t w;
+    memcpy(&w, area + bo, 4);
+    return (w >> bit) & ((1u << bits) - 1u);
+}
+
+static void put_sz(uint8_t *p, uint16_t s, uint16_t z) {
+    memcpy(p, &s, 2);
+    memcpy(p + 2, &z, 2);
+}
+
+/* ---------------- one (batch, kv-head) unit ---------------- */
+
+/* Quantize one unit's K and V (bf16 bits, [L][D]) and, if img != NULL, write its
+ * canonical image; if Kh/Vh != NULL, write the dequantized cache [L][D] (fp64;
+ * residual keys are the bf16 inputs themselves). */
+int orc_unit(const uint16_t *K, const uint16_t *V, int L, int D, int bk, int bv, int kmode,
+             uint8_t *img, double *Kh, double *Vh) {
+    if (D % 32 || D <= 0 || L < 0) return -1;
+    const int nj = D / 32;
+    const long REC = orc_record_bytes(D, bk, bv);
+    const long KC = 4L * D * bk, KS = 4L * D, VC = 4L * D * bv;
+    const int nblk = (L + 31) / 32;
+    const int nfull = L / 32;                       /* complete per-channel key groups */
+    if (img) memset(img, 0, (size_t)orc_unit_image_bytes(L, D, bk, bv, kmode));
+
+    float x[32];
+    uint8_t c[32];
+    uint16_t s16, z16;
+
+    /* values: per token, groups of 32 channels */
+    for (int tok = 0; tok < L; tok++) {
+        int blk = tok / 32, u = tok % 32;
+        for (int j = 0; j < nj; j++) {
+            for (int i = 0; i < 32; i++) x[i] = orc_bf16_to_f32(V[(long)tok * D + 32 * j + i]);
+            orc_quant(x, 32, 1, bv, &s16, &z16, c, 1);
+            if (img) {
+                uint8_t *rec = img + blk * REC;
+                put_sz(rec + KC + KS + VC + 4L * (u * nj + j), s16, z16);
+                for (int i = 0; i < 32; i++) orc_put_code(rec + KC + KS, 1, u, 32 * j + i, D, bv, c[i]);
+            }
+            if (Vh) {
+                double s = orc_f16_to_f64(s16), z = orc_f16_to_f64(z16);
+                for (int i = 0; i < 32; i++) Vh[(long)tok * D + 32 * j + i] = c[i] * s + z;
+            }
+        }
+    }
+
+    if (kmode == ORC_PER_CHANNEL) {
+        /* keys: per channel over each complete group of 32 tokens */
+        for (int blk = 0; blk < nfull; blk++) {
+            for (int d = 0; d < D; d++) {
+                for (int i = 0; i < 32; i++) x[i] = orc_bf16_to_f32(K[(long)(32 * blk + i) * D + d]);
+                orc_quant(x, 32, 1, bk, &s16, &z16, c, 1);
+                if (img) {
+                    uint8_t *rec = img + blk * REC;
+                    put_sz(rec + KC + 4L * d, s16, z16);
+                    for (int i = 0; i < 32; i++) orc_put_code(rec, 0, i, d, D, bk, c[i]);
+                }
+                if (Kh) {
+                    double s = orc_f16_to_f64(s16), z = orc_f16_to_f64(z16);
+                    for (int i = 0; i < 32; i++) Kh[(long)(32 * blk + i) * D + d] = c[i] * s + z;
+                }
+            }
+        }
+        /* the newest L mod 32 tokens stay in the bf16 residual */
+        for (int tok = 32 * nfull; tok < L; tok++) {
+            int u = tok - 32 * nfull;
+            if (img) memcpy(img + nblk * REC + 2L * u * D, K + (long)tok * D, 2L * D);
+            if (Kh)
+                for (int d = 0; d < D; d++) Kh[(long)tok * D + d] = orc_bf16_to_f32(K[(long)tok * D + d]);
+        }
+    } else {
+        /* keys per token, groups of 32 channels, like values */
+        for (int tok = 0; tok < L; tok++) {
+            int blk = tok / 32, u = tok % 32;
+            for (int j = 0; j < nj; j++) {
+                for (int i = 0; i < 32; i++) x[i] = orc_bf16_to_f32(K[(long)tok * D + 32 * j + i]);
+                orc_quant(x, 32, 1, bk, &s16, &z16, c, 1);
+                if (img) {
+                    uint8_t *rec = img + blk * REC;
+                    put_sz(rec + KC + 4L * (u * nj + j), s16, z16);
+                    for (int i = 0; i < 32; i++) orc_put_code(rec, 0, u, 32 * j + i, D, bk, c[i]);
+                }
+                if (Kh) {
+                    double s = orc_f16_to_f64(s16), z = orc_f16_to_f64(z16);
+                    for (int i = 0; i < 32; i++) Kh[(long)tok * D + 32 * j + i] = c[i] * s + z;
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+/* ---------------- Q4: attention in binary64 ---------------- */
+
+/* Unnormalised attention of G query heads (q: [G][D] bf16 bits) over tokens
+ * [t0, t1) of a dequantized cache: m = max score, l = sum exp(score - m),
+ * acc[g][d] = sum exp(score - m) * v^[d].  Scores are q.k^/sqrt(D). */
+void orc_attention_partial(const uint16_t *q, const double *Kh, const double *Vh, int t0, int t1,
+                           int D, int G, double *m, double *l, double *acc) {
+    const double scale = 1.0 / sqrt((double)D);
+    double *sc = (double *)malloc(sizeof(double) * (size_t)(t1 > t0 ? t1 - t0 : 1));
+    for (int g = 0; g < G; g++) {
+        double mx = -INFINITY;
+        for (int t = t0; t < t1; t++) {
+            double s = 0.0;
+            for (int d = 0; d < D; d++) s += (double)orc_bf16_to_f32(q[g * D + d]) * Kh[(long)t * D + d];
+            s *= scale;
+            sc[t - t0] = s;
+            if (s > mx) mx = s;
+        }
+        double sum = 0.0;
+        for (int d = 0; d < D; d++) acc[g * D + d] = 0.0;
+        for (int t = t0; t < t1; t++) {
+            double p = exp(sc[t - t0] - mx);
+            sum += p;
+            for (int d = 0; d < D; d++) acc[g * D + d] += p * Vh[(long)t * D + d];
+        }
+        m[g] = mx;
+        l[g] = sum;
+    }
+    free(sc);
+}
+
+/* Log-sum-exp merge of S partials ([S][G], [S][G], [S][G][D]) into out [G][D]
+ * ([TRI] Facts: splits merged by online log-sum-exp). */
+void orc_merge_partials(int S, int G, int D, const double *m, const double *l, const double *acc,
+                        double *out) {
+    for (int g = 0; g < G; g++) {
+        double M = -INFINITY;
+        for (int s = 0; s < S; s++)
+            if (m[s * G + g] > M) M = m[s * G + g];
+        double den = 0.0;
+        for (int d = 0; d < D; d++) out[g * D + d] = 0.0;
+        for (int s = 0; s < S; s++) {
+            if (m[s * G + g] == -INFINITY) continue;   /* empty partial */
+            double w = exp(m[s * G + g] - M);
+            den += w * l[s * G + g];
+            for (int d = 0; d < D; d++) out[g * D + d] += w * acc[((long)s * G + g) * D + d];
+        }
+        for (int d = 0; d < D; d++) out[g * D + d] /= den;
+    }
+}
+
+/* Softmax attention over all L tokens: out [G][D]. */
+void orc_attention(const uint16_t *q, const double *Kh, const double *Vh, int L, int D, int G,
+                   double *out) {
+    double *m = (double *)malloc(sizeof(double) * G);
+    double *l = (double *)malloc(sizeof(double) * G);
+    double *acc = (double *)malloc(sizeof(double) * (size_t)G * D);
+    orc_attention_partial(q, Kh, Vh, 0, L, D, G, m, l, acc);
+    orc_merge_partials(1, G, D, m, l, acc, out);
+    free(m);
+    free(l);
+    free(acc);
+}
+
+/* ---------------- a whole layer ---------------- */
+
+/* K, V: [B][Hkv][L][D] bf16 bits; Q: [B][Hkv*G][D] bf16 bits (query head hq uses
+ * kv head hq / G).  img (nullable): unit images concatenated in (b, h) order.
+ * out (nullable): [B][Hkv*G][D] binary64.  Units run in parallel (OpenMP). */
+int orc_layer(const uint16_t *K, const uint16_t *V, const uint16_t *Q, int B, int Hkv, int G, int L,
+              int D, int bk, int bv, int kmode, uint8_t *img, double *out) {
+    if (L < 1 && out) return -1;
+    const long unit_img = orc_unit_image_bytes(L, D, bk, bv, kmode);
+    const int units = B * Hkv;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+    for (int un = 0; un < units; un++) {
+        int b = un / Hkv, h = un % Hkv;
+        const uint16_t *Ku = K + (long)un * L * D;
+        const uint16_t *Vu = V + (long)un * L * D;
+        double *Kh = NULL, *Vh = NULL;
+        if (out) {
+            Kh = (double *)malloc(sizeof(double) * (size_t)L * D);
+            Vh = (double *)malloc(sizeof(double) * (size_t)L * D);
+        }
+        err |= orc_unit(Ku, Vu, L, D, bk, bv, kmode, img ? img + un * unit_img : NULL, Kh, Vh) != 0;
+        if (out) {
+            orc_attention(Q + ((long)b * Hkv * G + (long)h * G) * D, Kh, Vh, L, D, G,
+                          out + ((long)b * Hkv * G + (long)h * G) * D);
+            free(Kh);
+            free(Vh);
+        }
+    }
+    return err ? -1 : 0;
+}
+
+/* ---------------- exported scalar helpers (for pins) ---------------- */
+
+void orc_f32_to_f16_array(const float *x, uint16_t *out, long n) {
+    for (long i = 0; i < n; i++) out[i] = orc_f32_to_f16(x[i]);
+}
+void orc_f16_to_f64_array(const uint16_t *h, double *out, long n) {
+    for (long i = 0; i < n; i++) out[i] = orc_f16_to_f64(h[i]);
+}
+/* Quantize many groups: x [ngroups][32] binary32 -> s16, z16 [ngroups], codes [ngroups][32]. */
+void orc_quant_groups(const float *x, long ngroups, int bits, uint16_t *s16, uint16_t *z16,
+                      uint8_t *codes) {
+    for (long g = 0; g < ngroups; g++) orc_quant(x + g * 32, 32, 1, bits, s16 + g, z16 + g, codes + g * 32, 1);
+}
+int orc_format_version(void) { return 1; }
