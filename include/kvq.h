@@ -1,0 +1,167 @@
+/*
+ * kvq.h -- C ABI of the layer-wise mixed-precision KV-cache library for B200 (sm_100a).
+ *
+ * What the library computes (cited by page title and section):
+ *  - A static per-layer key/value precision pair {bk, bv} (e.g. K8V4, K4V2), chosen
+ *    offline and applied at inference with no online decision
+ *    ("KVTuner: Sensitivity-Aware Layer-Wise Mixed-Precision KV Cache Quantization",
+ *    atlas.scime.ai summary: Approach; "Mixed-precision KV-cache quantization
+ *    per-layer sensitivity", Facts).
+ *  - Asymmetric groupwise quantization with group size 32: keys per channel (KIVI
+ *    style, groups of 32 consecutive tokens of one channel) or per token, values per
+ *    token (groups of 32 consecutive channels) ("TriAxialKV per-role mixed-precision
+ *    KV quantization", Facts: quantizer; per-layer sensitivity Facts: per-channel
+ *    asymmetric keys).  For a group x_0..x_31 and b bits:
+ *        s = fp16_rne(fp32((max - min) / (2^b - 1))), z = fp16_rne(min),
+ *        code_i = clamp(rne(fp32((x_i - float(z)) / float(s))), 0, 2^b - 1)  (0 if s = 0)
+ *    every step a single correctly rounded binary32 operation (no FMA contraction);
+ *    dequant x^ = code * s + z.
+ *  - Keys in per-channel mode: the newest L mod 32 tokens that do not fill a group
+ *    stay unquantized in a bf16 residual (TriAxialKV Facts mention KIVI's
+ *    full-precision residual buffer).
+ *  - Single-token decode attention over the packed cache, dequantizing in
+ *    registers, split over the sequence into flash-decoding partials merged by
+ *    log-sum-exp (TriAxialKV Facts: bitwidth-homogeneous splits merged by online
+ *    log-sum-exp).  out[b, hq] = sum_t softmax_t(q . k^_t / sqrt(D)) v^_t over all L
+ *    cached tokens; query head hq uses kv head hq / G, G = n_q_heads / n_kv_heads.
+ *
+ * Storage format v1 (the pages fix none; chosen so that each decoder thread's tensor
+ * core operand fragments are contiguous).  Per layer, per (batch b, kv head h):
+ * capacity ceil(max_ctx/32) block records of 32 tokens, then (per-channel keys) a
+ * residual of 32 x D bf16.  Record of block beta, D = head_dim, nj = D/32:
+ *     [K codes 4*D*bk B][K s/z 4*D B][V codes 4*D*bv B][V s/z 4*D B]
+ *   s/z entry = (scale fp16, zero fp16); per-channel K: entry d at 4*d; per-token K
+ *   and V: entry (u, j) at 4*(u*nj + j) (u = token in block, j = d/32).
+ *   Code areas = two 16-token halves of 2*D*b bytes; token u in half u/16; in the half
+ *   each code has a lane (0..31) and a slot:
+ *     keys:   i=(u%16)/8, gk=u%8, k=d/16, e=d%16, t=(e%8)/2, r=e/8, hb=e%2,
+ *             lane=4*gk+t, slot=(2k+i)*2+r
+ *     values: e=u%16, t=(e%8)/2, ch=e/8, hb=e%2, m=d/16, rho=d%16, g=rho%8, rh=rho/8,
+ *             lane=4*g+t, slot=4m+2ch+rh
+ *   A lane has Wh = D*b/64 little-endian 32-bit words per half, F = 32/b fields of b
+ *   bits each (LSB first), P = F/2 slots per word: the code sits in lane word
+ *   slot/P, field slot%P + hb*P.  Lane words are stored in chunks of c = min(4, Wh):
+ *   word index in half = ((w/c)*32 + lane)*c + w%c.
+ *
+ * Conventions for every entry point:
+ *  - Return value: a kvq_status (0 = success).  Arguments are checked on the host
+ *    before any launch; on failure nothing is launched and kvq_last_error() returns
+ *    a message (thread-local, valid until the next call on that thread).
+ *  - Device pointers are plain CUDA global-memory pointers owned by the caller; the
+ *    library never allocates device memory.  `stream` is a cudaStream_t (NULL = the
+ *    legacy default stream); calls that take one are asynchronous on it.
+ *  - K/V/q/out pointers must be 16-byte aligned; the workspace 256-byte aligned.
+ *  - All sequences in the batch have the same length (the library tracks one L per
+ *    layer).  A handle is not thread-safe: serialize calls on one handle.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KVQ_OK = 0,
+    KVQ_EINVAL = -1,        /* bad argument (null pointer, layer index, sizes)   */
+    KVQ_EUNSUPPORTED = -2,  /* valid but not supported by this build (e.g. D)    */
+    KVQ_ECAPACITY = -3,     /* append would exceed max_ctx / a page pool         */
+    KVQ_EUNBOUND = -4,      /* no workspace bound, or workspace too small        */
+    KVQ_EALIGN = -5,        /* pointer alignment                                 */
+    KVQ_ECUDA = -6,         /* a CUDA runtime call or launch failed              */
+    KVQ_EDEVICE = -7        /* a kernel reported an error through the status word */
+} kvq_status;
+
+typedef enum { KVQ_PER_CHANNEL = 0, KVQ_PER_TOKEN = 1 } kvq_mode;
+
+/* One layer's precision pair.  bk, bv in {2, 4, 8}; vmode must be KVQ_PER_TOKEN. */
+typedef struct {
+    int bk, bv;
+    int kmode;   /* kvq_mode for keys   */
+    int vmode;   /* kvq_mode for values */
+} kvq_layer_cfg;
+
+typedef struct {
+    int num_layers;
+    int batch;
+    int n_kv_heads;
+    int n_q_heads;      /* multiple of n_kv_heads; G = n_q_heads / n_kv_heads <= 8 */
+    int head_dim;       /* 64 or 128 */
+    int group;          /* must be 32 */
+    int max_ctx;        /* token capacity per sequence and layer */
+    const kvq_layer_cfg *layers;   /* num_layers entries, copied by kvq_plan */
+    int paged;          /* 0: per-layer maps (this header's format); 1: INT2/INT4 paged */
+    int page_tokens;    /* paged: 16 */
+    float avg_bits;     /* paged: expected mean bits of the tag mask (sizes the pools) */
+} kvq_plan_desc;
+
+typedef struct kvq_handle kvq_handle;
+
+/* Validate a plan and create a host handle (host memory only). */
+KVQ_API int kvq_plan(const kvq_plan_desc *desc, kvq_handle **out);
+
+/* Device workspace size the plan needs: all layers' cache regions, the split
+ * partials and a status word. */
+KVQ_API int kvq_workspace_bytes(const kvq_handle *h, size_t *bytes);
+
+/* Bind caller-owned device memory (>= kvq_workspace_bytes, 256-byte aligned) and
+ * reset every layer to length 0.  No device work is issued. */
+KVQ_API int kvq_bind(kvq_handle *h, void *dev_ptr, size_t bytes);
+
+/* Append n_new tokens to every sequence of `layer`: K, V are bf16 [B][Hkv][n_new][D]
+ * (device).  Quantizes values per token, keys per channel (completing 32-token groups
+ * from residual + new tokens; the rest goes to the residual) or per token.  One kernel
+ * launch.  n_new >= 1; returns KVQ_ECAPACITY beyond max_ctx. */
+KVQ_API int kvq_append(kvq_handle *h, int layer, const void *K, const void *V, int n_new, void *stream);
+
+/* Decode attention of one query token per sequence over all L tokens of `layer`:
+ * q bf16 [B][Hq][D] (device); out [B][Hq][D] (device) bf16, or fp32 if out_fp32.
+ * Launches the split kernel and, when the sequence is split, the log-sum-exp merge
+ * kernel.  Requires L >= 1. */
+KVQ_API int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_fp32,
+                    void *stream);
+
+/* Force the number of sequence splits used by kvq_decode_attn (0 = automatic; the
+ * value is capped by the number of 32-token blocks and the partial buffer size). */
+KVQ_API int kvq_set_num_splits(kvq_handle *h, int num_splits);
+
+/* The split count kvq_decode_attn would use for `layer` at its current length. */
+KVQ_API int kvq_get_num_splits(const kvq_handle *h, int layer, int *num_splits);
+
+/* Copy one layer's cache to host memory in canonical order (parity checks): for each
+ * (b, h) the records 0..ceil(L/32)-1 then, for per-channel keys, the residual; bytes
+ * that hold no token of 0..L-1 are zero.  Synchronous (device-wide).  If host_buf is
+ * NULL or bytes is too small, only *needed is written (KVQ_EINVAL if too small). */
+KVQ_API int kvq_export_layer(const kvq_handle *h, int layer, void *host_buf, size_t bytes,
+                     size_t *needed);
+
+/* Current length L of `layer`. */
+KVQ_API int kvq_seq_len(const kvq_handle *h, int layer, int *L);
+
+/* Shorten `layer` to L tokens (host bookkeeping only).  L <= current length and
+ * L % 32 == 0 (so no token of a kept block is partially overwritten later). */
+KVQ_API int kvq_truncate(kvq_handle *h, int layer, int L);
+
+/* Read and clear the device status word (synchronizes `stream`).  KVQ_EDEVICE if a
+ * kernel reported a bounded wait that expired; *flags gets the raw bits. */
+KVQ_API int kvq_device_status(kvq_handle *h, void *stream, unsigned *flags);
+
+/* Free the handle (not the caller's workspace). */
+KVQ_API void kvq_destroy(kvq_handle *h);
+
+/* Message for the last failing call on this thread ("" if none). */
+KVQ_API const char *kvq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVQ_H */

@@ -1,0 +1,115 @@
+"""C-ABI library on the CPU: it loads, exports every symbol include/kvq.h declares, and
+its host-side checks reject bad plans and arguments before any CUDA call."""
+import ctypes
+
+import pytest
+
+from layer_wise_mixed_b200 import build as kbuild
+from layer_wise_mixed_b200 import kvq
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kvq.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = kvq.header_functions()
+    assert {"kvq_plan", "kvq_append", "kvq_decode_attn", "kvq_export_layer", "kvq_bind",
+            "kvq_workspace_bytes", "kvq_destroy", "kvq_last_error"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def desc(**kw):
+    a = dict(num_layers=2, batch=2, n_kv_heads=2, n_q_heads=4, head_dim=64, max_ctx=100,
+             layer_bits=[(4, 2), (8, 8)])
+    kmodes = kw.pop("kmodes", None)
+    a.update(kw)
+    return kvq.make_desc(a["num_layers"], a["batch"], a["n_kv_heads"], a["n_q_heads"], a["head_dim"],
+                         a["max_ctx"], a["layer_bits"], kmodes)
+
+
+def plan_rc(d):
+    h = ctypes.c_void_p()
+    rc = kvq.load().kvq_plan(ctypes.byref(d), ctypes.byref(h))
+    if rc == 0:
+        kvq.kvq_destroy(h.value)
+    return rc
+
+
+def test_plan_validation(lib):
+    assert plan_rc(desc()) == kvq.KVQ_OK
+    assert plan_rc(desc(layer_bits=[(3, 2), (8, 8)])) == kvq.KVQ_EINVAL
+    assert plan_rc(desc(layer_bits=[(4, 16), (8, 8)])) == kvq.KVQ_EINVAL
+    assert plan_rc(desc(n_q_heads=5)) == kvq.KVQ_EINVAL
+    assert plan_rc(desc(head_dim=96)) == kvq.KVQ_EUNSUPPORTED
+    assert plan_rc(desc(n_q_heads=18)) == kvq.KVQ_EUNSUPPORTED          # G = 9
+    assert plan_rc(desc(batch=0)) == kvq.KVQ_EINVAL
+    assert plan_rc(desc(kmodes=[1, 0])) == kvq.KVQ_OK
+    assert plan_rc(desc(kmodes=[1, 0], n_q_heads=6)) == kvq.KVQ_EUNSUPPORTED   # per-token keys, G = 3
+    d = desc()
+    d.group = 64
+    assert plan_rc(d) == kvq.KVQ_EUNSUPPORTED
+    d = desc()
+    d.layers[0].vmode = kvq.KVQ_PER_CHANNEL
+    assert plan_rc(d) == kvq.KVQ_EUNSUPPORTED
+    assert "per token" in kvq.kvq_last_error()
+
+
+def test_workspace_layout(lib):
+    d = desc(layer_bits=[(4, 2), (8, 8)], kmodes=[0, 1])
+    h = kvq.kvq_plan(d)
+    try:
+        D, B, Hkv, Hq, cap = 64, 2, 2, 4, (100 + 31) // 32
+        rec0 = 4 * D * 4 + 4 * D + 4 * D * 2 + 4 * D
+        rec1 = 4 * D * 8 + 4 * D + 4 * D * 8 + 4 * D
+        al = lambda x: (x + 255) // 256 * 256
+        expect = 256
+        expect = al(expect + rec0 * cap * B * Hkv)
+        expect = al(expect + 64 * D * B * Hkv)          # residual of the per-channel layer
+        expect = al(expect + rec1 * cap * B * Hkv)
+        expect = al(expect + B * Hq * 64 * D * 4)
+        expect = al(expect + B * Hq * 64 * 2 * 4)
+        assert kvq.kvq_workspace_bytes(h) == expect
+    finally:
+        kvq.kvq_destroy(h)
+
+
+def test_argument_checks_before_any_launch(lib):
+    h = kvq.kvq_plan(desc())
+    L = kvq.load()
+    try:
+        # not bound yet
+        assert L.kvq_append(h, 0, 4096, 4096, 1, None) == kvq.KVQ_EUNBOUND
+        n = kvq.kvq_workspace_bytes(h)
+        assert L.kvq_bind(h, 4096 + 16, n) == kvq.KVQ_EALIGN
+        assert L.kvq_bind(h, 4096, n - 1) == kvq.KVQ_EUNBOUND
+        fake = 1 << 40                      # never dereferenced: every call below fails on the host
+        assert L.kvq_bind(h, fake, n) == kvq.KVQ_OK
+        assert L.kvq_append(h, 2, fake, fake, 1, None) == kvq.KVQ_EINVAL      # layer
+        assert L.kvq_append(h, 0, None, fake, 1, None) == kvq.KVQ_EINVAL      # null
+        assert L.kvq_append(h, 0, fake + 8, fake, 1, None) == kvq.KVQ_EALIGN
+        assert L.kvq_append(h, 0, fake, fake, 0, None) == kvq.KVQ_EINVAL      # n_new
+        assert L.kvq_append(h, 0, fake, fake, 101, None) == kvq.KVQ_ECAPACITY
+        assert L.kvq_decode_attn(h, 0, fake, fake, 0, None) == kvq.KVQ_EINVAL  # empty layer
+        assert L.kvq_decode_attn(h, 0, fake + 4, fake, 0, None) == kvq.KVQ_EALIGN
+        assert "16-byte" in kvq.kvq_last_error()
+        assert kvq.kvq_seq_len(h, 1) == 0
+        need = ctypes.c_size_t()
+        assert L.kvq_export_layer(h, 0, None, 0, ctypes.byref(need)) == kvq.KVQ_OK
+        assert need.value == (2 * 2) * 32 * 64 * 2     # empty layer: a 32 x 64 bf16 residual per unit
+        assert L.kvq_truncate(h, 0, 1) == kvq.KVQ_EINVAL
+        assert L.kvq_set_num_splits(h, -1) == kvq.KVQ_EINVAL
+        assert L.kvq_set_num_splits(h, 3) == kvq.KVQ_OK
+    finally:
+        kvq.kvq_destroy(h)
+
+
+def test_product_path_has_no_fallback(monkeypatch, tmp_path):
+    """Without libkvq.so the binding raises; it never computes anything itself."""
+    monkeypatch.setattr(kvq, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(kvq, "_lib", None)
+    with pytest.raises(FileNotFoundError):
+        kvq.load()
