@@ -1,0 +1,395 @@
+"""Decode-step benchmark of the mixed-precision KV cache (one JSON line on stdout).
+
+A step = one decode token for every sequence of the batch through every layer: per
+layer, kvq_append of the new token's K/V (quantize + pack, group flush when a key group
+completes) then kvq_decode_attn (split kernel + log-sum-exp merge).  Each step of the
+decode schedule is captured once into a CUDA graph (untimed); the timed region replays
+K graphs.  Inputs are seeded synthetic tensors already resident in HBM; one step reads
+every layer's cache once (larger than L2 for every workload here).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c2-k8v8|c3|c4]
+    python bench.py --impl reference ...     # the CPU oracle on a bounded sample
+
+Under torchrun each rank runs its own replica of the workload (own seeds, no data-path
+collective: weak scaling); rank 0 prints the line with the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn tokens/s and HBM GB/s (% of roofline) over mixed-precision KV, 1 B200"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s pool figure)"
+
+
+def decode_bytes(B, Hkv, G, D, L, bk, bv, kmode):
+    """Algorithmic bytes of one decode-attention launch over L tokens: packed codes, fp16
+    scale+zero per 32 elements, the bf16 key residual, q in and out (bf16)."""
+    if kmode == 0:
+        kb = (L // 32) * 32 * D * (bk + 1) / 8 + (L % 32) * D * 2
+    else:
+        kb = L * D * (bk + 1) / 8
+    vb = L * D * (bv + 1) / 8
+    return B * Hkv * (kb + vb + 2 * G * D * 2)
+
+
+class ClockSampler:
+    """NVML sampling of SM clock and clock-event reasons in a background thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index, period=0.02):
+        self.samples = []
+        self.period = period
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+        self.t = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                clk = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                self.samples.append((clk, rs, util))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.t:
+            self._stop.set()
+            self.t.join()
+        busy = [s for s in self.samples if s[2] > 0] or self.samples
+        if not busy:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        reasons = set()
+        for _, rs, _ in busy:
+            for bit, name in self.REASONS.items():
+                if rs & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[0] for s in busy), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(busy)}
+
+
+# ---------------------------------------------------------------- CPU oracle arm
+def cpu_oracle_sample(wl, L, seqs, layers=1):
+    """Time the oracle (quantize the layer's cache + fp64 attention) on `seqs` sequences
+    of `layers` layers at context L; returns (seconds, tokens/s scaled to the workload)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from layer_wise_mixed_b200 import inputs
+    t = 0.0
+    for l in range(layers):
+        K, V = inputs.layer_kv(wl, l, L, "cpu", batch=seqs, tag="cpu-sample")
+        q = inputs.step_q(wl, l, 0, "cpu", batch=seqs)
+        b16 = lambda x: x.contiguous().view(torch.int16).numpy().view(np.uint16)
+        Kb, Vb, qb = b16(K), b16(V), b16(q)
+        bk, bv = wl.layer_bits[l % len(wl.layer_bits)]
+        t0 = time.perf_counter()
+        oracle.layer(Kb, Vb, qb, wl.G, bk, bv, wl.kmode, want_image=False)
+        t += time.perf_counter() - t0
+    step_s = t / layers * wl.num_layers * (wl.batch / seqs)
+    return t, wl.batch / step_s
+
+
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    cores = os.cpu_count()
+    seqs = max(1, min(wl.batch, args.ref_seqs))
+    Ls = [wl.prefill + 1 + (i % max(1, wl.decode_steps)) for i in range(args.warmup + args.steps)]
+    for i in range(args.warmup):
+        cpu_oracle_sample(wl, Ls[i], seqs)
+    tot, vals = 0.0, []
+    for i in range(args.steps):
+        s, v = cpu_oracle_sample(wl, Ls[args.warmup + i], seqs)
+        tot += s
+        vals.append(v)
+    value = len(vals) / sum(1.0 / v for v in vals)
+    sample = (f"per step: oracle quantize+fp64 attention of 1 of {wl.num_layers} layers for {seqs} of "
+              f"{wl.batch} sequences at the step's context, scaled to the full step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * wl.batch / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl):
+    bits = sorted(set(wl.layer_bits))
+    return {"workload": wl.name, "layers": wl.num_layers, "batch": wl.batch, "q_heads": wl.n_q_heads,
+            "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim,
+            "context": f"{wl.prefill + 1}..{wl.prefill + wl.decode_steps}",
+            "bits": ",".join(f"K{a}V{b}" for a, b in bits), "equivalent_bits": wl.equivalent_bits(),
+            "keys": "per-channel" if wl.kmode == 0 else "per-token", "values": "per-token", "group": 32,
+            "l2": "inputs larger than L2 (each step reads every layer's cache once)",
+            "launch": "one CUDA graph per decode step (append + decode for all layers)"}
+
+
+# ---------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=512)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="c2", choices=["c2", "c2-k8v8", "c2-k8v4", "c3", "c4"])
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--ref-seqs", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="use only the first N layers (small ncu captures; reported in config.layers)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    from layer_wise_mixed_b200 import configs
+    wl = configs.by_name(args.workload)
+    if args.layers:
+        import dataclasses
+        wl = dataclasses.replace(wl, num_layers=args.layers, layer_bits=wl.layer_bits[:args.layers])
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from layer_wise_mixed_b200 import inputs, kvq
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+
+    # replica per rank: its own sequences (weak scaling, no data-path collective)
+    if world > 1:
+        wl = configs.Workload(f"{wl.name}-rank{rank}", wl.num_layers, wl.batch, wl.n_q_heads, wl.n_kv_heads,
+                              wl.head_dim, wl.prefill, wl.decode_steps, wl.layer_bits, wl.kmode, wl.n_outlier,
+                              wl.outlier_lo, wl.outlier_hi)
+    B, Hkv, Hq, D, G, NL = wl.batch, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.G, wl.num_layers
+    cache = kvq.Cache(NL, B, Hkv, Hq, D, wl.max_ctx, list(wl.layer_bits), kmodes=[wl.kmode] * NL)
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for l in range(NL):
+            K, V = inputs.layer_kv(wl, l, wl.prefill, "cuda")
+            cache.append(l, K, V)
+            del K, V
+    stream.synchronize()
+
+    # decode schedule inputs, resident in HBM
+    nsched = wl.decode_steps
+    Kn = torch.empty((nsched, NL, B, Hkv, 1, D), dtype=torch.bfloat16, device="cuda")
+    Vn = torch.empty_like(Kn)
+    Qn = torch.empty((nsched, NL, B, Hq, D), dtype=torch.bfloat16, device="cuda")
+    for s in range(nsched):
+        for l in range(NL):
+            k, v = inputs.step_kv(wl, l, s, "cuda")
+            Kn[s, l].copy_(k)
+            Vn[s, l].copy_(v)
+            Qn[s, l].copy_(inputs.step_q(wl, l, s, "cuda"))
+    out = torch.empty((NL, B, Hq, D), dtype=torch.bfloat16, device="cuda")
+
+    # one eager decode per layer before capture (kernel attributes, occupancy, status clear)
+    with torch.cuda.stream(stream):
+        for l in range(NL):
+            cache.decode_attn(l, Qn[0, l], out[l], stream=stream)
+    stream.synchronize()
+
+    graphs, dec_graphs, splits, Ls = [], [], [], []
+    for s in range(nsched):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for l in range(NL):
+                kvq.kvq_append(cache.h, l, Kn[s, l], Vn[s, l], 1, stream)
+                kvq.kvq_decode_attn(cache.h, l, Qn[s, l], out[l], False, stream)
+        graphs.append(g)
+        splits.append([kvq.kvq_get_num_splits(cache.h, l) for l in range(NL)])
+        Ls.append(cache.seq_len(0))
+        gd = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gd, stream=stream):
+            for l in range(NL):
+                kvq.kvq_decode_attn(cache.h, l, Qn[s, l], out[l], False, stream)
+        dec_graphs.append(gd)
+    torch.cuda.synchronize()
+
+    order = [(args.warmup + i) % nsched for i in range(args.steps)]
+    sampler = ClockSampler(local)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- timed region: K full steps ----
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % nsched].replay()
+    sampler.start()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for s in order:
+            graphs[s].replay()
+        e1.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * B * args.steps / (ms / 1e3)
+
+    # ---- dominant kernel: decode-only graphs over the same schedule (live events) ----
+    with torch.cuda.stream(stream):
+        for s in order[: min(len(order), 8)]:
+            dec_graphs[s].replay()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for s in order:
+            dec_graphs[s].replay()
+        d1.record(stream)
+    stream.synchronize()
+    dec_ms = d0.elapsed_time(d1)
+    launches_dec = args.steps * NL
+    dec_bytes = sum(decode_bytes(B, Hkv, G, D, Ls[s], *wl.layer_bits[l], wl.kmode)
+                    for s in order for l in range(NL))
+    peak, peak_src = measured_hbm_peak()
+    achieved = dec_bytes / (dec_ms / 1e3) / 1e9
+    gpu_launches = sum(2 + (1 if splits[s][l] > 1 else 0) for s in order for l in range(NL))
+
+    # ---- e2e: public API with host buffers, H2D + D2H inside the timed region ----
+    e2e_steps = args.e2e_steps or min(args.steps, 64)
+    hK = Kn.cpu().pin_memory()
+    hV = Vn.cpu().pin_memory()
+    hQ = Qn.cpu().pin_memory()
+    hO = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dK = torch.empty_like(Kn[0])
+    dV = torch.empty_like(Vn[0])
+    dQ = torch.empty_like(Qn[0])
+    for l in range(NL):
+        kvq.kvq_truncate(cache.h, l, wl.prefill)
+
+    def e2e_step(s):
+        dK.copy_(hK[s], non_blocking=True)
+        dV.copy_(hV[s], non_blocking=True)
+        dQ.copy_(hQ[s], non_blocking=True)
+        for l in range(NL):
+            if cache.seq_len(l) >= wl.max_ctx:
+                kvq.kvq_truncate(cache.h, l, wl.prefill)
+            kvq.kvq_append(cache.h, l, dK[l], dV[l], 1, stream)
+            kvq.kvq_decode_attn(cache.h, l, dQ[l], out[l], False, stream)
+        hO.copy_(out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            e2e_step(i % nsched)
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(e2e_steps):
+            e2e_step((3 + i) % nsched)
+        f1.record(stream)
+    barrier()
+    e2e_ms = f0.elapsed_time(f1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * B * e2e_steps / (e2e_ms / 1e3)
+    h2d = (dK.numel() + dV.numel() + dQ.numel()) * 2
+    d2h = out.numel() * 2
+    status = kvq.kvq_device_status(cache.h, stream)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_cpu, v_cpu = 0.0, []
+        L_mid = wl.prefill + max(1, wl.decode_steps // 2)
+        while t_cpu < 10.0:
+            s_, v_ = cpu_oracle_sample(wl, L_mid, max(1, min(B, args.ref_seqs)))
+            t_cpu += s_
+            v_cpu.append(v_)
+        cpu = {"value": len(v_cpu) / sum(1 / v for v in v_cpu), "unit": "tokens/s", "cores": os.cpu_count(),
+               "kind": "oracle",
+               "sample": (f"{len(v_cpu)} x (quantize + fp64 attention of 1 layer, {min(B, args.ref_seqs)} of {B} "
+                          f"sequences, context {L_mid}), {t_cpu:.1f} s CPU, scaled to a full step")}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f16*f16->f32 (codes exact in f16), f32 quantizer",
+                "data": "synthetic (seeded normal K/V/Q, outlier key channels; no weights or datasets)",
+                "config": workload_config(wl),
+                "hbm_gbs_decode": achieved,
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                             "frac": achieved / peak, "traffic": None, "kernel": "decode_split_kernel (+merge)",
+                             "peak_source": peak_src, "avg_launch_us": 1e3 * dec_ms / launches_dec,
+                             "algorithmic_bytes_per_launch": dec_bytes / launches_dec},
+                "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                        "steps": e2e_steps, "how": "per step: pinned H2D of all layers' K/V/q, kvq_append + "
+                        "kvq_decode_attn per layer (eager C-ABI calls), D2H of all layers' outputs"},
+                "gpu_launches": gpu_launches, "clocks": clocks, "device_status": status,
+                "splits": sorted(set(x for s in order for x in splits[s]))}
+        print(json.dumps(line), flush=True)
+    del graphs, dec_graphs
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -83,7 +83,7 @@ __device__ __forceinline__ void word_lane(int widx, int Wh, int &lane, int &w) {
 // Per-token quantization of the new tokens of one 16-token half-block and repacking
 // of its words.  role 0 = keys (per-token mode), 1 = values.
 __device__ void per_token_half(const AppendParams &p, int role, int unit, int hbi,
-                               uint8_t (*codes)[kMaxD]) {
+                               uint8_t (*codes)[kMaxD], unsigned *cta_smax) {
     const int D = p.D, nj = D / 32;
     const int bits = role ? p.bv : p.bk;
     const uint16_t *src = (role ? p.V : p.K) + static_cast<long long>(unit) * p.n * D;
@@ -116,6 +116,7 @@ __device__ void per_token_half(const AppendParams &p, int role, int unit, int hb
             if (lane == 0) {
                 const uint32_t v = static_cast<uint32_t>(s16) | (static_cast<uint32_t>(z16) << 16);
                 *reinterpret_cast<uint32_t *>(sz + 4LL * (u * nj + j)) = v;
+                atomicMax(cta_smax, static_cast<unsigned>(s16));
             }
         }
     }
@@ -144,7 +145,7 @@ __device__ void per_token_half(const AppendParams &p, int role, int unit, int hb
 // Per-channel quantization of one completed 32-token key group; the CTA with
 // first == true also writes the new residual tokens of its (b, h) afterwards.
 __device__ void per_channel_group(const AppendParams &p, int unit, int q, bool do_group, bool first,
-                                  float (*xs)[kMaxD], uint8_t (*codes)[kMaxD]) {
+                                  float (*xs)[kMaxD], uint8_t (*codes)[kMaxD], unsigned *cta_smax) {
     const int D = p.D;
     const uint16_t *src = p.K + static_cast<long long>(unit) * p.n * D;
     uint16_t *res = p.res + static_cast<long long>(unit) * 32 * D;
@@ -171,6 +172,7 @@ __device__ void per_channel_group(const AppendParams &p, int unit, int q, bool d
             for (int u = 0; u < 32; ++u) codes[u][d] = static_cast<uint8_t>(group_code(xs[u][d], s, z, p.bk));
             *reinterpret_cast<uint32_t *>(rec + p.kc + 4LL * d) =
                 static_cast<uint32_t>(s16) | (static_cast<uint32_t>(z16) << 16);
+            atomicMax(cta_smax, static_cast<unsigned>(s16));
         }
         __syncthreads();
         const int bits = p.bk, Wh = D * bits / 64, F = 32 / bits, nwh = D * bits / 2;
@@ -199,24 +201,35 @@ __device__ void per_channel_group(const AppendParams &p, int unit, int q, bool d
     }
 }
 
+// Scales are non-negative, so their fp16 bit patterns order like their values: the
+// largest scale of the layer is kept with integer atomicMax (one per CTA), for the
+// decoder's choice of fp16 operand prescales.
 __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams p) {
     __shared__ __align__(16) float xs[32][kMaxD];
     __shared__ __align__(16) uint8_t codes[32][kMaxD];
+    __shared__ unsigned cta_smax;
+    if (threadIdx.x == 0) cta_smax = 0;
+    __syncthreads();
     const int cta = blockIdx.x;
+    int role;
     if (cta < p.nV) {
+        role = 1;
         const int unit = cta / p.nhb, hbi = p.hb0 + cta % p.nhb;
-        per_token_half(p, 1, unit, hbi, codes);
-        return;
+        per_token_half(p, 1, unit, hbi, codes, &cta_smax);
+    } else {
+        role = 0;
+        const int k = cta - p.nV;
+        if (p.kmode == 1) {
+            const int unit = k / p.nhb, hbi = p.hb0 + k % p.nhb;
+            per_token_half(p, 0, unit, hbi, codes, &cta_smax);
+        } else {
+            const int per_unit = p.ng > 0 ? p.ng : 1;
+            const int unit = k / per_unit, qi = k % per_unit;
+            per_channel_group(p, unit, p.g0 + qi, p.ng > 0, qi == 0, xs, codes, &cta_smax);
+        }
     }
-    const int k = cta - p.nV;
-    if (p.kmode == 1) {
-        const int unit = k / p.nhb, hbi = p.hb0 + k % p.nhb;
-        per_token_half(p, 0, unit, hbi, codes);
-        return;
-    }
-    const int per_unit = p.ng > 0 ? p.ng : 1;
-    const int unit = k / per_unit, qi = k % per_unit;
-    per_channel_group(p, unit, p.g0 + qi, p.ng > 0, qi == 0, xs, codes);
+    __syncthreads();
+    if (threadIdx.x == 0 && cta_smax) atomicMax(p.smax + role, cta_smax);
 }
 
 }  // namespace

@@ -28,6 +28,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <mutex>
+
 #include "kvq_internal.h"
 
 namespace kvq {
@@ -160,6 +162,31 @@ __device__ __forceinline__ void load_lane_words(const uint8_t *half_area, int la
 }
 
 // ------------------------------------------------------------------ kernel
+// Exponent-only power of two (exact scaling), e in [-126, 127].
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
+
+// Largest e with 2^e <= x (x > 0, normal).
+__device__ __forceinline__ int floor_log2(float x) { return ((__float_as_int(x) >> 23) & 0xFF) - 127; }
+
+__device__ __forceinline__ float half_lo_f(uint32_t w) { return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFF))); }
+__device__ __forceinline__ float half_hi_f(uint32_t w) { return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16))); }
+
+// hi/lo fp16 pair of x*s for a half2 x = xh + xl and a half2 s: hi = rn(xh*s),
+// lo = rn(rn_exact(xh*s - hi) + xl*s); the residual xh*s - hi is exact in fp16 (FMA).
+__device__ __forceinline__ void mul_hilo(uint32_t xh, uint32_t xl, uint32_t s, uint32_t &hi, uint32_t &lo) {
+    const __half2 h = __hmul2(bits_h2(xh), bits_h2(s));
+    const __half2 r = __hfma2(bits_h2(xh), bits_h2(s), __hneg2(h));
+    lo = h2_bits(__hfma2(bits_h2(xl), bits_h2(s), r));
+    hi = h2_bits(h);
+}
+
+// Split two floats into fp16 hi (11-bit truncation, exact) and lo (remainder) pairs.
+__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const float ha = trunc11(a), hb = trunc11(b);
+    hi = pack_h2(ha, hb);
+    lo = pack_h2(a - ha, b - hb);
+}
+
 template <int BK, int BV, int KM, int D, int NT>
 __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodeParams p) {
     constexpr int KS = D / 16;     // 16-channel steps (QK) / 16-channel row tiles (PV)
@@ -202,6 +229,12 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
     }
     issued = __shfl_sync(0xffffffffu, issued, 0);
 
+    // ---- operand prescales (powers of two) from the layer's largest scales ----
+    const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
+    const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
+    // values: p * 2^kp * s_v stays below 2^14 in fp16
+    const int kp = smax_v > 0.f ? max(-24, min(14, 14 - floor_log2(smax_v) - 1)) : 14;
+
     // ---- this thread's query head and channels (16k + 2t + {0, 1, 8, 9}) ----
     const int hh = g % G;
     const uint16_t *qrow = p.q + (static_cast<long long>(b) * p.Hkv * G + h * G + hh) * D;
@@ -217,12 +250,36 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
     }
     const float qscale = kLog2e * rsqrtf(static_cast<float>(D));
 
-    // per-token keys: constant masked A fragments (rows r = j*G + head) and q sums per group
-    uint32_t aq[KM == 1 ? KS : 1][4];
-    float qsum_g = 0.f, qsum_g8 = 0.f;   // sum of q over the channel group of rows g and g+8
+    // Per-channel keys: q~ = q log2(e)/sqrt(D) 2^kq as fp16 hi/lo fragments (rows g: hi,
+    // g+8: lo), kq chosen so that q~ s_k stays below 2^14 and q~ below 2^15.
+    // Per-token keys: raw q (exact in fp16), rows (group j, head) masked to group j.
+    uint32_t aq[KS][4];
+    float unscale = 1.f;                 // scores = accumulators * unscale
+    float qsum_g = 0.f, qsum_g8 = 0.f;   // per-token keys: sum of q over the rows' groups
     const int jg = g / G, jg8 = (g + 8) / G;
     const bool row_g = (KM == 1) && (g < G * NJ), row_g8 = (KM == 1) && (g + 8 < G * NJ);
-    if constexpr (KM == 1) {
+    if constexpr (KM == 0) {
+        float amax = 0.f;
+#pragma unroll
+        for (int k = 0; k < KS; ++k)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) amax = fmaxf(amax, fabsf(qv[k][c] * qscale));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        int kq = 0;
+        if (amax > 0.f) {
+            kq = 14 - floor_log2(amax);                              // q~ < 2^15
+            if (smax_k > 0.f) kq = min(kq, 13 - floor_log2(amax) - floor_log2(smax_k) - 1);   // q~ s < 2^14
+            kq = max(-60, min(60, kq));
+        }
+        const float sc = qscale * pow2f(kq > 0 ? min(kq, 126) : max(kq, -126));
+        unscale = pow2f(-kq);
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+            split2(qv[k][0] * sc, qv[k][1] * sc, aq[k][0], aq[k][1]);
+            split2(qv[k][2] * sc, qv[k][3] * sc, aq[k][2], aq[k][3]);
+        }
+    } else {
         float part[NJ];
 #pragma unroll
         for (int j = 0; j < NJ; ++j) part[j] = 0.f;
@@ -243,11 +300,7 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
             if (j == (jg < NJ ? jg : 0)) qsum_g = part[j];
             if (j == (jg8 < NJ ? jg8 : 0)) qsum_g8 = part[j];
         }
-    } else {
-#pragma unroll
-        for (int k = 0; k < KS; ++k)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) qv[k][c] *= qscale;
+        unscale = qscale;
     }
 
     float m_run = -INFINITY, l_run = 0.f;
@@ -262,10 +315,13 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
 #pragma unroll
             for (int c = 0; c < 4; ++c) oacc[m][n][c] = 0.f;
 
-    // B-operand column of this thread for P (NT == 1: hi, lo or zero by column)
-    const int col_kind = (NT == 1) ? (g < G ? 0 : (g < 2 * G ? 1 : 2)) : (g < G ? 0 : 2);
+    // B-operand column of this thread for P: NT == 1: hi (g < G), lo (G <= g < 2G) or
+    // zero; NT == 2: tile 0 hi, tile 1 lo for g < G.
+    const uint32_t m_hi = ((NT == 1 && g < G) || (NT == 2 && g < G)) ? 0xFFFFFFFFu : 0u;
+    const uint32_t m_lo = (NT == 1 && g >= G && g < 2 * G) ? 0xFFFFFFFFu : 0u;
     const int alpha_src0 = 4 * ((NT == 1) ? ((2 * t) % G) : min(2 * t, 7));
     const int alpha_src1 = 4 * ((NT == 1) ? ((2 * t + 1) % G) : min(2 * t + 1, 7));
+    const float pbias = static_cast<float>(kp);
 
     bool failed = false;
     int i = 0;
@@ -277,7 +333,8 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
             break;
         }
         const uint8_t *R = stages + st * REC;
-        const int valid = (blk == tail_blk) ? rem : 32;
+        const bool tail = blk == tail_blk;
+        const int valid = tail ? rem : 32;
 
         // ================= scores S^T (rows: heads, columns: 8-token tiles) =================
         float acc[4][4];
@@ -285,9 +342,8 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
         for (int n = 0; n < 4; ++n)
 #pragma unroll
             for (int c = 0; c < 4; ++c) acc[n][c] = 0.f;
-        float cz = 0.f;
-        const bool resid_block = (KM == 0) && (blk == tail_blk);
-        if (!resid_block) {
+        float czacc[4] = {0.f, 0.f, 0.f, 0.f};
+        if (KM == 1 || !tail) {
             uint32_t kw[2][WHK];
             load_lane_words<WHK>(R, lane, kw[0]);
             load_lane_words<WHK>(R + 2 * D * BK, lane, kw[1]);
@@ -295,26 +351,13 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
             for (int k = 0; k < KS; ++k) {
                 uint32_t a[4];
                 if constexpr (KM == 0) {
-                    const int c0 = 16 * k + 2 * t;
-                    const uint2 sz0 = *reinterpret_cast<const uint2 *>(R + KC + 4 * c0);
-                    const uint2 sz8 = *reinterpret_cast<const uint2 *>(R + KC + 4 * (c0 + 8));
-                    const __half2 s01 = __halves2half2(__ushort_as_half(sz0.x & 0xFFFF), __ushort_as_half(sz0.y & 0xFFFF));
-                    const __half2 z01 = __halves2half2(__ushort_as_half(sz0.x >> 16), __ushort_as_half(sz0.y >> 16));
-                    const __half2 s89 = __halves2half2(__ushort_as_half(sz8.x & 0xFFFF), __ushort_as_half(sz8.y & 0xFFFF));
-                    const __half2 z89 = __halves2half2(__ushort_as_half(sz8.x >> 16), __ushort_as_half(sz8.y >> 16));
-                    const float2 fs01 = __half22float2(s01), fz01 = __half22float2(z01);
-                    const float2 fs89 = __half22float2(s89), fz89 = __half22float2(z89);
-                    const float x0 = qv[k][0] * fs01.x, x1 = qv[k][1] * fs01.y;
-                    const float x8 = qv[k][2] * fs89.x, x9 = qv[k][3] * fs89.y;
-                    cz = fmaf(qv[k][0], fz01.x, cz);
-                    cz = fmaf(qv[k][1], fz01.y, cz);
-                    cz = fmaf(qv[k][2], fz89.x, cz);
-                    cz = fmaf(qv[k][3], fz89.y, cz);
-                    const float h0 = trunc11(x0), h1 = trunc11(x1), h8 = trunc11(x8), h9 = trunc11(x9);
-                    a[0] = pack_h2(h0, h1);
-                    a[1] = pack_h2(x0 - h0, x1 - h1);
-                    a[2] = pack_h2(h8, h9);
-                    a[3] = pack_h2(x8 - h8, x9 - h9);
+                    const uint2 sz0 = *reinterpret_cast<const uint2 *>(R + KC + 4 * (16 * k + 2 * t));
+                    const uint2 sz8 = *reinterpret_cast<const uint2 *>(R + KC + 4 * (16 * k + 2 * t + 8));
+                    const uint32_t s01 = prmt(sz0.x, sz0.y, 0x5410u), z01 = prmt(sz0.x, sz0.y, 0x7632u);
+                    const uint32_t s89 = prmt(sz8.x, sz8.y, 0x5410u), z89 = prmt(sz8.x, sz8.y, 0x7632u);
+                    mul_hilo(aq[k][0], aq[k][1], s01, a[0], a[1]);
+                    mul_hilo(aq[k][2], aq[k][3], s89, a[2], a[3]);
+                    mma16816(czacc, aq[k], z01, z89);   // sum_d q~_d z_d, same in every column
                 } else {
                     a[0] = aq[k][0];
                     a[1] = aq[k][1];
@@ -333,10 +376,6 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
             const uint16_t *res = p.res + (static_cast<long long>(b) * p.Hkv + h) * 32 * D;
 #pragma unroll
             for (int k = 0; k < KS; ++k) {
-                const float h0 = trunc11(qv[k][0]), h1 = trunc11(qv[k][1]);
-                const float h8 = trunc11(qv[k][2]), h9 = trunc11(qv[k][3]);
-                uint32_t a[4] = {pack_h2(h0, h1), pack_h2(qv[k][0] - h0, qv[k][1] - h1), pack_h2(h8, h9),
-                                 pack_h2(qv[k][2] - h8, qv[k][3] - h9)};
 #pragma unroll
                 for (int n = 0; n < 4; ++n) {
                     const int u = 8 * n + g;
@@ -347,19 +386,18 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
                         b0 = pack_h2(__uint_as_float(r0 << 16), __uint_as_float(r0 & 0xFFFF0000u));
                         b1 = pack_h2(__uint_as_float(r8 << 16), __uint_as_float(r8 & 0xFFFF0000u));
                     }
-                    mma16816(acc[n], a, b0, b1);
+                    mma16816(acc[n], aq[k], b0, b1);
                 }
             }
         }
 
         float sc[4][2];
         if constexpr (KM == 0) {
-            cz += __shfl_xor_sync(0xffffffffu, cz, 1);
-            cz += __shfl_xor_sync(0xffffffffu, cz, 2);
+            const float cz = czacc[0] + czacc[2];
 #pragma unroll
             for (int n = 0; n < 4; ++n) {
-                sc[n][0] = acc[n][0] + acc[n][2] + cz;
-                sc[n][1] = acc[n][1] + acc[n][3] + cz;
+                sc[n][0] = (acc[n][0] + acc[n][2] + cz) * unscale;
+                sc[n][1] = (acc[n][1] + acc[n][3] + cz) * unscale;
             }
         } else {
             // per-token key scales, then sum the (group, head) rows of each head
@@ -371,27 +409,27 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
                     float v = 0.f;
                     if (row_g) {
                         const uint32_t e = *reinterpret_cast<const uint32_t *>(R + KC + 4 * (u * NJ + jg));
-                        v = fmaf(__half2float(__ushort_as_half(e & 0xFFFF)), acc[n][c],
-                                 __half2float(__ushort_as_half(e >> 16)) * qsum_g);
+                        v = fmaf(half_lo_f(e), acc[n][c], half_hi_f(e) * qsum_g);
                     }
                     if (row_g8) {
                         const uint32_t e = *reinterpret_cast<const uint32_t *>(R + KC + 4 * (u * NJ + jg8));
-                        v += fmaf(__half2float(__ushort_as_half(e & 0xFFFF)), acc[n][2 + c],
-                                  __half2float(__ushort_as_half(e >> 16)) * qsum_g8);
+                        v += fmaf(half_lo_f(e), acc[n][2 + c], half_hi_f(e) * qsum_g8);
                     }
 #pragma unroll
                     for (int msk = G; msk < 8; msk <<= 1) v += __shfl_xor_sync(0xffffffffu, v, 4 * msk);
-                    sc[n][c] = v * qscale;
+                    sc[n][c] = v * unscale;
                 }
             }
         }
+        if (tail) {
 #pragma unroll
-        for (int n = 0; n < 4; ++n)
+            for (int n = 0; n < 4; ++n)
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-                if (8 * n + 2 * t + c >= valid) sc[n][c] = -INFINITY;
+                for (int c = 0; c < 2; ++c)
+                    if (8 * n + 2 * t + c >= valid) sc[n][c] = -INFINITY;
+        }
 
-        // ================= online softmax (base 2) =================
+        // ================= online softmax (base 2; p carries the factor 2^kp) =================
         float mloc = fmaxf(fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1])),
                            fmaxf(fmaxf(sc[2][0], sc[2][1]), fmaxf(sc[3][0], sc[3][1])));
         mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
@@ -399,13 +437,14 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
         const float m_new = fmaxf(m_run, mloc);
         const float alpha = fast_exp2(m_run - m_new);
         m_run = m_new;
+        const float shift = pbias - m_new;
         float pr[4][2];
         float psum = 0.f;
 #pragma unroll
         for (int n = 0; n < 4; ++n)
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                pr[n][c] = fast_exp2(sc[n][c] - m_new);
+                pr[n][c] = fast_exp2(sc[n][c] + shift);
                 psum += pr[n][c];
             }
         l_run = fmaf(l_run, alpha, psum);
@@ -430,55 +469,61 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
         for (int kk = 0; kk < 2; ++kk) {
             uint32_t vw[WHV];
             load_lane_words<WHV>(R + KC + KSZ + kk * 2 * D * BV, lane, vw);
-            const float pt[4] = {pr[2 * kk][0], pr[2 * kk][1], pr[2 * kk + 1][0], pr[2 * kk + 1][1]};
-            const int ut[4] = {16 * kk + 2 * t, 16 * kk + 2 * t + 1, 16 * kk + 8 + 2 * t, 16 * kk + 9 + 2 * t};
-            uint32_t szv[4][NJ];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const uint8_t *src = R + KC + KSZ + VC + 4 * (ut[e] * NJ);
+            // tokens 16kk + 2t + {0,1} (pair A) and 16kk + 8 + 2t + {0,1} (pair B)
+            const float pa0 = pr[2 * kk][0], pa1 = pr[2 * kk][1];
+            const float pb0 = pr[2 * kk + 1][0], pb1 = pr[2 * kk + 1][1];
+            uint32_t pah, pal, pbh, pbl;
+            split2(pa0, pa1, pah, pal);
+            split2(pb0, pb1, pbh, pbl);
+            uint32_t wa0[NJ], wa1[NJ], wb0[NJ], wb1[NJ];
+            {
+                const uint8_t *vs = R + KC + KSZ + VC;
+                const int u0 = 16 * kk + 2 * t;
                 if constexpr (NJ == 4) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(src);
-                    szv[e][0] = v.x;
-                    szv[e][1] = v.y;
-                    szv[e][2] = v.z;
-                    szv[e][3] = v.w;
-                } else if constexpr (NJ == 2) {
-                    const uint2 v = *reinterpret_cast<const uint2 *>(src);
-                    szv[e][0] = v.x;
-                    szv[e][1] = v.y;
+                    const uint4 x0 = *reinterpret_cast<const uint4 *>(vs + 16 * u0);
+                    const uint4 x1 = *reinterpret_cast<const uint4 *>(vs + 16 * (u0 + 1));
+                    const uint4 x2 = *reinterpret_cast<const uint4 *>(vs + 16 * (u0 + 8));
+                    const uint4 x3 = *reinterpret_cast<const uint4 *>(vs + 16 * (u0 + 9));
+                    wa0[0] = x0.x; wa0[1] = x0.y; wa0[2] = x0.z; wa0[3] = x0.w;
+                    wa1[0] = x1.x; wa1[1] = x1.y; wa1[2] = x1.z; wa1[3] = x1.w;
+                    wb0[0] = x2.x; wb0[1] = x2.y; wb0[2] = x2.z; wb0[3] = x2.w;
+                    wb1[0] = x3.x; wb1[1] = x3.y; wb1[2] = x3.z; wb1[3] = x3.w;
                 } else {
 #pragma unroll
-                    for (int j = 0; j < NJ; ++j) szv[e][j] = reinterpret_cast<const uint32_t *>(src)[j];
+                    for (int j = 0; j < NJ; ++j) {
+                        wa0[j] = reinterpret_cast<const uint32_t *>(vs + 4 * NJ * u0)[j];
+                        wa1[j] = reinterpret_cast<const uint32_t *>(vs + 4 * NJ * (u0 + 1))[j];
+                        wb0[j] = reinterpret_cast<const uint32_t *>(vs + 4 * NJ * (u0 + 8))[j];
+                        wb1[j] = reinterpret_cast<const uint32_t *>(vs + 4 * NJ * (u0 + 9))[j];
+                    }
                 }
             }
 #pragma unroll
             for (int j = 0; j < NJ; ++j) {
-                float pp[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float s = __half2float(__ushort_as_half(szv[e][j] & 0xFFFF));
-                    const float z = __half2float(__ushort_as_half(szv[e][j] >> 16));
-                    const bool live = pt[e] != 0.0f;
-                    pp[e] = live ? pt[e] * s : 0.f;
-                    zacc[j] += live ? pt[e] * z : 0.f;
+                uint32_t sa = prmt(wa0[j], wa1[j], 0x5410u), sb = prmt(wb0[j], wb1[j], 0x5410u);
+                float za0 = half_hi_f(wa0[j]), za1 = half_hi_f(wa1[j]);
+                float zb0 = half_hi_f(wb0[j]), zb1 = half_hi_f(wb1[j]);
+                if (tail) {
+                    // absent tokens: p = 0, and their scale/zero words may hold anything
+                    const int u0 = 16 * kk + 2 * t;
+                    if (u0 >= valid) { sa &= 0xFFFF0000u; za0 = 0.f; }
+                    if (u0 + 1 >= valid) { sa &= 0x0000FFFFu; za1 = 0.f; }
+                    if (u0 + 8 >= valid) { sb &= 0xFFFF0000u; zb0 = 0.f; }
+                    if (u0 + 9 >= valid) { sb &= 0x0000FFFFu; zb1 = 0.f; }
                 }
-                uint32_t bh0, bh1, bl0 = 0u, bl1 = 0u;
-                {
-                    const float h0 = trunc11(pp[0]), h1 = trunc11(pp[1]), h2 = trunc11(pp[2]), h3 = trunc11(pp[3]);
-                    if constexpr (NT == 1) {
-                        const float v0 = col_kind == 0 ? h0 : (col_kind == 1 ? pp[0] - h0 : 0.f);
-                        const float v1 = col_kind == 0 ? h1 : (col_kind == 1 ? pp[1] - h1 : 0.f);
-                        const float v2 = col_kind == 0 ? h2 : (col_kind == 1 ? pp[2] - h2 : 0.f);
-                        const float v3 = col_kind == 0 ? h3 : (col_kind == 1 ? pp[3] - h3 : 0.f);
-                        bh0 = pack_h2(v0, v1);
-                        bh1 = pack_h2(v2, v3);
-                    } else {
-                        const bool on = col_kind == 0;
-                        bh0 = on ? pack_h2(h0, h1) : 0u;
-                        bh1 = on ? pack_h2(h2, h3) : 0u;
-                        bl0 = on ? pack_h2(pp[0] - h0, pp[1] - h1) : 0u;
-                        bl1 = on ? pack_h2(pp[2] - h2, pp[3] - h3) : 0u;
-                    }
+                zacc[j] = fmaf(pa0, za0, fmaf(pa1, za1, fmaf(pb0, zb0, fmaf(pb1, zb1, zacc[j]))));
+                uint32_t ah, al, bh, bl;
+                mul_hilo(pah, pal, sa, ah, al);
+                mul_hilo(pbh, pbl, sb, bh, bl);
+                uint32_t b0, b1, c0 = 0u, c1 = 0u;
+                if constexpr (NT == 1) {
+                    b0 = (ah & m_hi) | (al & m_lo);
+                    b1 = (bh & m_hi) | (bl & m_lo);
+                } else {
+                    b0 = ah & m_hi;
+                    b1 = bh & m_hi;
+                    c0 = al & m_hi;
+                    c1 = bl & m_hi;
                 }
 #pragma unroll
                 for (int mm = 0; mm < 2; ++mm) {
@@ -489,8 +534,8 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
                         const int s = 4 * m + r;
                         a[r] = unpack<BV>(vw[s / PV], s % PV);
                     }
-                    mma16816(oacc[m][0], a, bh0, bh1);
-                    if constexpr (NT == 2) mma16816(oacc[m][NT - 1], a, bl0, bl1);
+                    mma16816(oacc[m][0], a, b0, b1);
+                    if constexpr (NT == 2) mma16816(oacc[m][NT - 1], a, c0, c1);
                 }
             }
         }
@@ -642,14 +687,49 @@ size_t decode_smem_bytes(long long rec_bytes, int nstage, int D, int G) {
     return base + static_cast<size_t>(NW) * nstage * 8;
 }
 
+// Per-kernel cache of the dynamic shared-memory attribute and occupancy, so launches
+// (including launches recorded into CUDA graphs) issue no attribute calls.
+struct KernelState {
+    KernelFn fn = nullptr;
+    size_t smem_set = 0;
+    size_t occ_smem = 0;
+    int occ = 0;
+};
+static std::mutex g_state_mu;
+static KernelState g_state[64];
+
+static cudaError_t prepare_kernel(KernelFn fn, size_t smem, int *occ_out) {
+    std::lock_guard<std::mutex> lk(g_state_mu);
+    KernelState *ks = nullptr;
+    for (auto &e : g_state) {
+        if (e.fn == fn || e.fn == nullptr) {
+            ks = &e;
+            break;
+        }
+    }
+    if (!ks) return cudaErrorInvalidValue;
+    ks->fn = fn;
+    if (smem > ks->smem_set) {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        ks->smem_set = smem;
+    }
+    if (occ_out) {
+        if (ks->occ_smem != smem) {
+            cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ks->occ, fn, NW * 32, smem);
+            if (e != cudaSuccess) return e;
+            ks->occ_smem = smem;
+        }
+        *occ_out = ks->occ;
+    }
+    return cudaSuccess;
+}
+
 cudaError_t decode_occupancy(int D, int bk, int bv, int kmode, int G, long long rec_bytes, int nstage,
                              int *ctas_per_sm) {
     KernelFn fn = pick_kernel(D, bk, bv, kmode, G);
     if (!fn) return cudaErrorInvalidValue;
-    const size_t smem = decode_smem_bytes(rec_bytes, nstage, D, G);
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, fn, NW * 32, smem);
+    return prepare_kernel(fn, decode_smem_bytes(rec_bytes, nstage, D, G), ctas_per_sm);
 }
 
 cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmode, cudaStream_t st,
@@ -657,9 +737,8 @@ cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmod
     KernelFn fn = pick_kernel(D, bk, bv, kmode, p.G);
     if (!fn) return cudaErrorInvalidValue;
     const size_t smem = decode_smem_bytes(p.rec_bytes, p.nstage, D, p.G);
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = prepare_kernel(fn, smem, ctas_per_sm_out);
     if (e != cudaSuccess) return e;
-    (void)ctas_per_sm_out;
     dim3 grid(p.S, p.Hkv, p.B);
     fn<<<grid, NW * 32, smem, st>>>(p);
     return cudaGetLastError();

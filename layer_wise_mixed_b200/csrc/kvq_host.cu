@@ -21,7 +21,7 @@ struct kvq_handle {
     std::vector<LayerGeom> geom;
     std::vector<int> len;
     int cap_blk = 0;
-    long long status_off = 0, part_acc_off = 0, part_ml_off = 0, total = 0;
+    long long status_off = 0, smax_off = 0, meta_bytes = 0, part_acc_off = 0, part_ml_off = 0, total = 0;
     uint8_t *ws = nullptr;
     size_t ws_bytes = 0;
     int forced_splits = 0;
@@ -67,11 +67,11 @@ int check_bound(const kvq_handle *h) {
 
 int cuda_fail(cudaError_t e, const char *what);
 
-// The status word lives in caller memory of unknown content: zero it on the stream of
-// the first launch after a bind.
+// The status word and the per-layer maximum scales live in caller memory of unknown
+// content: zero them on the stream of the first launch after a bind.
 int prepare_status(kvq_handle *h, cudaStream_t st) {
     if (h->status_clear) return KVQ_OK;
-    cudaError_t e = cudaMemsetAsync(h->ws + h->status_off, 0, 256, st);
+    cudaError_t e = cudaMemsetAsync(h->ws + h->status_off, 0, static_cast<size_t>(h->meta_bytes), st);
     if (e != cudaSuccess) return cuda_fail(e, "status clear");
     h->status_clear = true;
     return KVQ_OK;
@@ -131,8 +131,10 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
     h->desc.layers = nullptr;
     h->cap_blk = (d->max_ctx + 31) / 32;
     const int D = d->head_dim;
-    long long off = 256;   // status word
     h->status_off = 0;
+    h->smax_off = 256;                                      // after the status word
+    h->meta_bytes = align256(256 + 8LL * d->num_layers);   // {K, V} max scale per layer
+    long long off = h->meta_bytes;
     for (int l = 0; l < d->num_layers; ++l) {
         const kvq_layer_cfg &c = h->cfg[l];
         if (!valid_bits(c.bk) || !valid_bits(c.bv)) {
@@ -216,6 +218,7 @@ int kvq_append(kvq_handle *h, int layer, const void *K, const void *V, int n_new
     kvq::AppendParams p{};
     p.K = static_cast<const uint16_t *>(K);
     p.V = static_cast<const uint16_t *>(V);
+    p.smax = reinterpret_cast<unsigned *>(h->ws + h->smax_off) + 2 * layer;
     p.rec = h->ws + g.rec_off;
     p.res = g.res_off >= 0 ? reinterpret_cast<uint16_t *>(h->ws + g.res_off) : nullptr;
     p.B = h->desc.batch;
@@ -291,6 +294,7 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
     p.rec = h->ws + g.rec_off;
     p.res = g.res_off >= 0 ? reinterpret_cast<const uint16_t *>(h->ws + g.res_off) : nullptr;
     p.q = static_cast<const uint16_t *>(q);
+    p.smax = reinterpret_cast<const unsigned *>(h->ws + h->smax_off) + 2 * layer;
     p.out = out;
     p.part_acc = reinterpret_cast<float *>(h->ws + h->part_acc_off);
     p.part_ml = reinterpret_cast<float *>(h->ws + h->part_ml_off);

@@ -24,6 +24,7 @@ struct LayerGeom {
 
 struct AppendParams {
     const uint16_t *K, *V;      // bf16 [B][Hkv][n][D]
+    unsigned *smax;             // this layer's {max key scale, max value scale} (fp16 bits)
     uint8_t *rec;               // layer records [B][Hkv][cap][rec_bytes]
     uint16_t *res;              // residual [B][Hkv][32][D] bf16 (per-channel keys)
     int B, Hkv, D, bk, bv, kmode;
@@ -38,6 +39,7 @@ struct DecodeParams {
     const uint8_t *rec;         // layer records
     const uint16_t *res;        // residual (per-channel keys) or null
     const uint16_t *q;          // bf16 [B][Hq][D]
+    const unsigned *smax;       // this layer's {max key scale, max value scale} (fp16 bits)
     void *out;                  // [B][Hq][D] bf16 or fp32
     float *part_acc;            // [B][Hq][kMaxSplits][D]
     float *part_ml;             // [B][Hq][kMaxSplits][2]  (m in log2 units, l)

@@ -122,10 +122,11 @@ def test_gqa_groups(G, kmode):
 def test_chunked_equals_bulk():
     """Incremental appends (ragged chunks) give the same bytes as the oracle's image of
     the whole sequence, which is also what one bulk append gives."""
+    wl = workload(2, 2, 4, 128, name="chunked-vs-bulk")
     for kmode in (0, 1):
         chunks = [5, 27, 1, 64, 3, 100, 33, 1, 1, 65]
-        c1 = run_case(2, 2, 4, 128, [(4, 2)], kmode, chunks, tag="chunks")
-        c2 = run_case(2, 2, 4, 128, [(4, 2)], kmode, [sum(chunks)], tag="bulk")
+        c1 = run_case(2, 2, 4, 128, [(4, 2)], kmode, chunks, wl=wl, tag="chunks")
+        c2 = run_case(2, 2, 4, 128, [(4, 2)], kmode, [sum(chunks)], wl=wl, tag="bulk")
         assert np.array_equal(c1.export_layer(0), c2.export_layer(0))
 
 
