@@ -30,8 +30,11 @@
  * capacity ceil(max_ctx/32) block records of 32 tokens, then (per-channel keys) a
  * residual of 32 x D bf16.  Record of block beta, D = head_dim, nj = D/32:
  *     [K codes 4*D*bk B][K s/z 4*D B][V codes 4*D*bv B][V s/z 4*D B]
- *   s/z entry = (scale fp16, zero fp16); per-channel K: entry d at 4*d; per-token K
- *   and V: entry (u, j) at 4*(u*nj + j) (u = token in block, j = d/32).
+ *   Scales and zeros are fp16, at byte offsets inside their s/z area:
+ *     per-channel K, channel d: k=d/16, e=d%16, t=(e%8)/2, r=e/8, hb=e%2:
+ *       scale at 16*(4k+t) + 8r + 2hb, zero at +4;
+ *     per-token K and V, token u of the block, group j=d/32:
+ *       scale at 8*nj*(u/2) + 4j + 2*(u%2), zero at +4*nj.
  *   Code areas = two 16-token halves of 2*D*b bytes; token u in half u/16; in the half
  *   each code has a lane (0..31) and a slot:
  *     keys:   i=(u%16)/8, gk=u%8, k=d/16, e=d%16, t=(e%8)/2, r=e/8, hb=e%2,

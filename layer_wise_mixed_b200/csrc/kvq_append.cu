@@ -72,6 +72,15 @@ __device__ __forceinline__ void field_owner(int role, int lane, int w, int f, in
     }
 }
 
+// Byte offsets of a scale/zero pair in the s/z areas of the v1 format.
+__device__ __forceinline__ int chan_sz_off(int d) {   // per-channel keys: scale; zero at +4
+    const int k = d >> 4, e = d & 15;
+    return 16 * (4 * k + ((e & 7) >> 1)) + 8 * (e >> 3) + 2 * (e & 1);
+}
+__device__ __forceinline__ int tok_sz_off(int u, int j, int nj) {   // per token: scale; zero at +4*nj
+    return 8 * nj * (u >> 1) + 4 * j + 2 * (u & 1);
+}
+
 // Memory word index inside a half's code area -> (lane, lane word).
 __device__ __forceinline__ void word_lane(int widx, int Wh, int &lane, int &w) {
     const int c = Wh < 4 ? Wh : 4;
@@ -114,8 +123,9 @@ __device__ void per_token_half(const AppendParams &p, int role, int unit, int hb
             group_params(mn, mx, bits, s, z, s16, z16);
             codes[e][32 * j + lane] = static_cast<uint8_t>(group_code(x, s, z, bits));
             if (lane == 0) {
-                const uint32_t v = static_cast<uint32_t>(s16) | (static_cast<uint32_t>(z16) << 16);
-                *reinterpret_cast<uint32_t *>(sz + 4LL * (u * nj + j)) = v;
+                const int so = tok_sz_off(u, j, nj);
+                *reinterpret_cast<uint16_t *>(sz + so) = s16;
+                *reinterpret_cast<uint16_t *>(sz + so + 4 * nj) = z16;
                 atomicMax(cta_smax, static_cast<unsigned>(s16));
             }
         }
@@ -170,8 +180,9 @@ __device__ void per_channel_group(const AppendParams &p, int unit, int q, bool d
             uint16_t s16, z16;
             group_params(mn, mx, p.bk, s, z, s16, z16);
             for (int u = 0; u < 32; ++u) codes[u][d] = static_cast<uint8_t>(group_code(xs[u][d], s, z, p.bk));
-            *reinterpret_cast<uint32_t *>(rec + p.kc + 4LL * d) =
-                static_cast<uint32_t>(s16) | (static_cast<uint32_t>(z16) << 16);
+            const int so = chan_sz_off(d);
+            *reinterpret_cast<uint16_t *>(rec + p.kc + so) = s16;
+            *reinterpret_cast<uint16_t *>(rec + p.kc + so + 4) = z16;
             atomicMax(cta_smax, static_cast<unsigned>(s16));
         }
         __syncthreads();

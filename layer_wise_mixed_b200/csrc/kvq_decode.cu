@@ -29,6 +29,7 @@
 #include <cuda_fp16.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "kvq_internal.h"
 
@@ -79,7 +80,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned phase) {
 }
 
 __device__ __forceinline__ void mma16816(float *c, const uint32_t *a, uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};\n"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -187,8 +188,12 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t 
     lo = pack_h2(a - ha, b - hb);
 }
 
+// Floats of the per-warp combine buffer: O^T columns [8*NT][D], value zero-point
+// terms [8*NT][NJ], running max and sum per head [8] + [8].
+__host__ __device__ constexpr int comb_floats(int D, int NT) { return 8 * NT * D + 8 * NT * (D / 32) + 16; }
+
 template <int BK, int BV, int KM, int D, int NT>
-__global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(const DecodeParams p) {
     constexpr int KS = D / 16;     // 16-channel steps (QK) / 16-channel row tiles (PV)
     constexpr int NJ = D / 32;     // channel groups
     constexpr int WHK = D * BK / 64, WHV = D * BV / 64;
@@ -208,9 +213,11 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
 
     uint8_t *stages = smem + static_cast<size_t>(warp) * NS * REC;
     const size_t stage_bytes = static_cast<size_t>(NW) * NS * REC;
-    const size_t comb_bytes = static_cast<size_t>(NW) * (8 * NT * D + 8 * (2 + NJ)) * 4;
+    const size_t comb_bytes = static_cast<size_t>(NW) * comb_floats(D, NT) * 4;
     const size_t bar_off = ((stage_bytes > comb_bytes ? stage_bytes : comb_bytes) + 127) & ~size_t(127);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + bar_off) + warp * NS;
+    // q operand fragments, identical for the CTA's warps: [KS][32 lanes] x uint4
+    uint4 *aq_s = reinterpret_cast<uint4 *>(smem + bar_off + static_cast<size_t>(NW) * NS * 8 + 8 * ((NW * NS) & 1));
     const uint8_t *unit_rec = p.rec + (static_cast<long long>(b) * p.Hkv + h) * p.cap_blk * REC;
 
     const int nb = (blk1 - blk0 > warp) ? (blk1 - blk0 - warp + NW - 1) / NW : 0;
@@ -219,21 +226,19 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
         fence_mbar_init();
     }
     __syncwarp();
-    int issued = 0;
+    int issued = min(NS, nb);   // copies issued so far (every lane keeps the count)
     if (lane == 0) {
-        for (; issued < NS && issued < nb; ++issued) {
-            mbar_expect_tx(&bars[issued], REC);
-            bulk_g2s(stages + issued * REC, unit_rec + static_cast<long long>(blk0 + warp + NW * issued) * REC,
-                     REC, &bars[issued]);
+        for (int k = 0; k < issued; ++k) {
+            mbar_expect_tx(&bars[k], REC);
+            bulk_g2s(stages + k * REC, unit_rec + static_cast<long long>(blk0 + warp + NW * k) * REC, REC, &bars[k]);
         }
     }
-    issued = __shfl_sync(0xffffffffu, issued, 0);
 
     // ---- operand prescales (powers of two) from the layer's largest scales ----
     const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
     const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
     // values: p * 2^kp * s_v stays below 2^14 in fp16
-    const int kp = smax_v > 0.f ? max(-24, min(14, 14 - floor_log2(smax_v) - 1)) : 14;
+    const int kp = smax_v > 0.f ? max(-24, min(14, 13 - floor_log2(smax_v))) : 14;
 
     // ---- this thread's query head and channels (16k + 2t + {0, 1, 8, 9}) ----
     const int hh = g % G;
@@ -253,8 +258,8 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
     // Per-channel keys: q~ = q log2(e)/sqrt(D) 2^kq as fp16 hi/lo fragments (rows g: hi,
     // g+8: lo), kq chosen so that q~ s_k stays below 2^14 and q~ below 2^15.
     // Per-token keys: raw q (exact in fp16), rows (group j, head) masked to group j.
-    uint32_t aq[KS][4];
-    float unscale = 1.f;                 // scores = accumulators * unscale
+    uint32_t aq[KS][4];                  // built here, then kept in shared memory (aq_s)
+    float unscale = 1.f;                 // true score (log2 units) = raw * unscale
     float qsum_g = 0.f, qsum_g8 = 0.f;   // per-token keys: sum of q over the rows' groups
     const int jg = g / G, jg8 = (g + 8) / G;
     const bool row_g = (KM == 1) && (g < G * NJ), row_g8 = (KM == 1) && (g + 8 < G * NJ);
@@ -268,11 +273,11 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
         int kq = 0;
         if (amax > 0.f) {
-            kq = 14 - floor_log2(amax);                              // q~ < 2^15
-            if (smax_k > 0.f) kq = min(kq, 13 - floor_log2(amax) - floor_log2(smax_k) - 1);   // q~ s < 2^14
+            kq = 14 - floor_log2(amax);                                            // q~ < 2^15
+            if (smax_k > 0.f) kq = min(kq, 12 - floor_log2(amax) - floor_log2(smax_k));   // q~ s < 2^14
             kq = max(-60, min(60, kq));
         }
-        const float sc = qscale * pow2f(kq > 0 ? min(kq, 126) : max(kq, -126));
+        const float sc = qscale * pow2f(kq);
         unscale = pow2f(-kq);
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
@@ -302,80 +307,51 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
         }
         unscale = qscale;
     }
+    if (warp == 0) {
+#pragma unroll
+        for (int k = 0; k < KS; ++k) aq_s[k * 32 + lane] = make_uint4(aq[k][0], aq[k][1], aq[k][2], aq[k][3]);
+    }
+    __syncthreads();
 
     float m_run = -INFINITY, l_run = 0.f;
-    float zacc[NJ];
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) zacc[j] = 0.f;
     float oacc[KS][NT][4];
+    float zc[NT][4];     // value zero-point term: rows = channel group j (= g), cols as oacc
 #pragma unroll
-    for (int m = 0; m < KS; ++m)
+    for (int n = 0; n < NT; ++n) {
 #pragma unroll
-        for (int n = 0; n < NT; ++n)
+        for (int c = 0; c < 4; ++c) zc[n][c] = 0.f;
+#pragma unroll
+        for (int m = 0; m < KS; ++m)
 #pragma unroll
             for (int c = 0; c < 4; ++c) oacc[m][n][c] = 0.f;
+    }
 
     // B-operand column of this thread for P: NT == 1: hi (g < G), lo (G <= g < 2G) or
     // zero; NT == 2: tile 0 hi, tile 1 lo for g < G.
-    const uint32_t m_hi = ((NT == 1 && g < G) || (NT == 2 && g < G)) ? 0xFFFFFFFFu : 0u;
+    const uint32_t m_hi = (g < G) ? 0xFFFFFFFFu : 0u;
     const uint32_t m_lo = (NT == 1 && g >= G && g < 2 * G) ? 0xFFFFFFFFu : 0u;
     const int alpha_src0 = 4 * ((NT == 1) ? ((2 * t) % G) : min(2 * t, 7));
     const int alpha_src1 = 4 * ((NT == 1) ? ((2 * t + 1) % G) : min(2 * t + 1, 7));
     const float pbias = static_cast<float>(kp);
+    const int jz = g < NJ ? g : NJ - 1;
 
-    bool failed = false;
-    int i = 0;
-    for (; i < nb; ++i) {
-        const int blk = blk0 + warp + NW * i;
-        const int st = i % NS;
-        if (!mbar_wait(&bars[st], (i / NS) & 1)) {
-            failed = true;
-            break;
-        }
-        const uint8_t *R = stages + st * REC;
-        const bool tail = blk == tail_blk;
-        const int valid = tail ? rem : 32;
-
-        // ================= scores S^T (rows: heads, columns: 8-token tiles) =================
+    // ------------------------------------------------------------ one 32-token block
+    auto body = [&](auto tail_tag, const uint8_t *R, const int valid) {
+        constexpr bool TAIL = decltype(tail_tag)::value;
+        // ===== scores S^T (rows: heads, columns: 8-token tiles) =====
         float acc[4][4];
 #pragma unroll
         for (int n = 0; n < 4; ++n)
 #pragma unroll
             for (int c = 0; c < 4; ++c) acc[n][c] = 0.f;
         float czacc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (KM == 1 || !tail) {
-            uint32_t kw[2][WHK];
-            load_lane_words<WHK>(R, lane, kw[0]);
-            load_lane_words<WHK>(R + 2 * D * BK, lane, kw[1]);
-#pragma unroll
-            for (int k = 0; k < KS; ++k) {
-                uint32_t a[4];
-                if constexpr (KM == 0) {
-                    const uint2 sz0 = *reinterpret_cast<const uint2 *>(R + KC + 4 * (16 * k + 2 * t));
-                    const uint2 sz8 = *reinterpret_cast<const uint2 *>(R + KC + 4 * (16 * k + 2 * t + 8));
-                    const uint32_t s01 = prmt(sz0.x, sz0.y, 0x5410u), z01 = prmt(sz0.x, sz0.y, 0x7632u);
-                    const uint32_t s89 = prmt(sz8.x, sz8.y, 0x5410u), z89 = prmt(sz8.x, sz8.y, 0x7632u);
-                    mul_hilo(aq[k][0], aq[k][1], s01, a[0], a[1]);
-                    mul_hilo(aq[k][2], aq[k][3], s89, a[2], a[3]);
-                    mma16816(czacc, aq[k], z01, z89);   // sum_d q~_d z_d, same in every column
-                } else {
-                    a[0] = aq[k][0];
-                    a[1] = aq[k][1];
-                    a[2] = aq[k][2];
-                    a[3] = aq[k][3];
-                }
-#pragma unroll
-                for (int n = 0; n < 4; ++n) {
-                    const int s0 = (2 * k + (n & 1)) * 2;
-                    const uint32_t w = kw[n >> 1][s0 / PK];
-                    mma16816(acc[n], a, unpack<BK>(w, s0 % PK), unpack<BK>(w, s0 % PK + 1));
-                }
-            }
-        } else {
-            // bf16 residual keys of the last, incomplete group (per-channel layers)
+        if constexpr (KM == 0 && TAIL) {
+            // bf16 residual keys of the last, incomplete group
             const uint16_t *res = p.res + (static_cast<long long>(b) * p.Hkv + h) * 32 * D;
 #pragma unroll
             for (int k = 0; k < KS; ++k) {
+                const uint4 aqv = aq_s[k * 32 + lane];
+                const uint32_t ak[4] = {aqv.x, aqv.y, aqv.z, aqv.w};
 #pragma unroll
                 for (int n = 0; n < 4; ++n) {
                     const int u = 8 * n + g;
@@ -386,55 +362,99 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
                         b0 = pack_h2(__uint_as_float(r0 << 16), __uint_as_float(r0 & 0xFFFF0000u));
                         b1 = pack_h2(__uint_as_float(r8 << 16), __uint_as_float(r8 & 0xFFFF0000u));
                     }
-                    mma16816(acc[n], aq[k], b0, b1);
+                    mma16816(acc[n], ak, b0, b1);
+                }
+            }
+        } else {
+            // key words of k-step k: slots 4k..4k+3 of each half, lane word (4k + x) / PK
+            constexpr int WPK = PK >= 4 ? 1 : 4 / PK;   // words per k-step and half
+            constexpr int CH = WHK < 4 ? WHK : 4;        // lane words per chunk
+#pragma unroll
+            for (int k = 0; k < KS; ++k) {
+                uint32_t kw0[WPK], kw1[WPK];
+                const int w0 = (4 * k) / PK;
+#pragma unroll
+                for (int x = 0; x < WPK; ++x) {
+                    const int w = w0 + x;
+                    const int off = (((w / CH) * 32 + lane) * CH + (w % CH)) * 4;
+                    kw0[x] = *reinterpret_cast<const uint32_t *>(R + off);
+                    kw1[x] = *reinterpret_cast<const uint32_t *>(R + 2 * D * BK + off);
+                }
+                const uint4 aqv = aq_s[k * 32 + lane];
+                const uint32_t ak[4] = {aqv.x, aqv.y, aqv.z, aqv.w};
+                uint32_t a[4];
+                if constexpr (KM == 0) {
+                    // scales/zeros of channels (16k+2t, +1) and (16k+2t+8, +9) as half2
+                    const uint4 sz = *reinterpret_cast<const uint4 *>(R + KC + 16 * (4 * k + t));
+                    mul_hilo(ak[0], ak[1], sz.x, a[0], a[1]);
+                    mul_hilo(ak[2], ak[3], sz.z, a[2], a[3]);
+                    mma16816(czacc, ak, sz.y, sz.w);   // sum_d q~_d z_d, same in every column
+                } else {
+                    a[0] = ak[0];
+                    a[1] = ak[1];
+                    a[2] = ak[2];
+                    a[3] = ak[3];
+                }
+#pragma unroll
+                for (int n = 0; n < 4; ++n) {
+                    const int s0 = (2 * k + (n & 1)) * 2;
+                    const int wl = s0 / PK - w0;
+                    const uint32_t w = (n >> 1) ? kw1[wl] : kw0[wl];
+                    mma16816(acc[n], a, unpack<BK>(w, s0 % PK), unpack<BK>(w, s0 % PK + 1));
                 }
             }
         }
 
-        float sc[4][2];
+        float raw[4][2];
         if constexpr (KM == 0) {
             const float cz = czacc[0] + czacc[2];
 #pragma unroll
             for (int n = 0; n < 4; ++n) {
-                sc[n][0] = (acc[n][0] + acc[n][2] + cz) * unscale;
-                sc[n][1] = (acc[n][1] + acc[n][3] + cz) * unscale;
+                raw[n][0] = acc[n][0] + acc[n][2] + cz;
+                raw[n][1] = acc[n][1] + acc[n][3] + cz;
             }
         } else {
-            // per-token key scales, then sum the (group, head) rows of each head
+            // per-token key scales on the (group, head) rows, then sum the rows of a head
+            const uint8_t *ks = R + KC;
 #pragma unroll
             for (int n = 0; n < 4; ++n) {
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const int u = 8 * n + 2 * t + c;
-                    float v = 0.f;
-                    if (row_g) {
-                        const uint32_t e = *reinterpret_cast<const uint32_t *>(R + KC + 4 * (u * NJ + jg));
-                        v = fmaf(half_lo_f(e), acc[n][c], half_hi_f(e) * qsum_g);
-                    }
-                    if (row_g8) {
-                        const uint32_t e = *reinterpret_cast<const uint32_t *>(R + KC + 4 * (u * NJ + jg8));
-                        v += fmaf(half_lo_f(e), acc[n][2 + c], half_hi_f(e) * qsum_g8);
-                    }
-#pragma unroll
-                    for (int msk = G; msk < 8; msk <<= 1) v += __shfl_xor_sync(0xffffffffu, v, 4 * msk);
-                    sc[n][c] = v * unscale;
+                const int pi = 4 * n + t;   // token pair (8n + 2t, 8n + 2t + 1)
+                float v0 = 0.f, v1 = 0.f;
+                if (row_g) {
+                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * jg);
+                    const uint32_t zw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * NJ + 4 * jg);
+                    v0 = fmaf(half_lo_f(sw), acc[n][0], half_lo_f(zw) * qsum_g);
+                    v1 = fmaf(half_hi_f(sw), acc[n][1], half_hi_f(zw) * qsum_g);
                 }
+                if (row_g8) {
+                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * jg8);
+                    const uint32_t zw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * NJ + 4 * jg8);
+                    v0 += fmaf(half_lo_f(sw), acc[n][2], half_lo_f(zw) * qsum_g8);
+                    v1 += fmaf(half_hi_f(sw), acc[n][3], half_hi_f(zw) * qsum_g8);
+                }
+#pragma unroll
+                for (int msk = G; msk < 8; msk <<= 1) {
+                    v0 += __shfl_xor_sync(0xffffffffu, v0, 4 * msk);
+                    v1 += __shfl_xor_sync(0xffffffffu, v1, 4 * msk);
+                }
+                raw[n][0] = v0;
+                raw[n][1] = v1;
             }
         }
-        if (tail) {
+        if constexpr (TAIL) {
 #pragma unroll
             for (int n = 0; n < 4; ++n)
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
-                    if (8 * n + 2 * t + c >= valid) sc[n][c] = -INFINITY;
+                    if (8 * n + 2 * t + c >= valid) raw[n][c] = -INFINITY;
         }
 
-        // ================= online softmax (base 2; p carries the factor 2^kp) =================
-        float mloc = fmaxf(fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1])),
-                           fmaxf(fmaxf(sc[2][0], sc[2][1]), fmaxf(sc[3][0], sc[3][1])));
+        // ===== online softmax (base 2; p carries the factor 2^kp) =====
+        float mloc = fmaxf(fmaxf(fmaxf(raw[0][0], raw[0][1]), fmaxf(raw[1][0], raw[1][1])),
+                           fmaxf(fmaxf(raw[2][0], raw[2][1]), fmaxf(raw[3][0], raw[3][1])));
         mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
         mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-        const float m_new = fmaxf(m_run, mloc);
+        const float m_new = fmaxf(m_run, mloc * unscale);
         const float alpha = fast_exp2(m_run - m_new);
         m_run = m_new;
         const float shift = pbias - m_new;
@@ -444,77 +464,80 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
         for (int n = 0; n < 4; ++n)
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                pr[n][c] = fast_exp2(sc[n][c] + shift);
+                pr[n][c] = fast_exp2(fmaf(raw[n][c], unscale, shift));
                 psum += pr[n][c];
             }
         l_run = fmaf(l_run, alpha, psum);
         if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll
-            for (int j = 0; j < NJ; ++j) zacc[j] *= alpha;
             const float a0 = __shfl_sync(0xffffffffu, alpha, alpha_src0);
             const float a1 = __shfl_sync(0xffffffffu, alpha, alpha_src1);
 #pragma unroll
-            for (int m = 0; m < KS; ++m)
+            for (int n = 0; n < NT; ++n) {
+                zc[n][0] *= a0;
+                zc[n][1] *= a1;
 #pragma unroll
-                for (int n = 0; n < NT; ++n) {
+                for (int m = 0; m < KS; ++m) {
                     oacc[m][n][0] *= a0;
                     oacc[m][n][1] *= a1;
                     oacc[m][n][2] *= a0;
                     oacc[m][n][3] *= a1;
                 }
+            }
         }
 
-        // ================= O^T += V^T P'^T (two 16-token steps) =================
+        // ===== O^T += V^T P'^T and the zero-point term (two 16-token steps) =====
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) {
             uint32_t vw[WHV];
             load_lane_words<WHV>(R + KC + KSZ + kk * 2 * D * BV, lane, vw);
-            // tokens 16kk + 2t + {0,1} (pair A) and 16kk + 8 + 2t + {0,1} (pair B)
-            const float pa0 = pr[2 * kk][0], pa1 = pr[2 * kk][1];
-            const float pb0 = pr[2 * kk + 1][0], pb1 = pr[2 * kk + 1][1];
-            uint32_t pah, pal, pbh, pbl;
-            split2(pa0, pa1, pah, pal);
-            split2(pb0, pb1, pbh, pbl);
-            uint32_t wa0[NJ], wa1[NJ], wb0[NJ], wb1[NJ];
-            {
-                const uint8_t *vs = R + KC + KSZ + VC;
-                const int u0 = 16 * kk + 2 * t;
-                if constexpr (NJ == 4) {
-                    const uint4 x0 = *reinterpret_cast<const uint4 *>(vs + 16 * u0);
-                    const uint4 x1 = *reinterpret_cast<const uint4 *>(vs + 16 * (u0 + 1));
-                    const uint4 x2 = *reinterpret_cast<const uint4 *>(vs + 16 * (u0 + 8));
-                    const uint4 x3 = *reinterpret_cast<const uint4 *>(vs + 16 * (u0 + 9));
-                    wa0[0] = x0.x; wa0[1] = x0.y; wa0[2] = x0.z; wa0[3] = x0.w;
-                    wa1[0] = x1.x; wa1[1] = x1.y; wa1[2] = x1.z; wa1[3] = x1.w;
-                    wb0[0] = x2.x; wb0[1] = x2.y; wb0[2] = x2.z; wb0[3] = x2.w;
-                    wb1[0] = x3.x; wb1[1] = x3.y; wb1[2] = x3.z; wb1[3] = x3.w;
-                } else {
+            uint32_t pah, pal, pbh, pbl;   // p of token pairs A (16kk+2t, +1) and B (+8, +9)
+            split2(pr[2 * kk][0], pr[2 * kk][1], pah, pal);
+            split2(pr[2 * kk + 1][0], pr[2 * kk + 1][1], pbh, pbl);
+            const uint8_t *vs = R + KC + KSZ + VC;
+            const int iA = 8 * kk + t, iB = iA + 4;
+            uint32_t sA[NJ], sB[NJ];
+            if constexpr (NJ == 4) {
+                const uint4 xa = *reinterpret_cast<const uint4 *>(vs + 8 * NJ * iA);
+                const uint4 xb = *reinterpret_cast<const uint4 *>(vs + 8 * NJ * iB);
+                sA[0] = xa.x; sA[1] = xa.y; sA[2] = xa.z; sA[3] = xa.w;
+                sB[0] = xb.x; sB[1] = xb.y; sB[2] = xb.z; sB[3] = xb.w;
+            } else {
 #pragma unroll
-                    for (int j = 0; j < NJ; ++j) {
-                        wa0[j] = reinterpret_cast<const uint32_t *>(vs + 4 * NJ * u0)[j];
-                        wa1[j] = reinterpret_cast<const uint32_t *>(vs + 4 * NJ * (u0 + 1))[j];
-                        wb0[j] = reinterpret_cast<const uint32_t *>(vs + 4 * NJ * (u0 + 8))[j];
-                        wb1[j] = reinterpret_cast<const uint32_t *>(vs + 4 * NJ * (u0 + 9))[j];
-                    }
+                for (int j = 0; j < NJ; ++j) {
+                    sA[j] = reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iA)[j];
+                    sB[j] = reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iB)[j];
+                }
+            }
+            uint32_t zA = *reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iA + 4 * NJ + 4 * jz);
+            uint32_t zB = *reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iB + 4 * NJ + 4 * jz);
+            if constexpr (TAIL) {
+                // absent tokens: p = 0 and their scale/zero halves may hold anything
+                const int u0 = 16 * kk + 2 * t;
+                const uint32_t mA = (u0 < valid ? 0x0000FFFFu : 0u) | (u0 + 1 < valid ? 0xFFFF0000u : 0u);
+                const uint32_t mB = (u0 + 8 < valid ? 0x0000FFFFu : 0u) | (u0 + 9 < valid ? 0xFFFF0000u : 0u);
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+                    sA[j] &= mA;
+                    sB[j] &= mB;
+                }
+                zA &= mA;
+                zB &= mB;
+            }
+            // zero-point term: rows j = g of Z^T (tokens as columns) times the P columns
+            {
+                const uint32_t az[4] = {g < NJ ? zA : 0u, 0u, g < NJ ? zB : 0u, 0u};
+                if constexpr (NT == 1) {
+                    mma16816(zc[0], az, (pah & m_hi) | (pal & m_lo), (pbh & m_hi) | (pbl & m_lo));
+                } else {
+                    mma16816(zc[0], az, pah & m_hi, pbh & m_hi);
+                    mma16816(zc[1], az, pal & m_hi, pbl & m_hi);
                 }
             }
 #pragma unroll
             for (int j = 0; j < NJ; ++j) {
-                uint32_t sa = prmt(wa0[j], wa1[j], 0x5410u), sb = prmt(wb0[j], wb1[j], 0x5410u);
-                float za0 = half_hi_f(wa0[j]), za1 = half_hi_f(wa1[j]);
-                float zb0 = half_hi_f(wb0[j]), zb1 = half_hi_f(wb1[j]);
-                if (tail) {
-                    // absent tokens: p = 0, and their scale/zero words may hold anything
-                    const int u0 = 16 * kk + 2 * t;
-                    if (u0 >= valid) { sa &= 0xFFFF0000u; za0 = 0.f; }
-                    if (u0 + 1 >= valid) { sa &= 0x0000FFFFu; za1 = 0.f; }
-                    if (u0 + 8 >= valid) { sb &= 0xFFFF0000u; zb0 = 0.f; }
-                    if (u0 + 9 >= valid) { sb &= 0x0000FFFFu; zb1 = 0.f; }
-                }
-                zacc[j] = fmaf(pa0, za0, fmaf(pa1, za1, fmaf(pb0, zb0, fmaf(pb1, zb1, zacc[j]))));
                 uint32_t ah, al, bh, bl;
-                mul_hilo(pah, pal, sa, ah, al);
-                mul_hilo(pbh, pbl, sb, bh, bl);
+                mul_hilo(pah, pal, sA[j], ah, al);
+                mul_hilo(pbh, pbl, sB[j], bh, bl);
                 uint32_t b0, b1, c0 = 0u, c1 = 0u;
                 if constexpr (NT == 1) {
                     b0 = (ah & m_hi) | (al & m_lo);
@@ -539,16 +562,46 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
                 }
             }
         }
+    };
 
+    // ------------------------------------------------------------ main loop
+    const bool has_tail = tail_blk >= blk0 && tail_blk < blk1 && ((tail_blk - blk0) % NW) == warp;
+    const int nb_main = nb - (has_tail ? 1 : 0);
+    int st = 0;
+    unsigned ph = 0;
+    bool failed = false;
+    int i = 0;
+    auto refill = [&]() {
         __syncwarp();
-        if (lane == 0 && issued < nb) {
-            fence_proxy_async();
-            const int ni = issued++;
-            mbar_expect_tx(&bars[st], REC);
-            bulk_g2s(stages + st * REC, unit_rec + static_cast<long long>(blk0 + warp + NW * ni) * REC, REC,
-                     &bars[st]);
+        if (issued < nb) {
+            if (lane == 0) {
+                fence_proxy_async();
+                mbar_expect_tx(&bars[st], REC);
+                bulk_g2s(stages + st * REC, unit_rec + static_cast<long long>(blk0 + warp + NW * issued) * REC, REC,
+                         &bars[st]);
+            }
+            ++issued;
         }
-        issued = __shfl_sync(0xffffffffu, issued, 0);
+        if (++st == NS) {
+            st = 0;
+            ph ^= 1u;
+        }
+    };
+    for (; i < nb_main; ++i) {
+        if (!mbar_wait(&bars[st], ph)) {
+            failed = true;
+            break;
+        }
+        body(std::false_type{}, stages + st * REC, 32);
+        refill();
+    }
+    if (!failed && has_tail) {
+        if (!mbar_wait(&bars[st], ph)) {
+            failed = true;
+        } else {
+            body(std::true_type{}, stages + st * REC, rem);
+            ++i;
+        }
     }
     if (failed) {
         // drain the copies still in flight (bounded), then report
@@ -559,18 +612,12 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
     // ================= combine the warps of this split =================
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-        zacc[j] += __shfl_xor_sync(0xffffffffu, zacc[j], 1);
-        zacc[j] += __shfl_xor_sync(0xffffffffu, zacc[j], 2);
-    }
     __syncthreads();   // every warp is done with its stages
-    float *obuf = reinterpret_cast<float *>(smem);                 // [NW][8*NT][D]
-    float *mbuf = obuf + NW * 8 * NT * D;                          // [NW][8]
-    float *lbuf = mbuf + NW * 8;                                   // [NW][8]
-    float *zbuf = lbuf + NW * 8;                                   // [NW][8][NJ]
+    constexpr int CF = comb_floats(D, NT);
     {
-        float *ob = obuf + warp * 8 * NT * D;
+        float *ob = reinterpret_cast<float *>(smem) + warp * CF;   // [8*NT][D]
+        float *zb = ob + 8 * NT * D;                                // [8*NT][NJ]
+        float *ml = zb + 8 * NT * NJ;                               // m[8], l[8]
 #pragma unroll
         for (int m = 0; m < KS; ++m)
 #pragma unroll
@@ -581,30 +628,38 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_split_kernel(const DecodePa
                 ob[c0 * D + d0 + 8] = oacc[m][n][2];
                 ob[(c0 + 1) * D + d0 + 8] = oacc[m][n][3];
             }
-        if (t == 0 && g < G) {
-            mbuf[warp * 8 + g] = (nb > 0 && !failed) ? m_run : -INFINITY;
-            lbuf[warp * 8 + g] = l_run;
+        if (g < NJ) {
 #pragma unroll
-            for (int j = 0; j < NJ; ++j) zbuf[(warp * 8 + g) * NJ + j] = zacc[j];
+            for (int n = 0; n < NT; ++n) {
+                zb[(8 * n + 2 * t) * NJ + g] = zc[n][0];
+                zb[(8 * n + 2 * t + 1) * NJ + g] = zc[n][1];
+            }
+        }
+        if (t == 0 && g < G) {
+            ml[g] = (nb > 0 && !failed) ? m_run : -INFINITY;
+            ml[8 + g] = l_run;
         }
     }
     __syncthreads();
     const int Hq = p.Hkv * G;
     for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
         const int hd = idx / D, d = idx % D;
+        const int chi = hd, clo = (NT == 1) ? hd + G : 8 + hd;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, mbuf[w * 8 + hd]);
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, reinterpret_cast<const float *>(smem)[w * CF + 8 * NT * D + 8 * NT * NJ + hd]);
         float val = 0.f, den = 0.f;
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
-            const float mw = mbuf[w * 8 + hd];
+            const float *ob = reinterpret_cast<const float *>(smem) + w * CF;
+            const float *zb = ob + 8 * NT * D;
+            const float *ml = zb + 8 * NT * NJ;
+            const float mw = ml[hd];
             if (mw == -INFINITY) continue;
             const float wt = fast_exp2(mw - M);
-            const float *ob = obuf + w * 8 * NT * D;
-            const float o = (NT == 1) ? ob[hd * D + d] + ob[(hd + G) * D + d] : ob[hd * D + d] + ob[(8 + hd) * D + d];
-            val = fmaf(wt, o + zbuf[(w * 8 + hd) * NJ + d / 32], val);
-            den = fmaf(wt, lbuf[w * 8 + hd], den);
+            const float o = (ob[chi * D + d] + ob[clo * D + d]) + (zb[chi * NJ + d / 32] + zb[clo * NJ + d / 32]);
+            val = fmaf(wt, o, val);
+            den = fmaf(wt, ml[8 + hd], den);
         }
         const long long row = static_cast<long long>(b) * Hq + h * G + hd;
         if (p.S == 1) {
@@ -672,19 +727,25 @@ KernelFn pick_kernel(int D, int bk, int bv, int kmode, int G) {
 
 }  // namespace
 
-int decode_stages(long long rec_bytes) {
-    long long ns = 65536 / (NW * rec_bytes);
-    if (ns < 2) ns = 2;
-    if (ns > 6) ns = 6;
-    return static_cast<int>(ns);
+// Stages per warp: as many as fit when the CTAs that registers allow per SM (4 for
+// G <= 4, else 3) share the SM's 228 KB of shared memory; at least 2 (fewer CTAs then
+// fit), at most 6.
+int decode_stages(long long rec_bytes, int D, int G) {
+    const long long fixed = 1024 + (D / 16) * 32 * 16 + 64;   // per-CTA reserve, q fragments, barriers
+    for (int ctas = (G <= 4 ? 4 : 3); ctas >= 1; --ctas) {
+        const long long ns = (228LL * 1024 / ctas - fixed) / (NW * rec_bytes);
+        if (ns >= 2) return static_cast<int>(ns > 6 ? 6 : ns);
+    }
+    return 2;
 }
 
 size_t decode_smem_bytes(long long rec_bytes, int nstage, int D, int G) {
     const int NT = G <= 4 ? 1 : 2;
     const size_t stage = static_cast<size_t>(NW) * nstage * rec_bytes;
-    const size_t comb = static_cast<size_t>(NW) * (8 * NT * D + 8 * (2 + D / 32)) * 4;
+    const size_t comb = static_cast<size_t>(NW) * comb_floats(D, NT) * 4;
     const size_t base = ((stage > comb ? stage : comb) + 127) & ~size_t(127);
-    return base + static_cast<size_t>(NW) * nstage * 8;
+    const size_t bars = static_cast<size_t>(NW) * nstage * 8 + 8 * ((NW * nstage) & 1);   // keeps 16-B alignment
+    return base + bars + static_cast<size_t>(D / 16) * 32 * 16;
 }
 
 // Per-kernel cache of the dynamic shared-memory attribute and occupancy, so launches

@@ -266,7 +266,7 @@ static int splits_for(kvq_handle *h, int layer, int *S_out, int *nstage_out) {
     const int L = h->len[layer];
     const int nblk = (L + 31) / 32;
     const int G = h->desc.n_q_heads / h->desc.n_kv_heads;
-    const int nstage = kvq::decode_stages(g.rec_bytes);
+    const int nstage = kvq::decode_stages(g.rec_bytes, h->desc.head_dim, G);
     int rc = ensure_device_info(h);
     if (rc) return rc;
     int per_sm = 1;
@@ -390,14 +390,23 @@ int kvq_export_layer(const kvq_handle *h, int layer, void *host_buf, size_t byte
         if (r) {
             // zero every byte of the last block that holds no token of 0..L-1
             uint8_t *tail = img + (nblk - 1) * g.rec_bytes;
+            // per-token scale/zero of token u, group j: 8*nj*(u/2) + 4j + 2(u%2), zero +4*nj
+            auto zero_tok_sz = [&](uint8_t *area) {
+                for (int u = r; u < 32; ++u)
+                    for (int j = 0; j < nj; ++j) {
+                        const long long so = 8LL * nj * (u / 2) + 4LL * j + 2LL * (u % 2);
+                        std::memset(area + so, 0, 2);
+                        std::memset(area + so + 4LL * nj, 0, 2);
+                    }
+            };
             if (g.kmode == KVQ_PER_CHANNEL) {
                 std::memset(tail, 0, g.kc + g.ks);
             } else {
                 if (r <= 16) std::memset(tail + 2LL * D * g.bk, 0, 2LL * D * g.bk);
-                std::memset(tail + g.kc + 4LL * r * nj, 0, g.ks - 4LL * r * nj);
+                zero_tok_sz(tail + g.kc);
             }
             if (r <= 16) std::memset(tail + g.kc + g.ks + 2LL * D * g.bv, 0, 2LL * D * g.bv);
-            std::memset(tail + g.kc + g.ks + g.vc + 4LL * r * nj, 0, g.vs - 4LL * r * nj);
+            zero_tok_sz(tail + g.kc + g.ks + g.vc);
         }
     }
     return ok();

@@ -62,7 +62,7 @@ cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmod
 cudaError_t decode_occupancy(int D, int bk, int bv, int kmode, int G, long long rec_bytes,
                              int nstage, int *ctas_per_sm);
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t st);
-int decode_stages(long long rec_bytes);
+int decode_stages(long long rec_bytes, int D, int G);
 size_t decode_smem_bytes(long long rec_bytes, int nstage, int D, int G);
 
 }  // namespace kvq

@@ -52,6 +52,8 @@ def lib():
         L.orc_get_code.argtypes = [P, i32, i32, i32, i32, i32]
         L.orc_code_position.restype = None
         L.orc_code_position.argtypes = [i32, i32, i32, i32, i32, P, P]
+        L.orc_sz_position.restype = None
+        L.orc_sz_position.argtypes = [i32, i32, i32, i32, P, P]
         L.orc_unit.restype = i32
         L.orc_unit.argtypes = [P, P, i32, i32, i32, i32, i32, P, P, P]
         L.orc_attention_partial.restype = None
@@ -137,6 +139,15 @@ def code_position(role: int, u: int, d: int, D: int, bits: int):
     t = ctypes.c_int()
     lib().orc_code_position(role, u, d, D, bits, ctypes.byref(b), ctypes.byref(t))
     return b.value, t.value
+
+
+def sz_position(kind: int, index: int, j: int, nj: int):
+    """(scale offset, zero offset) inside an s/z area: kind 0 per-channel (index =
+    channel), kind 1 per-token (index = token in block, j = channel group)."""
+    so = ctypes.c_long()
+    zo = ctypes.c_long()
+    lib().orc_sz_position(kind, index, j, nj, ctypes.byref(so), ctypes.byref(zo))
+    return so.value, zo.value
 
 
 # ---------------------------------------------------------------- units / layers

@@ -48,10 +48,11 @@
  *     Per (batch b, kv head h) the cache is a sequence of 32-token block records.
  *     Record of block beta (tokens 32*beta .. 32*beta+31), D = head_dim, nj = D/32:
  *        [K codes: 4*D*bk bytes][K s/z: 4*D bytes][V codes: 4*D*bv][V s/z: 4*D]
- *     s/z entries are (scale fp16, zero fp16) pairs, 4 bytes:
- *        per-channel K: entry d (channel) at 4*d
- *        per-token K and V: entry (u, j) at 4*(u*nj + j), u = token in block,
- *                           j = channel group d/32
+ *     Scales and zeros are fp16, placed (byte offsets inside their s/z area):
+ *        per-channel K, channel d: k = d/16, e = d%16, t = (e%8)/2, r = e/8, hb = e%2:
+ *           scale at 16*(4k + t) + 8r + 2hb, zero at that + 4
+ *        per-token K and V, token u of the block, channel group j = d/32:
+ *           scale at 8*nj*(u/2) + 4j + 2*(u%2), zero at that + 4*nj
  *     Code areas are two 16-token halves of 2*D*b bytes each.  Token u of the
  *     block lies in half eta = u/16.  Inside a half, every code belongs to one of
  *     32 "lanes" and one half-word "slot" of that lane:
@@ -226,9 +227,38 @@ unsigned orc_get_code(const uint8_t *area, int role, int u, int d, int D, int bi
     return (w >> bit) & ((1u << bits) - 1u);
 }
 
-static void put_sz(uint8_t *p, uint16_t s, uint16_t z) {
-    memcpy(p, &s, 2);
-    memcpy(p + 2, &z, 2);
+/* Offsets of the scale and zero of channel d (per-channel key s/z area). */
+static void orc_chan_sz_pos(int d, long *s_off, long *z_off) {
+    int k = d / 16, e = d % 16, t = (e % 8) / 2, r = e / 8, hb = e % 2;
+    *s_off = 16L * (4 * k + t) + 8 * r + 2 * hb;
+    *z_off = *s_off + 4;
+}
+
+/* Offsets of the scale and zero of token u, channel group j (per-token s/z area). */
+static void orc_tok_sz_pos(int u, int j, int nj, long *s_off, long *z_off) {
+    *s_off = 8L * nj * (u / 2) + 4 * j + 2 * (u % 2);
+    *z_off = *s_off + 4L * nj;
+}
+
+static void put_chan_sz(uint8_t *area, int d, uint16_t s, uint16_t z) {
+    long so, zo;
+    orc_chan_sz_pos(d, &so, &zo);
+    memcpy(area + so, &s, 2);
+    memcpy(area + zo, &z, 2);
+}
+
+static void put_tok_sz(uint8_t *area, int u, int j, int nj, uint16_t s, uint16_t z) {
+    long so, zo;
+    orc_tok_sz_pos(u, j, nj, &so, &zo);
+    memcpy(area + so, &s, 2);
+    memcpy(area + zo, &z, 2);
+}
+
+/* Exported for tests: kind 0 = per-channel (index = channel), 1 = per-token
+ * (index = token, j = group). */
+void orc_sz_position(int kind, int index, int j, int nj, long *s_off, long *z_off) {
+    if (kind == 0) orc_chan_sz_pos(index, s_off, z_off);
+    else orc_tok_sz_pos(index, j, nj, s_off, z_off);
 }
 
 /* ---------------- one (batch, kv-head) unit ---------------- */
@@ -258,7 +288,7 @@ int orc_unit(const uint16_t *K, const uint16_t *V, int L, int D, int bk, int bv,
             orc_quant(x, 32, 1, bv, &s16, &z16, c, 1);
             if (img) {
                 uint8_t *rec = img + blk * REC;
-                put_sz(rec + KC + KS + VC + 4L * (u * nj + j), s16, z16);
+                put_tok_sz(rec + KC + KS + VC, u, j, nj, s16, z16);
                 for (int i = 0; i < 32; i++) orc_put_code(rec + KC + KS, 1, u, 32 * j + i, D, bv, c[i]);
             }
             if (Vh) {
@@ -276,7 +306,7 @@ int orc_unit(const uint16_t *K, const uint16_t *V, int L, int D, int bk, int bv,
                 orc_quant(x, 32, 1, bk, &s16, &z16, c, 1);
                 if (img) {
                     uint8_t *rec = img + blk * REC;
-                    put_sz(rec + KC + 4L * d, s16, z16);
+                    put_chan_sz(rec + KC, d, s16, z16);
                     for (int i = 0; i < 32; i++) orc_put_code(rec, 0, i, d, D, bk, c[i]);
                 }
                 if (Kh) {
@@ -301,7 +331,7 @@ int orc_unit(const uint16_t *K, const uint16_t *V, int L, int D, int bk, int bv,
                 orc_quant(x, 32, 1, bk, &s16, &z16, c, 1);
                 if (img) {
                     uint8_t *rec = img + blk * REC;
-                    put_sz(rec + KC + 4L * (u * nj + j), s16, z16);
+                    put_tok_sz(rec + KC, u, j, nj, s16, z16);
                     for (int i = 0; i < 32; i++) orc_put_code(rec, 0, u, 32 * j + i, D, bk, c[i]);
                 }
                 if (Kh) {

@@ -215,6 +215,20 @@ def test_worked_packing_examples():
     assert len(img) == rec + 64 * D
 
 
+def chan_sz_off(d):
+    """Test-side restatement of the per-channel key scale/zero placement."""
+    k, e = divmod(d, 16)
+    t, r, hb = (e % 8) // 2, e // 8, e % 2
+    so = 16 * (4 * k + t) + 8 * r + 2 * hb
+    return so, so + 4
+
+
+def tok_sz_off(u, j, nj):
+    """Test-side restatement of the per-token scale/zero placement."""
+    so = 8 * nj * (u // 2) + 4 * j + 2 * (u % 2)
+    return so, so + 4 * nj
+
+
 def decode_unit_image(img, L, D, bk, bv, kmode):
     """Independent reader: codes and s/z of a unit image -> dequantized K^, V^ (fp64)."""
     REC = oracle.record_bytes(D, bk, bv)
@@ -224,26 +238,55 @@ def decode_unit_image(img, L, D, bk, bv, kmode):
     Kh = np.zeros((L, D))
     Vh = np.zeros((L, D))
 
-    def sz(buf, off):
-        h = np.frombuffer(buf[off:off + 4].tobytes(), np.uint16)
-        return oracle.f16_bits_to_f64(h)
+    def h16(buf, off):
+        return oracle.f16_bits_to_f64(np.frombuffer(buf[off:off + 2].tobytes(), np.uint16))[0]
 
     for tok in range(L):
         blk, u = divmod(tok, 32)
         rec = img[blk * REC:(blk + 1) * REC]
         for d in range(D):
-            s, z = sz(rec, KC + KS + VC + 4 * (u * nj + d // 32))
+            so, zo = tok_sz_off(u, d // 32, nj)
+            s, z = h16(rec, KC + KS + VC + so), h16(rec, KC + KS + VC + zo)
             Vh[tok, d] = oracle.get_code(rec[KC + KS:KC + KS + VC], 1, u, d, D, bv) * s + z
             if kmode == oracle.PER_TOKEN:
-                s, z = sz(rec, KC + 4 * (u * nj + d // 32))
-                Kh[tok, d] = oracle.get_code(rec[:KC], 0, u, d, D, bk) * s + z
+                so, zo = tok_sz_off(u, d // 32, nj)
+                Kh[tok, d] = oracle.get_code(rec[:KC], 0, u, d, D, bk) * h16(rec, KC + so) + h16(rec, KC + zo)
             elif blk < L // 32:
-                s, z = sz(rec, KC + 4 * d)
-                Kh[tok, d] = oracle.get_code(rec[:KC], 0, u, d, D, bk) * s + z
+                so, zo = chan_sz_off(d)
+                Kh[tok, d] = oracle.get_code(rec[:KC], 0, u, d, D, bk) * h16(rec, KC + so) + h16(rec, KC + zo)
             else:
                 res = img[nblk * REC:]
                 Kh[tok, d] = oracle.bf16_bits_to_f32(np.frombuffer(res[2 * (u * D + d):2 * (u * D + d) + 2].tobytes(), np.uint16))[0]
     return Kh, Vh
+
+
+def test_golden_sz_positions():
+    """Hand-derived scale/zero offsets (no page fixes a layout)."""
+    rows = [list(map(int, ln.split())) for ln in open(os.path.join(GOLDEN, "format_v1_sz_positions.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    assert len(rows) >= 12
+    for kind, nj, index, j, so, zo in rows:
+        assert oracle.sz_position(kind, index, j, nj) == (so, zo), (kind, nj, index, j)
+
+
+@pytest.mark.parametrize("nj", [1, 2, 4, 8])
+def test_sz_layout_is_a_bijection(nj):
+    """Scales and zeros of every channel (per-channel area) and of every (token, group)
+    (per-token area) occupy distinct aligned fp16 slots that tile the 4*D-byte area."""
+    D = 32 * nj
+    seen = set()
+    for d in range(D):
+        so, zo = oracle.sz_position(0, d, 0, nj)
+        assert so % 2 == 0 and zo % 2 == 0 and so not in seen and zo not in seen
+        seen |= {so, zo}
+    assert seen == set(range(0, 4 * D, 2))
+    seen = set()
+    for u in range(32):
+        for j in range(nj):
+            so, zo = oracle.sz_position(1, u, j, nj)
+            assert so not in seen and zo not in seen
+            seen |= {so, zo}
+    assert seen == set(range(0, 4 * D, 2))
 
 
 @pytest.mark.parametrize("L,kmode,bk,bv", [(40, 0, 4, 2), (33, 1, 8, 4), (64, 0, 2, 8), (7, 0, 8, 8)])
@@ -272,7 +315,11 @@ def test_image_edges_and_zero_fill():
         if r:
             tail = img[(nblk - 1) * REC:nblk * REC]
             assert not tail[:KC + KS].any()                  # incomplete key group: not stored
-            assert not tail[KC + KS + VC + 4 * nj * r:].any()  # value s/z of absent tokens
+            vsz = tail[KC + KS + VC:]
+            for u in range(r, 32):                           # value s/z of absent tokens
+                for j in range(nj):
+                    so, zo = tok_sz_off(u, j, nj)
+                    assert not vsz[so:so + 2].any() and not vsz[zo:zo + 2].any()
             res = img[nblk * REC:]
             assert not res[2 * D * r:].any()
             assert np.array_equal(Kh[L - r:], bf16_vals(K[L - r:]).astype(np.float64))
