@@ -158,6 +158,21 @@ KVQ_API int kvq_truncate(kvq_handle *h, int layer, int L);
  * kernel reported a bounded wait that expired; *flags gets the raw bits. */
 KVQ_API int kvq_device_status(kvq_handle *h, void *stream, unsigned *flags);
 
+/* Decode attention without any caller-provided scratch: the same computation and
+ * arguments as kvq_decode_attn, but the split partials go to a 32 MiB buffer built
+ * into the library (one per GPU that loads it, held until the process exits)
+ * instead of the workspace.  For callers that cannot allocate or lend device scratch
+ * (hosts that plan every device byte up front, code living in another component's
+ * memory pool).  The pages describe no such entry point; it has no counterpart
+ * there.  The first call on a device, with that device current, looks up the
+ * buffer's device address; make that first call before any stream capture.  Returns
+ * KVQ_EUNSUPPORTED when the call needs more partial space than the buffer holds
+ * (B * Hq * 64 * (head_dim + 2) * 4 bytes whenever the sequence is split).  All
+ * calls share the one buffer: calls that may overlap on the GPU (different streams,
+ * no ordering between them) race on it and must not be issued. */
+KVQ_API int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, int out_fp32,
+                                    void *stream);
+
 /* Free the handle (not the caller's workspace). */
 KVQ_API void kvq_destroy(kvq_handle *h);
 

@@ -4,6 +4,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -446,5 +447,106 @@ int kvq_device_status(kvq_handle *h, void *stream, unsigned *flags) {
 }
 
 void kvq_destroy(kvq_handle *h) { delete h; }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Decode attention for callers that cannot allocate device memory.
+//
+// kvq_decode_attn keeps its split partials in the caller's workspace.  Some callers
+// cannot provide scratch at all: an embedded or real-time host that plans every
+// device byte ahead of time, a plugin that runs inside someone else's memory pool,
+// or code between the points where allocating would be unsafe.  For them the
+// partials live in a fixed buffer compiled into this library.  The buffer exists
+// once per GPU that loads the library and stays until the process exits.  Host code
+// cannot use the array's name as a device address: the address is looked up once
+// per device (the first call on that device, with that device current) and cached.
+static constexpr size_t kStaticScratchBytes = size_t(32) << 20;   // 32 MiB
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+std::mutex g_scratch_mu;
+void *g_scratch_addr[256];   // per device ordinal
+
+int static_scratch_address(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 256) return fail(KVQ_EUNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress (static scratch)");
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return KVQ_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, int out_fp32, void *stream) {
+    int rc = check_layer(h, layer);
+    if (rc) return rc;
+    if ((rc = check_bound(h))) return rc;
+    if (!q || !out) return fail(KVQ_EINVAL, "null q or out");
+    if (!aligned(q, 16) || !aligned(out, 16)) return fail(KVQ_EALIGN, "q and out must be 16-byte aligned");
+    const int L = h->len[layer];
+    if (L < 1) return fail(KVQ_EINVAL, "layer %d is empty", layer);
+    int S = 1, nstage = 2;
+    if ((rc = splits_for(h, layer, &S, &nstage))) return rc;
+    const LayerGeom &g = h->geom[layer];
+    const int nblk = (L + 31) / 32;
+    const int bps = (nblk + S - 1) / S;
+    S = (nblk + bps - 1) / bps;
+    const long long rows = static_cast<long long>(h->desc.batch) * h->desc.n_q_heads;
+    const long long acc_bytes = rows * kvq::kMaxSplits * h->desc.head_dim * 4;
+    const long long need = S > 1 ? acc_bytes + rows * kvq::kMaxSplits * 2 * 4 : 0;
+    if (need > static_cast<long long>(kStaticScratchBytes))
+        return fail(KVQ_EUNSUPPORTED,
+                    "split partials need %lld bytes but the built-in scratch holds %zu; use kvq_decode_attn",
+                    need, kStaticScratchBytes);
+    void *scratch = nullptr;
+    if ((rc = static_scratch_address(&scratch))) return rc;
+    kvq::DecodeParams p{};
+    p.rec = h->ws + g.rec_off;
+    p.res = g.res_off >= 0 ? reinterpret_cast<const uint16_t *>(h->ws + g.res_off) : nullptr;
+    p.q = static_cast<const uint16_t *>(q);
+    p.smax = reinterpret_cast<const unsigned *>(h->ws + h->smax_off) + 2 * layer;
+    p.out = out;
+    p.part_acc = static_cast<float *>(scratch);
+    p.part_ml = reinterpret_cast<float *>(static_cast<unsigned char *>(scratch) + acc_bytes);
+    p.status = reinterpret_cast<unsigned *>(h->ws + h->status_off);
+    p.B = h->desc.batch;
+    p.Hkv = h->desc.n_kv_heads;
+    p.G = h->desc.n_q_heads / h->desc.n_kv_heads;
+    p.L = L;
+    p.cap_blk = h->cap_blk;
+    p.bps = bps;
+    p.S = S;
+    p.out_fp32 = out_fp32 ? 1 : 0;
+    p.nstage = nstage;
+    p.rec_bytes = g.rec_bytes;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = prepare_status(h, st))) return rc;
+    cudaError_t e = kvq::launch_decode(p, h->desc.head_dim, g.bk, g.bv, g.kmode, st, nullptr);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    if (p.S > 1) {
+        kvq::MergeParams m{};
+        m.part_acc = p.part_acc;
+        m.part_ml = p.part_ml;
+        m.out = out;
+        m.B = p.B;
+        m.Hq = h->desc.n_q_heads;
+        m.D = h->desc.head_dim;
+        m.S = p.S;
+        m.out_fp32 = p.out_fp32;
+        e = kvq::launch_merge(m, st);
+        if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+    }
+    return ok();
+}
 
 }  // extern "C"

@@ -68,6 +68,7 @@ def load() -> ctypes.CDLL:
         "kvq_bind": (I, [P, P, SZ]),
         "kvq_append": (I, [P, I, P, P, I, P]),
         "kvq_decode_attn": (I, [P, I, P, P, I, P]),
+        "kvq_decode_attn_noalloc": (I, [P, I, P, P, I, P]),
         "kvq_set_num_splits": (I, [P, I]),
         "kvq_get_num_splits": (I, [P, I, ctypes.POINTER(I)]),
         "kvq_export_layer": (I, [P, I, P, SZ, ctypes.POINTER(SZ)]),
@@ -133,6 +134,10 @@ def kvq_append(h: int, layer: int, K, V, n_new: int, stream=None):
 
 def kvq_decode_attn(h: int, layer: int, q, out, out_fp32: bool, stream=None):
     _check(load().kvq_decode_attn(h, layer, _ptr(q), _ptr(out), int(bool(out_fp32)), _stream(stream)))
+
+
+def kvq_decode_attn_noalloc(h: int, layer: int, q, out, out_fp32: bool, stream=None):
+    _check(load().kvq_decode_attn_noalloc(h, layer, _ptr(q), _ptr(out), int(bool(out_fp32)), _stream(stream)))
 
 
 def kvq_set_num_splits(h: int, n: int):
