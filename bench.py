@@ -39,6 +39,49 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s pool figure)"
 
 
+def kernel_source_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("layer_wise_mixed_b200/csrc/kvq_decode.cu", "layer_wise_mixed_b200/csrc/kvq_internal.h"):
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()
+
+
+def captured_traffic(workload_name, alg_bytes_per_launch):
+    """DRAM bytes per launch of the decode kernel from the committed ncu capture, scaled by
+    algorithmic bytes; None when the kernel changed since the capture or the workload differs."""
+    p = os.path.join(ROOT, "profiles", "decode_split_traffic.txt")
+    try:
+        kv = dict(ln.split(":", 1) for ln in open(p) if ":" in ln and not ln.startswith("#"))
+        kv = {k.strip(): v.strip() for k, v in kv.items()}
+        if kv["source_sha256"] != kernel_source_sha256() or kv["workload"] != workload_name:
+            return None
+        return float(kv["dram_bytes"]) / float(kv["algorithmic_bytes"]) * alg_bytes_per_launch
+    except Exception:
+        return None
+
+
+def rank_workload(wl, rank, world):
+    """Weak scaling: at N > 1 every rank runs its own replica of the workload on its own
+    seeded sequences (the rank is part of the workload name, hence of every seed)."""
+    if world <= 1:
+        return wl
+    import dataclasses
+    return dataclasses.replace(wl, name=f"{wl.name}-rank{rank}")
+
+
+def max_over_ranks(value_ms, world):
+    """Max of a per-rank time over all ranks (rank 0 reports it); plain value at N=1."""
+    if world <= 1:
+        return value_ms
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value_ms], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def decode_bytes(B, Hkv, G, D, L, bk, bv, kmode):
     """Algorithmic bytes of one decode-attention launch over L tokens: packed codes, fp16
     scale+zero per 32 elements, the bf16 key residual, q in and out (bf16)."""
@@ -212,10 +255,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
 
     # replica per rank: its own sequences (weak scaling, no data-path collective)
-    if world > 1:
-        wl = configs.Workload(f"{wl.name}-rank{rank}", wl.num_layers, wl.batch, wl.n_q_heads, wl.n_kv_heads,
-                              wl.head_dim, wl.prefill, wl.decode_steps, wl.layer_bits, wl.kmode, wl.n_outlier,
-                              wl.outlier_lo, wl.outlier_hi)
+    wl = rank_workload(wl, rank, world)
     B, Hkv, Hq, D, G, NL = wl.batch, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.G, wl.num_layers
     cache = kvq.Cache(NL, B, Hkv, Hq, D, wl.max_ctx, list(wl.layer_bits), kmodes=[wl.kmode] * NL)
     stream = torch.cuda.Stream()
@@ -285,11 +325,7 @@ def main():
         e1.record(stream)
     barrier()
     clocks = sampler.stop()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
     ms_per_step = ms / args.steps
     value = world * B * args.steps / (ms / 1e3)
 
@@ -344,11 +380,7 @@ def main():
             e2e_step((3 + i) % nsched)
         f1.record(stream)
     barrier()
-    e2e_ms = f0.elapsed_time(f1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
     e2e_value = world * B * e2e_steps / (e2e_ms / 1e3)
     h2d = (dK.numel() + dV.numel() + dQ.numel()) * 2
     d2h = out.numel() * 2
@@ -375,7 +407,9 @@ def main():
                 "config": workload_config(wl),
                 "hbm_gbs_decode": achieved,
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                             "frac": achieved / peak, "traffic": None, "kernel": "decode_split_kernel (+merge)",
+                             "frac": achieved / peak,
+                             "traffic": captured_traffic(wl.name, dec_bytes / launches_dec),
+                             "kernel": "decode_split_kernel (+merge)",
                              "peak_source": peak_src, "avg_launch_us": 1e3 * dec_ms / launches_dec,
                              "algorithmic_bytes_per_launch": dec_bytes / launches_dec},
                 "cpu_baseline": cpu,

@@ -108,26 +108,24 @@ __device__ __forceinline__ uint32_t hfma2_bits(uint32_t x, uint32_t m, uint32_t 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) { return h2_bits(__floats2half2_rn(lo, hi)); }
 
 // Exact fp16 pair of the two codes of slot p of a word: field p (low half) and field
-// p + P (high half), P = 16/BITS.  Codes enter the fp16 mantissa under exponent 2^10
-// (value 1024 + c, or 1024 + 2^k c) and the offset is removed exactly.
+// p + P (high half), P = 16/BITS.  The masked code bits are OR-ed under an fp16
+// exponent M chosen so that one mantissa step of the code is 1.0: the half then
+// holds M + c exactly, and subtracting M leaves c (M = 1024, 256, 64 or 16 for code
+// bits starting at mantissa bit 0, 2, 4 or 6).
 template <int BITS>
 __device__ __forceinline__ uint32_t unpack(uint32_t w, int p) {
-    constexpr uint32_t kMagic = 0x64006400u;   // (1024, 1024)
     if constexpr (BITS == 8) {
         const uint32_t sel = static_cast<uint32_t>(p) | 0x40u | (static_cast<uint32_t>(p + 2) << 8) | 0x4000u;
-        return hsub2_bits(prmt(w, 0x64646464u, sel), kMagic);
+        return hsub2_bits(prmt(w, 0x64646464u, sel), 0x64006400u);
     } else if constexpr (BITS == 4) {
         const uint32_t src = p < 2 ? w : (w >> 8);
-        if ((p & 1) == 0) return hsub2_bits(lop_and_or(src, 0x000F000Fu, kMagic), kMagic);
-        return hfma2_bits(lop_and_or(src, 0x00F000F0u, kMagic), 0x2C002C00u /*1/16*/, 0xD400D400u /*-64*/);
+        if ((p & 1) == 0) return hsub2_bits(lop_and_or(src, 0x000F000Fu, 0x64006400u), 0x64006400u);   // 1024 + c
+        return hsub2_bits(lop_and_or(src, 0x00F000F0u, 0x54005400u), 0x54005400u);                     // 64 + c
     } else {
         const uint32_t src = p < 4 ? w : (w >> 8);
         const int q = p & 3;
-        const uint32_t x = lop_and_or(src, 0x00030003u << (2 * q), kMagic);
-        if (q == 0) return hsub2_bits(x, kMagic);
-        if (q == 1) return hfma2_bits(x, 0x34003400u /*1/4*/, 0xDC00DC00u /*-256*/);
-        if (q == 2) return hfma2_bits(x, 0x2C002C00u /*1/16*/, 0xD400D400u /*-64*/);
-        return hfma2_bits(x, 0x24002400u /*1/64*/, 0xCC00CC00u /*-16*/);
+        const uint32_t M = q == 0 ? 0x64006400u : (q == 1 ? 0x5C005C00u : (q == 2 ? 0x54005400u : 0x4C004C00u));
+        return hsub2_bits(lop_and_or(src, 0x00030003u << (2 * q), M), M);
     }
 }
 
