@@ -169,7 +169,11 @@ def cpu_oracle_sample(wl, L, seqs, layers=1):
         Kb, Vb, qb = b16(K), b16(V), b16(q)
         bk, bv = wl.layer_bits[l % len(wl.layer_bits)]
         t0 = time.perf_counter()
-        oracle.layer(Kb, Vb, qb, wl.G, bk, bv, wl.kmode, want_image=False)
+        if wl.paged:
+            tg = inputs.tags(wl, L, tag="cpu-sample", batch=seqs).numpy()
+            oracle.paged_layer(Kb, Vb, tg, qb, wl.G, want_image=False)
+        else:
+            oracle.layer(Kb, Vb, qb, wl.G, bk, bv, wl.kmode, want_image=False)
         t += time.perf_counter() - t0
     step_s = t / layers * wl.num_layers * (wl.batch / seqs)
     return t, wl.batch / step_s
@@ -204,6 +208,14 @@ def run_reference(args, wl, rank):
 
 def workload_config(wl):
     bits = sorted(set(wl.layer_bits))
+    if wl.paged:
+        return {"workload": wl.name, "layers": wl.num_layers, "batch": wl.batch, "q_heads": wl.n_q_heads,
+                "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim,
+                "context": f"{wl.prefill + 1}..{wl.prefill + wl.decode_steps}",
+                "bits": "INT2 groups (K per-channel, V per-token) + INT4 per-token, tags Bernoulli(0.5)",
+                "equivalent_bits": wl.avg_bits, "page_tokens": wl.page_tokens,
+                "l2": "inputs larger than L2 (each step reads every layer's cache once)",
+                "launch": "one CUDA graph per decode step (tagged append + paged decode for all layers)"}
     return {"workload": wl.name, "layers": wl.num_layers, "batch": wl.batch, "q_heads": wl.n_q_heads,
             "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim,
             "context": f"{wl.prefill + 1}..{wl.prefill + wl.decode_steps}",
@@ -220,7 +232,7 @@ def main():
     ap.add_argument("--steps", type=int, default=512)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="c2", choices=["c2", "c2-k8v8", "c2-k8v4", "c3", "c4"])
+    ap.add_argument("--workload", default="c2", choices=["c2", "c2-k8v8", "c2-k8v4", "c3", "c4", "c5"])
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--ref-seqs", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -257,15 +269,37 @@ def main():
     # replica per rank: its own sequences (weak scaling, no data-path collective)
     wl = rank_workload(wl, rank, world)
     B, Hkv, Hq, D, G, NL = wl.batch, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.G, wl.num_layers
-    cache = kvq.Cache(NL, B, Hkv, Hq, D, wl.max_ctx, list(wl.layer_bits), kmodes=[wl.kmode] * NL)
+    paged = wl.paged
+    if paged:
+        cache = kvq.Cache(NL, B, Hkv, Hq, D, wl.max_ctx, avg_bits=wl.avg_bits)
+        all_tags = inputs.tags(wl, wl.max_ctx)                 # [B, prefill + steps], shared by layers
+        tags_dev = all_tags.cuda()
+        tags_host = all_tags.numpy()
+    else:
+        cache = kvq.Cache(NL, B, Hkv, Hq, D, wl.max_ctx, list(wl.layer_bits), kmodes=[wl.kmode] * NL)
     stream = torch.cuda.Stream()
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for l in range(NL):
             K, V = inputs.layer_kv(wl, l, wl.prefill, "cuda")
-            cache.append(l, K, V)
+            if paged:
+                t0 = tags_dev[:, :wl.prefill].contiguous()
+                kvq.kvq_append_tagged(cache.h, l, K, V, wl.prefill, np.ascontiguousarray(tags_host[:, :wl.prefill]),
+                                      t0, stream)
+            else:
+                cache.append(l, K, V)
             del K, V
     stream.synchronize()
+    if paged:
+        step_tags_dev = [tags_dev[:, wl.prefill + s:wl.prefill + s + 1].contiguous() for s in range(wl.decode_steps)]
+        step_tags_host = [np.ascontiguousarray(tags_host[:, wl.prefill + s:wl.prefill + s + 1])
+                          for s in range(wl.decode_steps)]
+
+    def append_step(l, s, Kd, Vd):
+        if paged:
+            kvq.kvq_append_tagged(cache.h, l, Kd, Vd, 1, step_tags_host[s], step_tags_dev[s], stream)
+        else:
+            kvq.kvq_append(cache.h, l, Kd, Vd, 1, stream)
 
     # decode schedule inputs, resident in HBM
     nsched = wl.decode_steps
@@ -291,7 +325,7 @@ def main():
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for l in range(NL):
-                kvq.kvq_append(cache.h, l, Kn[s, l], Vn[s, l], 1, stream)
+                append_step(l, s, Kn[s, l], Vn[s, l])
                 kvq.kvq_decode_attn(cache.h, l, Qn[s, l], out[l], False, stream)
         graphs.append(g)
         splits.append([kvq.kvq_get_num_splits(cache.h, l) for l in range(NL)])
@@ -341,11 +375,28 @@ def main():
     stream.synchronize()
     dec_ms = d0.elapsed_time(d1)
     launches_dec = args.steps * NL
-    dec_bytes = sum(decode_bytes(B, Hkv, G, D, Ls[s], *wl.layer_bits[l], wl.kmode)
-                    for s in order for l in range(NL))
+    if paged:
+        # INT2 groups: 2-bit codes + fp16 scale/zero per 32 (keys and values); INT4 tokens
+        # (main and pending): 4-bit codes + scale/zero; q in and out
+        def paged_bytes(L):
+            t = tags_host[:, :L]
+            n2 = (t == 2).sum(1)
+            g2 = (n2 // 32) * 32
+            rest = L - g2
+            per = g2 * D * 2 * (2 + 1) / 8 + rest * D * 2 * (4 + 1) / 8 + 2 * G * D * 2
+            return float(Hkv * per.sum())
+        dec_bytes = sum(paged_bytes(Ls[s]) for s in order for l in range(NL))
+    else:
+        dec_bytes = sum(decode_bytes(B, Hkv, G, D, Ls[s], *wl.layer_bits[l], wl.kmode)
+                        for s in order for l in range(NL))
     peak, peak_src = measured_hbm_peak()
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
     gpu_launches = sum(2 + (1 if splits[s][l] > 1 else 0) for s in order for l in range(NL))
+    e2e_note = ("per step: pinned H2D of all layers' K/V/q, kvq_append + kvq_decode_attn per layer (eager "
+                "C-ABI calls), D2H of all layers' outputs")
+    if paged:
+        e2e_note = ("per step: pinned H2D of all layers' K/V/q and kvq_decode_attn per layer (eager C-ABI calls; "
+                    "the cache is not advanced), D2H of all layers' outputs")
 
     # ---- e2e: public API with host buffers, H2D + D2H inside the timed region ----
     e2e_steps = args.e2e_steps or min(args.steps, 64)
@@ -356,14 +407,18 @@ def main():
     dK = torch.empty_like(Kn[0])
     dV = torch.empty_like(Vn[0])
     dQ = torch.empty_like(Qn[0])
-    for l in range(NL):
-        kvq.kvq_truncate(cache.h, l, wl.prefill)
+    if not paged:
+        for l in range(NL):
+            kvq.kvq_truncate(cache.h, l, wl.prefill)
 
     def e2e_step(s):
         dK.copy_(hK[s], non_blocking=True)
         dV.copy_(hV[s], non_blocking=True)
         dQ.copy_(hQ[s], non_blocking=True)
         for l in range(NL):
+            if paged:
+                kvq.kvq_decode_attn(cache.h, l, dQ[l], out[l], False, stream)
+                continue
             if cache.seq_len(l) >= wl.max_ctx:
                 kvq.kvq_truncate(cache.h, l, wl.prefill)
             kvq.kvq_append(cache.h, l, dK[l], dV[l], 1, stream)
@@ -414,8 +469,7 @@ def main():
                              "algorithmic_bytes_per_launch": dec_bytes / launches_dec},
                 "cpu_baseline": cpu,
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                        "steps": e2e_steps, "how": "per step: pinned H2D of all layers' K/V/q, kvq_append + "
-                        "kvq_decode_attn per layer (eager C-ABI calls), D2H of all layers' outputs"},
+                        "steps": e2e_steps, "how": e2e_note},
                 "gpu_launches": gpu_launches, "clocks": clocks, "device_status": status,
                 "splits": sorted(set(x for s in order for x in splits[s]))}
         print(json.dumps(line), flush=True)

@@ -126,6 +126,22 @@ KVQ_API int kvq_bind(kvq_handle *h, void *dev_ptr, size_t bytes);
  * launch.  n_new >= 1; returns KVQ_ECAPACITY beyond max_ctx. */
 KVQ_API int kvq_append(kvq_handle *h, int layer, const void *K, const void *V, int n_new, void *stream);
 
+/* Paged plans (desc.paged = 1; head_dim 128, G in {1, 2, 4}, batch <= 64): append n_new
+ * tokens per request with their tags, 2 (INT2) or 4 (INT4), given twice: host_tags
+ * [B][n_new] for the host-side page planning, dev_tags (same bytes, device) for the
+ * kernels; the caller keeps them equal.  INT2-tagged tokens, in arrival order, form
+ * groups of 32 (keys per channel 2-bit, values per token 2-bit) in the INT2 pool; INT4
+ * tokens go to 16-token INT4 pages (keys and values per token 4-bit); INT2 tokens whose
+ * group is still open are held the INT4 way in two pending pages per request (with
+ * their bf16 originals) until the group completes ("TriAxialKV per-role
+ * mixed-precision KV quantization", Facts: quantizer, leftover routing, page pools).
+ * The INT2 and INT4 pools of each (layer, kv head) share one region split at an offset
+ * from avg_bits; KVQ_ECAPACITY when a pool or a page table would overflow (checked
+ * before any launch).  A multi-token call launches a tag scan first.  The per-layer bit
+ * map is not used by paged plans (layers may be NULL). */
+KVQ_API int kvq_append_tagged(kvq_handle *h, int layer, const void *K, const void *V, int n_new,
+                              const uint8_t *host_tags, const uint8_t *dev_tags, void *stream);
+
 /* Decode attention of one query token per sequence over all L tokens of `layer`:
  * q bf16 [B][Hq][D] (device); out [B][Hq][D] (device) bf16, or fp32 if out_fp32.
  * Launches the split kernel and, when the sequence is split, the log-sum-exp merge
@@ -142,7 +158,9 @@ KVQ_API int kvq_get_num_splits(const kvq_handle *h, int layer, int *num_splits);
 
 /* Copy one layer's cache to host memory in canonical order (parity checks): for each
  * (b, h) the records 0..ceil(L/32)-1 then, for per-channel keys, the residual; bytes
- * that hold no token of 0..L-1 are zero.  Synchronous (device-wide).  If host_buf is
+ * that hold no token of 0..L-1 are zero.  Paged plans: for each (b, h) the INT2 records
+ * in group order, the INT4 main pages in order, the two pending pages, then the bf16
+ * staging keys and values (32 x D each) of the open INT2 group.  Synchronous (device-wide).  If host_buf is
  * NULL or bytes is too small, only *needed is written (KVQ_EINVAL if too small). */
 KVQ_API int kvq_export_layer(const kvq_handle *h, int layer, void *host_buf, size_t bytes,
                      size_t *needed);

@@ -190,93 +190,67 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t 
 // terms [8*NT][NJ], running max and sum per head [8] + [8].
 __host__ __device__ constexpr int comb_floats(int D, int NT) { return 8 * NT * D + 8 * NT * (D / 32) + 16; }
 
-template <int BK, int BV, int KM, int D, int NT>
-__global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(const DecodeParams p) {
-    constexpr int KS = D / 16;     // 16-channel steps (QK) / 16-channel row tiles (PV)
-    constexpr int NJ = D / 32;     // channel groups
-    constexpr int WHK = D * BK / 64, WHV = D * BV / 64;
-    constexpr int PK = 16 / BK, PV = 16 / BV;   // slots per word
-    constexpr int KC = 4 * D * BK, KSZ = 4 * D, VC = 4 * D * BV;
-    constexpr int REC = KC + KSZ + VC + 4 * D;
+// Bytes of one unit record: NH 16-token halves of codes, fp16 scales/zeros.
+__host__ __device__ constexpr int unit_bytes(int D, int BK, int BV, int KM, int NH) {
+    return 2 * NH * D * BK + (KM == 0 ? 4 * D : 2 * NH * D) + 2 * NH * D * BV + 2 * NH * D;
+}
 
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int b = blockIdx.z, h = blockIdx.y, sp = blockIdx.x;
-    const int G = p.G, L = p.L, NS = p.nstage;
-    const int nblk = (L + 31) >> 5;
-    const int blk0 = sp * p.bps, blk1 = min(nblk, blk0 + p.bps);
-    const int rem = L & 31;
-    const int tail_blk = rem ? (L >> 5) : -1;
+// Per-thread constants of the block body.
+struct BodyCtx {
+    const uint4 *aq_s;          // q operand fragments in shared memory, [KS][32]
+    const uint16_t *res;        // bf16 residual keys of this (b, h) (per-channel tail) or null
+    int lane, g, t, G, jg, jg8, jz, alpha_src0, alpha_src1;
+    bool row_g, row_g8;
+    uint32_t m_hi, m_lo;
+    float unscale, qsum_g, qsum_g8, pbias;
+};
 
-    uint8_t *stages = smem + static_cast<size_t>(warp) * NS * REC;
-    const size_t stage_bytes = static_cast<size_t>(NW) * NS * REC;
-    const size_t comb_bytes = static_cast<size_t>(NW) * comb_floats(D, NT) * 4;
-    const size_t bar_off = ((stage_bytes > comb_bytes ? stage_bytes : comb_bytes) + 127) & ~size_t(127);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + bar_off) + warp * NS;
-    // q operand fragments, identical for the CTA's warps: [KS][32 lanes] x uint4
-    uint4 *aq_s = reinterpret_cast<uint4 *>(smem + bar_off + static_cast<size_t>(NW) * NS * 8 + 8 * ((NW * NS) & 1));
-    const uint8_t *unit_rec = p.rec + (static_cast<long long>(b) * p.Hkv + h) * p.cap_blk * REC;
+template <int D, int NT>
+struct WarpAcc {
+    float m_run, l_run;
+    float oacc[D / 16][NT][4];
+    float zc[NT][4];            // value zero-point term: rows = channel group j (= g)
+};
 
-    const int nb = (blk1 - blk0 > warp) ? (blk1 - blk0 - warp + NW - 1) / NW : 0;
-    if (lane == 0) {
-        for (int s = 0; s < NS; ++s) mbar_init(&bars[s], 1);
-        fence_mbar_init();
-    }
-    __syncwarp();
-    int issued = min(NS, nb);   // copies issued so far (every lane keeps the count)
-    if (lane == 0) {
-        for (int k = 0; k < issued; ++k) {
-            mbar_expect_tx(&bars[k], REC);
-            bulk_g2s(stages + k * REC, unit_rec + static_cast<long long>(blk0 + warp + NW * k) * REC, REC, &bars[k]);
-        }
-    }
-
-    // ---- operand prescales (powers of two) from the layer's largest scales ----
-    const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
-    const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
-    // values: p * 2^kp * s_v stays below 2^14 in fp16
-    const int kp = smax_v > 0.f ? max(-24, min(14, 13 - floor_log2(smax_v))) : 14;
-
-    // ---- this thread's query head and channels (16k + 2t + {0, 1, 8, 9}) ----
-    const int hh = g % G;
-    const uint16_t *qrow = p.q + (static_cast<long long>(b) * p.Hkv * G + h * G + hh) * D;
+// Query setup: q~ fragments into shared memory (written by warp 0), score scaling.
+//  per-channel keys: q~ = q log2(e)/sqrt(D) 2^kq as fp16 hi/lo (rows g: hi, g+8: lo),
+//    kq chosen so that q~ s_k < 2^14 and q~ < 2^15; scores = raw * 2^-kq.
+//  per-token keys: raw q (exact in fp16), rows (group j, head) masked to group j;
+//    scores = raw * log2(e)/sqrt(D).
+template <int KM, int D>
+__device__ __forceinline__ void setup_query(const uint16_t *qrow, float smax_k, uint4 *aq_s, BodyCtx &c,
+                                            int warp) {
+    constexpr int KS = D / 16, NJ = D / 32;
+    const int t = c.t;
     float qv[KS][4];
 #pragma unroll
     for (int k = 0; k < KS; ++k) {
         const uint32_t a = *reinterpret_cast<const uint32_t *>(qrow + 16 * k + 2 * t);
-        const uint32_t c = *reinterpret_cast<const uint32_t *>(qrow + 16 * k + 2 * t + 8);
+        const uint32_t b = *reinterpret_cast<const uint32_t *>(qrow + 16 * k + 2 * t + 8);
         qv[k][0] = __uint_as_float(a << 16);
         qv[k][1] = __uint_as_float(a & 0xFFFF0000u);
-        qv[k][2] = __uint_as_float(c << 16);
-        qv[k][3] = __uint_as_float(c & 0xFFFF0000u);
+        qv[k][2] = __uint_as_float(b << 16);
+        qv[k][3] = __uint_as_float(b & 0xFFFF0000u);
     }
     const float qscale = kLog2e * rsqrtf(static_cast<float>(D));
-
-    // Per-channel keys: q~ = q log2(e)/sqrt(D) 2^kq as fp16 hi/lo fragments (rows g: hi,
-    // g+8: lo), kq chosen so that q~ s_k stays below 2^14 and q~ below 2^15.
-    // Per-token keys: raw q (exact in fp16), rows (group j, head) masked to group j.
-    uint32_t aq[KS][4];                  // built here, then kept in shared memory (aq_s)
-    float unscale = 1.f;                 // true score (log2 units) = raw * unscale
-    float qsum_g = 0.f, qsum_g8 = 0.f;   // per-token keys: sum of q over the rows' groups
-    const int jg = g / G, jg8 = (g + 8) / G;
-    const bool row_g = (KM == 1) && (g < G * NJ), row_g8 = (KM == 1) && (g + 8 < G * NJ);
+    uint32_t aq[KS][4];
+    c.qsum_g = c.qsum_g8 = 0.f;
     if constexpr (KM == 0) {
         float amax = 0.f;
 #pragma unroll
         for (int k = 0; k < KS; ++k)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) amax = fmaxf(amax, fabsf(qv[k][c] * qscale));
+            for (int x = 0; x < 4; ++x) amax = fmaxf(amax, fabsf(qv[k][x] * qscale));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
         int kq = 0;
         if (amax > 0.f) {
-            kq = 14 - floor_log2(amax);                                            // q~ < 2^15
+            kq = 14 - floor_log2(amax);                                                  // q~ < 2^15
             if (smax_k > 0.f) kq = min(kq, 12 - floor_log2(amax) - floor_log2(smax_k));   // q~ s < 2^14
             kq = max(-60, min(60, kq));
         }
         const float sc = qscale * pow2f(kq);
-        unscale = pow2f(-kq);
+        c.unscale = pow2f(-kq);
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
             split2(qv[k][0] * sc, qv[k][1] * sc, aq[k][0], aq[k][1]);
@@ -291,323 +265,374 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
             const int j = k >> 1;
             part[j] += (qv[k][0] + qv[k][1]) + (qv[k][2] + qv[k][3]);
             const uint32_t lo = pack_h2(qv[k][0], qv[k][1]), hi = pack_h2(qv[k][2], qv[k][3]);
-            aq[k][0] = (row_g && jg == j) ? lo : 0u;
-            aq[k][1] = (row_g8 && jg8 == j) ? lo : 0u;
-            aq[k][2] = (row_g && jg == j) ? hi : 0u;
-            aq[k][3] = (row_g8 && jg8 == j) ? hi : 0u;
+            aq[k][0] = (c.row_g && c.jg == j) ? lo : 0u;
+            aq[k][1] = (c.row_g8 && c.jg8 == j) ? lo : 0u;
+            aq[k][2] = (c.row_g && c.jg == j) ? hi : 0u;
+            aq[k][3] = (c.row_g8 && c.jg8 == j) ? hi : 0u;
         }
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
             part[j] += __shfl_xor_sync(0xffffffffu, part[j], 1);
             part[j] += __shfl_xor_sync(0xffffffffu, part[j], 2);
-            if (j == (jg < NJ ? jg : 0)) qsum_g = part[j];
-            if (j == (jg8 < NJ ? jg8 : 0)) qsum_g8 = part[j];
+            if (j == (c.jg < NJ ? c.jg : 0)) c.qsum_g = part[j];
+            if (j == (c.jg8 < NJ ? c.jg8 : 0)) c.qsum_g8 = part[j];
         }
-        unscale = qscale;
+        c.unscale = qscale;
     }
     if (warp == 0) {
 #pragma unroll
-        for (int k = 0; k < KS; ++k) aq_s[k * 32 + lane] = make_uint4(aq[k][0], aq[k][1], aq[k][2], aq[k][3]);
+        for (int k = 0; k < KS; ++k) aq_s[k * 32 + c.lane] = make_uint4(aq[k][0], aq[k][1], aq[k][2], aq[k][3]);
     }
-    __syncthreads();
+}
 
-    float m_run = -INFINITY, l_run = 0.f;
-    float oacc[KS][NT][4];
-    float zc[NT][4];     // value zero-point term: rows = channel group j (= g), cols as oacc
+// Thread constants that depend only on the lane, the group size and the layer scales.
+template <int KM, int D, int NT>
+__device__ __forceinline__ BodyCtx make_ctx(int lane, int G, float smax_v, const uint4 *aq_s) {
+    constexpr int NJ = D / 32;
+    BodyCtx c{};
+    c.aq_s = aq_s;
+    c.lane = lane;
+    c.g = lane >> 2;
+    c.t = lane & 3;
+    c.G = G;
+    c.jg = c.g / G;
+    c.jg8 = (c.g + 8) / G;
+    c.row_g = (KM == 1) && (c.g < G * NJ);
+    c.row_g8 = (KM == 1) && (c.g + 8 < G * NJ);
+    c.jz = c.g < NJ ? c.g : NJ - 1;
+    // B-operand column of this thread for P: NT == 1: hi (g < G), lo (G <= g < 2G) or
+    // zero; NT == 2: tile 0 hi, tile 1 lo for g < G.
+    c.m_hi = (c.g < G) ? 0xFFFFFFFFu : 0u;
+    c.m_lo = (NT == 1 && c.g >= G && c.g < 2 * G) ? 0xFFFFFFFFu : 0u;
+    c.alpha_src0 = 4 * ((NT == 1) ? ((2 * c.t) % G) : min(2 * c.t, 7));
+    c.alpha_src1 = 4 * ((NT == 1) ? ((2 * c.t + 1) % G) : min(2 * c.t + 1, 7));
+    // values: p * 2^kp * s_v stays below 2^14 in fp16
+    const int kp = smax_v > 0.f ? max(-24, min(14, 13 - floor_log2(smax_v))) : 14;
+    c.pbias = static_cast<float>(kp);
+    return c;
+}
+
+template <int D, int NT>
+__device__ __forceinline__ void acc_init(WarpAcc<D, NT> &A) {
+    A.m_run = -INFINITY;
+    A.l_run = 0.f;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) zc[n][c] = 0.f;
+        for (int x = 0; x < 4; ++x) A.zc[n][x] = 0.f;
 #pragma unroll
-        for (int m = 0; m < KS; ++m)
+        for (int m = 0; m < D / 16; ++m)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) oacc[m][n][c] = 0.f;
+            for (int x = 0; x < 4; ++x) A.oacc[m][n][x] = 0.f;
+    }
+}
+
+// One unit of NH 16-token halves (32-token block record, or 16-token page when NH = 1)
+// staged at R; `valid` tokens are present (TAIL: valid may be < 16 NH; per-channel
+// TAIL blocks take their keys from the bf16 residual).
+template <int BK, int BV, int KM, int D, int NT, int NH, bool TAIL>
+__device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R, const int valid,
+                                             const BodyCtx &c) {
+    constexpr int KS = D / 16;
+    constexpr int NJ = D / 32;
+    constexpr int NTOK = 16 * NH;        // tokens in the unit
+    constexpr int NTI = 2 * NH;          // 8-token score tiles
+    constexpr int WHK = D * BK / 64, WHV = D * BV / 64;
+    constexpr int PK = 16 / BK, PV = 16 / BV;
+    constexpr int KC = 2 * NH * D * BK, KSZ = (KM == 0 ? 4 * D : 2 * NH * D), VC = 2 * NH * D * BV;
+    static_assert(KM == 1 || NH == 2, "per-channel keys come in 32-token groups");
+    const int lane = c.lane, g = c.g, t = c.t;
+
+    // ===== scores S^T (rows: heads, columns: 8-token tiles) =====
+    float acc[NTI][4];
+#pragma unroll
+    for (int n = 0; n < NTI; ++n)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) acc[n][x] = 0.f;
+    float czacc[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (KM == 0 && TAIL) {
+        // bf16 residual keys of the last, incomplete group
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+            const uint4 aqv = c.aq_s[k * 32 + lane];
+            const uint32_t ak[4] = {aqv.x, aqv.y, aqv.z, aqv.w};
+#pragma unroll
+            for (int n = 0; n < NTI; ++n) {
+                const int u = 8 * n + g;
+                uint32_t b0 = 0u, b1 = 0u;
+                if (u < valid) {
+                    const uint32_t r0 = *reinterpret_cast<const uint32_t *>(c.res + u * D + 16 * k + 2 * t);
+                    const uint32_t r8 = *reinterpret_cast<const uint32_t *>(c.res + u * D + 16 * k + 2 * t + 8);
+                    b0 = pack_h2(__uint_as_float(r0 << 16), __uint_as_float(r0 & 0xFFFF0000u));
+                    b1 = pack_h2(__uint_as_float(r8 << 16), __uint_as_float(r8 & 0xFFFF0000u));
+                }
+                mma16816(acc[n], ak, b0, b1);
+            }
+        }
+    } else {
+        // key words of k-step k: slots 4k..4k+3 of each half, lane word (4k + x) / PK
+        constexpr int WPK = PK >= 4 ? 1 : 4 / PK;   // words per k-step and half
+        constexpr int CH = WHK < 4 ? WHK : 4;        // lane words per chunk
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+            uint32_t kw[NH][WPK];
+            const int w0 = (4 * k) / PK;
+#pragma unroll
+            for (int x = 0; x < WPK; ++x) {
+                const int w = w0 + x;
+                const int off = (((w / CH) * 32 + lane) * CH + (w % CH)) * 4;
+#pragma unroll
+                for (int hf = 0; hf < NH; ++hf) kw[hf][x] = *reinterpret_cast<const uint32_t *>(R + hf * 2 * D * BK + off);
+            }
+            const uint4 aqv = c.aq_s[k * 32 + lane];
+            const uint32_t ak[4] = {aqv.x, aqv.y, aqv.z, aqv.w};
+            uint32_t a[4];
+            if constexpr (KM == 0) {
+                // scales/zeros of channels (16k+2t, +1) and (16k+2t+8, +9) as half2
+                const uint4 sz = *reinterpret_cast<const uint4 *>(R + KC + 16 * (4 * k + t));
+                mul_hilo(ak[0], ak[1], sz.x, a[0], a[1]);
+                mul_hilo(ak[2], ak[3], sz.z, a[2], a[3]);
+                mma16816(czacc, ak, sz.y, sz.w);   // sum_d q~_d z_d, same in every column
+            } else {
+                a[0] = ak[0];
+                a[1] = ak[1];
+                a[2] = ak[2];
+                a[3] = ak[3];
+            }
+#pragma unroll
+            for (int n = 0; n < NTI; ++n) {
+                const int s0 = (2 * k + (n & 1)) * 2;
+                const int wl = s0 / PK - w0;
+                const uint32_t w = kw[n >> 1][wl];
+                mma16816(acc[n], a, unpack<BK>(w, s0 % PK), unpack<BK>(w, s0 % PK + 1));
+            }
+        }
     }
 
-    // B-operand column of this thread for P: NT == 1: hi (g < G), lo (G <= g < 2G) or
-    // zero; NT == 2: tile 0 hi, tile 1 lo for g < G.
-    const uint32_t m_hi = (g < G) ? 0xFFFFFFFFu : 0u;
-    const uint32_t m_lo = (NT == 1 && g >= G && g < 2 * G) ? 0xFFFFFFFFu : 0u;
-    const int alpha_src0 = 4 * ((NT == 1) ? ((2 * t) % G) : min(2 * t, 7));
-    const int alpha_src1 = 4 * ((NT == 1) ? ((2 * t + 1) % G) : min(2 * t + 1, 7));
-    const float pbias = static_cast<float>(kp);
-    const int jz = g < NJ ? g : NJ - 1;
-
-    // ------------------------------------------------------------ one 32-token block
-    auto body = [&](auto tail_tag, const uint8_t *R, const int valid) {
-        constexpr bool TAIL = decltype(tail_tag)::value;
-        // ===== scores S^T (rows: heads, columns: 8-token tiles) =====
-        float acc[4][4];
+    float raw[NTI][2];
+    if constexpr (KM == 0) {
+        const float cz = czacc[0] + czacc[2];
 #pragma unroll
-        for (int n = 0; n < 4; ++n)
+        for (int n = 0; n < NTI; ++n) {
+            raw[n][0] = acc[n][0] + acc[n][2] + cz;
+            raw[n][1] = acc[n][1] + acc[n][3] + cz;
+        }
+    } else {
+        // per-token key scales on the (group, head) rows, then sum the rows of a head
+        const uint8_t *ks = R + KC;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) acc[n][c] = 0.f;
-        float czacc[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (KM == 0 && TAIL) {
-            // bf16 residual keys of the last, incomplete group
-            const uint16_t *res = p.res + (static_cast<long long>(b) * p.Hkv + h) * 32 * D;
-#pragma unroll
-            for (int k = 0; k < KS; ++k) {
-                const uint4 aqv = aq_s[k * 32 + lane];
-                const uint32_t ak[4] = {aqv.x, aqv.y, aqv.z, aqv.w};
-#pragma unroll
-                for (int n = 0; n < 4; ++n) {
-                    const int u = 8 * n + g;
-                    uint32_t b0 = 0u, b1 = 0u;
-                    if (u < valid) {
-                        const uint32_t r0 = *reinterpret_cast<const uint32_t *>(res + u * D + 16 * k + 2 * t);
-                        const uint32_t r8 = *reinterpret_cast<const uint32_t *>(res + u * D + 16 * k + 2 * t + 8);
-                        b0 = pack_h2(__uint_as_float(r0 << 16), __uint_as_float(r0 & 0xFFFF0000u));
-                        b1 = pack_h2(__uint_as_float(r8 << 16), __uint_as_float(r8 & 0xFFFF0000u));
-                    }
-                    mma16816(acc[n], ak, b0, b1);
-                }
+        for (int n = 0; n < NTI; ++n) {
+            const int pi = 4 * n + t;   // token pair (8n + 2t, 8n + 2t + 1)
+            float v0 = 0.f, v1 = 0.f;
+            if (c.row_g) {
+                const uint32_t sw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * c.jg);
+                const uint32_t zw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * NJ + 4 * c.jg);
+                v0 = fmaf(half_lo_f(sw), acc[n][0], half_lo_f(zw) * c.qsum_g);
+                v1 = fmaf(half_hi_f(sw), acc[n][1], half_hi_f(zw) * c.qsum_g);
             }
+            if (c.row_g8) {
+                const uint32_t sw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * c.jg8);
+                const uint32_t zw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * NJ + 4 * c.jg8);
+                v0 += fmaf(half_lo_f(sw), acc[n][2], half_lo_f(zw) * c.qsum_g8);
+                v1 += fmaf(half_hi_f(sw), acc[n][3], half_hi_f(zw) * c.qsum_g8);
+            }
+#pragma unroll
+            for (int msk = c.G; msk < 8; msk <<= 1) {
+                v0 += __shfl_xor_sync(0xffffffffu, v0, 4 * msk);
+                v1 += __shfl_xor_sync(0xffffffffu, v1, 4 * msk);
+            }
+            raw[n][0] = v0;
+            raw[n][1] = v1;
+        }
+    }
+    if constexpr (TAIL) {
+#pragma unroll
+        for (int n = 0; n < NTI; ++n)
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+                if (8 * n + 2 * t + x >= valid) raw[n][x] = -INFINITY;
+    }
+
+    // ===== online softmax (base 2; p carries the factor 2^kp) =====
+    float mloc = -INFINITY;
+#pragma unroll
+    for (int n = 0; n < NTI; ++n) mloc = fmaxf(mloc, fmaxf(raw[n][0], raw[n][1]));
+    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+    mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+    const float m_new = fmaxf(A.m_run, mloc * c.unscale);
+    const float alpha = fast_exp2(A.m_run - m_new);
+    A.m_run = m_new;
+    const float shift = c.pbias - m_new;
+    float pr[NTI][2];
+    float psum = 0.f;
+#pragma unroll
+    for (int n = 0; n < NTI; ++n)
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            pr[n][x] = fast_exp2(fmaf(raw[n][x], c.unscale, shift));
+            psum += pr[n][x];
+        }
+    A.l_run = fmaf(A.l_run, alpha, psum);
+    if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+        const float a0 = __shfl_sync(0xffffffffu, alpha, c.alpha_src0);
+        const float a1 = __shfl_sync(0xffffffffu, alpha, c.alpha_src1);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            A.zc[n][0] *= a0;
+            A.zc[n][1] *= a1;
+#pragma unroll
+            for (int m = 0; m < KS; ++m) {
+                A.oacc[m][n][0] *= a0;
+                A.oacc[m][n][1] *= a1;
+                A.oacc[m][n][2] *= a0;
+                A.oacc[m][n][3] *= a1;
+            }
+        }
+    }
+
+    // ===== O^T += V^T P'^T and the zero-point term (16-token steps) =====
+#pragma unroll
+    for (int kk = 0; kk < NH; ++kk) {
+        uint32_t vw[WHV];
+        load_lane_words<WHV>(R + KC + KSZ + kk * 2 * D * BV, lane, vw);
+        uint32_t pah, pal, pbh, pbl;   // p of token pairs A (16kk+2t, +1) and B (+8, +9)
+        split2(pr[2 * kk][0], pr[2 * kk][1], pah, pal);
+        split2(pr[2 * kk + 1][0], pr[2 * kk + 1][1], pbh, pbl);
+        const uint8_t *vs = R + KC + KSZ + VC;
+        const int iA = 8 * kk + t, iB = iA + 4;
+        uint32_t sA[NJ], sB[NJ];
+        if constexpr (NJ == 4) {
+            const uint4 xa = *reinterpret_cast<const uint4 *>(vs + 8 * NJ * iA);
+            const uint4 xb = *reinterpret_cast<const uint4 *>(vs + 8 * NJ * iB);
+            sA[0] = xa.x; sA[1] = xa.y; sA[2] = xa.z; sA[3] = xa.w;
+            sB[0] = xb.x; sB[1] = xb.y; sB[2] = xb.z; sB[3] = xb.w;
         } else {
-            // key words of k-step k: slots 4k..4k+3 of each half, lane word (4k + x) / PK
-            constexpr int WPK = PK >= 4 ? 1 : 4 / PK;   // words per k-step and half
-            constexpr int CH = WHK < 4 ? WHK : 4;        // lane words per chunk
-#pragma unroll
-            for (int k = 0; k < KS; ++k) {
-                uint32_t kw0[WPK], kw1[WPK];
-                const int w0 = (4 * k) / PK;
-#pragma unroll
-                for (int x = 0; x < WPK; ++x) {
-                    const int w = w0 + x;
-                    const int off = (((w / CH) * 32 + lane) * CH + (w % CH)) * 4;
-                    kw0[x] = *reinterpret_cast<const uint32_t *>(R + off);
-                    kw1[x] = *reinterpret_cast<const uint32_t *>(R + 2 * D * BK + off);
-                }
-                const uint4 aqv = aq_s[k * 32 + lane];
-                const uint32_t ak[4] = {aqv.x, aqv.y, aqv.z, aqv.w};
-                uint32_t a[4];
-                if constexpr (KM == 0) {
-                    // scales/zeros of channels (16k+2t, +1) and (16k+2t+8, +9) as half2
-                    const uint4 sz = *reinterpret_cast<const uint4 *>(R + KC + 16 * (4 * k + t));
-                    mul_hilo(ak[0], ak[1], sz.x, a[0], a[1]);
-                    mul_hilo(ak[2], ak[3], sz.z, a[2], a[3]);
-                    mma16816(czacc, ak, sz.y, sz.w);   // sum_d q~_d z_d, same in every column
-                } else {
-                    a[0] = ak[0];
-                    a[1] = ak[1];
-                    a[2] = ak[2];
-                    a[3] = ak[3];
-                }
-#pragma unroll
-                for (int n = 0; n < 4; ++n) {
-                    const int s0 = (2 * k + (n & 1)) * 2;
-                    const int wl = s0 / PK - w0;
-                    const uint32_t w = (n >> 1) ? kw1[wl] : kw0[wl];
-                    mma16816(acc[n], a, unpack<BK>(w, s0 % PK), unpack<BK>(w, s0 % PK + 1));
-                }
-            }
-        }
-
-        float raw[4][2];
-        if constexpr (KM == 0) {
-            const float cz = czacc[0] + czacc[2];
-#pragma unroll
-            for (int n = 0; n < 4; ++n) {
-                raw[n][0] = acc[n][0] + acc[n][2] + cz;
-                raw[n][1] = acc[n][1] + acc[n][3] + cz;
-            }
-        } else {
-            // per-token key scales on the (group, head) rows, then sum the rows of a head
-            const uint8_t *ks = R + KC;
-#pragma unroll
-            for (int n = 0; n < 4; ++n) {
-                const int pi = 4 * n + t;   // token pair (8n + 2t, 8n + 2t + 1)
-                float v0 = 0.f, v1 = 0.f;
-                if (row_g) {
-                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * jg);
-                    const uint32_t zw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * NJ + 4 * jg);
-                    v0 = fmaf(half_lo_f(sw), acc[n][0], half_lo_f(zw) * qsum_g);
-                    v1 = fmaf(half_hi_f(sw), acc[n][1], half_hi_f(zw) * qsum_g);
-                }
-                if (row_g8) {
-                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * jg8);
-                    const uint32_t zw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * NJ + 4 * jg8);
-                    v0 += fmaf(half_lo_f(sw), acc[n][2], half_lo_f(zw) * qsum_g8);
-                    v1 += fmaf(half_hi_f(sw), acc[n][3], half_hi_f(zw) * qsum_g8);
-                }
-#pragma unroll
-                for (int msk = G; msk < 8; msk <<= 1) {
-                    v0 += __shfl_xor_sync(0xffffffffu, v0, 4 * msk);
-                    v1 += __shfl_xor_sync(0xffffffffu, v1, 4 * msk);
-                }
-                raw[n][0] = v0;
-                raw[n][1] = v1;
-            }
-        }
-        if constexpr (TAIL) {
-#pragma unroll
-            for (int n = 0; n < 4; ++n)
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-                    if (8 * n + 2 * t + c >= valid) raw[n][c] = -INFINITY;
-        }
-
-        // ===== online softmax (base 2; p carries the factor 2^kp) =====
-        float mloc = fmaxf(fmaxf(fmaxf(raw[0][0], raw[0][1]), fmaxf(raw[1][0], raw[1][1])),
-                           fmaxf(fmaxf(raw[2][0], raw[2][1]), fmaxf(raw[3][0], raw[3][1])));
-        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-        const float m_new = fmaxf(m_run, mloc * unscale);
-        const float alpha = fast_exp2(m_run - m_new);
-        m_run = m_new;
-        const float shift = pbias - m_new;
-        float pr[4][2];
-        float psum = 0.f;
-#pragma unroll
-        for (int n = 0; n < 4; ++n)
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                pr[n][c] = fast_exp2(fmaf(raw[n][c], unscale, shift));
-                psum += pr[n][c];
-            }
-        l_run = fmaf(l_run, alpha, psum);
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-            const float a0 = __shfl_sync(0xffffffffu, alpha, alpha_src0);
-            const float a1 = __shfl_sync(0xffffffffu, alpha, alpha_src1);
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                zc[n][0] *= a0;
-                zc[n][1] *= a1;
-#pragma unroll
-                for (int m = 0; m < KS; ++m) {
-                    oacc[m][n][0] *= a0;
-                    oacc[m][n][1] *= a1;
-                    oacc[m][n][2] *= a0;
-                    oacc[m][n][3] *= a1;
-                }
-            }
-        }
-
-        // ===== O^T += V^T P'^T and the zero-point term (two 16-token steps) =====
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-            uint32_t vw[WHV];
-            load_lane_words<WHV>(R + KC + KSZ + kk * 2 * D * BV, lane, vw);
-            uint32_t pah, pal, pbh, pbl;   // p of token pairs A (16kk+2t, +1) and B (+8, +9)
-            split2(pr[2 * kk][0], pr[2 * kk][1], pah, pal);
-            split2(pr[2 * kk + 1][0], pr[2 * kk + 1][1], pbh, pbl);
-            const uint8_t *vs = R + KC + KSZ + VC;
-            const int iA = 8 * kk + t, iB = iA + 4;
-            uint32_t sA[NJ], sB[NJ];
-            if constexpr (NJ == 4) {
-                const uint4 xa = *reinterpret_cast<const uint4 *>(vs + 8 * NJ * iA);
-                const uint4 xb = *reinterpret_cast<const uint4 *>(vs + 8 * NJ * iB);
-                sA[0] = xa.x; sA[1] = xa.y; sA[2] = xa.z; sA[3] = xa.w;
-                sB[0] = xb.x; sB[1] = xb.y; sB[2] = xb.z; sB[3] = xb.w;
-            } else {
-#pragma unroll
-                for (int j = 0; j < NJ; ++j) {
-                    sA[j] = reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iA)[j];
-                    sB[j] = reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iB)[j];
-                }
-            }
-            uint32_t zA = *reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iA + 4 * NJ + 4 * jz);
-            uint32_t zB = *reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iB + 4 * NJ + 4 * jz);
-            if constexpr (TAIL) {
-                // absent tokens: p = 0 and their scale/zero halves may hold anything
-                const int u0 = 16 * kk + 2 * t;
-                const uint32_t mA = (u0 < valid ? 0x0000FFFFu : 0u) | (u0 + 1 < valid ? 0xFFFF0000u : 0u);
-                const uint32_t mB = (u0 + 8 < valid ? 0x0000FFFFu : 0u) | (u0 + 9 < valid ? 0xFFFF0000u : 0u);
-#pragma unroll
-                for (int j = 0; j < NJ; ++j) {
-                    sA[j] &= mA;
-                    sB[j] &= mB;
-                }
-                zA &= mA;
-                zB &= mB;
-            }
-            // zero-point term: rows j = g of Z^T (tokens as columns) times the P columns
-            {
-                const uint32_t az[4] = {g < NJ ? zA : 0u, 0u, g < NJ ? zB : 0u, 0u};
-                if constexpr (NT == 1) {
-                    mma16816(zc[0], az, (pah & m_hi) | (pal & m_lo), (pbh & m_hi) | (pbl & m_lo));
-                } else {
-                    mma16816(zc[0], az, pah & m_hi, pbh & m_hi);
-                    mma16816(zc[1], az, pal & m_hi, pbl & m_hi);
-                }
-            }
 #pragma unroll
             for (int j = 0; j < NJ; ++j) {
-                uint32_t ah, al, bh, bl;
-                mul_hilo(pah, pal, sA[j], ah, al);
-                mul_hilo(pbh, pbl, sB[j], bh, bl);
-                uint32_t b0, b1, c0 = 0u, c1 = 0u;
-                if constexpr (NT == 1) {
-                    b0 = (ah & m_hi) | (al & m_lo);
-                    b1 = (bh & m_hi) | (bl & m_lo);
-                } else {
-                    b0 = ah & m_hi;
-                    b1 = bh & m_hi;
-                    c0 = al & m_hi;
-                    c1 = bl & m_hi;
-                }
-#pragma unroll
-                for (int mm = 0; mm < 2; ++mm) {
-                    const int m = 2 * j + mm;
-                    uint32_t a[4];
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const int s = 4 * m + r;
-                        a[r] = unpack<BV>(vw[s / PV], s % PV);
-                    }
-                    mma16816(oacc[m][0], a, b0, b1);
-                    if constexpr (NT == 2) mma16816(oacc[m][NT - 1], a, c0, c1);
-                }
+                sA[j] = reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iA)[j];
+                sB[j] = reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iB)[j];
             }
         }
-    };
-
-    // ------------------------------------------------------------ main loop
-    const bool has_tail = tail_blk >= blk0 && tail_blk < blk1 && ((tail_blk - blk0) % NW) == warp;
-    const int nb_main = nb - (has_tail ? 1 : 0);
-    int st = 0;
-    unsigned ph = 0;
-    bool failed = false;
-    int i = 0;
-    auto refill = [&]() {
-        __syncwarp();
-        if (issued < nb) {
-            if (lane == 0) {
-                fence_proxy_async();
-                mbar_expect_tx(&bars[st], REC);
-                bulk_g2s(stages + st * REC, unit_rec + static_cast<long long>(blk0 + warp + NW * issued) * REC, REC,
-                         &bars[st]);
+        uint32_t zA = *reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iA + 4 * NJ + 4 * c.jz);
+        uint32_t zB = *reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iB + 4 * NJ + 4 * c.jz);
+        if constexpr (TAIL) {
+            // absent tokens: p = 0 and their scale/zero halves may hold anything
+            const int u0 = 16 * kk + 2 * t;
+            const uint32_t mA = (u0 < valid ? 0x0000FFFFu : 0u) | (u0 + 1 < valid ? 0xFFFF0000u : 0u);
+            const uint32_t mB = (u0 + 8 < valid ? 0x0000FFFFu : 0u) | (u0 + 9 < valid ? 0xFFFF0000u : 0u);
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) {
+                sA[j] &= mA;
+                sB[j] &= mB;
             }
-            ++issued;
+            zA &= mA;
+            zB &= mB;
         }
-        if (++st == NS) {
-            st = 0;
-            ph ^= 1u;
+        // zero-point term: rows j = g of Z^T (tokens as columns) times the P columns
+        {
+            const uint32_t az[4] = {g < NJ ? zA : 0u, 0u, g < NJ ? zB : 0u, 0u};
+            if constexpr (NT == 1) {
+                mma16816(A.zc[0], az, (pah & c.m_hi) | (pal & c.m_lo), (pbh & c.m_hi) | (pbl & c.m_lo));
+            } else {
+                mma16816(A.zc[0], az, pah & c.m_hi, pbh & c.m_hi);
+                mma16816(A.zc[1], az, pal & c.m_hi, pbl & c.m_hi);
+            }
         }
-    };
-    for (; i < nb_main; ++i) {
-        if (!mbar_wait(&bars[st], ph)) {
-            failed = true;
-            break;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            uint32_t ah, al, bh, bl;
+            mul_hilo(pah, pal, sA[j], ah, al);
+            mul_hilo(pbh, pbl, sB[j], bh, bl);
+            uint32_t b0, b1, c0 = 0u, c1 = 0u;
+            if constexpr (NT == 1) {
+                b0 = (ah & c.m_hi) | (al & c.m_lo);
+                b1 = (bh & c.m_hi) | (bl & c.m_lo);
+            } else {
+                b0 = ah & c.m_hi;
+                b1 = bh & c.m_hi;
+                c0 = al & c.m_hi;
+                c1 = bl & c.m_hi;
+            }
+#pragma unroll
+            for (int mm = 0; mm < 2; ++mm) {
+                const int m = 2 * j + mm;
+                uint32_t a[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int s = 4 * m + r;
+                    a[r] = unpack<BV>(vw[s / PV], s % PV);
+                }
+                mma16816(A.oacc[m][0], a, b0, b1);
+                if constexpr (NT == 2) mma16816(A.oacc[m][NT - 1], a, c0, c1);
+            }
         }
-        body(std::false_type{}, stages + st * REC, 32);
-        refill();
     }
-    if (!failed && has_tail) {
-        if (!mbar_wait(&bars[st], ph)) {
-            failed = true;
-        } else {
-            body(std::true_type{}, stages + st * REC, rem);
-            ++i;
-        }
-    }
-    if (failed) {
-        // drain the copies still in flight (bounded), then report
-        for (int k = i; k < issued; ++k) mbar_wait(&bars[k % NS], (k / NS) & 1);
-        if (lane == 0) atomicOr(p.status, kStatusWaitExpired);
-    }
+    (void)NTOK;
+}
 
-    // ================= combine the warps of this split =================
+// Per-warp ring of NS shared-memory stages filled by cp.async.bulk (one elected lane),
+// completion tracked by one mbarrier per stage with bounded waits.
+struct WarpPipe {
+    uint8_t *stages;
+    uint64_t *bars;
+    int NS, stage_bytes, lane;
+    int issued, st;   // units issued so far; stage of the next unit to consume
+    unsigned ph;      // its mbarrier phase
+    int ist;          // stage of the next unit to issue
+};
+
+__device__ __forceinline__ void pipe_init(WarpPipe &P) {
+    if (P.lane == 0) {
+        for (int s = 0; s < P.NS; ++s) mbar_init(&P.bars[s], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    P.issued = 0;
+    P.st = 0;
+    P.ph = 0;
+    P.ist = 0;
+}
+
+// Issue the copy of the next unit (bytes from src) into the next free stage; stages
+// are refilled in the order they are consumed, so the next free stage is P.ist.
+__device__ __forceinline__ void pipe_issue(WarpPipe &P, const void *src, unsigned bytes) {
+    const int s = P.ist;
+    if (P.lane == 0) {
+        fence_proxy_async();
+        mbar_expect_tx(&P.bars[s], bytes);
+        bulk_g2s(P.stages + static_cast<size_t>(s) * P.stage_bytes, src, bytes, &P.bars[s]);
+    }
+    ++P.issued;
+    if (++P.ist == P.NS) P.ist = 0;
+}
+
+__device__ __forceinline__ bool pipe_wait(WarpPipe &P) { return mbar_wait(&P.bars[P.st], P.ph); }
+
+__device__ __forceinline__ const uint8_t *pipe_front(const WarpPipe &P) {
+    return P.stages + static_cast<size_t>(P.st) * P.stage_bytes;
+}
+
+__device__ __forceinline__ void pipe_pop(WarpPipe &P) {
+    __syncwarp();
+    if (++P.st == P.NS) {
+        P.st = 0;
+        P.ph ^= 1u;
+    }
+}
+
+// After a failed wait: wait (bounded) for the copies still in flight, from `from`.
+__device__ __forceinline__ void pipe_drain(WarpPipe &P, int from) {
+    for (int k = from; k < P.issued; ++k) mbar_wait(&P.bars[k % P.NS], (k / P.NS) & 1);
+}
+
+// Combine the CTA's warps and store either the output (one split) or the split partial.
+template <int D, int NT>
+__device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &c, bool has_data, uint8_t *smem,
+                                              int warp, long long row0, int sp, int S, int out_fp32, void *out,
+                                              float *part_acc, float *part_ml) {
+    constexpr int KS = D / 16, NJ = D / 32;
+    const int g = c.g, t = c.t, G = c.G;
+    float l_run = A.l_run;
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
     __syncthreads();   // every warp is done with its stages
@@ -621,57 +646,238 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
                 const int d0 = 16 * m + g, c0 = 8 * n + 2 * t;
-                ob[c0 * D + d0] = oacc[m][n][0];
-                ob[(c0 + 1) * D + d0] = oacc[m][n][1];
-                ob[c0 * D + d0 + 8] = oacc[m][n][2];
-                ob[(c0 + 1) * D + d0 + 8] = oacc[m][n][3];
+                ob[c0 * D + d0] = A.oacc[m][n][0];
+                ob[(c0 + 1) * D + d0] = A.oacc[m][n][1];
+                ob[c0 * D + d0 + 8] = A.oacc[m][n][2];
+                ob[(c0 + 1) * D + d0 + 8] = A.oacc[m][n][3];
             }
         if (g < NJ) {
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
-                zb[(8 * n + 2 * t) * NJ + g] = zc[n][0];
-                zb[(8 * n + 2 * t + 1) * NJ + g] = zc[n][1];
+                zb[(8 * n + 2 * t) * NJ + g] = A.zc[n][0];
+                zb[(8 * n + 2 * t + 1) * NJ + g] = A.zc[n][1];
             }
         }
         if (t == 0 && g < G) {
-            ml[g] = (nb > 0 && !failed) ? m_run : -INFINITY;
+            ml[g] = has_data ? A.m_run : -INFINITY;
             ml[8 + g] = l_run;
         }
     }
     __syncthreads();
-    const int Hq = p.Hkv * G;
+    const float *base = reinterpret_cast<const float *>(smem);
     for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
         const int hd = idx / D, d = idx % D;
         const int chi = hd, clo = (NT == 1) ? hd + G : 8 + hd;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, reinterpret_cast<const float *>(smem)[w * CF + 8 * NT * D + 8 * NT * NJ + hd]);
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, base[w * CF + 8 * NT * D + 8 * NT * NJ + hd]);
         float val = 0.f, den = 0.f;
+        if (M != -INFINITY) {
 #pragma unroll
-        for (int w = 0; w < NW; ++w) {
-            const float *ob = reinterpret_cast<const float *>(smem) + w * CF;
-            const float *zb = ob + 8 * NT * D;
-            const float *ml = zb + 8 * NT * NJ;
-            const float mw = ml[hd];
-            if (mw == -INFINITY) continue;
-            const float wt = fast_exp2(mw - M);
-            const float o = (ob[chi * D + d] + ob[clo * D + d]) + (zb[chi * NJ + d / 32] + zb[clo * NJ + d / 32]);
-            val = fmaf(wt, o, val);
-            den = fmaf(wt, ml[8 + hd], den);
+            for (int w = 0; w < NW; ++w) {
+                const float *ob = base + w * CF;
+                const float *zb = ob + 8 * NT * D;
+                const float *ml = zb + 8 * NT * NJ;
+                const float mw = ml[hd];
+                if (mw == -INFINITY) continue;
+                const float wt = fast_exp2(mw - M);
+                const float o = (ob[chi * D + d] + ob[clo * D + d]) + (zb[chi * NJ + d / 32] + zb[clo * NJ + d / 32]);
+                val = fmaf(wt, o, val);
+                den = fmaf(wt, ml[8 + hd], den);
+            }
         }
-        const long long row = static_cast<long long>(b) * Hq + h * G + hd;
-        if (p.S == 1) {
+        const long long row = row0 + hd;
+        if (S == 1) {
             const float o = val / den;
-            if (p.out_fp32) reinterpret_cast<float *>(p.out)[row * D + d] = o;
-            else reinterpret_cast<__nv_bfloat16 *>(p.out)[row * D + d] = __float2bfloat16_rn(o);
+            if (out_fp32) reinterpret_cast<float *>(out)[row * D + d] = o;
+            else reinterpret_cast<__nv_bfloat16 *>(out)[row * D + d] = __float2bfloat16_rn(o);
         } else {
-            p.part_acc[(row * kMaxSplits + sp) * D + d] = val;
+            part_acc[(row * kMaxSplits + sp) * D + d] = val;
             if (d == 0) {
-                p.part_ml[(row * kMaxSplits + sp) * 2] = M;
-                p.part_ml[(row * kMaxSplits + sp) * 2 + 1] = den;
+                part_ml[(row * kMaxSplits + sp) * 2] = M;
+                part_ml[(row * kMaxSplits + sp) * 2 + 1] = den;
             }
         }
     }
+}
+
+// Shared-memory carve-up: [stages | combine buffer][barriers][q fragments].
+struct SmemParts {
+    uint8_t *stages;
+    uint64_t *bars;
+    uint4 *aq_s;
+};
+
+__host__ __device__ inline size_t smem_bars_off(int NS, int stage_bytes, int D, int NT) {
+    const size_t stage = static_cast<size_t>(NW) * NS * stage_bytes;
+    const size_t comb = static_cast<size_t>(NW) * comb_floats(D, NT) * 4;
+    return ((stage > comb ? stage : comb) + 127) & ~size_t(127);
+}
+
+__host__ __device__ inline size_t smem_total(int NS, int stage_bytes, int D, int NT) {
+    const size_t bars = static_cast<size_t>(NW) * NS * 8 + 8 * ((NW * NS) & 1);   // keeps 16-B alignment
+    return smem_bars_off(NS, stage_bytes, D, NT) + bars + static_cast<size_t>(D / 16) * 32 * 16;
+}
+
+__device__ __forceinline__ SmemParts carve(uint8_t *smem, int NS, int stage_bytes, int D, int NT) {
+    SmemParts s;
+    s.stages = smem;
+    const size_t bo = smem_bars_off(NS, stage_bytes, D, NT);
+    s.bars = reinterpret_cast<uint64_t *>(smem + bo);
+    s.aq_s = reinterpret_cast<uint4 *>(smem + bo + static_cast<size_t>(NW) * NS * 8 + 8 * ((NW * NS) & 1));
+    return s;
+}
+
+// ------------------------------------------------------------------ per-layer kernel
+template <int BK, int BV, int KM, int D, int NT>
+__global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(const DecodeParams p) {
+    constexpr int REC = unit_bytes(D, BK, BV, KM, 2);
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.z, h = blockIdx.y, sp = blockIdx.x;
+    const int G = p.G, L = p.L, NS = p.nstage;
+    const int nblk = (L + 31) >> 5;
+    const int blk0 = sp * p.bps, blk1 = min(nblk, blk0 + p.bps);
+    const int rem = L & 31;
+    const int tail_blk = rem ? (L >> 5) : -1;
+
+    const SmemParts sm = carve(smem, NS, REC, D, NT);
+    WarpPipe P{sm.stages + static_cast<size_t>(warp) * NS * REC, sm.bars + warp * NS, NS, REC, lane, 0, 0, 0u, 0};
+    pipe_init(P);
+    const uint8_t *unit_rec = p.rec + (static_cast<long long>(b) * p.Hkv + h) * p.cap_blk * REC;
+    const int nb = (blk1 - blk0 > warp) ? (blk1 - blk0 - warp + NW - 1) / NW : 0;
+    for (int k = 0; k < NS && k < nb; ++k) pipe_issue(P, unit_rec + static_cast<long long>(blk0 + warp + NW * k) * REC, REC);
+
+    const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
+    const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
+    BodyCtx c = make_ctx<KM, D, NT>(lane, G, smax_v, sm.aq_s);
+    c.res = p.res ? p.res + (static_cast<long long>(b) * p.Hkv + h) * 32 * D : nullptr;
+    const int hh = c.g % G;
+    setup_query<KM, D>(p.q + (static_cast<long long>(b) * p.Hkv * G + h * G + hh) * D, smax_k, sm.aq_s, c, warp);
+    __syncthreads();
+
+    WarpAcc<D, NT> A;
+    acc_init(A);
+    const bool has_tail = tail_blk >= blk0 && tail_blk < blk1 && ((tail_blk - blk0) % NW) == warp;
+    const int nb_main = nb - (has_tail ? 1 : 0);
+    bool failed = false;
+    int i = 0;
+    for (; i < nb_main; ++i) {
+        if (!pipe_wait(P)) {
+            failed = true;
+            break;
+        }
+        process_unit<BK, BV, KM, D, NT, 2, false>(A, pipe_front(P), 32, c);
+        pipe_pop(P);
+        if (P.issued < nb) pipe_issue(P, unit_rec + static_cast<long long>(blk0 + warp + NW * P.issued) * REC, REC);
+    }
+    if (!failed && has_tail) {
+        if (!pipe_wait(P)) {
+            failed = true;
+        } else {
+            process_unit<BK, BV, KM, D, NT, 2, true>(A, pipe_front(P), rem, c);
+            ++i;
+        }
+    }
+    if (failed) {
+        pipe_drain(P, i);
+        if (lane == 0) atomicOr(p.status, kStatusWaitExpired);
+    }
+    combine_store<D, NT>(A, c, nb > 0 && !failed, smem, warp, static_cast<long long>(b) * p.Hkv * G + h * G, sp,
+                         p.S, p.out_fp32, p.out, p.part_acc, p.part_ml);
+}
+
+// ------------------------------------------------------------------ paged kernel
+// Splits [0, S2) cover the request's INT2 records (32-token groups, 2-bit keys per
+// channel, 2-bit values per token); splits [S2, S2 + S4) its INT4 pages (16 tokens,
+// 4-bit keys and values per token): main pages, then the pending pages of INT2 tokens
+// whose group is still open.  Every split is bitwidth-homogeneous.
+__global__ void __launch_bounds__(NW * 32, 4) decode_paged_kernel(const PagedDecodeParams p) {
+    constexpr int D = 128, NT = 1;
+    constexpr int REC2 = unit_bytes(D, 2, 2, 0, 2), PAGE4 = unit_bytes(D, 4, 4, 1, 1);
+    constexpr int STAGE = REC2 > PAGE4 ? REC2 : PAGE4;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.z, h = blockIdx.y, sp = blockIdx.x;
+    const int G = p.G, NS = p.nstage;
+    const bool int2 = sp < p.S2;
+    const int n2g = p.cnt[b].n2g, n4 = p.cnt[b].n4, np = p.cnt[b].np;
+    const int n4p = (n4 + 15) >> 4, npp = (np + 15) >> 4;
+    int u0, u1;
+    if (int2) {
+        const int per = (n2g + p.S2 - 1) / p.S2;
+        u0 = min(n2g, sp * per);
+        u1 = min(n2g, u0 + per);
+    } else {
+        const int tot = n4p + npp, per = (tot + p.S4 - 1) / p.S4;
+        u0 = min(tot, (sp - p.S2) * per);
+        u1 = min(tot, u0 + per);
+    }
+    const SmemParts sm = carve(smem, NS, STAGE, D, NT);
+    WarpPipe P{sm.stages + static_cast<size_t>(warp) * NS * STAGE, sm.bars + warp * NS, NS, STAGE, lane, 0, 0, 0u, 0};
+    pipe_init(P);
+    const int *tab = p.table + static_cast<long long>(b) * p.P_cap;
+    const uint8_t *pool2 = p.pool2 + static_cast<long long>(h) * p.n2_cap * REC2;
+    const uint8_t *pool4 = p.pool4 + static_cast<long long>(h) * p.n4_cap * PAGE4;
+    // unit u of this request -> (source, valid tokens)
+    // table of request b: INT2 groups from the front (entry = the group's first 16-token
+    // page, groups occupy page pairs), INT4 main pages from the back
+    auto src_of = [&](int u) -> const uint8_t * {
+        if (int2) return pool2 + static_cast<long long>(tab[u] >> 1) * REC2;
+        const int page = u < n4p ? tab[p.P_cap - 1 - u] : p.pend_base + 2 * b + (u - n4p);
+        return pool4 + static_cast<long long>(page) * PAGE4;
+    };
+    auto valid_of = [&](int u) -> int {
+        if (int2) return 32;
+        if (u < n4p) return (u == n4p - 1 && (n4 & 15)) ? (n4 & 15) : 16;
+        const int v = u - n4p;
+        return (v == npp - 1 && (np & 15)) ? (np & 15) : 16;
+    };
+    const int nb = (u1 - u0 > warp) ? (u1 - u0 - warp + NW - 1) / NW : 0;
+    const unsigned bytes = int2 ? REC2 : PAGE4;
+    for (int k = 0; k < NS && k < nb; ++k) pipe_issue(P, src_of(u0 + warp + NW * k), bytes);
+
+    const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
+    const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
+    WarpAcc<D, NT> A;
+    acc_init(A);
+    BodyCtx c;
+    const long long qoff = (static_cast<long long>(b) * p.Hkv * G + h * G + (lane >> 2) % G) * D;
+    if (int2) {
+        c = make_ctx<0, D, NT>(lane, G, smax_v, sm.aq_s);
+        c.res = nullptr;
+        setup_query<0, D>(p.q + qoff, smax_k, sm.aq_s, c, warp);
+    } else {
+        c = make_ctx<1, D, NT>(lane, G, smax_v, sm.aq_s);
+        c.res = nullptr;
+        setup_query<1, D>(p.q + qoff, smax_k, sm.aq_s, c, warp);
+    }
+    __syncthreads();
+
+    bool failed = false;
+    int i = 0;
+    for (; i < nb; ++i) {
+        if (!pipe_wait(P)) {
+            failed = true;
+            break;
+        }
+        const int u = u0 + warp + NW * i;
+        if (int2) {
+            process_unit<2, 2, 0, D, NT, 2, false>(A, pipe_front(P), 32, c);
+        } else {
+            const int v = valid_of(u);
+            if (v == 16) process_unit<4, 4, 1, D, NT, 1, false>(A, pipe_front(P), 16, c);
+            else process_unit<4, 4, 1, D, NT, 1, true>(A, pipe_front(P), v, c);
+        }
+        pipe_pop(P);
+        if (P.issued < nb) pipe_issue(P, src_of(u0 + warp + NW * P.issued), bytes);
+    }
+    if (failed) {
+        pipe_drain(P, i);
+        if (lane == 0) atomicOr(p.status, kStatusWaitExpired);
+    }
+    combine_store<D, NT>(A, c, nb > 0 && !failed, smem, warp, static_cast<long long>(b) * p.Hkv * G + h * G, sp,
+                         p.S2 + p.S4, p.out_fp32, p.out, p.part_acc, p.part_ml);
 }
 
 // Log-sum-exp merge of the split partials ("merged by online log-sum-exp").
@@ -739,17 +945,13 @@ int decode_stages(long long rec_bytes, int D, int G) {
 
 size_t decode_smem_bytes(long long rec_bytes, int nstage, int D, int G) {
     const int NT = G <= 4 ? 1 : 2;
-    const size_t stage = static_cast<size_t>(NW) * nstage * rec_bytes;
-    const size_t comb = static_cast<size_t>(NW) * comb_floats(D, NT) * 4;
-    const size_t base = ((stage > comb ? stage : comb) + 127) & ~size_t(127);
-    const size_t bars = static_cast<size_t>(NW) * nstage * 8 + 8 * ((NW * nstage) & 1);   // keeps 16-B alignment
-    return base + bars + static_cast<size_t>(D / 16) * 32 * 16;
+    return smem_total(nstage, static_cast<int>(rec_bytes), D, NT);
 }
 
 // Per-kernel cache of the dynamic shared-memory attribute and occupancy, so launches
 // (including launches recorded into CUDA graphs) issue no attribute calls.
 struct KernelState {
-    KernelFn fn = nullptr;
+    const void *fn = nullptr;
     size_t smem_set = 0;
     size_t occ_smem = 0;
     int occ = 0;
@@ -757,7 +959,7 @@ struct KernelState {
 static std::mutex g_state_mu;
 static KernelState g_state[64];
 
-static cudaError_t prepare_kernel(KernelFn fn, size_t smem, int *occ_out) {
+static cudaError_t prepare_kernel(const void *fn, size_t smem, int *occ_out) {
     std::lock_guard<std::mutex> lk(g_state_mu);
     KernelState *ks = nullptr;
     for (auto &e : g_state) {
@@ -788,7 +990,7 @@ cudaError_t decode_occupancy(int D, int bk, int bv, int kmode, int G, long long 
                              int *ctas_per_sm) {
     KernelFn fn = pick_kernel(D, bk, bv, kmode, G);
     if (!fn) return cudaErrorInvalidValue;
-    return prepare_kernel(fn, decode_smem_bytes(rec_bytes, nstage, D, G), ctas_per_sm);
+    return prepare_kernel(reinterpret_cast<const void *>(fn), decode_smem_bytes(rec_bytes, nstage, D, G), ctas_per_sm);
 }
 
 cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmode, cudaStream_t st,
@@ -796,10 +998,36 @@ cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmod
     KernelFn fn = pick_kernel(D, bk, bv, kmode, p.G);
     if (!fn) return cudaErrorInvalidValue;
     const size_t smem = decode_smem_bytes(p.rec_bytes, p.nstage, D, p.G);
-    cudaError_t e = prepare_kernel(fn, smem, ctas_per_sm_out);
+    cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(fn), smem, ctas_per_sm_out);
     if (e != cudaSuccess) return e;
     dim3 grid(p.S, p.Hkv, p.B);
     fn<<<grid, NW * 32, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+int paged_rec2_bytes(int D) { return unit_bytes(D, 2, 2, 0, 2); }
+int paged_page4_bytes(int D) { return unit_bytes(D, 4, 4, 1, 1); }
+
+int decode_paged_stages() {
+    const int stage = paged_rec2_bytes(128) > paged_page4_bytes(128) ? paged_rec2_bytes(128) : paged_page4_bytes(128);
+    return decode_stages(stage, 128, 4);
+}
+
+size_t decode_paged_smem_bytes(int nstage) {
+    const int stage = paged_rec2_bytes(128) > paged_page4_bytes(128) ? paged_rec2_bytes(128) : paged_page4_bytes(128);
+    return smem_total(nstage, stage, 128, 1);
+}
+
+cudaError_t decode_paged_occupancy(int nstage, int *ctas_per_sm) {
+    return prepare_kernel(reinterpret_cast<const void *>(decode_paged_kernel), decode_paged_smem_bytes(nstage), ctas_per_sm);
+}
+
+cudaError_t launch_decode_paged(const PagedDecodeParams &p, cudaStream_t st) {
+    const size_t smem = decode_paged_smem_bytes(p.nstage);
+    cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(decode_paged_kernel), smem, nullptr);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.S2 + p.S4, p.Hkv, p.B);
+    decode_paged_kernel<<<grid, NW * 32, smem, st>>>(p);
     return cudaGetLastError();
 }
 

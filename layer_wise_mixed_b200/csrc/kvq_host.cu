@@ -29,6 +29,18 @@ struct kvq_handle {
     int sm_count = 0;
     int device = -1;
     bool status_clear = false;   // status word zeroed on the device since the last bind
+    // paged INT2/INT4 plans
+    struct PagedLayer {
+        std::vector<int> n2g, n4, np;            // per request
+        std::vector<std::vector<int>> rec2;      // INT2 record ids per request, in group order
+        std::vector<std::vector<int>> page4;     // INT4 main page ids per request, in order
+        int next2 = 0, next4 = 0;                // bump allocators of the two pools
+    };
+    long long n2_cap = 0, n4_main_cap = 0, n4_cap = 0;
+    int P_cap = 0, pend_base = 0, inv_stride = 0;
+    long long rec2_bytes = 0, page4_bytes = 0, inv_off = 0;
+    std::vector<long long> pool2_off, pool4_off, staging_off, table_off;
+    std::vector<PagedLayer> pl;
 };
 
 namespace {
@@ -120,16 +132,74 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
     if (d->group != kvq::kGroup) return fail(KVQ_EUNSUPPORTED, "group must be 32 (got %d)", d->group);
     if (d->head_dim != 64 && d->head_dim != 128)
         return fail(KVQ_EUNSUPPORTED, "head_dim %d not supported (64 or 128)", d->head_dim);
-    if (d->paged) return fail(KVQ_EUNSUPPORTED, "paged plans are not available in this build");
-    if (!d->layers) return fail(KVQ_EINVAL, "null layer map");
+    if (!d->paged && !d->layers) return fail(KVQ_EINVAL, "null layer map");
+    if (d->paged) {
+        if (d->head_dim != 128) return fail(KVQ_EUNSUPPORTED, "paged plans need head_dim 128");
+        if (!(G == 1 || G == 2 || G == 4)) return fail(KVQ_EUNSUPPORTED, "paged plans need G in {1, 2, 4}");
+        if (d->batch > kvq::kMaxPagedBatch) return fail(KVQ_EUNSUPPORTED, "paged plans take at most %d requests", kvq::kMaxPagedBatch);
+        if (d->page_tokens != 16) return fail(KVQ_EUNSUPPORTED, "page_tokens must be 16");
+        if (!(d->avg_bits >= 2.0f && d->avg_bits <= 4.0f)) return fail(KVQ_EINVAL, "avg_bits must be in [2, 4]");
+    }
     const long long max_units = static_cast<long long>(d->batch) * d->n_kv_heads;
     if (max_units > 65535LL * 65535LL) return fail(KVQ_EUNSUPPORTED, "too many (batch, head) units");
     if (d->batch > 65535 || d->n_kv_heads > 65535) return fail(KVQ_EUNSUPPORTED, "batch/heads exceed grid limits");
 
     auto *h = new kvq_handle();
     h->desc = *d;
-    h->cfg.assign(d->layers, d->layers + d->num_layers);
+    if (d->layers) h->cfg.assign(d->layers, d->layers + d->num_layers);
     h->desc.layers = nullptr;
+    if (d->paged) {
+        // INT2 and INT4 pools of one region per (layer, kv head), split at an offset from
+        // the expected mean bits: a fraction f2 = (4 - avg_bits)/2 of the tokens is INT2.
+        const int D = d->head_dim;
+        const double f2 = (4.0 - d->avg_bits) / 2.0;
+        const double tokens = static_cast<double>(d->batch) * d->max_ctx;
+        h->rec2_bytes = kvq::paged_rec2_bytes(D);
+        h->page4_bytes = kvq::paged_page4_bytes(D);
+        h->n2_cap = static_cast<long long>(std::ceil(f2 * tokens * 1.03 / 32.0)) + d->batch;
+        h->n4_main_cap = static_cast<long long>(std::ceil((1.0 - f2) * tokens * 1.03 / 16.0)) + d->batch;
+        h->pend_base = static_cast<int>(h->n4_main_cap);
+        h->n4_cap = h->n4_main_cap + 2LL * d->batch;
+        h->P_cap = (d->max_ctx + 31) / 32 + (d->max_ctx + 15) / 16 + 1;
+        h->inv_stride = d->max_ctx;
+        long long off = align256(256 + 8LL * d->num_layers);
+        h->meta_bytes = off;
+        h->status_off = 0;
+        h->smax_off = 256;
+        for (int l = 0; l < d->num_layers; ++l) {
+            h->pool2_off.push_back(off);
+            off = align256(off + h->n2_cap * h->rec2_bytes * d->n_kv_heads);
+            h->pool4_off.push_back(off);
+            off = align256(off + h->n4_cap * h->page4_bytes * d->n_kv_heads);
+            h->staging_off.push_back(off);
+            off = align256(off + 2LL * d->batch * d->n_kv_heads * 32 * D * 2);
+            h->table_off.push_back(off);
+            off = align256(off + 4LL * d->batch * h->P_cap);
+            LayerGeom g{};
+            g.bk = 2;
+            g.bv = 2;
+            h->geom.push_back(g);
+        }
+        h->inv_off = off;
+        off = align256(off + 2LL * 4 * d->batch * h->inv_stride);
+        const long long rows = static_cast<long long>(d->batch) * d->n_q_heads;
+        h->part_acc_off = off;
+        off = align256(off + rows * kvq::kMaxSplits * D * 4);
+        h->part_ml_off = off;
+        off = align256(off + rows * kvq::kMaxSplits * 2 * 4);
+        h->total = off;
+        h->len.assign(d->num_layers, 0);
+        h->pl.assign(d->num_layers, kvq_handle::PagedLayer{});
+        for (auto &x : h->pl) {
+            x.n2g.assign(d->batch, 0);
+            x.n4.assign(d->batch, 0);
+            x.np.assign(d->batch, 0);
+            x.rec2.assign(d->batch, {});
+            x.page4.assign(d->batch, {});
+        }
+        *out = h;
+        return ok();
+    }
     h->cap_blk = (d->max_ctx + 31) / 32;
     const int D = d->head_dim;
     h->status_off = 0;
@@ -200,6 +270,14 @@ int kvq_bind(kvq_handle *h, void *dev_ptr, size_t bytes) {
     h->ws_bytes = bytes;
     h->status_clear = false;
     std::fill(h->len.begin(), h->len.end(), 0);
+    for (auto &x : h->pl) {
+        std::fill(x.n2g.begin(), x.n2g.end(), 0);
+        std::fill(x.n4.begin(), x.n4.end(), 0);
+        std::fill(x.np.begin(), x.np.end(), 0);
+        for (auto &v : x.rec2) v.clear();
+        for (auto &v : x.page4) v.clear();
+        x.next2 = x.next4 = 0;
+    }
     return ok();
 }
 
@@ -210,6 +288,7 @@ int kvq_append(kvq_handle *h, int layer, const void *K, const void *V, int n_new
     if (!K || !V) return fail(KVQ_EINVAL, "null K or V");
     if (!aligned(K, 16) || !aligned(V, 16)) return fail(KVQ_EALIGN, "K and V must be 16-byte aligned");
     if (n_new < 1) return fail(KVQ_EINVAL, "n_new must be >= 1 (got %d)", n_new);
+    if (h->desc.paged) return fail(KVQ_EINVAL, "paged plans append with kvq_append_tagged");
     const int L_old = h->len[layer];
     if (static_cast<long long>(L_old) + n_new > h->desc.max_ctx)
         return fail(KVQ_ECAPACITY, "layer %d: %d + %d tokens exceed max_ctx %d", layer, L_old, n_new, h->desc.max_ctx);
@@ -251,6 +330,105 @@ int kvq_append(kvq_handle *h, int layer, const void *K, const void *V, int n_new
     return ok();
 }
 
+int kvq_append_tagged(kvq_handle *h, int layer, const void *K, const void *V, int n_new,
+                      const uint8_t *host_tags, const uint8_t *dev_tags, void *stream) {
+    int rc = check_layer(h, layer);
+    if (rc) return rc;
+    if ((rc = check_bound(h))) return rc;
+    if (!h->desc.paged) return fail(KVQ_EINVAL, "kvq_append_tagged needs a paged plan");
+    if (!K || !V || !host_tags || !dev_tags) return fail(KVQ_EINVAL, "null K, V or tags");
+    if (!aligned(K, 16) || !aligned(V, 16)) return fail(KVQ_EALIGN, "K and V must be 16-byte aligned");
+    if (n_new < 1) return fail(KVQ_EINVAL, "n_new must be >= 1 (got %d)", n_new);
+    if (static_cast<long long>(h->len[layer]) + n_new > h->desc.max_ctx)
+        return fail(KVQ_ECAPACITY, "layer %d: %d + %d tokens exceed max_ctx %d", layer, h->len[layer], n_new,
+                    h->desc.max_ctx);
+    const int B = h->desc.batch;
+    auto &P = h->pl[layer];
+    kvq::PagedAppendParams a{};
+    int next2 = P.next2, next4 = P.next4;
+    a.cta4_off[0] = a.cta2_off[0] = 0;
+    for (int b = 0; b < B; ++b) {
+        int k2 = 0, k4 = 0;
+        for (int j = 0; j < n_new; ++j) {
+            const uint8_t tg = host_tags[static_cast<long long>(b) * n_new + j];
+            if (tg == 2) ++k2;
+            else if (tg == 4) ++k4;
+            else return fail(KVQ_EINVAL, "tag %d of request %d is %u (must be 2 or 4)", j, b, tg);
+        }
+        kvq::PagedReq &r = a.req[b];
+        r.n2g_old = P.n2g[b];
+        r.n4_old = P.n4[b];
+        r.np_old = P.np[b];
+        r.k2 = k2;
+        r.k4 = k4;
+        const int c0 = 32 * r.n2g_old + r.np_old, c1 = c0 + k2;
+        r.ng = c1 / 32 - c0 / 32;
+        r.base2 = next2;
+        next2 += r.ng;
+        const int n4p_old = (r.n4_old + 15) / 16, n4p_new = (r.n4_old + k4 + 15) / 16;
+        r.base4 = next4;
+        next4 += n4p_new - n4p_old;
+        r.last4 = (r.n4_old % 16 && k4 > 0) ? P.page4[b].back() : -1;
+        r.c4 = k4 > 0 ? (r.n4_old + k4 - 1) / 16 - r.n4_old / 16 + 1 : 0;
+        r.c2 = std::max(r.ng, k2 > 0 ? 1 : 0);
+        if (r.n2g_old + r.ng + n4p_new > h->P_cap)
+            return fail(KVQ_ECAPACITY, "request %d: page table full", b);
+        a.cta4_off[b + 1] = a.cta4_off[b] + r.c4;
+        a.cta2_off[b + 1] = a.cta2_off[b] + r.c2;
+    }
+    if (next2 > h->n2_cap)
+        return fail(KVQ_ECAPACITY, "INT2 pool full (%d of %lld records): the tags hold more INT2 tokens than avg_bits planned for",
+                    next2, h->n2_cap);
+    if (next4 > h->n4_main_cap)
+        return fail(KVQ_ECAPACITY, "INT4 pool full (%d of %lld pages): the tags hold more INT4 tokens than avg_bits planned for",
+                    next4, h->n4_main_cap);
+    const int D = h->desc.head_dim;
+    a.K = static_cast<const uint16_t *>(K);
+    a.V = static_cast<const uint16_t *>(V);
+    a.tags = dev_tags;
+    a.inv2 = reinterpret_cast<const int *>(h->ws + h->inv_off);
+    a.inv4 = a.inv2 + static_cast<long long>(B) * h->inv_stride;
+    a.inv_stride = h->inv_stride;
+    a.pool2 = h->ws + h->pool2_off[layer];
+    a.pool4 = h->ws + h->pool4_off[layer];
+    a.n2_cap = h->n2_cap;
+    a.n4_cap = h->n4_cap;
+    a.table = reinterpret_cast<int *>(h->ws + h->table_off[layer]);
+    a.P_cap = h->P_cap;
+    a.pend_base = h->pend_base;
+    a.staging = reinterpret_cast<uint16_t *>(h->ws + h->staging_off[layer]);
+    a.smax = reinterpret_cast<unsigned *>(h->ws + h->smax_off) + 2 * layer;
+    a.B = B;
+    a.Hkv = h->desc.n_kv_heads;
+    a.D = D;
+    a.n = n_new;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = prepare_status(h, st))) return rc;
+    if (n_new > 1) {
+        cudaError_t e = kvq::launch_paged_scan(dev_tags, B, n_new, const_cast<int *>(a.inv2), const_cast<int *>(a.inv4),
+                                               h->inv_stride, st);
+        if (e != cudaSuccess) return cuda_fail(e, "tag scan launch");
+    }
+    const long long grid = static_cast<long long>(a.cta4_off[B] + a.cta2_off[B]) * a.Hkv;
+    if (grid > 0x7FFFFFFFLL) return fail(KVQ_EUNSUPPORTED, "append too large for one launch");
+    cudaError_t e = kvq::launch_paged_append(a, static_cast<int>(grid), st);
+    if (e != cudaSuccess) return cuda_fail(e, "paged append launch");
+    // commit the host-side tables
+    for (int b = 0; b < B; ++b) {
+        const kvq::PagedReq &r = a.req[b];
+        for (int i = 0; i < r.ng; ++i) P.rec2[b].push_back(r.base2 + i);
+        const int n4p_old = (r.n4_old + 15) / 16, n4p_new = (r.n4_old + r.k4 + 15) / 16;
+        for (int i = 0; i < n4p_new - n4p_old; ++i) P.page4[b].push_back(r.base4 + i);
+        P.n2g[b] += r.ng;
+        P.n4[b] += r.k4;
+        P.np[b] = (32 * r.n2g_old + r.np_old + r.k2) % 32;
+    }
+    P.next2 = next2;
+    P.next4 = next4;
+    h->len[layer] += n_new;
+    return ok();
+}
+
 static int ensure_device_info(kvq_handle *h) {
     if (h->sm_count > 0) return KVQ_OK;
     int dev = 0;
@@ -279,6 +457,100 @@ static int splits_for(kvq_handle *h, int layer, int *S_out, int *nstage_out) {
     return KVQ_OK;
 }
 
+// ------------------------------------------------------------------ paged plans
+static void paged_units(const kvq_handle *h, int layer, int *u2, int *u4) {
+    const auto &P = h->pl[layer];
+    *u2 = *u4 = 0;
+    for (int b = 0; b < h->desc.batch; ++b) {
+        *u2 = std::max(*u2, P.n2g[b]);
+        *u4 = std::max(*u4, (P.n4[b] + 15) / 16 + (P.np[b] + 15) / 16);
+    }
+}
+
+// INT2 and INT4 split counts: minimise (waves) x (slowest CTA), an INT2 unit (32 tokens,
+// 2-bit record) weighing 1 and an INT4 page (16 tokens) 0.55.
+static int paged_splits(kvq_handle *h, int layer, int *S2, int *S4) {
+    int u2, u4;
+    paged_units(h, layer, &u2, &u4);
+    int rc = ensure_device_info(h);
+    if (rc) return rc;
+    int per_sm = 1;
+    cudaError_t e = kvq::decode_paged_occupancy(kvq::decode_paged_stages(), &per_sm);
+    if (e != cudaSuccess) return cuda_fail(e, "paged decode occupancy");
+    const int slots = std::max(1, per_sm) * h->sm_count;
+    const int units = h->desc.batch * h->desc.n_kv_heads;
+    if (h->forced_splits > 0) {
+        const int f = std::min(h->forced_splits, kvq::kMaxSplits);
+        *S2 = u2 > 0 ? std::max(1, std::min(u2, (f + 1) / 2)) : 0;
+        *S4 = u4 > 0 ? std::max(1, std::min(u4, f - *S2 > 0 ? f - *S2 : 1)) : 0;
+        return KVQ_OK;
+    }
+    double best = 1e300;
+    *S2 = u2 > 0 ? 1 : 0;
+    *S4 = u4 > 0 ? 1 : 0;
+    for (int a = (u2 > 0 ? 1 : 0); a <= (u2 > 0 ? std::min(32, u2) : 0); ++a)
+        for (int c = (u4 > 0 ? 1 : 0); c <= (u4 > 0 ? std::min(48, u4) : 0); ++c) {
+            if (a + c < 1 || a + c > kvq::kMaxSplits) continue;
+            const double t2 = a ? std::ceil(std::ceil(static_cast<double>(u2) / a) / kvq::kDecodeWarps) : 0.0;
+            const double t4 = c ? 0.55 * std::ceil(std::ceil(static_cast<double>(u4) / c) / kvq::kDecodeWarps) : 0.0;
+            const double waves = std::ceil(static_cast<double>(units) * (a + c) / slots);
+            const double cost = waves * (std::max(t2, t4) + 1.0) * (1.0 + 0.002 * (a + c));
+            if (cost < best - 1e-9) {
+                best = cost;
+                *S2 = a;
+                *S4 = c;
+            }
+        }
+    return KVQ_OK;
+}
+
+static int decode_paged(kvq_handle *h, int layer, const void *q, void *out, int out_fp32, cudaStream_t st,
+                        float *part_acc, float *part_ml) {
+    int S2 = 0, S4 = 0;
+    int rc = paged_splits(h, layer, &S2, &S4);
+    if (rc) return rc;
+    const auto &P = h->pl[layer];
+    kvq::PagedDecodeParams p{};
+    p.pool2 = h->ws + h->pool2_off[layer];
+    p.pool4 = h->ws + h->pool4_off[layer];
+    p.n2_cap = h->n2_cap;
+    p.n4_cap = h->n4_cap;
+    p.table = reinterpret_cast<const int *>(h->ws + h->table_off[layer]);
+    p.P_cap = h->P_cap;
+    p.pend_base = h->pend_base;
+    for (int b = 0; b < h->desc.batch; ++b) p.cnt[b] = kvq::PagedCounts{P.n2g[b], P.n4[b], P.np[b], 0};
+    p.q = static_cast<const uint16_t *>(q);
+    p.smax = reinterpret_cast<const unsigned *>(h->ws + h->smax_off) + 2 * layer;
+    p.out = out;
+    p.part_acc = part_acc;
+    p.part_ml = part_ml;
+    p.status = reinterpret_cast<unsigned *>(h->ws + h->status_off);
+    p.B = h->desc.batch;
+    p.Hkv = h->desc.n_kv_heads;
+    p.G = h->desc.n_q_heads / h->desc.n_kv_heads;
+    p.S2 = S2;
+    p.S4 = S4;
+    p.out_fp32 = out_fp32 ? 1 : 0;
+    p.nstage = kvq::decode_paged_stages();
+    if ((rc = prepare_status(h, st))) return rc;
+    cudaError_t e = kvq::launch_decode_paged(p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "paged decode launch");
+    if (S2 + S4 > 1) {
+        kvq::MergeParams m{};
+        m.part_acc = part_acc;
+        m.part_ml = part_ml;
+        m.out = out;
+        m.B = p.B;
+        m.Hq = h->desc.n_q_heads;
+        m.D = h->desc.head_dim;
+        m.S = S2 + S4;
+        m.out_fp32 = p.out_fp32;
+        e = kvq::launch_merge(m, st);
+        if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+    }
+    return ok();
+}
+
 int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_fp32, void *stream) {
     int rc = check_layer(h, layer);
     if (rc) return rc;
@@ -287,6 +559,10 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
     if (!aligned(q, 16) || !aligned(out, 16)) return fail(KVQ_EALIGN, "q and out must be 16-byte aligned");
     const int L = h->len[layer];
     if (L < 1) return fail(KVQ_EINVAL, "layer %d is empty", layer);
+    if (h->desc.paged)
+        return decode_paged(h, layer, q, out, out_fp32, static_cast<cudaStream_t>(stream),
+                            reinterpret_cast<float *>(h->ws + h->part_acc_off),
+                            reinterpret_cast<float *>(h->ws + h->part_ml_off));
     int S = 1, nstage = 2;
     if ((rc = splits_for(h, layer, &S, &nstage))) return rc;
     const LayerGeom &g = h->geom[layer];
@@ -347,6 +623,12 @@ int kvq_get_num_splits(const kvq_handle *hc, int layer, int *num_splits) {
         *num_splits = 0;
         return ok();
     }
+    if (h->desc.paged) {
+        int S2 = 0, S4 = 0;
+        if ((rc = paged_splits(h, layer, &S2, &S4))) return rc;
+        *num_splits = S2 + S4;
+        return ok();
+    }
     int S = 1, nstage = 2;
     if ((rc = splits_for(h, layer, &S, &nstage))) return rc;
     const int nblk = (L + 31) / 32;
@@ -355,10 +637,79 @@ int kvq_get_num_splits(const kvq_handle *hc, int layer, int *num_splits) {
     return ok();
 }
 
+static int export_paged(const kvq_handle *h, int layer, void *host_buf, size_t bytes, size_t *needed) {
+    const int B = h->desc.batch, Hkv = h->desc.n_kv_heads, D = h->desc.head_dim, nj = D / 32;
+    const auto &P = h->pl[layer];
+    const long long REC2 = h->rec2_bytes, PAGE4 = h->page4_bytes, STG = 2LL * 32 * D * 2;
+    std::vector<long long> unit_bytes(B);
+    long long total = 0;
+    for (int b = 0; b < B; ++b) {
+        unit_bytes[b] = P.n2g[b] * REC2 + ((P.n4[b] + 15) / 16 + 2) * PAGE4 + STG;
+        total += unit_bytes[b] * Hkv;
+    }
+    *needed = static_cast<size_t>(total);
+    if (!host_buf) return ok();
+    if (bytes < *needed) return fail(KVQ_EINVAL, "export buffer too small: %zu < %zu", bytes, *needed);
+    int rc = check_bound(h);
+    if (rc) return rc;
+    if (!h->status_clear) return fail(KVQ_EINVAL, "nothing appended since the workspace was bound");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    std::vector<uint8_t> pool2(static_cast<size_t>(h->n2_cap * REC2 * Hkv));
+    std::vector<uint8_t> pool4(static_cast<size_t>(h->n4_cap * PAGE4 * Hkv));
+    std::vector<uint8_t> stg(static_cast<size_t>(STG * B * Hkv));
+    e = cudaMemcpy(pool2.data(), h->ws + h->pool2_off[layer], pool2.size(), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemcpy(pool4.data(), h->ws + h->pool4_off[layer], pool4.size(), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemcpy(stg.data(), h->ws + h->staging_off[layer], stg.size(), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy (paged pools)");
+    // zero the scale/zero entries of absent tokens u >= r of a 16-token page
+    auto zero_absent = [&](uint8_t *page, int r) {
+        for (int u = r; u < 16; ++u)
+            for (int j = 0; j < nj; ++j) {
+                const long long so = 8LL * nj * (u / 2) + 4LL * j + 2LL * (u % 2);
+                for (long long area : {2LL * D * 4, 2LL * D * 4 + 2LL * D + 2LL * D * 4}) {
+                    std::memset(page + area + so, 0, 2);
+                    std::memset(page + area + so + 4LL * nj, 0, 2);
+                }
+            }
+    };
+    uint8_t *dst = static_cast<uint8_t *>(host_buf);
+    for (int b = 0; b < B; ++b)
+        for (int h2 = 0; h2 < Hkv; ++h2) {
+            uint8_t *img = dst;
+            for (int g = 0; g < P.n2g[b]; ++g)
+                std::memcpy(img + g * REC2, pool2.data() + (static_cast<long long>(h2) * h->n2_cap + P.rec2[b][g]) * REC2, REC2);
+            uint8_t *pg = img + P.n2g[b] * REC2;
+            const int n4p = (P.n4[b] + 15) / 16;
+            for (int i = 0; i < n4p; ++i) {
+                std::memcpy(pg + i * PAGE4, pool4.data() + (static_cast<long long>(h2) * h->n4_cap + P.page4[b][i]) * PAGE4, PAGE4);
+                if (i == n4p - 1 && P.n4[b] % 16) zero_absent(pg + i * PAGE4, P.n4[b] % 16);
+            }
+            uint8_t *pend = pg + n4p * PAGE4;
+            const int np = P.np[b];
+            for (int i = 0; i < 2; ++i) {
+                if (np > 16 * i) {
+                    std::memcpy(pend + i * PAGE4, pool4.data() + (static_cast<long long>(h2) * h->n4_cap + h->pend_base + 2 * b + i) * PAGE4, PAGE4);
+                    if (np < 16 * (i + 1)) zero_absent(pend + i * PAGE4, np - 16 * i);
+                } else {
+                    std::memset(pend + i * PAGE4, 0, PAGE4);
+                }
+            }
+            uint8_t *sg = pend + 2 * PAGE4;
+            const uint8_t *src = stg.data() + (static_cast<long long>(b) * Hkv + h2) * STG;
+            std::memset(sg, 0, STG);
+            std::memcpy(sg, src, 2LL * np * D);                            // keys of slots [0, np)
+            std::memcpy(sg + STG / 2, src + STG / 2, 2LL * np * D);        // values
+            dst += unit_bytes[b];
+        }
+    return ok();
+}
+
 int kvq_export_layer(const kvq_handle *h, int layer, void *host_buf, size_t bytes, size_t *needed) {
     int rc = check_layer(h, layer);
     if (rc) return rc;
     if (!needed) return fail(KVQ_EINVAL, "null argument");
+    if (h->desc.paged) return export_paged(h, layer, host_buf, bytes, needed);
     const LayerGeom &g = h->geom[layer];
     const int L = h->len[layer];
     const int nblk = (L + 31) / 32;
@@ -426,6 +777,7 @@ int kvq_truncate(kvq_handle *h, int layer, int L) {
     if (rc) return rc;
     if (L < 0 || L > h->len[layer]) return fail(KVQ_EINVAL, "truncate length %d outside [0, %d]", L, h->len[layer]);
     if (L % 32) return fail(KVQ_EINVAL, "truncate length must be a multiple of 32 (got %d)", L);
+    if (h->desc.paged) return fail(KVQ_EUNSUPPORTED, "paged plans cannot be truncated");
     h->len[layer] = L;
     return ok();
 }
@@ -495,6 +847,7 @@ int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, 
     if (!aligned(q, 16) || !aligned(out, 16)) return fail(KVQ_EALIGN, "q and out must be 16-byte aligned");
     const int L = h->len[layer];
     if (L < 1) return fail(KVQ_EINVAL, "layer %d is empty", layer);
+    if (h->desc.paged) return fail(KVQ_EUNSUPPORTED, "paged plans are not supported by kvq_decode_attn_noalloc");
     int S = 1, nstage = 2;
     if ((rc = splits_for(h, layer, &S, &nstage))) return rc;
     const LayerGeom &g = h->geom[layer];

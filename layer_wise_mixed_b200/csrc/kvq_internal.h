@@ -48,6 +48,58 @@ struct DecodeParams {
     long long rec_bytes;
 };
 
+// ---------------------------------------------------------------- paged INT2/INT4
+constexpr int kMaxPagedBatch = 64;   // requests per paged plan (kernel-parameter tables)
+
+struct PagedCounts {
+    int n2g;    // complete INT2 groups (32 tokens each)
+    int n4;     // tokens in the INT4 main pages
+    int np;     // INT2 tokens of the open group (held as INT4 in the pending pages)
+    int pad;
+};
+
+struct PagedDecodeParams {
+    const uint8_t *pool2;       // [Hkv][n2_cap records] of 32-token INT2 records
+    const uint8_t *pool4;       // [Hkv][n4_cap pages] of 16-token INT4 pages (pending pages last)
+    long long n2_cap, n4_cap;
+    const int *table;           // [B][P_cap]: INT2 first pages from the front, INT4 pages from the back
+    int P_cap, pend_base;
+    PagedCounts cnt[kMaxPagedBatch];
+    const uint16_t *q;
+    const unsigned *smax;
+    void *out;
+    float *part_acc, *part_ml;
+    unsigned *status;
+    int B, Hkv, G, S2, S4, out_fp32, nstage;
+};
+
+struct PagedReq {               // one request's append plan
+    int n2g_old, n4_old, np_old;
+    int k2, k4;                 // new INT2 / INT4 tokens in this call
+    int ng;                     // INT2 groups completed by this call
+    int base2;                  // first new INT2 record id
+    int base4;                  // first new INT4 main page id
+    int last4;                  // page id of the partly filled INT4 main page (-1 if none)
+    int c4, c2;                 // CTAs of this request: INT4 main pages touched, INT2 work CTAs
+};
+
+struct PagedAppendParams {
+    const uint16_t *K, *V;      // bf16 [B][Hkv][n][D]
+    const uint8_t *tags;        // device [B][n]: 2 or 4
+    const int *inv2, *inv4;     // [B][n_max]: input index of the r-th new INT2 / INT4 token (n > 1)
+    int inv_stride;
+    uint8_t *pool2, *pool4;
+    long long n2_cap, n4_cap;
+    int *table;
+    int P_cap, pend_base;
+    uint16_t *staging;          // [B][Hkv][2][32][D] bf16 originals of the open INT2 group (K, V)
+    unsigned *smax;
+    int B, Hkv, D, n;
+    int cta4_off[kMaxPagedBatch + 1];   // prefix offsets of the INT4-page CTAs per request
+    int cta2_off[kMaxPagedBatch + 1];   // prefix offsets of the INT2 CTAs per request
+    PagedReq req[kMaxPagedBatch];
+};
+
 struct MergeParams {
     const float *part_acc;
     const float *part_ml;
@@ -62,6 +114,15 @@ cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmod
 cudaError_t decode_occupancy(int D, int bk, int bv, int kmode, int G, long long rec_bytes,
                              int nstage, int *ctas_per_sm);
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t st);
+cudaError_t launch_decode_paged(const PagedDecodeParams &p, cudaStream_t st);
+cudaError_t decode_paged_occupancy(int nstage, int *ctas_per_sm);
+int decode_paged_stages();
+size_t decode_paged_smem_bytes(int nstage);
+cudaError_t launch_paged_scan(const uint8_t *tags, int B, int n, int *inv2, int *inv4, int inv_stride,
+                              cudaStream_t st);
+cudaError_t launch_paged_append(const PagedAppendParams &p, int grid, cudaStream_t st);
+int paged_rec2_bytes(int D);
+int paged_page4_bytes(int D);
 int decode_stages(long long rec_bytes, int D, int G);
 size_t decode_smem_bytes(long long rec_bytes, int nstage, int D, int G);
 

@@ -67,6 +67,7 @@ def load() -> ctypes.CDLL:
         "kvq_workspace_bytes": (I, [P, ctypes.POINTER(SZ)]),
         "kvq_bind": (I, [P, P, SZ]),
         "kvq_append": (I, [P, I, P, P, I, P]),
+        "kvq_append_tagged": (I, [P, I, P, P, I, P, P, P]),
         "kvq_decode_attn": (I, [P, I, P, P, I, P]),
         "kvq_decode_attn_noalloc": (I, [P, I, P, P, I, P]),
         "kvq_set_num_splits": (I, [P, I]),
@@ -132,6 +133,13 @@ def kvq_append(h: int, layer: int, K, V, n_new: int, stream=None):
     _check(load().kvq_append(h, layer, _ptr(K), _ptr(V), n_new, _stream(stream)))
 
 
+def kvq_append_tagged(h: int, layer: int, K, V, n_new: int, host_tags, dev_tags, stream=None):
+    """host_tags: contiguous uint8 numpy array [B, n_new]; dev_tags: the same bytes on the device."""
+    host_tags = np.ascontiguousarray(host_tags, np.uint8)
+    _check(load().kvq_append_tagged(h, layer, _ptr(K), _ptr(V), n_new, host_tags.ctypes.data_as(ctypes.c_void_p),
+                                    _ptr(dev_tags), _stream(stream)))
+
+
 def kvq_decode_attn(h: int, layer: int, q, out, out_fp32: bool, stream=None):
     _check(load().kvq_decode_attn(h, layer, _ptr(q), _ptr(out), int(bool(out_fp32)), _stream(stream)))
 
@@ -185,6 +193,11 @@ def kvq_last_error() -> str:
 
 
 # ------------------------------------------------------------------ convenience owner
+def make_paged_desc(num_layers: int, batch: int, n_kv_heads: int, n_q_heads: int, head_dim: int, max_ctx: int,
+                    avg_bits: float):
+    return kvq_plan_desc(num_layers, batch, n_kv_heads, n_q_heads, head_dim, 32, max_ctx, None, 1, 16, avg_bits)
+
+
 def make_desc(num_layers: int, batch: int, n_kv_heads: int, n_q_heads: int, head_dim: int, max_ctx: int,
               layer_bits: Sequence[Tuple[int, int]], kmodes: Optional[Sequence[int]] = None):
     cfgs = (kvq_layer_cfg * num_layers)()
@@ -196,12 +209,16 @@ def make_desc(num_layers: int, batch: int, n_kv_heads: int, n_q_heads: int, head
 
 
 class Cache:
-    """A plan plus a torch-allocated workspace on the current CUDA device."""
+    """A plan plus a torch-allocated workspace on the current CUDA device.  Pass
+    avg_bits (and no layer_bits) for a paged INT2/INT4 plan."""
 
-    def __init__(self, num_layers, batch, n_kv_heads, n_q_heads, head_dim, max_ctx, layer_bits,
-                 kmodes=None, device="cuda"):
+    def __init__(self, num_layers, batch, n_kv_heads, n_q_heads, head_dim, max_ctx, layer_bits=None,
+                 kmodes=None, device="cuda", avg_bits=None):
         import torch
-        self.desc = make_desc(num_layers, batch, n_kv_heads, n_q_heads, head_dim, max_ctx, layer_bits, kmodes)
+        if avg_bits is not None:
+            self.desc = make_paged_desc(num_layers, batch, n_kv_heads, n_q_heads, head_dim, max_ctx, avg_bits)
+        else:
+            self.desc = make_desc(num_layers, batch, n_kv_heads, n_q_heads, head_dim, max_ctx, layer_bits, kmodes)
         self.h = kvq_plan(self.desc)
         self.nbytes = kvq_workspace_bytes(self.h)
         self.ws = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
@@ -213,6 +230,11 @@ class Cache:
     def append(self, layer, K, V, stream=None):
         assert K.is_contiguous() and V.is_contiguous() and K.shape == V.shape
         kvq_append(self.h, layer, K, V, K.shape[2], stream)
+
+    def append_tagged(self, layer, K, V, tags, stream=None):
+        """tags: uint8 torch tensor [B, n] (2 or 4) on the device."""
+        assert K.is_contiguous() and V.is_contiguous() and K.shape == V.shape
+        kvq_append_tagged(self.h, layer, K, V, K.shape[2], tags.cpu().numpy(), tags, stream)
 
     def decode_attn(self, layer, q, out=None, out_fp32=False, stream=None):
         import torch

@@ -64,6 +64,16 @@ def lib():
         L.orc_attention.argtypes = [P, P, P, i32, i32, i32, P]
         L.orc_layer.restype = i32
         L.orc_layer.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, P, P]
+        L.orc_paged_unit.restype = i32
+        L.orc_paged_unit.argtypes = [P, P, P, i32, i32, P, P, P]
+        L.orc_paged_unit_bytes.restype = i64
+        L.orc_paged_unit_bytes.argtypes = [P, i32, i32]
+        L.orc_paged_layer.restype = i32
+        L.orc_paged_layer.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, P, P]
+        L.orc_paged_page4_bytes.restype = i64
+        L.orc_paged_page4_bytes.argtypes = [i32]
+        L.orc_paged_rec2_bytes.restype = i64
+        L.orc_paged_rec2_bytes.argtypes = [i32]
         L.orc_f32_to_f16_array.restype = None
         L.orc_f32_to_f16_array.argtypes = [P, P, i64]
         L.orc_f16_to_f64_array.restype = None
@@ -224,3 +234,53 @@ def layer(K, V, Q, G: int, bk: int, bv: int, kmode: int, want_image=True, want_o
     if rc != 0:
         raise ValueError("orc_layer rejected its arguments")
     return img, out
+
+
+# ---------------------------------------------------------------- paged INT2/INT4
+def paged_unit(K, V, tags, D: int, want_image=True, want_dequant=True):
+    """One (batch, kv head) unit of the paged cache. K, V: [L, D] bf16 bits; tags: [L]
+    uint8 (2 or 4).  Returns (image, Kh, Vh) with Kh/Vh in token order."""
+    K = _u16(K).reshape(-1, D)
+    V = _u16(V).reshape(-1, D)
+    tags = np.ascontiguousarray(tags, np.uint8)
+    L = K.shape[0]
+    n = int(lib().orc_paged_unit_bytes(_p(tags), L, D))
+    img = np.empty(n, np.uint8) if want_image else None
+    Kh = np.empty((L, D), np.float64) if want_dequant else None
+    Vh = np.empty((L, D), np.float64) if want_dequant else None
+    rc = lib().orc_paged_unit(_p(K), _p(V), _p(tags), L, D, _p(img) if img is not None else None,
+                              _p(Kh) if Kh is not None else None, _p(Vh) if Vh is not None else None)
+    if rc != 0:
+        raise ValueError("orc_paged_unit rejected its arguments")
+    return img, Kh, Vh
+
+
+def paged_layer(K, V, tags, Q, G: int, want_image=True, want_out=True):
+    """K, V: [B, Hkv, L, D] bf16 bits; tags [B, L]; Q [B, Hkv*G, D].  Returns (image, out)."""
+    K = _u16(K)
+    V = _u16(V)
+    tags = np.ascontiguousarray(tags, np.uint8)
+    B, Hkv, L, D = K.shape
+    img = None
+    if want_image:
+        tot = sum(int(lib().orc_paged_unit_bytes(_p(np.ascontiguousarray(tags[b])), L, D)) for b in range(B)) * Hkv
+        img = np.empty(tot, np.uint8)
+    out = None
+    Qp = None
+    if want_out:
+        Q = _u16(Q)
+        out = np.empty((B, Hkv * G, D), np.float64)
+        Qp = _p(Q)
+    rc = lib().orc_paged_layer(_p(K), _p(V), _p(tags), Qp, B, Hkv, G, L, D,
+                               _p(img) if img is not None else None, _p(out) if out is not None else None)
+    if rc != 0:
+        raise ValueError("orc_paged_layer rejected its arguments")
+    return img, out
+
+
+def paged_page4_bytes(D: int) -> int:
+    return int(lib().orc_paged_page4_bytes(D))
+
+
+def paged_rec2_bytes(D: int) -> int:
+    return int(lib().orc_paged_rec2_bytes(D))

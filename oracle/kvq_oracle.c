@@ -75,6 +75,20 @@
  *     then (per-channel K only) the residual; every byte that holds no token of
  *     0..L-1 is zero (the unfilled part of the last block and of the residual).
  *
+ * Q5  Paged INT2/INT4 token-mixed cache ([TRI] Facts: quantizer, leftovers, page
+ *     pools, decode path).  Every token carries a tag, 2 or 4.  The INT2-tagged tokens,
+ *     in arrival order, form groups of 32: keys per channel with 2 bits, values per token
+ *     with 2 bits (a 32-token record as in Q3, bk = bv = 2).  INT4-tagged tokens are
+ *     quantized per token, keys and values with 4 bits, into 16-token pages
+ *     [K codes 2*D*4 B][K s/z 2*D B][V codes 2*D*4 B][V s/z 2*D B] (the Q3 layouts of one
+ *     16-token half).  The n2 mod 32 INT2 tokens after the last complete group are held
+ *     the same INT4 way in two pending pages, and their bf16 originals in a 32-slot
+ *     staging area (reading: the leftovers go through the INT4 per-token path, values
+ *     too, so pages stay homogeneous, until their group of 32 completes).
+ *     Canonical image of a (b, h) unit: the INT2 records in group order, the INT4 pages
+ *     in order, the two pending pages, then the staging keys and values (32 x D bf16
+ *     each); bytes that hold no token are zero.
+ *
  * Q4  Attention (fp64): O[hq] = sum_t softmax_t(q . k^_t / sqrt(D)) v^_t over all L
  *     cached tokens, quantized ones and residual alike, no mask; GQA: the kv head
  *     of query head hq is hq / G.
@@ -342,6 +356,160 @@ int orc_unit(const uint16_t *K, const uint16_t *V, int L, int D, int bk, int bv,
         }
     }
     return 0;
+}
+
+/* ---------------- Q5: paged INT2/INT4 unit ---------------- */
+
+void orc_attention(const uint16_t *q, const double *Kh, const double *Vh, int L, int D, int G, double *out);
+
+long orc_paged_page4_bytes(int D) { return 20L * D; }
+long orc_paged_rec2_bytes(int D) { return orc_record_bytes(D, 2, 2); }
+
+/* Counts of a tag sequence: complete INT2 groups, INT4 tokens, pending INT2 tokens. */
+void orc_paged_counts(const uint8_t *tags, int L, int *n2g, int *n4, int *np) {
+    int n2 = 0, c4 = 0;
+    for (int i = 0; i < L; i++) {
+        if (tags[i] == 2) n2++;
+        else c4++;
+    }
+    *n2g = n2 / 32;
+    *np = n2 % 32;
+    *n4 = c4;
+}
+
+long orc_paged_unit_bytes(const uint8_t *tags, int L, int D) {
+    int n2g, n4, np;
+    orc_paged_counts(tags, L, &n2g, &n4, &np);
+    return n2g * orc_paged_rec2_bytes(D) + ((n4 + 15) / 16 + 2) * orc_paged_page4_bytes(D) + 128L * D;
+}
+
+/* Per-token quantization of one token (bits) into slot u of a 16-token page half:
+ * codes into the code area (role 0 keys, 1 values), scale/zero into the s/z area. */
+static void orc_token_to_page(const uint16_t *row, int D, int bits, int role, uint8_t *codes_area,
+                              uint8_t *sz_area, int u, double *deq) {
+    const int nj = D / 32;
+    float x[32];
+    uint8_t c[32];
+    uint16_t s16, z16;
+    for (int j = 0; j < nj; j++) {
+        for (int i = 0; i < 32; i++) x[i] = orc_bf16_to_f32(row[32 * j + i]);
+        orc_quant(x, 32, 1, bits, &s16, &z16, c, 1);
+        put_tok_sz(sz_area, u, j, nj, s16, z16);
+        for (int i = 0; i < 32; i++) orc_put_code(codes_area, role, u, 32 * j + i, D, bits, c[i]);
+        if (deq) {
+            double s = orc_f16_to_f64(s16), z = orc_f16_to_f64(z16);
+            for (int i = 0; i < 32; i++) deq[32 * j + i] = c[i] * s + z;
+        }
+    }
+}
+
+/* One (b, h) unit of the paged cache from its K, V ([L][D] bf16) and tags [L]. */
+int orc_paged_unit(const uint16_t *K, const uint16_t *V, const uint8_t *tags, int L, int D, uint8_t *img,
+                   double *Kh, double *Vh) {
+    if (D % 32 || D <= 0 || D > 512 || L < 0) return -1;
+    const int nj = D / 32;
+    const long REC2 = orc_paged_rec2_bytes(D), PAGE4 = orc_paged_page4_bytes(D);
+    const long KC2 = 4L * D * 2, KS2 = 4L * D, VC2 = 4L * D * 2;
+    const long KC4 = 2L * D * 4, KS4 = 2L * D, VC4 = 2L * D * 4;
+    int n2g, n4, np;
+    orc_paged_counts(tags, L, &n2g, &n4, &np);
+    const int n4p = (n4 + 15) / 16;
+    int *i2 = (int *)malloc(sizeof(int) * (size_t)(L + 1));
+    int *i4 = (int *)malloc(sizeof(int) * (size_t)(L + 1));
+    int n2 = 0, c4 = 0;
+    for (int i = 0; i < L; i++) {
+        if (tags[i] == 2) i2[n2++] = i;
+        else i4[c4++] = i;
+    }
+    if (img) memset(img, 0, (size_t)orc_paged_unit_bytes(tags, L, D));
+    uint8_t *pg4 = img ? img + n2g * REC2 : NULL;
+    uint8_t *pend = img ? pg4 + n4p * PAGE4 : NULL;
+    uint8_t *stage = img ? pend + 2 * PAGE4 : NULL;
+    float x[32];
+    uint8_t c[32];
+    uint16_t s16, z16;
+
+    /* INT2 groups: keys per channel over the group's 32 tokens, values per token */
+    for (int g = 0; g < n2g; g++) {
+        uint8_t *rec = img ? img + g * REC2 : NULL;
+        for (int d = 0; d < D; d++) {
+            for (int u = 0; u < 32; u++) x[u] = orc_bf16_to_f32(K[(long)i2[32 * g + u] * D + d]);
+            orc_quant(x, 32, 1, 2, &s16, &z16, c, 1);
+            if (rec) {
+                put_chan_sz(rec + KC2, d, s16, z16);
+                for (int u = 0; u < 32; u++) orc_put_code(rec, 0, u, d, D, 2, c[u]);
+            }
+            if (Kh) {
+                double s = orc_f16_to_f64(s16), z = orc_f16_to_f64(z16);
+                for (int u = 0; u < 32; u++) Kh[(long)i2[32 * g + u] * D + d] = c[u] * s + z;
+            }
+        }
+        for (int u = 0; u < 32; u++) {
+            const int tok = i2[32 * g + u];
+            for (int j = 0; j < nj; j++) {
+                for (int i = 0; i < 32; i++) x[i] = orc_bf16_to_f32(V[(long)tok * D + 32 * j + i]);
+                orc_quant(x, 32, 1, 2, &s16, &z16, c, 1);
+                if (rec) {
+                    put_tok_sz(rec + KC2 + KS2 + VC2, u, j, nj, s16, z16);
+                    for (int i = 0; i < 32; i++) orc_put_code(rec + KC2 + KS2, 1, u, 32 * j + i, D, 2, c[i]);
+                }
+                if (Vh) {
+                    double s = orc_f16_to_f64(s16), z = orc_f16_to_f64(z16);
+                    for (int i = 0; i < 32; i++) Vh[(long)tok * D + 32 * j + i] = c[i] * s + z;
+                }
+            }
+        }
+    }
+    /* INT4 tokens (main pages), then the pending INT2 tokens (pending pages + staging) */
+    for (int r = 0; r < n4 + np; r++) {
+        const int pending = r >= n4;
+        const int tok = pending ? i2[32 * n2g + (r - n4)] : i4[r];
+        const int slot = pending ? r - n4 : r;
+        uint8_t *page = img ? (pending ? pend : pg4) + (slot / 16) * PAGE4 : NULL;
+        const int u = slot % 16;
+        uint8_t tmp_codes[4096];
+        uint8_t tmp_sz[1024];
+        uint8_t *kcodes = page ? page : tmp_codes, *ksz = page ? page + KC4 : tmp_sz;
+        uint8_t *vcodes = page ? page + KC4 + KS4 : tmp_codes, *vsz = page ? page + KC4 + KS4 + VC4 : tmp_sz;
+        orc_token_to_page(K + (long)tok * D, D, 4, 0, kcodes, ksz, u, Kh ? Kh + (long)tok * D : NULL);
+        orc_token_to_page(V + (long)tok * D, D, 4, 1, vcodes, vsz, u, Vh ? Vh + (long)tok * D : NULL);
+        if (pending && stage) {
+            memcpy(stage + 2L * slot * D, K + (long)tok * D, 2L * D);
+            memcpy(stage + 64L * D + 2L * slot * D, V + (long)tok * D, 2L * D);
+        }
+    }
+    free(i2);
+    free(i4);
+    return 0;
+}
+
+/* A whole paged layer: K, V [B][Hkv][L][D], tags [B][L] (shared by heads), Q [B][Hkv*G][D].
+ * img: unit images concatenated in (b, h) order; out [B][Hq][D]. */
+int orc_paged_layer(const uint16_t *K, const uint16_t *V, const uint8_t *tags, const uint16_t *Q, int B, int Hkv,
+                    int G, int L, int D, uint8_t *img, double *out) {
+    long *off = (long *)malloc(sizeof(long) * (size_t)(B * Hkv + 1));
+    off[0] = 0;
+    for (int un = 0; un < B * Hkv; un++) off[un + 1] = off[un] + orc_paged_unit_bytes(tags + (long)(un / Hkv) * L, L, D);
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+    for (int un = 0; un < B * Hkv; un++) {
+        int b = un / Hkv, h = un % Hkv;
+        double *Kh = NULL, *Vh = NULL;
+        if (out) {
+            Kh = (double *)malloc(sizeof(double) * (size_t)L * D);
+            Vh = (double *)malloc(sizeof(double) * (size_t)L * D);
+        }
+        err |= orc_paged_unit(K + (long)un * L * D, V + (long)un * L * D, tags + (long)b * L, L, D,
+                              img ? img + off[un] : NULL, Kh, Vh) != 0;
+        if (out) {
+            orc_attention(Q + ((long)b * Hkv * G + (long)h * G) * D, Kh, Vh, L, D, G,
+                          out + ((long)b * Hkv * G + (long)h * G) * D);
+            free(Kh);
+            free(Vh);
+        }
+    }
+    free(off);
+    return err ? -1 : 0;
 }
 
 /* ---------------- Q4: attention in binary64 ---------------- */

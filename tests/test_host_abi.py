@@ -113,3 +113,47 @@ def test_product_path_has_no_fallback(monkeypatch, tmp_path):
     monkeypatch.setattr(kvq, "_lib", None)
     with pytest.raises(FileNotFoundError):
         kvq.load()
+
+
+def paged_rc(**kw):
+    a = dict(num_layers=2, batch=3, n_kv_heads=2, n_q_heads=8, head_dim=128, max_ctx=200, avg_bits=3.0)
+    a.update(kw)
+    d = kvq.make_paged_desc(a["num_layers"], a["batch"], a["n_kv_heads"], a["n_q_heads"], a["head_dim"],
+                            a["max_ctx"], a["avg_bits"])
+    return plan_rc(d)
+
+
+def test_paged_plan_validation(lib):
+    assert paged_rc() == kvq.KVQ_OK
+    assert paged_rc(head_dim=64) == kvq.KVQ_EUNSUPPORTED
+    assert paged_rc(n_q_heads=14) == kvq.KVQ_EUNSUPPORTED          # G = 7
+    assert paged_rc(batch=65) == kvq.KVQ_EUNSUPPORTED
+    assert paged_rc(avg_bits=5.0) == kvq.KVQ_EINVAL
+    assert paged_rc(avg_bits=1.5) == kvq.KVQ_EINVAL
+
+
+def test_paged_host_checks(lib):
+    import numpy as np
+    d = kvq.make_paged_desc(1, 2, 2, 8, 128, 300, 4.0)    # avg 4 bits: the INT2 pool holds ~2 groups
+    h = kvq.kvq_plan(d)
+    L = kvq.load()
+    try:
+        n = kvq.kvq_workspace_bytes(h)
+        fake = 1 << 40
+        assert L.kvq_bind(h, fake, n) == kvq.KVQ_OK
+        assert L.kvq_append(h, 0, fake, fake, 1, None) == kvq.KVQ_EINVAL      # needs the tagged entry
+        bad = np.full((2, 3), 3, np.uint8)
+        ptr = bad.ctypes.data_as(ctypes.c_void_p)
+        assert L.kvq_append_tagged(h, 0, fake, fake, 3, ptr, fake, None) == kvq.KVQ_EINVAL
+        assert "must be 2 or 4" in kvq.kvq_last_error()
+        many2 = np.full((2, 200), 2, np.uint8)                   # 12 groups > INT2 pool
+        ptr = many2.ctypes.data_as(ctypes.c_void_p)
+        assert L.kvq_append_tagged(h, 0, fake, fake, 200, ptr, fake, None) == kvq.KVQ_ECAPACITY
+        assert "INT2 pool full" in kvq.kvq_last_error()
+        assert kvq.kvq_seq_len(h, 0) == 0                        # nothing committed
+        assert L.kvq_truncate(h, 0, 0) == kvq.KVQ_EUNSUPPORTED
+        need = ctypes.c_size_t()
+        assert L.kvq_export_layer(h, 0, None, 0, ctypes.byref(need)) == kvq.KVQ_OK
+        assert need.value == 2 * 2 * (2 * 20 * 128 + 2 * 32 * 128 * 2)   # empty: pending pages + staging
+    finally:
+        kvq.kvq_destroy(h)
