@@ -186,9 +186,11 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t 
     lo = pack_h2(a - ha, b - hb);
 }
 
-// Floats of the per-warp combine buffer: O^T columns [8*NT][D], value zero-point
-// terms [8*NT][NJ], running max and sum per head [8] + [8].
-__host__ __device__ constexpr int comb_floats(int D, int NT) { return 8 * NT * D + 8 * NT * (D / 32) + 16; }
+// Floats of the per-warp combine buffer: O^T columns [8*NT][D] (zero-point term folded
+// in), running max and sum per head [8] + [8]; plus kCombShared floats shared by the CTA
+// (per-warp merge weights and per-head denominators).
+__host__ __device__ constexpr int comb_floats(int D, int NT) { return 8 * NT * D + 16; }
+constexpr int kCombShared = 64;
 
 // Bytes of one unit record: NH 16-token halves of codes, fp16 scales/zeros.
 __host__ __device__ constexpr int unit_bytes(int D, int BK, int BV, int KM, int NH) {
@@ -217,10 +219,13 @@ struct WarpAcc {
 //    kq chosen so that q~ s_k < 2^14 and q~ < 2^15; scores = raw * 2^-kq.
 //  per-token keys: raw q (exact in fp16), rows (group j, head) masked to group j;
 //    scores = raw * log2(e)/sqrt(D).
+// Computed by warp 0 only; every lane's scalars (unscale, qsum_g, qsum_g8) go to
+// scal_s[lane] for the other warps (load_query_scalars after a CTA barrier).
 template <int KM, int D>
-__device__ __forceinline__ void setup_query(const uint16_t *qrow, float smax_k, uint4 *aq_s, BodyCtx &c,
-                                            int warp) {
+__device__ __forceinline__ void setup_query(const uint16_t *qrow, float smax_k, uint4 *aq_s, float4 *scal_s,
+                                            BodyCtx &c, int warp) {
     constexpr int KS = D / 16, NJ = D / 32;
+    if (warp != 0) return;
     const int t = c.t;
     float qv[KS][4];
 #pragma unroll
@@ -279,10 +284,16 @@ __device__ __forceinline__ void setup_query(const uint16_t *qrow, float smax_k, 
         }
         c.unscale = qscale;
     }
-    if (warp == 0) {
 #pragma unroll
-        for (int k = 0; k < KS; ++k) aq_s[k * 32 + c.lane] = make_uint4(aq[k][0], aq[k][1], aq[k][2], aq[k][3]);
-    }
+    for (int k = 0; k < KS; ++k) aq_s[k * 32 + c.lane] = make_uint4(aq[k][0], aq[k][1], aq[k][2], aq[k][3]);
+    scal_s[c.lane] = make_float4(c.unscale, c.qsum_g, c.qsum_g8, 0.f);
+}
+
+__device__ __forceinline__ void load_query_scalars(BodyCtx &c, const float4 *scal_s) {
+    const float4 v = scal_s[c.lane];
+    c.unscale = v.x;
+    c.qsum_g = v.y;
+    c.qsum_g8 = v.z;
 }
 
 // Thread constants that depend only on the lane, the group size and the layer scales.
@@ -593,14 +604,15 @@ __device__ __forceinline__ void pipe_init(WarpPipe &P) {
     P.ist = 0;
 }
 
-// Issue the copy of the next unit (bytes from src) into the next free stage; stages
-// are refilled in the order they are consumed, so the next free stage is P.ist.
-__device__ __forceinline__ void pipe_issue(WarpPipe &P, const void *src, unsigned bytes) {
+// Issue the copy of the next unit (bytes from src, landing `skip` bytes into the stage)
+// into the next free stage; stages are refilled in the order they are consumed, so the
+// next free stage is P.ist.
+__device__ __forceinline__ void pipe_issue(WarpPipe &P, const void *src, unsigned bytes, unsigned skip = 0) {
     const int s = P.ist;
     if (P.lane == 0) {
         fence_proxy_async();
         mbar_expect_tx(&P.bars[s], bytes);
-        bulk_g2s(P.stages + static_cast<size_t>(s) * P.stage_bytes, src, bytes, &P.bars[s]);
+        bulk_g2s(P.stages + static_cast<size_t>(s) * P.stage_bytes + skip, src, bytes, &P.bars[s]);
     }
     ++P.issued;
     if (++P.ist == P.NS) P.ist = 0;
@@ -630,17 +642,31 @@ template <int D, int NT>
 __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &c, bool has_data, uint8_t *smem,
                                               int warp, long long row0, int sp, int S, int out_fp32, void *out,
                                               float *part_acc, float *part_ml) {
-    constexpr int KS = D / 16, NJ = D / 32;
+    constexpr int KS = D / 16;
     const int g = c.g, t = c.t, G = c.G;
     float l_run = A.l_run;
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    // fold the value zero-point term of channel group j (held by lane 4j + t) into the
+    // O^T columns of the channels of that group
+#pragma unroll
+    for (int m = 0; m < KS; ++m)
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const float z0 = __shfl_sync(0xffffffffu, A.zc[n][0], 4 * (m >> 1) + t);
+            const float z1 = __shfl_sync(0xffffffffu, A.zc[n][1], 4 * (m >> 1) + t);
+            A.oacc[m][n][0] += z0;
+            A.oacc[m][n][2] += z0;
+            A.oacc[m][n][1] += z1;
+            A.oacc[m][n][3] += z1;
+        }
     __syncthreads();   // every warp is done with its stages
     constexpr int CF = comb_floats(D, NT);
+    float *base = reinterpret_cast<float *>(smem);
+    float *shared_tail = base + NW * CF;   // wts[NW][8], den[8], M[8]
     {
-        float *ob = reinterpret_cast<float *>(smem) + warp * CF;   // [8*NT][D]
-        float *zb = ob + 8 * NT * D;                                // [8*NT][NJ]
-        float *ml = zb + 8 * NT * NJ;                               // m[8], l[8]
+        float *ob = base + warp * CF;      // [8*NT][D]
+        float *ml = ob + 8 * NT * D;       // m[8], l[8]
 #pragma unroll
         for (int m = 0; m < KS; ++m)
 #pragma unroll
@@ -651,41 +677,39 @@ __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &
                 ob[c0 * D + d0 + 8] = A.oacc[m][n][2];
                 ob[(c0 + 1) * D + d0 + 8] = A.oacc[m][n][3];
             }
-        if (g < NJ) {
-#pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                zb[(8 * n + 2 * t) * NJ + g] = A.zc[n][0];
-                zb[(8 * n + 2 * t + 1) * NJ + g] = A.zc[n][1];
-            }
-        }
         if (t == 0 && g < G) {
             ml[g] = has_data ? A.m_run : -INFINITY;
             ml[8 + g] = l_run;
         }
     }
     __syncthreads();
-    const float *base = reinterpret_cast<const float *>(smem);
+    if (threadIdx.x < G) {   // per-head merge weights of the warps
+        const int hd = threadIdx.x;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, base[w * CF + 8 * NT * D + hd]);
+        float den = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float mw = base[w * CF + 8 * NT * D + hd];
+            const float wt = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+            shared_tail[w * 8 + hd] = wt;
+            den = fmaf(wt, base[w * CF + 8 * NT * D + 8 + hd], den);
+        }
+        shared_tail[NW * 8 + hd] = den;
+        shared_tail[NW * 8 + 8 + hd] = M;
+    }
+    __syncthreads();
     for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
         const int hd = idx / D, d = idx % D;
         const int chi = hd, clo = (NT == 1) ? hd + G : 8 + hd;
-        float M = -INFINITY;
+        float val = 0.f;
 #pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, base[w * CF + 8 * NT * D + 8 * NT * NJ + hd]);
-        float val = 0.f, den = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-                const float *ob = base + w * CF;
-                const float *zb = ob + 8 * NT * D;
-                const float *ml = zb + 8 * NT * NJ;
-                const float mw = ml[hd];
-                if (mw == -INFINITY) continue;
-                const float wt = fast_exp2(mw - M);
-                const float o = (ob[chi * D + d] + ob[clo * D + d]) + (zb[chi * NJ + d / 32] + zb[clo * NJ + d / 32]);
-                val = fmaf(wt, o, val);
-                den = fmaf(wt, ml[8 + hd], den);
-            }
+        for (int w = 0; w < NW; ++w) {
+            const float *ob = base + w * CF;
+            val = fmaf(shared_tail[w * 8 + hd], ob[chi * D + d] + ob[clo * D + d], val);
         }
+        const float den = shared_tail[NW * 8 + hd];
         const long long row = row0 + hd;
         if (S == 1) {
             const float o = val / den;
@@ -694,7 +718,7 @@ __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &
         } else {
             part_acc[(row * kMaxSplits + sp) * D + d] = val;
             if (d == 0) {
-                part_ml[(row * kMaxSplits + sp) * 2] = M;
+                part_ml[(row * kMaxSplits + sp) * 2] = shared_tail[NW * 8 + 8 + hd];
                 part_ml[(row * kMaxSplits + sp) * 2 + 1] = den;
             }
         }
@@ -706,17 +730,18 @@ struct SmemParts {
     uint8_t *stages;
     uint64_t *bars;
     uint4 *aq_s;
+    float4 *scal_s;
 };
 
 __host__ __device__ inline size_t smem_bars_off(int NS, int stage_bytes, int D, int NT) {
     const size_t stage = static_cast<size_t>(NW) * NS * stage_bytes;
-    const size_t comb = static_cast<size_t>(NW) * comb_floats(D, NT) * 4;
+    const size_t comb = (static_cast<size_t>(NW) * comb_floats(D, NT) + kCombShared) * 4;
     return ((stage > comb ? stage : comb) + 127) & ~size_t(127);
 }
 
 __host__ __device__ inline size_t smem_total(int NS, int stage_bytes, int D, int NT) {
     const size_t bars = static_cast<size_t>(NW) * NS * 8 + 8 * ((NW * NS) & 1);   // keeps 16-B alignment
-    return smem_bars_off(NS, stage_bytes, D, NT) + bars + static_cast<size_t>(D / 16) * 32 * 16;
+    return smem_bars_off(NS, stage_bytes, D, NT) + bars + static_cast<size_t>(D / 16) * 32 * 16 + 32 * 16;
 }
 
 __device__ __forceinline__ SmemParts carve(uint8_t *smem, int NS, int stage_bytes, int D, int NT) {
@@ -725,6 +750,7 @@ __device__ __forceinline__ SmemParts carve(uint8_t *smem, int NS, int stage_byte
     const size_t bo = smem_bars_off(NS, stage_bytes, D, NT);
     s.bars = reinterpret_cast<uint64_t *>(smem + bo);
     s.aq_s = reinterpret_cast<uint4 *>(smem + bo + static_cast<size_t>(NW) * NS * 8 + 8 * ((NW * NS) & 1));
+    s.scal_s = reinterpret_cast<float4 *>(s.aq_s + (D / 16) * 32);
     return s;
 }
 
@@ -746,15 +772,26 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     pipe_init(P);
     const uint8_t *unit_rec = p.rec + (static_cast<long long>(b) * p.Hkv + h) * p.cap_blk * REC;
     const int nb = (blk1 - blk0 > warp) ? (blk1 - blk0 - warp + NW - 1) / NW : 0;
-    for (int k = 0; k < NS && k < nb; ++k) pipe_issue(P, unit_rec + static_cast<long long>(blk0 + warp + NW * k) * REC, REC);
+    // per-channel keys of the last, incomplete group come from the residual: fetch only
+    // the value part of that block's record
+    constexpr unsigned VSKIP = KM == 0 ? 2 * 2 * D * BK + 4 * D : 0;
+    auto issue_block = [&](int k) {
+        const int blk = blk0 + warp + NW * k;
+        const uint8_t *src = unit_rec + static_cast<long long>(blk) * REC;
+        if (blk == tail_blk) pipe_issue(P, src + VSKIP, REC - VSKIP, VSKIP);
+        else pipe_issue(P, src, REC);
+    };
+    for (int k = 0; k < NS && k < nb; ++k) issue_block(k);
 
     const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
     const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
     BodyCtx c = make_ctx<KM, D, NT>(lane, G, smax_v, sm.aq_s);
     c.res = p.res ? p.res + (static_cast<long long>(b) * p.Hkv + h) * 32 * D : nullptr;
     const int hh = c.g % G;
-    setup_query<KM, D>(p.q + (static_cast<long long>(b) * p.Hkv * G + h * G + hh) * D, smax_k, sm.aq_s, c, warp);
+    setup_query<KM, D>(p.q + (static_cast<long long>(b) * p.Hkv * G + h * G + hh) * D, smax_k, sm.aq_s, sm.scal_s,
+                       c, warp);
     __syncthreads();
+    load_query_scalars(c, sm.scal_s);
 
     WarpAcc<D, NT> A;
     acc_init(A);
@@ -769,7 +806,7 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
         }
         process_unit<BK, BV, KM, D, NT, 2, false>(A, pipe_front(P), 32, c);
         pipe_pop(P);
-        if (P.issued < nb) pipe_issue(P, unit_rec + static_cast<long long>(blk0 + warp + NW * P.issued) * REC, REC);
+        if (P.issued < nb) issue_block(P.issued);
     }
     if (!failed && has_tail) {
         if (!pipe_wait(P)) {
@@ -846,13 +883,14 @@ __global__ void __launch_bounds__(NW * 32, 4) decode_paged_kernel(const PagedDec
     if (int2) {
         c = make_ctx<0, D, NT>(lane, G, smax_v, sm.aq_s);
         c.res = nullptr;
-        setup_query<0, D>(p.q + qoff, smax_k, sm.aq_s, c, warp);
+        setup_query<0, D>(p.q + qoff, smax_k, sm.aq_s, sm.scal_s, c, warp);
     } else {
         c = make_ctx<1, D, NT>(lane, G, smax_v, sm.aq_s);
         c.res = nullptr;
-        setup_query<1, D>(p.q + qoff, smax_k, sm.aq_s, c, warp);
+        setup_query<1, D>(p.q + qoff, smax_k, sm.aq_s, sm.scal_s, c, warp);
     }
     __syncthreads();
+    load_query_scalars(c, sm.scal_s);
 
     bool failed = false;
     int i = 0;
