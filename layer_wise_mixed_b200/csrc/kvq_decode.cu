@@ -991,8 +991,8 @@ size_t decode_smem_bytes(long long rec_bytes, int nstage, int D, int G) {
 struct KernelState {
     const void *fn = nullptr;
     size_t smem_set = 0;
-    size_t occ_smem = 0;
-    int occ = 0;
+    size_t occ_smem[8] = {};   // occupancy per dynamic shared-memory size (stage counts)
+    int occ[8] = {};
 };
 static std::mutex g_state_mu;
 static KernelState g_state[64];
@@ -1014,12 +1014,19 @@ static cudaError_t prepare_kernel(const void *fn, size_t smem, int *occ_out) {
         ks->smem_set = smem;
     }
     if (occ_out) {
-        if (ks->occ_smem != smem) {
-            cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ks->occ, fn, NW * 32, smem);
+        int slot = -1;
+        for (int i = 0; i < 8; ++i)
+            if (ks->occ_smem[i] == smem || ks->occ_smem[i] == 0) {
+                slot = i;
+                break;
+            }
+        if (slot < 0) slot = static_cast<int>(smem % 8);   // full: replace an entry
+        if (ks->occ_smem[slot] != smem) {
+            cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ks->occ[slot], fn, NW * 32, smem);
             if (e != cudaSuccess) return e;
-            ks->occ_smem = smem;
+            ks->occ_smem[slot] = smem;
         }
-        *occ_out = ks->occ;
+        *occ_out = ks->occ[slot];
     }
     return cudaSuccess;
 }

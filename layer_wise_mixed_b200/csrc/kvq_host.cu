@@ -94,24 +94,17 @@ int cuda_fail(cudaError_t e, const char *what) {
     return fail(KVQ_ECUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-// Sequence splits for decode: minimise (waves) x (blocks per warp + per-CTA overhead).
-int choose_splits(const kvq_handle *h, int units, int nblk, int slots) {
-    const int smax = std::min(kvq::kMaxSplits, nblk);
-    if (h->forced_splits > 0) return std::min(h->forced_splits, smax);
-    int best = 1;
-    double best_t = 1e300;
-    for (int s = 1; s <= smax; ++s) {
-        const int bps = (nblk + s - 1) / s;
-        const int sreal = (nblk + bps - 1) / bps;
-        const double waves = std::ceil(static_cast<double>(units) * sreal / std::max(1, slots));
-        const double per_cta = std::ceil(static_cast<double>(bps) / kvq::kDecodeWarps) + 1.0;
-        const double tcost = waves * per_cta * (1.0 + 0.002 * sreal);
-        if (tcost < best_t - 1e-9) {
-            best_t = tcost;
-            best = sreal;
-        }
-    }
-    return best;
+// Estimated time of a per-layer decode launch, in units of one block's processing by a
+// warp: waves x (blocks per warp + a per-CTA overhead of about one block); with a single
+// stage per warp the copy latency of every block after the first is exposed (about 0.6
+// of a block each).
+double decode_cost(int units, int nblk, int S, int nstage, int slots) {
+    const int bps = (nblk + S - 1) / S;
+    const int sreal = (nblk + bps - 1) / bps;
+    const double waves = std::ceil(static_cast<double>(units) * sreal / std::max(1, slots));
+    const double bpw = std::ceil(static_cast<double>(bps) / kvq::kDecodeWarps);
+    const double per_cta = bpw + 1.0 + (nstage == 1 ? 0.6 * (bpw - 1.0) : 0.0);
+    return waves * per_cta * (1.0 + 0.002 * sreal);
 }
 
 }  // namespace
@@ -440,20 +433,50 @@ static int ensure_device_info(kvq_handle *h) {
     return KVQ_OK;
 }
 
+// Split count and stages per warp of a per-layer decode launch: every split count and
+// every stage count from 1 to the most that fit is costed with the occupancy it allows
+// (deep rings fit fewer CTAs per SM; short sequences gain more from one wave than from
+// prefetch depth).
 static int splits_for(kvq_handle *h, int layer, int *S_out, int *nstage_out) {
     const LayerGeom &g = h->geom[layer];
     const int L = h->len[layer];
     const int nblk = (L + 31) / 32;
     const int G = h->desc.n_q_heads / h->desc.n_kv_heads;
-    const int nstage = kvq::decode_stages(g.rec_bytes, h->desc.head_dim, G);
+    const int ns_max = kvq::decode_stages(g.rec_bytes, h->desc.head_dim, G);
     int rc = ensure_device_info(h);
     if (rc) return rc;
-    int per_sm = 1;
-    cudaError_t e = kvq::decode_occupancy(h->desc.head_dim, g.bk, g.bv, g.kmode, G, g.rec_bytes, nstage, &per_sm);
-    if (e != cudaSuccess) return cuda_fail(e, "decode occupancy");
     const int units = h->desc.batch * h->desc.n_kv_heads;
-    *S_out = choose_splits(h, units, nblk, std::max(1, per_sm) * h->sm_count);
-    *nstage_out = nstage;
+    const int smax = std::min(kvq::kMaxSplits, nblk);
+    double best = 1e300;
+    *S_out = 1;
+    *nstage_out = ns_max;
+    for (int ns = 1; ns <= ns_max; ++ns) {
+        int per_sm = 1;
+        cudaError_t e = kvq::decode_occupancy(h->desc.head_dim, g.bk, g.bv, g.kmode, G, g.rec_bytes, ns, &per_sm);
+        if (e != cudaSuccess) return cuda_fail(e, "decode occupancy");
+        const int slots = std::max(1, per_sm) * h->sm_count;
+        if (h->forced_splits > 0) {
+            const int S = std::min(h->forced_splits, smax);
+            const double c = decode_cost(units, nblk, S, ns, slots);
+            if (c < best - 1e-9) {
+                best = c;
+                *S_out = S;
+                *nstage_out = ns;
+            }
+            continue;
+        }
+        for (int S = 1; S <= smax; ++S) {
+            const int bps = (nblk + S - 1) / S;
+            const int sreal = (nblk + bps - 1) / bps;
+            if (sreal != S) continue;
+            const double c = decode_cost(units, nblk, S, ns, slots);
+            if (c < best - 1e-9) {
+                best = c;
+                *S_out = S;
+                *nstage_out = ns;
+            }
+        }
+    }
     return KVQ_OK;
 }
 

@@ -119,6 +119,15 @@ def test_gqa_groups(G, kmode):
     run_case(2, 2, G, 128, [(8, 4)], kmode, [150, 30, 20], decode_at=[150, 200], splits=(0, 3), tag=f"G{G}")
 
 
+@pytest.mark.parametrize("kmode", [0, 1])
+def test_many_short_units(kmode):
+    """Many (batch, kv head) units with few blocks each (64 units; 3, 4 and 5 blocks per
+    unit at L = 65, 97, 129, with residual tails of 1 token), automatic splits; every
+    decode is done twice (fp32, bf16) on the same cache."""
+    run_case(16, 4, 2, 64, [(4, 2)], kmode, [65, 32, 32], decode_at=[65, 97, 129], splits=(0,),
+             tag=f"spans{kmode}")
+
+
 def test_chunked_equals_bulk():
     """Incremental appends (ragged chunks) give the same bytes as the oracle's image of
     the whole sequence, which is also what one bulk append gives."""
