@@ -92,6 +92,12 @@ __device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32
     asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(orv));
     return d;
 }
+// (a & m) | (b & ~m) in one LOP3
+__device__ __forceinline__ uint32_t lop_sel(uint32_t a, uint32_t b, uint32_t m) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(d) : "r"(a), "r"(b), "r"(m));
+    return d;
+}
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t d;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
@@ -203,7 +209,7 @@ struct BodyCtx {
     const uint16_t *res;        // bf16 residual keys of this (b, h) (per-channel tail) or null
     int lane, g, t, G, jg, jg8, jz, alpha_src0, alpha_src1;
     bool row_g, row_g8;
-    uint32_t m_hi, m_lo;
+    uint32_t m_hi;
     float unscale, qsum_g, qsum_g8, pbias;
 };
 
@@ -311,10 +317,9 @@ __device__ __forceinline__ BodyCtx make_ctx(int lane, int G, float smax_v, const
     c.row_g = (KM == 1) && (c.g < G * NJ);
     c.row_g8 = (KM == 1) && (c.g + 8 < G * NJ);
     c.jz = c.g < NJ ? c.g : NJ - 1;
-    // B-operand column of this thread for P: NT == 1: hi (g < G), lo (G <= g < 2G) or
-    // zero; NT == 2: tile 0 hi, tile 1 lo for g < G.
+    // B-operand column of this thread for P: NT == 1: hi (g < G), else lo (columns 2G..
+    // are computed but never read); NT == 2: tile 0 hi, tile 1 lo.
     c.m_hi = (c.g < G) ? 0xFFFFFFFFu : 0u;
-    c.m_lo = (NT == 1 && c.g >= G && c.g < 2 * G) ? 0xFFFFFFFFu : 0u;
     c.alpha_src0 = 4 * ((NT == 1) ? ((2 * c.t) % G) : min(2 * c.t, 7));
     c.alpha_src1 = 4 * ((NT == 1) ? ((2 * c.t + 1) % G) : min(2 * c.t + 1, 7));
     // values: p * 2^kp * s_v stays below 2^14 in fp16
@@ -540,13 +545,14 @@ __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R
             zB &= mB;
         }
         // zero-point term: rows j = g of Z^T (tokens as columns) times the P columns
+        // (rows g >= NJ load group NJ - 1 and are never read)
         {
-            const uint32_t az[4] = {g < NJ ? zA : 0u, 0u, g < NJ ? zB : 0u, 0u};
+            const uint32_t az[4] = {zA, 0u, zB, 0u};
             if constexpr (NT == 1) {
-                mma16816(A.zc[0], az, (pah & c.m_hi) | (pal & c.m_lo), (pbh & c.m_hi) | (pbl & c.m_lo));
+                mma16816(A.zc[0], az, lop_sel(pah, pal, c.m_hi), lop_sel(pbh, pbl, c.m_hi));
             } else {
-                mma16816(A.zc[0], az, pah & c.m_hi, pbh & c.m_hi);
-                mma16816(A.zc[1], az, pal & c.m_hi, pbl & c.m_hi);
+                mma16816(A.zc[0], az, pah, pbh);
+                mma16816(A.zc[1], az, pal, pbl);
             }
         }
 #pragma unroll
@@ -556,13 +562,13 @@ __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R
             mul_hilo(pbh, pbl, sB[j], bh, bl);
             uint32_t b0, b1, c0 = 0u, c1 = 0u;
             if constexpr (NT == 1) {
-                b0 = (ah & c.m_hi) | (al & c.m_lo);
-                b1 = (bh & c.m_hi) | (bl & c.m_lo);
+                b0 = lop_sel(ah, al, c.m_hi);
+                b1 = lop_sel(bh, bl, c.m_hi);
             } else {
-                b0 = ah & c.m_hi;
-                b1 = bh & c.m_hi;
-                c0 = al & c.m_hi;
-                c1 = bl & c.m_hi;
+                b0 = ah;
+                b1 = bh;
+                c0 = al;
+                c1 = bl;
             }
 #pragma unroll
             for (int mm = 0; mm < 2; ++mm) {
