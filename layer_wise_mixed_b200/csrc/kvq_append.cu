@@ -161,6 +161,7 @@ __device__ void per_channel_group(const AppendParams &p, int unit, int q, bool d
 // largest scale of the layer is kept with integer atomicMax (one per CTA), for the
 // decoder's choice of fp16 operand prescales.
 __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams p) {
+    pdl_enter();
     __shared__ __align__(16) float xs[32][kMaxD];
     __shared__ __align__(16) uint8_t codes[32][kMaxD];
     __shared__ unsigned cta_smax;
@@ -194,8 +195,8 @@ cudaError_t launch_append(const AppendParams &p, cudaStream_t st) {
     if (p.D > kMaxD) return cudaErrorInvalidValue;
     const int grid = p.nV + p.nK;
     if (grid <= 0) return cudaSuccess;
-    append_kernel<<<grid, kThreads, 0, st>>>(p);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(append_kernel, dim3(grid), dim3(kThreads), 0, st, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace kvq

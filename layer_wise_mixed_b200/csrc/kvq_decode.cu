@@ -763,6 +763,7 @@ __device__ __forceinline__ SmemParts carve(uint8_t *smem, int NS, int stage_byte
 // ------------------------------------------------------------------ per-layer kernel
 template <int BK, int BV, int KM, int D, int NT>
 __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(const DecodeParams p) {
+    pdl_enter();
     constexpr int REC = unit_bytes(D, BK, BV, KM, 2);
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -836,6 +837,7 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
 // 4-bit keys and values per token): main pages, then the pending pages of INT2 tokens
 // whose group is still open.  Every split is bitwidth-homogeneous.
 __global__ void __launch_bounds__(NW * 32, 4) decode_paged_kernel(const PagedDecodeParams p) {
+    pdl_enter();
     constexpr int D = 128, NT = 1;
     constexpr int REC2 = unit_bytes(D, 2, 2, 0, 2), PAGE4 = unit_bytes(D, 4, 4, 1, 1);
     constexpr int STAGE = REC2 > PAGE4 ? REC2 : PAGE4;
@@ -926,6 +928,7 @@ __global__ void __launch_bounds__(NW * 32, 4) decode_paged_kernel(const PagedDec
 
 // Log-sum-exp merge of the split partials ("merged by online log-sum-exp").
 __global__ void merge_kernel(const MergeParams p) {
+    pdl_enter();
     const long long row = blockIdx.x;   // b * Hq + hq
     const float *ml = p.part_ml + row * kMaxSplits * 2;
     float M = -INFINITY;
@@ -1052,8 +1055,8 @@ cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmod
     cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(fn), smem, ctas_per_sm_out);
     if (e != cudaSuccess) return e;
     dim3 grid(p.S, p.Hkv, p.B);
-    fn<<<grid, NW * 32, smem, st>>>(p);
-    return cudaGetLastError();
+    e = launch_pdl(fn, grid, dim3(NW * 32), smem, st, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 int paged_rec2_bytes(int D) { return unit_bytes(D, 2, 2, 0, 2); }
@@ -1078,13 +1081,13 @@ cudaError_t launch_decode_paged(const PagedDecodeParams &p, cudaStream_t st) {
     cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(decode_paged_kernel), smem, nullptr);
     if (e != cudaSuccess) return e;
     dim3 grid(p.S2 + p.S4, p.Hkv, p.B);
-    decode_paged_kernel<<<grid, NW * 32, smem, st>>>(p);
-    return cudaGetLastError();
+    e = launch_pdl(decode_paged_kernel, grid, dim3(NW * 32), smem, st, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t st) {
-    merge_kernel<<<p.B * p.Hq, p.D, 0, st>>>(p);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(merge_kernel, dim3(p.B * p.Hq), dim3(p.D), 0, st, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace kvq

@@ -5,6 +5,35 @@
 
 namespace kvq {
 
+// Programmatic dependent launch.  Every kernel of this library is launched with
+// launch_pdl: it may be scheduled while the previous kernel of the stream is still
+// running, and calls pdl_enter() first, which lets the next kernel's CTAs launch early
+// and then waits until the previous kernel has completed and its memory is visible
+// (griddepcontrol.wait) -- before any global-memory access, so stream order semantics
+// are unchanged and only launch latency and prologues overlap.
+#ifdef __CUDACC__
+__device__ __forceinline__ void pdl_enter() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+#endif
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 constexpr int kGroup = 32;          // quantization group (tokens or channels)
 constexpr int kMaxSplits = 64;      // partial slots per (batch, query head)
 constexpr int kDecodeWarps = 4;     // warps per decode CTA

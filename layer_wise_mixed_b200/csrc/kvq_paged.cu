@@ -162,6 +162,7 @@ __device__ void write_int2_group(uint8_t *rec, SrcFn src_row, float (*xs)[kD], u
 }
 
 __global__ void __launch_bounds__(kThreads) paged_append_kernel(const PagedAppendParams p) {
+    pdl_enter();
     __shared__ __align__(16) float xs[32][kD];
     __shared__ __align__(16) uint8_t kc[32][kD];
     __shared__ __align__(16) uint8_t vc[32][kD];
@@ -259,6 +260,7 @@ __global__ void __launch_bounds__(kThreads) paged_append_kernel(const PagedAppen
 // Per request: input index of the r-th INT2-tagged and r-th INT4-tagged new token.
 __global__ void __launch_bounds__(1024) paged_scan_kernel(const uint8_t *tags, int n, int *inv2, int *inv4,
                                                           int stride) {
+    pdl_enter();
     __shared__ int part2[1024];
     const int b = blockIdx.x;
     const uint8_t *tg = tags + static_cast<long long>(b) * n;
@@ -289,13 +291,15 @@ __global__ void __launch_bounds__(1024) paged_scan_kernel(const uint8_t *tags, i
 
 cudaError_t launch_paged_scan(const uint8_t *tags, int B, int n, int *inv2, int *inv4, int inv_stride,
                               cudaStream_t st) {
-    paged_scan_kernel<<<B, 1024, 0, st>>>(tags, n, inv2, inv4, inv_stride);
+    cudaError_t e = launch_pdl(paged_scan_kernel, dim3(B), dim3(1024), 0, st, tags, n, inv2, inv4, inv_stride);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 cudaError_t launch_paged_append(const PagedAppendParams &p, int grid, cudaStream_t st) {
     if (grid <= 0) return cudaSuccess;
-    paged_append_kernel<<<grid, kThreads, 0, st>>>(p);
+    cudaError_t e = launch_pdl(paged_append_kernel, dim3(grid), dim3(kThreads), 0, st, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
