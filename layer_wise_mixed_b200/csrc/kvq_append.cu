@@ -50,12 +50,24 @@ __device__ void per_token_half(const AppendParams &p, int role, int unit, int hb
     uint32_t *area = reinterpret_cast<uint32_t *>(rec + (role ? p.kc + p.ks : 0) +
                                                   static_cast<long long>(eta) * 2 * D * bits);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int Wh = D * bits / 64, F = 32 / bits, nw = D * bits / 2;
 
-    for (int e = es + warp; e < ee; e += kWarps) {
+    // the half's words this thread rewrites, loaded up front (fields of tokens already in
+    // the half are kept); a half that starts with these tokens is rebuilt from zero
+    uint32_t old[kMaxD * 8 / 2 / kThreads];
+#pragma unroll
+    for (int r = 0; r < kMaxD * 8 / 2 / kThreads; ++r) {
+        const int widx = threadIdx.x + r * kThreads;
+        old[r] = (es > 0 && widx < nw) ? area[widx] : 0u;
+    }
+
+    // one warp per (new token, 32-channel group)
+    for (int it = warp; it < (ee - es) * nj; it += kWarps) {
+        const int e = es + it / nj, j = it % nj;
         const int tok = u0 + e;
         const uint16_t *row = src + static_cast<long long>(tok - p.L_old) * D;
         const int u = 16 * eta + e;
-        for (int j = 0; j < nj; ++j) {
+        {
             const float x = bf16_to_f32(row[32 * j + lane]);
             float mn = x, mx = x;
 #pragma unroll
@@ -77,19 +89,20 @@ __device__ void per_token_half(const AppendParams &p, int role, int unit, int hb
     }
     __syncthreads();
 
-    const int Wh = D * bits / 64, F = 32 / bits, nw = D * bits / 2;
     const uint32_t mask = (1u << bits) - 1u;
-    for (int widx = threadIdx.x; widx < nw; widx += kThreads) {
+#pragma unroll
+    for (int r = 0; r < kMaxD * 8 / 2 / kThreads; ++r) {
+        const int widx = threadIdx.x + r * kThreads;
+        if (widx >= nw) break;
         int ln, w;
         word_lane(widx, Wh, ln, w);
-        const uint32_t old = es > 0 ? area[widx] : 0u;
         uint32_t out = 0;
         for (int f = 0; f < F; ++f) {
             int e, d;
             field_owner(role, ln, w, f, bits, e, d);
             uint32_t c;
             if (e >= es && e < ee) c = codes[e][d];
-            else if (e < es) c = (old >> (f * bits)) & mask;
+            else if (e < es) c = (old[r] >> (f * bits)) & mask;
             else c = 0;
             out |= c << (f * bits);
         }
