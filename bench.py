@@ -1,13 +1,16 @@
 """Decode-step benchmark of the mixed-precision KV cache (one JSON line on stdout).
 
 A step = one decode token for every sequence of the batch through every layer: per
-layer, kvq_append of the new token's K/V (quantize + pack, group flush when a key group
-completes) then kvq_decode_attn (split kernel + log-sum-exp merge).  Each step of the
-decode schedule is captured once into a CUDA graph (untimed); the timed region replays
-K graphs.  Inputs are seeded synthetic tensors already resident in HBM; one step reads
+layer, the new token's K/V is quantized and packed into the cache and decode attention
+runs over it -- kvq_append_decode, one launch (a token that completes a per-channel key
+group: kvq_append, then kvq_decode_attn; paged plans: kvq_append_tagged, then
+kvq_decode_attn), plus the log-sum-exp merge when the sequence is split.  Each step of
+the decode schedule is captured once into a CUDA graph (untimed); the timed region
+replays K graphs.  The dominant kernel's roofline comes from decode-only replays of the
+same schedule.  Inputs are seeded synthetic tensors already resident in HBM; one step reads
 every layer's cache once (larger than L2 for every workload here).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c2-k8v8|c3|c4]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c2-k8v8|c3|c4|c5]
     python bench.py --impl reference ...     # the CPU oracle on a bounded sample
 
 Under torchrun each rank runs its own replica of the workload (own seeds, no data-path
@@ -222,7 +225,7 @@ def workload_config(wl):
             "bits": ",".join(f"K{a}V{b}" for a, b in bits), "equivalent_bits": wl.equivalent_bits(),
             "keys": "per-channel" if wl.kmode == 0 else "per-token", "values": "per-token", "group": 32,
             "l2": "inputs larger than L2 (each step reads every layer's cache once)",
-            "launch": "one CUDA graph per decode step (append + decode for all layers)"}
+            "launch": "one CUDA graph per decode step (fused append + decode launch per layer)"}
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -325,8 +328,11 @@ def main():
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for l in range(NL):
-                append_step(l, s, Kn[s, l], Vn[s, l])
-                kvq.kvq_decode_attn(cache.h, l, Qn[s, l], out[l], False, stream)
+                if paged:
+                    append_step(l, s, Kn[s, l], Vn[s, l])
+                    kvq.kvq_decode_attn(cache.h, l, Qn[s, l], out[l], False, stream)
+                else:
+                    kvq.kvq_append_decode(cache.h, l, Kn[s, l], Vn[s, l], Qn[s, l], out[l], False, stream)
         graphs.append(g)
         splits.append([kvq.kvq_get_num_splits(cache.h, l) for l in range(NL)])
         Ls.append(cache.seq_len(0))
@@ -391,8 +397,14 @@ def main():
                         for s in order for l in range(NL))
     peak, peak_src = measured_hbm_peak()
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
-    gpu_launches = sum(2 + (1 if splits[s][l] > 1 else 0) for s in order for l in range(NL))
-    e2e_note = ("per step: pinned H2D of all layers' K/V/q, kvq_append + kvq_decode_attn per layer (eager "
+    # per layer and step: one fused append + decode launch, or (a token that completes a
+    # per-channel key group; paged plans) an append and a decode launch; plus the merge
+    # launch when the sequence is split
+    def step_launches(s, l):
+        two = paged or (wl.kmode == 0 and Ls[s] % 32 == 0)
+        return (2 if two else 1) + (1 if splits[s][l] > 1 else 0)
+    gpu_launches = sum(step_launches(s, l) for s in order for l in range(NL))
+    e2e_note = ("per step: pinned H2D of all layers' K/V/q, kvq_append_decode per layer (eager "
                 "C-ABI calls), D2H of all layers' outputs")
     if paged:
         e2e_note = ("per step: pinned H2D of all layers' K/V/q and kvq_decode_attn per layer (eager C-ABI calls; "
@@ -421,8 +433,7 @@ def main():
                 continue
             if cache.seq_len(l) >= wl.max_ctx:
                 kvq.kvq_truncate(cache.h, l, wl.prefill)
-            kvq.kvq_append(cache.h, l, dK[l], dV[l], 1, stream)
-            kvq.kvq_decode_attn(cache.h, l, dQ[l], out[l], False, stream)
+            kvq.kvq_append_decode(cache.h, l, dK[l], dV[l], dQ[l], out[l], False, stream)
         hO.copy_(out, non_blocking=True)
 
     with torch.cuda.stream(stream):

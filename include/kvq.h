@@ -149,6 +149,17 @@ KVQ_API int kvq_append_tagged(kvq_handle *h, int layer, const void *K, const voi
 KVQ_API int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_fp32,
                     void *stream);
 
+/* One decode step in one launch: append one token (K, V bf16 [B][Hkv][1][D], device)
+ * to `layer` and then run kvq_decode_attn with q over all L + 1 tokens; same results
+ * and errors as kvq_append(..., n_new = 1, ...) followed by kvq_decode_attn.  The CTA
+ * that decodes a sequence's last block first quantizes and packs the new token into it
+ * (the pages apply quantize-and-pack and decode attention per step; fusing them is this
+ * library's choice).  A token that completes a 32-token per-channel key group takes the
+ * two-launch path, since the whole group is quantized then.  Per-layer plans only
+ * (paged plans: KVQ_EINVAL). */
+KVQ_API int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, const void *q,
+                              void *out, int out_fp32, void *stream);
+
 /* Force the number of sequence splits used by kvq_decode_attn (0 = automatic; the
  * value is capped by the number of 32-token blocks and the partial buffer size). */
 KVQ_API int kvq_set_num_splits(kvq_handle *h, int num_splits);

@@ -200,6 +200,11 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams p) {
     }
     __syncthreads();
     if (threadIdx.x == 0 && cta_smax) atomicMax(p.smax + role, cta_smax);
+    // carry the maxima of the old length into the new length's slot
+    if (cta == 0 && threadIdx.x == 0 && p.smax_prev != p.smax) {
+        atomicMax(p.smax, p.smax_prev[0]);
+        atomicMax(p.smax + 1, p.smax_prev[1]);
+    }
 }
 
 }  // namespace

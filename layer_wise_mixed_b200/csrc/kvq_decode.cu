@@ -32,6 +32,7 @@
 #include <type_traits>
 
 #include "kvq_internal.h"
+#include "kvq_quant.cuh"
 
 namespace kvq {
 namespace {
@@ -745,9 +746,14 @@ __host__ __device__ inline size_t smem_bars_off(int NS, int stage_bytes, int D, 
     return ((stage > comb ? stage : comb) + 127) & ~size_t(127);
 }
 
+// Bytes after the per-lane scalars: codes of a fused append's token (values, keys) and
+// the CTA's two scale maxima.
+__host__ __device__ constexpr int append_scratch_bytes(int D) { return 2 * D + 16; }
+
 __host__ __device__ inline size_t smem_total(int NS, int stage_bytes, int D, int NT) {
     const size_t bars = static_cast<size_t>(NW) * NS * 8 + 8 * ((NW * NS) & 1);   // keeps 16-B alignment
-    return smem_bars_off(NS, stage_bytes, D, NT) + bars + static_cast<size_t>(D / 16) * 32 * 16 + 32 * 16;
+    return smem_bars_off(NS, stage_bytes, D, NT) + bars + static_cast<size_t>(D / 16) * 32 * 16 + 32 * 16 +
+           append_scratch_bytes(D);
 }
 
 __device__ __forceinline__ SmemParts carve(uint8_t *smem, int NS, int stage_bytes, int D, int NT) {
@@ -758,6 +764,98 @@ __device__ __forceinline__ SmemParts carve(uint8_t *smem, int NS, int stage_byte
     s.aq_s = reinterpret_cast<uint4 *>(smem + bo + static_cast<size_t>(NW) * NS * 8 + 8 * ((NW * NS) & 1));
     s.scal_s = reinterpret_cast<float4 *>(s.aq_s + (D / 16) * 32);
     return s;
+}
+
+// ------------------------------------------------------------------ fused append
+// Bits of token e's codes inside word widx of a 16-token half's code area (role 0 key
+// operand, 1 value operand), from the token's codes code[d].
+template <int BITS>
+__device__ __forceinline__ uint32_t token_bits(int role, int widx, int e, const uint8_t *code, int D) {
+    constexpr int F = 32 / BITS;
+    int ln, w;
+    quant::word_lane(widx, D * BITS / 64, ln, w);
+    uint32_t out = 0;
+#pragma unroll
+    for (int f = 0; f < F; ++f) {
+        int ee, d;
+        quant::field_owner(role, ln, w, f, BITS, ee, d);
+        if (ee == e) out |= static_cast<uint32_t>(code[d]) << (f * BITS);
+    }
+    return out;
+}
+
+// Write one half's words for token e: the first token of a half rebuilds the half (its
+// words hold no other token yet, and stale bytes must read as zero); a later token ORs
+// its fields, which are zero until now.
+template <int BITS>
+__device__ __forceinline__ void pack_token(uint32_t *area, int role, int e, const uint8_t *code, int D) {
+    const int nw = D * BITS / 2;
+    for (int widx = threadIdx.x; widx < nw; widx += NW * 32) {
+        const uint32_t bits = token_bits<BITS>(role, widx, e, code, D);
+        if (e == 0) area[widx] = bits;
+        else if (bits) atomicOr(area + widx, bits);
+    }
+}
+
+// Quantize and pack the token appended by a fused launch, token u of block `blk` of unit
+// `unit`, with the same arithmetic as the append kernel: values per token
+// (one warp per 32-channel group), keys per token the same way or, per channel, the new
+// row into the residual (slot u: the host takes the two-launch path when the token
+// completes a key group).  All threads of the CTA take part; afterwards the writes are
+// visible to the bulk copy of the block, and own_k / own_v hold this CTA's largest new
+// scales.
+template <int BK, int BV, int KM, int D>
+__device__ __forceinline__ void append_token(const DecodeParams &p, long long unit, int blk, int u,
+                                             uint8_t *scratch, float &own_k, float &own_v) {
+    constexpr int NJ = D / 32;
+    constexpr int KC = 4 * D * BK, KSZ = 4 * D, VC = 4 * D * BV;
+    constexpr int REC = KC + KSZ + VC + 4 * D;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = u & 15, eta = u >> 4;
+    uint8_t *rec = p.rec_w + (unit * p.cap_blk + blk) * static_cast<long long>(REC);
+    uint8_t *codes = scratch;                                   // [0, D): values, [D, 2D): keys
+    unsigned *cmax = reinterpret_cast<unsigned *>(scratch + 2 * D);   // keys, values (fp16 bits)
+    if (threadIdx.x < 2) cmax[threadIdx.x] = 0u;
+    __syncthreads();
+    constexpr int NROLE = KM == 1 ? 2 : 1;
+    for (int it = warp; it < NROLE * NJ; it += NW) {
+        const int role = it < NJ ? 1 : 0;
+        const int j = it % NJ;
+        const int bits = role ? BV : BK;
+        const uint16_t *src = (role ? p.v_new : p.k_new) + unit * D;
+        const float x = quant::bf16_to_f32(src[32 * j + lane]);
+        float mn = x, mx = x;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        float sc, z;
+        uint16_t s16, z16;
+        quant::group_params(mn, mx, bits, sc, z, s16, z16);
+        codes[(role ? 0 : D) + 32 * j + lane] = static_cast<uint8_t>(quant::group_code(x, sc, z, bits));
+        if (lane == 0) {
+            uint8_t *sz = rec + (role ? KC + KSZ + VC : KC);
+            const int so = quant::tok_sz_off(u, j, NJ);
+            *reinterpret_cast<uint16_t *>(sz + so) = s16;
+            *reinterpret_cast<uint16_t *>(sz + so + 4 * NJ) = z16;
+            atomicMax(cmax + role, static_cast<unsigned>(s16));
+        }
+    }
+    if constexpr (KM == 0) {
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(p.k_new + unit * D);
+        uint32_t *dst = reinterpret_cast<uint32_t *>(p.res_w + (unit * 32 + u) * D);
+        for (int i = threadIdx.x; i < D / 2; i += NW * 32) dst[i] = src[i];
+    }
+    __syncthreads();
+    pack_token<BV>(reinterpret_cast<uint32_t *>(rec + KC + KSZ + eta * 2 * D * BV), 1, e, codes, D);
+    if constexpr (KM == 1) pack_token<BK>(reinterpret_cast<uint32_t *>(rec + eta * 2 * D * BK), 0, e, codes + D, D);
+    __threadfence();                                   // the new bytes are performed GPU-wide ...
+    asm volatile("fence.proxy.async;" ::: "memory");   // ... and ordered before async-proxy reads
+    __syncthreads();
+    own_k = __half2float(__ushort_as_half(static_cast<unsigned short>(cmax[0])));
+    own_v = __half2float(__ushort_as_half(static_cast<unsigned short>(cmax[1])));
+    if (threadIdx.x < 2 && cmax[threadIdx.x]) atomicMax(p.smax_out + threadIdx.x, cmax[threadIdx.x]);
 }
 
 // ------------------------------------------------------------------ per-layer kernel
@@ -788,10 +886,30 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
         if (blk == tail_blk) pipe_issue(P, src + VSKIP, REC - VSKIP, VSKIP);
         else pipe_issue(P, src, REC);
     };
-    for (int k = 0; k < NS && k < nb; ++k) issue_block(k);
+    // a fused launch first writes the new token, token L - 1 (the last of its block);
+    // that block is fetched after it
+    const bool fused = p.k_new != nullptr;
+    const int new_blk = (L - 1) >> 5;
+    const bool append_here = fused && new_blk >= blk0 && new_blk < blk1;   // CTA-uniform
+    for (int k = 0; k < NS && k < nb; ++k) {
+        if (append_here && blk0 + warp + NW * k == new_blk) break;
+        issue_block(k);
+    }
 
-    const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
-    const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
+    float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
+    float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
+    if (fused && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) {
+        atomicMax(p.smax_out, p.smax[0]);   // carry the old length's maxima forward
+        atomicMax(p.smax_out + 1, p.smax[1]);
+    }
+    if (append_here) {
+        float own_k, own_v;
+        append_token<BK, BV, KM, D>(p, static_cast<long long>(b) * p.Hkv + h, new_blk, (L - 1) & 31,
+                                    reinterpret_cast<uint8_t *>(sm.scal_s + 32), own_k, own_v);
+        smax_k = fmaxf(smax_k, own_k);
+        smax_v = fmaxf(smax_v, own_v);
+        while (P.issued < nb && P.issued < NS) issue_block(P.issued);
+    }
     BodyCtx c = make_ctx<KM, D, NT>(lane, G, smax_v, sm.aq_s);
     c.res = p.res ? p.res + (static_cast<long long>(b) * p.Hkv + h) * 32 * D : nullptr;
     const int hh = c.g % G;

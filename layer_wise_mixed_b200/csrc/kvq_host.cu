@@ -80,6 +80,15 @@ int check_bound(const kvq_handle *h) {
 
 int cuda_fail(cudaError_t e, const char *what);
 
+// Per-layer maxima of the fp16 scales {K, V}, kept in two slots by the parity of the
+// sequence length they describe: an operation that leaves a layer at length L writes slot
+// L & 1 (carrying the other slot forward), a decode at length L reads it.  A launch that
+// appends and decodes reads the slot of L - 1, which nothing writes during it.  Paged
+// plans use slot 0 only.
+unsigned *smax_slot(const kvq_handle *h, int layer, int parity) {
+    return reinterpret_cast<unsigned *>(h->ws + h->smax_off) + 4 * layer + 2 * (parity & 1);
+}
+
 // The status word and the per-layer maximum scales live in caller memory of unknown
 // content: zero them on the stream of the first launch after a bind.
 int prepare_status(kvq_handle *h, cudaStream_t st) {
@@ -155,7 +164,7 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
         h->n4_cap = h->n4_main_cap + 2LL * d->batch;
         h->P_cap = (d->max_ctx + 31) / 32 + (d->max_ctx + 15) / 16 + 1;
         h->inv_stride = d->max_ctx;
-        long long off = align256(256 + 8LL * d->num_layers);
+        long long off = align256(256 + 16LL * d->num_layers);
         h->meta_bytes = off;
         h->status_off = 0;
         h->smax_off = 256;
@@ -196,8 +205,8 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
     h->cap_blk = (d->max_ctx + 31) / 32;
     const int D = d->head_dim;
     h->status_off = 0;
-    h->smax_off = 256;                                      // after the status word
-    h->meta_bytes = align256(256 + 8LL * d->num_layers);   // {K, V} max scale per layer
+    h->smax_off = 256;                                       // after the status word
+    h->meta_bytes = align256(256 + 16LL * d->num_layers);   // {K, V} max scale per layer and parity
     long long off = h->meta_bytes;
     for (int l = 0; l < d->num_layers; ++l) {
         const kvq_layer_cfg &c = h->cfg[l];
@@ -291,7 +300,8 @@ int kvq_append(kvq_handle *h, int layer, const void *K, const void *V, int n_new
     kvq::AppendParams p{};
     p.K = static_cast<const uint16_t *>(K);
     p.V = static_cast<const uint16_t *>(V);
-    p.smax = reinterpret_cast<unsigned *>(h->ws + h->smax_off) + 2 * layer;
+    p.smax = smax_slot(h, layer, L_new);
+    p.smax_prev = smax_slot(h, layer, L_old);
     p.rec = h->ws + g.rec_off;
     p.res = g.res_off >= 0 ? reinterpret_cast<uint16_t *>(h->ws + g.res_off) : nullptr;
     p.B = h->desc.batch;
@@ -390,7 +400,7 @@ int kvq_append_tagged(kvq_handle *h, int layer, const void *K, const void *V, in
     a.P_cap = h->P_cap;
     a.pend_base = h->pend_base;
     a.staging = reinterpret_cast<uint16_t *>(h->ws + h->staging_off[layer]);
-    a.smax = reinterpret_cast<unsigned *>(h->ws + h->smax_off) + 2 * layer;
+    a.smax = smax_slot(h, layer, 0);
     a.B = B;
     a.Hkv = h->desc.n_kv_heads;
     a.D = D;
@@ -543,7 +553,7 @@ static int decode_paged(kvq_handle *h, int layer, const void *q, void *out, int 
     p.pend_base = h->pend_base;
     for (int b = 0; b < h->desc.batch; ++b) p.cnt[b] = kvq::PagedCounts{P.n2g[b], P.n4[b], P.np[b], 0};
     p.q = static_cast<const uint16_t *>(q);
-    p.smax = reinterpret_cast<const unsigned *>(h->ws + h->smax_off) + 2 * layer;
+    p.smax = smax_slot(h, layer, 0);
     p.out = out;
     p.part_acc = part_acc;
     p.part_ml = part_ml;
@@ -594,7 +604,7 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
     p.rec = h->ws + g.rec_off;
     p.res = g.res_off >= 0 ? reinterpret_cast<const uint16_t *>(h->ws + g.res_off) : nullptr;
     p.q = static_cast<const uint16_t *>(q);
-    p.smax = reinterpret_cast<const unsigned *>(h->ws + h->smax_off) + 2 * layer;
+    p.smax = smax_slot(h, layer, L);
     p.out = out;
     p.part_acc = reinterpret_cast<float *>(h->ws + h->part_acc_off);
     p.part_ml = reinterpret_cast<float *>(h->ws + h->part_ml_off);
@@ -613,6 +623,82 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
     if ((rc = prepare_status(h, st))) return rc;
     cudaError_t e = kvq::launch_decode(p, h->desc.head_dim, g.bk, g.bv, g.kmode, st, nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    if (p.S > 1) {
+        kvq::MergeParams m{};
+        m.part_acc = p.part_acc;
+        m.part_ml = p.part_ml;
+        m.out = out;
+        m.B = p.B;
+        m.Hq = h->desc.n_q_heads;
+        m.D = h->desc.head_dim;
+        m.S = p.S;
+        m.out_fp32 = p.out_fp32;
+        e = kvq::launch_merge(m, st);
+        if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+    }
+    return ok();
+}
+
+int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, const void *q, void *out,
+                      int out_fp32, void *stream) {
+    int rc = check_layer(h, layer);
+    if (rc) return rc;
+    if ((rc = check_bound(h))) return rc;
+    if (!K || !V || !q || !out) return fail(KVQ_EINVAL, "null K, V, q or out");
+    if (!aligned(K, 16) || !aligned(V, 16) || !aligned(q, 16) || !aligned(out, 16))
+        return fail(KVQ_EALIGN, "K, V, q and out must be 16-byte aligned");
+    if (h->desc.paged) return fail(KVQ_EINVAL, "paged plans append with kvq_append_tagged");
+    const int L_old = h->len[layer];
+    if (static_cast<long long>(L_old) + 1 > h->desc.max_ctx)
+        return fail(KVQ_ECAPACITY, "layer %d: %d + 1 tokens exceed max_ctx %d", layer, L_old, h->desc.max_ctx);
+    const LayerGeom &g = h->geom[layer];
+    const int L = L_old + 1;
+    if (g.kmode == KVQ_PER_CHANNEL && L % 32 == 0) {
+        // the token completes a key group: the group is quantized by the append kernel
+        if ((rc = kvq_append(h, layer, K, V, 1, stream))) return rc;
+        return kvq_decode_attn(h, layer, q, out, out_fp32, stream);
+    }
+    h->len[layer] = L;   // the schedule is chosen for the new length
+    int S = 1, nstage = 2;
+    if ((rc = splits_for(h, layer, &S, &nstage))) {
+        h->len[layer] = L_old;
+        return rc;
+    }
+    const int nblk = (L + 31) / 32;
+    kvq::DecodeParams p{};
+    p.rec = h->ws + g.rec_off;
+    p.res = g.res_off >= 0 ? reinterpret_cast<const uint16_t *>(h->ws + g.res_off) : nullptr;
+    p.q = static_cast<const uint16_t *>(q);
+    p.smax = smax_slot(h, layer, L_old);
+    p.out = out;
+    p.part_acc = reinterpret_cast<float *>(h->ws + h->part_acc_off);
+    p.part_ml = reinterpret_cast<float *>(h->ws + h->part_ml_off);
+    p.status = reinterpret_cast<unsigned *>(h->ws + h->status_off);
+    p.B = h->desc.batch;
+    p.Hkv = h->desc.n_kv_heads;
+    p.G = h->desc.n_q_heads / h->desc.n_kv_heads;
+    p.L = L;
+    p.cap_blk = h->cap_blk;
+    p.bps = (nblk + S - 1) / S;
+    p.S = (nblk + p.bps - 1) / p.bps;
+    p.out_fp32 = out_fp32 ? 1 : 0;
+    p.nstage = nstage;
+    p.rec_bytes = g.rec_bytes;
+    p.k_new = static_cast<const uint16_t *>(K);
+    p.v_new = static_cast<const uint16_t *>(V);
+    p.rec_w = h->ws + g.rec_off;
+    p.res_w = g.res_off >= 0 ? reinterpret_cast<uint16_t *>(h->ws + g.res_off) : nullptr;
+    p.smax_out = smax_slot(h, layer, L);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((rc = prepare_status(h, st))) {
+        h->len[layer] = L_old;
+        return rc;
+    }
+    cudaError_t e = kvq::launch_decode(p, h->desc.head_dim, g.bk, g.bv, g.kmode, st, nullptr);
+    if (e != cudaSuccess) {
+        h->len[layer] = L_old;
+        return cuda_fail(e, "fused append + decode launch");
+    }
     if (p.S > 1) {
         kvq::MergeParams m{};
         m.part_acc = p.part_acc;
@@ -890,7 +976,7 @@ int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, 
     p.rec = h->ws + g.rec_off;
     p.res = g.res_off >= 0 ? reinterpret_cast<const uint16_t *>(h->ws + g.res_off) : nullptr;
     p.q = static_cast<const uint16_t *>(q);
-    p.smax = reinterpret_cast<const unsigned *>(h->ws + h->smax_off) + 2 * layer;
+    p.smax = smax_slot(h, layer, L);
     p.out = out;
     p.part_acc = static_cast<float *>(scratch);
     p.part_ml = reinterpret_cast<float *>(static_cast<unsigned char *>(scratch) + acc_bytes);

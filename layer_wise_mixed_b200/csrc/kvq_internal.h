@@ -53,7 +53,8 @@ struct LayerGeom {
 
 struct AppendParams {
     const uint16_t *K, *V;      // bf16 [B][Hkv][n][D]
-    unsigned *smax;             // this layer's {max key scale, max value scale} (fp16 bits)
+    unsigned *smax;             // {max key scale, max value scale} (fp16 bits) at the new length
+    const unsigned *smax_prev;  // the same at the old length (other parity slot), or smax
     uint8_t *rec;               // layer records [B][Hkv][cap][rec_bytes]
     uint16_t *res;              // residual [B][Hkv][32][D] bf16 (per-channel keys)
     int B, Hkv, D, bk, bv, kmode;
@@ -75,6 +76,13 @@ struct DecodeParams {
     unsigned *status;
     int B, Hkv, G, L, cap_blk, S, bps, out_fp32, nstage;
     long long rec_bytes;
+    // Fused one-token append (kvq_append_decode), null otherwise: the new token's K and V
+    // rows (bf16 [B][Hkv][D]), now token L - 1; writable records and residual; the
+    // scale-maximum slot of length L (smax above is the slot of length L - 1).
+    const uint16_t *k_new, *v_new;
+    uint8_t *rec_w;
+    uint16_t *res_w;
+    unsigned *smax_out;
 };
 
 // ---------------------------------------------------------------- paged INT2/INT4

@@ -69,6 +69,7 @@ def load() -> ctypes.CDLL:
         "kvq_append": (I, [P, I, P, P, I, P]),
         "kvq_append_tagged": (I, [P, I, P, P, I, P, P, P]),
         "kvq_decode_attn": (I, [P, I, P, P, I, P]),
+        "kvq_append_decode": (I, [P, I, P, P, P, P, I, P]),
         "kvq_decode_attn_noalloc": (I, [P, I, P, P, I, P]),
         "kvq_set_num_splits": (I, [P, I]),
         "kvq_get_num_splits": (I, [P, I, ctypes.POINTER(I)]),
@@ -142,6 +143,11 @@ def kvq_append_tagged(h: int, layer: int, K, V, n_new: int, host_tags, dev_tags,
 
 def kvq_decode_attn(h: int, layer: int, q, out, out_fp32: bool, stream=None):
     _check(load().kvq_decode_attn(h, layer, _ptr(q), _ptr(out), int(bool(out_fp32)), _stream(stream)))
+
+
+def kvq_append_decode(h: int, layer: int, K, V, q, out, out_fp32: bool, stream=None):
+    _check(load().kvq_append_decode(h, layer, _ptr(K), _ptr(V), _ptr(q), _ptr(out), int(bool(out_fp32)),
+                                    _stream(stream)))
 
 
 def kvq_decode_attn_noalloc(h: int, layer: int, q, out, out_fp32: bool, stream=None):
@@ -242,6 +248,16 @@ class Cache:
             out = torch.empty((self.B, self.Hq, self.D), dtype=torch.float32 if out_fp32 else torch.bfloat16,
                               device=q.device)
         kvq_decode_attn(self.h, layer, q, out, out_fp32, stream)
+        return out
+
+    def append_decode(self, layer, K, V, q, out=None, out_fp32=False, stream=None):
+        """One decode step: append the token K, V [B, Hkv, 1, D] and attend with q."""
+        import torch
+        assert K.is_contiguous() and V.is_contiguous() and K.shape == V.shape and K.shape[2] == 1
+        if out is None:
+            out = torch.empty((self.B, self.Hq, self.D), dtype=torch.float32 if out_fp32 else torch.bfloat16,
+                              device=q.device)
+        kvq_append_decode(self.h, layer, K, V, q, out, out_fp32, stream)
         return out
 
     def export_layer(self, layer):

@@ -1,0 +1,99 @@
+"""GPU parity of kvq_append_decode (one-token append and decode attention in one launch)
+against the CPU oracle.
+
+Every step appends one token through the fused entry point; at the checked lengths the
+exported cache image must equal the oracle's image of the same token sequence byte for
+byte, and the step's fp32 output (and a bf16 decode at the same length) must meet the
+T1/T2 tolerances of the parity tests.  Steps that complete a 32-token per-channel key
+group take the two-launch path inside the call and are covered too.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from layer_wise_mixed_b200 import configs, inputs, kvq
+
+from test_gpu_parity import bits16, check_outputs, workload
+
+pytestmark = pytest.mark.gpu
+
+
+def run_fused(B, Hkv, G, D, bits, kmode, prefill, steps, check_at, splits=0, wl=None, tag="fused"):
+    bk, bv = bits
+    L_total = prefill + steps
+    wl = wl or workload(B, Hkv, G, D, name=tag)
+    cache = kvq.Cache(1, B, Hkv, Hkv * G, D, L_total, [bits], kmodes=[kmode])
+    kvq.kvq_set_num_splits(cache.h, splits)
+    K, V = inputs.layer_kv(wl, 0, L_total, "cuda")
+    Kb, Vb = bits16(K), bits16(V)
+    if prefill:
+        cache.append(0, K[:, :, :prefill].contiguous(), V[:, :, :prefill].contiguous())
+    check_at = set(check_at)
+    for L in range(prefill + 1, L_total + 1):
+        q = inputs.step_q(wl, 0, L, "cuda")
+        out32 = cache.append_decode(0, K[:, :, L - 1:L].contiguous(), V[:, :, L - 1:L].contiguous(), q,
+                                    out_fp32=True)
+        assert cache.seq_len(0) == L
+        if L not in check_at:
+            continue
+        out16 = cache.decode_attn(0, q, out_fp32=False)
+        torch.cuda.synchronize()
+        img_ref, out_ref = oracle.layer(Kb[:, :, :L], Vb[:, :, :L], bits16(q), G, bk, bv, kmode)
+        img = cache.export_layer(0)
+        if not np.array_equal(img, img_ref):
+            bad = np.flatnonzero(img != img_ref)
+            pytest.fail(f"{tag} L={L}: image differs at {bad.size} bytes, first {bad[:8]}")
+        check_outputs(out32, out16, out_ref, f"{tag} L={L} splits={splits}")
+    assert kvq.kvq_device_status(cache.h) == 0
+
+
+@pytest.mark.parametrize("kmode", [0, 1])
+@pytest.mark.parametrize("splits", [0, 1, 2, 3])
+def test_fused_from_empty(kmode, splits):
+    """Token by token from an empty cache: first token of a half (16, 48), of a block
+    (32, 64 with per-channel flushes), ragged lengths in between."""
+    run_fused(2, 2, 2, 64, (4, 2), kmode, 0, 70, [1, 2, 15, 16, 17, 31, 32, 33, 48, 49, 63, 64, 65, 70],
+              splits=splits, tag=f"empty{kmode}{splits}")
+
+
+@pytest.mark.parametrize("kmode", [0, 1])
+@pytest.mark.parametrize("bk", [2, 4, 8])
+@pytest.mark.parametrize("bv", [2, 4, 8])
+def test_fused_bit_pairs(kmode, bk, bv):
+    run_fused(2, 2, 4, 128, (bk, bv), kmode, 90, 40, [91, 96, 97, 112, 113, 128, 129, 130],
+              tag=f"K{bk}V{bv}m{kmode}")
+
+
+@pytest.mark.parametrize("G,kmode", [(1, 0), (3, 0), (7, 0), (8, 0), (1, 1), (4, 1)])
+def test_fused_gqa(G, kmode):
+    run_fused(2, 2, G, 128, (8, 4), kmode, 150, 20, [151, 160, 170], splits=0, tag=f"G{G}m{kmode}")
+
+
+def test_fused_llama_c2_schedule():
+    """Llama-3.1-8B attention shape, prompt 128 then 128 fused steps (K8V4, flushes at
+    160, 192, 224, 256 through the two-launch path); batch 4 to keep the oracle fast."""
+    wl = configs.Workload("fused-c2", 1, 4, 32, 8, 128, 128, 128, ((8, 4),))
+    run_fused(4, 8, 4, 128, (8, 4), 0, 128, 128, [129, 144, 145, 159, 160, 161, 200, 255, 256], wl=wl, tag="c2")
+
+
+def test_fused_matches_two_launches():
+    """The fused step leaves the same cache bytes as kvq_append followed by
+    kvq_decode_attn, and both outputs agree within the parity tolerance."""
+    B, Hkv, G, D, L0, n = 3, 4, 4, 128, 100, 40
+    wl = workload(B, Hkv, G, D, name="fused-vs-two")
+    K, V = inputs.layer_kv(wl, 0, L0 + n, "cuda")
+    a = kvq.Cache(1, B, Hkv, Hkv * G, D, L0 + n, [(4, 2)])
+    b = kvq.Cache(1, B, Hkv, Hkv * G, D, L0 + n, [(4, 2)])
+    for c in (a, b):
+        c.append(0, K[:, :, :L0].contiguous(), V[:, :, :L0].contiguous())
+    for L in range(L0 + 1, L0 + n + 1):
+        q = inputs.step_q(wl, 0, L, "cuda")
+        k1, v1 = K[:, :, L - 1:L].contiguous(), V[:, :, L - 1:L].contiguous()
+        oa = a.append_decode(0, k1, v1, q, out_fp32=True)
+        b.append(0, k1, v1)
+        ob = b.decode_attn(0, q, out_fp32=True)
+        torch.cuda.synchronize()
+        assert np.array_equal(a.export_layer(0), b.export_layer(0)), L
+        d = (oa - ob).double().abs().max().item()
+        assert d <= 1e-4, (L, d)

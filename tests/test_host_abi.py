@@ -66,7 +66,7 @@ def test_workspace_layout(lib):
         rec0 = 4 * D * 4 + 4 * D + 4 * D * 2 + 4 * D
         rec1 = 4 * D * 8 + 4 * D + 4 * D * 8 + 4 * D
         al = lambda x: (x + 255) // 256 * 256
-        expect = al(256 + 8 * 2)                       # status word + {K, V} max scale per layer
+        expect = al(256 + 16 * 2)                      # status word + {K, V} max scale per layer and parity
         expect = al(expect + rec0 * cap * B * Hkv)
         expect = al(expect + 64 * D * B * Hkv)          # residual of the per-channel layer
         expect = al(expect + rec1 * cap * B * Hkv)
@@ -96,6 +96,9 @@ def test_argument_checks_before_any_launch(lib):
         assert L.kvq_decode_attn(h, 0, fake, fake, 0, None) == kvq.KVQ_EINVAL  # empty layer
         assert L.kvq_decode_attn(h, 0, fake + 4, fake, 0, None) == kvq.KVQ_EALIGN
         assert "16-byte" in kvq.kvq_last_error()
+        assert L.kvq_append_decode(h, 0, fake, fake + 8, fake, fake, 0, None) == kvq.KVQ_EALIGN
+        assert L.kvq_append_decode(h, 0, fake, None, fake, fake, 0, None) == kvq.KVQ_EINVAL
+        assert L.kvq_append_decode(h, 5, fake, fake, fake, fake, 0, None) == kvq.KVQ_EINVAL
         assert kvq.kvq_seq_len(h, 1) == 0
         need = ctypes.c_size_t()
         assert L.kvq_export_layer(h, 0, None, 0, ctypes.byref(need)) == kvq.KVQ_OK
