@@ -303,6 +303,12 @@ __device__ __forceinline__ void load_query_scalars(BodyCtx &c, const float4 *sca
     c.qsum_g8 = v.z;
 }
 
+// Exponent kp of the power of two carried by p: p * 2^kp * s_v stays below 2^14 in fp16.
+__device__ __forceinline__ float value_bias(float smax_v) {
+    const int kp = smax_v > 0.f ? max(-24, min(14, 13 - floor_log2(smax_v))) : 14;
+    return static_cast<float>(kp);
+}
+
 // Thread constants that depend only on the lane, the group size and the layer scales.
 template <int KM, int D, int NT>
 __device__ __forceinline__ BodyCtx make_ctx(int lane, int G, float smax_v, const uint4 *aq_s) {
@@ -323,9 +329,7 @@ __device__ __forceinline__ BodyCtx make_ctx(int lane, int G, float smax_v, const
     c.m_hi = (c.g < G) ? 0xFFFFFFFFu : 0u;
     c.alpha_src0 = 4 * ((NT == 1) ? ((2 * c.t) % G) : min(2 * c.t, 7));
     c.alpha_src1 = 4 * ((NT == 1) ? ((2 * c.t + 1) % G) : min(2 * c.t + 1, 7));
-    // values: p * 2^kp * s_v stays below 2^14 in fp16
-    const int kp = smax_v > 0.f ? max(-24, min(14, 13 - floor_log2(smax_v))) : 14;
-    c.pbias = static_cast<float>(kp);
+    c.pbias = value_bias(smax_v);
     return c;
 }
 
@@ -896,25 +900,27 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
         issue_block(k);
     }
 
-    float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
-    float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
+    const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
+    const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
     if (fused && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) {
         atomicMax(p.smax_out, p.smax[0]);   // carry the old length's maxima forward
         atomicMax(p.smax_out + 1, p.smax[1]);
     }
+    BodyCtx c = make_ctx<KM, D, NT>(lane, G, smax_v, sm.aq_s);
+    c.res = p.res ? p.res + (static_cast<long long>(b) * p.Hkv + h) * 32 * D : nullptr;
+    const int hh = c.g % G;
+    // the key prescale needs no new scale (a token that completes a per-channel key group
+    // is never fused; per-token keys are scaled in fp32), so warp 0 sets up q first and
+    // its loads overlap the append
+    setup_query<KM, D>(p.q + (static_cast<long long>(b) * p.Hkv * G + h * G + hh) * D, smax_k, sm.aq_s, sm.scal_s,
+                       c, warp);
     if (append_here) {
         float own_k, own_v;
         append_token<BK, BV, KM, D>(p, static_cast<long long>(b) * p.Hkv + h, new_blk, (L - 1) & 31,
                                     reinterpret_cast<uint8_t *>(sm.scal_s + 32), own_k, own_v);
-        smax_k = fmaxf(smax_k, own_k);
-        smax_v = fmaxf(smax_v, own_v);
+        c.pbias = value_bias(fmaxf(smax_v, own_v));   // CTA-uniform: every warp's p carries it
         while (P.issued < nb && P.issued < NS) issue_block(P.issued);
     }
-    BodyCtx c = make_ctx<KM, D, NT>(lane, G, smax_v, sm.aq_s);
-    c.res = p.res ? p.res + (static_cast<long long>(b) * p.Hkv + h) * 32 * D : nullptr;
-    const int hh = c.g % G;
-    setup_query<KM, D>(p.q + (static_cast<long long>(b) * p.Hkv * G + h * G + hh) * D, smax_k, sm.aq_s, sm.scal_s,
-                       c, warp);
     __syncthreads();
     load_query_scalars(c, sm.scal_s);
 
