@@ -750,9 +750,9 @@ __host__ __device__ inline size_t smem_bars_off(int NS, int stage_bytes, int D, 
     return ((stage > comb ? stage : comb) + 127) & ~size_t(127);
 }
 
-// Bytes after the per-lane scalars: codes of a fused append's token (values, keys) and
-// the CTA's two scale maxima.
-__host__ __device__ constexpr int append_scratch_bytes(int D) { return 2 * D + 16; }
+// Bytes after the per-lane scalars: a fused append's token codes (values, keys: 2D), the
+// CTA's two scale maxima (16) and the token's fp16 scales/zeros per role and group.
+__host__ __device__ constexpr int append_scratch_bytes(int D) { return 2 * D + 16 + 2 * (D / 32) * 2 * 2; }
 
 __host__ __device__ inline size_t smem_total(int NS, int stage_bytes, int D, int NT) {
     const size_t bars = static_cast<size_t>(NW) * NS * 8 + 8 * ((NW * NS) & 1);   // keeps 16-B alignment
@@ -771,43 +771,32 @@ __device__ __forceinline__ SmemParts carve(uint8_t *smem, int NS, int stage_byte
 }
 
 // ------------------------------------------------------------------ fused append
-// Bits of token e's codes inside word widx of a 16-token half's code area (role 0 key
-// operand, 1 value operand), from the token's codes code[d].
+// Put token e's codes code[0..D) into a 16-token half's code area `area` (global or
+// shared memory) with per-code atomic ORs, `step` threads from `tid`.  The first token
+// of a half rebuilds the half: its words are zeroed first (stale bytes must read as
+// zero); the caller orders the zeroing before the ORs of other threads.
 template <int BITS>
-__device__ __forceinline__ uint32_t token_bits(int role, int widx, int e, const uint8_t *code, int D) {
-    constexpr int F = 32 / BITS;
-    int ln, w;
-    quant::word_lane(widx, D * BITS / 64, ln, w);
-    uint32_t out = 0;
-#pragma unroll
-    for (int f = 0; f < F; ++f) {
-        int ee, d;
-        quant::field_owner(role, ln, w, f, BITS, ee, d);
-        if (ee == e) out |= static_cast<uint32_t>(code[d]) << (f * BITS);
-    }
-    return out;
+__device__ __forceinline__ void zero_half(uint32_t *area, int tid, int step, int D) {
+    for (int widx = tid; widx < D * BITS / 2; widx += step) area[widx] = 0u;
 }
-
-// Write one half's words for token e: the first token of a half rebuilds the half (its
-// words hold no other token yet, and stale bytes must read as zero); a later token ORs
-// its fields, which are zero until now.
 template <int BITS>
-__device__ __forceinline__ void pack_token(uint32_t *area, int role, int e, const uint8_t *code, int D) {
-    const int nw = D * BITS / 2;
-    for (int widx = threadIdx.x; widx < nw; widx += NW * 32) {
-        const uint32_t bits = token_bits<BITS>(role, widx, e, code, D);
-        if (e == 0) area[widx] = bits;
-        else if (bits) atomicOr(area + widx, bits);
+__device__ __forceinline__ void or_token(uint32_t *area, int role, int e, const uint8_t *code, int tid, int step,
+                                         int D) {
+    for (int d = tid; d < D; d += step) {
+        int w, bit;
+        quant::code_place(role, e, d, D, BITS, w, bit);
+        atomicOr(area + w, static_cast<uint32_t>(code[d]) << bit);
     }
 }
 
 // Quantize and pack the token appended by a fused launch, token u of block `blk` of unit
-// `unit`, with the same arithmetic as the append kernel: values per token
-// (one warp per 32-channel group), keys per token the same way or, per channel, the new
-// row into the residual (slot u: the host takes the two-launch path when the token
-// completes a key group).  All threads of the CTA take part; afterwards the writes are
-// visible to the bulk copy of the block, and own_k / own_v hold this CTA's largest new
-// scales.
+// `unit`, with the same arithmetic as the append kernel: values per token (one warp per
+// 32-channel group), keys per token the same way or, per channel, the new row into the
+// residual (slot u: the host takes the two-launch path when the token completes a key
+// group).  All threads of the CTA take part.  The cache in HBM gets the new bytes for
+// later steps; this launch does not read them back: the warp that processes the block
+// patches its staged copy (patch_stage) from the codes, scales and zeros kept in
+// `scratch`.  own_k / own_v: the CTA's largest new scales.
 template <int BK, int BV, int KM, int D>
 __device__ __forceinline__ void append_token(const DecodeParams &p, long long unit, int blk, int u,
                                              uint8_t *scratch, float &own_k, float &own_v) {
@@ -817,8 +806,9 @@ __device__ __forceinline__ void append_token(const DecodeParams &p, long long un
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = u & 15, eta = u >> 4;
     uint8_t *rec = p.rec_w + (unit * p.cap_blk + blk) * static_cast<long long>(REC);
-    uint8_t *codes = scratch;                                   // [0, D): values, [D, 2D): keys
+    uint8_t *codes = scratch;                                          // [0, D): values, [D, 2D): keys
     unsigned *cmax = reinterpret_cast<unsigned *>(scratch + 2 * D);   // keys, values (fp16 bits)
+    uint16_t *szs = reinterpret_cast<uint16_t *>(scratch + 2 * D + 16);   // [role][j][scale, zero]
     if (threadIdx.x < 2) cmax[threadIdx.x] = 0u;
     __syncthreads();
     constexpr int NROLE = KM == 1 ? 2 : 1;
@@ -843,6 +833,8 @@ __device__ __forceinline__ void append_token(const DecodeParams &p, long long un
             const int so = quant::tok_sz_off(u, j, NJ);
             *reinterpret_cast<uint16_t *>(sz + so) = s16;
             *reinterpret_cast<uint16_t *>(sz + so + 4 * NJ) = z16;
+            szs[(role * NJ + j) * 2] = s16;
+            szs[(role * NJ + j) * 2 + 1] = z16;
             atomicMax(cmax + role, static_cast<unsigned>(s16));
         }
     }
@@ -851,15 +843,51 @@ __device__ __forceinline__ void append_token(const DecodeParams &p, long long un
         uint32_t *dst = reinterpret_cast<uint32_t *>(p.res_w + (unit * 32 + u) * D);
         for (int i = threadIdx.x; i < D / 2; i += NW * 32) dst[i] = src[i];
     }
+    uint32_t *vwords = reinterpret_cast<uint32_t *>(rec + KC + KSZ + eta * 2 * D * BV);
+    uint32_t *kwords = reinterpret_cast<uint32_t *>(rec + eta * 2 * D * BK);
+    if (e == 0) {   // the half's first token: its words are rebuilt from zero
+        zero_half<BV>(vwords, threadIdx.x, NW * 32, D);
+        if constexpr (KM == 1) zero_half<BK>(kwords, threadIdx.x, NW * 32, D);
+    }
     __syncthreads();
-    pack_token<BV>(reinterpret_cast<uint32_t *>(rec + KC + KSZ + eta * 2 * D * BV), 1, e, codes, D);
-    if constexpr (KM == 1) pack_token<BK>(reinterpret_cast<uint32_t *>(rec + eta * 2 * D * BK), 0, e, codes + D, D);
-    __threadfence();                                   // the new bytes are performed GPU-wide ...
-    asm volatile("fence.proxy.async;" ::: "memory");   // ... and ordered before async-proxy reads
-    __syncthreads();
+    or_token<BV>(vwords, 1, e, codes, threadIdx.x, NW * 32, D);
+    if constexpr (KM == 1) or_token<BK>(kwords, 0, e, codes + D, threadIdx.x, NW * 32, D);
     own_k = __half2float(__ushort_as_half(static_cast<unsigned short>(cmax[0])));
     own_v = __half2float(__ushort_as_half(static_cast<unsigned short>(cmax[1])));
     if (threadIdx.x < 2 && cmax[threadIdx.x]) atomicMax(p.smax_out + threadIdx.x, cmax[threadIdx.x]);
+}
+
+// The warp that processes the appended token's block writes the token into its staged
+// copy of the block (taken before or while the new bytes reached HBM), so the copy equals
+// the block after the append: the code fields of the token (the half's words rebuilt when
+// it is the half's first token, as in HBM) and its scales and zeros.  One warp; the
+// stage's bulk copy has completed.
+template <int BK, int BV, int KM, int D>
+__device__ __forceinline__ void patch_stage(uint8_t *stage, int u, const uint8_t *scratch, int lane) {
+    constexpr int NJ = D / 32;
+    constexpr int KC = 4 * D * BK, KSZ = 4 * D, VC = 4 * D * BV;
+    const int e = u & 15, eta = u >> 4;
+    const uint16_t *szs = reinterpret_cast<const uint16_t *>(scratch + 2 * D + 16);
+    uint32_t *vwords = reinterpret_cast<uint32_t *>(stage + KC + KSZ + eta * 2 * D * BV);
+    uint32_t *kwords = reinterpret_cast<uint32_t *>(stage + eta * 2 * D * BK);
+    if (e == 0) {
+        zero_half<BV>(vwords, lane, 32, D);
+        if constexpr (KM == 1) zero_half<BK>(kwords, lane, 32, D);
+        __syncwarp();
+    }
+    or_token<BV>(vwords, 1, e, scratch, lane, 32, D);
+    if constexpr (KM == 1) or_token<BK>(kwords, 0, e, scratch + D, lane, 32, D);
+    if (lane < NJ) {
+        uint8_t *sz = stage + KC + KSZ + VC + quant::tok_sz_off(u, lane, NJ);
+        *reinterpret_cast<uint16_t *>(sz) = szs[(NJ + lane) * 2];
+        *reinterpret_cast<uint16_t *>(sz + 4 * NJ) = szs[(NJ + lane) * 2 + 1];
+        if constexpr (KM == 1) {
+            uint8_t *kz = stage + KC + quant::tok_sz_off(u, lane, NJ);
+            *reinterpret_cast<uint16_t *>(kz) = szs[lane * 2];
+            *reinterpret_cast<uint16_t *>(kz + 4 * NJ) = szs[lane * 2 + 1];
+        }
+    }
+    __syncwarp();
 }
 
 // ------------------------------------------------------------------ per-layer kernel
@@ -890,15 +918,13 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
         if (blk == tail_blk) pipe_issue(P, src + VSKIP, REC - VSKIP, VSKIP);
         else pipe_issue(P, src, REC);
     };
-    // a fused launch first writes the new token, token L - 1 (the last of its block);
-    // that block is fetched after it
+    for (int k = 0; k < NS && k < nb; ++k) issue_block(k);
+    // a fused launch appends token L - 1 (the last of block new_blk) in the CTA that holds
+    // that block; the block's warp patches its staged copy with the token
     const bool fused = p.k_new != nullptr;
     const int new_blk = (L - 1) >> 5;
     const bool append_here = fused && new_blk >= blk0 && new_blk < blk1;   // CTA-uniform
-    for (int k = 0; k < NS && k < nb; ++k) {
-        if (append_here && blk0 + warp + NW * k == new_blk) break;
-        issue_block(k);
-    }
+    uint8_t *append_scratch = reinterpret_cast<uint8_t *>(sm.scal_s + 32);
 
     const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
     const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
@@ -917,9 +943,8 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     if (append_here) {
         float own_k, own_v;
         append_token<BK, BV, KM, D>(p, static_cast<long long>(b) * p.Hkv + h, new_blk, (L - 1) & 31,
-                                    reinterpret_cast<uint8_t *>(sm.scal_s + 32), own_k, own_v);
+                                    append_scratch, own_k, own_v);
         c.pbias = value_bias(fmaxf(smax_v, own_v));   // CTA-uniform: every warp's p carries it
-        while (P.issued < nb && P.issued < NS) issue_block(P.issued);
     }
     __syncthreads();
     load_query_scalars(c, sm.scal_s);
@@ -935,6 +960,8 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
             failed = true;
             break;
         }
+        if (append_here && blk0 + warp + NW * i == new_blk)
+            patch_stage<BK, BV, KM, D>(const_cast<uint8_t *>(pipe_front(P)), (L - 1) & 31, append_scratch, lane);
         process_unit<BK, BV, KM, D, NT, 2, false>(A, pipe_front(P), 32, c);
         pipe_pop(P);
         if (P.issued < nb) issue_block(P.issued);
@@ -943,6 +970,8 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
         if (!pipe_wait(P)) {
             failed = true;
         } else {
+            if (append_here && tail_blk == new_blk)
+                patch_stage<BK, BV, KM, D>(const_cast<uint8_t *>(pipe_front(P)), (L - 1) & 31, append_scratch, lane);
             process_unit<BK, BV, KM, D, NT, 2, true>(A, pipe_front(P), rem, c);
             ++i;
         }

@@ -49,6 +49,31 @@ __device__ __forceinline__ void field_owner(int role, int lane, int w, int f, in
     }
 }
 
+// Word index (inside a half's code area) and bit offset of the code of token e (0..15
+// inside the half), channel d, for the key operand role (role 0) or the value operand
+// role (role 1) of the v1 format: the inverse of field_owner.
+__device__ __forceinline__ void code_place(int role, int e, int d, int D, int bits, int &word, int &bit) {
+    const int P = 16 / bits;
+    int lane, slot, hb;
+    if (role == 0) {   // token e = 8i + gk, channel d = 16k + 8r + 2t + hb
+        const int i = e >> 3, gk = e & 7, k = d >> 4, ee = d & 15;
+        const int t = (ee & 7) >> 1, r = ee >> 3;
+        hb = ee & 1;
+        lane = 4 * gk + t;
+        slot = (2 * k + i) * 2 + r;
+    } else {           // token e = 8ch + 2t + hb, channel d = 16m + g + 8rh
+        const int t = (e & 7) >> 1, ch = e >> 3, m = d >> 4, rho = d & 15;
+        const int g = rho & 7, rh = rho >> 3;
+        hb = e & 1;
+        lane = 4 * g + t;
+        slot = 4 * m + 2 * ch + rh;
+    }
+    const int Wh = D * bits / 64, c = Wh < 4 ? Wh : 4;
+    const int w = slot / P, field = slot % P + hb * P;
+    word = ((w / c) * 32 + lane) * c + (w % c);
+    bit = field * bits;
+}
+
 // Byte offsets of a scale/zero pair in the s/z areas of the v1 format.
 __device__ __forceinline__ int chan_sz_off(int d) {   // per-channel keys: scale; zero at +4
     const int k = d >> 4, e = d & 15;
