@@ -953,18 +953,33 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     acc_init(A);
     const bool has_tail = tail_blk >= blk0 && tail_blk < blk1 && ((tail_blk - blk0) % NW) == warp;
     const int nb_main = nb - (has_tail ? 1 : 0);
+    // the appended token is in the unit's last block, the last block of its warp: the
+    // tail block, or (per-token keys, L % 32 == 0) the last full block, which is then
+    // taken out of the main loop
+    const bool patch_full = KM == 1 && append_here && !has_tail && nb > 0 && blk0 + warp + NW * (nb - 1) == new_blk;
+    const int nb_loop = nb_main - (patch_full ? 1 : 0);
     bool failed = false;
     int i = 0;
-    for (; i < nb_main; ++i) {
+    for (; i < nb_loop; ++i) {
         if (!pipe_wait(P)) {
             failed = true;
             break;
         }
-        if (append_here && blk0 + warp + NW * i == new_blk)
-            patch_stage<BK, BV, KM, D>(const_cast<uint8_t *>(pipe_front(P)), (L - 1) & 31, append_scratch, lane);
         process_unit<BK, BV, KM, D, NT, 2, false>(A, pipe_front(P), 32, c);
         pipe_pop(P);
         if (P.issued < nb) issue_block(P.issued);
+    }
+    if constexpr (KM == 1) {
+        if (!failed && patch_full) {
+            if (!pipe_wait(P)) {
+                failed = true;
+            } else {
+                patch_stage<BK, BV, KM, D>(const_cast<uint8_t *>(pipe_front(P)), (L - 1) & 31, append_scratch, lane);
+                process_unit<BK, BV, KM, D, NT, 2, false>(A, pipe_front(P), 32, c);
+                pipe_pop(P);
+                ++i;
+            }
+        }
     }
     if (!failed && has_tail) {
         if (!pipe_wait(P)) {
