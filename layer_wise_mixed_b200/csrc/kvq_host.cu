@@ -501,7 +501,8 @@ static void paged_units(const kvq_handle *h, int layer, int *u2, int *u4) {
 }
 
 // INT2 and INT4 split counts: minimise (waves) x (slowest CTA), an INT2 unit (32 tokens,
-// 2-bit record) weighing 1 and an INT4 page (16 tokens) 0.55.
+// 2-bit record) weighing 1 and an INT4 page (16 tokens) 0.8 (measured: ~700 and ~560
+// warp-instructions).
 static int paged_splits(kvq_handle *h, int layer, int *S2, int *S4) {
     int u2, u4;
     paged_units(h, layer, &u2, &u4);
@@ -525,7 +526,7 @@ static int paged_splits(kvq_handle *h, int layer, int *S2, int *S4) {
         for (int c = (u4 > 0 ? 1 : 0); c <= (u4 > 0 ? std::min(48, u4) : 0); ++c) {
             if (a + c < 1 || a + c > kvq::kMaxSplits) continue;
             const double t2 = a ? std::ceil(std::ceil(static_cast<double>(u2) / a) / kvq::kDecodeWarps) : 0.0;
-            const double t4 = c ? 0.55 * std::ceil(std::ceil(static_cast<double>(u4) / c) / kvq::kDecodeWarps) : 0.0;
+            const double t4 = c ? 0.8 * std::ceil(std::ceil(static_cast<double>(u4) / c) / kvq::kDecodeWarps) : 0.0;
             const double waves = std::ceil(static_cast<double>(units) * (a + c) / slots);
             const double cost = waves * (std::max(t2, t4) + 1.0) * (1.0 + 0.002 * (a + c));
             if (cost < best - 1e-9) {
