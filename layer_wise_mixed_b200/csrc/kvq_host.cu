@@ -104,16 +104,20 @@ int cuda_fail(cudaError_t e, const char *what) {
 }
 
 // Estimated time of a per-layer decode launch, in units of one block's processing by a
-// warp: waves x (blocks per warp + a per-CTA overhead of about one block); with a single
-// stage per warp the copy latency of every block after the first is exposed (about 0.6
-// of a block each).
-double decode_cost(int units, int nblk, int S, int nstage, int slots) {
+// warp.  CTAs are handed to SMs as slots free up, so the launch lasts about as long as
+// the busiest SM's share: ceil(CTAs / SMs) CTAs, of which `occ` run at once; with fewer
+// than `occ` an SM is not full and the CTAs' own latency decides.  A CTA costs its
+// blocks per warp plus about two blocks of fixed latency (first copy, q set-up,
+// combine); with a single stage per warp the copy latency of every block after the
+// first is exposed too (about 0.6 of a block each).  Splitting adds the merge launch.
+double decode_cost(int units, int nblk, int S, int nstage, int occ, int sms) {
     const int bps = (nblk + S - 1) / S;
     const int sreal = (nblk + bps - 1) / bps;
-    const double waves = std::ceil(static_cast<double>(units) * sreal / std::max(1, slots));
+    const double per_sm = std::ceil(static_cast<double>(units) * sreal / std::max(1, sms));
+    const double load = std::max(1.0, per_sm / std::max(1, occ));
     const double bpw = std::ceil(static_cast<double>(bps) / kvq::kDecodeWarps);
-    const double per_cta = bpw + 1.0 + (nstage == 1 ? 0.6 * (bpw - 1.0) : 0.0);
-    return waves * per_cta * (1.0 + 0.002 * sreal);
+    const double per_cta = bpw + 2.0 + (nstage == 1 ? 0.6 * (bpw - 1.0) : 0.0);
+    return load * per_cta * (1.0 + 0.002 * sreal) + (sreal > 1 ? 0.5 : 0.0);
 }
 
 }  // namespace
@@ -464,10 +468,9 @@ static int splits_for(kvq_handle *h, int layer, int *S_out, int *nstage_out) {
         int per_sm = 1;
         cudaError_t e = kvq::decode_occupancy(h->desc.head_dim, g.bk, g.bv, g.kmode, G, g.rec_bytes, ns, &per_sm);
         if (e != cudaSuccess) return cuda_fail(e, "decode occupancy");
-        const int slots = std::max(1, per_sm) * h->sm_count;
         if (h->forced_splits > 0) {
             const int S = std::min(h->forced_splits, smax);
-            const double c = decode_cost(units, nblk, S, ns, slots);
+            const double c = decode_cost(units, nblk, S, ns, per_sm, h->sm_count);
             if (c < best - 1e-9) {
                 best = c;
                 *S_out = S;
@@ -479,7 +482,7 @@ static int splits_for(kvq_handle *h, int layer, int *S_out, int *nstage_out) {
             const int bps = (nblk + S - 1) / S;
             const int sreal = (nblk + bps - 1) / bps;
             if (sreal != S) continue;
-            const double c = decode_cost(units, nblk, S, ns, slots);
+            const double c = decode_cost(units, nblk, S, ns, per_sm, h->sm_count);
             if (c < best - 1e-9) {
                 best = c;
                 *S_out = S;
