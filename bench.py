@@ -475,7 +475,7 @@ def main():
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                              "frac": achieved / peak,
                              "traffic": captured_traffic(wl.name, dec_bytes / launches_dec),
-                             "kernel": "decode_split_kernel (+merge)",
+                             "kernel": ("decode_paged_kernel" if wl.paged else "decode_split_kernel") + " (+merge)",
                              "peak_source": peak_src, "avg_launch_us": 1e3 * dec_ms / launches_dec,
                              "algorithmic_bytes_per_launch": dec_bytes / launches_dec},
                 "cpu_baseline": cpu,

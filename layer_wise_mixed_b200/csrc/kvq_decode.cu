@@ -351,7 +351,9 @@ __device__ __forceinline__ void acc_init(WarpAcc<D, NT> &A) {
 // One unit of NH 16-token halves (32-token block record, or 16-token page when NH = 1)
 // staged at R; `valid` tokens are present (TAIL: valid may be < 16 NH; per-channel
 // TAIL blocks take their keys from the bf16 residual).
-template <int BK, int BV, int KM, int D, int NT, int NH, bool TAIL>
+// PAIR: R holds two 16-token pages (per-token keys), one per half, each laid out
+// [K codes][K scales/zeros][V codes][V scales/zeros], instead of one 32-token record.
+template <int BK, int BV, int KM, int D, int NT, int NH, bool TAIL, bool PAIR = false>
 __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R, const int valid,
                                              const BodyCtx &c) {
     constexpr int KS = D / 16;
@@ -362,6 +364,15 @@ __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R
     constexpr int PK = 16 / BK, PV = 16 / BV;
     constexpr int KC = 2 * NH * D * BK, KSZ = (KM == 0 ? 4 * D : 2 * NH * D), VC = 2 * NH * D * BV;
     static_assert(KM == 1 || NH == 2, "per-channel keys come in 32-token groups");
+    static_assert(!PAIR || (KM == 1 && NH == 2), "page pairs hold per-token keys");
+    // areas of half hf (record: the halves share each area; pair: one page per half)
+    constexpr int KCH = 2 * D * BK, KSZH = 2 * D, VCH = 2 * D * BV, PAGE = KCH + KSZH + VCH + 2 * D;
+    auto kcode = [&](int hf) { return R + (PAIR ? hf * PAGE : hf * KCH); };
+    auto ksz_pair = [&](int pi) { return PAIR ? R + (pi >> 3) * PAGE + KCH + 8 * NJ * (pi & 7) : R + KC + 8 * NJ * pi; };
+    auto vcode = [&](int kk) { return PAIR ? R + kk * PAGE + KCH + KSZH : R + KC + KSZ + kk * VCH; };
+    auto vsz_pair = [&](int kk, int i) {
+        return PAIR ? R + kk * PAGE + KCH + KSZH + VCH + 8 * NJ * (i - 8 * kk) : R + KC + KSZ + VC + 8 * NJ * i;
+    };
     const int lane = c.lane, g = c.g, t = c.t;
 
     // ===== scores S^T (rows: heads, columns: 8-token tiles) =====
@@ -403,7 +414,7 @@ __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R
                 const int w = w0 + x;
                 const int off = (((w / CH) * 32 + lane) * CH + (w % CH)) * 4;
 #pragma unroll
-                for (int hf = 0; hf < NH; ++hf) kw[hf][x] = *reinterpret_cast<const uint32_t *>(R + hf * 2 * D * BK + off);
+                for (int hf = 0; hf < NH; ++hf) kw[hf][x] = *reinterpret_cast<const uint32_t *>(kcode(hf) + off);
             }
             const uint4 aqv = c.aq_s[k * 32 + lane];
             const uint32_t ak[4] = {aqv.x, aqv.y, aqv.z, aqv.w};
@@ -440,20 +451,20 @@ __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R
         }
     } else {
         // per-token key scales on the (group, head) rows, then sum the rows of a head
-        const uint8_t *ks = R + KC;
 #pragma unroll
         for (int n = 0; n < NTI; ++n) {
             const int pi = 4 * n + t;   // token pair (8n + 2t, 8n + 2t + 1)
+            const uint8_t *kp = ksz_pair(pi);
             float v0 = 0.f, v1 = 0.f;
             if (c.row_g) {
-                const uint32_t sw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * c.jg);
-                const uint32_t zw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * NJ + 4 * c.jg);
+                const uint32_t sw = *reinterpret_cast<const uint32_t *>(kp + 4 * c.jg);
+                const uint32_t zw = *reinterpret_cast<const uint32_t *>(kp + 4 * NJ + 4 * c.jg);
                 v0 = fmaf(half_lo_f(sw), acc[n][0], half_lo_f(zw) * c.qsum_g);
                 v1 = fmaf(half_hi_f(sw), acc[n][1], half_hi_f(zw) * c.qsum_g);
             }
             if (c.row_g8) {
-                const uint32_t sw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * c.jg8);
-                const uint32_t zw = *reinterpret_cast<const uint32_t *>(ks + 8 * NJ * pi + 4 * NJ + 4 * c.jg8);
+                const uint32_t sw = *reinterpret_cast<const uint32_t *>(kp + 4 * c.jg8);
+                const uint32_t zw = *reinterpret_cast<const uint32_t *>(kp + 4 * NJ + 4 * c.jg8);
                 v0 += fmaf(half_lo_f(sw), acc[n][2], half_lo_f(zw) * c.qsum_g8);
                 v1 += fmaf(half_hi_f(sw), acc[n][3], half_hi_f(zw) * c.qsum_g8);
             }
@@ -515,27 +526,27 @@ __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R
 #pragma unroll
     for (int kk = 0; kk < NH; ++kk) {
         uint32_t vw[WHV];
-        load_lane_words<WHV>(R + KC + KSZ + kk * 2 * D * BV, lane, vw);
+        load_lane_words<WHV>(vcode(kk), lane, vw);
         uint32_t pah, pal, pbh, pbl;   // p of token pairs A (16kk+2t, +1) and B (+8, +9)
         split2(pr[2 * kk][0], pr[2 * kk][1], pah, pal);
         split2(pr[2 * kk + 1][0], pr[2 * kk + 1][1], pbh, pbl);
-        const uint8_t *vs = R + KC + KSZ + VC;
         const int iA = 8 * kk + t, iB = iA + 4;
+        const uint8_t *vsA = vsz_pair(kk, iA), *vsB = vsz_pair(kk, iB);
         uint32_t sA[NJ], sB[NJ];
         if constexpr (NJ == 4) {
-            const uint4 xa = *reinterpret_cast<const uint4 *>(vs + 8 * NJ * iA);
-            const uint4 xb = *reinterpret_cast<const uint4 *>(vs + 8 * NJ * iB);
+            const uint4 xa = *reinterpret_cast<const uint4 *>(vsA);
+            const uint4 xb = *reinterpret_cast<const uint4 *>(vsB);
             sA[0] = xa.x; sA[1] = xa.y; sA[2] = xa.z; sA[3] = xa.w;
             sB[0] = xb.x; sB[1] = xb.y; sB[2] = xb.z; sB[3] = xb.w;
         } else {
 #pragma unroll
             for (int j = 0; j < NJ; ++j) {
-                sA[j] = reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iA)[j];
-                sB[j] = reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iB)[j];
+                sA[j] = reinterpret_cast<const uint32_t *>(vsA)[j];
+                sB[j] = reinterpret_cast<const uint32_t *>(vsB)[j];
             }
         }
-        uint32_t zA = *reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iA + 4 * NJ + 4 * c.jz);
-        uint32_t zB = *reinterpret_cast<const uint32_t *>(vs + 8 * NJ * iB + 4 * NJ + 4 * c.jz);
+        uint32_t zA = *reinterpret_cast<const uint32_t *>(vsA + 4 * NJ + 4 * c.jz);
+        uint32_t zB = *reinterpret_cast<const uint32_t *>(vsB + 4 * NJ + 4 * c.jz);
         if constexpr (TAIL) {
             // absent tokens: p = 0 and their scale/zero halves may hold anything
             const int u0 = 16 * kk + 2 * t;
@@ -1003,68 +1014,78 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
 // Splits [0, S2) cover the request's INT2 records (32-token groups, 2-bit keys per
 // channel, 2-bit values per token); splits [S2, S2 + S4) its INT4 pages (16 tokens,
 // 4-bit keys and values per token): main pages, then the pending pages of INT2 tokens
-// whose group is still open.  Every split is bitwidth-homogeneous.
-__global__ void __launch_bounds__(NW * 32, 4) decode_paged_kernel(const PagedDecodeParams p) {
-    pdl_enter();
+// whose group is still open.  Every split is bitwidth-homogeneous.  INT4 work items are
+// pairs of full pages, staged side by side and processed as one 32-token unit (the
+// attention is a sum over tokens: their order does not matter), then the odd full page
+// and the partly filled pages one by one.
+template <bool INT2>
+__device__ __forceinline__ void paged_body(const PagedDecodeParams &p, uint8_t *smem, int warp, int lane, int b,
+                                           int h, int sp) {
     constexpr int D = 128, NT = 1;
     constexpr int REC2 = unit_bytes(D, 2, 2, 0, 2), PAGE4 = unit_bytes(D, 4, 4, 1, 1);
-    constexpr int STAGE = REC2 > PAGE4 ? REC2 : PAGE4;
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = blockIdx.z, h = blockIdx.y, sp = blockIdx.x;
+    constexpr int STAGE = REC2 > 2 * PAGE4 ? REC2 : 2 * PAGE4;
     const int G = p.G, NS = p.nstage;
-    const bool int2 = sp < p.S2;
     const int n2g = p.cnt[b].n2g, n4 = p.cnt[b].n4, np = p.cnt[b].np;
-    const int n4p = (n4 + 15) >> 4, npp = (np + 15) >> 4;
-    int u0, u1;
-    if (int2) {
-        const int per = (n2g + p.S2 - 1) / p.S2;
-        u0 = min(n2g, sp * per);
-        u1 = min(n2g, u0 + per);
-    } else {
-        const int tot = n4p + npp, per = (tot + p.S4 - 1) / p.S4;
-        u0 = min(tot, (sp - p.S2) * per);
-        u1 = min(tot, u0 + per);
-    }
+    // INT4 pages: f4 full main pages (then a partial one of pm tokens), fp full pending
+    // pages (0 or 1, then a partial one of pp tokens)
+    const int f4 = n4 >> 4, pm = n4 & 15, fp = np >> 4, pp = np & 15;
+    const int F = f4 + fp, npair = F >> 1;
+    const int nitems = INT2 ? n2g : npair + (F & 1) + (pm ? 1 : 0) + (pp ? 1 : 0);
+    const int nsplit = INT2 ? p.S2 : p.S4, si = INT2 ? sp : sp - p.S2;
+    const int per = (nitems + nsplit - 1) / nsplit;
+    const int u0 = min(nitems, si * per), u1 = min(nitems, u0 + per);
     const SmemParts sm = carve(smem, NS, STAGE, D, NT);
     WarpPipe P{sm.stages + static_cast<size_t>(warp) * NS * STAGE, sm.bars + warp * NS, NS, STAGE, lane, 0, 0, 0u, 0};
     pipe_init(P);
     const int *tab = p.table + static_cast<long long>(b) * p.P_cap;
     const uint8_t *pool2 = p.pool2 + static_cast<long long>(h) * p.n2_cap * REC2;
     const uint8_t *pool4 = p.pool4 + static_cast<long long>(h) * p.n4_cap * PAGE4;
-    // unit u of this request -> (source, valid tokens)
     // table of request b: INT2 groups from the front (entry = the group's first 16-token
     // page, groups occupy page pairs), INT4 main pages from the back
-    auto src_of = [&](int u) -> const uint8_t * {
-        if (int2) return pool2 + static_cast<long long>(tab[u] >> 1) * REC2;
-        const int page = u < n4p ? tab[p.P_cap - 1 - u] : p.pend_base + 2 * b + (u - n4p);
+    auto full_page = [&](int f) -> const uint8_t * {   // f-th full INT4 page
+        const int page = f < f4 ? tab[p.P_cap - 1 - f] : p.pend_base + 2 * b;
         return pool4 + static_cast<long long>(page) * PAGE4;
     };
-    auto valid_of = [&](int u) -> int {
-        if (int2) return 32;
-        if (u < n4p) return (u == n4p - 1 && (n4 & 15)) ? (n4 & 15) : 16;
-        const int v = u - n4p;
-        return (v == npp - 1 && (np & 15)) ? (np & 15) : 16;
+    // item u after the pairs: 0 = odd full page, 1 = partial main page, 2 = partial pending page
+    auto single_kind = [&](int u) -> int {
+        int k = u - npair;
+        if (!(F & 1)) ++k;
+        if (k >= 1 && !pm) ++k;
+        return k;
+    };
+    auto issue_item = [&](int u) {
+        if (INT2) {
+            pipe_issue(P, pool2 + static_cast<long long>(tab[u] >> 1) * REC2, REC2);
+        } else if (u < npair) {
+            const uint8_t *a = full_page(2 * u), *bb = full_page(2 * u + 1);
+            const int st = P.ist;
+            if (lane == 0) {
+                fence_proxy_async();
+                mbar_expect_tx(&P.bars[st], 2 * PAGE4);
+                uint8_t *dst = P.stages + static_cast<size_t>(st) * P.stage_bytes;
+                bulk_g2s(dst, a, PAGE4, &P.bars[st]);
+                bulk_g2s(dst + PAGE4, bb, PAGE4, &P.bars[st]);
+            }
+            ++P.issued;
+            if (++P.ist == P.NS) P.ist = 0;
+        } else {
+            const int k = single_kind(u);
+            const int page = k == 0 ? (F - 1 < f4 ? tab[p.P_cap - 1 - (F - 1)] : p.pend_base + 2 * b)
+                           : k == 1 ? tab[p.P_cap - 1 - f4] : p.pend_base + 2 * b + fp;
+            pipe_issue(P, pool4 + static_cast<long long>(page) * PAGE4, PAGE4);
+        }
     };
     const int nb = (u1 - u0 > warp) ? (u1 - u0 - warp + NW - 1) / NW : 0;
-    const unsigned bytes = int2 ? REC2 : PAGE4;
-    for (int k = 0; k < NS && k < nb; ++k) pipe_issue(P, src_of(u0 + warp + NW * k), bytes);
+    for (int k = 0; k < NS && k < nb; ++k) issue_item(u0 + warp + NW * k);
 
     const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
     const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
     WarpAcc<D, NT> A;
     acc_init(A);
-    BodyCtx c;
     const long long qoff = (static_cast<long long>(b) * p.Hkv * G + h * G + (lane >> 2) % G) * D;
-    if (int2) {
-        c = make_ctx<0, D, NT>(lane, G, smax_v, sm.aq_s);
-        c.res = nullptr;
-        setup_query<0, D>(p.q + qoff, smax_k, sm.aq_s, sm.scal_s, c, warp);
-    } else {
-        c = make_ctx<1, D, NT>(lane, G, smax_v, sm.aq_s);
-        c.res = nullptr;
-        setup_query<1, D>(p.q + qoff, smax_k, sm.aq_s, sm.scal_s, c, warp);
-    }
+    BodyCtx c = make_ctx<INT2 ? 0 : 1, D, NT>(lane, G, smax_v, sm.aq_s);
+    c.res = nullptr;
+    setup_query<INT2 ? 0 : 1, D>(p.q + qoff, smax_k, sm.aq_s, sm.scal_s, c, warp);
     __syncthreads();
     load_query_scalars(c, sm.scal_s);
 
@@ -1076,15 +1097,18 @@ __global__ void __launch_bounds__(NW * 32, 4) decode_paged_kernel(const PagedDec
             break;
         }
         const int u = u0 + warp + NW * i;
-        if (int2) {
+        if (INT2) {
             process_unit<2, 2, 0, D, NT, 2, false>(A, pipe_front(P), 32, c);
+        } else if (u < npair) {
+            process_unit<4, 4, 1, D, NT, 2, false, true>(A, pipe_front(P), 32, c);
         } else {
-            const int v = valid_of(u);
+            const int k = single_kind(u);
+            const int v = k == 0 ? 16 : (k == 1 ? pm : pp);
             if (v == 16) process_unit<4, 4, 1, D, NT, 1, false>(A, pipe_front(P), 16, c);
             else process_unit<4, 4, 1, D, NT, 1, true>(A, pipe_front(P), v, c);
         }
         pipe_pop(P);
-        if (P.issued < nb) pipe_issue(P, src_of(u0 + warp + NW * P.issued), bytes);
+        if (P.issued < nb) issue_item(u0 + warp + NW * P.issued);
     }
     if (failed) {
         pipe_drain(P, i);
@@ -1092,6 +1116,15 @@ __global__ void __launch_bounds__(NW * 32, 4) decode_paged_kernel(const PagedDec
     }
     combine_store<D, NT>(A, c, nb > 0 && !failed, smem, warp, static_cast<long long>(b) * p.Hkv * G + h * G, sp,
                          p.S2 + p.S4, p.out_fp32, p.out, p.part_acc, p.part_ml);
+}
+
+__global__ void __launch_bounds__(NW * 32, 4) decode_paged_kernel(const PagedDecodeParams p) {
+    pdl_enter();
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.z, h = blockIdx.y, sp = blockIdx.x;
+    if (sp < p.S2) paged_body<true>(p, smem, warp, lane, b, h, sp);
+    else paged_body<false>(p, smem, warp, lane, b, h, sp);
 }
 
 // Log-sum-exp merge of the split partials ("merged by online log-sum-exp").
@@ -1230,15 +1263,14 @@ cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmod
 int paged_rec2_bytes(int D) { return unit_bytes(D, 2, 2, 0, 2); }
 int paged_page4_bytes(int D) { return unit_bytes(D, 4, 4, 1, 1); }
 
-int decode_paged_stages() {
-    const int stage = paged_rec2_bytes(128) > paged_page4_bytes(128) ? paged_rec2_bytes(128) : paged_page4_bytes(128);
-    return decode_stages(stage, 128, 4);
+// A paged stage holds an INT2 record or two INT4 pages.
+static int paged_stage_bytes() {
+    return paged_rec2_bytes(128) > 2 * paged_page4_bytes(128) ? paged_rec2_bytes(128) : 2 * paged_page4_bytes(128);
 }
 
-size_t decode_paged_smem_bytes(int nstage) {
-    const int stage = paged_rec2_bytes(128) > paged_page4_bytes(128) ? paged_rec2_bytes(128) : paged_page4_bytes(128);
-    return smem_total(nstage, stage, 128, 1);
-}
+int decode_paged_stages() { return decode_stages(paged_stage_bytes(), 128, 4); }
+
+size_t decode_paged_smem_bytes(int nstage) { return smem_total(nstage, paged_stage_bytes(), 128, 1); }
 
 cudaError_t decode_paged_occupancy(int nstage, int *ctas_per_sm) {
     return prepare_kernel(reinterpret_cast<const void *>(decode_paged_kernel), decode_paged_smem_bytes(nstage), ctas_per_sm);

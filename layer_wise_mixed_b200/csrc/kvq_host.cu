@@ -499,13 +499,15 @@ static void paged_units(const kvq_handle *h, int layer, int *u2, int *u4) {
     *u2 = *u4 = 0;
     for (int b = 0; b < h->desc.batch; ++b) {
         *u2 = std::max(*u2, P.n2g[b]);
-        *u4 = std::max(*u4, (P.n4[b] + 15) / 16 + (P.np[b] + 15) / 16);
+        // INT4 work items: pairs of full pages, the odd full page, the partial main and
+        // pending pages
+        const int F = P.n4[b] / 16 + P.np[b] / 16;
+        *u4 = std::max(*u4, F / 2 + F % 2 + (P.n4[b] % 16 ? 1 : 0) + (P.np[b] % 16 ? 1 : 0));
     }
 }
 
 // INT2 and INT4 split counts: minimise (waves) x (slowest CTA), an INT2 unit (32 tokens,
-// 2-bit record) weighing 1 and an INT4 page (16 tokens) 0.8 (measured: ~700 and ~560
-// warp-instructions).
+// 2-bit record) weighing 1 and an INT4 item (mostly a pair of 16-token pages) 1.2.
 static int paged_splits(kvq_handle *h, int layer, int *S2, int *S4) {
     int u2, u4;
     paged_units(h, layer, &u2, &u4);
@@ -529,7 +531,7 @@ static int paged_splits(kvq_handle *h, int layer, int *S2, int *S4) {
         for (int c = (u4 > 0 ? 1 : 0); c <= (u4 > 0 ? std::min(48, u4) : 0); ++c) {
             if (a + c < 1 || a + c > kvq::kMaxSplits) continue;
             const double t2 = a ? std::ceil(std::ceil(static_cast<double>(u2) / a) / kvq::kDecodeWarps) : 0.0;
-            const double t4 = c ? 0.8 * std::ceil(std::ceil(static_cast<double>(u4) / c) / kvq::kDecodeWarps) : 0.0;
+            const double t4 = c ? 1.2 * std::ceil(std::ceil(static_cast<double>(u4) / c) / kvq::kDecodeWarps) : 0.0;
             const double waves = std::ceil(static_cast<double>(units) * (a + c) / slots);
             const double cost = waves * (std::max(t2, t4) + 1.0) * (1.0 + 0.002 * (a + c));
             if (cost < best - 1e-9) {

@@ -226,6 +226,7 @@ class Cache:
         else:
             self.desc = make_desc(num_layers, batch, n_kv_heads, n_q_heads, head_dim, max_ctx, layer_bits, kmodes)
         self.h = kvq_plan(self.desc)
+        self._destroy = load().kvq_destroy   # held so that teardown at interpreter exit still works
         self.nbytes = kvq_workspace_bytes(self.h)
         self.ws = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device)
         base = self.ws.data_ptr()
@@ -268,6 +269,7 @@ class Cache:
 
     def __del__(self):
         h = getattr(self, "h", None)
-        if h:
-            kvq_destroy(h)
+        destroy = getattr(self, "_destroy", None)
+        if h and destroy is not None:
+            destroy(h)
             self.h = None
