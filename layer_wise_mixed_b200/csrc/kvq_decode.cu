@@ -74,6 +74,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned phase) {
     return ok != 0;
 }
 // Bounded wait: gives up after ~2^20 polls (each suspends at most ~1 ms).
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned phase) {
     for (int i = 0; i < (1 << 20); ++i)
         if (mbar_try_wait(bar, phase)) return true;
@@ -193,11 +197,9 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t 
     lo = pack_h2(a - ha, b - hb);
 }
 
-// Floats of the per-warp combine buffer: O^T columns [8*NT][D] (zero-point term folded
-// in), running max and sum per head [8] + [8]; plus kCombShared floats shared by the CTA
-// (per-warp merge weights and per-head denominators).
+// Floats of the per-warp combine buffer: the heads' O^T columns (zero-point term and lo
+// parts folded in, at most [8][D + 4]), then running max and sum per head [8] + [8].
 __host__ __device__ constexpr int comb_floats(int D, int NT) { return 8 * NT * D + 16; }
-constexpr int kCombShared = 64;
 
 // Bytes of one unit record: NH 16-token halves of codes, fp16 scales/zeros.
 __host__ __device__ constexpr int unit_bytes(int D, int BK, int BV, int KM, int NH) {
@@ -684,20 +686,40 @@ __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &
         }
     __syncthreads();   // every warp is done with its stages
     constexpr int CF = comb_floats(D, NT);
+    constexpr int DP = D + 4;   // head stride of the buffer: one store's head columns hit distinct banks
     float *base = reinterpret_cast<float *>(smem);
-    float *shared_tail = base + NW * CF;   // wts[NW][8], den[8], M[8]
     {
-        float *ob = base + warp * CF;      // [8*NT][D]
-        float *ml = ob + 8 * NT * D;       // m[8], l[8]
+        // each head's O^T column = hi part + lo part (NT == 2: tile 1; NT == 1: column
+        // head + G, on lane t + G/2 for even G), summed in registers; buffer [G][DP]
+        float *ob = base + warp * CF;
+        float *ml = ob + 8 * NT * D;   // m[8], l[8]
 #pragma unroll
         for (int m = 0; m < KS; ++m)
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                const int d0 = 16 * m + g, c0 = 8 * n + 2 * t;
-                ob[c0 * D + d0] = A.oacc[m][n][0];
-                ob[(c0 + 1) * D + d0] = A.oacc[m][n][1];
-                ob[c0 * D + d0 + 8] = A.oacc[m][n][2];
-                ob[(c0 + 1) * D + d0 + 8] = A.oacc[m][n][3];
+            for (int rh = 0; rh < 2; ++rh) {
+                const int d = 16 * m + g + 8 * rh;
+                const float r0 = A.oacc[m][0][2 * rh], r1 = A.oacc[m][0][2 * rh + 1];   // columns 2t, 2t + 1
+                float v0, v1;
+                if constexpr (NT == 2) {
+                    v0 = r0 + A.oacc[m][NT - 1][2 * rh];
+                    v1 = r1 + A.oacc[m][NT - 1][2 * rh + 1];
+                } else if (G == 1) {
+                    v0 = r0 + r1;
+                    v1 = 0.f;
+                } else if ((G & 1) == 0) {
+                    v0 = r0 + __shfl_down_sync(0xffffffffu, r0, G >> 1);
+                    v1 = r1 + __shfl_down_sync(0xffffffffu, r1, G >> 1);
+                } else {   // G = 3: the lo column's lane and register vary with the column
+                    const int c0 = 2 * t + G, c1 = 2 * t + 1 + G;
+                    const float a0 = __shfl_sync(0xffffffffu, r0, 4 * g + (c0 >> 1));
+                    const float b0 = __shfl_sync(0xffffffffu, r1, 4 * g + (c0 >> 1));
+                    const float a1 = __shfl_sync(0xffffffffu, r0, 4 * g + (c1 >> 1));
+                    const float b1 = __shfl_sync(0xffffffffu, r1, 4 * g + (c1 >> 1));
+                    v0 = r0 + ((c0 & 1) ? b0 : a0);
+                    v1 = r1 + ((c1 & 1) ? b1 : a1);
+                }
+                if (2 * t < G) ob[(2 * t) * DP + d] = v0;
+                if (2 * t + 1 < G) ob[(2 * t + 1) * DP + d] = v1;
             }
         if (t == 0 && g < G) {
             ml[g] = has_data ? A.m_run : -INFINITY;
@@ -705,42 +727,31 @@ __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &
         }
     }
     __syncthreads();
-    if (threadIdx.x < G) {   // per-head merge weights of the warps
-        const int hd = threadIdx.x;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, base[w * CF + 8 * NT * D + hd]);
-        float den = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-            const float mw = base[w * CF + 8 * NT * D + hd];
-            const float wt = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-            shared_tail[w * 8 + hd] = wt;
-            den = fmaf(wt, base[w * CF + 8 * NT * D + 8 + hd], den);
-        }
-        shared_tail[NW * 8 + hd] = den;
-        shared_tail[NW * 8 + 8 + hd] = M;
-    }
-    __syncthreads();
     for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
         const int hd = idx / D, d = idx % D;
-        const int chi = hd, clo = (NT == 1) ? hd + G : 8 + hd;
-        float val = 0.f;
+        // per-head merge weights of the warps (every thread of the head)
+        float mw[NW], M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
-            const float *ob = base + w * CF;
-            val = fmaf(shared_tail[w * 8 + hd], ob[chi * D + d] + ob[clo * D + d], val);
+            mw[w] = base[w * CF + 8 * NT * D + hd];
+            M = fmaxf(M, mw[w]);
         }
-        const float den = shared_tail[NW * 8 + hd];
+        float val = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const float wt = (mw[w] == -INFINITY) ? 0.f : fast_exp2(mw[w] - M);
+            den = fmaf(wt, base[w * CF + 8 * NT * D + 8 + hd], den);
+            val = fmaf(wt, base[w * CF + hd * DP + d], val);
+        }
         const long long row = row0 + hd;
         if (S == 1) {
-            const float o = val / den;
+            const float o = val * __frcp_rn(den);
             if (out_fp32) reinterpret_cast<float *>(out)[row * D + d] = o;
             else reinterpret_cast<__nv_bfloat16 *>(out)[row * D + d] = __float2bfloat16_rn(o);
         } else {
             part_acc[(row * kMaxSplits + sp) * D + d] = val;
             if (d == 0) {
-                part_ml[(row * kMaxSplits + sp) * 2] = shared_tail[NW * 8 + 8 + hd];
+                part_ml[(row * kMaxSplits + sp) * 2] = M;
                 part_ml[(row * kMaxSplits + sp) * 2 + 1] = den;
             }
         }
@@ -757,18 +768,21 @@ struct SmemParts {
 
 __host__ __device__ inline size_t smem_bars_off(int NS, int stage_bytes, int D, int NT) {
     const size_t stage = static_cast<size_t>(NW) * NS * stage_bytes;
-    const size_t comb = (static_cast<size_t>(NW) * comb_floats(D, NT) + kCombShared) * 4;
+    const size_t comb = static_cast<size_t>(NW) * comb_floats(D, NT) * 4;
     return ((stage > comb ? stage : comb) + 127) & ~size_t(127);
 }
 
 // Bytes after the per-lane scalars: a fused append's token codes (values, keys: 2D), the
 // CTA's two scale maxima (16) and the token's fp16 scales/zeros per role and group.
 __host__ __device__ constexpr int append_scratch_bytes(int D) { return 2 * D + 16 + 2 * (D / 32) * 2 * 2; }
+// Then the prologue area: the CTA's q rows (up to 8 heads), the appended token's K and V
+// rows (bf16) and the mbarrier of their bulk copies, issued with the first block copies.
+__host__ __device__ constexpr int prologue_bytes(int D) { return 8 * D * 2 + 2 * D * 2 + 16; }
 
 __host__ __device__ inline size_t smem_total(int NS, int stage_bytes, int D, int NT) {
     const size_t bars = static_cast<size_t>(NW) * NS * 8 + 8 * ((NW * NS) & 1);   // keeps 16-B alignment
     return smem_bars_off(NS, stage_bytes, D, NT) + bars + static_cast<size_t>(D / 16) * 32 * 16 + 32 * 16 +
-           append_scratch_bytes(D);
+           append_scratch_bytes(D) + prologue_bytes(D);
 }
 
 __device__ __forceinline__ SmemParts carve(uint8_t *smem, int NS, int stage_bytes, int D, int NT) {
@@ -810,7 +824,8 @@ __device__ __forceinline__ void or_token(uint32_t *area, int role, int e, const 
 // `scratch`.  own_k / own_v: the CTA's largest new scales.
 template <int BK, int BV, int KM, int D>
 __device__ __forceinline__ void append_token(const DecodeParams &p, long long unit, int blk, int u,
-                                             uint8_t *scratch, float &own_k, float &own_v) {
+                                             uint8_t *scratch, const uint16_t *kn, const uint16_t *vn,
+                                             uint64_t *pro_bar, float &own_k, float &own_v) {
     constexpr int NJ = D / 32;
     constexpr int KC = 4 * D * BK, KSZ = 4 * D, VC = 4 * D * BV;
     constexpr int REC = KC + KSZ + VC + 4 * D;
@@ -822,12 +837,14 @@ __device__ __forceinline__ void append_token(const DecodeParams &p, long long un
     uint16_t *szs = reinterpret_cast<uint16_t *>(scratch + 2 * D + 16);   // [role][j][scale, zero]
     if (threadIdx.x < 2) cmax[threadIdx.x] = 0u;
     __syncthreads();
+    // the token's rows (kn, vn) arrive by bulk copy with the q rows
+    if (!mbar_wait(pro_bar, 0) && (threadIdx.x & 31) == 0) atomicOr(p.status, kStatusWaitExpired);
     constexpr int NROLE = KM == 1 ? 2 : 1;
     for (int it = warp; it < NROLE * NJ; it += NW) {
         const int role = it < NJ ? 1 : 0;
         const int j = it % NJ;
         const int bits = role ? BV : BK;
-        const uint16_t *src = (role ? p.v_new : p.k_new) + unit * D;
+        const uint16_t *src = role ? vn : kn;
         const float x = quant::bf16_to_f32(src[32 * j + lane]);
         float mn = x, mx = x;
 #pragma unroll
@@ -850,7 +867,7 @@ __device__ __forceinline__ void append_token(const DecodeParams &p, long long un
         }
     }
     if constexpr (KM == 0) {
-        const uint32_t *src = reinterpret_cast<const uint32_t *>(p.k_new + unit * D);
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(kn);
         uint32_t *dst = reinterpret_cast<uint32_t *>(p.res_w + (unit * 32 + u) * D);
         for (int i = threadIdx.x; i < D / 2; i += NW * 32) dst[i] = src[i];
     }
@@ -914,6 +931,9 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     const int blk0 = sp * p.bps, blk1 = min(nblk, blk0 + p.bps);
     const int rem = L & 31;
     const int tail_blk = rem ? (L >> 5) : -1;
+    // the layer's scale maxima: loaded first, their latency overlaps the set-up
+    const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
+    const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
 
     const SmemParts sm = carve(smem, NS, REC, D, NT);
     WarpPipe P{sm.stages + static_cast<size_t>(warp) * NS * REC, sm.bars + warp * NS, NS, REC, lane, 0, 0, 0u, 0};
@@ -929,16 +949,39 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
         if (blk == tail_blk) pipe_issue(P, src + VSKIP, REC - VSKIP, VSKIP);
         else pipe_issue(P, src, REC);
     };
-    for (int k = 0; k < NS && k < nb; ++k) issue_block(k);
     // a fused launch appends token L - 1 (the last of block new_blk) in the CTA that holds
     // that block; the block's warp patches its staged copy with the token
     const bool fused = p.k_new != nullptr;
     const int new_blk = (L - 1) >> 5;
     const bool append_here = fused && new_blk >= blk0 && new_blk < blk1;   // CTA-uniform
     uint8_t *append_scratch = reinterpret_cast<uint8_t *>(sm.scal_s + 32);
+    // the prologue copies (the q rows of the kv head's G query heads and, in the CTA that
+    // appends, the token's K and V rows; all 16-byte aligned: rows of 2D bytes) go out
+    // before the block copies, which fill the memory queues for microseconds
+    const long long unit = static_cast<long long>(b) * p.Hkv + h;
+    uint16_t *q_s = reinterpret_cast<uint16_t *>(append_scratch + append_scratch_bytes(D));
+    uint16_t *kn_s = q_s + 8 * D, *vn_s = kn_s + D;
+    uint64_t *pro_bar = reinterpret_cast<uint64_t *>(vn_s + D);
+    if (threadIdx.x == 0) {
+        mbar_init(pro_bar, 1);
+        fence_mbar_init();
+        const unsigned qbytes = static_cast<unsigned>(G * D * 2);
+        mbar_expect_tx(pro_bar, qbytes + (append_here ? 4 * D : 0));
+        bulk_g2s(q_s, p.q + unit * G * D, qbytes, pro_bar);
+        if (append_here) {
+            bulk_g2s(kn_s, p.k_new + unit * D, 2 * D, pro_bar);
+            bulk_g2s(vn_s, p.v_new + unit * D, 2 * D, pro_bar);
+        }
+    }
+    if constexpr (KM == 0) {
+        // the bf16 residual rows of the tail block: into L2 now, read after the tail's copy
+        if (p.res && tail_blk >= blk0 && tail_blk < blk1 && ((tail_blk - blk0) % NW) == warp) {
+            const char *r = reinterpret_cast<const char *>(p.res + unit * 32 * D);
+            for (int i = lane; i < rem * D * 2 / 128; i += 32) prefetch_l2(r + i * 128);
+        }
+    }
+    for (int k = 0; k < NS && k < nb; ++k) issue_block(k);
 
-    const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
-    const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
     if (fused && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) {
         atomicMax(p.smax_out, p.smax[0]);   // carry the old length's maxima forward
         atomicMax(p.smax_out + 1, p.smax[1]);
@@ -949,12 +992,12 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     // the key prescale needs no new scale (a token that completes a per-channel key group
     // is never fused; per-token keys are scaled in fp32), so warp 0 sets up q first and
     // its loads overlap the append
-    setup_query<KM, D>(p.q + (static_cast<long long>(b) * p.Hkv * G + h * G + hh) * D, smax_k, sm.aq_s, sm.scal_s,
-                       c, warp);
+    if (warp == 0 && !mbar_wait(pro_bar, 0) && lane == 0) atomicOr(p.status, kStatusWaitExpired);
+    setup_query<KM, D>(q_s + hh * D, smax_k, sm.aq_s, sm.scal_s, c, warp);
     if (append_here) {
         float own_k, own_v;
-        append_token<BK, BV, KM, D>(p, static_cast<long long>(b) * p.Hkv + h, new_blk, (L - 1) & 31,
-                                    append_scratch, own_k, own_v);
+        append_token<BK, BV, KM, D>(p, unit, new_blk, (L - 1) & 31, append_scratch, kn_s, vn_s, pro_bar, own_k,
+                                    own_v);
         c.pbias = value_bias(fmaxf(smax_v, own_v));   // CTA-uniform: every warp's p carries it
     }
     __syncthreads();
@@ -1183,7 +1226,8 @@ KernelFn pick_kernel(int D, int bk, int bv, int kmode, int G) {
 // G <= 4, else 3) share the SM's 228 KB of shared memory; at least 2 (fewer CTAs then
 // fit), at most 6.
 int decode_stages(long long rec_bytes, int D, int G) {
-    const long long fixed = 1024 + (D / 16) * 32 * 16 + 64;   // per-CTA reserve, q fragments, barriers
+    // per-CTA reserve, q fragments, barriers, prologue
+    const long long fixed = 1024 + (D / 16) * 32 * 16 + 64 + prologue_bytes(D);
     for (int ctas = (G <= 4 ? 4 : 3); ctas >= 1; --ctas) {
         const long long ns = (228LL * 1024 / ctas - fixed) / (NW * rec_bytes);
         if (ns >= 2) return static_cast<int>(ns > 6 ? 6 : ns);
