@@ -727,29 +727,43 @@ __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &
         }
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
-        const int hd = idx / D, d = idx % D;
-        // per-head merge weights of the warps (every thread of the head)
+    // outputs in groups of 4 channels of one head (16-byte smem reads and global stores);
+    // the warps' merge weights once per group
+    for (int i4 = threadIdx.x; i4 < G * D / 4; i4 += NW * 32) {
+        const int hd = (4 * i4) / D, d = (4 * i4) % D;
         float mw[NW], M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
             mw[w] = base[w * CF + 8 * NT * D + hd];
             M = fmaxf(M, mw[w]);
         }
-        float val = 0.f, den = 0.f;
+        float den = 0.f;
+        float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
             const float wt = (mw[w] == -INFINITY) ? 0.f : fast_exp2(mw[w] - M);
             den = fmaf(wt, base[w * CF + 8 * NT * D + 8 + hd], den);
-            val = fmaf(wt, base[w * CF + hd * DP + d], val);
+            const float4 o = *reinterpret_cast<const float4 *>(base + w * CF + hd * DP + d);
+            val.x = fmaf(wt, o.x, val.x);
+            val.y = fmaf(wt, o.y, val.y);
+            val.z = fmaf(wt, o.z, val.z);
+            val.w = fmaf(wt, o.w, val.w);
         }
         const long long row = row0 + hd;
         if (S == 1) {
-            const float o = val * __frcp_rn(den);
-            if (out_fp32) reinterpret_cast<float *>(out)[row * D + d] = o;
-            else reinterpret_cast<__nv_bfloat16 *>(out)[row * D + d] = __float2bfloat16_rn(o);
+            const float r = __frcp_rn(den);
+            const float4 o = make_float4(val.x * r, val.y * r, val.z * r, val.w * r);
+            if (out_fp32) {
+                *reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + row * D + d) = o;
+            } else {
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y), hi = __floats2bfloat162_rn(o.z, o.w);
+                uint2 u;
+                u.x = *reinterpret_cast<const uint32_t *>(&lo);
+                u.y = *reinterpret_cast<const uint32_t *>(&hi);
+                *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(out) + row * D + d) = u;
+            }
         } else {
-            part_acc[(row * kMaxSplits + sp) * D + d] = val;
+            *reinterpret_cast<float4 *>(part_acc + (row * kMaxSplits + sp) * D + d) = val;
             if (d == 0) {
                 part_ml[(row * kMaxSplits + sp) * 2] = M;
                 part_ml[(row * kMaxSplits + sp) * 2 + 1] = den;
