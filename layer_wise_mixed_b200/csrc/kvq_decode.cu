@@ -197,9 +197,9 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t 
     lo = pack_h2(a - ha, b - hb);
 }
 
-// Floats of the per-warp combine buffer: the heads' O^T columns (zero-point term and lo
-// parts folded in, at most [8][D + 4]), then running max and sum per head [8] + [8].
-__host__ __device__ constexpr int comb_floats(int D, int NT) { return 8 * NT * D + 16; }
+// Floats of the per-warp combine buffer: O^T columns [8 NT][D + 4], value zero-point
+// terms [D/32][8 NT], running max and sum per head [8] + [8].
+__host__ __device__ constexpr int comb_floats(int D, int NT) { return 8 * NT * (D + 4) + (D / 32) * 8 * NT + 16; }
 
 // Bytes of one unit record: NH 16-token halves of codes, fp16 scales/zeros.
 __host__ __device__ constexpr int unit_bytes(int D, int BK, int BV, int KM, int NH) {
@@ -671,56 +671,33 @@ __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &
     float l_run = A.l_run;
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-    // fold the value zero-point term of channel group j (held by lane 4j + t) into the
-    // O^T columns of the channels of that group
-#pragma unroll
-    for (int m = 0; m < KS; ++m)
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const float z0 = __shfl_sync(0xffffffffu, A.zc[n][0], 4 * (m >> 1) + t);
-            const float z1 = __shfl_sync(0xffffffffu, A.zc[n][1], 4 * (m >> 1) + t);
-            A.oacc[m][n][0] += z0;
-            A.oacc[m][n][2] += z0;
-            A.oacc[m][n][1] += z1;
-            A.oacc[m][n][3] += z1;
-        }
     __syncthreads();   // every warp is done with its stages
-    constexpr int CF = comb_floats(D, NT);
-    constexpr int DP = D + 4;   // head stride of the buffer: one store's head columns hit distinct banks
+    // each warp's O^T columns (hi and lo parts, [8 NT][DP]: a store's 32 lanes hit 32
+    // banks), its value zero-point terms ([NJ][8 NT]: row j = channel group, on lanes
+    // g = j) and per-head m, l; hi + lo + zero term are added while merging
+    constexpr int CF = comb_floats(D, NT), DP = D + 4, NJ = D / 32;
     float *base = reinterpret_cast<float *>(smem);
     {
-        // each head's O^T column = hi part + lo part (NT == 2: tile 1; NT == 1: column
-        // head + G, on lane t + G/2 for even G), summed in registers; buffer [G][DP]
         float *ob = base + warp * CF;
-        float *ml = ob + 8 * NT * D;   // m[8], l[8]
+        float *zb = ob + 8 * NT * DP;
+        float *ml = zb + NJ * 8 * NT;
 #pragma unroll
         for (int m = 0; m < KS; ++m)
 #pragma unroll
-            for (int rh = 0; rh < 2; ++rh) {
-                const int d = 16 * m + g + 8 * rh;
-                const float r0 = A.oacc[m][0][2 * rh], r1 = A.oacc[m][0][2 * rh + 1];   // columns 2t, 2t + 1
-                float v0, v1;
-                if constexpr (NT == 2) {
-                    v0 = r0 + A.oacc[m][NT - 1][2 * rh];
-                    v1 = r1 + A.oacc[m][NT - 1][2 * rh + 1];
-                } else if (G == 1) {
-                    v0 = r0 + r1;
-                    v1 = 0.f;
-                } else if ((G & 1) == 0) {
-                    v0 = r0 + __shfl_down_sync(0xffffffffu, r0, G >> 1);
-                    v1 = r1 + __shfl_down_sync(0xffffffffu, r1, G >> 1);
-                } else {   // G = 3: the lo column's lane and register vary with the column
-                    const int c0 = 2 * t + G, c1 = 2 * t + 1 + G;
-                    const float a0 = __shfl_sync(0xffffffffu, r0, 4 * g + (c0 >> 1));
-                    const float b0 = __shfl_sync(0xffffffffu, r1, 4 * g + (c0 >> 1));
-                    const float a1 = __shfl_sync(0xffffffffu, r0, 4 * g + (c1 >> 1));
-                    const float b1 = __shfl_sync(0xffffffffu, r1, 4 * g + (c1 >> 1));
-                    v0 = r0 + ((c0 & 1) ? b0 : a0);
-                    v1 = r1 + ((c1 & 1) ? b1 : a1);
-                }
-                if (2 * t < G) ob[(2 * t) * DP + d] = v0;
-                if (2 * t + 1 < G) ob[(2 * t + 1) * DP + d] = v1;
+            for (int n = 0; n < NT; ++n) {
+                const int d0 = 16 * m + g, c0 = 8 * n + 2 * t;
+                ob[c0 * DP + d0] = A.oacc[m][n][0];
+                ob[(c0 + 1) * DP + d0] = A.oacc[m][n][1];
+                ob[c0 * DP + d0 + 8] = A.oacc[m][n][2];
+                ob[(c0 + 1) * DP + d0 + 8] = A.oacc[m][n][3];
             }
+        if (g < NJ) {
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                zb[g * 8 * NT + 8 * n + 2 * t] = A.zc[n][0];
+                zb[g * 8 * NT + 8 * n + 2 * t + 1] = A.zc[n][1];
+            }
+        }
         if (t == 0 && g < G) {
             ml[g] = has_data ? A.m_run : -INFINITY;
             ml[8 + g] = l_run;
@@ -731,23 +708,29 @@ __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &
     // the warps' merge weights once per group
     for (int i4 = threadIdx.x; i4 < G * D / 4; i4 += NW * 32) {
         const int hd = (4 * i4) / D, d = (4 * i4) % D;
+        const int chi = hd, clo = (NT == 1) ? hd + G : 8 + hd, j = d >> 5;
+        constexpr int MLO = 8 * NT * DP + NJ * 8 * NT;   // m, l offset in a warp's buffer
         float mw[NW], M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
-            mw[w] = base[w * CF + 8 * NT * D + hd];
+            mw[w] = base[w * CF + MLO + hd];
             M = fmaxf(M, mw[w]);
         }
         float den = 0.f;
         float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
+            const float *ob = base + w * CF;
+            const float *zb = ob + 8 * NT * DP;
             const float wt = (mw[w] == -INFINITY) ? 0.f : fast_exp2(mw[w] - M);
-            den = fmaf(wt, base[w * CF + 8 * NT * D + 8 + hd], den);
-            const float4 o = *reinterpret_cast<const float4 *>(base + w * CF + hd * DP + d);
-            val.x = fmaf(wt, o.x, val.x);
-            val.y = fmaf(wt, o.y, val.y);
-            val.z = fmaf(wt, o.z, val.z);
-            val.w = fmaf(wt, o.w, val.w);
+            den = fmaf(wt, ob[MLO + 8 + hd], den);
+            const float4 oh = *reinterpret_cast<const float4 *>(ob + chi * DP + d);
+            const float4 ol = *reinterpret_cast<const float4 *>(ob + clo * DP + d);
+            const float z = zb[j * 8 * NT + chi] + zb[j * 8 * NT + clo];
+            val.x = fmaf(wt, oh.x + ol.x + z, val.x);
+            val.y = fmaf(wt, oh.y + ol.y + z, val.y);
+            val.z = fmaf(wt, oh.z + ol.z + z, val.z);
+            val.w = fmaf(wt, oh.w + ol.w + z, val.w);
         }
         const long long row = row0 + hd;
         if (S == 1) {
@@ -945,9 +928,9 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     const int blk0 = sp * p.bps, blk1 = min(nblk, blk0 + p.bps);
     const int rem = L & 31;
     const int tail_blk = rem ? (L >> 5) : -1;
-    // the layer's scale maxima: loaded first, their latency overlaps the set-up
-    const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
-    const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
+    // the layer's scale maxima: loaded first (converted at first use), their latency
+    // overlaps the set-up
+    const unsigned smax_bits_k = p.smax[0], smax_bits_v = p.smax[1];
 
     const SmemParts sm = carve(smem, NS, REC, D, NT);
     WarpPipe P{sm.stages + static_cast<size_t>(warp) * NS * REC, sm.bars + warp * NS, NS, REC, lane, 0, 0, 0u, 0};
@@ -996,9 +979,11 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     }
     for (int k = 0; k < NS && k < nb; ++k) issue_block(k);
 
+    const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(smax_bits_k)));
+    const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(smax_bits_v)));
     if (fused && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) {
-        atomicMax(p.smax_out, p.smax[0]);   // carry the old length's maxima forward
-        atomicMax(p.smax_out + 1, p.smax[1]);
+        atomicMax(p.smax_out, smax_bits_k);   // carry the old length's maxima forward
+        atomicMax(p.smax_out + 1, smax_bits_v);
     }
     BodyCtx c = make_ctx<KM, D, NT>(lane, G, smax_v, sm.aq_s);
     c.res = p.res ? p.res + (static_cast<long long>(b) * p.Hkv + h) * 32 * D : nullptr;
