@@ -4,7 +4,8 @@ A step = one decode token for every sequence of the batch through every layer: p
 layer, the new token's K/V is quantized and packed into the cache and decode attention
 runs over it -- kvq_append_decode, one launch (a token that completes a per-channel key
 group: kvq_append, then kvq_decode_attn; paged plans: kvq_append_tagged, then
-kvq_decode_attn), plus the log-sum-exp merge when the sequence is split.  Each step of
+kvq_decode_attn), plus the log-sum-exp merge launch when a sequence is split in two or
+three (from four splits the decode launch merges its own partials).  Each step of
 the decode schedule is captured once into a CUDA graph (untimed); the timed region
 replays K graphs.  The dominant kernel's roofline comes from decode-only replays of the
 same schedule.  Inputs are seeded synthetic tensors already resident in HBM; one step reads
@@ -399,10 +400,10 @@ def main():
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
     # per layer and step: one fused append + decode launch, or (a token that completes a
     # per-channel key group; paged plans) an append and a decode launch; plus the merge
-    # launch when the sequence is split
+    # launch for two or three splits
     def step_launches(s, l):
         two = paged or (wl.kmode == 0 and Ls[s] % 32 == 0)
-        return (2 if two else 1) + (1 if splits[s][l] > 1 else 0)
+        return (2 if two else 1) + (1 if 1 < splits[s][l] < 4 else 0)
     gpu_launches = sum(step_launches(s, l) for s in order for l in range(NL))
     e2e_note = ("per step: pinned H2D of all layers' K/V/q, kvq_append_decode per layer (eager "
                 "C-ABI calls), D2H of all layers' outputs")
@@ -475,7 +476,7 @@ def main():
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                              "frac": achieved / peak,
                              "traffic": captured_traffic(wl.name, dec_bytes / launches_dec),
-                             "kernel": ("decode_paged_kernel" if wl.paged else "decode_split_kernel") + " (+merge)",
+                             "kernel": "decode_paged_kernel" if wl.paged else "decode_split_kernel",
                              "peak_source": peak_src, "avg_launch_us": 1e3 * dec_ms / launches_dec,
                              "algorithmic_bytes_per_launch": dec_bytes / launches_dec},
                 "cpu_baseline": cpu,

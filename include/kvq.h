@@ -113,7 +113,7 @@ typedef struct kvq_handle kvq_handle;
 KVQ_API int kvq_plan(const kvq_plan_desc *desc, kvq_handle **out);
 
 /* Device workspace size the plan needs: all layers' cache regions, the split
- * partials and a status word. */
+ * partials, split arrival counters and a status word. */
 KVQ_API int kvq_workspace_bytes(const kvq_handle *h, size_t *bytes);
 
 /* Bind caller-owned device memory (>= kvq_workspace_bytes, 256-byte aligned) and
@@ -144,8 +144,9 @@ KVQ_API int kvq_append_tagged(kvq_handle *h, int layer, const void *K, const voi
 
 /* Decode attention of one query token per sequence over all L tokens of `layer`:
  * q bf16 [B][Hq][D] (device); out [B][Hq][D] (device) bf16, or fp32 if out_fp32.
- * Launches the split kernel and, when the sequence is split, the log-sum-exp merge
- * kernel.  Requires L >= 1. */
+ * One kernel launch.  A sequence split in two or three parts adds a log-sum-exp merge
+ * launch; from four splits the last CTA of each (batch, kv head) to finish merges the
+ * partials inside the decode launch.  Requires L >= 1. */
 KVQ_API int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_fp32,
                     void *stream);
 

@@ -24,7 +24,8 @@
 // m16n8k16 (fp16 in, fp32 accumulate) does both contractions; online softmax in
 // base 2.  The last block of a per-channel layer takes its keys from the bf16
 // residual.  Warps are combined in shared memory; one split writes the output
-// directly, several write fp32 partials for the merge kernel.
+// directly, several write fp32 partials that the (batch, kv head)'s last CTA to finish
+// merges by log-sum-exp.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -661,11 +662,13 @@ __device__ __forceinline__ void pipe_drain(WarpPipe &P, int from) {
     for (int k = from; k < P.issued; ++k) mbar_wait(&P.bars[k % P.NS], (k / P.NS) & 1);
 }
 
-// Combine the CTA's warps and store either the output (one split) or the split partial.
+// Combine the CTA's warps and store either the output (one split) or the split partial;
+// with several splits and a counter `arrive`, the unit's last CTA to arrive (it resets
+// the counter) merges the S partials by log-sum-exp and stores the output.
 template <int D, int NT>
 __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &c, bool has_data, uint8_t *smem,
                                               int warp, long long row0, int sp, int S, int out_fp32, void *out,
-                                              float *part_acc, float *part_ml) {
+                                              float *part_acc, float *part_ml, unsigned *arrive) {
     constexpr int KS = D / 16;
     const int g = c.g, t = c.t, G = c.G;
     float l_run = A.l_run;
@@ -753,6 +756,50 @@ __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &
             }
         }
     }
+    if (S == 1 || arrive == nullptr) return;
+    // split partials: the CTA's stores precede (barrier) thread 0's release-acquire count
+    // of the arrival; the last CTA merges (no CTA waits for another)
+    __shared__ int s_last;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned prev;
+        asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(prev) : "l"(arrive) : "memory");
+        s_last = prev == static_cast<unsigned>(S - 1);
+    }
+    __syncthreads();
+    if (!s_last) return;
+    for (int i4 = threadIdx.x; i4 < G * D / 4; i4 += NW * 32) {
+        const int hd = (4 * i4) / D, d = (4 * i4) % D;
+        const long long row = row0 + hd;
+        const float *ml = part_ml + row * kMaxSplits * 2;
+        float M = -INFINITY;
+        for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(ml + 2 * s));
+        float den = 0.f;
+        float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < S; ++s) {
+            const float ms = __ldcg(ml + 2 * s);
+            if (ms == -INFINITY) continue;
+            const float wt = fast_exp2(ms - M);
+            den = fmaf(wt, __ldcg(ml + 2 * s + 1), den);
+            const float4 a = __ldcg(reinterpret_cast<const float4 *>(part_acc + (row * kMaxSplits + s) * D + d));
+            val.x = fmaf(wt, a.x, val.x);
+            val.y = fmaf(wt, a.y, val.y);
+            val.z = fmaf(wt, a.z, val.z);
+            val.w = fmaf(wt, a.w, val.w);
+        }
+        const float r = __frcp_rn(den);
+        const float4 o = make_float4(val.x * r, val.y * r, val.z * r, val.w * r);
+        if (out_fp32) {
+            *reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + row * D + d) = o;
+        } else {
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y), hi = __floats2bfloat162_rn(o.z, o.w);
+            uint2 u;
+            u.x = *reinterpret_cast<const uint32_t *>(&lo);
+            u.y = *reinterpret_cast<const uint32_t *>(&hi);
+            *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(out) + row * D + d) = u;
+        }
+    }
+    if (threadIdx.x == 0) *arrive = 0u;   // ready for the next launch
 }
 
 // Shared-memory carve-up: [stages | combine buffer][barriers][q fragments].
@@ -1049,7 +1096,7 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
         if (lane == 0) atomicOr(p.status, kStatusWaitExpired);
     }
     combine_store<D, NT>(A, c, nb > 0 && !failed, smem, warp, static_cast<long long>(b) * p.Hkv * G + h * G, sp,
-                         p.S, p.out_fp32, p.out, p.part_acc, p.part_ml);
+                         p.S, p.out_fp32, p.out, p.part_acc, p.part_ml, p.arrive ? p.arrive + unit : nullptr);
 }
 
 // ------------------------------------------------------------------ paged kernel
@@ -1157,7 +1204,8 @@ __device__ __forceinline__ void paged_body(const PagedDecodeParams &p, uint8_t *
         if (lane == 0) atomicOr(p.status, kStatusWaitExpired);
     }
     combine_store<D, NT>(A, c, nb > 0 && !failed, smem, warp, static_cast<long long>(b) * p.Hkv * G + h * G, sp,
-                         p.S2 + p.S4, p.out_fp32, p.out, p.part_acc, p.part_ml);
+                         p.S2 + p.S4, p.out_fp32, p.out, p.part_acc, p.part_ml,
+                         p.arrive ? p.arrive + static_cast<long long>(b) * p.Hkv + h : nullptr);
 }
 
 __global__ void __launch_bounds__(NW * 32, 4) decode_paged_kernel(const PagedDecodeParams p) {
@@ -1169,7 +1217,8 @@ __global__ void __launch_bounds__(NW * 32, 4) decode_paged_kernel(const PagedDec
     else paged_body<false>(p, smem, warp, lane, b, h, sp);
 }
 
-// Log-sum-exp merge of the split partials ("merged by online log-sum-exp").
+// Log-sum-exp merge of the split partials ("merged by online log-sum-exp"), for split
+// counts below kInLaunchMergeSplits.
 __global__ void merge_kernel(const MergeParams p) {
     pdl_enter();
     const long long row = blockIdx.x;   // b * Hq + hq
@@ -1185,7 +1234,7 @@ __global__ void merge_kernel(const MergeParams p) {
             val = fmaf(wt, p.part_acc[(row * kMaxSplits + s) * p.D + d], val);
             den = fmaf(wt, ml[2 * s + 1], den);
         }
-        const float o = val / den;
+        const float o = val * __frcp_rn(den);
         if (p.out_fp32) reinterpret_cast<float *>(p.out)[row * p.D + d] = o;
         else reinterpret_cast<__nv_bfloat16 *>(p.out)[row * p.D + d] = __float2bfloat16_rn(o);
     }
@@ -1319,6 +1368,11 @@ cudaError_t decode_paged_occupancy(int nstage, int *ctas_per_sm) {
     return prepare_kernel(reinterpret_cast<const void *>(decode_paged_kernel), decode_paged_smem_bytes(nstage), ctas_per_sm);
 }
 
+cudaError_t launch_merge(const MergeParams &p, cudaStream_t st) {
+    cudaError_t e = launch_pdl(merge_kernel, dim3(p.B * p.Hq), dim3(p.D), 0, st, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 cudaError_t launch_decode_paged(const PagedDecodeParams &p, cudaStream_t st) {
     const size_t smem = decode_paged_smem_bytes(p.nstage);
     cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(decode_paged_kernel), smem, nullptr);
@@ -1328,9 +1382,5 @@ cudaError_t launch_decode_paged(const PagedDecodeParams &p, cudaStream_t st) {
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_merge(const MergeParams &p, cudaStream_t st) {
-    cudaError_t e = launch_pdl(merge_kernel, dim3(p.B * p.Hq), dim3(p.D), 0, st, p);
-    return e != cudaSuccess ? e : cudaGetLastError();
-}
 
 }  // namespace kvq

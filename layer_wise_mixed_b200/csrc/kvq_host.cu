@@ -22,7 +22,8 @@ struct kvq_handle {
     std::vector<LayerGeom> geom;
     std::vector<int> len;
     int cap_blk = 0;
-    long long status_off = 0, smax_off = 0, meta_bytes = 0, part_acc_off = 0, part_ml_off = 0, total = 0;
+    long long status_off = 0, smax_off = 0, arrive_off = 0, meta_bytes = 0, part_acc_off = 0, part_ml_off = 0,
+              total = 0;
     uint8_t *ws = nullptr;
     size_t ws_bytes = 0;
     int forced_splits = 0;
@@ -109,7 +110,8 @@ int cuda_fail(cudaError_t e, const char *what) {
 // than `occ` an SM is not full and the CTAs' own latency decides.  A CTA costs its
 // blocks per warp plus about two blocks of fixed latency (first copy, q set-up,
 // combine); with a single stage per warp the copy latency of every block after the
-// first is exposed too (about 0.6 of a block each).  Splitting adds the merge launch.
+// first is exposed too (about 0.6 of a block each).  Splitting adds the partial writes and
+// the merge by each unit's last CTA.
 double decode_cost(int units, int nblk, int S, int nstage, int occ, int sms) {
     const int bps = (nblk + S - 1) / S;
     const int sreal = (nblk + bps - 1) / bps;
@@ -168,10 +170,11 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
         h->n4_cap = h->n4_main_cap + 2LL * d->batch;
         h->P_cap = (d->max_ctx + 31) / 32 + (d->max_ctx + 15) / 16 + 1;
         h->inv_stride = d->max_ctx;
-        long long off = align256(256 + 16LL * d->num_layers);
-        h->meta_bytes = off;
         h->status_off = 0;
         h->smax_off = 256;
+        h->arrive_off = align256(256 + 16LL * d->num_layers);
+        h->meta_bytes = align256(h->arrive_off + 4LL * d->batch * d->n_kv_heads);
+        long long off = h->meta_bytes;
         for (int l = 0; l < d->num_layers; ++l) {
             h->pool2_off.push_back(off);
             off = align256(off + h->n2_cap * h->rec2_bytes * d->n_kv_heads);
@@ -209,8 +212,9 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
     h->cap_blk = (d->max_ctx + 31) / 32;
     const int D = d->head_dim;
     h->status_off = 0;
-    h->smax_off = 256;                                       // after the status word
-    h->meta_bytes = align256(256 + 16LL * d->num_layers);   // {K, V} max scale per layer and parity
+    h->smax_off = 256;                                             // after the status word
+    h->arrive_off = align256(256 + 16LL * d->num_layers);         // {K, V} max scale per layer and parity
+    h->meta_bytes = align256(h->arrive_off + 4LL * d->batch * d->n_kv_heads);   // split arrival counters
     long long off = h->meta_bytes;
     for (int l = 0; l < d->num_layers; ++l) {
         const kvq_layer_cfg &c = h->cfg[l];
@@ -569,12 +573,13 @@ static int decode_paged(kvq_handle *h, int layer, const void *q, void *out, int 
     p.G = h->desc.n_q_heads / h->desc.n_kv_heads;
     p.S2 = S2;
     p.S4 = S4;
+    p.arrive = S2 + S4 >= kvq::kInLaunchMergeSplits ? reinterpret_cast<unsigned *>(h->ws + h->arrive_off) : nullptr;
     p.out_fp32 = out_fp32 ? 1 : 0;
     p.nstage = kvq::decode_paged_stages();
     if ((rc = prepare_status(h, st))) return rc;
     cudaError_t e = kvq::launch_decode_paged(p, st);
     if (e != cudaSuccess) return cuda_fail(e, "paged decode launch");
-    if (S2 + S4 > 1) {
+    if (S2 + S4 > 1 && !p.arrive) {
         kvq::MergeParams m{};
         m.part_acc = part_acc;
         m.part_ml = part_ml;
@@ -625,11 +630,12 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
     p.out_fp32 = out_fp32 ? 1 : 0;
     p.nstage = nstage;
     p.rec_bytes = g.rec_bytes;
+    p.arrive = p.S >= kvq::kInLaunchMergeSplits ? reinterpret_cast<unsigned *>(h->ws + h->arrive_off) : nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = prepare_status(h, st))) return rc;
     cudaError_t e = kvq::launch_decode(p, h->desc.head_dim, g.bk, g.bv, g.kmode, st, nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-    if (p.S > 1) {
+    if (p.S > 1 && !p.arrive) {
         kvq::MergeParams m{};
         m.part_acc = p.part_acc;
         m.part_ml = p.part_ml;
@@ -690,6 +696,7 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
     p.out_fp32 = out_fp32 ? 1 : 0;
     p.nstage = nstage;
     p.rec_bytes = g.rec_bytes;
+    p.arrive = p.S >= kvq::kInLaunchMergeSplits ? reinterpret_cast<unsigned *>(h->ws + h->arrive_off) : nullptr;
     p.k_new = static_cast<const uint16_t *>(K);
     p.v_new = static_cast<const uint16_t *>(V);
     p.rec_w = h->ws + g.rec_off;
@@ -705,7 +712,7 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
         h->len[layer] = L_old;
         return cuda_fail(e, "fused append + decode launch");
     }
-    if (p.S > 1) {
+    if (p.S > 1 && !p.arrive) {
         kvq::MergeParams m{};
         m.part_acc = p.part_acc;
         m.part_ml = p.part_ml;
@@ -997,11 +1004,12 @@ int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, 
     p.out_fp32 = out_fp32 ? 1 : 0;
     p.nstage = nstage;
     p.rec_bytes = g.rec_bytes;
+    p.arrive = p.S >= kvq::kInLaunchMergeSplits ? reinterpret_cast<unsigned *>(h->ws + h->arrive_off) : nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = prepare_status(h, st))) return rc;
     cudaError_t e = kvq::launch_decode(p, h->desc.head_dim, g.bk, g.bv, g.kmode, st, nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-    if (p.S > 1) {
+    if (p.S > 1 && !p.arrive) {
         kvq::MergeParams m{};
         m.part_acc = p.part_acc;
         m.part_ml = p.part_ml;

@@ -73,6 +73,8 @@ struct DecodeParams {
     void *out;                  // [B][Hq][D] bf16 or fp32
     float *part_acc;            // [B][Hq][kMaxSplits][D]
     float *part_ml;             // [B][Hq][kMaxSplits][2]  (m in log2 units, l)
+    unsigned *arrive;           // [B][Hkv] split arrival counters (zero between launches), or null:
+                                // split partials merged by merge_kernel
     unsigned *status;
     int B, Hkv, G, L, cap_blk, S, bps, out_fp32, nstage;
     long long rec_bytes;
@@ -106,6 +108,7 @@ struct PagedDecodeParams {
     const unsigned *smax;
     void *out;
     float *part_acc, *part_ml;
+    unsigned *arrive;           // as in DecodeParams
     unsigned *status;
     int B, Hkv, G, S2, S4, out_fp32, nstage;
 };
@@ -143,6 +146,12 @@ struct MergeParams {
     void *out;
     int B, Hq, D, S, out_fp32;
 };
+
+// Split counts from which the decode launch merges its own partials (the last CTA of a
+// (batch, kv head) to finish); below, merge_kernel follows.  Measured on one B200: two or
+// three splits are faster with the separate launch (every CTA's arrival costs a global
+// round trip at its exit), nine (the paged 32K-context workload) with the in-launch merge.
+constexpr int kInLaunchMergeSplits = 4;
 
 cudaError_t launch_append(const AppendParams &p, cudaStream_t st);
 // Returns cudaErrorInvalidValue if no kernel exists for the combination.

@@ -97,3 +97,10 @@ def test_fused_matches_two_launches():
         assert np.array_equal(a.export_layer(0), b.export_layer(0)), L
         d = (oa - ob).double().abs().max().item()
         assert d <= 1e-4, (L, d)
+
+
+@pytest.mark.parametrize("kmode", [0, 1])
+def test_fused_in_launch_merge(kmode):
+    """Five splits: the split partials are merged by the last CTA of each (b, kv head)
+    inside the fused launch, step after step (the arrival counters reset themselves)."""
+    run_fused(2, 2, 4, 128, (4, 2), kmode, 150, 40, [151, 160, 161, 175, 190], splits=5, tag=f"merge{kmode}")

@@ -67,6 +67,7 @@ def test_workspace_layout(lib):
         rec1 = 4 * D * 8 + 4 * D + 4 * D * 8 + 4 * D
         al = lambda x: (x + 255) // 256 * 256
         expect = al(256 + 16 * 2)                      # status word + {K, V} max scale per layer and parity
+        expect = al(expect + 4 * B * Hkv)               # split arrival counters per (b, kv head)
         expect = al(expect + rec0 * cap * B * Hkv)
         expect = al(expect + 64 * D * B * Hkv)          # residual of the per-channel layer
         expect = al(expect + rec1 * cap * B * Hkv)
