@@ -810,8 +810,9 @@ struct SmemParts {
     float4 *scal_s;
 };
 
-__host__ __device__ inline size_t smem_bars_off(int NS, int stage_bytes, int D, int NT) {
-    const size_t stage = static_cast<size_t>(NW) * NS * stage_bytes;
+// PS: the CTA's stages (all warps).
+__host__ __device__ inline size_t smem_bars_off(int PS, int stage_bytes, int D, int NT) {
+    const size_t stage = static_cast<size_t>(PS) * stage_bytes;
     const size_t comb = static_cast<size_t>(NW) * comb_floats(D, NT) * 4;
     return ((stage > comb ? stage : comb) + 127) & ~size_t(127);
 }
@@ -823,18 +824,18 @@ __host__ __device__ constexpr int append_scratch_bytes(int D) { return 2 * D + 1
 // rows (bf16) and the mbarrier of their bulk copies, issued with the first block copies.
 __host__ __device__ constexpr int prologue_bytes(int D) { return 8 * D * 2 + 2 * D * 2 + 16; }
 
-__host__ __device__ inline size_t smem_total(int NS, int stage_bytes, int D, int NT) {
-    const size_t bars = static_cast<size_t>(NW) * NS * 8 + 8 * ((NW * NS) & 1);   // keeps 16-B alignment
-    return smem_bars_off(NS, stage_bytes, D, NT) + bars + static_cast<size_t>(D / 16) * 32 * 16 + 32 * 16 +
+__host__ __device__ inline size_t smem_total(int PS, int stage_bytes, int D, int NT) {
+    const size_t bars = static_cast<size_t>(PS) * 8 + 8 * (PS & 1);   // keeps 16-B alignment
+    return smem_bars_off(PS, stage_bytes, D, NT) + bars + static_cast<size_t>(D / 16) * 32 * 16 + 32 * 16 +
            append_scratch_bytes(D) + prologue_bytes(D);
 }
 
-__device__ __forceinline__ SmemParts carve(uint8_t *smem, int NS, int stage_bytes, int D, int NT) {
+__device__ __forceinline__ SmemParts carve(uint8_t *smem, int PS, int stage_bytes, int D, int NT) {
     SmemParts s;
     s.stages = smem;
-    const size_t bo = smem_bars_off(NS, stage_bytes, D, NT);
+    const size_t bo = smem_bars_off(PS, stage_bytes, D, NT);
     s.bars = reinterpret_cast<uint64_t *>(smem + bo);
-    s.aq_s = reinterpret_cast<uint4 *>(smem + bo + static_cast<size_t>(NW) * NS * 8 + 8 * ((NW * NS) & 1));
+    s.aq_s = reinterpret_cast<uint4 *>(smem + bo + static_cast<size_t>(PS) * 8 + 8 * (PS & 1));
     s.scal_s = reinterpret_cast<float4 *>(s.aq_s + (D / 16) * 32);
     return s;
 }
@@ -970,7 +971,10 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.z, h = blockIdx.y, sp = blockIdx.x;
-    const int G = p.G, L = p.L, NS = p.nstage;
+    const int G = p.G, L = p.L;
+    // nstage stages per warp, one more for warps 0 .. nextra - 1 (those with the most blocks)
+    const int NS = p.nstage + (warp < p.nextra ? 1 : 0);
+    const int sbase = warp * p.nstage + min(warp, p.nextra);
     const int nblk = (L + 31) >> 5;
     const int blk0 = sp * p.bps, blk1 = min(nblk, blk0 + p.bps);
     const int rem = L & 31;
@@ -979,8 +983,8 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     // overlaps the set-up
     const unsigned smax_bits_k = p.smax[0], smax_bits_v = p.smax[1];
 
-    const SmemParts sm = carve(smem, NS, REC, D, NT);
-    WarpPipe P{sm.stages + static_cast<size_t>(warp) * NS * REC, sm.bars + warp * NS, NS, REC, lane, 0, 0, 0u, 0};
+    const SmemParts sm = carve(smem, NW * p.nstage + p.nextra, REC, D, NT);
+    WarpPipe P{sm.stages + static_cast<size_t>(sbase) * REC, sm.bars + sbase, NS, REC, lane, 0, 0, 0u, 0};
     pipe_init(P);
     const uint8_t *unit_rec = p.rec + (static_cast<long long>(b) * p.Hkv + h) * p.cap_blk * REC;
     const int nb = (blk1 - blk0 > warp) ? (blk1 - blk0 - warp + NW - 1) / NW : 0;
@@ -1123,7 +1127,7 @@ __device__ __forceinline__ void paged_body(const PagedDecodeParams &p, uint8_t *
     const int nsplit = INT2 ? p.S2 : p.S4, si = INT2 ? sp : sp - p.S2;
     const int per = (nitems + nsplit - 1) / nsplit;
     const int u0 = min(nitems, si * per), u1 = min(nitems, u0 + per);
-    const SmemParts sm = carve(smem, NS, STAGE, D, NT);
+    const SmemParts sm = carve(smem, NW * NS, STAGE, D, NT);
     WarpPipe P{sm.stages + static_cast<size_t>(warp) * NS * STAGE, sm.bars + warp * NS, NS, STAGE, lane, 0, 0, 0u, 0};
     pipe_init(P);
     const int *tab = p.table + static_cast<long long>(b) * p.P_cap;
@@ -1283,9 +1287,9 @@ int decode_stages(long long rec_bytes, int D, int G) {
     return 2;
 }
 
-size_t decode_smem_bytes(long long rec_bytes, int nstage, int D, int G) {
+size_t decode_smem_bytes(long long rec_bytes, int nstage, int nextra, int D, int G) {
     const int NT = G <= 4 ? 1 : 2;
-    return smem_total(nstage, static_cast<int>(rec_bytes), D, NT);
+    return smem_total(NW * nstage + nextra, static_cast<int>(rec_bytes), D, NT);
 }
 
 // Per-kernel cache of the dynamic shared-memory attribute and occupancy, so launches
@@ -1334,17 +1338,18 @@ static cudaError_t prepare_kernel(const void *fn, size_t smem, int *occ_out) {
 }
 
 cudaError_t decode_occupancy(int D, int bk, int bv, int kmode, int G, long long rec_bytes, int nstage,
-                             int *ctas_per_sm) {
+                             int nextra, int *ctas_per_sm) {
     KernelFn fn = pick_kernel(D, bk, bv, kmode, G);
     if (!fn) return cudaErrorInvalidValue;
-    return prepare_kernel(reinterpret_cast<const void *>(fn), decode_smem_bytes(rec_bytes, nstage, D, G), ctas_per_sm);
+    return prepare_kernel(reinterpret_cast<const void *>(fn), decode_smem_bytes(rec_bytes, nstage, nextra, D, G),
+                          ctas_per_sm);
 }
 
 cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmode, cudaStream_t st,
                           int *ctas_per_sm_out) {
     KernelFn fn = pick_kernel(D, bk, bv, kmode, p.G);
     if (!fn) return cudaErrorInvalidValue;
-    const size_t smem = decode_smem_bytes(p.rec_bytes, p.nstage, D, p.G);
+    const size_t smem = decode_smem_bytes(p.rec_bytes, p.nstage, p.nextra, D, p.G);
     cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(fn), smem, ctas_per_sm_out);
     if (e != cudaSuccess) return e;
     dim3 grid(p.S, p.Hkv, p.B);
@@ -1362,7 +1367,7 @@ static int paged_stage_bytes() {
 
 int decode_paged_stages() { return decode_stages(paged_stage_bytes(), 128, 4); }
 
-size_t decode_paged_smem_bytes(int nstage) { return smem_total(nstage, paged_stage_bytes(), 128, 1); }
+size_t decode_paged_smem_bytes(int nstage) { return smem_total(NW * nstage, paged_stage_bytes(), 128, 1); }
 
 cudaError_t decode_paged_occupancy(int nstage, int *ctas_per_sm) {
     return prepare_kernel(reinterpret_cast<const void *>(decode_paged_kernel), decode_paged_smem_bytes(nstage), ctas_per_sm);

@@ -455,7 +455,9 @@ static int ensure_device_info(kvq_handle *h) {
 // every stage count from 1 to the most that fit is costed with the occupancy it allows
 // (deep rings fit fewer CTAs per SM; short sequences gain more from one wave than from
 // prefetch depth).
-static int splits_for(kvq_handle *h, int layer, int *S_out, int *nstage_out) {
+// Split count S, stages per warp and extra stages (for the warps with the most blocks
+// when one stage per warp is used) of a per-layer decode launch.
+static int splits_for(kvq_handle *h, int layer, int *S_out, int *nstage_out, int *nextra_out) {
     const LayerGeom &g = h->geom[layer];
     const int L = h->len[layer];
     const int nblk = (L + 31) / 32;
@@ -468,32 +470,32 @@ static int splits_for(kvq_handle *h, int layer, int *S_out, int *nstage_out) {
     double best = 1e300;
     *S_out = 1;
     *nstage_out = ns_max;
-    for (int ns = 1; ns <= ns_max; ++ns) {
-        int per_sm = 1;
-        cudaError_t e = kvq::decode_occupancy(h->desc.head_dim, g.bk, g.bv, g.kmode, G, g.rec_bytes, ns, &per_sm);
-        if (e != cudaSuccess) return cuda_fail(e, "decode occupancy");
-        if (h->forced_splits > 0) {
-            const int S = std::min(h->forced_splits, smax);
-            const double c = decode_cost(units, nblk, S, ns, per_sm, h->sm_count);
-            if (c < best - 1e-9) {
-                best = c;
-                *S_out = S;
-                *nstage_out = ns;
+    *nextra_out = 0;
+    constexpr int NW = kvq::kDecodeWarps;
+    for (int ns = 1; ns <= ns_max; ++ns)
+        for (int nx = 0; nx < (ns == 1 ? NW : 1); ++nx) {
+            int per_sm = 1;
+            cudaError_t e =
+                kvq::decode_occupancy(h->desc.head_dim, g.bk, g.bv, g.kmode, G, g.rec_bytes, ns, nx, &per_sm);
+            if (e != cudaSuccess) return cuda_fail(e, "decode occupancy");
+            for (int S = 1; S <= smax; ++S) {
+                if (h->forced_splits > 0 && S != std::min(h->forced_splits, smax)) continue;
+                const int bps = (nblk + S - 1) / S;
+                const int sreal = (nblk + bps - 1) / bps;
+                if (h->forced_splits <= 0 && sreal != S) continue;
+                // extra stages: for exactly the warps with two blocks (warps 0 .. bps % NW
+                // - 1) when every other warp has one, so that no warp waits for a copy
+                // issued after its previous block
+                if (nx > 0 && !(bps > NW && bps < 2 * NW && nx == bps % NW)) continue;
+                const double c = decode_cost(units, nblk, S, nx > 0 ? 2 : ns, per_sm, h->sm_count);
+                if (c < best - 1e-9) {
+                    best = c;
+                    *S_out = S;
+                    *nstage_out = ns;
+                    *nextra_out = nx;
+                }
             }
-            continue;
         }
-        for (int S = 1; S <= smax; ++S) {
-            const int bps = (nblk + S - 1) / S;
-            const int sreal = (nblk + bps - 1) / bps;
-            if (sreal != S) continue;
-            const double c = decode_cost(units, nblk, S, ns, per_sm, h->sm_count);
-            if (c < best - 1e-9) {
-                best = c;
-                *S_out = S;
-                *nstage_out = ns;
-            }
-        }
-    }
     return KVQ_OK;
 }
 
@@ -607,8 +609,8 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
         return decode_paged(h, layer, q, out, out_fp32, static_cast<cudaStream_t>(stream),
                             reinterpret_cast<float *>(h->ws + h->part_acc_off),
                             reinterpret_cast<float *>(h->ws + h->part_ml_off));
-    int S = 1, nstage = 2;
-    if ((rc = splits_for(h, layer, &S, &nstage))) return rc;
+    int S = 1, nstage = 2, nextra = 0;
+    if ((rc = splits_for(h, layer, &S, &nstage, &nextra))) return rc;
     const LayerGeom &g = h->geom[layer];
     const int nblk = (L + 31) / 32;
     kvq::DecodeParams p{};
@@ -629,6 +631,7 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
     p.S = (nblk + p.bps - 1) / p.bps;
     p.out_fp32 = out_fp32 ? 1 : 0;
     p.nstage = nstage;
+    p.nextra = nextra;
     p.rec_bytes = g.rec_bytes;
     p.arrive = p.S >= kvq::kInLaunchMergeSplits ? reinterpret_cast<unsigned *>(h->ws + h->arrive_off) : nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -671,8 +674,8 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
         return kvq_decode_attn(h, layer, q, out, out_fp32, stream);
     }
     h->len[layer] = L;   // the schedule is chosen for the new length
-    int S = 1, nstage = 2;
-    if ((rc = splits_for(h, layer, &S, &nstage))) {
+    int S = 1, nstage = 2, nextra = 0;
+    if ((rc = splits_for(h, layer, &S, &nstage, &nextra))) {
         h->len[layer] = L_old;
         return rc;
     }
@@ -695,6 +698,7 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
     p.S = (nblk + p.bps - 1) / p.bps;
     p.out_fp32 = out_fp32 ? 1 : 0;
     p.nstage = nstage;
+    p.nextra = nextra;
     p.rec_bytes = g.rec_bytes;
     p.arrive = p.S >= kvq::kInLaunchMergeSplits ? reinterpret_cast<unsigned *>(h->ws + h->arrive_off) : nullptr;
     p.k_new = static_cast<const uint16_t *>(K);
@@ -751,8 +755,8 @@ int kvq_get_num_splits(const kvq_handle *hc, int layer, int *num_splits) {
         *num_splits = S2 + S4;
         return ok();
     }
-    int S = 1, nstage = 2;
-    if ((rc = splits_for(h, layer, &S, &nstage))) return rc;
+    int S = 1, nstage = 2, nextra = 0;
+    if ((rc = splits_for(h, layer, &S, &nstage, &nextra))) return rc;
     const int nblk = (L + 31) / 32;
     const int bps = (nblk + S - 1) / S;
     *num_splits = (nblk + bps - 1) / bps;
@@ -970,8 +974,8 @@ int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, 
     const int L = h->len[layer];
     if (L < 1) return fail(KVQ_EINVAL, "layer %d is empty", layer);
     if (h->desc.paged) return fail(KVQ_EUNSUPPORTED, "paged plans are not supported by kvq_decode_attn_noalloc");
-    int S = 1, nstage = 2;
-    if ((rc = splits_for(h, layer, &S, &nstage))) return rc;
+    int S = 1, nstage = 2, nextra = 0;
+    if ((rc = splits_for(h, layer, &S, &nstage, &nextra))) return rc;
     const LayerGeom &g = h->geom[layer];
     const int nblk = (L + 31) / 32;
     const int bps = (nblk + S - 1) / S;
@@ -1003,6 +1007,7 @@ int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, 
     p.S = S;
     p.out_fp32 = out_fp32 ? 1 : 0;
     p.nstage = nstage;
+    p.nextra = nextra;
     p.rec_bytes = g.rec_bytes;
     p.arrive = p.S >= kvq::kInLaunchMergeSplits ? reinterpret_cast<unsigned *>(h->ws + h->arrive_off) : nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -76,7 +76,8 @@ struct DecodeParams {
     unsigned *arrive;           // [B][Hkv] split arrival counters (zero between launches), or null:
                                 // split partials merged by merge_kernel
     unsigned *status;
-    int B, Hkv, G, L, cap_blk, S, bps, out_fp32, nstage;
+    int B, Hkv, G, L, cap_blk, S, bps, out_fp32;
+    int nstage, nextra;         // stages per warp; one more for warps 0 .. nextra - 1
     long long rec_bytes;
     // Fused one-token append (kvq_append_decode), null otherwise: the new token's K and V
     // rows (bf16 [B][Hkv][D]), now token L - 1; writable records and residual; the
@@ -158,7 +159,7 @@ cudaError_t launch_append(const AppendParams &p, cudaStream_t st);
 cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmode,
                           cudaStream_t st, int *ctas_per_sm_out);
 cudaError_t decode_occupancy(int D, int bk, int bv, int kmode, int G, long long rec_bytes,
-                             int nstage, int *ctas_per_sm);
+                             int nstage, int nextra, int *ctas_per_sm);
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t st);
 cudaError_t launch_decode_paged(const PagedDecodeParams &p, cudaStream_t st);
 cudaError_t decode_paged_occupancy(int nstage, int *ctas_per_sm);
@@ -170,6 +171,6 @@ cudaError_t launch_paged_append(const PagedAppendParams &p, int grid, cudaStream
 int paged_rec2_bytes(int D);
 int paged_page4_bytes(int D);
 int decode_stages(long long rec_bytes, int D, int G);
-size_t decode_smem_bytes(long long rec_bytes, int nstage, int D, int G);
+size_t decode_smem_bytes(long long rec_bytes, int nstage, int nextra, int D, int G);
 
 }  // namespace kvq
