@@ -1021,6 +1021,8 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
             bulk_g2s(vn_s, p.v_new + unit * D, 2 * D, pro_bar);
         }
     }
+    __syncwarp();   // warp 0's other lanes wait on pro_bar after lane 0 initialised it; the
+                    // other warps wait on it only after a CTA barrier
     if constexpr (KM == 0) {
         // the bf16 residual rows of the tail block: into L2 now, read after the tail's copy
         if (p.res && tail_blk >= blk0 && tail_blk < blk1 && ((tail_blk - blk0) % NW) == warp) {
