@@ -104,3 +104,52 @@ def test_fused_in_launch_merge(kmode):
     """Five splits: the split partials are merged by the last CTA of each (b, kv head)
     inside the fused launch, step after step (the arrival counters reset themselves)."""
     run_fused(2, 2, 4, 128, (4, 2), kmode, 150, 40, [151, 160, 161, 175, 190], splits=5, tag=f"merge{kmode}")
+
+
+def test_fused_c2_full_size_graphs():
+    """The default bench workload at full size (Llama-3.1-8B shape, batch 64, 8 kv heads,
+    GQA 4, K8V4, per-channel keys; 2 of its 32 layers), in the bench's launch
+    configuration: prompt 128, then every decode step of each layer captured into a CUDA
+    graph (fused append + decode; steps completing a key group take two launches inside
+    the call) and replayed.  At the checked lengths the step's graph is replayed a second
+    time: replays are idempotent (same image, same output)."""
+    wl = configs.llama_c2((8, 4))
+    B, Hkv, G, D, NL, P = wl.batch, wl.n_kv_heads, wl.G, wl.head_dim, 2, wl.prefill
+    steps = 128
+    cache = kvq.Cache(NL, B, Hkv, Hkv * G, D, P + steps, [(8, 4)] * NL)
+    KV = [inputs.layer_kv(wl, l, P + steps, "cuda") for l in range(NL)]
+    for l in range(NL):
+        cache.append(l, KV[l][0][:, :, :P].contiguous(), KV[l][1][:, :, :P].contiguous())
+    stream = torch.cuda.Stream()
+    check = {129, 144, 159, 160, 161, 200, 255, 256}
+    for L in range(P + 1, P + steps + 1):
+        qs = [inputs.step_q(wl, l, L, "cuda") for l in range(NL)]
+        ks = [KV[l][0][:, :, L - 1:L].contiguous() for l in range(NL)]
+        vs = [KV[l][1][:, :, L - 1:L].contiguous() for l in range(NL)]
+        outs = [torch.empty((B, Hkv * G, D), dtype=torch.float32, device="cuda") for _ in range(NL)]
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for l in range(NL):
+                cache.append_decode(l, ks[l], vs[l], qs[l], outs[l], out_fp32=True, stream=stream.cuda_stream)
+        g.replay()
+        torch.cuda.synchronize()
+        if L not in check:
+            continue
+        first = [o.clone() for o in outs]
+        imgs = [cache.export_layer(l) for l in range(NL)]
+        g.replay()
+        torch.cuda.synchronize()
+        for l in range(NL):
+            assert torch.equal(first[l], outs[l]), (L, l)
+            assert np.array_equal(imgs[l], cache.export_layer(l)), (L, l)
+            Kb, Vb = bits16(KV[l][0][:, :, :L]), bits16(KV[l][1][:, :, :L])
+            img_ref, out_ref = oracle.layer(Kb, Vb, bits16(qs[l]), G, 8, 4, 0)
+            if not np.array_equal(imgs[l], img_ref):
+                bad = np.flatnonzero(imgs[l] != img_ref)
+                pytest.fail(f"c2 full L={L} layer {l}: image differs at {bad.size} bytes, first {bad[:8]}")
+            out16 = cache.decode_attn(l, qs[l], out_fp32=False)
+            torch.cuda.synchronize()
+            check_outputs(outs[l], out16, out_ref, f"c2 full L={L} layer {l}")
+        del g
+    assert kvq.kvq_device_status(cache.h) == 0
