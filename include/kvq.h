@@ -203,6 +203,45 @@ KVQ_API int kvq_device_status(kvq_handle *h, void *stream, unsigned *flags);
 KVQ_API int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, int out_fp32,
                                     void *stream);
 
+/* ---- Per-tag bit allocation of paged plans (host memory, no device work) ----------
+ * From "TriAxialKV per-role mixed-precision KV quantization for agentic prefills",
+ * Facts: the per-tag distortion D_k(b) is the attention-output MSE, taken as the max over
+ * heads, the mean over requests and the sum over layers; each tag gets INT2 or INT4 under
+ * an average-bit budget, by exhaustive search for 22 or fewer tags and a greedy
+ * per-bit-gain rule otherwise.  The tagger (chat-template markers) is not part of this
+ * library: tags arrive as integers. */
+
+/* D_k(2) and D_k(4) for every tag k from calibration prefills (host pointers):
+ *   Q bf16 [num_layers][num_requests][n_q_heads][T][head_dim],
+ *   K, V bf16 [num_layers][num_requests][n_kv_heads][T][head_dim],
+ *   tags int32 [num_requests][T] in [0, num_tags), shared by layers and heads.
+ * For (tag k, b): the tokens of tag k are quantized at b bits and every other token is
+ * kept exact; b = 4 quantizes K and V per token (groups of 32 channels); b = 2 quantizes
+ * K per channel over consecutive 32-token groups of the tag's tokens of that request
+ * (in token order) and V per token, and the tag's last T_k mod 32 tokens take the 4-bit
+ * per-token path for K and V (leftover routing of the pages).  The error measure is the
+ * mean squared difference of the causal attention outputs (all T queries, fp64) against
+ * the exact keys and values, per query head; D_k(b) = sum over layers of the mean over
+ * requests of the max over query heads.  Tags with no token get 0.  counts[k] receives
+ * the number of tokens of tag k over all requests.  Cost O(layers x requests x tags x
+ * n_q_heads x T^2 x head_dim), spread over the host's cores: a calibration tool for
+ * prefills of up to a few thousand tokens.  Errors: KVQ_EINVAL (counts, shapes: head_dim
+ * a multiple of 32, n_q_heads a multiple of n_kv_heads; tags out of range; null). */
+KVQ_API int kvq_tag_distortion(int num_layers, int num_requests, int n_q_heads, int n_kv_heads, int head_dim,
+                               int T, const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                               const int32_t *tags, int num_tags, double *D2, double *D4, int64_t *counts);
+
+/* bits[k] in {2, 4} for every tag: minimise sum_k D_{b_k}(k) subject to
+ * sum_k counts[k] * bits[k] <= avg_bits * sum_k counts[k].  Tags with counts[k] == 0
+ * take no part and get 4.  With P <= 22 tags present: exhaustive over all 2^P choices,
+ * distortion summed in ascending tag order, the first least-distortion choice in
+ * ascending mask order (bit i = the i-th present tag at INT2).  Otherwise greedy: start
+ * from all INT4 and move to INT2 the tag of least (D_k(2) - D_k(4)) / (2 counts[k])
+ * (ties: lower index) until the budget holds.  *total_distortion (if not NULL) gets the
+ * chosen sum.  Errors: KVQ_EINVAL (avg_bits outside [2, 4], negative counts, null). */
+KVQ_API int kvq_tag_allocate(int num_tags, const double *D2, const double *D4, const int64_t *counts,
+                             double avg_bits, int *bits, double *total_distortion);
+
 /* Free the handle (not the caller's workspace). */
 KVQ_API void kvq_destroy(kvq_handle *h);
 

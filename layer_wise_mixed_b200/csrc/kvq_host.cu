@@ -124,6 +124,11 @@ double decode_cost(int units, int nblk, int S, int nstage, int occ, int sms) {
 
 }  // namespace
 
+namespace kvq {
+int host_fail(int code, const char *msg) { return fail(code, "%s", msg); }
+int host_ok() { return ok(); }
+}  // namespace kvq
+
 extern "C" {
 
 const char *kvq_last_error(void) { return g_err.c_str(); }

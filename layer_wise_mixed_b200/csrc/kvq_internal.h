@@ -154,6 +154,11 @@ struct MergeParams {
 // round trip at its exit), nine (the paged 32K-context workload) with the in-launch merge.
 constexpr int kInLaunchMergeSplits = 4;
 
+// Set the thread's kvq_last_error message and return code / clear it and return KVQ_OK
+// (for entry points outside kvq_host.cu).
+int host_fail(int code, const char *msg);
+int host_ok();
+
 cudaError_t launch_append(const AppendParams &p, cudaStream_t st);
 // Returns cudaErrorInvalidValue if no kernel exists for the combination.
 cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmode,

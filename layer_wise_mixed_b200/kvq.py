@@ -77,6 +77,8 @@ def load() -> ctypes.CDLL:
         "kvq_seq_len": (I, [P, I, ctypes.POINTER(I)]),
         "kvq_truncate": (I, [P, I, I]),
         "kvq_device_status": (I, [P, P, ctypes.POINTER(ctypes.c_uint)]),
+        "kvq_tag_distortion": (I, [I, I, I, I, I, I, P, P, P, P, I, P, P, P]),
+        "kvq_tag_allocate": (I, [I, P, P, P, ctypes.c_double, P, P]),
         "kvq_destroy": (None, [P]),
         "kvq_last_error": (ctypes.c_char_p, []),
     }
@@ -196,6 +198,42 @@ def kvq_destroy(h: int):
 
 def kvq_last_error() -> str:
     return load().kvq_last_error().decode()
+
+
+def kvq_tag_distortion(Q, K, V, tags, num_tags: int):
+    """Per-tag distortion from calibration prefills (host numpy arrays): Q uint16 (bf16
+    bits) [NL, R, Hq, T, D], K/V [NL, R, Hkv, T, D], tags int32 [R, T].
+    Returns (D2, D4, counts)."""
+    import numpy as np
+    Q = np.ascontiguousarray(Q, np.uint16)
+    K = np.ascontiguousarray(K, np.uint16)
+    V = np.ascontiguousarray(V, np.uint16)
+    tags = np.ascontiguousarray(tags, np.int32)
+    NL, R, Hq, T, D = Q.shape
+    Hkv = K.shape[2]
+    if K.shape != (NL, R, Hkv, T, D) or V.shape != K.shape or tags.shape != (R, T):
+        raise ValueError("shape mismatch")
+    D2 = np.zeros(num_tags, np.float64)
+    D4 = np.zeros(num_tags, np.float64)
+    counts = np.zeros(num_tags, np.int64)
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    _check(load().kvq_tag_distortion(NL, R, Hq, Hkv, D, T, p(Q), p(K), p(V), p(tags), num_tags, p(D2), p(D4),
+                                     p(counts)))
+    return D2, D4, counts
+
+
+def kvq_tag_allocate(D2, D4, counts, avg_bits: float):
+    """INT2/INT4 per tag under the average-bit budget: (bits int32 [K], total distortion)."""
+    import numpy as np
+    D2 = np.ascontiguousarray(D2, np.float64)
+    D4 = np.ascontiguousarray(D4, np.float64)
+    counts = np.ascontiguousarray(counts, np.int64)
+    bits = np.zeros(len(counts), np.int32)
+    total = ctypes.c_double(0.0)
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    _check(load().kvq_tag_allocate(len(counts), p(D2), p(D4), p(counts), float(avg_bits), p(bits),
+                                   ctypes.byref(total)))
+    return bits, total.value
 
 
 # ------------------------------------------------------------------ convenience owner
