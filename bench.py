@@ -11,7 +11,7 @@ replays K graphs.  The dominant kernel's roofline comes from decode-only replays
 same schedule.  Inputs are seeded synthetic tensors already resident in HBM; one step reads
 every layer's cache once (larger than L2 for every workload here).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c2-k8v8|c3|c4|c5]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2|c2-k8v8|c3|c4|c5|c5-alloc]
     python bench.py --impl reference ...     # the CPU oracle on a bounded sample
 
 Under torchrun each rank runs its own replica of the workload (own seeds, no data-path
@@ -63,6 +63,14 @@ def captured_traffic(workload_name, alg_bytes_per_launch):
         return float(kv["dram_bytes"]) / float(kv["algorithmic_bytes"]) * alg_bytes_per_launch
     except Exception:
         return None
+
+
+def paged_tags(wl, n_tokens, tag="prefill", batch=None):
+    """INT2/INT4 mask of a paged workload: seeded Bernoulli, or the per-tag allocation."""
+    from layer_wise_mixed_b200 import inputs, tagalloc
+    if wl.tag_source == "alloc":
+        return tagalloc.token_mask(wl, n_tokens, tag=tag, batch=batch)
+    return inputs.tags(wl, n_tokens, tag=tag, batch=batch)
 
 
 def rank_workload(wl, rank, world):
@@ -174,7 +182,7 @@ def cpu_oracle_sample(wl, L, seqs, layers=1):
         bk, bv = wl.layer_bits[l % len(wl.layer_bits)]
         t0 = time.perf_counter()
         if wl.paged:
-            tg = inputs.tags(wl, L, tag="cpu-sample", batch=seqs).numpy()
+            tg = paged_tags(wl, L, tag="cpu-sample", batch=seqs).numpy()
             oracle.paged_layer(Kb, Vb, tg, qb, wl.G, want_image=False)
         else:
             oracle.layer(Kb, Vb, qb, wl.G, bk, bv, wl.kmode, want_image=False)
@@ -216,7 +224,9 @@ def workload_config(wl):
         return {"workload": wl.name, "layers": wl.num_layers, "batch": wl.batch, "q_heads": wl.n_q_heads,
                 "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim,
                 "context": f"{wl.prefill + 1}..{wl.prefill + wl.decode_steps}",
-                "bits": "INT2 groups (K per-channel, V per-token) + INT4 per-token, tags Bernoulli(0.5)",
+                "bits": "INT2 groups (K per-channel, V per-token) + INT4 per-token, tags " +
+                        ("from the per-tag allocation at 3.0 bits (synthetic segment tag ids, seeded calibration)"
+                         if wl.tag_source == "alloc" else "Bernoulli(0.5)"),
                 "equivalent_bits": wl.avg_bits, "page_tokens": wl.page_tokens,
                 "l2": "inputs larger than L2 (each step reads every layer's cache once)",
                 "launch": "one CUDA graph per decode step (tagged append + paged decode for all layers)"}
@@ -236,7 +246,7 @@ def main():
     ap.add_argument("--steps", type=int, default=512)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="c2", choices=["c2", "c2-k8v8", "c2-k8v4", "c3", "c4", "c5"])
+    ap.add_argument("--workload", default="c2", choices=["c2", "c2-k8v8", "c2-k8v4", "c3", "c4", "c5", "c5-alloc"])
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--ref-seqs", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -275,8 +285,10 @@ def main():
     B, Hkv, Hq, D, G, NL = wl.batch, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.G, wl.num_layers
     paged = wl.paged
     if paged:
-        cache = kvq.Cache(NL, B, Hkv, Hq, D, wl.max_ctx, avg_bits=wl.avg_bits)
-        all_tags = inputs.tags(wl, wl.max_ctx)                 # [B, prefill + steps], shared by layers
+        all_tags = paged_tags(wl, wl.max_ctx)                  # [B, prefill + steps], shared by layers
+        # the pools split at the mask's own mean bits (an allocation may land under its budget)
+        plan_bits = min(wl.avg_bits, 4.0 - 2.0 * float((all_tags == 2).float().mean()))
+        cache = kvq.Cache(NL, B, Hkv, Hq, D, wl.max_ctx, avg_bits=plan_bits)
         tags_dev = all_tags.cuda()
         tags_host = all_tags.numpy()
     else:

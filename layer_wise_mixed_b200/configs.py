@@ -38,6 +38,7 @@ class Workload:
     page_tokens: int = 16
     avg_bits: float = 0.0     # paged: average bits of the tag mask
     int2_prob: float = 0.5    # paged: probability that a token is tagged INT2
+    tag_source: str = "bernoulli"   # paged: "bernoulli" mask, or "alloc" (per-tag allocation)
 
     @property
     def G(self) -> int:
@@ -104,7 +105,17 @@ def paged_c5() -> Workload:
                     int2_prob=0.5)
 
 
+def paged_c5_alloc() -> Workload:
+    """C5 with the INT2/INT4 mask from the per-tag allocation at 3.0 bits: tokens carry
+    synthetic (temporal, modal, semantic) tag ids in segments; a small seeded calibration
+    set of the same shape gives D_k(b); each tag's tokens take its bits."""
+    return Workload("llama8b-b16-ctx32768-paged-alloc", 32, 16, 32, 8, 128, 32768, 17,
+                    tuple([(2, 2)] * 32), paged=True, page_tokens=16, avg_bits=3.0,
+                    tag_source="alloc")
+
+
 def by_name(name: str) -> Workload:
     table = {"tiny": tiny(), "c2": llama_c2((8, 4)), "c2-k8v8": llama_c2((8, 8)),
-             "c2-k8v4": llama_c2((8, 4)), "c3": llama_c3(), "c4": qwen_c4(), "c5": paged_c5()}
+             "c2-k8v4": llama_c2((8, 4)), "c3": llama_c3(), "c4": qwen_c4(), "c5": paged_c5(),
+             "c5-alloc": paged_c5_alloc()}
     return table[name]

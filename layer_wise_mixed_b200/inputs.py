@@ -13,6 +13,11 @@ Recipe (per layer l, kv head h):
   * V ~ N(0, 1), Q ~ N(0, 1).
   * Tags (paged workloads): per (batch row, token) INT2 with probability
     int2_prob, else INT4, shared by all layers and heads.
+  * Tag ids (per-tag allocation): each sequence is cut into segments (16-256 tokens;
+    calibration sets 16-64);
+    a segment's id is (temporal * 2 + modal) * 7 + semantic with temporal = the
+    quarter of the sequence it starts in, modal = 1 (image) with probability 0.3 and
+    semantic uniform in 0..6: 56 possible ids, of which a sequence uses some.
 """
 from __future__ import annotations
 
@@ -69,3 +74,30 @@ def tags(w: Workload, n_tokens: int, tag="prefill", batch=None) -> torch.Tensor:
     g = _gen("cpu", w.name, tag, "tags", B, n_tokens)
     u = torch.rand((B, n_tokens), generator=g)
     return torch.where(u < w.int2_prob, 2, 4).to(torch.uint8)
+
+
+def prefill_q(w: Workload, layer: int, n_tokens: int, device="cpu", batch=None, tag="prefill"):
+    """Q bf16 [B, Hq, n_tokens, D] for the prefill tokens of one layer (calibration)."""
+    B = w.batch if batch is None else batch
+    g = _gen(device, w.name, layer, tag, "Qp", B, n_tokens)
+    q = torch.randn((B, w.n_q_heads, n_tokens, w.head_dim), generator=g, device=device, dtype=torch.float32)
+    return q.to(torch.bfloat16)
+
+
+def tag_ids(w: Workload, n_tokens: int, tag="prefill", batch=None, seg=(16, 256)) -> torch.Tensor:
+    """int32 [B, n_tokens] segment tag ids in [0, 56) (recipe in the module docstring;
+    segment lengths uniform in seg)."""
+    B = w.batch if batch is None else batch
+    g = _gen("cpu", w.name, tag, "tagids", B, n_tokens, seg[0], seg[1])
+    out = torch.empty((B, n_tokens), dtype=torch.int32)
+    for b in range(B):
+        t = 0
+        while t < n_tokens:
+            n = int(torch.randint(seg[0], seg[1] + 1, (1,), generator=g))
+            temporal = min(3, 4 * t // n_tokens)
+            modal = int(torch.rand(1, generator=g) < 0.3)
+            semantic = int(torch.randint(0, 7, (1,), generator=g))
+            out[b, t:t + n] = (temporal * 2 + modal) * 7 + semantic
+            t += n
+    return out
+

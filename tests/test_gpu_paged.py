@@ -103,3 +103,15 @@ def test_paged_c5_full_layer():
     tags = inputs.tags(wl, L0 + steps).numpy()
     run_paged(wl.batch, wl.n_kv_heads, wl.G, [L0] + [1] * steps, tags, decode_at=[L0 + 1, L0 + steps],
               wl=wl, avg_bits=wl.avg_bits)
+
+
+def test_paged_segment_tag_mask():
+    """Masks with the per-tag allocation's structure: runs of 16-256 tokens share one
+    precision (segment tag ids mapped by a fixed table: even ids INT2, odd INT4), so INT2
+    groups complete in the middle of runs and pending pages fill from several runs;
+    prompt of 1500 tokens, then 40 single tokens, splits automatic and forced."""
+    B, L0, n = 4, 1500, 40
+    wl = configs.Workload("paged-seg", 1, B, 2 * 4, 2, 128, 0, 0, ((2, 2),))
+    ids = inputs.tag_ids(wl, L0 + n).numpy()
+    tags = np.where(ids % 2 == 0, 2, 4).astype(np.uint8)
+    run_paged(B, 2, 4, [L0] + [1] * n, tags, decode_at=[L0, L0 + 1, L0 + 17, L0 + n], splits=(0, 3, 6), wl=wl)
