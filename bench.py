@@ -417,51 +417,100 @@ def main():
         two = paged or (wl.kmode == 0 and Ls[s] % 32 == 0)
         return (2 if two else 1) + (1 if 1 < splits[s][l] < 4 else 0)
     gpu_launches = sum(step_launches(s, l) for s in order for l in range(NL))
-    e2e_note = ("per step: pinned H2D of all layers' K/V/q, kvq_append_decode per layer (eager "
-                "C-ABI calls), D2H of all layers' outputs")
+    e2e_note = ("per step and group of 4 layers: pinned H2D of the group's K/V/q (copy stream), "
+                "kvq_append_decode per layer (eager C-ABI calls, compute stream), D2H of the group's outputs "
+                "(second copy stream); groups overlap")
     if paged:
-        e2e_note = ("per step: pinned H2D of all layers' K/V/q and kvq_decode_attn per layer (eager C-ABI calls; "
-                    "the cache is not advanced), D2H of all layers' outputs")
+        e2e_note = ("per step and group of 4 layers: pinned H2D of the group's K/V/q, kvq_decode_attn per layer "
+                    "(eager C-ABI calls; the cache is not advanced), D2H of the group's outputs; groups overlap")
 
     # ---- e2e: public API with host buffers, H2D + D2H inside the timed region ----
+    # Per step and group of CH layers: one H2D of the group's K|V|q (pinned host, packed per
+    # layer) on a copy stream, the group's C-ABI calls on the compute stream, one D2H of
+    # the group's outputs on a second copy stream (the other PCIe direction), so that
+    # transfers of one group overlap the calls of another; device buffers alternate
+    # between even and odd steps.
     e2e_steps = args.e2e_steps or min(args.steps, 64)
-    hK = Kn.cpu().pin_memory()
-    hV = Vn.cpu().pin_memory()
-    hQ = Qn.cpu().pin_memory()
-    hO = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    dK = torch.empty_like(Kn[0])
-    dV = torch.empty_like(Vn[0])
-    dQ = torch.empty_like(Qn[0])
+    CH = 4
+    groups = [list(range(g0, min(NL, g0 + CH))) for g0 in range(0, NL, CH)]
+    nk, nq = B * Hkv * D, B * Hq * D                      # bf16 elements per layer
+    per = 2 * nk + nq
+    hIn = torch.cat([Kn.reshape(nsched, NL, nk), Vn.reshape(nsched, NL, nk), Qn.reshape(nsched, NL, nq)],
+                    dim=2).cpu().pin_memory()             # [step, layer, K|V|q]
+    hO = torch.empty((NL,) + tuple(out.shape[1:]), dtype=out.dtype).pin_memory()
+    dIn = torch.empty((2, NL, per), dtype=torch.bfloat16, device="cuda")
+    dOut = torch.empty((2,) + tuple(out.shape), dtype=out.dtype, device="cuda")
+    h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = {k: [[torch.cuda.Event() for _ in groups] for _ in range(2)] for k in ("in", "comp", "out")}
+    used = [[False] * len(groups) for _ in range(2)]
     if not paged:
         for l in range(NL):
             kvq.kvq_truncate(cache.h, l, wl.prefill)
+    # raw C-ABI calls with pointers taken once (the Python wrappers cost more host time
+    # per call than the transfers they would overlap)
+    lib = kvq.load()
+    sptr = stream.cuda_stream
+    ptrs = [[(dIn[par, l].data_ptr(), dIn[par, l].data_ptr() + 2 * nk, dIn[par, l].data_ptr() + 4 * nk,
+              dOut[par, l].data_ptr()) for l in range(NL)] for par in range(2)]
+    lens = [wl.prefill] * NL
 
-    def e2e_step(s):
-        dK.copy_(hK[s], non_blocking=True)
-        dV.copy_(hV[s], non_blocking=True)
-        dQ.copy_(hQ[s], non_blocking=True)
-        for l in range(NL):
-            if paged:
-                kvq.kvq_decode_attn(cache.h, l, dQ[l], out[l], False, stream)
-                continue
-            if cache.seq_len(l) >= wl.max_ctx:
+    def call(l, par):
+        pk, pv, pq, po = ptrs[par][l]
+        if paged:
+            rc = lib.kvq_decode_attn(cache.h, l, pq, po, 0, sptr)
+        else:
+            if lens[l] >= wl.max_ctx:
                 kvq.kvq_truncate(cache.h, l, wl.prefill)
-            kvq.kvq_append_decode(cache.h, l, dK[l], dV[l], dQ[l], out[l], False, stream)
-        hO.copy_(out, non_blocking=True)
+                lens[l] = wl.prefill
+            rc = lib.kvq_append_decode(cache.h, l, pk, pv, pq, po, 0, sptr)
+            lens[l] += 1
+        if rc != kvq.KVQ_OK:
+            raise kvq.KvqError(rc, lib.kvq_last_error().decode())
+
+    def e2e_step(i, s):
+        par = i & 1
+        for gi, grp in enumerate(groups):
+            l0, l1 = grp[0], grp[-1] + 1
+            with torch.cuda.stream(h2d_stream):
+                if used[par][gi]:
+                    h2d_stream.wait_event(ev["comp"][par][gi])     # the calls of step i - 2 read this buffer
+                dIn[par, l0:l1].copy_(hIn[s, l0:l1], non_blocking=True)
+                ev["in"][par][gi].record(h2d_stream)
+            stream.wait_event(ev["in"][par][gi])
+            if used[par][gi]:
+                stream.wait_event(ev["out"][par][gi])              # step i - 2's outputs are on the host
+            for l in grp:
+                call(l, par)
+            ev["comp"][par][gi].record(stream)
+            with torch.cuda.stream(d2h_stream):
+                d2h_stream.wait_event(ev["comp"][par][gi])
+                hO[l0:l1].copy_(dOut[par, l0:l1], non_blocking=True)
+                ev["out"][par][gi].record(d2h_stream)
+            used[par][gi] = True
+
+    def drain():
+        for par in range(2):
+            for gi in range(len(groups)):
+                if used[par][gi]:
+                    stream.wait_event(ev["out"][par][gi])
 
     with torch.cuda.stream(stream):
         for i in range(3):
-            e2e_step(i % nsched)
+            e2e_step(i, i % nsched)
+        drain()
         barrier()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(stream)
+        h2d_stream.wait_stream(stream)
+        d2h_stream.wait_stream(stream)
         for i in range(e2e_steps):
-            e2e_step((3 + i) % nsched)
+            e2e_step(3 + i, (3 + i) % nsched)
+        drain()
         f1.record(stream)
     barrier()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
     e2e_value = world * B * e2e_steps / (e2e_ms / 1e3)
-    h2d = (dK.numel() + dV.numel() + dQ.numel()) * 2
+    h2d = NL * per * 2
     d2h = out.numel() * 2
     status = kvq.kvq_device_status(cache.h, stream)
 
