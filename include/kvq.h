@@ -126,6 +126,18 @@ KVQ_API int kvq_bind(kvq_handle *h, void *dev_ptr, size_t bytes);
  * launch.  n_new >= 1; returns KVQ_ECAPACITY beyond max_ctx. */
 KVQ_API int kvq_append(kvq_handle *h, int layer, const void *K, const void *V, int n_new, void *stream);
 
+/* Append n_new[b] tokens to sequence b of `layer` (0 <= n_new[b] <= n_max; n_new is a
+ * host array of batch entries): K, V bf16 [B][Hkv][n_max][D] (device), request b's
+ * tokens in its first n_new[b] slots.  Sequences may then differ in length (ragged
+ * batches); every other entry point works per request from then on: decode attends
+ * over each sequence's own tokens, kvq_append_decode appends one token to each,
+ * kvq_export_layer exports each unit at its own length, kvq_truncate cuts every
+ * sequence to the same length.  Plans with more than 64 requests accept only equal
+ * lengths (KVQ_EUNSUPPORTED): the per-request lengths travel in the kernels' parameters.
+ * Errors as kvq_append, plus KVQ_EINVAL for a count outside [0, n_max]. */
+KVQ_API int kvq_append_ragged(kvq_handle *h, int layer, const void *K, const void *V, const int32_t *n_new,
+                              int n_max, void *stream);
+
 /* Paged plans (desc.paged = 1; head_dim 128, G in {1, 2, 4}, batch <= 64): append n_new
  * tokens per request with their tags, 2 (INT2) or 4 (INT4), given twice: host_tags
  * [B][n_new] for the host-side page planning, dev_tags (same bytes, device) for the
@@ -177,11 +189,16 @@ KVQ_API int kvq_get_num_splits(const kvq_handle *h, int layer, int *num_splits);
 KVQ_API int kvq_export_layer(const kvq_handle *h, int layer, void *host_buf, size_t bytes,
                      size_t *needed);
 
-/* Current length L of `layer`. */
+/* Current length L of `layer` (the largest over its sequences). */
 KVQ_API int kvq_seq_len(const kvq_handle *h, int layer, int *L);
 
-/* Shorten `layer` to L tokens (host bookkeeping only).  L <= current length and
- * L % 32 == 0 (so no token of a kept block is partially overwritten later). */
+/* Current length of every sequence of `layer`: L host int32 [batch].  Per-layer plans
+ * only (paged plans: KVQ_EUNSUPPORTED). */
+KVQ_API int kvq_seq_lens(const kvq_handle *h, int layer, int32_t *L);
+
+/* Shorten every sequence of `layer` to L tokens (host bookkeeping only).  L <= the
+ * shortest sequence and L % 32 == 0 (so no token of a kept block is partially
+ * overwritten later). */
 KVQ_API int kvq_truncate(kvq_handle *h, int layer, int L);
 
 /* Read and clear the device status word (synchronizes `stream`).  KVQ_EDEVICE if a

@@ -36,14 +36,14 @@ constexpr int kMaxD = 256;
 
 // Per-token quantization of the new tokens of one 16-token half-block and repacking
 // of its words.  role 0 = keys (per-token mode), 1 = values.
-__device__ void per_token_half(const AppendParams &p, int role, int unit, int hbi,
+__device__ void per_token_half(const AppendParams &p, int role, int unit, int hbi, int L_old, int n,
                                uint8_t (*codes)[kMaxD], unsigned *cta_smax) {
     const int D = p.D, nj = D / 32;
     const int bits = role ? p.bv : p.bk;
     const uint16_t *src = (role ? p.V : p.K) + static_cast<long long>(unit) * p.n * D;
-    const int L_new = p.L_old + p.n;
+    const int L_new = L_old + n;
     const int u0 = 16 * hbi;
-    const int es = max(p.L_old, u0) - u0, ee = min(L_new, u0 + 16) - u0;
+    const int es = max(L_old, u0) - u0, ee = min(L_new, u0 + 16) - u0;
     const int blk = hbi >> 1, eta = hbi & 1;
     uint8_t *rec = p.rec + (static_cast<long long>(unit) * p.cap_blk + blk) * p.rec_bytes;
     uint8_t *sz = rec + (role ? p.kc + p.ks + p.vc : p.kc);
@@ -65,7 +65,7 @@ __device__ void per_token_half(const AppendParams &p, int role, int unit, int hb
     for (int it = warp; it < (ee - es) * nj; it += kWarps) {
         const int e = es + it / nj, j = it % nj;
         const int tok = u0 + e;
-        const uint16_t *row = src + static_cast<long long>(tok - p.L_old) * D;
+        const uint16_t *row = src + static_cast<long long>(tok - L_old) * D;
         const int u = 16 * eta + e;
         {
             const float x = bf16_to_f32(row[32 * j + lane]);
@@ -112,18 +112,17 @@ __device__ void per_token_half(const AppendParams &p, int role, int unit, int hb
 
 // Per-channel quantization of one completed 32-token key group; the CTA with
 // first == true also writes the new residual tokens of its (b, h) afterwards.
-__device__ void per_channel_group(const AppendParams &p, int unit, int q, bool do_group, bool first,
-                                  float (*xs)[kMaxD], uint8_t (*codes)[kMaxD], unsigned *cta_smax) {
+__device__ void per_channel_group(const AppendParams &p, int unit, int q, bool do_group, bool first, int L_old,
+                                  int n, float (*xs)[kMaxD], uint8_t (*codes)[kMaxD], unsigned *cta_smax) {
     const int D = p.D;
     const uint16_t *src = p.K + static_cast<long long>(unit) * p.n * D;
     uint16_t *res = p.res + static_cast<long long>(unit) * 32 * D;
-    const int L_new = p.L_old + p.n;
+    const int L_new = L_old + n;
     if (do_group) {
         const int t0 = 32 * q;
         for (int idx = threadIdx.x; idx < 32 * D; idx += kThreads) {
             const int u = idx / D, d = idx % D, tok = t0 + u;
-            const uint16_t v = tok < p.L_old ? res[u * D + d]
-                                             : src[static_cast<long long>(tok - p.L_old) * D + d];
+            const uint16_t v = tok < L_old ? res[u * D + d] : src[static_cast<long long>(tok - L_old) * D + d];
             xs[u][d] = bf16_to_f32(v);
         }
         __syncthreads();
@@ -161,11 +160,11 @@ __device__ void per_channel_group(const AppendParams &p, int unit, int q, bool d
         __syncthreads();   // the residual reads above complete before the rewrite below
     }
     if (first) {
-        const int res_start = max(p.L_old, 32 * (L_new / 32));
+        const int res_start = max(L_old, 32 * (L_new / 32));
         const int cnt = L_new - res_start;
         for (int idx = threadIdx.x; idx < cnt * D; idx += kThreads) {
             const int tok = res_start + idx / D, d = idx % D;
-            res[(tok % 32) * D + d] = src[static_cast<long long>(tok - p.L_old) * D + d];
+            res[(tok % 32) * D + d] = src[static_cast<long long>(tok - L_old) * D + d];
         }
     }
 }
@@ -181,21 +180,40 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams p) {
     if (threadIdx.x == 0) cta_smax = 0;
     __syncthreads();
     const int cta = blockIdx.x;
-    int role;
+    // this CTA's request range: the launch's own, or (ragged) its request's
+    auto range = [&](int unit, int &L_old, int &n, int &hb0, int &nhb, int &g0, int &ng) {
+        if (!p.ragged) {
+            L_old = p.L_old, n = p.n, hb0 = p.hb0, nhb = p.nhb, g0 = p.g0, ng = p.ng;
+            return;
+        }
+        const int b = unit / p.Hkv;
+        L_old = p.L_old_r[b];
+        n = p.n_r[b];
+        const int L_new = L_old + n;
+        hb0 = L_old / 16;
+        nhb = n > 0 ? (L_new - 1) / 16 - hb0 + 1 : 0;
+        g0 = L_old / 32;
+        ng = L_new / 32 - g0;
+    };
+    int role, L_old, n, hb0, nhb, g0, ng;
     if (cta < p.nV) {
         role = 1;
-        const int unit = cta / p.nhb, hbi = p.hb0 + cta % p.nhb;
-        per_token_half(p, 1, unit, hbi, codes, &cta_smax);
+        const int unit = cta / p.nhb, hi = cta % p.nhb;
+        range(unit, L_old, n, hb0, nhb, g0, ng);
+        if (hi < nhb) per_token_half(p, 1, unit, hb0 + hi, L_old, n, codes, &cta_smax);
     } else {
         role = 0;
         const int k = cta - p.nV;
         if (p.kmode == 1) {
-            const int unit = k / p.nhb, hbi = p.hb0 + k % p.nhb;
-            per_token_half(p, 0, unit, hbi, codes, &cta_smax);
+            const int unit = k / p.nhb, hi = k % p.nhb;
+            range(unit, L_old, n, hb0, nhb, g0, ng);
+            if (hi < nhb) per_token_half(p, 0, unit, hb0 + hi, L_old, n, codes, &cta_smax);
         } else {
             const int per_unit = p.ng > 0 ? p.ng : 1;
             const int unit = k / per_unit, qi = k % per_unit;
-            per_channel_group(p, unit, p.g0 + qi, p.ng > 0, qi == 0, xs, codes, &cta_smax);
+            range(unit, L_old, n, hb0, nhb, g0, ng);
+            if (qi < ng || qi == 0)
+                per_channel_group(p, unit, g0 + qi, qi < ng, qi == 0, L_old, n, xs, codes, &cta_smax);
         }
     }
     __syncthreads();

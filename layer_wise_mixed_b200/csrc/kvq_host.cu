@@ -20,7 +20,9 @@ struct kvq_handle {
     kvq_plan_desc desc{};
     std::vector<kvq_layer_cfg> cfg;
     std::vector<LayerGeom> geom;
-    std::vector<int> len;
+    std::vector<int> len;                    // per layer: the largest request length
+    std::vector<std::vector<int>> rlen;      // per-layer plans: per layer, per request
+    std::vector<unsigned> ver;               // per layer: appends since bind (scale-maximum slot)
     int cap_blk = 0;
     long long status_off = 0, smax_off = 0, arrive_off = 0, meta_bytes = 0, part_acc_off = 0, part_ml_off = 0,
               total = 0;
@@ -82,10 +84,10 @@ int check_bound(const kvq_handle *h) {
 int cuda_fail(cudaError_t e, const char *what);
 
 // Per-layer maxima of the fp16 scales {K, V}, kept in two slots by the parity of the
-// sequence length they describe: an operation that leaves a layer at length L writes slot
-// L & 1 (carrying the other slot forward), a decode at length L reads it.  A launch that
-// appends and decodes reads the slot of L - 1, which nothing writes during it.  Paged
-// plans use slot 0 only.
+// layer's append count v: an append reads slot v & 1, writes slot (v + 1) & 1 (carrying
+// the other slot forward) and makes v + 1; a decode reads slot v & 1.  A launch that
+// appends and decodes reads slot v and writes slot v + 1, which nothing else touches
+// during it.  Paged plans use slot 0 only.
 unsigned *smax_slot(const kvq_handle *h, int layer, int parity) {
     return reinterpret_cast<unsigned *>(h->ws + h->smax_off) + 4 * layer + 2 * (parity & 1);
 }
@@ -203,6 +205,7 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
         off = align256(off + rows * kvq::kMaxSplits * 2 * 4);
         h->total = off;
         h->len.assign(d->num_layers, 0);
+    h->ver.assign(d->num_layers, 0u);
         h->pl.assign(d->num_layers, kvq_handle::PagedLayer{});
         for (auto &x : h->pl) {
             x.n2g.assign(d->batch, 0);
@@ -266,6 +269,8 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
     off = align256(off + rows * kvq::kMaxSplits * 2 * 4);
     h->total = off;
     h->len.assign(d->num_layers, 0);
+    h->ver.assign(d->num_layers, 0u);
+    h->rlen.assign(d->num_layers, std::vector<int>(d->batch, 0));
     *out = h;
     return ok();
 }
@@ -285,6 +290,8 @@ int kvq_bind(kvq_handle *h, void *dev_ptr, size_t bytes) {
     h->ws_bytes = bytes;
     h->status_clear = false;
     std::fill(h->len.begin(), h->len.end(), 0);
+    std::fill(h->ver.begin(), h->ver.end(), 0u);
+    for (auto &r : h->rlen) std::fill(r.begin(), r.end(), 0);
     for (auto &x : h->pl) {
         std::fill(x.n2g.begin(), x.n2g.end(), 0);
         std::fill(x.n4.begin(), x.n4.end(), 0);
@@ -296,54 +303,129 @@ int kvq_bind(kvq_handle *h, void *dev_ptr, size_t bytes) {
     return ok();
 }
 
-int kvq_append(kvq_handle *h, int layer, const void *K, const void *V, int n_new, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Whether the requests of a per-layer plan's layer have different lengths.
+bool layer_ragged(const kvq_handle *h, int layer) {
+    const auto &r = h->rlen[layer];
+    return std::any_of(r.begin(), r.end(), [&](int x) { return x != r[0]; });
+}
+
+// Append n[b] tokens to request b (n == nullptr: n_max to every request); K, V hold
+// n_max token slots per (b, kv head).
+int append_impl(kvq_handle *h, int layer, const void *K, const void *V, const int *n, int n_max, void *stream) {
     int rc = check_layer(h, layer);
     if (rc) return rc;
     if ((rc = check_bound(h))) return rc;
     if (!K || !V) return fail(KVQ_EINVAL, "null K or V");
     if (!aligned(K, 16) || !aligned(V, 16)) return fail(KVQ_EALIGN, "K and V must be 16-byte aligned");
-    if (n_new < 1) return fail(KVQ_EINVAL, "n_new must be >= 1 (got %d)", n_new);
+    if (n_max < 1) return fail(KVQ_EINVAL, "n_new must be >= 1 (got %d)", n_max);
     if (h->desc.paged) return fail(KVQ_EINVAL, "paged plans append with kvq_append_tagged");
-    const int L_old = h->len[layer];
-    if (static_cast<long long>(L_old) + n_new > h->desc.max_ctx)
-        return fail(KVQ_ECAPACITY, "layer %d: %d + %d tokens exceed max_ctx %d", layer, L_old, n_new, h->desc.max_ctx);
+    const int B = h->desc.batch;
+    std::vector<int> Lo(h->rlen[layer]), nn(B, n_max);
+    if (n)
+        for (int b = 0; b < B; ++b) {
+            if (n[b] < 0 || n[b] > n_max) return fail(KVQ_EINVAL, "request %d: n_new %d outside [0, %d]", b, n[b], n_max);
+            nn[b] = n[b];
+        }
+    for (int b = 0; b < B; ++b)
+        if (static_cast<long long>(Lo[b]) + nn[b] > h->desc.max_ctx)
+            return fail(KVQ_ECAPACITY, "layer %d request %d: %d + %d tokens exceed max_ctx %d", layer, b, Lo[b], nn[b],
+                        h->desc.max_ctx);
+    const bool uniform = !layer_ragged(h, layer) && std::all_of(nn.begin(), nn.end(), [&](int x) { return x == nn[0]; });
+    if (!uniform && B > kvq::kMaxRagged)
+        return fail(KVQ_EUNSUPPORTED, "requests of different lengths need batch <= %d (got %d)", kvq::kMaxRagged, B);
     const LayerGeom &g = h->geom[layer];
-    const int units = h->desc.batch * h->desc.n_kv_heads;
-    const int L_new = L_old + n_new;
+    const int units = B * h->desc.n_kv_heads;
     kvq::AppendParams p{};
     p.K = static_cast<const uint16_t *>(K);
     p.V = static_cast<const uint16_t *>(V);
-    p.smax = smax_slot(h, layer, L_new);
-    p.smax_prev = smax_slot(h, layer, L_old);
+    p.smax = smax_slot(h, layer, static_cast<int>(h->ver[layer] + 1));
+    p.smax_prev = smax_slot(h, layer, static_cast<int>(h->ver[layer]));
     p.rec = h->ws + g.rec_off;
     p.res = g.res_off >= 0 ? reinterpret_cast<uint16_t *>(h->ws + g.res_off) : nullptr;
-    p.B = h->desc.batch;
+    p.B = B;
     p.Hkv = h->desc.n_kv_heads;
     p.D = h->desc.head_dim;
     p.bk = g.bk;
     p.bv = g.bv;
     p.kmode = g.kmode;
-    p.L_old = L_old;
-    p.n = n_new;
+    p.n = n_max;
     p.cap_blk = h->cap_blk;
     p.rec_bytes = g.rec_bytes;
     p.kc = g.kc;
     p.ks = g.ks;
     p.vc = g.vc;
-    p.hb0 = L_old / 16;
-    p.nhb = (L_new - 1) / 16 - p.hb0 + 1;
-    p.g0 = L_old / 32;
-    p.ng = L_new / 32 - L_old / 32;
+    if (uniform) {
+        const int L_old = Lo[0], L_new = L_old + nn[0];
+        p.L_old = L_old;
+        p.hb0 = L_old / 16;
+        p.nhb = nn[0] > 0 ? (L_new - 1) / 16 - p.hb0 + 1 : 0;
+        p.g0 = L_old / 32;
+        p.ng = L_new / 32 - L_old / 32;
+        if (nn[0] != n_max) {   // every request appends the same n < n_max: the ragged path
+            p.ragged = 1;
+        }
+    } else {
+        p.ragged = 1;
+    }
+    if (p.ragged) {
+        int nhb = 0, ng = 0;
+        for (int b = 0; b < B; ++b) {
+            p.L_old_r[b] = Lo[b];
+            p.n_r[b] = nn[b];
+            const int L_new = Lo[b] + nn[b];
+            if (nn[b] > 0) nhb = std::max(nhb, (L_new - 1) / 16 - Lo[b] / 16 + 1);
+            ng = std::max(ng, L_new / 32 - Lo[b] / 32);
+        }
+        p.nhb = nhb;
+        p.ng = ng;
+    }
     const long long nV = static_cast<long long>(units) * p.nhb;
     const long long nK = g.kmode == KVQ_PER_TOKEN ? nV : static_cast<long long>(units) * std::max(p.ng, 1);
     if (nV + nK > 0x7FFFFFFFLL) return fail(KVQ_EUNSUPPORTED, "append too large for one launch");
     p.nV = static_cast<int>(nV);
     p.nK = static_cast<int>(nK);
+    if (p.nV + p.nK == 0) return ok();   // no token appended: nothing changes (the slot neither)
     if ((rc = prepare_status(h, static_cast<cudaStream_t>(stream)))) return rc;
     cudaError_t e = kvq::launch_append(p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
-    h->len[layer] = L_new;
+    int mx = 0;
+    for (int b = 0; b < B; ++b) {
+        h->rlen[layer][b] = Lo[b] + nn[b];
+        mx = std::max(mx, h->rlen[layer][b]);
+    }
+    h->len[layer] = mx;
+    ++h->ver[layer];
     return ok();
+}
+
+// Decode parameters' per-request lengths (ragged layers); false if a request is empty.
+bool fill_lengths(const kvq_handle *h, int layer, kvq::DecodeParams &p) {
+    p.ragged = 0;
+    if (!layer_ragged(h, layer)) return true;
+    p.ragged = 1;
+    for (int b = 0; b < h->desc.batch; ++b) {
+        if (h->rlen[layer][b] < 1) return false;
+        p.lens[b] = h->rlen[layer][b];
+    }
+    return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvq_append(kvq_handle *h, int layer, const void *K, const void *V, int n_new, void *stream) {
+    return append_impl(h, layer, K, V, nullptr, n_new, stream);
+}
+
+int kvq_append_ragged(kvq_handle *h, int layer, const void *K, const void *V, const int32_t *n_new, int n_max,
+                      void *stream) {
+    if (!n_new) return fail(KVQ_EINVAL, "null n_new");
+    return append_impl(h, layer, K, V, n_new, n_max, stream);
 }
 
 int kvq_append_tagged(kvq_handle *h, int layer, const void *K, const void *V, int n_new,
@@ -622,7 +704,8 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
     p.rec = h->ws + g.rec_off;
     p.res = g.res_off >= 0 ? reinterpret_cast<const uint16_t *>(h->ws + g.res_off) : nullptr;
     p.q = static_cast<const uint16_t *>(q);
-    p.smax = smax_slot(h, layer, L);
+    p.smax = smax_slot(h, layer, static_cast<int>(h->ver[layer]));
+    if (!fill_lengths(h, layer, p)) return fail(KVQ_EINVAL, "layer %d: a request is empty", layer);
     p.out = out;
     p.part_acc = reinterpret_cast<float *>(h->ws + h->part_acc_off);
     p.part_ml = reinterpret_cast<float *>(h->ws + h->part_ml_off);
@@ -669,15 +752,23 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
         return fail(KVQ_EALIGN, "K, V, q and out must be 16-byte aligned");
     if (h->desc.paged) return fail(KVQ_EINVAL, "paged plans append with kvq_append_tagged");
     const int L_old = h->len[layer];
-    if (static_cast<long long>(L_old) + 1 > h->desc.max_ctx)
-        return fail(KVQ_ECAPACITY, "layer %d: %d + 1 tokens exceed max_ctx %d", layer, L_old, h->desc.max_ctx);
+    const int B = h->desc.batch;
+    for (int b = 0; b < B; ++b)
+        if (static_cast<long long>(h->rlen[layer][b]) + 1 > h->desc.max_ctx)
+            return fail(KVQ_ECAPACITY, "layer %d request %d: %d + 1 tokens exceed max_ctx %d", layer, b,
+                        h->rlen[layer][b], h->desc.max_ctx);
     const LayerGeom &g = h->geom[layer];
     const int L = L_old + 1;
-    if (g.kmode == KVQ_PER_CHANNEL && L % 32 == 0) {
-        // the token completes a key group: the group is quantized by the append kernel
+    bool completes = false;   // the token completes some request's key group
+    for (int b = 0; b < B; ++b) completes = completes || (h->rlen[layer][b] + 1) % 32 == 0;
+    if (g.kmode == KVQ_PER_CHANNEL && completes) {
+        // the group is quantized by the append kernel
         if ((rc = kvq_append(h, layer, K, V, 1, stream))) return rc;
         return kvq_decode_attn(h, layer, q, out, out_fp32, stream);
     }
+    const bool ragged = layer_ragged(h, layer);
+    if (ragged && B > kvq::kMaxRagged)
+        return fail(KVQ_EUNSUPPORTED, "requests of different lengths need batch <= %d (got %d)", kvq::kMaxRagged, B);
     h->len[layer] = L;   // the schedule is chosen for the new length
     int S = 1, nstage = 2, nextra = 0;
     if ((rc = splits_for(h, layer, &S, &nstage, &nextra))) {
@@ -689,7 +780,9 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
     p.rec = h->ws + g.rec_off;
     p.res = g.res_off >= 0 ? reinterpret_cast<const uint16_t *>(h->ws + g.res_off) : nullptr;
     p.q = static_cast<const uint16_t *>(q);
-    p.smax = smax_slot(h, layer, L_old);
+    p.smax = smax_slot(h, layer, static_cast<int>(h->ver[layer]));
+    p.ragged = ragged ? 1 : 0;
+    for (int b = 0; ragged && b < B; ++b) p.lens[b] = h->rlen[layer][b] + 1;
     p.out = out;
     p.part_acc = reinterpret_cast<float *>(h->ws + h->part_acc_off);
     p.part_ml = reinterpret_cast<float *>(h->ws + h->part_ml_off);
@@ -710,7 +803,7 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
     p.v_new = static_cast<const uint16_t *>(V);
     p.rec_w = h->ws + g.rec_off;
     p.res_w = g.res_off >= 0 ? reinterpret_cast<uint16_t *>(h->ws + g.res_off) : nullptr;
-    p.smax_out = smax_slot(h, layer, L);
+    p.smax_out = smax_slot(h, layer, static_cast<int>(h->ver[layer] + 1));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = prepare_status(h, st))) {
         h->len[layer] = L_old;
@@ -721,6 +814,8 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
         h->len[layer] = L_old;
         return cuda_fail(e, "fused append + decode launch");
     }
+    for (int b = 0; b < B; ++b) ++h->rlen[layer][b];
+    ++h->ver[layer];
     if (p.S > 1 && !p.arrive) {
         kvq::MergeParams m{};
         m.part_acc = p.part_acc;
@@ -842,24 +937,24 @@ int kvq_export_layer(const kvq_handle *h, int layer, void *host_buf, size_t byte
     if (!needed) return fail(KVQ_EINVAL, "null argument");
     if (h->desc.paged) return export_paged(h, layer, host_buf, bytes, needed);
     const LayerGeom &g = h->geom[layer];
-    const int L = h->len[layer];
-    const int nblk = (L + 31) / 32;
-    const int D = h->desc.head_dim;
+    const int D = h->desc.head_dim, Hkv = h->desc.n_kv_heads;
     const long long res_bytes = g.kmode == KVQ_PER_CHANNEL ? 64LL * D : 0;
-    const long long unit_img = nblk * g.rec_bytes + res_bytes;
-    const int units = h->desc.batch * h->desc.n_kv_heads;
-    *needed = static_cast<size_t>(unit_img * units);
+    const int units = h->desc.batch * Hkv;
+    auto unit_len = [&](int u) { return h->rlen[layer][u / Hkv]; };
+    auto unit_img = [&](int u) { return (unit_len(u) + 31) / 32 * g.rec_bytes + res_bytes; };
+    long long total = 0;
+    for (int u = 0; u < units; ++u) total += unit_img(u);
+    *needed = static_cast<size_t>(total);
     if (!host_buf) return ok();
     if (bytes < *needed) return fail(KVQ_EINVAL, "export buffer too small: %zu < %zu", bytes, *needed);
     if ((rc = check_bound(h))) return rc;
     if (!h->status_clear) return fail(KVQ_EINVAL, "nothing appended since the workspace was bound");
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-    uint8_t *dst = static_cast<uint8_t *>(host_buf);
-    const int r = L % 32;
+    uint8_t *img = static_cast<uint8_t *>(host_buf);
     const int nj = D / 32;
-    for (int u = 0; u < units; ++u) {
-        uint8_t *img = dst + u * unit_img;
+    for (int u = 0; u < units; img += unit_img(u), ++u) {
+        const int L = unit_len(u), nblk = (L + 31) / 32, r = L % 32;
         if (nblk > 0) {
             e = cudaMemcpy(img, h->ws + g.rec_off + u * g.unit_bytes, nblk * g.rec_bytes, cudaMemcpyDeviceToHost);
             if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy (records)");
@@ -903,13 +998,24 @@ int kvq_seq_len(const kvq_handle *h, int layer, int *L) {
     return ok();
 }
 
+int kvq_seq_lens(const kvq_handle *h, int layer, int32_t *L) {
+    int rc = check_layer(h, layer);
+    if (rc) return rc;
+    if (!L) return fail(KVQ_EINVAL, "null argument");
+    if (h->desc.paged) return fail(KVQ_EUNSUPPORTED, "paged plans report one length per layer");
+    for (int b = 0; b < h->desc.batch; ++b) L[b] = h->rlen[layer][b];
+    return ok();
+}
+
 int kvq_truncate(kvq_handle *h, int layer, int L) {
     int rc = check_layer(h, layer);
     if (rc) return rc;
-    if (L < 0 || L > h->len[layer]) return fail(KVQ_EINVAL, "truncate length %d outside [0, %d]", L, h->len[layer]);
-    if (L % 32) return fail(KVQ_EINVAL, "truncate length must be a multiple of 32 (got %d)", L);
     if (h->desc.paged) return fail(KVQ_EUNSUPPORTED, "paged plans cannot be truncated");
+    const int shortest = *std::min_element(h->rlen[layer].begin(), h->rlen[layer].end());
+    if (L < 0 || L > shortest) return fail(KVQ_EINVAL, "truncate length %d outside [0, %d]", L, shortest);
+    if (L % 32) return fail(KVQ_EINVAL, "truncate length must be a multiple of 32 (got %d)", L);
     h->len[layer] = L;
+    std::fill(h->rlen[layer].begin(), h->rlen[layer].end(), L);
     return ok();
 }
 
@@ -998,7 +1104,8 @@ int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, 
     p.rec = h->ws + g.rec_off;
     p.res = g.res_off >= 0 ? reinterpret_cast<const uint16_t *>(h->ws + g.res_off) : nullptr;
     p.q = static_cast<const uint16_t *>(q);
-    p.smax = smax_slot(h, layer, L);
+    p.smax = smax_slot(h, layer, static_cast<int>(h->ver[layer]));
+    if (!fill_lengths(h, layer, p)) return fail(KVQ_EINVAL, "layer %d: a request is empty", layer);
     p.out = out;
     p.part_acc = static_cast<float *>(scratch);
     p.part_ml = reinterpret_cast<float *>(static_cast<unsigned char *>(scratch) + acc_bytes);

@@ -36,6 +36,8 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 
 constexpr int kGroup = 32;          // quantization group (tokens or channels)
 constexpr int kMaxSplits = 64;      // partial slots per (batch, query head)
+constexpr int kMaxRagged = 64;      // requests per per-layer plan with per-request lengths
+                                    // (kernel-parameter tables)
 constexpr int kDecodeWarps = 4;     // warps per decode CTA
 
 // Device status word bits (written with atomicOr, read by kvq_device_status).
@@ -52,7 +54,8 @@ struct LayerGeom {
 };
 
 struct AppendParams {
-    const uint16_t *K, *V;      // bf16 [B][Hkv][n][D]
+    const uint16_t *K, *V;      // bf16 [B][Hkv][n][D] (ragged: n = the largest count, request b
+                                // uses its first n_r[b] tokens)
     unsigned *smax;             // {max key scale, max value scale} (fp16 bits) at the new length
     const unsigned *smax_prev;  // the same at the old length (other parity slot), or smax
     uint8_t *rec;               // layer records [B][Hkv][cap][rec_bytes]
@@ -63,6 +66,11 @@ struct AppendParams {
     int hb0, nhb;               // first touched 16-token half-block, count per unit
     int g0, ng;                 // first completed key group, count per unit
     int nV, nK;                 // CTA counts of the two roles
+    // per-request lengths (ragged != 0): request b appends n_r[b] tokens at L_old_r[b];
+    // nhb and ng are then the largest counts over the requests (grid sizing) and each CTA
+    // derives its request's own range, idling when it has none
+    int ragged;
+    int L_old_r[kMaxRagged], n_r[kMaxRagged];
 };
 
 struct DecodeParams {
@@ -78,6 +86,10 @@ struct DecodeParams {
     unsigned *status;
     int B, Hkv, G, L, cap_blk, S, bps, out_fp32;
     int nstage, nextra;         // stages per warp; one more for warps 0 .. nextra - 1
+    // per-request lengths (ragged != 0): request b has lens[b] tokens (L above is the
+    // largest, which sets the split partition)
+    int ragged;
+    int lens[kMaxRagged];
     long long rec_bytes;
     // Fused one-token append (kvq_append_decode), null otherwise: the new token's K and V
     // rows (bf16 [B][Hkv][D]), now token L - 1; writable records and residual; the

@@ -68,6 +68,8 @@ def load() -> ctypes.CDLL:
         "kvq_bind": (I, [P, P, SZ]),
         "kvq_append": (I, [P, I, P, P, I, P]),
         "kvq_append_tagged": (I, [P, I, P, P, I, P, P, P]),
+        "kvq_append_ragged": (I, [P, I, P, P, P, I, P]),
+        "kvq_seq_lens": (I, [P, I, P]),
         "kvq_decode_attn": (I, [P, I, P, P, I, P]),
         "kvq_append_decode": (I, [P, I, P, P, P, P, I, P]),
         "kvq_decode_attn_noalloc": (I, [P, I, P, P, I, P]),
@@ -141,6 +143,21 @@ def kvq_append_tagged(h: int, layer: int, K, V, n_new: int, host_tags, dev_tags,
     host_tags = np.ascontiguousarray(host_tags, np.uint8)
     _check(load().kvq_append_tagged(h, layer, _ptr(K), _ptr(V), n_new, host_tags.ctypes.data_as(ctypes.c_void_p),
                                     _ptr(dev_tags), _stream(stream)))
+
+
+def kvq_append_ragged(h: int, layer: int, K, V, n_new, stream=None):
+    """K, V [B, Hkv, n_max, D]; request b appends its first n_new[b] tokens."""
+    import numpy as np
+    n = np.ascontiguousarray(n_new, np.int32)
+    _check(load().kvq_append_ragged(h, layer, _ptr(K), _ptr(V), n.ctypes.data_as(ctypes.c_void_p), K.shape[2],
+                                    _stream(stream)))
+
+
+def kvq_seq_lens(h: int, layer: int, batch: int):
+    import numpy as np
+    out = np.zeros(batch, np.int32)
+    _check(load().kvq_seq_lens(h, layer, out.ctypes.data_as(ctypes.c_void_p)))
+    return out
 
 
 def kvq_decode_attn(h: int, layer: int, q, out, out_fp32: bool, stream=None):
@@ -298,6 +315,14 @@ class Cache:
                               device=q.device)
         kvq_append_decode(self.h, layer, K, V, q, out, out_fp32, stream)
         return out
+
+    def append_ragged(self, layer, K, V, n_new, stream=None):
+        """K, V [B, Hkv, n_max, D] (contiguous); request b appends its first n_new[b] tokens."""
+        assert K.is_contiguous() and V.is_contiguous() and K.shape == V.shape
+        kvq_append_ragged(self.h, layer, K, V, n_new, stream)
+
+    def seq_lens(self, layer):
+        return kvq_seq_lens(self.h, layer, self.B)
 
     def export_layer(self, layer):
         return kvq_export_layer(self.h, layer)
