@@ -111,3 +111,18 @@ def test_ragged_truncate_and_equal_again():
     r.check(inputs.step_q(r.wl, 0, 3, "cuda"), splits=(0, 2), what="truncated")
     with pytest.raises(kvq.KvqError):
         kvq.kvq_truncate(r.cache.h, 0, 64)      # longer than the sequences
+
+
+@pytest.mark.parametrize("splits", [1, 3, 5])
+def test_ragged_noalloc_matches_workspace_entry(splits):
+    """The entry point without caller scratch gives the same bytes on a ragged layer."""
+    r = Ragged(4, 2, 4, 128, (8, 4), 0, 400, f"ragnoalloc{splits}")
+    r.append([130, 33, 200, 1])
+    kvq.kvq_set_num_splits(r.cache.h, splits)
+    q = inputs.step_q(r.wl, 0, 9, "cuda")
+    a = r.cache.decode_attn(0, q, out_fp32=True)
+    b = torch.empty_like(a)
+    kvq.kvq_decode_attn_noalloc(r.cache.h, 0, q, b, True)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    r.check(q, splits=(splits,), what="noalloc")
