@@ -123,7 +123,7 @@ KVQ_API int kvq_bind(kvq_handle *h, void *dev_ptr, size_t bytes);
 /* Append n_new tokens to every sequence of `layer`: K, V are bf16 [B][Hkv][n_new][D]
  * (device).  Quantizes values per token, keys per channel (completing 32-token groups
  * from residual + new tokens; the rest goes to the residual) or per token.  One kernel
- * launch.  n_new >= 1; returns KVQ_ECAPACITY beyond max_ctx. */
+ * launch.  n_new >= 1; returns KVQ_ECAPACITY beyond max_ctx (for any sequence). */
 KVQ_API int kvq_append(kvq_handle *h, int layer, const void *K, const void *V, int n_new, void *stream);
 
 /* Append n_new[b] tokens to sequence b of `layer` (0 <= n_new[b] <= n_max; n_new is a
@@ -167,8 +167,9 @@ KVQ_API int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, 
  * and errors as kvq_append(..., n_new = 1, ...) followed by kvq_decode_attn.  The CTA
  * that decodes a sequence's last block first quantizes and packs the new token into it
  * (the pages apply quantize-and-pack and decode attention per step; fusing them is this
- * library's choice).  A token that completes a 32-token per-channel key group takes the
- * two-launch path, since the whole group is quantized then.  Per-layer plans only
+ * library's choice).  A token that completes a 32-token per-channel key group (of any
+ * sequence) takes the two-launch path, since the whole group is quantized then.  On a
+ * ragged layer each sequence gets one token at its own length.  Per-layer plans only
  * (paged plans: KVQ_EINVAL). */
 KVQ_API int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, const void *q,
                               void *out, int out_fp32, void *stream);
