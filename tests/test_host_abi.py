@@ -111,6 +111,41 @@ def test_argument_checks_before_any_launch(lib):
         kvq.kvq_destroy(h)
 
 
+def test_ragged_argument_checks_before_any_launch(lib):
+    import numpy as np
+    L = kvq.load()
+    h = kvq.kvq_plan(desc())                         # batch 2, max_ctx 100
+    try:
+        fake = 1 << 40
+        assert L.kvq_bind(h, fake, kvq.kvq_workspace_bytes(h)) == kvq.KVQ_OK
+        p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+        assert L.kvq_append_ragged(h, 0, fake, fake, None, 4, None) == kvq.KVQ_EINVAL            # null counts
+        assert L.kvq_append_ragged(h, 0, fake, fake, p(np.array([5, 1], np.int32)), 4, None) == kvq.KVQ_EINVAL
+        assert L.kvq_append_ragged(h, 0, fake, fake, p(np.array([-1, 1], np.int32)), 4, None) == kvq.KVQ_EINVAL
+        assert L.kvq_append_ragged(h, 0, fake, fake, p(np.array([1, 101], np.int32)), 120, None) == kvq.KVQ_ECAPACITY
+        assert "request 1" in kvq.kvq_last_error()
+        assert L.kvq_append_ragged(h, 0, fake, fake, p(np.array([1, 1], np.int32)), 0, None) == kvq.KVQ_EINVAL
+        assert list(kvq.kvq_seq_lens(h, 0, 2)) == [0, 0]
+    finally:
+        kvq.kvq_destroy(h)
+    h = kvq.kvq_plan(desc(batch=65))                 # different lengths need batch <= 64
+    try:
+        fake = 1 << 40
+        assert L.kvq_bind(h, fake, kvq.kvq_workspace_bytes(h)) == kvq.KVQ_OK
+        counts = np.ones(65, np.int32)
+        counts[3] = 2
+        assert L.kvq_append_ragged(h, 0, fake, fake, counts.ctypes.data_as(ctypes.c_void_p), 2, None) == \
+            kvq.KVQ_EUNSUPPORTED
+    finally:
+        kvq.kvq_destroy(h)
+    h = kvq.kvq_plan(kvq.make_paged_desc(1, 2, 2, 8, 128, 64, 3.0))
+    try:
+        with pytest.raises(kvq.KvqError):
+            kvq.kvq_seq_lens(h, 0, 2)
+    finally:
+        kvq.kvq_destroy(h)
+
+
 def test_product_path_has_no_fallback(monkeypatch, tmp_path):
     """Without libkvq.so the binding raises; it never computes anything itself."""
     monkeypatch.setattr(kvq, "LIB_PATH", str(tmp_path / "missing.so"))
