@@ -242,8 +242,9 @@ KVQ_API int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, voi
  * the exact keys and values, per query head; D_k(b) = sum over layers of the mean over
  * requests of the max over query heads.  Tags with no token get 0.  counts[k] receives
  * the number of tokens of tag k over all requests.  Cost O(layers x requests x tags x
- * n_q_heads x T^2 x head_dim), spread over the host's cores: a calibration tool for
- * prefills of up to a few thousand tokens.  Errors: KVQ_EINVAL (counts, shapes: head_dim
+ * n_q_heads x T^2 x head_dim), spread over the host's cores (as many as keep the
+ * workers' T x T fp64 score buffers within about 2 GB): a calibration tool for prefills
+ * of up to a few thousand tokens.  Errors: KVQ_EINVAL (counts, shapes: head_dim
  * a multiple of 32, n_q_heads a multiple of n_kv_heads; tags out of range; null). */
 KVQ_API int kvq_tag_distortion(int num_layers, int num_requests, int n_q_heads, int n_kv_heads, int head_dim,
                                int T, const uint16_t *Q, const uint16_t *K, const uint16_t *V,

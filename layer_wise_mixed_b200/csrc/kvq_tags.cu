@@ -188,7 +188,11 @@ int kvq_tag_distortion(int num_layers, int num_requests, int n_q_heads, int n_kv
             }
         }
     };
-    const unsigned nth = std::max(1u, std::min(std::thread::hardware_concurrency(), 64u));
+    // threads: the host's cores, at most 64, and as many as keep every worker's buffers
+    // (the T x T fp64 scores and ~10 T x D rows) within about 2 GB
+    const double per_thread = 8.0 * (static_cast<double>(T) * T + 12.0 * static_cast<double>(TD));
+    const unsigned by_mem = static_cast<unsigned>(std::max(1.0, std::floor(2.0e9 / per_thread)));
+    const unsigned nth = std::max(1u, std::min({std::thread::hardware_concurrency(), 64u, by_mem}));
     std::vector<std::thread> pool;
     for (unsigned i = 1; i < nth; ++i) pool.emplace_back(work);
     work();
