@@ -526,6 +526,17 @@ def main():
                "kind": "oracle",
                "sample": (f"{len(v_cpu)} x (quantize + fp64 attention of 1 layer, {min(B, args.ref_seqs)} of {B} "
                           f"sequences, context {L_mid}), {t_cpu:.1f} s CPU, scaled to a full step")}
+        # the same sample on one thread (about 3 s)
+        import oracle
+        threads = oracle.set_threads(0)
+        oracle.set_threads(1)
+        t1, v1 = 0.0, []
+        while t1 < 3.0:
+            s_, v_ = cpu_oracle_sample(wl, L_mid, max(1, min(B, args.ref_seqs)))
+            t1 += s_
+            v1.append(v_)
+        oracle.set_threads(threads)
+        cpu["single_thread"] = {"value": len(v1) / sum(1 / v for v in v1), "unit": "tokens/s", "cores": 1}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,

@@ -78,6 +78,8 @@ def lib():
         L.orc_f32_to_f16_array.argtypes = [P, P, i64]
         L.orc_f16_to_f64_array.restype = None
         L.orc_f16_to_f64_array.argtypes = [P, P, i64]
+        L.orc_set_threads.restype = i32
+        L.orc_set_threads.argtypes = [i32]
         L.orc_quant_groups.restype = None
         L.orc_quant_groups.argtypes = [P, i64, i32, P, P, P]
         L.orc_format_version.restype = i32
@@ -116,6 +118,12 @@ def f16_bits_to_f64(h) -> np.ndarray:
 def bf16_bits_to_f32(b) -> np.ndarray:
     b = _u16(b)
     return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def set_threads(n: int) -> int:
+    """Threads of the oracle's OpenMP loops (n <= 0: default); returns the count in use.
+    Timing only: results do not depend on it."""
+    return int(lib().orc_set_threads(int(n)))
 
 
 def quant_groups(x, bits: int):

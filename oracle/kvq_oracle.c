@@ -608,6 +608,22 @@ int orc_layer(const uint16_t *K, const uint16_t *V, const uint16_t *Q, int B, in
     return err ? -1 : 0;
 }
 
+/* ---------------- threads (timing only; no effect on any result) ---------------- */
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+/* Threads of the OpenMP loops above (n <= 0: the runtime's default); returns the count. */
+int orc_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
 /* ---------------- exported scalar helpers (for pins) ---------------- */
 
 void orc_f32_to_f16_array(const float *x, uint16_t *out, long n) {
