@@ -215,3 +215,33 @@ def test_distortion_argument_checks():
         kvq.kvq_tag_distortion(Q, K, K, np.full((1, 4), 3, np.int32), 3)      # tag out of range
     with pytest.raises(kvq.KvqError):
         kvq.kvq_tag_distortion(Q[..., :48], K[..., :48], K[..., :48], np.zeros((1, 4), np.int32), 1)   # D % 32
+
+
+def test_segment_tag_ids_recipe():
+    """Synthetic tag ids: segments of 16-256 tokens sharing one id in [0, 56), the
+    temporal axis being the quarter of the sequence the segment starts in."""
+    from layer_wise_mixed_b200 import configs, inputs
+    w = configs.by_name("c5-alloc")
+    ids = inputs.tag_ids(w, 3000, batch=3).numpy()
+    assert ids.min() >= 0 and ids.max() < 56
+    for row in ids:
+        cuts = np.flatnonzero(np.diff(row)) + 1
+        starts = np.concatenate([[0], cuts])
+        lens = np.diff(np.concatenate([starts, [len(row)]]))
+        assert np.all(lens[:-1] >= 16)           # a run may span segments that drew one id
+        for s0 in starts:                        # every run starts a segment: id // 14 = its quarter
+            assert row[s0] // 14 == min(3, 4 * s0 // len(row))
+    assert np.array_equal(ids, inputs.tag_ids(w, 3000, batch=3).numpy())   # seeded
+
+
+def test_allocation_mask_meets_budget():
+    """The workload's INT2/INT4 mask from the per-tag allocation keeps the average bits at
+    or under the workload's budget, and every token takes its tag's bits."""
+    from layer_wise_mixed_b200 import configs, inputs, tagalloc
+    w = configs.by_name("c5-alloc")
+    m = tagalloc.token_mask(w, w.max_ctx).numpy()
+    assert set(np.unique(m)) <= {2, 4}
+    assert m.astype(np.float64).mean() <= w.avg_bits + 1e-12
+    ids = inputs.tag_ids(w, w.max_ctx).numpy()
+    bits = tagalloc.tag_bits(w)
+    assert np.array_equal(m, bits[ids])
