@@ -247,6 +247,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="c2", choices=["c2", "c2-k8v8", "c2-k8v4", "c3", "c4", "c5", "c5-alloc"])
+    ap.add_argument("--e2e-group", type=int, default=16, help="layers per H2D/D2H transfer group of the e2e loop")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--ref-seqs", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -417,21 +418,22 @@ def main():
         two = paged or (wl.kmode == 0 and Ls[s] % 32 == 0)
         return (2 if two else 1) + (1 if 1 < splits[s][l] < 4 else 0)
     gpu_launches = sum(step_launches(s, l) for s in order for l in range(NL))
-    e2e_note = ("per step and group of 4 layers: pinned H2D of the group's K/V/q (copy stream), "
+    e2e_note = (f"per step and group of {max(1, args.e2e_group)} layers: pinned H2D of the group's K/V/q (copy stream), "
                 "kvq_append_decode per layer (eager C-ABI calls, compute stream), D2H of the group's outputs "
                 "(second copy stream); groups overlap")
     if paged:
-        e2e_note = ("per step and group of 4 layers: pinned H2D of the group's K/V/q, kvq_decode_attn per layer "
+        e2e_note = (f"per step and group of {max(1, args.e2e_group)} layers: pinned H2D of the group's K/V/q, kvq_decode_attn per layer "
                     "(eager C-ABI calls; the cache is not advanced), D2H of the group's outputs; groups overlap")
 
     # ---- e2e: public API with host buffers, H2D + D2H inside the timed region ----
-    # Per step and group of CH layers: one H2D of the group's K|V|q (pinned host, packed per
-    # layer) on a copy stream, the group's C-ABI calls on the compute stream, one D2H of
+    # Per step and group of CH layers (--e2e-group; fewer, larger groups issue fewer copies
+    # and events: measured best at 16 of 32 layers): one H2D of the group's K|V|q (pinned
+    # host, packed per layer) on a copy stream, the group's C-ABI calls on the compute stream, one D2H of
     # the group's outputs on a second copy stream (the other PCIe direction), so that
     # transfers of one group overlap the calls of another; device buffers alternate
     # between even and odd steps.
     e2e_steps = args.e2e_steps or min(args.steps, 64)
-    CH = 4
+    CH = max(1, args.e2e_group)
     groups = [list(range(g0, min(NL, g0 + CH))) for g0 in range(0, NL, CH)]
     nk, nq = B * Hkv * D, B * Hq * D                      # bf16 elements per layer
     per = 2 * nk + nq
