@@ -114,7 +114,7 @@ int kvq_tag_distortion(int num_layers, int num_requests, int n_q_heads, int n_kv
     auto work = [&]() {
         std::vector<float> kf(TD), vf(TD);
         std::vector<double> kx(TD), vx(TD), kq(TD), vq(TD), qd(TD), S(static_cast<size_t>(T) * T), m(T), l(T),
-            N(TD), dN(D);
+            N(TD), dN(D), kxT(TD), kqT, sq;
         for (;;) {
             const long long task = next.fetch_add(1);
             if (task >= ntask) break;
@@ -128,24 +128,32 @@ int kvq_tag_distortion(int num_layers, int num_requests, int n_q_heads, int n_kv
                 kx[i] = kf[i];
                 vx[i] = vf[i];
             }
+            for (int j = 0; j < T; ++j)   // keys channel-major: score rows accumulate as axpys
+                for (int c = 0; c < D; ++c) kxT[static_cast<long long>(c) * T + j] = kx[static_cast<long long>(j) * D + c];
             for (int gg = 0; gg < G; ++gg) {
                 const int hq = h * G + gg;
                 const long long qo = ((static_cast<long long>(lay) * R + r) * n_q_heads + hq) * TD;
                 for (long long i = 0; i < TD; ++i) qd[i] = bf16f(Q[qo + i]);
                 for (int i = 0; i < T; ++i) {
+                    double *Si = S.data() + static_cast<size_t>(i) * T;
+                    for (int j = 0; j <= i; ++j) Si[j] = 0.0;
+                    for (int c = 0; c < D; ++c) {
+                        const double qc = qd[static_cast<long long>(i) * D + c];
+                        const double *kc = kxT.data() + static_cast<long long>(c) * T;
+                        for (int j = 0; j <= i; ++j) Si[j] += qc * kc[j];
+                    }
                     double mx = -INFINITY;
                     for (int j = 0; j <= i; ++j) {
-                        double d = 0.0;
-                        for (int c = 0; c < D; ++c) d += qd[i * D + c] * kx[j * D + c];
-                        S[static_cast<size_t>(i) * T + j] = d * rs;
-                        mx = std::max(mx, d * rs);
+                        Si[j] *= rs;
+                        mx = std::max(mx, Si[j]);
                     }
                     m[i] = mx;
                     double li = 0.0;
                     double *Ni = N.data() + static_cast<long long>(i) * D;
                     for (int c = 0; c < D; ++c) Ni[c] = 0.0;
                     for (int j = 0; j <= i; ++j) {
-                        const double pij = std::exp(S[static_cast<size_t>(i) * T + j] - mx);
+                        const double pij = std::exp(Si[j] - mx);
+                        Si[j] = pij;   // S now holds the exact weights exp(s_ij - m_i)
                         li += pij;
                         for (int c = 0; c < D; ++c) Ni[c] += pij * vx[j * D + c];
                     }
@@ -161,16 +169,30 @@ int kvq_tag_distortion(int num_layers, int num_requests, int n_q_heads, int n_kv
                                 vq[t * D + c] = vx[t * D + c];
                             }
                         quantize_tag(kf.data(), vf.data(), tk, D, bi == 0 ? 2 : 4, kq.data(), vq.data());
+                        // the tag's quantized keys channel-major: a row's scores against its
+                        // first cnt tag tokens accumulate as axpys over those tokens
+                        const int nt = static_cast<int>(tk.size());
+                        kqT.resize(static_cast<size_t>(D) * nt);
+                        sq.resize(nt);
+                        for (int ti = 0; ti < nt; ++ti)
+                            for (int c = 0; c < D; ++c)
+                                kqT[static_cast<size_t>(c) * nt + ti] = kq[static_cast<long long>(tk[ti]) * D + c];
                         double err = 0.0;
+                        int cnt = 0;
                         for (int i = tk[0]; i < T; ++i) {
+                            while (cnt < nt && tk[cnt] <= i) ++cnt;
+                            for (int ti = 0; ti < cnt; ++ti) sq[ti] = 0.0;
+                            for (int c = 0; c < D; ++c) {
+                                const double qc = qd[static_cast<long long>(i) * D + c];
+                                const double *kc = kqT.data() + static_cast<size_t>(c) * nt;
+                                for (int ti = 0; ti < cnt; ++ti) sq[ti] += qc * kc[ti];
+                            }
                             double dl = 0.0;
                             for (int c = 0; c < D; ++c) dN[c] = 0.0;
-                            for (int t : tk) {
-                                if (t > i) break;
-                                double d = 0.0;
-                                for (int c = 0; c < D; ++c) d += qd[i * D + c] * kq[t * D + c];
-                                const double pq = std::exp(d * rs - m[i]);
-                                const double pe = std::exp(S[static_cast<size_t>(i) * T + t] - m[i]);
+                            for (int ti = 0; ti < cnt; ++ti) {
+                                const int t = tk[ti];
+                                const double pq = std::exp(sq[ti] * rs - m[i]);
+                                const double pe = S[static_cast<size_t>(i) * T + t];
                                 dl += pq - pe;
                                 for (int c = 0; c < D; ++c) dN[c] += pq * vq[t * D + c] - pe * vx[t * D + c];
                             }
