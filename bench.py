@@ -52,15 +52,30 @@ def kernel_source_sha256():
 
 
 def captured_traffic(workload_name, alg_bytes_per_launch):
-    """DRAM bytes per launch of the decode kernel from the committed ncu capture, scaled by
-    algorithmic bytes; None when the kernel changed since the capture or the workload differs."""
+    """DRAM bytes per launch of the decode kernel from the committed ncu captures (one
+    block of `key: value` lines per workload, blank-line separated), scaled by algorithmic
+    bytes; None when the kernel changed since the capture or no capture covers the workload."""
     p = os.path.join(ROOT, "profiles", "decode_split_traffic.txt")
     try:
-        kv = dict(ln.split(":", 1) for ln in open(p) if ":" in ln and not ln.startswith("#"))
-        kv = {k.strip(): v.strip() for k, v in kv.items()}
-        if kv["source_sha256"] != kernel_source_sha256() or kv["workload"] != workload_name:
-            return None
-        return float(kv["dram_bytes"]) / float(kv["algorithmic_bytes"]) * alg_bytes_per_launch
+        blocks, cur = [], {}
+        for ln in open(p):
+            if ln.startswith("#"):
+                continue
+            if not ln.strip():
+                if cur:
+                    blocks.append(cur)
+                cur = {}
+                continue
+            if ":" in ln:
+                k, v = ln.split(":", 1)
+                cur[k.strip()] = v.strip()
+        if cur:
+            blocks.append(cur)
+        sha = kernel_source_sha256()
+        for kv in blocks:
+            if kv.get("source_sha256") == sha and kv.get("workload") == workload_name:
+                return float(kv["dram_bytes"]) / float(kv["algorithmic_bytes"]) * alg_bytes_per_launch
+        return None
     except Exception:
         return None
 
@@ -240,6 +255,185 @@ def workload_config(wl):
 
 
 # ---------------------------------------------------------------- GPU arm
+class WorkloadRun:
+    """One workload on the current device: the cache after the prefill, the decode
+    schedule's inputs resident in HBM, and per decode step two CUDA graphs (captured
+    once, untimed): the full step over every layer (fused append + decode launch; a
+    token that completes a per-channel key group: append, then decode; paged plans:
+    tagged append, then decode) and decode alone over every layer."""
+
+    def __init__(self, wl, stream):
+        import numpy as np
+        import torch
+
+        from layer_wise_mixed_b200 import inputs, kvq
+        self.wl, self.stream = wl, stream
+        B, Hkv, Hq, D, NL = wl.batch, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.num_layers
+        self.paged = paged = wl.paged
+        if paged:
+            all_tags = paged_tags(wl, wl.max_ctx)                  # [B, prefill + steps], shared by layers
+            # the pools split at the mask's own mean bits (an allocation may land under its budget)
+            plan_bits = min(wl.avg_bits, 4.0 - 2.0 * float((all_tags == 2).float().mean()))
+            self.cache = kvq.Cache(NL, B, Hkv, Hq, D, wl.max_ctx, avg_bits=plan_bits)
+            tags_dev = all_tags.cuda()
+            self.tags_host = tags_host = all_tags.numpy()
+        else:
+            self.cache = kvq.Cache(NL, B, Hkv, Hq, D, wl.max_ctx, list(wl.layer_bits), kmodes=[wl.kmode] * NL)
+        cache = self.cache
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for l in range(NL):
+                K, V = inputs.layer_kv(wl, l, wl.prefill, "cuda")
+                if paged:
+                    t0 = tags_dev[:, :wl.prefill].contiguous()
+                    kvq.kvq_append_tagged(cache.h, l, K, V, wl.prefill,
+                                          np.ascontiguousarray(tags_host[:, :wl.prefill]), t0, stream)
+                else:
+                    cache.append(l, K, V)
+                del K, V
+        stream.synchronize()
+        nsched = self.nsched = wl.decode_steps
+        if paged:
+            step_tags_dev = [tags_dev[:, wl.prefill + s:wl.prefill + s + 1].contiguous() for s in range(nsched)]
+            step_tags_host = [np.ascontiguousarray(tags_host[:, wl.prefill + s:wl.prefill + s + 1])
+                              for s in range(nsched)]
+        # decode schedule inputs, resident in HBM
+        self.Kn = Kn = torch.empty((nsched, NL, B, Hkv, 1, D), dtype=torch.bfloat16, device="cuda")
+        self.Vn = Vn = torch.empty_like(Kn)
+        self.Qn = Qn = torch.empty((nsched, NL, B, Hq, D), dtype=torch.bfloat16, device="cuda")
+        for s in range(nsched):
+            for l in range(NL):
+                k, v = inputs.step_kv(wl, l, s, "cuda")
+                Kn[s, l].copy_(k)
+                Vn[s, l].copy_(v)
+                Qn[s, l].copy_(inputs.step_q(wl, l, s, "cuda"))
+        self.out = out = torch.empty((NL, B, Hq, D), dtype=torch.bfloat16, device="cuda")
+        # one eager decode per layer before capture (kernel attributes, occupancy, status clear)
+        with torch.cuda.stream(stream):
+            for l in range(NL):
+                cache.decode_attn(l, Qn[0, l], out[l], stream=stream)
+        stream.synchronize()
+        self.graphs, self.dec_graphs, self.splits, self.Ls = [], [], [], []
+        for s in range(nsched):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for l in range(NL):
+                    if paged:
+                        kvq.kvq_append_tagged(cache.h, l, Kn[s, l], Vn[s, l], 1, step_tags_host[s], step_tags_dev[s],
+                                              stream)
+                        kvq.kvq_decode_attn(cache.h, l, Qn[s, l], out[l], False, stream)
+                    else:
+                        kvq.kvq_append_decode(cache.h, l, Kn[s, l], Vn[s, l], Qn[s, l], out[l], False, stream)
+            self.graphs.append(g)
+            self.splits.append([kvq.kvq_get_num_splits(cache.h, l) for l in range(NL)])
+            self.Ls.append(cache.seq_len(0))
+            gd = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gd, stream=stream):
+                for l in range(NL):
+                    kvq.kvq_decode_attn(cache.h, l, Qn[s, l], out[l], False, stream)
+            self.dec_graphs.append(gd)
+        torch.cuda.synchronize()
+
+    def release(self):
+        self.graphs, self.dec_graphs = [], []
+
+    def time_steps(self, order, warmup, barrier):
+        """Device time (ms) of the full steps in `order`, after `warmup` untimed steps."""
+        import torch
+        stream = self.stream
+        with torch.cuda.stream(stream):
+            for i in range(warmup):
+                self.graphs[i % self.nsched].replay()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for s in order:
+                self.graphs[s].replay()
+            e1.record(stream)
+        barrier()
+        return e0.elapsed_time(e1)
+
+    def time_decode(self, order, min_ms=100.0, min_reps=3):
+        """Decode-only graphs over the steps in `order`, replayed as a whole until at least
+        min_ms of device time (and min_reps passes) are timed; returns (ms per launch,
+        passes, timed ms).  Live CUDA events on the launching stream."""
+        import torch
+        stream = self.stream
+        with torch.cuda.stream(stream):
+            for s in order[: min(len(order), 8)]:
+                self.dec_graphs[s].replay()
+            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            d0.record(stream)
+            for s in order:
+                self.dec_graphs[s].replay()
+            d1.record(stream)
+        stream.synchronize()
+        one = d0.elapsed_time(d1)
+        reps = max(min_reps, int(min_ms / max(one, 1e-3)) + 1)
+        with torch.cuda.stream(stream):
+            d0.record(stream)
+            for _ in range(reps):
+                for s in order:
+                    self.dec_graphs[s].replay()
+            d1.record(stream)
+        stream.synchronize()
+        tot = d0.elapsed_time(d1)
+        return tot / (reps * len(order) * self.wl.num_layers), reps, tot
+
+    def decode_bytes_per_launch(self, order):
+        wl = self.wl
+        B, Hkv, G, D, NL = wl.batch, wl.n_kv_heads, wl.G, wl.head_dim, wl.num_layers
+        if self.paged:
+            # INT2 groups: 2-bit codes + fp16 scale/zero per 32 (keys and values); INT4 tokens
+            # (main and pending): 4-bit codes + scale/zero; q in and out
+            def paged_bytes(L):
+                t = self.tags_host[:, :L]
+                n2 = (t == 2).sum(1)
+                g2 = (n2 // 32) * 32
+                rest = L - g2
+                per = g2 * D * 2 * (2 + 1) / 8 + rest * D * 2 * (4 + 1) / 8 + 2 * G * D * 2
+                return float(Hkv * per.sum())
+            tot = sum(paged_bytes(self.Ls[s]) for s in order for l in range(NL))
+        else:
+            tot = sum(decode_bytes(B, Hkv, G, D, self.Ls[s], *wl.layer_bits[l], wl.kmode)
+                      for s in order for l in range(NL))
+        return tot / (len(order) * NL)
+
+    def launches(self, order):
+        """Kernel launches of the steps in `order`: per layer one fused launch, or (a token
+        that completes a per-channel key group; paged plans) an append and a decode launch
+        (plus the tag scan of multi-token paged appends: none here); plus the merge launch
+        for two or three splits."""
+        wl = self.wl
+
+        def step_launches(s, l):
+            two = self.paged or (wl.kmode == 0 and self.Ls[s] % 32 == 0)
+            return (2 if two else 1) + (1 if 1 < self.splits[s][l] < 4 else 0)
+        return sum(step_launches(s, l) for s in order for l in range(wl.num_layers))
+
+    def context(self, order):
+        Ls = [self.Ls[s] for s in order]
+        return f"{min(Ls)}..{max(Ls)}"
+
+
+def reduced_workload(wl, n_layers):
+    """The first n_layers layers of `wl` with the same precision mix as the full map (layers
+    taken from each distinct bit pair in proportion), renumbered 0..n-1."""
+    import dataclasses
+    from collections import Counter
+    cnt = Counter(wl.layer_bits)
+    total = len(wl.layer_bits)
+    bits = []
+    for pair, c in sorted(cnt.items(), key=lambda x: -x[1]):
+        bits += [pair] * max(1, round(n_layers * c / total))
+    bits = tuple(sorted(bits, key=lambda p: wl.layer_bits.index(p)))
+    return dataclasses.replace(wl, num_layers=len(bits), layer_bits=bits)
+
+
+PER_CONFIG_LAYERS = {"c3": 4, "c4": 2, "c5": 2, "c5-alloc": 2, "c2-k8v8": 32, "c2": 32, "c2-k8v4": 32}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -253,6 +447,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="use only the first N layers (small ncu captures; reported in config.layers)")
+    ap.add_argument("--per-config", default="c3,c4,c5",
+                    help="comma list of further workloads measured after the headline (reduced layer counts with "
+                         "the same precision mix; 'none' to skip)")
+    ap.add_argument("--decode-ms", type=float, default=100.0,
+                    help="minimum device time of the decode-only replays behind the roofline figure")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -270,154 +469,44 @@ def main():
         run_reference(args, wl, rank)
         return
 
-    import numpy as np
     import torch
     import torch.distributed as dist
     from datetime import timedelta
 
-    from layer_wise_mixed_b200 import inputs, kvq
+    from layer_wise_mixed_b200 import kvq
 
     torch.cuda.set_device(local)
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-
-    # replica per rank: its own sequences (weak scaling, no data-path collective)
-    wl = rank_workload(wl, rank, world)
-    B, Hkv, Hq, D, G, NL = wl.batch, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.G, wl.num_layers
-    paged = wl.paged
-    if paged:
-        all_tags = paged_tags(wl, wl.max_ctx)                  # [B, prefill + steps], shared by layers
-        # the pools split at the mask's own mean bits (an allocation may land under its budget)
-        plan_bits = min(wl.avg_bits, 4.0 - 2.0 * float((all_tags == 2).float().mean()))
-        cache = kvq.Cache(NL, B, Hkv, Hq, D, wl.max_ctx, avg_bits=plan_bits)
-        tags_dev = all_tags.cuda()
-        tags_host = all_tags.numpy()
-    else:
-        cache = kvq.Cache(NL, B, Hkv, Hq, D, wl.max_ctx, list(wl.layer_bits), kmodes=[wl.kmode] * NL)
-    stream = torch.cuda.Stream()
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        for l in range(NL):
-            K, V = inputs.layer_kv(wl, l, wl.prefill, "cuda")
-            if paged:
-                t0 = tags_dev[:, :wl.prefill].contiguous()
-                kvq.kvq_append_tagged(cache.h, l, K, V, wl.prefill, np.ascontiguousarray(tags_host[:, :wl.prefill]),
-                                      t0, stream)
-            else:
-                cache.append(l, K, V)
-            del K, V
-    stream.synchronize()
-    if paged:
-        step_tags_dev = [tags_dev[:, wl.prefill + s:wl.prefill + s + 1].contiguous() for s in range(wl.decode_steps)]
-        step_tags_host = [np.ascontiguousarray(tags_host[:, wl.prefill + s:wl.prefill + s + 1])
-                          for s in range(wl.decode_steps)]
-
-    def append_step(l, s, Kd, Vd):
-        if paged:
-            kvq.kvq_append_tagged(cache.h, l, Kd, Vd, 1, step_tags_host[s], step_tags_dev[s], stream)
-        else:
-            kvq.kvq_append(cache.h, l, Kd, Vd, 1, stream)
-
-    # decode schedule inputs, resident in HBM
-    nsched = wl.decode_steps
-    Kn = torch.empty((nsched, NL, B, Hkv, 1, D), dtype=torch.bfloat16, device="cuda")
-    Vn = torch.empty_like(Kn)
-    Qn = torch.empty((nsched, NL, B, Hq, D), dtype=torch.bfloat16, device="cuda")
-    for s in range(nsched):
-        for l in range(NL):
-            k, v = inputs.step_kv(wl, l, s, "cuda")
-            Kn[s, l].copy_(k)
-            Vn[s, l].copy_(v)
-            Qn[s, l].copy_(inputs.step_q(wl, l, s, "cuda"))
-    out = torch.empty((NL, B, Hq, D), dtype=torch.bfloat16, device="cuda")
-
-    # one eager decode per layer before capture (kernel attributes, occupancy, status clear)
-    with torch.cuda.stream(stream):
-        for l in range(NL):
-            cache.decode_attn(l, Qn[0, l], out[l], stream=stream)
-    stream.synchronize()
-
-    graphs, dec_graphs, splits, Ls = [], [], [], []
-    for s in range(nsched):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for l in range(NL):
-                if paged:
-                    append_step(l, s, Kn[s, l], Vn[s, l])
-                    kvq.kvq_decode_attn(cache.h, l, Qn[s, l], out[l], False, stream)
-                else:
-                    kvq.kvq_append_decode(cache.h, l, Kn[s, l], Vn[s, l], Qn[s, l], out[l], False, stream)
-        graphs.append(g)
-        splits.append([kvq.kvq_get_num_splits(cache.h, l) for l in range(NL)])
-        Ls.append(cache.seq_len(0))
-        gd = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gd, stream=stream):
-            for l in range(NL):
-                kvq.kvq_decode_attn(cache.h, l, Qn[s, l], out[l], False, stream)
-        dec_graphs.append(gd)
-    torch.cuda.synchronize()
-
-    order = [(args.warmup + i) % nsched for i in range(args.steps)]
-    sampler = ClockSampler(local)
 
     def barrier():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
 
-    # ---- timed region: K full steps ----
-    with torch.cuda.stream(stream):
-        for i in range(args.warmup):
-            graphs[i % nsched].replay()
+    # replica per rank: its own sequences (weak scaling, no data-path collective)
+    wl = rank_workload(wl, rank, world)
+    B, Hkv, Hq, D, G, NL = wl.batch, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.G, wl.num_layers
+    paged = wl.paged
+    stream = torch.cuda.Stream()
+    run = WorkloadRun(wl, stream)
+    cache, Kn, Vn, Qn, out, nsched = run.cache, run.Kn, run.Vn, run.Qn, run.out, run.nsched
+    order = [(args.warmup + i) % nsched for i in range(args.steps)]
+    peak, peak_src = measured_hbm_peak()
+
+    # ---- timed region: K full steps; then the dominant kernel: decode-only graphs over
+    # the same steps (live events), replayed for at least --decode-ms of device time ----
+    sampler = ClockSampler(local)
     sampler.start()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for s in order:
-            graphs[s].replay()
-        e1.record(stream)
-    barrier()
+    ms = max_over_ranks(run.time_steps(order, args.warmup, barrier), world)
+    dec_launch_ms, dec_reps, dec_total_ms = run.time_decode(order, args.decode_ms)
     clocks = sampler.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1), world)
     ms_per_step = ms / args.steps
     value = world * B * args.steps / (ms / 1e3)
-
-    # ---- dominant kernel: decode-only graphs over the same schedule (live events) ----
-    with torch.cuda.stream(stream):
-        for s in order[: min(len(order), 8)]:
-            dec_graphs[s].replay()
-        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        d0.record(stream)
-        for s in order:
-            dec_graphs[s].replay()
-        d1.record(stream)
-    stream.synchronize()
-    dec_ms = d0.elapsed_time(d1)
-    launches_dec = args.steps * NL
-    if paged:
-        # INT2 groups: 2-bit codes + fp16 scale/zero per 32 (keys and values); INT4 tokens
-        # (main and pending): 4-bit codes + scale/zero; q in and out
-        def paged_bytes(L):
-            t = tags_host[:, :L]
-            n2 = (t == 2).sum(1)
-            g2 = (n2 // 32) * 32
-            rest = L - g2
-            per = g2 * D * 2 * (2 + 1) / 8 + rest * D * 2 * (4 + 1) / 8 + 2 * G * D * 2
-            return float(Hkv * per.sum())
-        dec_bytes = sum(paged_bytes(Ls[s]) for s in order for l in range(NL))
-    else:
-        dec_bytes = sum(decode_bytes(B, Hkv, G, D, Ls[s], *wl.layer_bits[l], wl.kmode)
-                        for s in order for l in range(NL))
-    peak, peak_src = measured_hbm_peak()
-    achieved = dec_bytes / (dec_ms / 1e3) / 1e9
-    # per layer and step: one fused append + decode launch, or (a token that completes a
-    # per-channel key group; paged plans) an append and a decode launch; plus the merge
-    # launch for two or three splits
-    def step_launches(s, l):
-        two = paged or (wl.kmode == 0 and Ls[s] % 32 == 0)
-        return (2 if two else 1) + (1 if 1 < splits[s][l] < 4 else 0)
-    gpu_launches = sum(step_launches(s, l) for s in order for l in range(NL))
+    launches_dec = len(order) * NL
+    bytes_launch = run.decode_bytes_per_launch(order)
+    achieved = bytes_launch / (dec_launch_ms / 1e3) / 1e9
+    gpu_launches = run.launches(order)
     e2e_note = (f"per step and group of {max(1, args.e2e_group)} layers: pinned H2D of the group's K/V/q (copy stream), "
                 "kvq_append_decode per layer (eager C-ABI calls, compute stream), D2H of the group's outputs "
                 "(second copy stream); groups overlap")
@@ -515,6 +604,53 @@ def main():
     h2d = NL * per * 2
     d2h = out.numel() * 2
     status = kvq.kvq_device_status(cache.h, stream)
+    head_cfg = workload_config(wl)
+    head_cfg["context"] = run.context(order)
+    head_cfg["schedule"] = f"{wl.prefill + 1}..{wl.prefill + wl.decode_steps}"
+    traffic = captured_traffic(wl.name, bytes_launch)
+    head_splits = sorted(set(x for s in order for x in run.splits[s]))
+    run.release()
+    del run, cache, hIn, dIn, dOut
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    # ---- further workloads (rank 0 of a 1-GPU run): the long-context maps and the paged
+    # cache, reduced to a few layers with the same precision mix; step throughput scaled to
+    # the full layer count, the decode kernel's roofline per launch ----
+    per_config = {}
+    wanted = [] if args.per_config in ("", "none") else [x for x in args.per_config.split(",") if x]
+    if world == 1:
+        for name in wanted:
+            full = configs.by_name(name)
+            wc = reduced_workload(full, PER_CONFIG_LAYERS.get(name, 2))
+            r = WorkloadRun(wc, stream)
+            ordc = list(range(r.nsched))
+            smp = ClockSampler(local)
+            smp.start()
+            ms_c = r.time_steps(ordc, 3, barrier)
+            dl_ms, dl_reps, _ = r.time_decode(ordc, args.decode_ms)
+            clk = smp.stop()
+            bl = r.decode_bytes_per_launch(ordc)
+            ach = bl / (dl_ms / 1e3) / 1e9
+            st = kvq.kvq_device_status(r.cache.h, stream)
+            per_config[name] = {
+                "workload": full.name, "layers_measured": wc.num_layers, "layers_full": full.num_layers,
+                "bits_measured": ",".join(f"K{a}V{b}" for a, b in wc.layer_bits) if not wc.paged else "INT2/INT4",
+                "batch": wc.batch, "timed_context": r.context(ordc), "steps": len(ordc),
+                "tokens_per_s": wc.batch / (ms_c / len(ordc) * full.num_layers / wc.num_layers / 1e3),
+                "step_ms_per_layer": ms_c / len(ordc) / wc.num_layers,
+                "hbm_gbs_decode": ach, "frac": ach / peak, "avg_launch_us": 1e3 * dl_ms,
+                "algorithmic_bytes_per_launch": bl, "decode_replays": dl_reps,
+                "traffic": captured_traffic(full.name, bl),
+                "kernel": "decode_paged_kernel" if wc.paged else "decode_split_kernel",
+                "splits": sorted(set(x for s in ordc for x in r.splits[s])), "clocks": clk, "device_status": st,
+                "how": (f"{wc.num_layers} of {full.num_layers} layers with the full map's precision mix; tokens/s = "
+                        "batch / (step time scaled to the full layer count); decode GB/s = algorithmic bytes / "
+                        "CUDA-event time of decode-only graph replays")}
+            r.release()
+            del r
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -545,21 +681,22 @@ def main():
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f16*f16->f32 (codes exact in f16), f32 quantizer",
                 "data": "synthetic (seeded normal K/V/Q, outlier key channels; no weights or datasets)",
-                "config": workload_config(wl),
+                "config": head_cfg,
                 "hbm_gbs_decode": achieved,
                 "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                             "frac": achieved / peak,
-                             "traffic": captured_traffic(wl.name, dec_bytes / launches_dec),
+                             "frac": achieved / peak, "traffic": traffic,
                              "kernel": "decode_paged_kernel" if wl.paged else "decode_split_kernel",
-                             "peak_source": peak_src, "avg_launch_us": 1e3 * dec_ms / launches_dec,
-                             "algorithmic_bytes_per_launch": dec_bytes / launches_dec},
+                             "peak_source": peak_src, "avg_launch_us": 1e3 * dec_launch_ms,
+                             "algorithmic_bytes_per_launch": bytes_launch,
+                             "decode_region": {"replays_of_timed_steps": dec_reps, "ms": dec_total_ms,
+                                               "launches": dec_reps * launches_dec}},
                 "cpu_baseline": cpu,
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                         "steps": e2e_steps, "how": e2e_note},
                 "gpu_launches": gpu_launches, "clocks": clocks, "device_status": status,
-                "splits": sorted(set(x for s in order for x in splits[s]))}
+                "splits": head_splits,
+                "per_config": per_config}
         print(json.dumps(line), flush=True)
-    del graphs, dec_graphs
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

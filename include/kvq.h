@@ -25,8 +25,9 @@
  *    log-sum-exp).  out[b, hq] = sum_t softmax_t(q . k^_t / sqrt(D)) v^_t over all L
  *    cached tokens; query head hq uses kv head hq / G, G = n_q_heads / n_kv_heads.
  *
- * Storage format v1 (the pages fix none; chosen so that each decoder thread's tensor
- * core operand fragments are contiguous).  Per layer, per (batch b, kv head h):
+ * Storage format v2 (the pages fix none; chosen so that each decoder thread's tensor
+ * core operand fragments are contiguous; v1, whose scales and zeros were in plain index
+ * order, is not readable as v2).  Per layer, per (batch b, kv head h):
  * capacity ceil(max_ctx/32) block records of 32 tokens, then (per-channel keys) a
  * residual of 32 x D bf16.  Record of block beta, D = head_dim, nj = D/32:
  *     [K codes 4*D*bk B][K s/z 4*D B][V codes 4*D*bv B][V s/z 4*D B]
@@ -214,8 +215,10 @@ KVQ_API int kvq_device_status(kvq_handle *h, void *stream, unsigned *flags);
  * memory pool).  The pages describe no such entry point; it has no counterpart
  * there.  The first call on a device, with that device current, looks up the
  * buffer's device address; make that first call before any stream capture.  Returns
- * KVQ_EUNSUPPORTED when the call needs more partial space than the buffer holds
- * (B * Hq * 64 * (head_dim + 2) * 4 bytes whenever the sequence is split).  All
+ * KVQ_EUNSUPPORTED when the call needs more partial space than the buffer holds:
+ * a call split in S > 1 parts needs about B * Hq * S * (head_dim + 2) * 4 bytes
+ * (batch 64 with 32 query heads at head_dim 128: up to 31 splits; no space without
+ * splits).  All
  * calls share the one buffer: calls that may overlap on the GPU (different streams,
  * no ordering between them) race on it and must not be issued. */
 KVQ_API int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, int out_fp32,

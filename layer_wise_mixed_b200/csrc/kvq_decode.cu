@@ -70,24 +70,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned phase) {
     asm volatile(
         "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(phase), "r"(1000000u)
+        : "r"(smem_u32(bar)), "r"(phase), "r"(100000u)
         : "memory");
     return ok != 0;
 }
-// Bounded wait: gives up after ~2^20 polls (each suspends at most ~1 ms).
 __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait: polls until the phase completes or kWaitLimitNs of wall time (the GPU's
+// global nanosecond timer) have passed since the first failed poll, then reports
+// failure; the caller records kStatusWaitExpired and returns normally.  A copy lands
+// in microseconds, so the limit is only reached when something is broken.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned phase) {
-    for (int i = 0; i < (1 << 20); ++i)
+    if (mbar_try_wait(bar, phase)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
         if (mbar_try_wait(bar, phase)) return true;
-    return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
 }
 
 __device__ __forceinline__ void mma16816(float *c, const uint32_t *a, uint32_t b0, uint32_t b1) {
     asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The same shape with bf16 operands (the bf16 residual keys of a per-channel layer).
+__device__ __forceinline__ void mma16816_bf16(float *c, const uint32_t *a, uint32_t b0, uint32_t b1) {
+    asm(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};\n"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -113,9 +134,6 @@ __device__ __forceinline__ uint32_t h2_bits(__half2 v) { return *reinterpret_cas
 __device__ __forceinline__ __half2 bits_h2(uint32_t v) { return *reinterpret_cast<__half2 *>(&v); }
 __device__ __forceinline__ uint32_t hsub2_bits(uint32_t x, uint32_t y) {
     return h2_bits(__hsub2(bits_h2(x), bits_h2(y)));
-}
-__device__ __forceinline__ uint32_t hfma2_bits(uint32_t x, uint32_t m, uint32_t a) {
-    return h2_bits(__hfma2(bits_h2(x), bits_h2(m), bits_h2(a)));
 }
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) { return h2_bits(__floats2half2_rn(lo, hi)); }
 
@@ -191,6 +209,21 @@ __device__ __forceinline__ void mul_hilo(uint32_t xh, uint32_t xl, uint32_t s, u
     hi = h2_bits(h);
 }
 
+// Split two floats into three bf16 pairs: hi and mid by 8-bit truncation (exact), lo the
+// remainder rounded to bf16; hi + mid + lo carries 24 significant bits (error below
+// 2^-24 of |v|), as much as the float itself.
+__device__ __forceinline__ void split3_bf16(float a, float b, uint32_t &hi, uint32_t &mid, uint32_t &lo) {
+    const float ha = __uint_as_float(__float_as_uint(a) & 0xFFFF0000u);
+    const float hb = __uint_as_float(__float_as_uint(b) & 0xFFFF0000u);
+    hi = (__float_as_uint(ha) >> 16) | (__float_as_uint(hb) & 0xFFFF0000u);
+    const float ra = a - ha, rb = b - hb;   // exact
+    const float ma = __uint_as_float(__float_as_uint(ra) & 0xFFFF0000u);
+    const float mb = __uint_as_float(__float_as_uint(rb) & 0xFFFF0000u);
+    mid = (__float_as_uint(ma) >> 16) | (__float_as_uint(mb) & 0xFFFF0000u);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(ra - ma, rb - mb);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
 // Split two floats into fp16 hi (11-bit truncation, exact) and lo (remainder) pairs.
 __device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
     const float ha = trunc11(a), hb = trunc11(b);
@@ -209,7 +242,9 @@ __host__ __device__ constexpr int unit_bytes(int D, int BK, int BV, int KM, int 
 
 // Per-thread constants of the block body.
 struct BodyCtx {
-    const uint4 *aq_s;          // q operand fragments in shared memory, [KS][32]
+    const uint4 *aq_s;          // q operand fragments in shared memory: [KS][32] fp16 hi/lo,
+                                // then (per-channel keys) [KS][32] bf16 hi/mid and [KS][32]
+                                // bf16 lo (as uint4 {lo, 0, lo', 0}) for the residual
     const uint16_t *res;        // bf16 residual keys of this (b, h) (per-channel tail) or null
     int lane, g, t, G, jg, jg8, jz, alpha_src0, alpha_src1;
     bool row_g, row_g8;
@@ -226,9 +261,15 @@ struct WarpAcc {
 
 // Query setup: q~ fragments into shared memory (written by warp 0), score scaling.
 //  per-channel keys: q~ = q log2(e)/sqrt(D) 2^kq as fp16 hi/lo (rows g: hi, g+8: lo),
-//    kq chosen so that q~ s_k < 2^14 and q~ < 2^15; scores = raw * 2^-kq.
-//  per-token keys: raw q (exact in fp16), rows (group j, head) masked to group j;
-//    scores = raw * log2(e)/sqrt(D).
+//    kq chosen so that q~ s_k < 2^14 and q~ < 2^15; scores = raw * 2^-kq.  The same q~
+//    as bf16 hi/mid/lo parts for the bf16 residual keys of the open group (bf16
+//    operands take the residual rows as they are, at any magnitude, with no fp16
+//    conversion; three parts keep q~'s 24 bits).
+//  per-token keys: q~ = q 2^kq with kq chosen so that |q~| < 2^15 (a bf16 value times a
+//    power of two is exact in fp16 down to 2^-14 of that bound; smaller entries lose
+//    bits far below the largest product), rows (group j, head) masked to group j;
+//    scores = raw * log2(e)/sqrt(D) * 2^-kq.
+// kq is clamped so that 2^kq and 2^-kq stay normal binary32 numbers.
 // Computed by warp 0 only; every lane's scalars (unscale, qsum_g, qsum_g8) go to
 // scal_s[lane] for the other warps (load_query_scalars after a CTA barrier).
 template <int KM, int D>
@@ -250,28 +291,40 @@ __device__ __forceinline__ void setup_query(const uint16_t *qrow, float smax_k, 
     const float qscale = kLog2e * rsqrtf(static_cast<float>(D));
     uint32_t aq[KS][4];
     c.qsum_g = c.qsum_g8 = 0.f;
+    // the head's largest |q| (times the score scale for per-channel keys): the 4 lanes
+    // of a row group hold all D channels of head hh
+    float amax = 0.f;
+#pragma unroll
+    for (int k = 0; k < KS; ++k)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) amax = fmaxf(amax, fabsf(KM == 0 ? qv[k][x] * qscale : qv[k][x]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    int kq = 0;
+    if (amax > 0.f) {
+        kq = 14 - floor_log2(amax);                                                                // q~ < 2^15
+        if (KM == 0 && smax_k > 0.f) kq = min(kq, 12 - floor_log2(amax) - floor_log2(smax_k));   // q~ s < 2^14
+        kq = max(-120, min(100, kq));
+    }
     if constexpr (KM == 0) {
-        float amax = 0.f;
-#pragma unroll
-        for (int k = 0; k < KS; ++k)
-#pragma unroll
-            for (int x = 0; x < 4; ++x) amax = fmaxf(amax, fabsf(qv[k][x] * qscale));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        int kq = 0;
-        if (amax > 0.f) {
-            kq = 14 - floor_log2(amax);                                                  // q~ < 2^15
-            if (smax_k > 0.f) kq = min(kq, 12 - floor_log2(amax) - floor_log2(smax_k));   // q~ s < 2^14
-            kq = max(-60, min(60, kq));
-        }
         const float sc = qscale * pow2f(kq);
         c.unscale = pow2f(-kq);
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
             split2(qv[k][0] * sc, qv[k][1] * sc, aq[k][0], aq[k][1]);
             split2(qv[k][2] * sc, qv[k][3] * sc, aq[k][2], aq[k][3]);
+            uint32_t h0, m0, l0, h2, m2, l2;
+            split3_bf16(qv[k][0] * sc, qv[k][1] * sc, h0, m0, l0);
+            split3_bf16(qv[k][2] * sc, qv[k][3] * sc, h2, m2, l2);
+            aq_s[(KS + k) * 32 + c.lane] = make_uint4(h0, m0, h2, m2);       // rows g: hi, g + 8: mid
+            aq_s[(2 * KS + k) * 32 + c.lane] = make_uint4(l0, 0u, l2, 0u);   // rows g: lo
         }
     } else {
+        const float sc = pow2f(kq);
+#pragma unroll
+        for (int k = 0; k < KS; ++k)
+#pragma unroll
+            for (int x = 0; x < 4; ++x) qv[k][x] *= sc;
         float part[NJ];
 #pragma unroll
         for (int j = 0; j < NJ; ++j) part[j] = 0.f;
@@ -292,7 +345,7 @@ __device__ __forceinline__ void setup_query(const uint16_t *qrow, float smax_k, 
             if (j == (c.jg < NJ ? c.jg : 0)) c.qsum_g = part[j];
             if (j == (c.jg8 < NJ ? c.jg8 : 0)) c.qsum_g8 = part[j];
         }
-        c.unscale = qscale;
+        c.unscale = qscale * pow2f(-kq);
     }
 #pragma unroll
     for (int k = 0; k < KS; ++k) aq_s[k * 32 + c.lane] = make_uint4(aq[k][0], aq[k][1], aq[k][2], aq[k][3]);
@@ -386,22 +439,24 @@ __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R
         for (int x = 0; x < 4; ++x) acc[n][x] = 0.f;
     float czacc[4] = {0.f, 0.f, 0.f, 0.f};
     if constexpr (KM == 0 && TAIL) {
-        // bf16 residual keys of the last, incomplete group
+        // bf16 residual keys of the last, incomplete group: bf16 MMAs with the bf16
+        // hi/mid (rows g, g + 8) and lo (rows g) query parts, the rows taken as stored
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
-            const uint4 aqv = c.aq_s[k * 32 + lane];
+            const uint4 aqv = c.aq_s[(KS + k) * 32 + lane];
+            const uint4 aql = c.aq_s[(2 * KS + k) * 32 + lane];
             const uint32_t ak[4] = {aqv.x, aqv.y, aqv.z, aqv.w};
+            const uint32_t al[4] = {aql.x, aql.y, aql.z, aql.w};
 #pragma unroll
             for (int n = 0; n < NTI; ++n) {
                 const int u = 8 * n + g;
                 uint32_t b0 = 0u, b1 = 0u;
                 if (u < valid) {
-                    const uint32_t r0 = *reinterpret_cast<const uint32_t *>(c.res + u * D + 16 * k + 2 * t);
-                    const uint32_t r8 = *reinterpret_cast<const uint32_t *>(c.res + u * D + 16 * k + 2 * t + 8);
-                    b0 = pack_h2(__uint_as_float(r0 << 16), __uint_as_float(r0 & 0xFFFF0000u));
-                    b1 = pack_h2(__uint_as_float(r8 << 16), __uint_as_float(r8 & 0xFFFF0000u));
+                    b0 = *reinterpret_cast<const uint32_t *>(c.res + u * D + 16 * k + 2 * t);
+                    b1 = *reinterpret_cast<const uint32_t *>(c.res + u * D + 16 * k + 2 * t + 8);
                 }
-                mma16816(acc[n], ak, b0, b1);
+                mma16816_bf16(acc[n], ak, b0, b1);
+                mma16816_bf16(acc[n], al, b0, b1);
             }
         }
     } else {
@@ -668,7 +723,7 @@ __device__ __forceinline__ void pipe_drain(WarpPipe &P, int from) {
 template <int D, int NT>
 __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &c, bool has_data, uint8_t *smem,
                                               int warp, long long row0, int sp, int S, int out_fp32, void *out,
-                                              float *part_acc, float *part_ml, unsigned *arrive) {
+                                              float *part_acc, float *part_ml, int sstride, unsigned *arrive) {
     constexpr int KS = D / 16;
     const int g = c.g, t = c.t, G = c.G;
     float l_run = A.l_run;
@@ -749,10 +804,10 @@ __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &
                 *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(out) + row * D + d) = u;
             }
         } else {
-            *reinterpret_cast<float4 *>(part_acc + (row * kMaxSplits + sp) * D + d) = val;
+            *reinterpret_cast<float4 *>(part_acc + (row * sstride + sp) * D + d) = val;
             if (d == 0) {
-                part_ml[(row * kMaxSplits + sp) * 2] = M;
-                part_ml[(row * kMaxSplits + sp) * 2 + 1] = den;
+                part_ml[(row * sstride + sp) * 2] = M;
+                part_ml[(row * sstride + sp) * 2 + 1] = den;
             }
         }
     }
@@ -771,7 +826,7 @@ __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &
     for (int i4 = threadIdx.x; i4 < G * D / 4; i4 += NW * 32) {
         const int hd = (4 * i4) / D, d = (4 * i4) % D;
         const long long row = row0 + hd;
-        const float *ml = part_ml + row * kMaxSplits * 2;
+        const float *ml = part_ml + row * sstride * 2;
         float M = -INFINITY;
         for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(ml + 2 * s));
         float den = 0.f;
@@ -781,7 +836,7 @@ __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &
             if (ms == -INFINITY) continue;
             const float wt = fast_exp2(ms - M);
             den = fmaf(wt, __ldcg(ml + 2 * s + 1), den);
-            const float4 a = __ldcg(reinterpret_cast<const float4 *>(part_acc + (row * kMaxSplits + s) * D + d));
+            const float4 a = __ldcg(reinterpret_cast<const float4 *>(part_acc + (row * sstride + s) * D + d));
             val.x = fmaf(wt, a.x, val.x);
             val.y = fmaf(wt, a.y, val.y);
             val.z = fmaf(wt, a.z, val.z);
@@ -826,7 +881,7 @@ __host__ __device__ constexpr int prologue_bytes(int D) { return 8 * D * 2 + 2 *
 
 __host__ __device__ inline size_t smem_total(int PS, int stage_bytes, int D, int NT) {
     const size_t bars = static_cast<size_t>(PS) * 8 + 8 * (PS & 1);   // keeps 16-B alignment
-    return smem_bars_off(PS, stage_bytes, D, NT) + bars + static_cast<size_t>(D / 16) * 32 * 16 + 32 * 16 +
+    return smem_bars_off(PS, stage_bytes, D, NT) + bars + static_cast<size_t>(D / 16) * 32 * 16 * 3 + 32 * 16 +
            append_scratch_bytes(D) + prologue_bytes(D);
 }
 
@@ -836,7 +891,7 @@ __device__ __forceinline__ SmemParts carve(uint8_t *smem, int PS, int stage_byte
     const size_t bo = smem_bars_off(PS, stage_bytes, D, NT);
     s.bars = reinterpret_cast<uint64_t *>(smem + bo);
     s.aq_s = reinterpret_cast<uint4 *>(smem + bo + static_cast<size_t>(PS) * 8 + 8 * (PS & 1));
-    s.scal_s = reinterpret_cast<float4 *>(s.aq_s + (D / 16) * 32);
+    s.scal_s = reinterpret_cast<float4 *>(s.aq_s + 3 * (D / 16) * 32);
     return s;
 }
 
@@ -1102,7 +1157,7 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
         if (lane == 0) atomicOr(p.status, kStatusWaitExpired);
     }
     combine_store<D, NT>(A, c, nb > 0 && !failed, smem, warp, static_cast<long long>(b) * p.Hkv * G + h * G, sp,
-                         p.S, p.out_fp32, p.out, p.part_acc, p.part_ml, p.arrive ? p.arrive + unit : nullptr);
+                         p.S, p.out_fp32, p.out, p.part_acc, p.part_ml, p.sstride, p.arrive ? p.arrive + unit : nullptr);
 }
 
 // ------------------------------------------------------------------ paged kernel
@@ -1210,7 +1265,7 @@ __device__ __forceinline__ void paged_body(const PagedDecodeParams &p, uint8_t *
         if (lane == 0) atomicOr(p.status, kStatusWaitExpired);
     }
     combine_store<D, NT>(A, c, nb > 0 && !failed, smem, warp, static_cast<long long>(b) * p.Hkv * G + h * G, sp,
-                         p.S2 + p.S4, p.out_fp32, p.out, p.part_acc, p.part_ml,
+                         p.S2 + p.S4, p.out_fp32, p.out, p.part_acc, p.part_ml, p.sstride,
                          p.arrive ? p.arrive + static_cast<long long>(b) * p.Hkv + h : nullptr);
 }
 
@@ -1228,7 +1283,7 @@ __global__ void __launch_bounds__(NW * 32, 4) decode_paged_kernel(const PagedDec
 __global__ void merge_kernel(const MergeParams p) {
     pdl_enter();
     const long long row = blockIdx.x;   // b * Hq + hq
-    const float *ml = p.part_ml + row * kMaxSplits * 2;
+    const float *ml = p.part_ml + row * p.sstride * 2;
     float M = -INFINITY;
     for (int s = 0; s < p.S; ++s) M = fmaxf(M, ml[2 * s]);
     for (int d = threadIdx.x; d < p.D; d += blockDim.x) {
@@ -1237,7 +1292,7 @@ __global__ void merge_kernel(const MergeParams p) {
             const float ms = ml[2 * s];
             if (ms == -INFINITY) continue;
             const float wt = fast_exp2(ms - M);
-            val = fmaf(wt, p.part_acc[(row * kMaxSplits + s) * p.D + d], val);
+            val = fmaf(wt, p.part_acc[(row * p.sstride + s) * p.D + d], val);
             den = fmaf(wt, ml[2 * s + 1], den);
         }
         const float o = val * __frcp_rn(den);
@@ -1281,7 +1336,7 @@ KernelFn pick_kernel(int D, int bk, int bv, int kmode, int G) {
 // fit), at most 6.
 int decode_stages(long long rec_bytes, int D, int G) {
     // per-CTA reserve, q fragments, barriers, prologue
-    const long long fixed = 1024 + (D / 16) * 32 * 16 + 64 + prologue_bytes(D);
+    const long long fixed = 1024 + 3 * (D / 16) * 32 * 16 + 64 + prologue_bytes(D);
     for (int ctas = (G <= 4 ? 4 : 3); ctas >= 1; --ctas) {
         const long long ns = (228LL * 1024 / ctas - fixed) / (NW * rec_bytes);
         if (ns >= 2) return static_cast<int>(ns > 6 ? 6 : ns);

@@ -656,6 +656,7 @@ static int decode_paged(kvq_handle *h, int layer, const void *q, void *out, int 
     p.out = out;
     p.part_acc = part_acc;
     p.part_ml = part_ml;
+    p.sstride = kvq::kMaxSplits;
     p.status = reinterpret_cast<unsigned *>(h->ws + h->status_off);
     p.B = h->desc.batch;
     p.Hkv = h->desc.n_kv_heads;
@@ -678,6 +679,7 @@ static int decode_paged(kvq_handle *h, int layer, const void *q, void *out, int 
         m.D = h->desc.head_dim;
         m.S = S2 + S4;
         m.out_fp32 = p.out_fp32;
+        m.sstride = p.sstride;
         e = kvq::launch_merge(m, st);
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");
     }
@@ -709,6 +711,7 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
     p.out = out;
     p.part_acc = reinterpret_cast<float *>(h->ws + h->part_acc_off);
     p.part_ml = reinterpret_cast<float *>(h->ws + h->part_ml_off);
+    p.sstride = kvq::kMaxSplits;
     p.status = reinterpret_cast<unsigned *>(h->ws + h->status_off);
     p.B = h->desc.batch;
     p.Hkv = h->desc.n_kv_heads;
@@ -736,6 +739,7 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
         m.D = h->desc.head_dim;
         m.S = p.S;
         m.out_fp32 = p.out_fp32;
+        m.sstride = p.sstride;
         e = kvq::launch_merge(m, st);
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");
     }
@@ -786,6 +790,7 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
     p.out = out;
     p.part_acc = reinterpret_cast<float *>(h->ws + h->part_acc_off);
     p.part_ml = reinterpret_cast<float *>(h->ws + h->part_ml_off);
+    p.sstride = kvq::kMaxSplits;
     p.status = reinterpret_cast<unsigned *>(h->ws + h->status_off);
     p.B = h->desc.batch;
     p.Hkv = h->desc.n_kv_heads;
@@ -826,6 +831,7 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
         m.D = h->desc.head_dim;
         m.S = p.S;
         m.out_fp32 = p.out_fp32;
+        m.sstride = p.sstride;
         e = kvq::launch_merge(m, st);
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");
     }
@@ -1092,8 +1098,9 @@ int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, 
     const int bps = (nblk + S - 1) / S;
     S = (nblk + bps - 1) / bps;
     const long long rows = static_cast<long long>(h->desc.batch) * h->desc.n_q_heads;
-    const long long acc_bytes = rows * kvq::kMaxSplits * h->desc.head_dim * 4;
-    const long long need = S > 1 ? acc_bytes + rows * kvq::kMaxSplits * 2 * 4 : 0;
+    // partials packed at the launch's own split count: [B][Hq][S][D] then [B][Hq][S][2]
+    const long long acc_bytes = (rows * S * h->desc.head_dim * 4 + 255) / 256 * 256;
+    const long long need = S > 1 ? acc_bytes + rows * S * 2 * 4 : 0;
     if (need > static_cast<long long>(kStaticScratchBytes))
         return fail(KVQ_EUNSUPPORTED,
                     "split partials need %lld bytes but the built-in scratch holds %zu; use kvq_decode_attn",
@@ -1109,6 +1116,7 @@ int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, 
     p.out = out;
     p.part_acc = static_cast<float *>(scratch);
     p.part_ml = reinterpret_cast<float *>(static_cast<unsigned char *>(scratch) + acc_bytes);
+    p.sstride = S;
     p.status = reinterpret_cast<unsigned *>(h->ws + h->status_off);
     p.B = h->desc.batch;
     p.Hkv = h->desc.n_kv_heads;
@@ -1136,6 +1144,7 @@ int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, 
         m.D = h->desc.head_dim;
         m.S = p.S;
         m.out_fp32 = p.out_fp32;
+        m.sstride = p.sstride;
         e = kvq::launch_merge(m, st);
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");
     }

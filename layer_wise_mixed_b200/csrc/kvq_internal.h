@@ -42,6 +42,9 @@ constexpr int kDecodeWarps = 4;     // warps per decode CTA
 
 // Device status word bits (written with atomicOr, read by kvq_device_status).
 constexpr unsigned kStatusWaitExpired = 1u;   // a bounded mbarrier wait gave up
+// Wall-time limit of one bounded wait inside a kernel (nanoseconds of the GPU's global
+// timer): 100 ms, far above any copy's latency, far below what would hold a GPU.
+constexpr unsigned long long kWaitLimitNs = 100ull * 1000 * 1000;
 
 // Per-layer geometry and precision, resolved by the host.
 struct LayerGeom {
@@ -79,8 +82,10 @@ struct DecodeParams {
     const uint16_t *q;          // bf16 [B][Hq][D]
     const unsigned *smax;       // this layer's {max key scale, max value scale} (fp16 bits)
     void *out;                  // [B][Hq][D] bf16 or fp32
-    float *part_acc;            // [B][Hq][kMaxSplits][D]
-    float *part_ml;             // [B][Hq][kMaxSplits][2]  (m in log2 units, l)
+    float *part_acc;            // [B][Hq][sstride][D]
+    float *part_ml;             // [B][Hq][sstride][2]  (m in log2 units, l)
+    int sstride;                // partial slots per (batch, query head): kMaxSplits in the
+                                // workspace, the launch's split count in the built-in scratch
     unsigned *arrive;           // [B][Hkv] split arrival counters (zero between launches), or null:
                                 // split partials merged by merge_kernel
     unsigned *status;
@@ -121,6 +126,7 @@ struct PagedDecodeParams {
     const unsigned *smax;
     void *out;
     float *part_acc, *part_ml;
+    int sstride;                // as in DecodeParams
     unsigned *arrive;           // as in DecodeParams
     unsigned *status;
     int B, Hkv, G, S2, S4, out_fp32, nstage;
@@ -158,6 +164,7 @@ struct MergeParams {
     const float *part_ml;
     void *out;
     int B, Hq, D, S, out_fp32;
+    int sstride;                // partial slots per (batch, query head)
 };
 
 // Split counts from which the decode launch merges its own partials (the last CTA of a

@@ -1,4 +1,4 @@
-// Device helpers shared by the append kernels: the group quantizer and the v1 storage
+// Device helpers shared by the append kernels: the group quantizer and the v2 storage
 // format's positions (see include/kvq.h).  Each quantizer step is one correctly rounded
 // binary32 operation; nothing here is contracted into FMA.
 #pragma once
@@ -32,7 +32,7 @@ __device__ __forceinline__ int group_code(float x, float s, float z, int bits) {
 }
 
 // Owner (token in half e, channel d) of field f of lane word w, for the key operand
-// role (role 0) or the value operand role (role 1) of the v1 format.
+// role (role 0) or the value operand role (role 1) of the v2 format.
 __device__ __forceinline__ void field_owner(int role, int lane, int w, int f, int bits, int &e,
                                             int &d) {
     const int P = 16 / bits;
@@ -51,7 +51,7 @@ __device__ __forceinline__ void field_owner(int role, int lane, int w, int f, in
 
 // Word index (inside a half's code area) and bit offset of the code of token e (0..15
 // inside the half), channel d, for the key operand role (role 0) or the value operand
-// role (role 1) of the v1 format: the inverse of field_owner.
+// role (role 1) of the v2 format: the inverse of field_owner.
 __device__ __forceinline__ void code_place(int role, int e, int d, int D, int bits, int &word, int &bit) {
     const int P = 16 / bits;
     int lane, slot, hb;
@@ -74,7 +74,7 @@ __device__ __forceinline__ void code_place(int role, int e, int d, int D, int bi
     bit = field * bits;
 }
 
-// Byte offsets of a scale/zero pair in the s/z areas of the v1 format.
+// Byte offsets of a scale/zero pair in the s/z areas of the v2 format.
 __device__ __forceinline__ int chan_sz_off(int d) {   // per-channel keys: scale; zero at +4
     const int k = d >> 4, e = d & 15;
     return 16 * (4 * k + ((e & 7) >> 1)) + 8 * (e >> 3) + 2 * (e & 1);

@@ -95,6 +95,11 @@ int kvq_tag_distortion(int num_layers, int num_requests, int n_q_heads, int n_kv
     const int D = head_dim, G = n_q_heads / n_kv_heads, R = num_requests, NL = num_layers;
     for (long long i = 0; i < static_cast<long long>(R) * T; ++i)
         if (tags[i] < 0 || tags[i] >= num_tags) return kvq::host_fail(KVQ_EINVAL, "tag out of range");
+    // every worker holds a T x T fp64 score matrix and ~12 T x D rows: refuse sizes whose
+    // buffers would not fit the 2 GB the workers share, before anything is allocated
+    const double per_thread = 8.0 * (static_cast<double>(T) * T + 12.0 * static_cast<double>(T) * head_dim);
+    if (per_thread > 2.0e9)
+        return kvq::host_fail(KVQ_EINVAL, "T too large for the host calibration (worker buffers exceed 2 GB)");
     for (int k = 0; k < num_tags; ++k) counts[k] = 0;
     for (long long i = 0; i < static_cast<long long>(R) * T; ++i) ++counts[tags[i]];
 
@@ -111,7 +116,8 @@ int kvq_tag_distortion(int num_layers, int num_requests, int n_q_heads, int n_kv
     const long long ntask = static_cast<long long>(NL) * R * n_kv_heads;
     const double rs = 1.0 / std::sqrt(static_cast<double>(D));
     std::atomic<long long> next{0};
-    auto work = [&]() {
+    std::atomic<int> failed{0};
+    auto work_body = [&]() {
         std::vector<float> kf(TD), vf(TD);
         std::vector<double> kx(TD), vx(TD), kq(TD), vq(TD), qd(TD), S(static_cast<size_t>(T) * T), m(T), l(T),
             N(TD), dN(D), kxT(TD), kqT, sq;
@@ -210,15 +216,25 @@ int kvq_tag_distortion(int num_layers, int num_requests, int n_q_heads, int n_kv
             }
         }
     };
+    // a worker that cannot allocate its buffers stops the others and the call fails
+    // (no exception leaves a worker thread)
+    auto work = [&]() {
+        try {
+            work_body();
+        } catch (...) {
+            failed.store(1);
+            next.store(ntask);
+        }
+    };
     // threads: the host's cores, at most 64, and as many as keep every worker's buffers
-    // (the T x T fp64 scores and ~10 T x D rows) within about 2 GB
-    const double per_thread = 8.0 * (static_cast<double>(T) * T + 12.0 * static_cast<double>(TD));
+    // (the T x T fp64 scores and ~12 T x D rows) within about 2 GB
     const unsigned by_mem = static_cast<unsigned>(std::max(1.0, std::floor(2.0e9 / per_thread)));
     const unsigned nth = std::max(1u, std::min({std::thread::hardware_concurrency(), 64u, by_mem}));
     std::vector<std::thread> pool;
     for (unsigned i = 1; i < nth; ++i) pool.emplace_back(work);
     work();
     for (auto &th : pool) th.join();
+    if (failed.load()) return kvq::host_fail(KVQ_EINVAL, "host memory exhausted during calibration");
     auto head_max = [&](int lay, int r, int k, int bi) {
         double w = 0.0;
         const double *e = mse.data() + (((static_cast<size_t>(lay) * R + r) * num_tags + k) * 2 + bi) * n_q_heads;

@@ -3,7 +3,7 @@
 * Equivalent precision of a map: the mean over layers of (key bits + value bits)/2
   (KVTuner summary, Key results: "3.25-bit equivalent precision"; per-layer
   sensitivity facts: a K8V2 pair is "5-bit", a K4V8 pair "6-bit").
-* Storage bits per cached element of the v1 format: codes plus one fp16 scale and
+* Storage bits per cached element of the v2 format: codes plus one fp16 scale and
   one fp16 zero per 32 elements, for keys and values alike (asymmetric groupwise
   quantizer with g = 32, TriAxialKV facts).
 """

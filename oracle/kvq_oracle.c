@@ -43,8 +43,11 @@
  *     residual.  Values, and keys in per-token mode: 32 consecutive channels of
  *     one token.
  *
- * Q3  Storage format (version 1).  The pages fix no layout; this one is chosen so
+ * Q3  Storage format (version 2).  The pages fix no layout; this one is chosen so
  *     that a decoder thread's tensor-core operand fragments are contiguous.
+ *     (Version 1 kept the scales and zeros of each area in plain index order; version
+ *     2 places them in fragment order, as below.  Images of the two versions are not
+ *     interchangeable.)
  *     Per (batch b, kv head h) the cache is a sequence of 32-token block records.
  *     Record of block beta (tokens 32*beta .. 32*beta+31), D = head_dim, nj = D/32:
  *        [K codes: 4*D*bk bytes][K s/z: 4*D bytes][V codes: 4*D*bv][V s/z: 4*D]
@@ -637,4 +640,4 @@ void orc_quant_groups(const float *x, long ngroups, int bits, uint16_t *s16, uin
                       uint8_t *codes) {
     for (long g = 0; g < ngroups; g++) orc_quant(x + g * 32, 32, 1, bits, s16 + g, z16 + g, codes + g * 32, 1);
 }
-int orc_format_version(void) { return 1; }
+int orc_format_version(void) { return 2; }

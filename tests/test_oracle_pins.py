@@ -154,7 +154,7 @@ def test_numpy_restatement_agrees():
 # ----------------------------------------------------------------- storage format (Q3)
 def test_golden_positions():
     """Hand-derived positions of single codes (no page prints a layout)."""
-    rows = [list(map(int, ln.split())) for ln in open(os.path.join(GOLDEN, "format_v1_positions.txt"))
+    rows = [list(map(int, ln.split())) for ln in open(os.path.join(GOLDEN, "format_v2_positions.txt"))
             if ln.strip() and not ln.startswith("#")]
     assert len(rows) > 30
     for role, D, bits, u, d, byte, bit in rows:
@@ -262,7 +262,7 @@ def decode_unit_image(img, L, D, bk, bv, kmode):
 
 def test_golden_sz_positions():
     """Hand-derived scale/zero offsets (no page fixes a layout)."""
-    rows = [list(map(int, ln.split())) for ln in open(os.path.join(GOLDEN, "format_v1_sz_positions.txt"))
+    rows = [list(map(int, ln.split())) for ln in open(os.path.join(GOLDEN, "format_v2_sz_positions.txt"))
             if ln.strip() and not ln.startswith("#")]
     assert len(rows) >= 12
     for kind, nj, index, j, so, zo in rows:
