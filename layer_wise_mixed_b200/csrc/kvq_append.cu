@@ -187,8 +187,13 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams p) {
             return;
         }
         const int b = unit / p.Hkv;
-        L_old = p.L_old_r[b];
-        n = p.n_r[b];
+        if (p.ragged_dev) {
+            L_old = p.ragged_dev[b];
+            n = p.ragged_dev[p.B + b];
+        } else {
+            L_old = p.L_old_r[b];
+            n = p.n_r[b];
+        }
         const int L_new = L_old + n;
         hb0 = L_old / 16;
         nhb = n > 0 ? (L_new - 1) / 16 - hb0 + 1 : 0;
@@ -225,9 +230,33 @@ __global__ void __launch_bounds__(kThreads) append_kernel(AppendParams p) {
     }
 }
 
+struct TableChunk {
+    int *dst;
+    int n;
+    int v[1000];   // keeps the parameter block under 4 KB
+};
+
+__global__ void set_table_kernel(const TableChunk c) {
+    pdl_enter();
+    for (int i = threadIdx.x; i < c.n; i += blockDim.x) c.dst[i] = c.v[i];
+}
+
 }  // namespace
 
+cudaError_t launch_set_table(int *dst, const int *vals, int n, cudaStream_t st) {
+    for (int i0 = 0; i0 < n; i0 += 1000) {
+        TableChunk c;
+        c.dst = dst + i0;
+        c.n = n - i0 < 1000 ? n - i0 : 1000;
+        for (int i = 0; i < c.n; ++i) c.v[i] = vals[i0 + i];
+        cudaError_t e = launch_pdl(set_table_kernel, dim3(1), dim3(256), 0, st, c);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaGetLastError();
+}
+
 cudaError_t launch_append(const AppendParams &p, cudaStream_t st) {
+
     if (p.D > kMaxD) return cudaErrorInvalidValue;
     const int grid = p.nV + p.nK;
     if (grid <= 0) return cudaSuccess;

@@ -1026,7 +1026,8 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.z, h = blockIdx.y, sp = blockIdx.x;
-    const int G = p.G, L = p.ragged ? p.lens[b] : p.L;   // this request's length
+    const int G = p.G, L = p.ragged ? (p.lens_dev ? p.lens_dev[b] : p.lens[b]) : p.L;   // this request's length
+
     // nstage stages per warp, one more for warps 0 .. nextra - 1 (those with the most blocks)
     const int NS = p.nstage + (warp < p.nextra ? 1 : 0);
     const int sbase = warp * p.nstage + min(warp, p.nextra);

@@ -26,6 +26,7 @@ struct kvq_handle {
     int cap_blk = 0;
     long long status_off = 0, smax_off = 0, arrive_off = 0, meta_bytes = 0, part_acc_off = 0, part_ml_off = 0,
               total = 0;
+    long long lens_off = 0;                  // per-layer plans: per layer [2][B] int32 length tables
     uint8_t *ws = nullptr;
     size_t ws_bytes = 0;
     int forced_splits = 0;
@@ -82,6 +83,13 @@ int check_bound(const kvq_handle *h) {
 }
 
 int cuda_fail(cudaError_t e, const char *what);
+
+// The layer's device length table (per-layer plans): [B] lengths, or [B] old lengths then
+// [B] counts for an append.
+int *lens_table(const kvq_handle *h, int layer) {
+    return reinterpret_cast<int *>(h->ws + h->lens_off) + 2LL * h->desc.batch * layer;
+}
+
 
 // Per-layer maxima of the fp16 scales {K, V}, kept in two slots by the parity of the
 // layer's append count v: an append reads slot v & 1, writes slot (v + 1) & 1 (carrying
@@ -224,6 +232,10 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
     h->arrive_off = align256(256 + 16LL * d->num_layers);         // {K, V} max scale per layer and parity
     h->meta_bytes = align256(h->arrive_off + 4LL * d->batch * d->n_kv_heads);   // split arrival counters
     long long off = h->meta_bytes;
+    // per-request length tables of batches above kvq::kMaxRagged (one per layer, so calls
+    // on different layers never share one)
+    h->lens_off = off;
+    off = align256(off + 8LL * d->batch * d->num_layers);
     for (int l = 0; l < d->num_layers; ++l) {
         const kvq_layer_cfg &c = h->cfg[l];
         if (!valid_bits(c.bk) || !valid_bits(c.bv)) {
@@ -335,8 +347,6 @@ int append_impl(kvq_handle *h, int layer, const void *K, const void *V, const in
             return fail(KVQ_ECAPACITY, "layer %d request %d: %d + %d tokens exceed max_ctx %d", layer, b, Lo[b], nn[b],
                         h->desc.max_ctx);
     const bool uniform = !layer_ragged(h, layer) && std::all_of(nn.begin(), nn.end(), [&](int x) { return x == nn[0]; });
-    if (!uniform && B > kvq::kMaxRagged)
-        return fail(KVQ_EUNSUPPORTED, "requests of different lengths need batch <= %d (got %d)", kvq::kMaxRagged, B);
     const LayerGeom &g = h->geom[layer];
     const int units = B * h->desc.n_kv_heads;
     kvq::AppendParams p{};
@@ -371,11 +381,18 @@ int append_impl(kvq_handle *h, int layer, const void *K, const void *V, const in
     } else {
         p.ragged = 1;
     }
+    std::vector<int> table;   // [B] old lengths, then [B] counts (batches above kMaxRagged)
     if (p.ragged) {
         int nhb = 0, ng = 0;
+        if (B > kvq::kMaxRagged) {
+            table.assign(Lo.begin(), Lo.end());
+            table.insert(table.end(), nn.begin(), nn.end());
+        }
         for (int b = 0; b < B; ++b) {
-            p.L_old_r[b] = Lo[b];
-            p.n_r[b] = nn[b];
+            if (B <= kvq::kMaxRagged) {
+                p.L_old_r[b] = Lo[b];
+                p.n_r[b] = nn[b];
+            }
             const int L_new = Lo[b] + nn[b];
             if (nn[b] > 0) nhb = std::max(nhb, (L_new - 1) / 16 - Lo[b] / 16 + 1);
             ng = std::max(ng, L_new / 32 - Lo[b] / 32);
@@ -390,6 +407,13 @@ int append_impl(kvq_handle *h, int layer, const void *K, const void *V, const in
     p.nK = static_cast<int>(nK);
     if (p.nV + p.nK == 0) return ok();   // no token appended: nothing changes (the slot neither)
     if ((rc = prepare_status(h, static_cast<cudaStream_t>(stream)))) return rc;
+    if (!table.empty()) {
+        int *dev = lens_table(h, layer);
+        cudaError_t e = kvq::launch_set_table(dev, table.data(), static_cast<int>(table.size()),
+                                              static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "length table launch");
+        p.ragged_dev = dev;
+    }
     cudaError_t e = kvq::launch_append(p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
     int mx = 0;
@@ -402,16 +426,28 @@ int append_impl(kvq_handle *h, int layer, const void *K, const void *V, const in
     return ok();
 }
 
-// Decode parameters' per-request lengths (ragged layers); false if a request is empty.
-bool fill_lengths(const kvq_handle *h, int layer, kvq::DecodeParams &p) {
+// Decode parameters' per-request lengths (ragged layers), each request's length plus
+// `extra`: in the parameters, or (batches above kMaxRagged) in the layer's device table,
+// written on `st`.  KVQ_EINVAL if a request would be empty.
+int fill_lengths(kvq_handle *h, int layer, kvq::DecodeParams &p, int extra, cudaStream_t st) {
     p.ragged = 0;
-    if (!layer_ragged(h, layer)) return true;
+    p.lens_dev = nullptr;
+    if (!layer_ragged(h, layer)) return KVQ_OK;
     p.ragged = 1;
-    for (int b = 0; b < h->desc.batch; ++b) {
-        if (h->rlen[layer][b] < 1) return false;
-        p.lens[b] = h->rlen[layer][b];
+    const int B = h->desc.batch;
+    std::vector<int> lens(B);
+    for (int b = 0; b < B; ++b) {
+        lens[b] = h->rlen[layer][b] + extra;
+        if (lens[b] < 1) return fail(KVQ_EINVAL, "layer %d: request %d is empty", layer, b);
+        if (B <= kvq::kMaxRagged) p.lens[b] = lens[b];
     }
-    return true;
+    if (B > kvq::kMaxRagged) {
+        int *dev = lens_table(h, layer);
+        cudaError_t e = kvq::launch_set_table(dev, lens.data(), B, st);
+        if (e != cudaSuccess) return cuda_fail(e, "length table launch");
+        p.lens_dev = dev;
+    }
+    return KVQ_OK;
 }
 
 }  // namespace
@@ -707,7 +743,7 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
     p.res = g.res_off >= 0 ? reinterpret_cast<const uint16_t *>(h->ws + g.res_off) : nullptr;
     p.q = static_cast<const uint16_t *>(q);
     p.smax = smax_slot(h, layer, static_cast<int>(h->ver[layer]));
-    if (!fill_lengths(h, layer, p)) return fail(KVQ_EINVAL, "layer %d: a request is empty", layer);
+    if ((rc = fill_lengths(h, layer, p, 0, static_cast<cudaStream_t>(stream)))) return rc;
     p.out = out;
     p.part_acc = reinterpret_cast<float *>(h->ws + h->part_acc_off);
     p.part_ml = reinterpret_cast<float *>(h->ws + h->part_ml_off);
@@ -770,9 +806,6 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
         if ((rc = kvq_append(h, layer, K, V, 1, stream))) return rc;
         return kvq_decode_attn(h, layer, q, out, out_fp32, stream);
     }
-    const bool ragged = layer_ragged(h, layer);
-    if (ragged && B > kvq::kMaxRagged)
-        return fail(KVQ_EUNSUPPORTED, "requests of different lengths need batch <= %d (got %d)", kvq::kMaxRagged, B);
     h->len[layer] = L;   // the schedule is chosen for the new length
     int S = 1, nstage = 2, nextra = 0;
     if ((rc = splits_for(h, layer, &S, &nstage, &nextra))) {
@@ -785,8 +818,10 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
     p.res = g.res_off >= 0 ? reinterpret_cast<const uint16_t *>(h->ws + g.res_off) : nullptr;
     p.q = static_cast<const uint16_t *>(q);
     p.smax = smax_slot(h, layer, static_cast<int>(h->ver[layer]));
-    p.ragged = ragged ? 1 : 0;
-    for (int b = 0; ragged && b < B; ++b) p.lens[b] = h->rlen[layer][b] + 1;
+    if ((rc = fill_lengths(h, layer, p, 1, static_cast<cudaStream_t>(stream)))) {
+        h->len[layer] = L_old;
+        return rc;
+    }
     p.out = out;
     p.part_acc = reinterpret_cast<float *>(h->ws + h->part_acc_off);
     p.part_ml = reinterpret_cast<float *>(h->ws + h->part_ml_off);
@@ -1112,7 +1147,7 @@ int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, 
     p.res = g.res_off >= 0 ? reinterpret_cast<const uint16_t *>(h->ws + g.res_off) : nullptr;
     p.q = static_cast<const uint16_t *>(q);
     p.smax = smax_slot(h, layer, static_cast<int>(h->ver[layer]));
-    if (!fill_lengths(h, layer, p)) return fail(KVQ_EINVAL, "layer %d: a request is empty", layer);
+    if ((rc = fill_lengths(h, layer, p, 0, static_cast<cudaStream_t>(stream)))) return rc;
     p.out = out;
     p.part_acc = static_cast<float *>(scratch);
     p.part_ml = reinterpret_cast<float *>(static_cast<unsigned char *>(scratch) + acc_bytes);

@@ -36,8 +36,8 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 
 constexpr int kGroup = 32;          // quantization group (tokens or channels)
 constexpr int kMaxSplits = 64;      // partial slots per (batch, query head)
-constexpr int kMaxRagged = 64;      // requests per per-layer plan with per-request lengths
-                                    // (kernel-parameter tables)
+constexpr int kMaxRagged = 64;      // requests whose per-request lengths travel in the kernel
+                                    // parameters; larger batches use a device table
 constexpr int kDecodeWarps = 4;     // warps per decode CTA
 
 // Device status word bits (written with atomicOr, read by kvq_device_status).
@@ -71,9 +71,12 @@ struct AppendParams {
     int nV, nK;                 // CTA counts of the two roles
     // per-request lengths (ragged != 0): request b appends n_r[b] tokens at L_old_r[b];
     // nhb and ng are then the largest counts over the requests (grid sizing) and each CTA
-    // derives its request's own range, idling when it has none
+    // derives its request's own range, idling when it has none.  Batches of more than
+    // kMaxRagged requests read them from the device table ragged_dev instead: [B] L_old,
+    // then [B] n (written on the stream by launch_set_table just before).
     int ragged;
     int L_old_r[kMaxRagged], n_r[kMaxRagged];
+    const int *ragged_dev;
 };
 
 struct DecodeParams {
@@ -92,9 +95,11 @@ struct DecodeParams {
     int B, Hkv, G, L, cap_blk, S, bps, out_fp32;
     int nstage, nextra;         // stages per warp; one more for warps 0 .. nextra - 1
     // per-request lengths (ragged != 0): request b has lens[b] tokens (L above is the
-    // largest, which sets the split partition)
+    // largest, which sets the split partition); batches of more than kMaxRagged requests
+    // read them from the device table lens_dev [B] (written by launch_set_table)
     int ragged;
     int lens[kMaxRagged];
+    const int *lens_dev;
     long long rec_bytes;
     // Fused one-token append (kvq_append_decode), null otherwise: the new token's K and V
     // rows (bf16 [B][Hkv][D]), now token L - 1; writable records and residual; the
@@ -179,6 +184,12 @@ int host_fail(int code, const char *msg);
 int host_ok();
 
 cudaError_t launch_append(const AppendParams &p, cudaStream_t st);
+// Write n host integers into the device table dst on stream st, as kernel launches that
+// carry the values in their parameters (1000 per launch): the values are captured by
+// value into CUDA graphs, and each launch writes only after the preceding kernel of the
+// stream has completed (programmatic dependent launch waits first).
+cudaError_t launch_set_table(int *dst, const int *vals, int n, cudaStream_t st);
+
 // Returns cudaErrorInvalidValue if no kernel exists for the combination.
 cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmode,
                           cudaStream_t st, int *ctas_per_sm_out);

@@ -126,3 +126,31 @@ def test_ragged_noalloc_matches_workspace_entry(splits):
     torch.cuda.synchronize()
     assert torch.equal(a, b)
     r.check(q, splits=(splits,), what="noalloc")
+
+
+@pytest.mark.parametrize("kmode", [0, 1])
+def test_ragged_batch_96(kmode):
+    """96 requests of different lengths (above the 64 whose lengths fit the kernel
+    parameters: the lengths go through the layer's device table): ragged appends with
+    zero counts and group completions, decode with automatic and forced splits, fused
+    one-token steps (and the two-launch path), the entry point without caller scratch."""
+    B = 96
+    r = Ragged(B, 2, 4, 128, (4, 2), kmode, 260, f"ragged96-{kmode}")
+    rng = np.random.default_rng(96 + kmode)
+    r.append([int(x) for x in rng.integers(1, 160, B)])
+    r.check(inputs.step_q(r.wl, 0, 1, "cuda"), splits=(0, 3, 5), what="b96 prompts")
+    counts = [int(x) for x in rng.integers(0, 40, B)]
+    counts[0] = 0
+    r.append(counts)
+    r.check(inputs.step_q(r.wl, 0, 2, "cuda"), splits=(0, 4), what="b96 appends")
+    for step in range(1, 4):
+        q, out32 = r.fused(step)
+        r.check(q, out32, splits=(0,), what=f"b96 fused {step}")
+    q = inputs.step_q(r.wl, 0, 7, "cuda")
+    kvq.kvq_set_num_splits(r.cache.h, 3)
+    a = r.cache.decode_attn(0, q, out_fp32=True)
+    b = torch.empty_like(a)
+    kvq.kvq_decode_attn_noalloc(r.cache.h, 0, q, b, True)
+    kvq.kvq_set_num_splits(r.cache.h, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)

@@ -68,6 +68,7 @@ def test_workspace_layout(lib):
         al = lambda x: (x + 255) // 256 * 256
         expect = al(256 + 16 * 2)                      # status word + {K, V} max scale per layer and parity
         expect = al(expect + 4 * B * Hkv)               # split arrival counters per (b, kv head)
+        expect = al(expect + 8 * B * 2)                 # per-layer [2][B] length tables (large ragged batches)
         expect = al(expect + rec0 * cap * B * Hkv)
         expect = al(expect + 64 * D * B * Hkv)          # residual of the per-channel layer
         expect = al(expect + rec1 * cap * B * Hkv)
@@ -128,16 +129,19 @@ def test_ragged_argument_checks_before_any_launch(lib):
         assert list(kvq.kvq_seq_lens(h, 0, 2)) == [0, 0]
     finally:
         kvq.kvq_destroy(h)
-    h = kvq.kvq_plan(desc(batch=65))                 # different lengths need batch <= 64
+    h = kvq.kvq_plan(desc(batch=65))                 # above 64 requests: lengths in a device table
     try:
         fake = 1 << 40
         assert L.kvq_bind(h, fake, kvq.kvq_workspace_bytes(h)) == kvq.KVQ_OK
         counts = np.ones(65, np.int32)
-        counts[3] = 2
+        counts[3] = 3                                 # outside [0, n_max]: refused before any launch
         assert L.kvq_append_ragged(h, 0, fake, fake, counts.ctypes.data_as(ctypes.c_void_p), 2, None) == \
-            kvq.KVQ_EUNSUPPORTED
+            kvq.KVQ_EINVAL
+        assert "request 3" in kvq.kvq_last_error()
+        assert list(kvq.kvq_seq_lens(h, 0, 65)) == [0] * 65
     finally:
         kvq.kvq_destroy(h)
+
     h = kvq.kvq_plan(kvq.make_paged_desc(1, 2, 2, 8, 128, 64, 3.0))
     try:
         with pytest.raises(kvq.KvqError):
