@@ -441,7 +441,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="c2", choices=["c2", "c2-k8v8", "c2-k8v4", "c3", "c4", "c5", "c5-alloc"])
-    ap.add_argument("--e2e-group", type=int, default=16, help="layers per H2D/D2H transfer group of the e2e loop")
+    ap.add_argument("--e2e-group", type=int, default=16, help="layers per H2D/D2H transfer group of the eager e2e loop")
+    ap.add_argument("--e2e-mode", default="graph", choices=["graph", "eager"],
+                    help="graph: per step one H2D of the step's inputs, the step's captured graph of C-ABI calls, one "
+                         "D2H of its outputs; eager: per group of layers, eager C-ABI calls")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--ref-seqs", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -513,6 +516,12 @@ def main():
     if paged:
         e2e_note = (f"per step and group of {max(1, args.e2e_group)} layers: pinned H2D of the group's K/V/q, kvq_decode_attn per layer "
                     "(eager C-ABI calls; the cache is not advanced), D2H of the group's outputs; groups overlap")
+    if args.e2e_mode == "graph":
+        e2e_note = ("per step: pinned H2D of the step's K/V/q for every layer into the step's device inputs (copy stream), "
+                    "replay of the step's CUDA graph of C-ABI calls (" +
+                    ("kvq_append_tagged + kvq_decode_attn" if paged else "kvq_append_decode") +
+                    " per layer, captured once through the public API; compute stream), D2D of the outputs into a "
+                    "double buffer and their D2H (second copy stream); consecutive steps overlap")
 
     # ---- e2e: public API with host buffers, H2D + D2H inside the timed region ----
     # Per step and group of CH layers (--e2e-group; fewer, larger groups issue fewer copies
@@ -522,72 +531,106 @@ def main():
     # transfers of one group overlap the calls of another; device buffers alternate
     # between even and odd steps.
     e2e_steps = args.e2e_steps or min(args.steps, 64)
-    CH = max(1, args.e2e_group)
-    groups = [list(range(g0, min(NL, g0 + CH))) for g0 in range(0, NL, CH)]
     nk, nq = B * Hkv * D, B * Hq * D                      # bf16 elements per layer
     per = 2 * nk + nq
-    hIn = torch.cat([Kn.reshape(nsched, NL, nk), Vn.reshape(nsched, NL, nk), Qn.reshape(nsched, NL, nq)],
-                    dim=2).cpu().pin_memory()             # [step, layer, K|V|q]
-    hO = torch.empty((NL,) + tuple(out.shape[1:]), dtype=out.dtype).pin_memory()
-    dIn = torch.empty((2, NL, per), dtype=torch.bfloat16, device="cuda")
-    dOut = torch.empty((2,) + tuple(out.shape), dtype=out.dtype, device="cuda")
     h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
-    ev = {k: [[torch.cuda.Event() for _ in groups] for _ in range(2)] for k in ("in", "comp", "out")}
-    used = [[False] * len(groups) for _ in range(2)]
-    if not paged:
-        for l in range(NL):
-            kvq.kvq_truncate(cache.h, l, wl.prefill)
-    # raw C-ABI calls with pointers taken once (the Python wrappers cost more host time
-    # per call than the transfers they would overlap)
-    lib = kvq.load()
-    sptr = stream.cuda_stream
-    ptrs = [[(dIn[par, l].data_ptr(), dIn[par, l].data_ptr() + 2 * nk, dIn[par, l].data_ptr() + 4 * nk,
-              dOut[par, l].data_ptr()) for l in range(NL)] for par in range(2)]
-    lens = [wl.prefill] * NL
-
-    def call(l, par):
-        pk, pv, pq, po = ptrs[par][l]
-        if paged:
-            rc = lib.kvq_decode_attn(cache.h, l, pq, po, 0, sptr)
-        else:
-            if lens[l] >= wl.max_ctx:
+    if args.e2e_mode == "eager":
+        CH = max(1, args.e2e_group)
+        groups = [list(range(g0, min(NL, g0 + CH))) for g0 in range(0, NL, CH)]
+        hIn = torch.cat([Kn.reshape(nsched, NL, nk), Vn.reshape(nsched, NL, nk), Qn.reshape(nsched, NL, nq)],
+                        dim=2).cpu().pin_memory()             # [step, layer, K|V|q]
+        hO = torch.empty((NL,) + tuple(out.shape[1:]), dtype=out.dtype).pin_memory()
+        dIn = torch.empty((2, NL, per), dtype=torch.bfloat16, device="cuda")
+        dOut = torch.empty((2,) + tuple(out.shape), dtype=out.dtype, device="cuda")
+        ev = {k: [[torch.cuda.Event() for _ in groups] for _ in range(2)] for k in ("in", "comp", "out")}
+        used = [[False] * len(groups) for _ in range(2)]
+        if not paged and args.e2e_mode == "eager":
+            for l in range(NL):
                 kvq.kvq_truncate(cache.h, l, wl.prefill)
-                lens[l] = wl.prefill
-            rc = lib.kvq_append_decode(cache.h, l, pk, pv, pq, po, 0, sptr)
-            lens[l] += 1
-        if rc != kvq.KVQ_OK:
-            raise kvq.KvqError(rc, lib.kvq_last_error().decode())
+        # raw C-ABI calls with pointers taken once (the Python wrappers cost more host time
+        # per call than the transfers they would overlap)
+        lib = kvq.load()
+        sptr = stream.cuda_stream
+        ptrs = [[(dIn[par, l].data_ptr(), dIn[par, l].data_ptr() + 2 * nk, dIn[par, l].data_ptr() + 4 * nk,
+                  dOut[par, l].data_ptr()) for l in range(NL)] for par in range(2)]
+        lens = [wl.prefill] * NL
 
-    def e2e_step(i, s):
-        par = i & 1
-        for gi, grp in enumerate(groups):
-            l0, l1 = grp[0], grp[-1] + 1
+        def call(l, par):
+            pk, pv, pq, po = ptrs[par][l]
+            if paged:
+                rc = lib.kvq_decode_attn(cache.h, l, pq, po, 0, sptr)
+            else:
+                if lens[l] >= wl.max_ctx:
+                    kvq.kvq_truncate(cache.h, l, wl.prefill)
+                    lens[l] = wl.prefill
+                rc = lib.kvq_append_decode(cache.h, l, pk, pv, pq, po, 0, sptr)
+                lens[l] += 1
+            if rc != kvq.KVQ_OK:
+                raise kvq.KvqError(rc, lib.kvq_last_error().decode())
+
+        def e2e_step(i, s):
+            par = i & 1
+            for gi, grp in enumerate(groups):
+                l0, l1 = grp[0], grp[-1] + 1
+                with torch.cuda.stream(h2d_stream):
+                    if used[par][gi]:
+                        h2d_stream.wait_event(ev["comp"][par][gi])     # the calls of step i - 2 read this buffer
+                    dIn[par, l0:l1].copy_(hIn[s, l0:l1], non_blocking=True)
+                    ev["in"][par][gi].record(h2d_stream)
+                stream.wait_event(ev["in"][par][gi])
+                if used[par][gi]:
+                    stream.wait_event(ev["out"][par][gi])              # step i - 2's outputs are on the host
+                for l in grp:
+                    call(l, par)
+                ev["comp"][par][gi].record(stream)
+                with torch.cuda.stream(d2h_stream):
+                    d2h_stream.wait_event(ev["comp"][par][gi])
+                    hO[l0:l1].copy_(dOut[par, l0:l1], non_blocking=True)
+                    ev["out"][par][gi].record(d2h_stream)
+                used[par][gi] = True
+
+        def drain():
+            for par in range(2):
+                for gi in range(len(groups)):
+                    if used[par][gi]:
+                        stream.wait_event(ev["out"][par][gi])
+
+    if args.e2e_mode == "graph":
+        # the step's inputs land in the device tensors its graph reads (Kn/Vn/Qn[s], one
+        # per step of the schedule); outputs alternate between two device buffers for the D2H
+        hK, hV, hQ = Kn.cpu().pin_memory(), Vn.cpu().pin_memory(), Qn.cpu().pin_memory()
+        out2 = torch.empty((2,) + tuple(out.shape), dtype=out.dtype, device="cuda")
+        hO2 = torch.empty((2,) + tuple(out.shape), dtype=out.dtype).pin_memory()
+        gev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "comp", "out")}
+        gused = [False, False]
+
+        def e2e_step(i, s):
+            par = i & 1
             with torch.cuda.stream(h2d_stream):
-                if used[par][gi]:
-                    h2d_stream.wait_event(ev["comp"][par][gi])     # the calls of step i - 2 read this buffer
-                dIn[par, l0:l1].copy_(hIn[s, l0:l1], non_blocking=True)
-                ev["in"][par][gi].record(h2d_stream)
-            stream.wait_event(ev["in"][par][gi])
-            if used[par][gi]:
-                stream.wait_event(ev["out"][par][gi])              # step i - 2's outputs are on the host
-            for l in grp:
-                call(l, par)
-            ev["comp"][par][gi].record(stream)
+                Kn[s].copy_(hK[s], non_blocking=True)
+                Vn[s].copy_(hV[s], non_blocking=True)
+                Qn[s].copy_(hQ[s], non_blocking=True)
+                gev["in"][par].record(h2d_stream)
+            stream.wait_event(gev["in"][par])
+            run.graphs[s].replay()
+            if gused[par]:
+                stream.wait_event(gev["out"][par])           # step i - 2's outputs are on the host
+            out2[par].copy_(out, non_blocking=True)
+            gev["comp"][par].record(stream)
             with torch.cuda.stream(d2h_stream):
-                d2h_stream.wait_event(ev["comp"][par][gi])
-                hO[l0:l1].copy_(dOut[par, l0:l1], non_blocking=True)
-                ev["out"][par][gi].record(d2h_stream)
-            used[par][gi] = True
+                d2h_stream.wait_event(gev["comp"][par])
+                hO2[par].copy_(out2[par], non_blocking=True)
+                gev["out"][par].record(d2h_stream)
+            gused[par] = True
 
-    def drain():
-        for par in range(2):
-            for gi in range(len(groups)):
-                if used[par][gi]:
-                    stream.wait_event(ev["out"][par][gi])
-
+        def drain():
+            for par in range(2):
+                if gused[par]:
+                    stream.wait_event(gev["out"][par])
+    e2e_first = args.warmup + args.steps   # continue the schedule where the timed steps ended
     with torch.cuda.stream(stream):
         for i in range(3):
-            e2e_step(i, i % nsched)
+            e2e_step(i, (e2e_first + i) % nsched)
         drain()
         barrier()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -595,7 +638,7 @@ def main():
         h2d_stream.wait_stream(stream)
         d2h_stream.wait_stream(stream)
         for i in range(e2e_steps):
-            e2e_step(3 + i, (3 + i) % nsched)
+            e2e_step(3 + i, (e2e_first + 3 + i) % nsched)
         drain()
         f1.record(stream)
     barrier()
@@ -610,7 +653,7 @@ def main():
     traffic = captured_traffic(wl.name, bytes_launch)
     head_splits = sorted(set(x for s in order for x in run.splits[s]))
     run.release()
-    del run, cache, hIn, dIn, dOut
+    del run, cache
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
 
@@ -692,7 +735,9 @@ def main():
                                                "launches": dec_reps * launches_dec}},
                 "cpu_baseline": cpu,
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                        "steps": e2e_steps, "how": e2e_note},
+                        "steps": e2e_steps, "how": e2e_note,
+                        "host_link_gbs": {"h2d": h2d * e2e_steps / (e2e_ms / 1e3) / 1e9,
+                                          "d2h": d2h * e2e_steps / (e2e_ms / 1e3) / 1e9}},
                 "gpu_launches": gpu_launches, "clocks": clocks, "device_status": status,
                 "splits": head_splits,
                 "per_config": per_config}

@@ -106,7 +106,16 @@ typedef struct {
     int paged;          /* 0: per-layer maps (this header's format); 1: INT2/INT4 paged */
     int page_tokens;    /* paged: 16 */
     float avg_bits;     /* paged: expected mean bits of the tag mask (sizes the pools) */
+    int pool_blocks;    /* per-layer plans: 0 = every sequence reserves max_ctx tokens of every
+                         * layer (a slab of ceil(max_ctx/32) records per (sequence, kv head));
+                         * > 0 = block pools: each layer's 32-token records come from a pool of
+                         * pool_blocks blocks (one record per kv head each), assigned to a
+                         * sequence's blocks through a block table as it grows and returned by
+                         * kvq_truncate / kvq_reset_sequences, so sequences of very different
+                         * lengths share the memory; a sequence still holds at most max_ctx
+                         * tokens.  Ignored by paged plans. */
 } kvq_plan_desc;
+
 
 typedef struct kvq_handle kvq_handle;
 
@@ -202,6 +211,15 @@ KVQ_API int kvq_seq_lens(const kvq_handle *h, int layer, int32_t *L);
  * shortest sequence and L % 32 == 0 (so no token of a kept block is partially
  * overwritten later). */
 KVQ_API int kvq_truncate(kvq_handle *h, int layer, int L);
+
+/* Empty the sequences seqs[0..n) in every layer (host bookkeeping only): their lengths
+ * become 0 and, with block pools (desc.pool_blocks > 0), their blocks return to each
+ * layer's pool for any sequence to take (continuous batching: a finished request leaves,
+ * a new one takes its slot).  An emptied sequence must be appended to before the next
+ * decode of a layer (decode needs every sequence non-empty).  Per-layer plans only
+ * (paged plans: KVQ_EUNSUPPORTED); KVQ_EINVAL for an index outside [0, batch). */
+KVQ_API int kvq_reset_sequences(kvq_handle *h, const int32_t *seqs, int n);
+
 
 /* Read and clear the device status word (synchronizes `stream`).  KVQ_EDEVICE if a
  * kernel reported a bounded wait that expired; *flags gets the raw bits. */

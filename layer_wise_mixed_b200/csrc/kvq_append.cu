@@ -45,7 +45,7 @@ __device__ void per_token_half(const AppendParams &p, int role, int unit, int hb
     const int u0 = 16 * hbi;
     const int es = max(L_old, u0) - u0, ee = min(L_new, u0 + 16) - u0;
     const int blk = hbi >> 1, eta = hbi & 1;
-    uint8_t *rec = p.rec + (static_cast<long long>(unit) * p.cap_blk + blk) * p.rec_bytes;
+    uint8_t *rec = p.rec + rec_index(p.btab, unit / p.Hkv, p.Hkv, unit % p.Hkv, p.cap_blk, blk) * p.rec_bytes;
     uint8_t *sz = rec + (role ? p.kc + p.ks + p.vc : p.kc);
     uint32_t *area = reinterpret_cast<uint32_t *>(rec + (role ? p.kc + p.ks : 0) +
                                                   static_cast<long long>(eta) * 2 * D * bits);
@@ -126,7 +126,7 @@ __device__ void per_channel_group(const AppendParams &p, int unit, int q, bool d
             xs[u][d] = bf16_to_f32(v);
         }
         __syncthreads();
-        uint8_t *rec = p.rec + (static_cast<long long>(unit) * p.cap_blk + q) * p.rec_bytes;
+        uint8_t *rec = p.rec + rec_index(p.btab, unit / p.Hkv, p.Hkv, unit % p.Hkv, p.cap_blk, q) * p.rec_bytes;
         for (int d = threadIdx.x; d < D; d += kThreads) {
             float mn = xs[0][d], mx = xs[0][d];
             for (int u = 1; u < 32; ++u) {
@@ -241,6 +241,17 @@ __global__ void set_table_kernel(const TableChunk c) {
     for (int i = threadIdx.x; i < c.n; i += blockDim.x) c.dst[i] = c.v[i];
 }
 
+struct ScatterChunk {
+    int *dst;
+    int n;
+    int idx[500], v[500];   // keeps the parameter block under 4 KB
+};
+
+__global__ void scatter_table_kernel(const ScatterChunk c) {
+    pdl_enter();
+    for (int i = threadIdx.x; i < c.n; i += blockDim.x) c.dst[c.idx[i]] = c.v[i];
+}
+
 }  // namespace
 
 cudaError_t launch_set_table(int *dst, const int *vals, int n, cudaStream_t st) {
@@ -255,7 +266,23 @@ cudaError_t launch_set_table(int *dst, const int *vals, int n, cudaStream_t st) 
     return cudaGetLastError();
 }
 
+cudaError_t launch_scatter_table(int *dst, const int *idx, const int *vals, int n, cudaStream_t st) {
+    for (int i0 = 0; i0 < n; i0 += 500) {
+        ScatterChunk c;
+        c.dst = dst;
+        c.n = n - i0 < 500 ? n - i0 : 500;
+        for (int i = 0; i < c.n; ++i) {
+            c.idx[i] = idx[i0 + i];
+            c.v[i] = vals[i0 + i];
+        }
+        cudaError_t e = launch_pdl(scatter_table_kernel, dim3(1), dim3(256), 0, st, c);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaGetLastError();
+}
+
 cudaError_t launch_append(const AppendParams &p, cudaStream_t st) {
+
 
     if (p.D > kMaxD) return cudaErrorInvalidValue;
     const int grid = p.nV + p.nK;

@@ -272,7 +272,7 @@ struct WarpAcc {
 // kq is clamped so that 2^kq and 2^-kq stay normal binary32 numbers.
 // Computed by warp 0 only; every lane's scalars (unscale, qsum_g, qsum_g8) go to
 // scal_s[lane] for the other warps (load_query_scalars after a CTA barrier).
-template <int KM, int D>
+template <int KM, int D, int NT>
 __device__ __forceinline__ void setup_query(const uint16_t *qrow, float smax_k, uint4 *aq_s, float4 *scal_s,
                                             BodyCtx &c, int warp) {
     constexpr int KS = D / 16, NJ = D / 32;
@@ -316,8 +316,12 @@ __device__ __forceinline__ void setup_query(const uint16_t *qrow, float smax_k, 
             uint32_t h0, m0, l0, h2, m2, l2;
             split3_bf16(qv[k][0] * sc, qv[k][1] * sc, h0, m0, l0);
             split3_bf16(qv[k][2] * sc, qv[k][3] * sc, h2, m2, l2);
-            aq_s[(KS + k) * 32 + c.lane] = make_uint4(h0, m0, h2, m2);       // rows g: hi, g + 8: mid
-            aq_s[(2 * KS + k) * 32 + c.lane] = make_uint4(l0, 0u, l2, 0u);   // rows g: lo
+            if constexpr (NT == 1) {   // one MMA: rows 0-3 hi, 4-7 mid, 8-11 lo (head g % G on every lane)
+                aq_s[(KS + k) * 32 + c.lane] = c.g < 4 ? make_uint4(h0, l0, h2, l2) : make_uint4(m0, 0u, m2, 0u);
+            } else {        // two MMAs: rows g hi and g + 8 mid, then rows g lo
+                aq_s[(KS + k) * 32 + c.lane] = make_uint4(h0, m0, h2, m2);
+                aq_s[(2 * KS + k) * 32 + c.lane] = make_uint4(l0, 0u, l2, 0u);
+            }
         }
     } else {
         const float sc = pow2f(kq);
@@ -439,14 +443,19 @@ __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R
         for (int x = 0; x < 4; ++x) acc[n][x] = 0.f;
     float czacc[4] = {0.f, 0.f, 0.f, 0.f};
     if constexpr (KM == 0 && TAIL) {
-        // bf16 residual keys of the last, incomplete group: bf16 MMAs with the bf16
-        // hi/mid (rows g, g + 8) and lo (rows g) query parts, the rows taken as stored
+        // bf16 residual keys of the last, incomplete group: bf16 MMAs with the three bf16
+        // query parts (packed into one MMA's rows, or hi/mid then lo), the rows taken as
+        // stored
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
             const uint4 aqv = c.aq_s[(KS + k) * 32 + lane];
-            const uint4 aql = c.aq_s[(2 * KS + k) * 32 + lane];
             const uint32_t ak[4] = {aqv.x, aqv.y, aqv.z, aqv.w};
-            const uint32_t al[4] = {aql.x, aql.y, aql.z, aql.w};
+            uint32_t al[4] = {0u, 0u, 0u, 0u};
+            if constexpr (NT == 2) {
+                const uint4 aql = c.aq_s[(2 * KS + k) * 32 + lane];
+                al[0] = aql.x;
+                al[2] = aql.z;
+            }
 #pragma unroll
             for (int n = 0; n < NTI; ++n) {
                 const int u = 8 * n + g;
@@ -456,7 +465,7 @@ __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R
                     b1 = *reinterpret_cast<const uint32_t *>(c.res + u * D + 16 * k + 2 * t + 8);
                 }
                 mma16816_bf16(acc[n], ak, b0, b1);
-                mma16816_bf16(acc[n], al, b0, b1);
+                if constexpr (NT == 2) mma16816_bf16(acc[n], al, b0, b1);
             }
         }
     } else {
@@ -506,6 +515,15 @@ __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R
         for (int n = 0; n < NTI; ++n) {
             raw[n][0] = acc[n][0] + acc[n][2] + cz;
             raw[n][1] = acc[n][1] + acc[n][3] + cz;
+        }
+        if constexpr (TAIL) {
+            if constexpr (NT == 1) {   // rows g (hi, lo) and g ^ 4 (mid) of the packed residual MMA
+#pragma unroll
+                for (int n = 0; n < NTI; ++n) {
+                    raw[n][0] += __shfl_xor_sync(0xffffffffu, raw[n][0], 16);
+                    raw[n][1] += __shfl_xor_sync(0xffffffffu, raw[n][1], 16);
+                }
+            }
         }
     } else {
         // per-token key scales on the (group, head) rows, then sum the rows of a head
@@ -931,7 +949,8 @@ __device__ __forceinline__ void append_token(const DecodeParams &p, long long un
     constexpr int REC = KC + KSZ + VC + 4 * D;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = u & 15, eta = u >> 4;
-    uint8_t *rec = p.rec_w + (unit * p.cap_blk + blk) * static_cast<long long>(REC);
+    uint8_t *rec = p.rec_w + rec_index(p.btab, static_cast<int>(unit / p.Hkv), p.Hkv, static_cast<int>(unit % p.Hkv),
+                                       p.cap_blk, blk) * static_cast<long long>(REC);
     uint8_t *codes = scratch;                                          // [0, D): values, [D, 2D): keys
     unsigned *cmax = reinterpret_cast<unsigned *>(scratch + 2 * D);   // keys, values (fp16 bits)
     uint16_t *szs = reinterpret_cast<uint16_t *>(scratch + 2 * D + 16);   // [role][j][scale, zero]
@@ -1021,7 +1040,8 @@ __device__ __forceinline__ void patch_stage(uint8_t *stage, int u, const uint8_t
 // ------------------------------------------------------------------ per-layer kernel
 template <int BK, int BV, int KM, int D, int NT>
 __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(const DecodeParams p) {
-    pdl_enter();
+    const bool early = p.early != 0;   // CTA-uniform
+    if (!early) pdl_enter();
     constexpr int REC = unit_bytes(D, BK, BV, KM, 2);
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1035,24 +1055,39 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     const int blk0 = sp * p.bps, blk1 = min(nblk, blk0 + p.bps);
     const int rem = L & 31;
     const int tail_blk = rem ? (L >> 5) : -1;
-    // the layer's scale maxima: loaded first (converted at first use), their latency
-    // overlaps the set-up
-    const unsigned smax_bits_k = p.smax[0], smax_bits_v = p.smax[1];
 
     const SmemParts sm = carve(smem, NW * p.nstage + p.nextra, REC, D, NT);
     WarpPipe P{sm.stages + static_cast<size_t>(sbase) * REC, sm.bars + sbase, NS, REC, lane, 0, 0, 0u, 0};
     pipe_init(P);
-    const uint8_t *unit_rec = p.rec + (static_cast<long long>(b) * p.Hkv + h) * p.cap_blk * REC;
     const int nb = (blk1 - blk0 > warp) ? (blk1 - blk0 - warp + NW - 1) / NW : 0;
     // per-channel keys of the last, incomplete group come from the residual: fetch only
     // the value part of that block's record
     constexpr unsigned VSKIP = KM == 0 ? 2 * 2 * D * BK + 4 * D : 0;
     auto issue_block = [&](int k) {
         const int blk = blk0 + warp + NW * k;
-        const uint8_t *src = unit_rec + static_cast<long long>(blk) * REC;
+        const uint8_t *src = p.rec + rec_index(p.btab, b, p.Hkv, h, p.cap_blk, blk) * REC;
         if (blk == tail_blk) pipe_issue(P, src + VSKIP, REC - VSKIP, VSKIP);
         else pipe_issue(P, src, REC);
     };
+    const long long unit = static_cast<long long>(b) * p.Hkv + h;
+    // the first stages' block copies and (per-channel keys) the bf16 residual rows of the
+    // tail block into L2 (read after the tail's copy)
+    auto issue_first = [&]() {
+        if constexpr (KM == 0) {
+            if (p.res && tail_blk >= blk0 && tail_blk < blk1 && ((tail_blk - blk0) % NW) == warp) {
+                const char *r = reinterpret_cast<const char *>(p.res + unit * 32 * D);
+                for (int i = lane; i < rem * D * 2 / 128; i += 32) prefetch_l2(r + i * 128);
+            }
+        }
+        for (int k = 0; k < NS && k < nb; ++k) issue_block(k);
+    };
+    if (early) {
+        issue_first();
+        pdl_enter();
+    }
+    // the layer's scale maxima: loaded first (converted at first use), their latency
+    // overlaps the set-up
+    const unsigned smax_bits_k = p.smax[0], smax_bits_v = p.smax[1];
     // a fused launch appends token L - 1 (the last of block new_blk) in the CTA that holds
     // that block; the block's warp patches its staged copy with the token
     const bool fused = p.k_new != nullptr;
@@ -1061,8 +1096,8 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     uint8_t *append_scratch = reinterpret_cast<uint8_t *>(sm.scal_s + 32);
     // the prologue copies (the q rows of the kv head's G query heads and, in the CTA that
     // appends, the token's K and V rows; all 16-byte aligned: rows of 2D bytes) go out
-    // before the block copies, which fill the memory queues for microseconds
-    const long long unit = static_cast<long long>(b) * p.Hkv + h;
+    // before the block copies (unless those went out early), which fill the memory queues
+    // for microseconds
     uint16_t *q_s = reinterpret_cast<uint16_t *>(append_scratch + append_scratch_bytes(D));
     uint16_t *kn_s = q_s + 8 * D, *vn_s = kn_s + D;
     uint64_t *pro_bar = reinterpret_cast<uint64_t *>(vn_s + D);
@@ -1079,14 +1114,8 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     }
     __syncwarp();   // warp 0's other lanes wait on pro_bar after lane 0 initialised it; the
                     // other warps wait on it only after a CTA barrier
-    if constexpr (KM == 0) {
-        // the bf16 residual rows of the tail block: into L2 now, read after the tail's copy
-        if (p.res && tail_blk >= blk0 && tail_blk < blk1 && ((tail_blk - blk0) % NW) == warp) {
-            const char *r = reinterpret_cast<const char *>(p.res + unit * 32 * D);
-            for (int i = lane; i < rem * D * 2 / 128; i += 32) prefetch_l2(r + i * 128);
-        }
-    }
-    for (int k = 0; k < NS && k < nb; ++k) issue_block(k);
+    if (!early) issue_first();
+
 
     const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(smax_bits_k)));
     const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(smax_bits_v)));
@@ -1101,7 +1130,7 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     // is never fused; per-token keys are scaled in fp32), so warp 0 sets up q first and
     // its loads overlap the append
     if (warp == 0 && !mbar_wait(pro_bar, 0) && lane == 0) atomicOr(p.status, kStatusWaitExpired);
-    setup_query<KM, D>(q_s + hh * D, smax_k, sm.aq_s, sm.scal_s, c, warp);
+    setup_query<KM, D, NT>(q_s + hh * D, smax_k, sm.aq_s, sm.scal_s, c, warp);
     if (append_here) {
         float own_k, own_v;
         append_token<BK, BV, KM, D>(p, unit, new_blk, (L - 1) & 31, append_scratch, kn_s, vn_s, pro_bar, own_k,
@@ -1236,7 +1265,7 @@ __device__ __forceinline__ void paged_body(const PagedDecodeParams &p, uint8_t *
     const long long qoff = (static_cast<long long>(b) * p.Hkv * G + h * G + (lane >> 2) % G) * D;
     BodyCtx c = make_ctx<INT2 ? 0 : 1, D, NT>(lane, G, smax_v, sm.aq_s);
     c.res = nullptr;
-    setup_query<INT2 ? 0 : 1, D>(p.q + qoff, smax_k, sm.aq_s, sm.scal_s, c, warp);
+    setup_query<INT2 ? 0 : 1, D, NT>(p.q + qoff, smax_k, sm.aq_s, sm.scal_s, c, warp);
     __syncthreads();
     load_query_scalars(c, sm.scal_s);
 
@@ -1282,7 +1311,11 @@ __global__ void __launch_bounds__(NW * 32, 4) decode_paged_kernel(const PagedDec
 // Log-sum-exp merge of the split partials ("merged by online log-sum-exp"), for split
 // counts below kInLaunchMergeSplits.
 __global__ void merge_kernel(const MergeParams p) {
-    pdl_enter();
+    // trigger first: the next kernel (usually the next layer's decode) may launch while the
+    // decode this merge follows is still running (the host counts both as launches the
+    // next one may overlap)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const long long row = blockIdx.x;   // b * Hq + hq
     const float *ml = p.part_ml + row * p.sstride * 2;
     float M = -INFINITY;
@@ -1315,8 +1348,13 @@ KernelFn pick_bits(int bk, int bv) {
     return nullptr;
 }
 
+// Column tiles of the value MMA and layout of the residual query parts: one tile (hi and
+// lo columns side by side, the three residual parts in one MMA) when G divides 4, two
+// tiles otherwise.
+static int nt_for(int G) { return (G == 1 || G == 2 || G == 4) ? 1 : 2; }
+
 KernelFn pick_kernel(int D, int bk, int bv, int kmode, int G) {
-    const int NT = G <= 4 ? 1 : 2;
+    const int NT = nt_for(G);
     if (G < 1 || G > 8) return nullptr;
     if (kmode == 1) {
         // rows (group, head) must fit one 16-row tile and heads must divide 8
@@ -1338,7 +1376,7 @@ KernelFn pick_kernel(int D, int bk, int bv, int kmode, int G) {
 int decode_stages(long long rec_bytes, int D, int G) {
     // per-CTA reserve, q fragments, barriers, prologue
     const long long fixed = 1024 + 3 * (D / 16) * 32 * 16 + 64 + prologue_bytes(D);
-    for (int ctas = (G <= 4 ? 4 : 3); ctas >= 1; --ctas) {
+    for (int ctas = (nt_for(G) == 1 ? 4 : 3); ctas >= 1; --ctas) {
         const long long ns = (228LL * 1024 / ctas - fixed) / (NW * rec_bytes);
         if (ns >= 2) return static_cast<int>(ns > 6 ? 6 : ns);
     }
@@ -1346,7 +1384,7 @@ int decode_stages(long long rec_bytes, int D, int G) {
 }
 
 size_t decode_smem_bytes(long long rec_bytes, int nstage, int nextra, int D, int G) {
-    const int NT = G <= 4 ? 1 : 2;
+    const int NT = nt_for(G);
     return smem_total(NW * nstage + nextra, static_cast<int>(rec_bytes), D, NT);
 }
 

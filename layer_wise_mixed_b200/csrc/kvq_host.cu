@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstring>
 #include <string>
+#include <unordered_map>
 #include <vector>
 
 #include "kvq.h"
@@ -20,6 +21,10 @@ struct kvq_handle {
     kvq_plan_desc desc{};
     std::vector<kvq_layer_cfg> cfg;
     std::vector<LayerGeom> geom;
+    // per stream: the layers whose records or residual the last two launches of this
+    // handle wrote (-1: none), for the decode's early block copies (kvq_internal.h,
+    // pdl_enter)
+    std::unordered_map<const void *, std::pair<int, int>> last_write;
     std::vector<int> len;                    // per layer: the largest request length
     std::vector<std::vector<int>> rlen;      // per-layer plans: per layer, per request
     std::vector<unsigned> ver;               // per layer: appends since bind (scale-maximum slot)
@@ -27,6 +32,11 @@ struct kvq_handle {
     long long status_off = 0, smax_off = 0, arrive_off = 0, meta_bytes = 0, part_acc_off = 0, part_ml_off = 0,
               total = 0;
     long long lens_off = 0;                  // per-layer plans: per layer [2][B] int32 length tables
+    // block pools of per-layer plans (desc.pool_blocks > 0)
+    bool pools = false;
+    std::vector<long long> btab_off;                   // per layer: device block table [B][cap_blk]
+    std::vector<std::vector<int>> free_blocks;         // per layer: free pool blocks (a stack)
+    std::vector<std::vector<std::vector<int>>> blocks; // per layer, per request: pool blocks in order
     uint8_t *ws = nullptr;
     size_t ws_bytes = 0;
     int forced_splits = 0;
@@ -88,6 +98,80 @@ int cuda_fail(cudaError_t e, const char *what);
 // [B] counts for an append.
 int *lens_table(const kvq_handle *h, int layer) {
     return reinterpret_cast<int *>(h->ws + h->lens_off) + 2LL * h->desc.batch * layer;
+}
+
+// A decode launch of `layer` on stream st may copy its first cache blocks before its
+// PDL wait unless one of the two previous launches of this handle on st wrote that
+// layer's cache.  Every launch is noted, with the layer whose cache it writes or -1.
+int may_start_early(const kvq_handle *h, cudaStream_t st, int layer) {
+    const auto it = h->last_write.find(static_cast<const void *>(st));
+    if (it == h->last_write.end()) return 1;
+    return (it->second.first != layer && it->second.second != layer) ? 1 : 0;
+}
+// Block pools: the device block table of `layer` ([B][cap_blk] int32), or null.
+const int *block_table(const kvq_handle *h, int layer) {
+    return h->pools ? reinterpret_cast<const int *>(h->ws + h->btab_off[layer]) : nullptr;
+}
+
+// Block pools: take from the layer's free stack the blocks that every request's new
+// length L_new[b] needs (request order) and list the new table entries (index b * cap_blk
+// + i, value = pool block) in idx / val.  KVQ_ECAPACITY, with nothing taken, if the pool
+// has too few free blocks.
+int reserve_blocks(kvq_handle *h, int layer, const std::vector<int> &L_new, std::vector<int> &idx,
+                   std::vector<int> &val) {
+    if (!h->pools) return KVQ_OK;
+    auto &fb = h->free_blocks[layer];
+    auto &bl = h->blocks[layer];
+    long long need = 0;
+    for (int b = 0; b < h->desc.batch; ++b)
+        need += std::max(0LL, static_cast<long long>((L_new[b] + 31) / 32) - static_cast<long long>(bl[b].size()));
+    if (need > static_cast<long long>(fb.size()))
+        return fail(KVQ_ECAPACITY, "layer %d: block pool exhausted (%lld more blocks needed, %zu of %d free)", layer,
+                    need, fb.size(), h->desc.pool_blocks);
+    for (int b = 0; b < h->desc.batch; ++b)
+        while (static_cast<int>(bl[b].size()) < (L_new[b] + 31) / 32) {
+            const int pid = fb.back();
+            fb.pop_back();
+            idx.push_back(b * h->cap_blk + static_cast<int>(bl[b].size()));
+            val.push_back(pid);
+            bl[b].push_back(pid);
+        }
+    return KVQ_OK;
+}
+
+// Block pools: return the blocks of request b beyond its first `keep` to the free stack.
+void release_blocks(kvq_handle *h, int layer, int b, int keep) {
+    if (!h->pools) return;
+    auto &v = h->blocks[layer][b];
+    while (static_cast<int>(v.size()) > keep) {
+        h->free_blocks[layer].push_back(v.back());
+        v.pop_back();
+    }
+}
+
+void note_write(kvq_handle *h, cudaStream_t st, int layer);
+
+// Block pools: write new table entries on the stream (a launch that writes the layer's
+// table: the next decode of the layer starts no copy before its wait).
+int upload_blocks(kvq_handle *h, int layer, const std::vector<int> &idx, const std::vector<int> &val,
+                  cudaStream_t st) {
+    if (idx.empty()) return KVQ_OK;
+    int *tab = reinterpret_cast<int *>(h->ws + h->btab_off[layer]);
+    cudaError_t e = kvq::launch_scatter_table(tab, idx.data(), val.data(), static_cast<int>(idx.size()), st);
+    if (e != cudaSuccess) return cuda_fail(e, "block table launch");
+    for (size_t i = 0; i < idx.size(); i += 500) note_write(h, st, layer);
+    return KVQ_OK;
+}
+
+void note_write(kvq_handle *h, cudaStream_t st, int layer) {
+
+    auto it = h->last_write.find(static_cast<const void *>(st));
+    if (it == h->last_write.end()) {
+        h->last_write[static_cast<const void *>(st)] = {layer, -1};
+    } else {
+        it->second.second = it->second.first;
+        it->second.first = layer;
+    }
 }
 
 
@@ -226,6 +310,12 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
         return ok();
     }
     h->cap_blk = (d->max_ctx + 31) / 32;
+    if (d->pool_blocks < 0) {
+        delete h;
+        return fail(KVQ_EINVAL, "pool_blocks must be >= 0 (got %d)", d->pool_blocks);
+    }
+    h->pools = d->pool_blocks > 0;
+
     const int D = d->head_dim;
     h->status_off = 0;
     h->smax_off = 256;                                             // after the status word
@@ -265,7 +355,13 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
         g.rec_bytes = g.kc + g.ks + g.vc + g.vs;
         g.unit_bytes = g.rec_bytes * h->cap_blk;
         g.rec_off = off;
-        off = align256(off + g.unit_bytes * max_units);
+        if (h->pools) {   // the layer's pool: pool_blocks blocks of one record per kv head
+            off = align256(off + g.rec_bytes * d->n_kv_heads * static_cast<long long>(d->pool_blocks));
+            h->btab_off.push_back(off);
+            off = align256(off + 4LL * d->batch * h->cap_blk);
+        } else {
+            off = align256(off + g.unit_bytes * max_units);
+        }
         if (c.kmode == KVQ_PER_CHANNEL) {
             g.res_off = off;
             off = align256(off + 64LL * D * max_units);
@@ -283,6 +379,11 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
     h->len.assign(d->num_layers, 0);
     h->ver.assign(d->num_layers, 0u);
     h->rlen.assign(d->num_layers, std::vector<int>(d->batch, 0));
+    if (h->pools) {
+        h->free_blocks.assign(d->num_layers, {});
+        h->blocks.assign(d->num_layers, std::vector<std::vector<int>>(d->batch));
+    }
+
     *out = h;
     return ok();
 }
@@ -312,6 +413,15 @@ int kvq_bind(kvq_handle *h, void *dev_ptr, size_t bytes) {
         for (auto &v : x.page4) v.clear();
         x.next2 = x.next4 = 0;
     }
+    if (h->pools) {   // every block free (taken from the stack's end: block 0 first)
+        for (int l = 0; l < h->desc.num_layers; ++l) {
+            auto &fb = h->free_blocks[l];
+            fb.resize(h->desc.pool_blocks);
+            for (int i = 0; i < h->desc.pool_blocks; ++i) fb[i] = h->desc.pool_blocks - 1 - i;
+            for (auto &v : h->blocks[l]) v.clear();
+        }
+    }
+    h->last_write.clear();
     return ok();
 }
 
@@ -406,16 +516,27 @@ int append_impl(kvq_handle *h, int layer, const void *K, const void *V, const in
     p.nV = static_cast<int>(nV);
     p.nK = static_cast<int>(nK);
     if (p.nV + p.nK == 0) return ok();   // no token appended: nothing changes (the slot neither)
+    std::vector<int> bidx, bval;         // block pools: new table entries
+    {
+        std::vector<int> L_new(B);
+        for (int b = 0; b < B; ++b) L_new[b] = Lo[b] + nn[b];
+        if ((rc = reserve_blocks(h, layer, L_new, bidx, bval))) return rc;
+    }
+    p.btab = block_table(h, layer);
     if ((rc = prepare_status(h, static_cast<cudaStream_t>(stream)))) return rc;
+    if ((rc = upload_blocks(h, layer, bidx, bval, static_cast<cudaStream_t>(stream)))) return rc;
     if (!table.empty()) {
+
         int *dev = lens_table(h, layer);
         cudaError_t e = kvq::launch_set_table(dev, table.data(), static_cast<int>(table.size()),
                                               static_cast<cudaStream_t>(stream));
         if (e != cudaSuccess) return cuda_fail(e, "length table launch");
+        for (size_t i = 0; i < table.size(); i += 1000) note_write(h, static_cast<cudaStream_t>(stream), -1);
         p.ragged_dev = dev;
     }
     cudaError_t e = kvq::launch_append(p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    note_write(h, static_cast<cudaStream_t>(stream), layer);
     int mx = 0;
     for (int b = 0; b < B; ++b) {
         h->rlen[layer][b] = Lo[b] + nn[b];
@@ -445,6 +566,7 @@ int fill_lengths(kvq_handle *h, int layer, kvq::DecodeParams &p, int extra, cuda
         int *dev = lens_table(h, layer);
         cudaError_t e = kvq::launch_set_table(dev, lens.data(), B, st);
         if (e != cudaSuccess) return cuda_fail(e, "length table launch");
+        for (int i = 0; i < B; i += 1000) note_write(h, st, -1);
         p.lens_dev = dev;
     }
     return KVQ_OK;
@@ -542,11 +664,14 @@ int kvq_append_tagged(kvq_handle *h, int layer, const void *K, const void *V, in
         cudaError_t e = kvq::launch_paged_scan(dev_tags, B, n_new, const_cast<int *>(a.inv2), const_cast<int *>(a.inv4),
                                                h->inv_stride, st);
         if (e != cudaSuccess) return cuda_fail(e, "tag scan launch");
+        note_write(h, st, -1);
+
     }
     const long long grid = static_cast<long long>(a.cta4_off[B] + a.cta2_off[B]) * a.Hkv;
     if (grid > 0x7FFFFFFFLL) return fail(KVQ_EUNSUPPORTED, "append too large for one launch");
     cudaError_t e = kvq::launch_paged_append(a, static_cast<int>(grid), st);
     if (e != cudaSuccess) return cuda_fail(e, "paged append launch");
+    note_write(h, st, layer);
     // commit the host-side tables
     for (int b = 0; b < B; ++b) {
         const kvq::PagedReq &r = a.req[b];
@@ -620,6 +745,21 @@ static int splits_for(kvq_handle *h, int layer, int *S_out, int *nstage_out, int
             }
         }
     return KVQ_OK;
+}
+
+// Early block copies pay only for short launches: one wave of CTAs whose warps hold one
+// or two blocks each (the copies then land during the previous kernel's tail).  In longer
+// launches they only put the q rows behind a CTA's block copies (measured on one B200:
+// context-4096 and -8192 layers 3-7% slower with them, the 128-256-token layers of the
+// batch-64 Llama shape 9% faster).
+static bool early_pays(kvq_handle *h, int layer, const kvq::DecodeParams &p) {
+    const LayerGeom &g = h->geom[layer];
+    int occ = 1;
+    if (kvq::decode_occupancy(h->desc.head_dim, g.bk, g.bv, g.kmode, p.G, g.rec_bytes, p.nstage, p.nextra, &occ) !=
+        cudaSuccess)
+        return false;
+    const long long ctas = static_cast<long long>(p.B) * p.Hkv * p.S;
+    return ctas <= static_cast<long long>(occ) * h->sm_count && (p.bps + kvq::kDecodeWarps - 1) / kvq::kDecodeWarps <= 2;
 }
 
 // ------------------------------------------------------------------ paged plans
@@ -705,6 +845,7 @@ static int decode_paged(kvq_handle *h, int layer, const void *q, void *out, int 
     if ((rc = prepare_status(h, st))) return rc;
     cudaError_t e = kvq::launch_decode_paged(p, st);
     if (e != cudaSuccess) return cuda_fail(e, "paged decode launch");
+    note_write(h, st, -1);
     if (S2 + S4 > 1 && !p.arrive) {
         kvq::MergeParams m{};
         m.part_acc = part_acc;
@@ -718,6 +859,7 @@ static int decode_paged(kvq_handle *h, int layer, const void *q, void *out, int 
         m.sstride = p.sstride;
         e = kvq::launch_merge(m, st);
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+        note_write(h, st, -1);
     }
     return ok();
 }
@@ -763,8 +905,11 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
     p.arrive = p.S >= kvq::kInLaunchMergeSplits ? reinterpret_cast<unsigned *>(h->ws + h->arrive_off) : nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = prepare_status(h, st))) return rc;
+    p.btab = block_table(h, layer);
+    p.early = !p.lens_dev && may_start_early(h, st, layer) && early_pays(h, layer, p);
     cudaError_t e = kvq::launch_decode(p, h->desc.head_dim, g.bk, g.bv, g.kmode, st, nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    note_write(h, st, -1);
     if (p.S > 1 && !p.arrive) {
         kvq::MergeParams m{};
         m.part_acc = p.part_acc;
@@ -778,6 +923,7 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
         m.sstride = p.sstride;
         e = kvq::launch_merge(m, st);
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+        note_write(h, st, -1);
     }
     return ok();
 }
@@ -805,6 +951,12 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
         // the group is quantized by the append kernel
         if ((rc = kvq_append(h, layer, K, V, 1, stream))) return rc;
         return kvq_decode_attn(h, layer, q, out, out_fp32, stream);
+    }
+    std::vector<int> bidx, bval;   // block pools: a token that opens a block takes one
+    {
+        std::vector<int> L_new(B);
+        for (int b = 0; b < B; ++b) L_new[b] = h->rlen[layer][b] + 1;
+        if ((rc = reserve_blocks(h, layer, L_new, bidx, bval))) return rc;
     }
     h->len[layer] = L;   // the schedule is chosen for the new length
     int S = 1, nstage = 2, nextra = 0;
@@ -849,11 +1001,19 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
         h->len[layer] = L_old;
         return rc;
     }
+    if ((rc = upload_blocks(h, layer, bidx, bval, st))) {
+        h->len[layer] = L_old;
+        return rc;
+    }
+    p.btab = block_table(h, layer);
+    p.early = !p.lens_dev && may_start_early(h, st, layer) && early_pays(h, layer, p);
+
     cudaError_t e = kvq::launch_decode(p, h->desc.head_dim, g.bk, g.bv, g.kmode, st, nullptr);
     if (e != cudaSuccess) {
         h->len[layer] = L_old;
         return cuda_fail(e, "fused append + decode launch");
     }
+    note_write(h, st, layer);
     for (int b = 0; b < B; ++b) ++h->rlen[layer][b];
     ++h->ver[layer];
     if (p.S > 1 && !p.arrive) {
@@ -869,6 +1029,7 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
         m.sstride = p.sstride;
         e = kvq::launch_merge(m, st);
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+        note_write(h, st, -1);
     }
     return ok();
 }
@@ -996,8 +1157,14 @@ int kvq_export_layer(const kvq_handle *h, int layer, void *host_buf, size_t byte
     const int nj = D / 32;
     for (int u = 0; u < units; img += unit_img(u), ++u) {
         const int L = unit_len(u), nblk = (L + 31) / 32, r = L % 32;
-        if (nblk > 0) {
+        if (nblk > 0 && !h->pools) {
             e = cudaMemcpy(img, h->ws + g.rec_off + u * g.unit_bytes, nblk * g.rec_bytes, cudaMemcpyDeviceToHost);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy (records)");
+        }
+        for (int blk = 0; blk < nblk && h->pools; ++blk) {   // gathered through the block table
+            const long long ri = static_cast<long long>(h->blocks[layer][u / Hkv][blk]) * Hkv + u % Hkv;
+            e = cudaMemcpy(img + blk * g.rec_bytes, h->ws + g.rec_off + ri * g.rec_bytes, g.rec_bytes,
+                           cudaMemcpyDeviceToHost);
             if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy (records)");
         }
         if (res_bytes) {
@@ -1057,8 +1224,27 @@ int kvq_truncate(kvq_handle *h, int layer, int L) {
     if (L % 32) return fail(KVQ_EINVAL, "truncate length must be a multiple of 32 (got %d)", L);
     h->len[layer] = L;
     std::fill(h->rlen[layer].begin(), h->rlen[layer].end(), L);
+    for (int b = 0; b < h->desc.batch; ++b) release_blocks(h, layer, b, L / 32);
     return ok();
 }
+
+int kvq_reset_sequences(kvq_handle *h, const int32_t *seqs, int n) {
+    if (!h || (n > 0 && !seqs)) return fail(KVQ_EINVAL, "null argument");
+    if (h->desc.paged) return fail(KVQ_EUNSUPPORTED, "paged plans cannot reset single sequences");
+    if (n < 0) return fail(KVQ_EINVAL, "n must be >= 0 (got %d)", n);
+    for (int i = 0; i < n; ++i)
+        if (seqs[i] < 0 || seqs[i] >= h->desc.batch)
+            return fail(KVQ_EINVAL, "sequence %d out of range [0, %d)", seqs[i], h->desc.batch);
+    for (int l = 0; l < h->desc.num_layers; ++l) {
+        for (int i = 0; i < n; ++i) {
+            h->rlen[l][seqs[i]] = 0;
+            release_blocks(h, l, seqs[i], 0);
+        }
+        h->len[l] = *std::max_element(h->rlen[l].begin(), h->rlen[l].end());
+    }
+    return ok();
+}
+
 
 int kvq_device_status(kvq_handle *h, void *stream, unsigned *flags) {
     if (!h) return fail(KVQ_EINVAL, "null handle");
@@ -1167,8 +1353,11 @@ int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, 
     p.arrive = p.S >= kvq::kInLaunchMergeSplits ? reinterpret_cast<unsigned *>(h->ws + h->arrive_off) : nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if ((rc = prepare_status(h, st))) return rc;
+    p.btab = block_table(h, layer);
+    p.early = !p.lens_dev && may_start_early(h, st, layer) && early_pays(h, layer, p);
     cudaError_t e = kvq::launch_decode(p, h->desc.head_dim, g.bk, g.bv, g.kmode, st, nullptr);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    note_write(h, st, -1);
     if (p.S > 1 && !p.arrive) {
         kvq::MergeParams m{};
         m.part_acc = p.part_acc;
@@ -1182,6 +1371,7 @@ int kvq_decode_attn_noalloc(kvq_handle *h, int layer, const void *q, void *out, 
         m.sstride = p.sstride;
         e = kvq::launch_merge(m, st);
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+        note_write(h, st, -1);
     }
     return ok();
 }

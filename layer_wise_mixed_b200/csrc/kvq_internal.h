@@ -7,14 +7,21 @@ namespace kvq {
 
 // Programmatic dependent launch.  Every kernel of this library is launched with
 // launch_pdl: it may be scheduled while the previous kernel of the stream is still
-// running, and calls pdl_enter() first, which lets the next kernel's CTAs launch early
-// and then waits until the previous kernel has completed and its memory is visible
-// (griddepcontrol.wait) -- before any global-memory access, so stream order semantics
-// are unchanged and only launch latency and prologues overlap.
+// running.  pdl_enter() first waits until the previous kernel has completed and its
+// memory is visible (griddepcontrol.wait), then lets the next kernel's CTAs launch
+// (griddepcontrol.launch_dependents).  Every global-memory access comes after it, so
+// stream order semantics are unchanged and only launch latency and prologues overlap --
+// with one exception: a decode launch whose host-side plan marks it `early` copies its
+// first cache blocks before pdl_enter().  That is safe because of the order above: when
+// a kernel of this library starts, the kernel before it in the stream has passed its own
+// wait, so every kernel two or more launches back has completed.  The merge kernel alone
+// lets its dependents launch before it waits; it always follows a decode launch, so a
+// kernel may overlap at most the two launches before it, and the host marks a decode
+// launch early only if neither of those writes the blocks it reads.
 #ifdef __CUDACC__
 __device__ __forceinline__ void pdl_enter() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 #endif
 
@@ -35,6 +42,16 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 }
 
 constexpr int kGroup = 32;          // quantization group (tokens or channels)
+
+#ifdef __CUDACC__
+// Index of the record of block blk of (request b, kv head h) in a layer's record area:
+// the unit's slab of cap_blk records, or (block pools, btab != null) the pool block that
+// the table btab [B][cap_blk] assigns to that block of the request, one record per kv head.
+__host__ __device__ __forceinline__ long long rec_index(const int *btab, int b, int Hkv, int h, int cap_blk, int blk) {
+    return btab ? static_cast<long long>(btab[static_cast<long long>(b) * cap_blk + blk]) * Hkv + h
+                : (static_cast<long long>(b) * Hkv + h) * cap_blk + blk;
+}
+#endif
 constexpr int kMaxSplits = 64;      // partial slots per (batch, query head)
 constexpr int kMaxRagged = 64;      // requests whose per-request lengths travel in the kernel
                                     // parameters; larger batches use a device table
@@ -77,6 +94,7 @@ struct AppendParams {
     int ragged;
     int L_old_r[kMaxRagged], n_r[kMaxRagged];
     const int *ragged_dev;
+    const int *btab;            // block pools: [B][cap_blk] pool block of each block (rec is the pool)
 };
 
 struct DecodeParams {
@@ -108,7 +126,13 @@ struct DecodeParams {
     uint8_t *rec_w;
     uint16_t *res_w;
     unsigned *smax_out;
+    // early != 0: the first stages' block copies (and the L2 prefetch of the residual
+    // rows) are issued before pdl_enter(); the host sets it only when the previous launch
+    // in the stream writes none of this layer's records or residual (see pdl_enter)
+    int early;
+    const int *btab;            // block pools: [B][cap_blk] pool block of each block (rec is the pool)
 };
+
 
 // ---------------------------------------------------------------- paged INT2/INT4
 constexpr int kMaxPagedBatch = 64;   // requests per paged plan (kernel-parameter tables)
@@ -189,6 +213,9 @@ cudaError_t launch_append(const AppendParams &p, cudaStream_t st);
 // value into CUDA graphs, and each launch writes only after the preceding kernel of the
 // stream has completed (programmatic dependent launch waits first).
 cudaError_t launch_set_table(int *dst, const int *vals, int n, cudaStream_t st);
+// The same for n scattered entries: dst[idx[i]] = vals[i] (500 per launch).
+cudaError_t launch_scatter_table(int *dst, const int *idx, const int *vals, int n, cudaStream_t st);
+
 
 // Returns cudaErrorInvalidValue if no kernel exists for the combination.
 cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmode,

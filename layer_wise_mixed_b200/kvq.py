@@ -47,7 +47,8 @@ class kvq_plan_desc(ctypes.Structure):
     _fields_ = [("num_layers", ctypes.c_int), ("batch", ctypes.c_int), ("n_kv_heads", ctypes.c_int),
                 ("n_q_heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("group", ctypes.c_int),
                 ("max_ctx", ctypes.c_int), ("layers", ctypes.POINTER(kvq_layer_cfg)),
-                ("paged", ctypes.c_int), ("page_tokens", ctypes.c_int), ("avg_bits", ctypes.c_float)]
+                ("paged", ctypes.c_int), ("page_tokens", ctypes.c_int), ("avg_bits", ctypes.c_float),
+                ("pool_blocks", ctypes.c_int)]
 
 
 _lib = None
@@ -78,6 +79,7 @@ def load() -> ctypes.CDLL:
         "kvq_export_layer": (I, [P, I, P, SZ, ctypes.POINTER(SZ)]),
         "kvq_seq_len": (I, [P, I, ctypes.POINTER(I)]),
         "kvq_truncate": (I, [P, I, I]),
+        "kvq_reset_sequences": (I, [P, P, I]),
         "kvq_device_status": (I, [P, P, ctypes.POINTER(ctypes.c_uint)]),
         "kvq_tag_distortion": (I, [I, I, I, I, I, I, P, P, P, P, I, P, P, P]),
         "kvq_tag_allocate": (I, [I, P, P, P, ctypes.c_double, P, P]),
@@ -202,6 +204,11 @@ def kvq_truncate(h: int, layer: int, L: int):
     _check(load().kvq_truncate(h, layer, L))
 
 
+def kvq_reset_sequences(h: int, seqs):
+    n = np.ascontiguousarray(seqs, np.int32)
+    _check(load().kvq_reset_sequences(h, n.ctypes.data_as(ctypes.c_void_p), n.size))
+
+
 def kvq_device_status(h: int, stream=None) -> int:
     f = ctypes.c_uint()
     rc = load().kvq_device_status(h, _stream(stream), ctypes.byref(f))
@@ -256,15 +263,15 @@ def kvq_tag_allocate(D2, D4, counts, avg_bits: float):
 # ------------------------------------------------------------------ convenience owner
 def make_paged_desc(num_layers: int, batch: int, n_kv_heads: int, n_q_heads: int, head_dim: int, max_ctx: int,
                     avg_bits: float):
-    return kvq_plan_desc(num_layers, batch, n_kv_heads, n_q_heads, head_dim, 32, max_ctx, None, 1, 16, avg_bits)
+    return kvq_plan_desc(num_layers, batch, n_kv_heads, n_q_heads, head_dim, 32, max_ctx, None, 1, 16, avg_bits, 0)
 
 
 def make_desc(num_layers: int, batch: int, n_kv_heads: int, n_q_heads: int, head_dim: int, max_ctx: int,
-              layer_bits: Sequence[Tuple[int, int]], kmodes: Optional[Sequence[int]] = None):
+              layer_bits: Sequence[Tuple[int, int]], kmodes: Optional[Sequence[int]] = None, pool_blocks: int = 0):
     cfgs = (kvq_layer_cfg * num_layers)()
     for i, (bk, bv) in enumerate(layer_bits):
         cfgs[i] = kvq_layer_cfg(bk, bv, KVQ_PER_CHANNEL if kmodes is None else kmodes[i], KVQ_PER_TOKEN)
-    d = kvq_plan_desc(num_layers, batch, n_kv_heads, n_q_heads, head_dim, 32, max_ctx, cfgs, 0, 16, 0.0)
+    d = kvq_plan_desc(num_layers, batch, n_kv_heads, n_q_heads, head_dim, 32, max_ctx, cfgs, 0, 16, 0.0, pool_blocks)
     d._cfgs = cfgs   # keep the array alive with the descriptor
     return d
 
@@ -274,12 +281,13 @@ class Cache:
     avg_bits (and no layer_bits) for a paged INT2/INT4 plan."""
 
     def __init__(self, num_layers, batch, n_kv_heads, n_q_heads, head_dim, max_ctx, layer_bits=None,
-                 kmodes=None, device="cuda", avg_bits=None):
+                 kmodes=None, device="cuda", avg_bits=None, pool_blocks=0):
         import torch
         if avg_bits is not None:
             self.desc = make_paged_desc(num_layers, batch, n_kv_heads, n_q_heads, head_dim, max_ctx, avg_bits)
         else:
-            self.desc = make_desc(num_layers, batch, n_kv_heads, n_q_heads, head_dim, max_ctx, layer_bits, kmodes)
+            self.desc = make_desc(num_layers, batch, n_kv_heads, n_q_heads, head_dim, max_ctx, layer_bits, kmodes,
+                                  pool_blocks)
         self.h = kvq_plan(self.desc)
         self._destroy = load().kvq_destroy   # held so that teardown at interpreter exit still works
         self.nbytes = kvq_workspace_bytes(self.h)

@@ -200,3 +200,44 @@ def test_paged_host_checks(lib):
         assert need.value == 2 * 2 * (2 * 20 * 128 + 2 * 32 * 128 * 2)   # empty: pending pages + staging
     finally:
         kvq.kvq_destroy(h)
+
+
+def test_block_pool_plan_layout_and_checks(lib):
+    """Block pools: the layer regions hold the pool and the block table instead of the
+    slabs; an append the pool cannot hold is refused before any launch and leaves the
+    lengths as they were; kvq_reset_sequences checks its arguments."""
+    import numpy as np
+    L = kvq.load()
+    D, B, Hkv, Hq, cap, P = 64, 2, 2, 4, (100 + 31) // 32, 3
+    d = kvq.make_desc(2, B, Hkv, Hq, D, 100, [(4, 2), (8, 8)], None, pool_blocks=P)
+    h = kvq.kvq_plan(d)
+    try:
+        rec0 = 4 * D * 4 + 4 * D + 4 * D * 2 + 4 * D
+        rec1 = 4 * D * 8 + 4 * D + 4 * D * 8 + 4 * D
+        al = lambda x: (x + 255) // 256 * 256
+        expect = al(256 + 16 * 2)
+        expect = al(expect + 4 * B * Hkv)
+        expect = al(expect + 8 * B * 2)
+        expect = al(expect + rec0 * Hkv * P)            # layer 0 pool
+        expect = al(expect + 4 * B * cap)               # layer 0 block table
+        expect = al(expect + 64 * D * B * Hkv)          # residual (per-channel keys)
+        expect = al(expect + rec1 * Hkv * P)
+        expect = al(expect + 4 * B * cap)
+        expect = al(expect + 64 * D * B * Hkv)
+        expect = al(expect + B * Hq * 64 * D * 4)
+        expect = al(expect + B * Hq * 64 * 2 * 4)
+        assert kvq.kvq_workspace_bytes(h) == expect
+        fake = 1 << 40
+        assert L.kvq_bind(h, fake, expect) == kvq.KVQ_OK
+        # 2 sequences x 2 blocks (64 tokens) > 3 pool blocks: refused before any launch
+        assert L.kvq_append(h, 0, fake, fake, 64, None) == kvq.KVQ_ECAPACITY
+        assert "block pool" in kvq.kvq_last_error()
+        assert list(kvq.kvq_seq_lens(h, 0, B)) == [0, 0]
+        p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+        assert L.kvq_reset_sequences(h, p(np.array([0, 2], np.int32)), 2) == kvq.KVQ_EINVAL   # out of range
+        assert L.kvq_reset_sequences(h, None, 1) == kvq.KVQ_EINVAL
+        assert L.kvq_reset_sequences(h, p(np.array([1], np.int32)), 1) == kvq.KVQ_OK
+    finally:
+        kvq.kvq_destroy(h)
+    d = kvq.make_desc(1, B, Hkv, Hq, D, 100, [(4, 2)], None, pool_blocks=-1)
+    assert plan_rc(d) == kvq.KVQ_EINVAL
