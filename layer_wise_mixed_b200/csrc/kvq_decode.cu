@@ -1060,12 +1060,14 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     WarpPipe P{sm.stages + static_cast<size_t>(sbase) * REC, sm.bars + sbase, NS, REC, lane, 0, 0, 0u, 0};
     pipe_init(P);
     const int nb = (blk1 - blk0 > warp) ? (blk1 - blk0 - warp + NW - 1) / NW : 0;
+    const uint8_t *unit_rec = p.rec + (static_cast<long long>(b) * p.Hkv + h) * p.cap_blk * REC;   // slab plans
     // per-channel keys of the last, incomplete group come from the residual: fetch only
     // the value part of that block's record
     constexpr unsigned VSKIP = KM == 0 ? 2 * 2 * D * BK + 4 * D : 0;
     auto issue_block = [&](int k) {
         const int blk = blk0 + warp + NW * k;
-        const uint8_t *src = p.rec + rec_index(p.btab, b, p.Hkv, h, p.cap_blk, blk) * REC;
+        const uint8_t *src = p.btab ? p.rec + rec_index(p.btab, b, p.Hkv, h, p.cap_blk, blk) * REC
+                                    : unit_rec + static_cast<long long>(blk) * REC;
         if (blk == tail_blk) pipe_issue(P, src + VSKIP, REC - VSKIP, VSKIP);
         else pipe_issue(P, src, REC);
     };
