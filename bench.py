@@ -97,6 +97,43 @@ def rank_workload(wl, rank, world):
     return dataclasses.replace(wl, name=f"{wl.name}-rank{rank}")
 
 
+def link_bound(h2d, d2h, stream, h2d_stream, d2h_stream, world, barrier, steps=16):
+    """Bound of the end-to-end loop set by the host link alone: per step one pinned H2D of
+    the step's input bytes and one D2H of its output bytes, issued on two copy streams at
+    once (the loop's own pattern), nothing else on the GPU; CUDA events, max over ranks."""
+    import torch
+    hi = torch.empty(h2d // 2, dtype=torch.bfloat16).pin_memory()
+    di = torch.empty(h2d // 2, dtype=torch.bfloat16, device="cuda")
+    do = torch.zeros(d2h // 2, dtype=torch.bfloat16, device="cuda")
+    ho = torch.empty(d2h // 2, dtype=torch.bfloat16).pin_memory()
+
+    def run(n):
+        h2d_stream.wait_stream(stream)
+        d2h_stream.wait_stream(stream)
+        for _ in range(n):
+            with torch.cuda.stream(h2d_stream):
+                di.copy_(hi, non_blocking=True)
+            with torch.cuda.stream(d2h_stream):
+                ho.copy_(do, non_blocking=True)
+        stream.wait_stream(h2d_stream)
+        stream.wait_stream(d2h_stream)
+
+    with torch.cuda.stream(stream):
+        run(3)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run(steps)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    del hi, di, do, ho
+    return {"ms_per_step": ms, "h2d_gbs": h2d / (ms / 1e3) / 1e9, "d2h_gbs": d2h / (ms / 1e3) / 1e9,
+            "how": "pinned H2D of the step's input bytes and D2H of its output bytes on two copy streams at once, "
+                   "nothing else running; tokens_s = batch per such step, frac = e2e / tokens_s"}
+
+
 def max_over_ranks(value_ms, world):
     """Max of a per-rank time over all ranks (rank 0 reports it); plain value at N=1."""
     if world <= 1:
@@ -646,6 +683,9 @@ def main():
     e2e_value = world * B * e2e_steps / (e2e_ms / 1e3)
     h2d = NL * per * 2
     d2h = out.numel() * 2
+    link = link_bound(h2d, d2h, stream, h2d_stream, d2h_stream, world, barrier)
+    link["tokens_s"] = world * B / (link["ms_per_step"] / 1e3)
+    link["frac"] = e2e_value / link["tokens_s"]
     status = kvq.kvq_device_status(cache.h, stream)
     head_cfg = workload_config(wl)
     head_cfg["context"] = run.context(order)
@@ -737,7 +777,8 @@ def main():
                 "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                         "steps": e2e_steps, "how": e2e_note,
                         "host_link_gbs": {"h2d": h2d * e2e_steps / (e2e_ms / 1e3) / 1e9,
-                                          "d2h": d2h * e2e_steps / (e2e_ms / 1e3) / 1e9}},
+                                          "d2h": d2h * e2e_steps / (e2e_ms / 1e3) / 1e9},
+                        "link_bound": link},
                 "gpu_launches": gpu_launches, "clocks": clocks, "device_status": status,
                 "splits": head_splits,
                 "per_config": per_config}

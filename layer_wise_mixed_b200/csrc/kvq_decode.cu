@@ -824,7 +824,7 @@ __device__ __forceinline__ void combine_store(WarpAcc<D, NT> &A, const BodyCtx &
         } else {
             *reinterpret_cast<float4 *>(part_acc + (row * sstride + sp) * D + d) = val;
             if (d == 0) {
-                part_ml[(row * sstride + sp) * 2] = M;
+                part_ml[(row * sstride + sp) * 2] = M - c.pbias;   // den and val carry 2^pbias
                 part_ml[(row * sstride + sp) * 2 + 1] = den;
             }
         }
@@ -932,76 +932,128 @@ __device__ __forceinline__ void or_token(uint32_t *area, int role, int e, const 
     }
 }
 
-// Quantize and pack the token appended by a fused launch, token u of block `blk` of unit
-// `unit`, with the same arithmetic as the append kernel: values per token (one warp per
-// 32-channel group), keys per token the same way or, per channel, the new row into the
-// residual (slot u: the host takes the two-launch path when the token completes a key
-// group).  All threads of the CTA take part.  The cache in HBM gets the new bytes for
-// later steps; this launch does not read them back: the warp that processes the block
-// patches its staged copy (patch_stage) from the codes, scales and zeros kept in
-// `scratch`.  own_k / own_v: the CTA's largest new scales.
+// Quantize the token appended by a fused launch (token u of its block) in one warp, with
+// the append kernel's arithmetic: each 32-channel group of the value row (and, per-token
+// keys, of the key row) is held by 32/CPL lanes of CPL channels, so the warp quantizes
+// every group at once.  Codes, scales and zeros go to `scratch` (shared memory), from
+// which the warp that processes the block patches its staged copy (patch_stage); the
+// cache in HBM gets them from append_token_store.  Returns the new scale maxima (keys,
+// values; fp16 bits) on every lane.
 template <int BK, int BV, int KM, int D>
-__device__ __forceinline__ void append_token(const DecodeParams &p, long long unit, int blk, int u,
-                                             uint8_t *scratch, const uint16_t *kn, const uint16_t *vn,
-                                             uint64_t *pro_bar, float &own_k, float &own_v) {
-    constexpr int NJ = D / 32;
-    constexpr int KC = 4 * D * BK, KSZ = 4 * D, VC = 4 * D * BV;
-    constexpr int REC = KC + KSZ + VC + 4 * D;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = u & 15, eta = u >> 4;
-    uint8_t *rec = p.rec_w + rec_index(p.btab, static_cast<int>(unit / p.Hkv), p.Hkv, static_cast<int>(unit % p.Hkv),
-                                       p.cap_blk, blk) * static_cast<long long>(REC);
-    uint8_t *codes = scratch;                                          // [0, D): values, [D, 2D): keys
-    unsigned *cmax = reinterpret_cast<unsigned *>(scratch + 2 * D);   // keys, values (fp16 bits)
+__device__ __forceinline__ void append_token_quantize(uint8_t *scratch, const uint16_t *kn, const uint16_t *vn,
+                                                      int lane, unsigned smax_new[2]) {
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    constexpr int NJ = D / 32, CPL = D / 32, LPG = 32 / CPL;
+    uint8_t *codes = scratch;                                              // [0, D): values, [D, 2D): keys
     uint16_t *szs = reinterpret_cast<uint16_t *>(scratch + 2 * D + 16);   // [role][j][scale, zero]
-    if (threadIdx.x < 2) cmax[threadIdx.x] = 0u;
-    __syncthreads();
-    // the token's rows (kn, vn) arrive by bulk copy with the q rows
-    if (!mbar_wait(pro_bar, 0) && (threadIdx.x & 31) == 0) atomicOr(p.status, kStatusWaitExpired);
+    const int j = lane / LPG, d0 = CPL * lane;   // this lane's group and first channel
+    smax_new[0] = smax_new[1] = 0u;
     constexpr int NROLE = KM == 1 ? 2 : 1;
-    for (int it = warp; it < NROLE * NJ; it += NW) {
-        const int role = it < NJ ? 1 : 0;
-        const int j = it % NJ;
-        const int bits = role ? BV : BK;
-        const uint16_t *src = role ? vn : kn;
-        const float x = quant::bf16_to_f32(src[32 * j + lane]);
-        float mn = x, mx = x;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
+    for (int r = 0; r < NROLE; ++r) {
+        const int role = r == 0 ? 1 : 0;   // values, then (per-token keys) keys
+        const int bits = role ? BV : BK;
+        const uint16_t *src = (role ? vn : kn) + d0;
+        float x[CPL];
+        if constexpr (CPL == 4) {
+            const uint2 w = *reinterpret_cast<const uint2 *>(src);
+            x[0] = __uint_as_float(w.x << 16);
+            x[1] = __uint_as_float(w.x & 0xFFFF0000u);
+            x[2] = __uint_as_float(w.y << 16);
+            x[3] = __uint_as_float(w.y & 0xFFFF0000u);
+        } else {
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(src);
+            x[0] = __uint_as_float(w << 16);
+            x[1] = __uint_as_float(w & 0xFFFF0000u);
+        }
+        float mn = x[0], mx = x[0];
+#pragma unroll
+        for (int i = 1; i < CPL; ++i) {
+            mn = fminf(mn, x[i]);
+            mx = fmaxf(mx, x[i]);
+        }
+#pragma unroll
+        for (int o = LPG / 2; o > 0; o >>= 1) {
             mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         }
         float sc, z;
         uint16_t s16, z16;
         quant::group_params(mn, mx, bits, sc, z, s16, z16);
-        codes[(role ? 0 : D) + 32 * j + lane] = static_cast<uint8_t>(quant::group_code(x, sc, z, bits));
-        if (lane == 0) {
-            uint8_t *sz = rec + (role ? KC + KSZ + VC : KC);
-            const int so = quant::tok_sz_off(u, j, NJ);
-            *reinterpret_cast<uint16_t *>(sz + so) = s16;
-            *reinterpret_cast<uint16_t *>(sz + so + 4 * NJ) = z16;
+        uint32_t packed = 0u;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) packed |= static_cast<uint32_t>(quant::group_code(x[i], sc, z, bits)) << (8 * i);
+        if constexpr (CPL == 4) *reinterpret_cast<uint32_t *>(codes + (role ? 0 : D) + d0) = packed;
+        else *reinterpret_cast<uint16_t *>(codes + (role ? 0 : D) + d0) = static_cast<uint16_t>(packed);
+        if (lane % LPG == 0) {
             szs[(role * NJ + j) * 2] = s16;
             szs[(role * NJ + j) * 2 + 1] = z16;
-            atomicMax(cmax + role, static_cast<unsigned>(s16));
         }
+        smax_new[role] = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(s16));
     }
-    if constexpr (KM == 0) {
-        const uint32_t *src = reinterpret_cast<const uint32_t *>(kn);
-        uint32_t *dst = reinterpret_cast<uint32_t *>(p.res_w + (unit * 32 + u) * D);
-        for (int i = threadIdx.x; i < D / 2; i += NW * 32) dst[i] = src[i];
+    __syncwarp();
+}
+
+// Per-channel keys: the new key row into the residual of unit `unit` (slot u: the host
+// takes the two-launch path when the token completes a key group).  One warp.
+template <int D>
+__device__ __forceinline__ void append_residual_row(const DecodeParams &p, long long unit, int u, const uint16_t *kn,
+                                                    int lane) {
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(kn);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(p.res_w + (unit * 32 + u) * D);
+    for (int i = lane; i < D / 2; i += 32) dst[i] = src[i];
+    __syncwarp();   // the warp's own later reads of the row (when it holds the block)
+}
+
+// The quantized token (append_token_quantize's `scratch`) into the cache in HBM for later
+// launches: its code fields (the half's words rebuilt from zero when it is the half's
+// first token), scales and zeros in the block record of unit `unit`, and the layer's scale
+// maxima.  One warp.
+template <int BK, int BV, int KM, int D>
+__device__ __forceinline__ void append_token_store(const DecodeParams &p, long long unit, int blk, int u,
+                                                   const uint8_t *scratch, int lane, const unsigned smax_new[2]) {
+    constexpr int NJ = D / 32;
+    constexpr int KC = 4 * D * BK, KSZ = 4 * D, VC = 4 * D * BV;
+    constexpr int REC = KC + KSZ + VC + 4 * D;
+    const int e = u & 15, eta = u >> 4;
+    uint8_t *rec = p.rec_w + rec_index(p.btab, static_cast<int>(unit / p.Hkv), p.Hkv, static_cast<int>(unit % p.Hkv),
+                                       p.cap_blk, blk) * static_cast<long long>(REC);
+    const uint8_t *codes = scratch;
+    const uint16_t *szs = reinterpret_cast<const uint16_t *>(scratch + 2 * D + 16);
+    if (lane < (KM == 1 ? 2 : 1) * NJ) {   // lane = role-major (values, then keys) group
+        const int role = lane < NJ ? 1 : 0, j = lane % NJ;
+        uint8_t *sz = rec + (role ? KC + KSZ + VC : KC);
+        const int so = quant::tok_sz_off(u, j, NJ);
+        *reinterpret_cast<uint16_t *>(sz + so) = szs[(role * NJ + j) * 2];
+        *reinterpret_cast<uint16_t *>(sz + so + 4 * NJ) = szs[(role * NJ + j) * 2 + 1];
     }
     uint32_t *vwords = reinterpret_cast<uint32_t *>(rec + KC + KSZ + eta * 2 * D * BV);
     uint32_t *kwords = reinterpret_cast<uint32_t *>(rec + eta * 2 * D * BK);
     if (e == 0) {   // the half's first token: its words are rebuilt from zero
-        zero_half<BV>(vwords, threadIdx.x, NW * 32, D);
-        if constexpr (KM == 1) zero_half<BK>(kwords, threadIdx.x, NW * 32, D);
+        zero_half<BV>(vwords, lane, 32, D);
+        if constexpr (KM == 1) zero_half<BK>(kwords, lane, 32, D);
+        __syncwarp();
     }
-    __syncthreads();
-    or_token<BV>(vwords, 1, e, codes, threadIdx.x, NW * 32, D);
-    if constexpr (KM == 1) or_token<BK>(kwords, 0, e, codes + D, threadIdx.x, NW * 32, D);
-    own_k = __half2float(__ushort_as_half(static_cast<unsigned short>(cmax[0])));
-    own_v = __half2float(__ushort_as_half(static_cast<unsigned short>(cmax[1])));
-    if (threadIdx.x < 2 && cmax[threadIdx.x]) atomicMax(p.smax_out + threadIdx.x, cmax[threadIdx.x]);
+    or_token<BV>(vwords, 1, e, codes, lane, 32, D);
+    if constexpr (KM == 1) or_token<BK>(kwords, 0, e, codes + D, lane, 32, D);
+    if (lane == 0) {
+        if (smax_new[0]) atomicMax(p.smax_out, smax_new[0]);
+        if (smax_new[1]) atomicMax(p.smax_out + 1, smax_new[1]);
+    }
+}
+
+// Upper bound of the fp16 value scales of a new row: a 32-channel group's scale is at
+// most 2 max|v| / (2^BV - 1), and rounding it to fp16 (or to a subnormal step) raises it
+// by less than the margin.  Warp-wide (every lane gets it).
+template <int BV, int D>
+__device__ __forceinline__ float new_value_scale_bound(const uint16_t *vn, int lane) {
+    // max |v| from the bf16 magnitude bits (ordered like the values they encode)
+    unsigned mb = 0u;
+#pragma unroll
+    for (int d = lane; d < D; d += 32) mb = max(mb, static_cast<unsigned>(vn[d]) & 0x7FFFu);
+    mb = __reduce_max_sync(0xffffffffu, mb);
+    const float m = quant::bf16_to_f32(static_cast<uint16_t>(mb));
+    return m * (2.0f / static_cast<float>((1 << BV) - 1)) * (1.0f + 0x1p-9f) + 0x1p-24f;
 }
 
 // The warp that processes the appended token's block writes the token into its staged
@@ -1129,18 +1181,40 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     c.res = p.res ? p.res + (static_cast<long long>(b) * p.Hkv + h) * 32 * D : nullptr;
     const int hh = c.g % G;
     // the key prescale needs no new scale (a token that completes a per-channel key group
-    // is never fused; per-token keys are scaled in fp32), so warp 0 sets up q first and
-    // its loads overlap the append
+    // is never fused; per-token keys are scaled in fp32)
     if (warp == 0 && !mbar_wait(pro_bar, 0) && lane == 0) atomicOr(p.status, kStatusWaitExpired);
     setup_query<KM, D, NT>(q_s + hh * D, smax_k, sm.aq_s, sm.scal_s, c, warp);
-    if (append_here) {
-        float own_k, own_v;
-        append_token<BK, BV, KM, D>(p, unit, new_blk, (L - 1) & 31, append_scratch, kn_s, vn_s, pro_bar, own_k,
-                                    own_v);
-        c.pbias = value_bias(fmaxf(smax_v, own_v));   // CTA-uniform: every warp's p carries it
-    }
     __syncthreads();
     load_query_scalars(c, sm.scal_s);
+    // the value prescale must cover the new token's scales: every warp bounds them from
+    // the new row (the same CTA-uniform result; the row has arrived: warp 0 waited for it)
+    if (append_here) {
+        if (!mbar_wait(pro_bar, 0) && lane == 0) atomicOr(p.status, kStatusWaitExpired);
+        c.pbias = value_bias(fmaxf(smax_v, new_value_scale_bound<BV, D>(vn_s, lane)));
+    }
+    // the append runs in the warp with the fewest blocks (the block's own warp when none
+    // has fewer), before its blocks; the block's warp waits for it (named barrier 1) only
+    // before patching its staged copy, its last block
+    int owner = 0, helper = 0;
+    if (append_here) {
+        auto blocks_of = [&](int w) { return (blk1 - blk0 > w) ? (blk1 - blk0 - w + NW - 1) / NW : 0; };
+        owner = (new_blk - blk0) % NW;
+        helper = owner;
+        for (int w = NW - 1; w >= 0; --w)
+            if (blocks_of(w) < blocks_of(helper)) helper = w;
+        if (warp == helper) {
+            // the token's rows (kn, vn) arrive by bulk copy with the q rows
+            if (!mbar_wait(pro_bar, 0) && lane == 0) atomicOr(p.status, kStatusWaitExpired);
+            unsigned smax_new[2];
+            append_token_quantize<BK, BV, KM, D>(append_scratch, kn_s, vn_s, lane, smax_new);
+            // the tail reads the new residual row from HBM after the hand-over; the record's
+            // words, scales and the maxima are only for later launches: written after it,
+            // so the barrier's release does not wait for them
+            if constexpr (KM == 0) append_residual_row<D>(p, unit, (L - 1) & 31, kn_s, lane);
+            if (helper != owner) asm volatile("bar.arrive 1, %0;" ::"n"(64) : "memory");
+            append_token_store<BK, BV, KM, D>(p, unit, new_blk, (L - 1) & 31, append_scratch, lane, smax_new);
+        }
+    }
 
     WarpAcc<D, NT> A;
     acc_init(A);
@@ -1162,6 +1236,10 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
         pipe_pop(P);
         if (P.issued < nb) issue_block(P.issued);
     }
+    // the helper's codes, scales and zeros are in shared memory and the new residual row
+    // in HBM (every path of the owner passes here once; the helper arrives after its
+    // quantize, whose wait is bounded)
+    if (append_here && warp == owner && helper != owner) asm volatile("bar.sync 1, %0;" ::"n"(64) : "memory");
     if constexpr (KM == 1) {
         if (!failed && patch_full) {
             if (!pipe_wait(P)) {
@@ -1178,7 +1256,8 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
         if (!pipe_wait(P)) {
             failed = true;
         } else {
-            if (append_here && tail_blk == new_blk)
+            const bool patch = append_here && tail_blk == new_blk;
+            if (patch)
                 patch_stage<BK, BV, KM, D>(const_cast<uint8_t *>(pipe_front(P)), (L - 1) & 31, append_scratch, lane);
             process_unit<BK, BV, KM, D, NT, 2, true>(A, pipe_front(P), rem, c);
             ++i;

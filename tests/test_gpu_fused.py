@@ -153,3 +153,43 @@ def test_fused_c2_full_size_graphs():
             check_outputs(outs[l], out16, out_ref, f"c2 full L={L} layer {l}")
         del g
     assert kvq.kvq_device_status(cache.h) == 0
+
+
+@pytest.mark.parametrize("kmode", [0, 1])
+@pytest.mark.parametrize("bits", [(8, 4), (4, 2)], ids=["K8V4", "K4V2"])
+def test_fused_split_value_scale_jump(kmode, bits):
+    """Fused steps whose new value row is 2^4 to 2^11 times larger than every value before
+    it, under forced splits: the CTA that appends the token takes a smaller value
+    prescale than the other splits of the same (b, kv head) (it sees the new scale, they
+    see the layer's old maxima), and the split merge must weigh the partials by their
+    true maxima (a sum over tokens split into parts: the KVTuner summary's flash-decoding
+    kernels and the TriAxialKV page's LSE merge of splits)."""
+    bk, bv = bits
+    B, Hkv, G, D = 2, 2, 4, 128
+    prefill = 100
+    wl = workload(B, Hkv, G, D, name=f"jump{kmode}{bk}{bv}")
+    jumps = [(2, 5), (3, 9), (5, 12)]   # (splits, log2 of the new row's scale-up)
+    L_total = prefill + len(jumps)
+    K, V = inputs.layer_kv(wl, 0, L_total, "cuda")
+    V = V.float()
+    V[:, :, :prefill] *= 2.0                                  # value scales near 1
+    for i, (_, e) in enumerate(jumps):
+        V[:, :, prefill + i] *= 2.0 ** e
+    V = V.to(torch.bfloat16)
+    Kb, Vb = bits16(K), bits16(V)
+    cache = kvq.Cache(1, B, Hkv, Hkv * G, D, L_total, [bits], kmodes=[kmode])
+    cache.append(0, K[:, :, :prefill].contiguous(), V[:, :, :prefill].contiguous())
+    for i, (S, _) in enumerate(jumps):
+        L = prefill + i + 1
+        kvq.kvq_set_num_splits(cache.h, S)
+        q = inputs.step_q(wl, 0, L, "cuda")
+        out32 = cache.append_decode(0, K[:, :, L - 1:L].contiguous(), V[:, :, L - 1:L].contiguous(), q,
+                                    out_fp32=True)
+        torch.cuda.synchronize()
+        img_ref, out_ref = oracle.layer(Kb[:, :, :L], Vb[:, :, :L], bits16(q), G, bk, bv, kmode)
+        img = cache.export_layer(0)
+        if not np.array_equal(img, img_ref):
+            bad = np.flatnonzero(img != img_ref)
+            pytest.fail(f"L={L}: image differs at {bad.size} bytes, first {bad[:8]}")
+        check_outputs(out32, out32.to(torch.bfloat16), out_ref, f"jump splits={S} L={L}")
+    assert kvq.kvq_device_status(cache.h) == 0
