@@ -1090,7 +1090,9 @@ __device__ __forceinline__ void patch_stage(uint8_t *stage, int u, const uint8_t
 }
 
 // ------------------------------------------------------------------ per-layer kernel
-template <int BK, int BV, int KM, int D, int NT>
+// FUSED: the instance for kvq_append_decode launches (p.k_new set); decode-only launches
+// take the instance without the append code.
+template <int BK, int BV, int KM, int D, int NT, bool FUSED>
 __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(const DecodeParams p) {
     const bool early = p.early != 0;   // CTA-uniform
     if (!early) pdl_enter();
@@ -1144,7 +1146,7 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
     const unsigned smax_bits_k = p.smax[0], smax_bits_v = p.smax[1];
     // a fused launch appends token L - 1 (the last of block new_blk) in the CTA that holds
     // that block; the block's warp patches its staged copy with the token
-    const bool fused = p.k_new != nullptr;
+    const bool fused = FUSED && p.k_new != nullptr;
     const int new_blk = (L - 1) >> 5;
     const bool append_here = fused && new_blk >= blk0 && new_blk < blk1;   // CTA-uniform
     uint8_t *append_scratch = reinterpret_cast<uint8_t *>(sm.scal_s + 32);
@@ -1418,10 +1420,10 @@ __global__ void merge_kernel(const MergeParams p) {
 
 using KernelFn = void (*)(const DecodeParams);
 
-template <int D, int NT, int KM>
+template <int D, int NT, int KM, bool FUSED>
 KernelFn pick_bits(int bk, int bv) {
 #define KVQ_CASE(BKv, BVv) \
-    if (bk == BKv && bv == BVv) return decode_split_kernel<BKv, BVv, KM, D, NT>;
+    if (bk == BKv && bv == BVv) return decode_split_kernel<BKv, BVv, KM, D, NT, FUSED>;
     KVQ_CASE(2, 2) KVQ_CASE(2, 4) KVQ_CASE(2, 8)
     KVQ_CASE(4, 2) KVQ_CASE(4, 4) KVQ_CASE(4, 8)
     KVQ_CASE(8, 2) KVQ_CASE(8, 4) KVQ_CASE(8, 8)
@@ -1434,19 +1436,24 @@ KernelFn pick_bits(int bk, int bv) {
 // tiles otherwise.
 static int nt_for(int G) { return (G == 1 || G == 2 || G == 4) ? 1 : 2; }
 
-KernelFn pick_kernel(int D, int bk, int bv, int kmode, int G) {
+template <bool FUSED>
+KernelFn pick_kernel_t(int D, int bk, int bv, int kmode, int G) {
     const int NT = nt_for(G);
     if (G < 1 || G > 8) return nullptr;
     if (kmode == 1) {
         // rows (group, head) must fit one 16-row tile and heads must divide 8
         if (!(G == 1 || G == 2 || G == 4) || G * (D / 32) > 16) return nullptr;
-        if (D == 64) return pick_bits<64, 1, 1>(bk, bv);
-        if (D == 128) return pick_bits<128, 1, 1>(bk, bv);
+        if (D == 64) return pick_bits<64, 1, 1, FUSED>(bk, bv);
+        if (D == 128) return pick_bits<128, 1, 1, FUSED>(bk, bv);
         return nullptr;
     }
-    if (D == 64) return NT == 1 ? pick_bits<64, 1, 0>(bk, bv) : pick_bits<64, 2, 0>(bk, bv);
-    if (D == 128) return NT == 1 ? pick_bits<128, 1, 0>(bk, bv) : pick_bits<128, 2, 0>(bk, bv);
+    if (D == 64) return NT == 1 ? pick_bits<64, 1, 0, FUSED>(bk, bv) : pick_bits<64, 2, 0, FUSED>(bk, bv);
+    if (D == 128) return NT == 1 ? pick_bits<128, 1, 0, FUSED>(bk, bv) : pick_bits<128, 2, 0, FUSED>(bk, bv);
     return nullptr;
+}
+
+KernelFn pick_kernel(int D, int bk, int bv, int kmode, int G, bool fused) {
+    return fused ? pick_kernel_t<true>(D, bk, bv, kmode, G) : pick_kernel_t<false>(D, bk, bv, kmode, G);
 }
 
 }  // namespace
@@ -1478,7 +1485,7 @@ struct KernelState {
     int occ[8] = {};
 };
 static std::mutex g_state_mu;
-static KernelState g_state[64];
+static KernelState g_state[160];   // every decode instance (2 x 54), the paged and merge kernels
 
 static cudaError_t prepare_kernel(const void *fn, size_t smem, int *occ_out) {
     std::lock_guard<std::mutex> lk(g_state_mu);
@@ -1516,7 +1523,7 @@ static cudaError_t prepare_kernel(const void *fn, size_t smem, int *occ_out) {
 
 cudaError_t decode_occupancy(int D, int bk, int bv, int kmode, int G, long long rec_bytes, int nstage,
                              int nextra, int *ctas_per_sm) {
-    KernelFn fn = pick_kernel(D, bk, bv, kmode, G);
+    KernelFn fn = pick_kernel(D, bk, bv, kmode, G, false);   // the fused instance has the same occupancy
     if (!fn) return cudaErrorInvalidValue;
     return prepare_kernel(reinterpret_cast<const void *>(fn), decode_smem_bytes(rec_bytes, nstage, nextra, D, G),
                           ctas_per_sm);
@@ -1524,7 +1531,7 @@ cudaError_t decode_occupancy(int D, int bk, int bv, int kmode, int G, long long 
 
 cudaError_t launch_decode(const DecodeParams &p, int D, int bk, int bv, int kmode, cudaStream_t st,
                           int *ctas_per_sm_out) {
-    KernelFn fn = pick_kernel(D, bk, bv, kmode, p.G);
+    KernelFn fn = pick_kernel(D, bk, bv, kmode, p.G, p.k_new != nullptr);
     if (!fn) return cudaErrorInvalidValue;
     const size_t smem = decode_smem_bytes(p.rec_bytes, p.nstage, p.nextra, D, p.G);
     cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(fn), smem, ctas_per_sm_out);
