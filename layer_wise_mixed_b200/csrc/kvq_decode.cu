@@ -922,13 +922,39 @@ template <int BITS>
 __device__ __forceinline__ void zero_half(uint32_t *area, int tid, int step, int D) {
     for (int widx = tid; widx < D * BITS / 2; widx += step) area[widx] = 0u;
 }
+// Insert token e's codes into a half's code words (one warp): the code fields of the
+// token that share a lane word are OR-ed in at once.  Values (role 1): the fields of
+// channels 16m + g and 16m + g + 8 are adjacent slots of lane 4g + t, one word (2 codes;
+// with 2-bit codes two such pairs share a word).  Keys (role 0): channels
+// 16k + 8r + 2t + hb of lane 4 gk + t fill slots 4k + 2i + r, one word (4 codes).
+// (e = 8 ch + 2t + hb for values, e = 8i + gk for keys; the positions are those of
+// quant::code_place, channel by channel.)
 template <int BITS>
-__device__ __forceinline__ void or_token(uint32_t *area, int role, int e, const uint8_t *code, int tid, int step,
-                                         int D) {
-    for (int d = tid; d < D; d += step) {
-        int w, bit;
-        quant::code_place(role, e, d, D, BITS, w, bit);
-        atomicOr(area + w, static_cast<uint32_t>(code[d]) << bit);
+__device__ __forceinline__ void or_token_words(uint32_t *area, int role, int e, const uint8_t *code, int lane,
+                                               int D) {
+    constexpr int P = 16 / BITS;
+    const int Wh = D * BITS / 64, c = Wh < 4 ? Wh : 4;
+    auto mem_word = [&](int lw, int w) { return ((w / c) * 32 + lw) * c + (w % c); };
+    if (role == 1) {
+        const int t = (e & 7) >> 1, ch = e >> 3, hb = e & 1;
+        for (int pi = lane; pi < D / 2; pi += 32) {
+            const int g = pi & 7, m = pi >> 3;
+            const int slot = 4 * m + 2 * ch, f = slot % P + hb * P, d = 16 * m + g;
+            const uint32_t v = (static_cast<uint32_t>(code[d]) << (f * BITS)) |
+                               (static_cast<uint32_t>(code[d + 8]) << ((f + 1) * BITS));
+            atomicOr(area + mem_word(4 * g + t, slot / P), v);
+        }
+    } else {
+        const int i = e >> 3, gk = e & 7;
+        for (int pi = lane; pi < D / 4; pi += 32) {
+            const int t = pi & 3, k = pi >> 2;
+            const int slot = 4 * k + 2 * i, f = slot % P, d = 16 * k + 2 * t;
+            const uint32_t v = (static_cast<uint32_t>(code[d]) << (f * BITS)) |
+                               (static_cast<uint32_t>(code[d + 1]) << ((f + P) * BITS)) |
+                               (static_cast<uint32_t>(code[d + 8]) << ((f + 1) * BITS)) |
+                               (static_cast<uint32_t>(code[d + 9]) << ((f + 1 + P) * BITS));
+            atomicOr(area + mem_word(4 * gk + t, slot / P), v);
+        }
     }
 }
 
@@ -1034,8 +1060,8 @@ __device__ __forceinline__ void append_token_store(const DecodeParams &p, long l
         if constexpr (KM == 1) zero_half<BK>(kwords, lane, 32, D);
         __syncwarp();
     }
-    or_token<BV>(vwords, 1, e, codes, lane, 32, D);
-    if constexpr (KM == 1) or_token<BK>(kwords, 0, e, codes + D, lane, 32, D);
+    or_token_words<BV>(vwords, 1, e, codes, lane, D);
+    if constexpr (KM == 1) or_token_words<BK>(kwords, 0, e, codes + D, lane, D);
     if (lane == 0) {
         if (smax_new[0]) atomicMax(p.smax_out, smax_new[0]);
         if (smax_new[1]) atomicMax(p.smax_out + 1, smax_new[1]);
@@ -1074,8 +1100,8 @@ __device__ __forceinline__ void patch_stage(uint8_t *stage, int u, const uint8_t
         if constexpr (KM == 1) zero_half<BK>(kwords, lane, 32, D);
         __syncwarp();
     }
-    or_token<BV>(vwords, 1, e, scratch, lane, 32, D);
-    if constexpr (KM == 1) or_token<BK>(kwords, 0, e, scratch + D, lane, 32, D);
+    or_token_words<BV>(vwords, 1, e, scratch, lane, D);
+    if constexpr (KM == 1) or_token_words<BK>(kwords, 0, e, scratch + D, lane, D);
     if (lane < NJ) {
         uint8_t *sz = stage + KC + KSZ + VC + quant::tok_sz_off(u, lane, NJ);
         *reinterpret_cast<uint16_t *>(sz) = szs[(NJ + lane) * 2];
