@@ -184,6 +184,25 @@ KVQ_API int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, 
 KVQ_API int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, const void *q,
                               void *out, int out_fp32, void *stream);
 
+/* Decode path of kvq_decode_attn on per-layer plans (default KVQ_DECODE_MMA_SYNC).
+ *
+ * KVQ_DECODE_MMA_SYNC: decode_split_kernel, mma.sync tensor-core tiles in registers; every
+ *   plan kvq_plan accepts.
+ * KVQ_DECODE_TCGEN05: the same attention (the pages' flash-decoding splits merged by
+ *   log-sum-exp, "TriAxialKV per-role mixed-precision KV quantization", Facts: decode
+ *   path) with both contractions on the 5th-generation tensor cores: tcgen05.mma with
+ *   operands staged in shared memory and accumulators in tensor memory.  Layers with
+ *   per-channel keys, head_dim 128 and at most 4 query heads per kv head; any other layer
+ *   fails with KVQ_EUNSUPPORTED (nothing is launched).  Results meet the same tolerances
+ *   as the default path, not bit for bit the same values.
+ *
+ * kvq_append_decode (the fused step) and paged plans always use their own kernels.
+ * Returns KVQ_EINVAL for an unknown path or a null handle; the setting applies to the
+ * handle's later kvq_decode_attn calls. */
+#define KVQ_DECODE_MMA_SYNC 0
+#define KVQ_DECODE_TCGEN05 1
+KVQ_API int kvq_set_decode_path(kvq_handle *h, int path);
+
 /* Force the number of sequence splits used by kvq_decode_attn (0 = automatic; the
  * value is capped by the number of 32-token blocks and the partial buffer size). */
 KVQ_API int kvq_set_num_splits(kvq_handle *h, int num_splits);

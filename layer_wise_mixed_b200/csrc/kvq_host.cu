@@ -40,6 +40,7 @@ struct kvq_handle {
     uint8_t *ws = nullptr;
     size_t ws_bytes = 0;
     int forced_splits = 0;
+    int decode_path = KVQ_DECODE_MMA_SYNC;   // kvq_set_decode_path
     int sm_count = 0;
     int device = -1;
     bool status_clear = false;   // status word zeroed on the device since the last bind
@@ -864,6 +865,94 @@ static int decode_paged(kvq_handle *h, int layer, const void *q, void *out, int 
     return ok();
 }
 
+// Split count of the tcgen05 decode: the one with the fewest CTA waves times chunks (4
+// blocks) per CTA, one chunk of set-up counted per CTA; a forced count is taken as given.
+static int umma_splits(kvq_handle *h, int layer, int *S_out) {
+    const LayerGeom &g = h->geom[layer];
+    const int nblk = (h->len[layer] + 31) / 32;
+    int rc = ensure_device_info(h);
+    if (rc) return rc;
+    int occ = 1;
+    cudaError_t e = kvq::decode_umma_occupancy(g.bk, g.bv, &occ);
+    if (e != cudaSuccess) return cuda_fail(e, "tcgen05 decode occupancy");
+    const long long units = static_cast<long long>(h->desc.batch) * h->desc.n_kv_heads;
+    const long long slots = static_cast<long long>(std::max(occ, 1)) * h->sm_count;
+    const int smax = std::min(kvq::kMaxSplits, nblk);
+    if (h->forced_splits > 0) {
+        *S_out = std::min(h->forced_splits, smax);
+        return KVQ_OK;
+    }
+    double best = 1e300;
+    *S_out = 1;
+    for (int S = 1; S <= smax; ++S) {
+        const int bps = (nblk + S - 1) / S;
+        if ((nblk + bps - 1) / bps != S) continue;
+        const double waves = static_cast<double>((units * S + slots - 1) / slots);
+        const double c = waves * ((bps + 3) / 4 + 1);
+        if (c < best - 1e-9) {
+            best = c;
+            *S_out = S;
+        }
+    }
+    return KVQ_OK;
+}
+
+// kvq_decode_attn on the tcgen05 kernel (per-channel keys, head_dim 128, G <= 4).
+static int decode_umma(kvq_handle *h, int layer, const void *q, void *out, int out_fp32, cudaStream_t st) {
+    const LayerGeom &g = h->geom[layer];
+    const int G = h->desc.n_q_heads / h->desc.n_kv_heads;
+    if (g.kmode != 0 || h->desc.head_dim != 128 || G > 4)
+        return fail(KVQ_EUNSUPPORTED,
+                    "the tcgen05 decode path takes per-channel keys, head_dim 128 and at most 4 query heads per "
+                    "kv head (layer %d: kmode %d, head_dim %d, %d heads per kv head)",
+                    layer, g.kmode, h->desc.head_dim, G);
+    const int L = h->len[layer];
+    const int nblk = (L + 31) / 32;
+    int S = 1, rc;
+    if ((rc = umma_splits(h, layer, &S))) return rc;
+    kvq::DecodeParams p{};
+    p.rec = h->ws + g.rec_off;
+    p.res = reinterpret_cast<const uint16_t *>(h->ws + g.res_off);
+    p.q = static_cast<const uint16_t *>(q);
+    p.smax = smax_slot(h, layer, static_cast<int>(h->ver[layer]));
+    if ((rc = fill_lengths(h, layer, p, 0, st))) return rc;
+    p.out = out;
+    p.part_acc = reinterpret_cast<float *>(h->ws + h->part_acc_off);
+    p.part_ml = reinterpret_cast<float *>(h->ws + h->part_ml_off);
+    p.sstride = kvq::kMaxSplits;
+    p.status = reinterpret_cast<unsigned *>(h->ws + h->status_off);
+    p.B = h->desc.batch;
+    p.Hkv = h->desc.n_kv_heads;
+    p.G = G;
+    p.L = L;
+    p.cap_blk = h->cap_blk;
+    p.bps = (nblk + S - 1) / S;
+    p.S = (nblk + p.bps - 1) / p.bps;
+    p.out_fp32 = out_fp32 ? 1 : 0;
+    p.rec_bytes = g.rec_bytes;
+    p.btab = block_table(h, layer);
+    if ((rc = prepare_status(h, st))) return rc;
+    cudaError_t e = kvq::launch_decode_umma(p, g.bk, g.bv, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tcgen05 decode launch");
+    note_write(h, st, -1);
+    if (p.S > 1) {
+        kvq::MergeParams m{};
+        m.part_acc = p.part_acc;
+        m.part_ml = p.part_ml;
+        m.out = out;
+        m.B = p.B;
+        m.Hq = h->desc.n_q_heads;
+        m.D = h->desc.head_dim;
+        m.S = p.S;
+        m.out_fp32 = p.out_fp32;
+        m.sstride = p.sstride;
+        e = kvq::launch_merge(m, st);
+        if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+        note_write(h, st, -1);
+    }
+    return ok();
+}
+
 int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_fp32, void *stream) {
     int rc = check_layer(h, layer);
     if (rc) return rc;
@@ -876,6 +965,8 @@ int kvq_decode_attn(kvq_handle *h, int layer, const void *q, void *out, int out_
         return decode_paged(h, layer, q, out, out_fp32, static_cast<cudaStream_t>(stream),
                             reinterpret_cast<float *>(h->ws + h->part_acc_off),
                             reinterpret_cast<float *>(h->ws + h->part_ml_off));
+    if (h->decode_path == KVQ_DECODE_TCGEN05)
+        return decode_umma(h, layer, q, out, out_fp32, static_cast<cudaStream_t>(stream));
     int S = 1, nstage = 2, nextra = 0;
     if ((rc = splits_for(h, layer, &S, &nstage, &nextra))) return rc;
     const LayerGeom &g = h->geom[layer];
@@ -1031,6 +1122,13 @@ int kvq_append_decode(kvq_handle *h, int layer, const void *K, const void *V, co
         if (e != cudaSuccess) return cuda_fail(e, "merge launch");
         note_write(h, st, -1);
     }
+    return ok();
+}
+
+int kvq_set_decode_path(kvq_handle *h, int path) {
+    if (!h) return fail(KVQ_EINVAL, "null handle");
+    if (path != KVQ_DECODE_MMA_SYNC && path != KVQ_DECODE_TCGEN05) return fail(KVQ_EINVAL, "unknown decode path %d", path);
+    h->decode_path = path;
     return ok();
 }
 

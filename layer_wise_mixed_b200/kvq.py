@@ -28,6 +28,8 @@ KVQ_ECUDA = -6
 KVQ_EDEVICE = -7
 KVQ_PER_CHANNEL = 0
 KVQ_PER_TOKEN = 1
+KVQ_DECODE_MMA_SYNC = 0
+KVQ_DECODE_TCGEN05 = 1
 
 _NAMES = {0: "KVQ_OK", -1: "KVQ_EINVAL", -2: "KVQ_EUNSUPPORTED", -3: "KVQ_ECAPACITY",
           -4: "KVQ_EUNBOUND", -5: "KVQ_EALIGN", -6: "KVQ_ECUDA", -7: "KVQ_EDEVICE"}
@@ -75,6 +77,7 @@ def load() -> ctypes.CDLL:
         "kvq_append_decode": (I, [P, I, P, P, P, P, I, P]),
         "kvq_decode_attn_noalloc": (I, [P, I, P, P, I, P]),
         "kvq_set_num_splits": (I, [P, I]),
+        "kvq_set_decode_path": (I, [P, I]),
         "kvq_get_num_splits": (I, [P, I, ctypes.POINTER(I)]),
         "kvq_export_layer": (I, [P, I, P, SZ, ctypes.POINTER(SZ)]),
         "kvq_seq_len": (I, [P, I, ctypes.POINTER(I)]),
@@ -177,6 +180,10 @@ def kvq_decode_attn_noalloc(h: int, layer: int, q, out, out_fp32: bool, stream=N
 
 def kvq_set_num_splits(h: int, n: int):
     _check(load().kvq_set_num_splits(h, n))
+
+
+def kvq_set_decode_path(h: int, path: int):
+    _check(load().kvq_set_decode_path(h, path))
 
 
 def kvq_get_num_splits(h: int, layer: int) -> int:

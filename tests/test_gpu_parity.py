@@ -61,9 +61,11 @@ def workload(B, Hkv, G, D, n_out=8, lo=10.0, hi=20.0, name="case"):
                             outlier_lo=lo, outlier_hi=hi)
 
 
-def run_case(B, Hkv, G, D, layer_bits, kmode, chunks, decode_at=None, splits=(0,), wl=None, tag="case"):
+def run_case(B, Hkv, G, D, layer_bits, kmode, chunks, decode_at=None, splits=(0,), wl=None, tag="case",
+             paths=(kvq.KVQ_DECODE_MMA_SYNC,)):
     """Append the token sequence in `chunks` (sizes), checking the image and decode output
-    against the oracle whenever the running length is in decode_at (default: the end)."""
+    against the oracle whenever the running length is in decode_at (default: the end),
+    on each decode path in `paths` and each split count in `splits`."""
     L_total = sum(chunks)
     wl = wl or workload(B, Hkv, G, D, name=tag)
     nl = len(layer_bits)
@@ -85,12 +87,15 @@ def run_case(B, Hkv, G, D, layer_bits, kmode, chunks, decode_at=None, splits=(0,
             if not np.array_equal(img, img_ref):
                 bad = np.flatnonzero(img != img_ref)
                 pytest.fail(f"{tag} layer {l} L={L}: image differs at {bad.size} bytes, first {bad[:8]}")
-            for S in splits:
-                kvq.kvq_set_num_splits(cache.h, S)
-                out32 = cache.decode_attn(l, q, out_fp32=True)
-                out16 = cache.decode_attn(l, q, out_fp32=False)
-                torch.cuda.synchronize()
-                check_outputs(out32, out16, out_ref, f"{tag} layer {l} L={L} splits={S}")
+            for path in paths:
+                kvq.kvq_set_decode_path(cache.h, path)
+                for S in splits:
+                    kvq.kvq_set_num_splits(cache.h, S)
+                    out32 = cache.decode_attn(l, q, out_fp32=True)
+                    out16 = cache.decode_attn(l, q, out_fp32=False)
+                    torch.cuda.synchronize()
+                    check_outputs(out32, out16, out_ref, f"{tag} layer {l} L={L} path={path} splits={S}")
+            kvq.kvq_set_decode_path(cache.h, kvq.KVQ_DECODE_MMA_SYNC)
             kvq.kvq_set_num_splits(cache.h, 0)
     assert kvq.kvq_device_status(cache.h) == 0
     return cache
