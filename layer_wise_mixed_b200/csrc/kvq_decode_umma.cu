@@ -112,6 +112,22 @@ __device__ __forceinline__ float block_max128(float v, float *red, int warp, int
     return fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
 }
 
+// CTA-wide maxima of four values per thread (one barrier pair); red holds [4 warps][4]
+__device__ __forceinline__ void block_max4(const float *v, float *out, float *red, int warp, int lane) {
+    float m[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        m[i] = v[i];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m[i] = fmaxf(m[i], __shfl_xor_sync(0xffffffffu, m[i], o));
+    }
+    __syncthreads();
+    if (lane == 0) *reinterpret_cast<float4 *>(red + 4 * warp) = make_float4(m[0], m[1], m[2], m[3]);
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) out[i] = fmaxf(fmaxf(red[i], red[4 + i]), fmaxf(red[8 + i], red[12 + i]));
+}
+
 __device__ __forceinline__ float block_sum128(float v, float *red, int warp, int lane) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -129,9 +145,13 @@ struct UmmaSmem {
     static constexpr int off_tile = 0;
     static constexpr int off_ak = off_tile + TILE;
     static constexpr int off_bv = off_ak + UCHUNK * AK;
-    static constexpr int off_qs = off_bv + BV;           // q~ [4][128] fp32
-    static constexpr int off_sc = off_qs + 4 * UD * 4;   // per warp: scores [8][32] fp32
-    static constexpr int off_zk = off_sc + UCHUNK * 8 * 32 * 4;   // per warp: key zero terms [4]
+    static constexpr int QS_ROW = UD + 4;                // q~ row stride (floats): heads on different banks
+    static constexpr int PB_ROW = 36;                    // p row stride (floats)
+    static constexpr int off_qs = off_bv + BV;           // q~ [4][QS_ROW] fp32
+    static constexpr int SC_ROW = 36;                    // score row stride (floats): conflict-free 16-byte stores
+    static constexpr int off_sc = off_qs + 4 * QS_ROW * 4;   // per warp: scores [8][SC_ROW] fp32
+    static constexpr int off_pb = off_sc + UCHUNK * 8 * SC_ROW * 4;   // per warp: p [4 heads][PB_ROW]
+    static constexpr int off_zk = off_pb + UCHUNK * 4 * PB_ROW * 4;   // per warp: key zero terms [4]
     static constexpr int off_zv = off_zk + UCHUNK * 4 * 4;        // per warp: value zero terms [4 j][4 h]
     static constexpr int off_red = off_zv + UCHUNK * 16 * 4;      // reductions [4 warps][4]
     static constexpr int off_bar = off_red + 16 * 4;              // copy, mma, q barriers + tmem slot
@@ -164,6 +184,7 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
     uint8_t *bv = smem + UmmaSmem::off_bv;
     float *qs = reinterpret_cast<float *>(smem + UmmaSmem::off_qs);
     float *sc = reinterpret_cast<float *>(smem + UmmaSmem::off_sc);
+    float *pb = reinterpret_cast<float *>(smem + UmmaSmem::off_pb);
     float *zk = reinterpret_cast<float *>(smem + UmmaSmem::off_zk);
     float *zv = reinterpret_cast<float *>(smem + UmmaSmem::off_zv);
     float *red = reinterpret_cast<float *>(smem + UmmaSmem::off_red);
@@ -221,7 +242,7 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
             if (smax_k > 0.f) kq = min(kq, 12 - floor_log2(amax) - floor_log2(smax_k));
             kq = max(-120, min(100, kq));
         }
-        qs[hh * D + tid] = qv * pow2f(kq);
+        qs[hh * UmmaSmem::QS_ROW + tid] = qv * pow2f(kq);
         unscale[hh] = pow2f(-kq);
     }
     const int kp = smax_v > 0.f ? max(-24, min(14, 13 - floor_log2(smax_v))) : 14;
@@ -251,50 +272,59 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
 
         // ---- (1) key tiles of this warp's block: B_K codes, A_K = q~ s hi/lo, zero term
         if (mine && !is_tail) {
+            uint32_t kw[2][WHK];   // this lane's code words of both halves
+            load_lane_words<WHK>(R, lane, kw[0]);
+            load_lane_words<WHK>(R + 2 * D * BK, lane, kw[1]);
 #pragma unroll
-            for (int k = 0; k < KS; ++k) {
-                constexpr int WPK = PK >= 4 ? 1 : 4 / PK;
-                constexpr int CH = WHK < 4 ? WHK : 4;
-                const int w0 = (4 * k) / PK;
+            for (int k = 0; k < KS; ++k)
 #pragma unroll
                 for (int n = 0; n < 4; ++n) {   // 8-token tiles: half n >> 1, rows 8 (n & 1) + g
                     const int s0 = (2 * k + (n & 1)) * 2;
-                    const int w = w0 + (s0 / PK - w0);
-                    const int off = (((w / CH) * 32 + lane) * CH + (w % CH)) * 4;
-                    const uint32_t word = *reinterpret_cast<const uint32_t *>(R + (n >> 1) * 2 * D * BK + off);
+                    const uint32_t word = kw[n >> 1][s0 / PK];
                     const int tok = 32 * warp + 8 * n + g;
                     *reinterpret_cast<uint32_t *>(tile + kmaj(tok, 16 * k + 2 * t, 128)) = unpack<BK>(word, s0 % PK);
                     *reinterpret_cast<uint32_t *>(tile + kmaj(tok, 16 * k + 8 + 2 * t, 128)) =
                         unpack<BK>(word, s0 % PK + 1);
                 }
-                (void)WPK;
-            }
-            // A_K rows: hi (0-3) and lo (4-7) of q~_c s_c, channels 4 lane .. 4 lane + 3
+            // A_K: lane = (row r = lane & 7, 8-channel chunks lane >> 3, + 4, + 8, + 12); row r:
+            // head r & 3, the hi (r < 4) or lo (r >= 4) part of q~_c s_c; one 16-byte store per
+            // chunk (8 lanes fill a 128-byte core matrix).  The hi-row lanes also sum q~_c z_c.
             uint8_t *a = ak + warp * UmmaSmem::AK;
-            float z4[4];
+            const int r = lane & 7, hh = r & 3;
+            const bool hi_row = r < 4, live = hh < G;
+            float zs = 0.f;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int c = 4 * lane + i;
-                const int so = quant::chan_sz_off(c);
-                const float s = __half2float(*reinterpret_cast<const __half *>(R + KC + so));
-                z4[i] = __half2float(*reinterpret_cast<const __half *>(R + KC + so + 4));
+            for (int it = 0; it < 4; ++it) {
+                const int c8 = (lane >> 3) + 4 * it, d0 = 8 * c8;
+                // scales/zeros of channels d0 .. d0 + 7: half2 pairs 16 bytes apart
+                const uint8_t *szp = R + KC + quant::chan_sz_off(d0);
+                float sv[8], zv8[8], qv[8];
 #pragma unroll
-                for (int hh = 0; hh < 4; ++hh) {
-                    const float v = hh < G ? qs[hh * D + c] * s : 0.f;
-                    const float hi = trunc11(v);
-                    *reinterpret_cast<__half *>(a + kmaj(hh, c, 8)) = __float2half_rn(hi);
-                    *reinterpret_cast<__half *>(a + kmaj(4 + hh, c, 8)) = __float2half_rn(v - hi);
+                for (int e = 0; e < 8; e += 2) {
+                    const __half2 s2 = *reinterpret_cast<const __half2 *>(szp + 8 * e);
+                    const __half2 z2 = *reinterpret_cast<const __half2 *>(szp + 8 * e + 4);
+                    sv[e] = __low2float(s2);
+                    sv[e + 1] = __high2float(s2);
+                    zv8[e] = __low2float(z2);
+                    zv8[e + 1] = __high2float(z2);
                 }
+                const float4 q0 = *reinterpret_cast<const float4 *>(qs + hh * UmmaSmem::QS_ROW + d0);
+                const float4 q1 = *reinterpret_cast<const float4 *>(qs + hh * UmmaSmem::QS_ROW + d0 + 4);
+                qv[0] = q0.x; qv[1] = q0.y; qv[2] = q0.z; qv[3] = q0.w;
+                qv[4] = q1.x; qv[5] = q1.y; qv[6] = q1.z; qv[7] = q1.w;
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    float v0 = live ? qv[e] * sv[e] : 0.f, v1 = live ? qv[e + 1] * sv[e + 1] : 0.f;
+                    const float h0 = trunc11(v0), h1 = trunc11(v1);
+                    w4[e >> 1] = hi_row ? pack_h2(h0, h1) : pack_h2(v0 - h0, v1 - h1);
+                    zs = fmaf(qv[e], zv8[e], fmaf(qv[e + 1], zv8[e + 1], zs));
+                }
+                *reinterpret_cast<uint4 *>(a + kmaj(r, d0, 8)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-#pragma unroll
-            for (int hh = 0; hh < 4; ++hh) {
-                float zs = 0.f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) zs = fmaf(hh < G ? qs[hh * D + 4 * lane + i] : 0.f, z4[i], zs);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
-                if (lane == 0) zk[warp * 4 + hh] = zs;
-            }
+            zs += __shfl_xor_sync(0xffffffffu, zs, 8);
+            zs += __shfl_xor_sync(0xffffffffu, zs, 16);
+            if (lane < 4) zk[warp * 4 + lane] = live ? zs : 0.f;
         }
         fence_proxy_async();
         tc_fence_before();
@@ -326,14 +356,15 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
             float v[32];
             tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32 * warp, v);
             if (lane < 8) {
+                float *row = sc + (warp * 8 + lane) * UmmaSmem::SC_ROW;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) sc[(warp * 8 + lane) * 32 + i] = v[i];
+                for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4 *>(row + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
             }
             __syncwarp();
 #pragma unroll
             for (int hh = 0; hh < 4; ++hh)
-                s4[hh] = (sc[(warp * 8 + hh) * 32 + lane] + sc[(warp * 8 + 4 + hh) * 32 + lane] + zk[warp * 4 + hh]) *
-                         unscale[hh];
+                s4[hh] = (sc[(warp * 8 + hh) * UmmaSmem::SC_ROW + lane] + sc[(warp * 8 + 4 + hh) * UmmaSmem::SC_ROW + lane] +
+                          zk[warp * 4 + hh]) * unscale[hh];
         } else if (is_tail) {
             // the open group's keys: bf16 residual rows, fp32 dot products
             float acc4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -343,7 +374,7 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
                     const uint32_t w2 = *reinterpret_cast<const uint32_t *>(row + c);
                     const float k0 = __uint_as_float(w2 << 16), k1 = __uint_as_float(w2 & 0xFFFF0000u);
 #pragma unroll
-                    for (int hh = 0; hh < 4; ++hh) acc4[hh] = fmaf(qs[hh * D + c], k0, fmaf(qs[hh * D + c + 1], k1, acc4[hh]));
+                    for (int hh = 0; hh < 4; ++hh) acc4[hh] = fmaf(qs[hh * UmmaSmem::QS_ROW + c], k0, fmaf(qs[hh * UmmaSmem::QS_ROW + c + 1], k1, acc4[hh]));
                 }
             }
 #pragma unroll
@@ -354,10 +385,11 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
         for (int hh = 0; hh < 4; ++hh)
             if (!tok_ok || hh >= G) s4[hh] = -INFINITY;
         // ---- (4) online softmax over the chunk (CTA-wide per head)
-        float alpha[4], m_new[4];
+        float alpha[4], m_new[4], cm4[4];
+        block_max4(s4, cm4, red, warp, lane);
 #pragma unroll
         for (int hh = 0; hh < 4; ++hh) {
-            const float cm = block_max128(s4[hh], red, warp, lane);
+            const float cm = cm4[hh];
             m_new[hh] = fmaxf(m_run[hh], cm);
             alpha[hh] = (m_new[hh] == -INFINITY) ? 1.f : fast_exp2(m_run[hh] - m_new[hh]);
             m_run[hh] = m_new[hh];
@@ -368,36 +400,39 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
             p4[hh] = tok_ok && hh < G ? fast_exp2(s4[hh] - m_new[hh] + pbias) : 0.f;
             l_acc[hh] = fmaf(l_acc[hh], alpha[hh], p4[hh]);
         }
-        // ---- (5) B_V = p s_V hi/lo per (group, head), value zero terms; lane = token
+        // ---- (5) B_V = p s_V hi/lo per (group, head): lane = column n = (group j, head, part),
+        // the warp's 4 token octets, one 16-byte store each (8 lanes fill a core matrix); the
+        // hi lanes also sum the value zero term p_t z_tj over the block's tokens
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh) pb[(warp * 4 + hh) * UmmaSmem::PB_ROW + lane] = p4[hh];
+        __syncwarp();
         {
-            const int tokc = 32 * warp + lane;
-            const int u = lane;
-            float zsum[16];
+            const int n = lane, j = n >> 3, hh = (n >> 1) & 3, part = n & 1;
+            float zsum = 0.f;
 #pragma unroll
-            for (int j = 0; j < NJ; ++j) {
-                float s = 0.f, z = 0.f;
-                if (tok_ok) {
-                    const uint8_t *szp = R + KC + KSZ + VC + quant::tok_sz_off(u, j, NJ);
-                    s = __half2float(*reinterpret_cast<const __half *>(szp));
-                    z = __half2float(*reinterpret_cast<const __half *>(szp + 4 * NJ));
+            for (int o = 0; o < 4; ++o) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const int u = 8 * o + e;   // token pair (u, u + 1) of the block
+                    float v0 = 0.f, v1 = 0.f;
+                    if (u < valid) {
+                        const uint8_t *szp = R + KC + KSZ + VC + quant::tok_sz_off(u, j, NJ);
+                        const __half2 s2 = *reinterpret_cast<const __half2 *>(szp);
+                        const __half2 z2 = *reinterpret_cast<const __half2 *>(szp + 4 * NJ);
+                        const float p0 = pb[(warp * 4 + hh) * UmmaSmem::PB_ROW + u];
+                        const float p1 = u + 1 < valid ? pb[(warp * 4 + hh) * UmmaSmem::PB_ROW + u + 1] : 0.f;
+                        v0 = p0 * __low2float(s2);
+                        v1 = u + 1 < valid ? p1 * __high2float(s2) : 0.f;
+                        zsum = fmaf(p0, __low2float(z2), zsum);
+                        if (u + 1 < valid) zsum = fmaf(p1, __high2float(z2), zsum);
+                    }
+                    const float h0 = trunc11(v0), h1 = trunc11(v1);
+                    w4[e >> 1] = part == 0 ? pack_h2(h0, h1) : pack_h2(v0 - h0, v1 - h1);
                 }
-#pragma unroll
-                for (int hh = 0; hh < 4; ++hh) {
-                    const float v = tok_ok ? p4[hh] * s : 0.f;
-                    const float hi = trunc11(v);
-                    const int n = j * 8 + hh * 2;
-                    *reinterpret_cast<__half *>(bv + kmaj(n, tokc, 32)) = __float2half_rn(hi);
-                    *reinterpret_cast<__half *>(bv + kmaj(n + 1, tokc, 32)) = __float2half_rn(v - hi);
-                    zsum[j * 4 + hh] = tok_ok ? p4[hh] * z : 0.f;
-                }
+                *reinterpret_cast<uint4 *>(bv + kmaj(n, 32 * warp + 8 * o, 32)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float v = zsum[i];
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (lane == 0) zv[warp * 16 + i] = v;
-            }
+            if (part == 0) zv[warp * 16 + j * 4 + hh] = zsum;
         }
         // ---- (6) A_V = value codes (channel x token) of this warp's block (zeros for none)
         if (mine) {
