@@ -46,7 +46,8 @@ def measured_hbm_peak():
 def kernel_source_sha256():
     import hashlib
     h = hashlib.sha256()
-    for f in ("layer_wise_mixed_b200/csrc/kvq_decode.cu", "layer_wise_mixed_b200/csrc/kvq_internal.h"):
+    for f in ("layer_wise_mixed_b200/csrc/kvq_decode.cu", "layer_wise_mixed_b200/csrc/kvq_device.cuh",
+              "layer_wise_mixed_b200/csrc/kvq_internal.h"):
         h.update(open(os.path.join(ROOT, f), "rb").read())
     return h.hexdigest()
 
@@ -132,6 +133,19 @@ def link_bound(h2d, d2h, stream, h2d_stream, d2h_stream, world, barrier, steps=1
     return {"ms_per_step": ms, "h2d_gbs": h2d / (ms / 1e3) / 1e9, "d2h_gbs": d2h / (ms / 1e3) / 1e9,
             "how": "pinned H2D of the step's input bytes and D2H of its output bytes on two copy streams at once, "
                    "nothing else running; tokens_s = batch per such step, frac = e2e / tokens_s"}
+
+
+def decode_paths_entry(bytes_launch, ms_default, ms_tcgen05, peak, kernel):
+    """Decode-only launch time and roofline fraction per decode path on the same schedule:
+    the default (mma.sync tiles; the paged kernel for paged plans) and, where the layer
+    qualifies, the tcgen05 path (kvq_set_decode_path)."""
+    def one(k, ms):
+        gbs = bytes_launch / (ms / 1e3) / 1e9
+        return {"kernel": k, "avg_launch_us": 1e3 * ms, "hbm_gbs": gbs, "frac": gbs / peak}
+    d = {"mma_sync": one(kernel, ms_default)}
+    if ms_tcgen05 is not None:
+        d["tcgen05"] = one("decode_umma_kernel", ms_tcgen05)
+    return d
 
 
 def max_over_ranks(value_ms, world):
@@ -297,9 +311,11 @@ class WorkloadRun:
     schedule's inputs resident in HBM, and per decode step two CUDA graphs (captured
     once, untimed): the full step over every layer (fused append + decode launch; a
     token that completes a per-channel key group: append, then decode; paged plans:
-    tagged append, then decode) and decode alone over every layer."""
+    tagged append, then decode) and decode alone over every layer; with tcgen05=True, for
+    layers the tcgen05 decode path takes (per-channel keys, head_dim 128, G <= 4), also
+    decode alone on that path."""
 
-    def __init__(self, wl, stream):
+    def __init__(self, wl, stream, tcgen05=False):
         import numpy as np
         import torch
 
@@ -350,7 +366,8 @@ class WorkloadRun:
             for l in range(NL):
                 cache.decode_attn(l, Qn[0, l], out[l], stream=stream)
         stream.synchronize()
-        self.graphs, self.dec_graphs, self.splits, self.Ls = [], [], [], []
+        self.graphs, self.dec_graphs, self.tc_graphs, self.splits, self.Ls = [], [], [], [], []
+        tc = tcgen05 and not paged and wl.kmode == 0 and D == 128 and wl.G <= 4
         for s in range(nsched):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
@@ -369,10 +386,18 @@ class WorkloadRun:
                 for l in range(NL):
                     kvq.kvq_decode_attn(cache.h, l, Qn[s, l], out[l], False, stream)
             self.dec_graphs.append(gd)
+            if tc:
+                kvq.kvq_set_decode_path(cache.h, kvq.KVQ_DECODE_TCGEN05)
+                gt = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gt, stream=stream):
+                    for l in range(NL):
+                        kvq.kvq_decode_attn(cache.h, l, Qn[s, l], out[l], False, stream)
+                kvq.kvq_set_decode_path(cache.h, kvq.KVQ_DECODE_MMA_SYNC)
+                self.tc_graphs.append(gt)
         torch.cuda.synchronize()
 
     def release(self):
-        self.graphs, self.dec_graphs = [], []
+        self.graphs, self.dec_graphs, self.tc_graphs = [], [], []
 
     def time_steps(self, order, warmup, barrier):
         """Device time (ms) of the full steps in `order`, after `warmup` untimed steps."""
@@ -391,19 +416,21 @@ class WorkloadRun:
         barrier()
         return e0.elapsed_time(e1)
 
-    def time_decode(self, order, min_ms=100.0, min_reps=3):
-        """Decode-only graphs over the steps in `order`, replayed as a whole until at least
-        min_ms of device time (and min_reps passes) are timed; returns (ms per launch,
-        passes, timed ms).  Live CUDA events on the launching stream."""
+    def time_decode(self, order, min_ms=100.0, min_reps=3, tcgen05=False):
+        """Decode-only graphs over the steps in `order` (the tcgen05 path's with
+        tcgen05=True), replayed as a whole until at least min_ms of device time (and
+        min_reps passes) are timed; returns (ms per decode launch, passes, timed ms).  Live
+        CUDA events on the launching stream."""
         import torch
         stream = self.stream
+        dec_graphs = self.tc_graphs if tcgen05 else self.dec_graphs
         with torch.cuda.stream(stream):
             for s in order[: min(len(order), 8)]:
-                self.dec_graphs[s].replay()
+                dec_graphs[s].replay()
             d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             d0.record(stream)
             for s in order:
-                self.dec_graphs[s].replay()
+                dec_graphs[s].replay()
             d1.record(stream)
         stream.synchronize()
         one = d0.elapsed_time(d1)
@@ -412,7 +439,7 @@ class WorkloadRun:
             d0.record(stream)
             for _ in range(reps):
                 for s in order:
-                    self.dec_graphs[s].replay()
+                    dec_graphs[s].replay()
             d1.record(stream)
         stream.synchronize()
         tot = d0.elapsed_time(d1)
@@ -492,6 +519,8 @@ def main():
                          "the same precision mix; 'none' to skip)")
     ap.add_argument("--decode-ms", type=float, default=100.0,
                     help="minimum device time of the decode-only replays behind the roofline figure")
+    ap.add_argument("--no-tcgen05", action="store_true",
+                    help="skip the decode-only replays on the tcgen05 path (decode_paths in the JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -529,7 +558,7 @@ def main():
     B, Hkv, Hq, D, G, NL = wl.batch, wl.n_kv_heads, wl.n_q_heads, wl.head_dim, wl.G, wl.num_layers
     paged = wl.paged
     stream = torch.cuda.Stream()
-    run = WorkloadRun(wl, stream)
+    run = WorkloadRun(wl, stream, tcgen05=not args.no_tcgen05)
     cache, Kn, Vn, Qn, out, nsched = run.cache, run.Kn, run.Vn, run.Qn, run.out, run.nsched
     order = [(args.warmup + i) % nsched for i in range(args.steps)]
     peak, peak_src = measured_hbm_peak()
@@ -540,12 +569,15 @@ def main():
     sampler.start()
     ms = max_over_ranks(run.time_steps(order, args.warmup, barrier), world)
     dec_launch_ms, dec_reps, dec_total_ms = run.time_decode(order, args.decode_ms)
+    tc_launch_ms = run.time_decode(order, args.decode_ms, tcgen05=True)[0] if run.tc_graphs else None
     clocks = sampler.stop()
     ms_per_step = ms / args.steps
     value = world * B * args.steps / (ms / 1e3)
     launches_dec = len(order) * NL
     bytes_launch = run.decode_bytes_per_launch(order)
     achieved = bytes_launch / (dec_launch_ms / 1e3) / 1e9
+    decode_paths = decode_paths_entry(bytes_launch, dec_launch_ms, tc_launch_ms, peak,
+                                      "decode_paged_kernel" if paged else "decode_split_kernel")
     gpu_launches = run.launches(order)
     e2e_note = (f"per step and group of {max(1, args.e2e_group)} layers: pinned H2D of the group's K/V/q (copy stream), "
                 "kvq_append_decode per layer (eager C-ABI calls, compute stream), D2H of the group's outputs "
@@ -706,12 +738,13 @@ def main():
         for name in wanted:
             full = configs.by_name(name)
             wc = reduced_workload(full, PER_CONFIG_LAYERS.get(name, 2))
-            r = WorkloadRun(wc, stream)
+            r = WorkloadRun(wc, stream, tcgen05=not args.no_tcgen05)
             ordc = list(range(r.nsched))
             smp = ClockSampler(local)
             smp.start()
             ms_c = r.time_steps(ordc, 3, barrier)
             dl_ms, dl_reps, _ = r.time_decode(ordc, args.decode_ms)
+            tl_ms = r.time_decode(ordc, args.decode_ms, tcgen05=True)[0] if r.tc_graphs else None
             clk = smp.stop()
             bl = r.decode_bytes_per_launch(ordc)
             ach = bl / (dl_ms / 1e3) / 1e9
@@ -727,6 +760,8 @@ def main():
                 "traffic": captured_traffic(full.name, bl),
                 "kernel": "decode_paged_kernel" if wc.paged else "decode_split_kernel",
                 "splits": sorted(set(x for s in ordc for x in r.splits[s])), "clocks": clk, "device_status": st,
+                "decode_paths": decode_paths_entry(bl, dl_ms, tl_ms, peak,
+                                                   "decode_paged_kernel" if wc.paged else "decode_split_kernel"),
                 "how": (f"{wc.num_layers} of {full.num_layers} layers with the full map's precision mix; tokens/s = "
                         "batch / (step time scaled to the full layer count); decode GB/s = algorithmic bytes / "
                         "CUDA-event time of decode-only graph replays")}
@@ -781,6 +816,7 @@ def main():
                         "link_bound": link},
                 "gpu_launches": gpu_launches, "clocks": clocks, "device_status": status,
                 "splits": head_splits,
+                "decode_paths": decode_paths,
                 "per_config": per_config}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -108,6 +108,12 @@ def test_argument_checks_before_any_launch(lib):
         assert L.kvq_truncate(h, 0, 1) == kvq.KVQ_EINVAL
         assert L.kvq_set_num_splits(h, -1) == kvq.KVQ_EINVAL
         assert L.kvq_set_num_splits(h, 3) == kvq.KVQ_OK
+        assert L.kvq_set_decode_path(None, kvq.KVQ_DECODE_TCGEN05) == kvq.KVQ_EINVAL
+        assert L.kvq_set_decode_path(h, 2) == kvq.KVQ_EINVAL
+        assert L.kvq_set_decode_path(h, kvq.KVQ_DECODE_TCGEN05) == kvq.KVQ_OK
+        # the tcgen05 path takes head_dim 128 only; this plan's is 64: refused on the host
+        assert L.kvq_decode_attn(h, 0, fake, fake, 0, None) == kvq.KVQ_EINVAL      # still: empty layer first
+        assert L.kvq_set_decode_path(h, kvq.KVQ_DECODE_MMA_SYNC) == kvq.KVQ_OK
     finally:
         kvq.kvq_destroy(h)
 
