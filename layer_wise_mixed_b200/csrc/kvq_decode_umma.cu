@@ -1,6 +1,6 @@
 // Split-KV decode attention over the packed per-layer cache on the 5th-generation tensor
 // cores (tcgen05.mma, accumulators in tensor memory): a variant of decode_split_kernel
-// for per-channel keys, head_dim 128 and up to 4 query heads per kv head.
+// for per-channel keys, head_dim 128 and up to 8 query heads per kv head.
 //
 // The same attention as the mma.sync kernel (flash-decoding splits merged by log-sum-exp:
 // "TriAxialKV per-role mixed-precision KV quantization", Facts: decode path; one static
@@ -9,9 +9,11 @@
 // in the no-swizzle K-major layout (8-row x 16-byte core matrices):
 //
 //   scores, per 32-token block:  D_K [row][token] = sum_c A_K [row][c] B_K [token][c]
-//     A_K rows = (part, head): q~_c s_c as an exact fp16 hi (rows 0-3) + lo (rows 4-7) pair,
-//       8 rows read with stride-byte-offset 0, so all 128 accumulator lanes hold copies of
-//       the 8 rows and each warp reads its own block's scores from its lane quarter;
+//     A_K rows = (part, head): q~_c s_c as an exact fp16 hi + lo pair.  Up to 4 heads: 8
+//       rows read with stride-byte-offset 0, so all 128 accumulator lanes hold copies of
+//       the 8 rows and each warp reads its own block's scores from its lane quarter; 5 to 8
+//       heads: 16 rows (the tile's other rows read past them and are not used), whose
+//       scores warp 0 reads and passes on through shared memory;
 //     B_K = the block's key codes as exact fp16 integers; the zero term sum_c q~_c z_c is
 //       added on the CUDA cores.
 //   values, per 4-block chunk:  D_V [c][n] = sum_t A_V [c][t] B_V [n][t]
@@ -103,29 +105,24 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *v) {
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ float block_max128(float v, float *red, int warp, int lane) {
+// CTA-wide maxima of N values per thread (one barrier pair); red holds [4 warps][N]
+template <int N>
+__device__ __forceinline__ void block_maxn(const float *v, float *out, float *red, int warp, int lane) {
+    float m[N];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    __syncthreads();
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    return fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-}
-
-// CTA-wide maxima of four values per thread (one barrier pair); red holds [4 warps][4]
-__device__ __forceinline__ void block_max4(const float *v, float *out, float *red, int warp, int lane) {
-    float m[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < N; ++i) {
         m[i] = v[i];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m[i] = fmaxf(m[i], __shfl_xor_sync(0xffffffffu, m[i], o));
     }
     __syncthreads();
-    if (lane == 0) *reinterpret_cast<float4 *>(red + 4 * warp) = make_float4(m[0], m[1], m[2], m[3]);
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < N; i += 4) *reinterpret_cast<float4 *>(red + N * warp + i) = make_float4(m[i], m[i + 1], m[i + 2], m[i + 3]);
+    }
     __syncthreads();
 #pragma unroll
-    for (int i = 0; i < 4; ++i) out[i] = fmaxf(fmaxf(red[i], red[4 + i]), fmaxf(red[8 + i], red[12 + i]));
+    for (int i = 0; i < N; ++i) out[i] = fmaxf(fmaxf(red[i], red[N + i]), fmaxf(red[2 * N + i], red[3 * N + i]));
 }
 
 __device__ __forceinline__ float block_sum128(float v, float *red, int warp, int lane) {
@@ -137,37 +134,60 @@ __device__ __forceinline__ float block_sum128(float v, float *red, int warp, int
     return (red[0] + red[1]) + (red[2] + red[3]);
 }
 
-// Shared memory of one CTA (dynamic, 1024-byte aligned base).
+// 32 lanes x 16 columns
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared memory of one CTA (dynamic, 1024-byte aligned base) for up to GM query heads per
+// kv head (GM = 4 or 8).
+template <int GM>
 struct UmmaSmem {
-    static constexpr int TILE = UD * 128 * 2;           // B_K (128 tokens x 128 channels) / A_V (128 x 128)
-    static constexpr int AK = 8 * UD * 2;               // one block's A_K: 8 rows x 128 channels
-    static constexpr int BV = 32 * 128 * 2;             // B_V: 32 columns x 128 tokens
+    static constexpr int RK = 2 * GM;                    // A_K rows: hi and lo per head
+    static constexpr int NV = 8 * GM;                    // B_V columns: (group, head, part)
+    static constexpr int TILE = UD * 128 * 2;            // B_K (128 tokens x 128 channels) / A_V (128 x 128)
+    static constexpr int AK = RK * UD * 2;               // one block's A_K
+    static constexpr int BV = NV * 128 * 2;              // B_V: NV columns x 128 tokens
+    static constexpr int QS_ROW = UD + 4;                // q~ row stride (floats): heads on different banks
+    static constexpr int PB_ROW = 36;                    // p row stride (floats)
+    static constexpr int SC_ROW = 36;                    // score row stride (floats): conflict-free 16-byte stores
     static constexpr int off_tile = 0;
     static constexpr int off_ak = off_tile + TILE;
     static constexpr int off_bv = off_ak + UCHUNK * AK;
-    static constexpr int QS_ROW = UD + 4;                // q~ row stride (floats): heads on different banks
-    static constexpr int PB_ROW = 36;                    // p row stride (floats)
-    static constexpr int off_qs = off_bv + BV;           // q~ [4][QS_ROW] fp32
-    static constexpr int SC_ROW = 36;                    // score row stride (floats): conflict-free 16-byte stores
-    static constexpr int off_sc = off_qs + 4 * QS_ROW * 4;   // per warp: scores [8][SC_ROW] fp32
-    static constexpr int off_pb = off_sc + UCHUNK * 8 * SC_ROW * 4;   // per warp: p [4 heads][PB_ROW]
-    static constexpr int off_zk = off_pb + UCHUNK * 4 * PB_ROW * 4;   // per warp: key zero terms [4]
-    static constexpr int off_zv = off_zk + UCHUNK * 4 * 4;        // per warp: value zero terms [4 j][4 h]
-    static constexpr int off_red = off_zv + UCHUNK * 16 * 4;      // reductions [4 warps][4]
-    static constexpr int off_bar = off_red + 16 * 4;              // copy, mma, q barriers + tmem slot
-    static constexpr int off_q = off_bar + 64;                    // bf16 q rows [G][128]
-    static constexpr int off_stage = ((off_q + 4 * UD * 2 + 127) / 128) * 128;
+    static constexpr int off_qs = off_bv + BV;                        // q~ [GM][QS_ROW] fp32
+    static constexpr int off_sc = off_qs + GM * QS_ROW * 4;           // per block: scores [RK][SC_ROW] fp32
+    static constexpr int off_pb = off_sc + UCHUNK * RK * SC_ROW * 4;  // per warp: p [GM][PB_ROW]
+    static constexpr int off_zk = off_pb + UCHUNK * GM * PB_ROW * 4;  // per warp: key zero terms [GM]
+    static constexpr int off_zv = off_zk + UCHUNK * GM * 4;           // per warp: value zero terms [4 j][GM]
+    static constexpr int off_red = off_zv + UCHUNK * 4 * GM * 4;      // reductions [4 warps][GM]
+    static constexpr int off_bar = off_red + 4 * GM * 4;              // copy, mma, q barriers + tmem slot
+    static constexpr int off_q = off_bar + 64;                        // bf16 q rows [G][128]
+    static constexpr int off_stage = ((off_q + GM * UD * 2 + 127) / 128) * 128;
     static constexpr int bytes(int rec) { return off_stage + UCHUNK * rec; }
 };
 
-template <int BK, int BV>
+template <int BK, int BV, int GM>
 __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams p) {
     pdl_enter();
+    using SM = UmmaSmem<GM>;
     constexpr int D = UD, NJ = D / 32, KS = D / 16;
+    constexpr int RK = SM::RK, NV = SM::NV;
     constexpr int REC = unit_bytes(D, BK, BV, 0, 2);
     constexpr int KC = 4 * D * BK, KSZ = 4 * D, VC = 4 * D * BV;
     constexpr int PK = 16 / BK, PV = 16 / BV;
     constexpr int WHK = D * BK / 64, WHV = D * BV / 64;
+    // GM = 4: the 8 A_K rows are read with stride-byte-offset 0, so every lane quarter
+    // holds them and each warp reads its own block's scores; GM = 8: 16 rows, lanes 0-15
+    // (warp 0's quarter) hold them and warp 0 passes every block's scores on
+    constexpr bool ALIAS = GM == 4;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -179,21 +199,21 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
     const int blk0 = sp * p.bps, blk1 = min(nblk, blk0 + p.bps);
     const long long unit = static_cast<long long>(b) * p.Hkv + h;
 
-    uint8_t *tile = smem + UmmaSmem::off_tile;
-    uint8_t *ak = smem + UmmaSmem::off_ak;
-    uint8_t *bv = smem + UmmaSmem::off_bv;
-    float *qs = reinterpret_cast<float *>(smem + UmmaSmem::off_qs);
-    float *sc = reinterpret_cast<float *>(smem + UmmaSmem::off_sc);
-    float *pb = reinterpret_cast<float *>(smem + UmmaSmem::off_pb);
-    float *zk = reinterpret_cast<float *>(smem + UmmaSmem::off_zk);
-    float *zv = reinterpret_cast<float *>(smem + UmmaSmem::off_zv);
-    float *red = reinterpret_cast<float *>(smem + UmmaSmem::off_red);
-    uint64_t *copy_bar = reinterpret_cast<uint64_t *>(smem + UmmaSmem::off_bar);
+    uint8_t *tile = smem + SM::off_tile;
+    uint8_t *ak = smem + SM::off_ak;
+    uint8_t *bv = smem + SM::off_bv;
+    float *qs = reinterpret_cast<float *>(smem + SM::off_qs);
+    float *sc = reinterpret_cast<float *>(smem + SM::off_sc);
+    float *pb = reinterpret_cast<float *>(smem + SM::off_pb);
+    float *zk = reinterpret_cast<float *>(smem + SM::off_zk);
+    float *zv = reinterpret_cast<float *>(smem + SM::off_zv);
+    float *red = reinterpret_cast<float *>(smem + SM::off_red);
+    uint64_t *copy_bar = reinterpret_cast<uint64_t *>(smem + SM::off_bar);
     uint64_t *mma_bar = copy_bar + 1;
     uint64_t *q_bar = copy_bar + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(copy_bar + 3);
-    uint16_t *q_s = reinterpret_cast<uint16_t *>(smem + UmmaSmem::off_q);
-    uint8_t *stage = smem + UmmaSmem::off_stage;
+    uint16_t *q_s = reinterpret_cast<uint16_t *>(smem + SM::off_q);
+    uint8_t *stage = smem + SM::off_stage;
 
     auto rec_src = [&](int blk) {
         return p.rec + rec_index(p.btab, b, p.Hkv, h, p.cap_blk, blk) * static_cast<long long>(REC);
@@ -231,33 +251,40 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
     const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
     const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
     const float qscale = kLog2eU * rsqrtf(static_cast<float>(D));
-    float unscale[4];
+    float unscale[GM];
+    {
+        float qv[GM], aq[GM], amax[GM];
 #pragma unroll
-    for (int hh = 0; hh < 4; ++hh) {
-        const float qv = hh < G ? quant::bf16_to_f32(q_s[hh * D + tid]) * qscale : 0.f;
-        const float amax = block_max128(fabsf(qv), red, warp, lane);
-        int kq = 0;
-        if (amax > 0.f) {
-            kq = 14 - floor_log2(amax);
-            if (smax_k > 0.f) kq = min(kq, 12 - floor_log2(amax) - floor_log2(smax_k));
-            kq = max(-120, min(100, kq));
+        for (int hh = 0; hh < GM; ++hh) {
+            qv[hh] = hh < G ? quant::bf16_to_f32(q_s[hh * D + tid]) * qscale : 0.f;
+            aq[hh] = fabsf(qv[hh]);
         }
-        qs[hh * UmmaSmem::QS_ROW + tid] = qv * pow2f(kq);
-        unscale[hh] = pow2f(-kq);
+        block_maxn<GM>(aq, amax, red, warp, lane);
+#pragma unroll
+        for (int hh = 0; hh < GM; ++hh) {
+            int kq = 0;
+            if (amax[hh] > 0.f) {
+                kq = 14 - floor_log2(amax[hh]);
+                if (smax_k > 0.f) kq = min(kq, 12 - floor_log2(amax[hh]) - floor_log2(smax_k));
+                kq = max(-120, min(100, kq));
+            }
+            qs[hh * SM::QS_ROW + tid] = qv[hh] * pow2f(kq);
+            unscale[hh] = pow2f(-kq);
+        }
     }
     const int kp = smax_v > 0.f ? max(-24, min(14, 13 - floor_log2(smax_v))) : 14;
     const float pbias = static_cast<float>(kp);
     __syncthreads();
 
-    float m_run[4], l_acc[4], o_acc[4];
+    float m_run[GM], l_acc[GM], o_acc[GM];
 #pragma unroll
-    for (int hh = 0; hh < 4; ++hh) {
+    for (int hh = 0; hh < GM; ++hh) {
         m_run[hh] = -INFINITY;
         l_acc[hh] = 0.f;
         o_acc[hh] = 0.f;
     }
     constexpr uint32_t IDESC_K = umma_idesc(128, 32);
-    constexpr uint32_t IDESC_V = umma_idesc(128, 32);
+    constexpr uint32_t IDESC_V = umma_idesc(128, NV);
     unsigned copy_phase = 0, mma_phase = 0;
 
     for (int c0 = blk0; c0 < blk1; c0 += UCHUNK) {
@@ -286,16 +313,16 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
                     *reinterpret_cast<uint32_t *>(tile + kmaj(tok, 16 * k + 8 + 2 * t, 128)) =
                         unpack<BK>(word, s0 % PK + 1);
                 }
-            // A_K: lane = (row r = lane & 7, 8-channel chunks lane >> 3, + 4, + 8, + 12); row r:
-            // head r & 3, the hi (r < 4) or lo (r >= 4) part of q~_c s_c; one 16-byte store per
-            // chunk (8 lanes fill a 128-byte core matrix).  The hi-row lanes also sum q~_c z_c.
-            uint8_t *a = ak + warp * UmmaSmem::AK;
-            const int r = lane & 7, hh = r & 3;
-            const bool hi_row = r < 4, live = hh < G;
+            // A_K: lane = (row r = lane % RK, 8-channel chunks lane / RK + (32 / RK) i); row r:
+            // head r % GM, the hi (r < GM) or lo part of q~_c s_c; one 16-byte store per chunk
+            // (8 lanes fill a 128-byte core matrix).  The hi-row lanes also sum q~_c z_c.
+            uint8_t *a = ak + warp * SM::AK;
+            const int r = lane % RK, hh = r % GM;
+            const bool hi_row = r < GM, live = hh < G;
             float zs = 0.f;
 #pragma unroll
-            for (int it = 0; it < 4; ++it) {
-                const int c8 = (lane >> 3) + 4 * it, d0 = 8 * c8;
+            for (int it = 0; it < 16 * RK / 32; ++it) {
+                const int c8 = lane / RK + (32 / RK) * it, d0 = 8 * c8;
                 // scales/zeros of channels d0 .. d0 + 7: half2 pairs 16 bytes apart
                 const uint8_t *szp = R + KC + quant::chan_sz_off(d0);
                 float sv[8], zv8[8], qv[8];
@@ -308,8 +335,8 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
                     zv8[e] = __low2float(z2);
                     zv8[e + 1] = __high2float(z2);
                 }
-                const float4 q0 = *reinterpret_cast<const float4 *>(qs + hh * UmmaSmem::QS_ROW + d0);
-                const float4 q1 = *reinterpret_cast<const float4 *>(qs + hh * UmmaSmem::QS_ROW + d0 + 4);
+                const float4 q0 = *reinterpret_cast<const float4 *>(qs + hh * SM::QS_ROW + d0);
+                const float4 q1 = *reinterpret_cast<const float4 *>(qs + hh * SM::QS_ROW + d0 + 4);
                 qv[0] = q0.x; qv[1] = q0.y; qv[2] = q0.z; qv[3] = q0.w;
                 qv[4] = q1.x; qv[5] = q1.y; qv[6] = q1.z; qv[7] = q1.w;
                 uint32_t w4[4];
@@ -320,11 +347,11 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
                     w4[e >> 1] = hi_row ? pack_h2(h0, h1) : pack_h2(v0 - h0, v1 - h1);
                     zs = fmaf(qv[e], zv8[e], fmaf(qv[e + 1], zv8[e + 1], zs));
                 }
-                *reinterpret_cast<uint4 *>(a + kmaj(r, d0, 8)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                *reinterpret_cast<uint4 *>(a + kmaj(r, d0, RK)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-            zs += __shfl_xor_sync(0xffffffffu, zs, 8);
-            zs += __shfl_xor_sync(0xffffffffu, zs, 16);
-            if (lane < 4) zk[warp * 4 + lane] = live ? zs : 0.f;
+#pragma unroll
+            for (int o = RK; o < 32; o <<= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
+            if (lane < GM) zk[warp * GM + lane] = live ? zs : 0.f;
         }
         fence_proxy_async();
         tc_fence_before();
@@ -338,7 +365,7 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
                 if (c0 + i == tail_blk) continue;
 #pragma unroll
                 for (int s = 0; s < KS; ++s) {
-                    const uint64_t ad = umma_desc(smem_u32(ak + i * UmmaSmem::AK) + s * 256, 128, 0);
+                    const uint64_t ad = umma_desc(smem_u32(ak + i * SM::AK) + s * 2 * RK * 16, RK * 16, ALIAS ? 0 : 128);
                     const uint64_t bd = umma_desc(smem_u32(tile) + 512 * i + s * 4096, 2048, 128);
                     umma_f16(tmem + 32 * i, ad, bd, IDESC_K, s > 0 ? 1u : 0u);
                 }
@@ -350,64 +377,86 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
             mma_phase ^= 1u;
         }
         tc_fence_after();
-        // ---- (3) this warp's block scores: lane = token, 4 heads (log2 units)
-        float s4[4];
-        if (mine && !is_tail) {
-            float v[32];
-            tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32 * warp, v);
-            if (lane < 8) {
-                float *row = sc + (warp * 8 + lane) * UmmaSmem::SC_ROW;
+        // ---- (3) scores: lane = token of this warp's block, GM heads (log2 units)
+        float s4[GM];
+        if constexpr (ALIAS) {
+            if (mine && !is_tail) {
+                float v[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32 * warp, v);
+                if (lane < RK) {
+                    float *row = sc + (warp * RK + lane) * SM::SC_ROW;
 #pragma unroll
-                for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4 *>(row + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                    for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4 *>(row + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+                }
+                __syncwarp();
             }
-            __syncwarp();
+        } else {
+            // rows 0 .. RK - 1 sit in lanes 0 .. RK - 1: warp 0 reads every block's columns
+            if (warp == 0) {
+                for (int i = 0; i < nb; ++i) {
+                    if (c0 + i == tail_blk) continue;
+                    float v[32];
+                    tmem_ld32(tmem + 32 * i, v);
+                    if (lane < RK) {
+                        float *row = sc + (i * RK + lane) * SM::SC_ROW;
 #pragma unroll
-            for (int hh = 0; hh < 4; ++hh)
-                s4[hh] = (sc[(warp * 8 + hh) * UmmaSmem::SC_ROW + lane] + sc[(warp * 8 + 4 + hh) * UmmaSmem::SC_ROW + lane] +
-                          zk[warp * 4 + hh]) * unscale[hh];
+                        for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4 *>(row + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                    }
+                }
+            }
+            __syncthreads();
+        }
+        if (mine && !is_tail) {
+#pragma unroll
+            for (int hh = 0; hh < GM; ++hh)
+                s4[hh] = (sc[(warp * RK + hh) * SM::SC_ROW + lane] + sc[(warp * RK + GM + hh) * SM::SC_ROW + lane] +
+                          zk[warp * GM + hh]) * unscale[hh];
         } else if (is_tail) {
             // the open group's keys: bf16 residual rows, fp32 dot products
-            float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+            float acc[GM];
+#pragma unroll
+            for (int hh = 0; hh < GM; ++hh) acc[hh] = 0.f;
             if (lane < rem) {
                 const uint16_t *row = p.res + (unit * 32 + lane) * D;
                 for (int c = 0; c < D; c += 2) {
                     const uint32_t w2 = *reinterpret_cast<const uint32_t *>(row + c);
                     const float k0 = __uint_as_float(w2 << 16), k1 = __uint_as_float(w2 & 0xFFFF0000u);
 #pragma unroll
-                    for (int hh = 0; hh < 4; ++hh) acc4[hh] = fmaf(qs[hh * UmmaSmem::QS_ROW + c], k0, fmaf(qs[hh * UmmaSmem::QS_ROW + c + 1], k1, acc4[hh]));
+                    for (int hh = 0; hh < GM; ++hh)
+                        acc[hh] = fmaf(qs[hh * SM::QS_ROW + c], k0, fmaf(qs[hh * SM::QS_ROW + c + 1], k1, acc[hh]));
                 }
             }
 #pragma unroll
-            for (int hh = 0; hh < 4; ++hh) s4[hh] = acc4[hh] * unscale[hh];
+            for (int hh = 0; hh < GM; ++hh) s4[hh] = acc[hh] * unscale[hh];
         }
         const bool tok_ok = lane < valid;
 #pragma unroll
-        for (int hh = 0; hh < 4; ++hh)
+        for (int hh = 0; hh < GM; ++hh)
             if (!tok_ok || hh >= G) s4[hh] = -INFINITY;
         // ---- (4) online softmax over the chunk (CTA-wide per head)
-        float alpha[4], m_new[4], cm4[4];
-        block_max4(s4, cm4, red, warp, lane);
+        float alpha[GM], m_new[GM], cm[GM];
+        block_maxn<GM>(s4, cm, red, warp, lane);
 #pragma unroll
-        for (int hh = 0; hh < 4; ++hh) {
-            const float cm = cm4[hh];
-            m_new[hh] = fmaxf(m_run[hh], cm);
+        for (int hh = 0; hh < GM; ++hh) {
+            m_new[hh] = fmaxf(m_run[hh], cm[hh]);
             alpha[hh] = (m_new[hh] == -INFINITY) ? 1.f : fast_exp2(m_run[hh] - m_new[hh]);
             m_run[hh] = m_new[hh];
         }
-        float p4[4];
+        float p4[GM];
 #pragma unroll
-        for (int hh = 0; hh < 4; ++hh) {
+        for (int hh = 0; hh < GM; ++hh) {
             p4[hh] = tok_ok && hh < G ? fast_exp2(s4[hh] - m_new[hh] + pbias) : 0.f;
             l_acc[hh] = fmaf(l_acc[hh], alpha[hh], p4[hh]);
         }
-        // ---- (5) B_V = p s_V hi/lo per (group, head): lane = column n = (group j, head, part),
-        // the warp's 4 token octets, one 16-byte store each (8 lanes fill a core matrix); the
-        // hi lanes also sum the value zero term p_t z_tj over the block's tokens
+        // ---- (5) B_V = p s_V hi/lo per (group, head): lane = column n = (group j, head, part)
+        // (GM = 8: two columns per lane), the warp's 4 token octets, one 16-byte store each
+        // (8 lanes fill a core matrix); the hi lanes also sum the value zero term p_t z_tj
 #pragma unroll
-        for (int hh = 0; hh < 4; ++hh) pb[(warp * 4 + hh) * UmmaSmem::PB_ROW + lane] = p4[hh];
+        for (int hh = 0; hh < GM; ++hh) pb[(warp * GM + hh) * SM::PB_ROW + lane] = p4[hh];
         __syncwarp();
-        {
-            const int n = lane, j = n >> 3, hh = (n >> 1) & 3, part = n & 1;
+#pragma unroll
+        for (int nn = 0; nn < NV / 32; ++nn) {
+            const int n = lane + 32 * nn, j = n / (2 * GM), hh = (n >> 1) % GM, part = n & 1;
             float zsum = 0.f;
 #pragma unroll
             for (int o = 0; o < 4; ++o) {
@@ -420,8 +469,8 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
                         const uint8_t *szp = R + KC + KSZ + VC + quant::tok_sz_off(u, j, NJ);
                         const __half2 s2 = *reinterpret_cast<const __half2 *>(szp);
                         const __half2 z2 = *reinterpret_cast<const __half2 *>(szp + 4 * NJ);
-                        const float p0 = pb[(warp * 4 + hh) * UmmaSmem::PB_ROW + u];
-                        const float p1 = u + 1 < valid ? pb[(warp * 4 + hh) * UmmaSmem::PB_ROW + u + 1] : 0.f;
+                        const float p0 = pb[(warp * GM + hh) * SM::PB_ROW + u];
+                        const float p1 = u + 1 < valid ? pb[(warp * GM + hh) * SM::PB_ROW + u + 1] : 0.f;
                         v0 = p0 * __low2float(s2);
                         v1 = u + 1 < valid ? p1 * __high2float(s2) : 0.f;
                         zsum = fmaf(p0, __low2float(z2), zsum);
@@ -430,9 +479,9 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
                     const float h0 = trunc11(v0), h1 = trunc11(v1);
                     w4[e >> 1] = part == 0 ? pack_h2(h0, h1) : pack_h2(v0 - h0, v1 - h1);
                 }
-                *reinterpret_cast<uint4 *>(bv + kmaj(n, 32 * warp + 8 * o, 32)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                *reinterpret_cast<uint4 *>(bv + kmaj(n, 32 * warp + 8 * o, NV)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-            if (part == 0) zv[warp * 16 + j * 4 + hh] = zsum;
+            if (part == 0) zv[warp * 4 * GM + j * GM + hh] = zsum;
         }
         // ---- (6) A_V = value codes (channel x token) of this warp's block (zeros for none)
         if (mine) {
@@ -465,7 +514,7 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
 #pragma unroll
             for (int s = 0; s < 8; ++s) {   // K = 128 tokens
                 const uint64_t ad = umma_desc(smem_u32(tile) + s * 4096, 2048, 128);
-                const uint64_t bd = umma_desc(smem_u32(bv) + s * 1024, 512, 128);
+                const uint64_t bd = umma_desc(smem_u32(bv) + s * 2 * NV * 16, NV * 16, 128);
                 umma_f16(tmem, ad, bd, IDESC_V, s > 0 ? 1u : 0u);
             }
             umma_commit(mma_bar);
@@ -473,14 +522,15 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
         if (!mbar_wait(mma_bar, mma_phase)) failed = true;
         mma_phase ^= 1u;
         tc_fence_after();
-        // ---- (7) channel tid = 32 warp + lane of group j = warp: its 8 columns
+        // ---- (7) channel tid = 32 warp + lane of group j = warp: its 2 GM columns
         {
-            float v[8];
-            tmem_ld8(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 8 * warp, v);
+            float v[2 * GM];
+            if constexpr (GM == 4) tmem_ld8(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 2 * GM * warp, v);
+            else tmem_ld16(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 2 * GM * warp, v);
 #pragma unroll
-            for (int hh = 0; hh < 4; ++hh) {
-                const float z = (zv[0 * 16 + warp * 4 + hh] + zv[1 * 16 + warp * 4 + hh]) +
-                                (zv[2 * 16 + warp * 4 + hh] + zv[3 * 16 + warp * 4 + hh]);
+            for (int hh = 0; hh < GM; ++hh) {
+                const float z = (zv[0 * 4 * GM + warp * GM + hh] + zv[1 * 4 * GM + warp * GM + hh]) +
+                                (zv[2 * 4 * GM + warp * GM + hh] + zv[3 * 4 * GM + warp * GM + hh]);
                 o_acc[hh] = fmaf(o_acc[hh], alpha[hh], v[2 * hh] + v[2 * hh + 1] + z);
             }
         }
@@ -490,11 +540,11 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
     }
 
     // ---- epilogue: l over the CTA, output or split partials (thread = channel)
-    float l_tot[4];
+    float l_tot[GM];
 #pragma unroll
-    for (int hh = 0; hh < 4; ++hh) l_tot[hh] = block_sum128(l_acc[hh], red, warp, lane);
+    for (int hh = 0; hh < GM; ++hh) l_tot[hh] = block_sum128(l_acc[hh], red, warp, lane);
 #pragma unroll
-    for (int hh = 0; hh < 4; ++hh) {
+    for (int hh = 0; hh < GM; ++hh) {
         if (hh >= G) continue;
         const long long row = unit * G + hh;
         if (p.S == 1) {
@@ -517,9 +567,10 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
 
 using UmmaFn = void (*)(const DecodeParams);
 
-UmmaFn pick_umma(int bk, int bv) {
+template <int GM>
+UmmaFn pick_umma_g(int bk, int bv) {
 #define KVQ_UCASE(BKv, BVv) \
-    if (bk == BKv && bv == BVv) return decode_umma_kernel<BKv, BVv>;
+    if (bk == BKv && bv == BVv) return decode_umma_kernel<BKv, BVv, GM>;
     KVQ_UCASE(2, 2) KVQ_UCASE(2, 4) KVQ_UCASE(2, 8)
     KVQ_UCASE(4, 2) KVQ_UCASE(4, 4) KVQ_UCASE(4, 8)
     KVQ_UCASE(8, 2) KVQ_UCASE(8, 4) KVQ_UCASE(8, 8)
@@ -527,33 +578,39 @@ UmmaFn pick_umma(int bk, int bv) {
     return nullptr;
 }
 
+UmmaFn pick_umma(int bk, int bv, int G) {
+    if (G < 1 || G > 8) return nullptr;
+    return G <= 4 ? pick_umma_g<4>(bk, bv) : pick_umma_g<8>(bk, bv);
+}
+
 std::mutex g_umma_mu;
-const void *g_umma_set[9] = {};
-size_t g_umma_smem[9] = {};
+const void *g_umma_set[18] = {};
+size_t g_umma_smem[18] = {};
 
 }  // namespace
 
-size_t decode_umma_smem_bytes(int bk, int bv) {
-    return static_cast<size_t>(UmmaSmem::bytes(unit_bytes(UD, bk, bv, 0, 2)));
+size_t decode_umma_smem_bytes(int bk, int bv, int G) {
+    const int rec = unit_bytes(UD, bk, bv, 0, 2);
+    return static_cast<size_t>(G <= 4 ? UmmaSmem<4>::bytes(rec) : UmmaSmem<8>::bytes(rec));
 }
 
-cudaError_t decode_umma_occupancy(int bk, int bv, int *ctas_per_sm) {
-    UmmaFn fn = pick_umma(bk, bv);
+cudaError_t decode_umma_occupancy(int bk, int bv, int G, int *ctas_per_sm) {
+    UmmaFn fn = pick_umma(bk, bv, G);
     if (!fn) return cudaErrorInvalidValue;
-    const size_t smem = decode_umma_smem_bytes(bk, bv);
+    const size_t smem = decode_umma_smem_bytes(bk, bv, G);
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, fn, 128, smem);
 }
 
 cudaError_t launch_decode_umma(const DecodeParams &p, int bk, int bv, cudaStream_t st) {
-    UmmaFn fn = pick_umma(bk, bv);
-    if (!fn || p.G < 1 || p.G > 4) return cudaErrorInvalidValue;
-    const size_t smem = decode_umma_smem_bytes(bk, bv);
+    UmmaFn fn = pick_umma(bk, bv, p.G);
+    if (!fn) return cudaErrorInvalidValue;
+    const size_t smem = decode_umma_smem_bytes(bk, bv, p.G);
     {
         std::lock_guard<std::mutex> lk(g_umma_mu);
         int slot = -1;
-        for (int k = 0; k < 9; ++k)
+        for (int k = 0; k < 18; ++k)
             if (g_umma_set[k] == reinterpret_cast<const void *>(fn) || g_umma_set[k] == nullptr) {
                 slot = k;
                 break;

@@ -873,7 +873,7 @@ static int umma_splits(kvq_handle *h, int layer, int *S_out) {
     int rc = ensure_device_info(h);
     if (rc) return rc;
     int occ = 1;
-    cudaError_t e = kvq::decode_umma_occupancy(g.bk, g.bv, &occ);
+    cudaError_t e = kvq::decode_umma_occupancy(g.bk, g.bv, h->desc.n_q_heads / h->desc.n_kv_heads, &occ);
     if (e != cudaSuccess) return cuda_fail(e, "tcgen05 decode occupancy");
     const long long units = static_cast<long long>(h->desc.batch) * h->desc.n_kv_heads;
     const long long slots = static_cast<long long>(std::max(occ, 1)) * h->sm_count;
@@ -897,13 +897,13 @@ static int umma_splits(kvq_handle *h, int layer, int *S_out) {
     return KVQ_OK;
 }
 
-// kvq_decode_attn on the tcgen05 kernel (per-channel keys, head_dim 128, G <= 4).
+// kvq_decode_attn on the tcgen05 kernel (per-channel keys, head_dim 128, G <= 8).
 static int decode_umma(kvq_handle *h, int layer, const void *q, void *out, int out_fp32, cudaStream_t st) {
     const LayerGeom &g = h->geom[layer];
     const int G = h->desc.n_q_heads / h->desc.n_kv_heads;
-    if (g.kmode != 0 || h->desc.head_dim != 128 || G > 4)
+    if (g.kmode != 0 || h->desc.head_dim != 128 || G > 8)
         return fail(KVQ_EUNSUPPORTED,
-                    "the tcgen05 decode path takes per-channel keys, head_dim 128 and at most 4 query heads per "
+                    "the tcgen05 decode path takes per-channel keys, head_dim 128 and at most 8 query heads per "
                     "kv head (layer %d: kmode %d, head_dim %d, %d heads per kv head)",
                     layer, g.kmode, h->desc.head_dim, G);
     const int L = h->len[layer];

@@ -1,9 +1,9 @@
 """GPU parity of the tcgen05 decode path (kvq_set_decode_path(h, KVQ_DECODE_TCGEN05))
 against the CPU oracle: both contractions of the per-layer decode on tcgen05.mma with
-tensor-memory accumulators, for per-channel keys, head_dim 128 and up to 4 query heads
-per kv head (the flash-decoding splits merged by log-sum-exp of the "TriAxialKV per-role
-mixed-precision KV quantization" page, Facts: decode path).  The same T1/T2 bounds as the
-mma.sync path; layers outside the path's scope are refused without a launch."""
+tensor-memory accumulators, for per-channel keys and head_dim 128 (the flash-decoding splits merged by log-sum-exp of the "TriAxialKV per-role
+mixed-precision KV quantization" page, Facts: decode path), up to 8 query heads per kv
+head.  The same T1/T2 bounds as the mma.sync path; layers outside the path's scope are
+refused without a launch."""
 import numpy as np
 import pytest
 import torch
@@ -28,7 +28,7 @@ def test_umma_bit_pairs(bk, bv):
              tag=f"umma-K{bk}V{bv}")
 
 
-@pytest.mark.parametrize("G", [1, 2, 3, 4])
+@pytest.mark.parametrize("G", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_umma_gqa(G):
     run_case(2, 2, G, 128, [(8, 4)], 0, [150, 30, 20], decode_at=[150, 200], splits=(0, 3), paths=UMMA,
              tag=f"umma-G{G}")
@@ -105,6 +105,38 @@ def test_umma_edge(kind, bits):
     assert kvq.kvq_device_status(cache.h) == 0
 
 
+@pytest.mark.parametrize("bits", [(8, 2), (4, 2), (2, 8)], ids=["K8V2", "K4V2", "K2V8"])
+def test_umma_qwen_gqa7(bits):
+    """Qwen2.5-7B attention shape (28 q / 4 kv heads, GQA 7) with 16 outlier key channels
+    per head x30, batch 4, context 1000 then single-token steps, forced and automatic splits,
+    both paths."""
+    wl = configs.Workload("umma-qwen", 1, 4, 28, 4, 128, 1000, 4, (bits,), n_outlier=16, outlier_lo=30.0,
+                          outlier_hi=30.0)
+    run_case(4, 4, 7, 128, [bits], 0, [1000, 1, 1, 1, 1], decode_at=[1000, 1003, 1004], splits=(0, 3), wl=wl,
+             paths=BOTH, tag=f"umma-qwen-K{bits[0]}V{bits[1]}")
+
+
+@pytest.mark.parametrize("kind", ["const", "zero_kv", "tiny", "large", "ties", "q_huge", "q_small"])
+def test_umma_edge_g8(kind):
+    """The boundary inputs at 8 query heads per kv head (the 16-row key operand)."""
+    B, Hkv, G, D, bits = 2, 2, 8, 128, (4, 4)
+    wl = workload(B, Hkv, G, D, name=f"umma-edge8-{kind}")
+    L = 100
+    cache = kvq.Cache(1, B, Hkv, Hkv * G, D, L, [bits], kmodes=[0])
+    K, V = inputs.edge_kv(kind, wl, 0, L, "cuda", bits=bits, kmode=0)
+    cache.append(0, K, V)
+    q = inputs.edge_q(kind, wl, 0, L, "cuda", bits=bits)
+    _, ref = oracle.layer(bits16(K), bits16(V), bits16(q), G, bits[0], bits[1], 0)
+    kvq.kvq_set_decode_path(cache.h, kvq.KVQ_DECODE_TCGEN05)
+    for S in (0, 2):
+        kvq.kvq_set_num_splits(cache.h, S)
+        out32 = cache.decode_attn(0, q, out_fp32=True)
+        out16 = cache.decode_attn(0, q, out_fp32=False)
+        torch.cuda.synchronize()
+        check_outputs(out32, out16, ref, f"G=8 {kind} splits={S}")
+    assert kvq.kvq_device_status(cache.h) == 0
+
+
 @pytest.mark.slow
 def test_umma_llama_c3_full_layer():
     """Full C3 size for a K4V2 layer: batch 64, 8 kv heads, context 4096 + 4 decode
@@ -113,11 +145,11 @@ def test_umma_llama_c3_full_layer():
     run_case(64, 8, 4, 128, [(4, 2)], 0, [4096] + [1] * 4, decode_at=[4100], wl=wl, paths=BOTH, tag="umma-c3")
 
 
-@pytest.mark.parametrize("case", ["per-token keys", "G=8", "head_dim 64"])
+@pytest.mark.parametrize("case", ["per-token keys", "head_dim 64"])
 def test_umma_refuses_other_layers(case):
-    """Per-token keys, more than 4 query heads per kv head or head_dim 64: KVQ_EUNSUPPORTED
-    from kvq_decode_attn on the tcgen05 path, and the default path still decodes."""
-    kmode, G, D = {"per-token keys": (1, 4, 128), "G=8": (0, 8, 128), "head_dim 64": (0, 4, 64)}[case]
+    """Per-token keys or head_dim 64: KVQ_EUNSUPPORTED from kvq_decode_attn on the tcgen05
+    path, and the default path still decodes."""
+    kmode, G, D = {"per-token keys": (1, 4, 128), "head_dim 64": (0, 4, 64)}[case]
     wl = workload(1, 2, G, D, name=f"umma-refuse-{G}-{D}")
     cache = kvq.Cache(1, 1, 2, 2 * G, D, 64, [(4, 4)], kmodes=[kmode])
     K, V = inputs.layer_kv(wl, 0, 40, "cuda")
