@@ -312,7 +312,7 @@ class WorkloadRun:
     once, untimed): the full step over every layer (fused append + decode launch; a
     token that completes a per-channel key group: append, then decode; paged plans:
     tagged append, then decode) and decode alone over every layer; with tcgen05=True, for
-    layers the tcgen05 decode path takes (per-channel keys, head_dim 128, G <= 8), also
+    layers the tcgen05 decode path takes (head_dim 128, G <= 8), also
     decode alone on that path."""
 
     def __init__(self, wl, stream, tcgen05=False):
@@ -367,7 +367,7 @@ class WorkloadRun:
                 cache.decode_attn(l, Qn[0, l], out[l], stream=stream)
         stream.synchronize()
         self.graphs, self.dec_graphs, self.tc_graphs, self.splits, self.Ls = [], [], [], [], []
-        tc = tcgen05 and not paged and wl.kmode == 0 and D == 128 and wl.G <= 8
+        tc = tcgen05 and not paged and D == 128 and wl.G <= 8
         for s in range(nsched):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):

@@ -192,7 +192,7 @@ KVQ_API int kvq_append_decode(kvq_handle *h, int layer, const void *K, const voi
  *   log-sum-exp, "TriAxialKV per-role mixed-precision KV quantization", Facts: decode
  *   path) with both contractions on the 5th-generation tensor cores: tcgen05.mma with
  *   operands staged in shared memory and accumulators in tensor memory.  Layers with
- *   per-channel keys, head_dim 128 and at most 8 query heads per kv head; any other layer
+ *   head_dim 128 and at most 8 query heads per kv head, either key mode; head_dim 64
  *   fails with KVQ_EUNSUPPORTED (nothing is launched).  Results meet the same tolerances
  *   as the default path, not bit for bit the same values.
  *

@@ -1,6 +1,6 @@
 // Split-KV decode attention over the packed per-layer cache on the 5th-generation tensor
 // cores (tcgen05.mma, accumulators in tensor memory): a variant of decode_split_kernel
-// for per-channel keys, head_dim 128 and up to 8 query heads per kv head.
+// for head_dim 128, up to 8 query heads per kv head and either key mode.
 //
 // The same attention as the mma.sync kernel (flash-decoding splits merged by log-sum-exp:
 // "TriAxialKV per-role mixed-precision KV quantization", Facts: decode path; one static
@@ -16,6 +16,8 @@
 //       scores warp 0 reads and passes on through shared memory;
 //     B_K = the block's key codes as exact fp16 integers; the zero term sum_c q~_c z_c is
 //       added on the CUDA cores.
+//     Per-token keys: A_K rows = (32-channel group j, head) with q~ masked to group j, one
+//       tile for every block; score = sum_j (s_tj D_K [(j, head)][t] + z_tj sum_{c in j} q~_c).
 //   values, per 4-block chunk:  D_V [c][n] = sum_t A_V [c][t] B_V [n][t]
 //     A_V = value codes (channel x token), B_V columns n = (group j, head, part): p_t s_tj
 //       as an fp16 hi/lo pair; channel c reads the 8 columns of its group j = c / 32; the
@@ -148,24 +150,28 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
 }
 
 // Shared memory of one CTA (dynamic, 1024-byte aligned base) for up to GM query heads per
-// kv head (GM = 4 or 8).
-template <int GM>
+// kv head (GM = 4 or 8) and key mode KM.
+template <int GM, int KM>
 struct UmmaSmem {
-    static constexpr int RK = 2 * GM;                    // A_K rows: hi and lo per head
+    // A_K rows: per-channel keys, hi and lo per head (one tile per block); per-token keys,
+    // (32-channel group, head) with q masked to the group (one tile for every block)
+    static constexpr int RK = KM == 0 ? 2 * GM : (UD / 32) * GM;
+    static constexpr int NAK = KM == 0 ? UCHUNK : 1;
     static constexpr int NV = 8 * GM;                    // B_V columns: (group, head, part)
     static constexpr int TILE = UD * 128 * 2;            // B_K (128 tokens x 128 channels) / A_V (128 x 128)
-    static constexpr int AK = RK * UD * 2;               // one block's A_K
+    static constexpr int AK = RK * UD * 2;               // one A_K tile
     static constexpr int BV = NV * 128 * 2;              // B_V: NV columns x 128 tokens
     static constexpr int QS_ROW = UD + 4;                // q~ row stride (floats): heads on different banks
     static constexpr int PB_ROW = 36;                    // p row stride (floats)
     static constexpr int SC_ROW = 36;                    // score row stride (floats): conflict-free 16-byte stores
     static constexpr int off_tile = 0;
     static constexpr int off_ak = off_tile + TILE;
-    static constexpr int off_bv = off_ak + UCHUNK * AK;
+    static constexpr int off_bv = off_ak + NAK * AK;
     static constexpr int off_qs = off_bv + BV;                        // q~ [GM][QS_ROW] fp32
     static constexpr int off_sc = off_qs + GM * QS_ROW * 4;           // per block: scores [RK][SC_ROW] fp32
     static constexpr int off_pb = off_sc + UCHUNK * RK * SC_ROW * 4;  // per warp: p [GM][PB_ROW]
-    static constexpr int off_zk = off_pb + UCHUNK * GM * PB_ROW * 4;  // per warp: key zero terms [GM]
+    static constexpr int off_zk = off_pb + UCHUNK * GM * PB_ROW * 4;  // per warp: key zero terms [GM] (KM = 0);
+                                                                      // q~ sums [group][GM] (KM = 1)
     static constexpr int off_zv = off_zk + UCHUNK * GM * 4;           // per warp: value zero terms [4 j][GM]
     static constexpr int off_red = off_zv + UCHUNK * 4 * GM * 4;      // reductions [4 warps][GM]
     static constexpr int off_bar = off_red + 4 * GM * 4;              // copy, mma, q barriers + tmem slot
@@ -174,20 +180,20 @@ struct UmmaSmem {
     static constexpr int bytes(int rec) { return off_stage + UCHUNK * rec; }
 };
 
-template <int BK, int BV, int GM>
+template <int BK, int BV, int GM, int KM>
 __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams p) {
     pdl_enter();
-    using SM = UmmaSmem<GM>;
+    using SM = UmmaSmem<GM, KM>;
     constexpr int D = UD, NJ = D / 32, KS = D / 16;
     constexpr int RK = SM::RK, NV = SM::NV;
-    constexpr int REC = unit_bytes(D, BK, BV, 0, 2);
+    constexpr int REC = unit_bytes(D, BK, BV, KM, 2);
     constexpr int KC = 4 * D * BK, KSZ = 4 * D, VC = 4 * D * BV;
     constexpr int PK = 16 / BK, PV = 16 / BV;
     constexpr int WHK = D * BK / 64, WHV = D * BV / 64;
     // GM = 4: the 8 A_K rows are read with stride-byte-offset 0, so every lane quarter
     // holds them and each warp reads its own block's scores; GM = 8: 16 rows, lanes 0-15
     // (warp 0's quarter) hold them and warp 0 passes every block's scores on
-    constexpr bool ALIAS = GM == 4;
+    constexpr bool ALIAS = KM == 0 && GM == 4;   // per-token keys: RK = 4 GM rows, never aliased
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -245,8 +251,10 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
     const uint32_t tmem = *tmem_slot;
     bool failed = false;
 
-    // ---- q~ = q log2(e)/sqrt(D) 2^kq per head (thread = channel), kq as in the mma.sync
-    // kernel: q~ < 2^15 and q~ s_k < 2^14 for the layer's largest key scale
+    // ---- q~ per head (thread = channel), kq as in the mma.sync kernel.  Per-channel keys:
+    // q~ = q log2(e)/sqrt(D) 2^kq with q~ < 2^15 and q~ s_k < 2^14 for the layer's largest
+    // key scale; per-token keys: q~ = q 2^kq < 2^15 (exact in fp16), the score scale applied
+    // with unscale
     if (!mbar_wait(q_bar, 0)) failed = true;
     const float smax_k = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[0])));
     const float smax_v = __half2float(__ushort_as_half(static_cast<unsigned short>(p.smax[1])));
@@ -256,7 +264,7 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
         float qv[GM], aq[GM], amax[GM];
 #pragma unroll
         for (int hh = 0; hh < GM; ++hh) {
-            qv[hh] = hh < G ? quant::bf16_to_f32(q_s[hh * D + tid]) * qscale : 0.f;
+            qv[hh] = hh < G ? quant::bf16_to_f32(q_s[hh * D + tid]) * (KM == 0 ? qscale : 1.f) : 0.f;
             aq[hh] = fabsf(qv[hh]);
         }
         block_maxn<GM>(aq, amax, red, warp, lane);
@@ -265,11 +273,31 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
             int kq = 0;
             if (amax[hh] > 0.f) {
                 kq = 14 - floor_log2(amax[hh]);
-                if (smax_k > 0.f) kq = min(kq, 12 - floor_log2(amax[hh]) - floor_log2(smax_k));
+                if (KM == 0 && smax_k > 0.f) kq = min(kq, 12 - floor_log2(amax[hh]) - floor_log2(smax_k));
                 kq = max(-120, min(100, kq));
             }
-            qs[hh * SM::QS_ROW + tid] = qv[hh] * pow2f(kq);
-            unscale[hh] = pow2f(-kq);
+            qv[hh] *= pow2f(kq);
+            qs[hh * SM::QS_ROW + tid] = qv[hh];
+            unscale[hh] = KM == 0 ? pow2f(-kq) : qscale * pow2f(-kq);
+        }
+        if constexpr (KM == 1) {
+            // A_K rows (group j, head hh): q~ of channel tid in row (tid / 32) GM + hh, zeros
+            // in the other groups' rows (fp16, exact: a bf16 value times a power of two below
+            // 2^15); the groups' q~ sums for the zero terms (warp = group)
+            const int j = tid >> 5;
+#pragma unroll
+            for (int r = 0; r < RK; ++r) {
+                const int hh = r % GM;
+                const float v = (r / GM == j && hh < G) ? qv[hh] : 0.f;
+                *reinterpret_cast<__half *>(ak + kmaj(r, tid, RK)) = __float2half_rn(v);
+            }
+#pragma unroll
+            for (int hh = 0; hh < GM; ++hh) {
+                float sum = qv[hh];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                if (lane == 0) zk[j * GM + hh] = sum;   // qsum [group][head]
+            }
         }
     }
     const int kp = smax_v > 0.f ? max(-24, min(14, 13 - floor_log2(smax_v))) : 14;
@@ -297,8 +325,10 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
         if (!mbar_wait(copy_bar, copy_phase)) failed = true;
         copy_phase ^= 1u;
 
-        // ---- (1) key tiles of this warp's block: B_K codes, A_K = q~ s hi/lo, zero term
-        if (mine && !is_tail) {
+        // ---- (1) key tiles of this warp's block: B_K codes; per-channel keys also A_K = q~ s
+        // hi/lo and the zero term (their open group's keys are the residual rows instead)
+        const bool has_codes = mine && (KM == 1 || !is_tail);
+        if (has_codes) {
             uint32_t kw[2][WHK];   // this lane's code words of both halves
             load_lane_words<WHK>(R, lane, kw[0]);
             load_lane_words<WHK>(R + 2 * D * BK, lane, kw[1]);
@@ -313,6 +343,8 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
                     *reinterpret_cast<uint32_t *>(tile + kmaj(tok, 16 * k + 8 + 2 * t, 128)) =
                         unpack<BK>(word, s0 % PK + 1);
                 }
+        }
+        if (KM == 0 && has_codes) {
             // A_K: lane = (row r = lane % RK, 8-channel chunks lane / RK + (32 / RK) i); row r:
             // head r % GM, the hi (r < GM) or lo part of q~_c s_c; one 16-byte store per chunk
             // (8 lanes fill a 128-byte core matrix).  The hi-row lanes also sum q~_c z_c.
@@ -359,13 +391,14 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
         tc_fence_after();
         // ---- (2) score MMAs: block i of the chunk into accumulator columns 32 i .. 32 i + 31
         bool any_k = false;
-        for (int i = 0; i < nb; ++i) any_k |= (c0 + i != tail_blk);
+        for (int i = 0; i < nb; ++i) any_k |= (KM == 1 || c0 + i != tail_blk);
         if (tid == 0 && any_k) {
             for (int i = 0; i < nb; ++i) {
-                if (c0 + i == tail_blk) continue;
+                if (KM == 0 && c0 + i == tail_blk) continue;
 #pragma unroll
                 for (int s = 0; s < KS; ++s) {
-                    const uint64_t ad = umma_desc(smem_u32(ak + i * SM::AK) + s * 2 * RK * 16, RK * 16, ALIAS ? 0 : 128);
+                    const uint8_t *a_tile = ak + (KM == 0 ? i * SM::AK : 0);
+                    const uint64_t ad = umma_desc(smem_u32(a_tile) + s * 2 * RK * 16, RK * 16, ALIAS ? 0 : 128);
                     const uint64_t bd = umma_desc(smem_u32(tile) + 512 * i + s * 4096, 2048, 128);
                     umma_f16(tmem + 32 * i, ad, bd, IDESC_K, s > 0 ? 1u : 0u);
                 }
@@ -394,7 +427,7 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
             // rows 0 .. RK - 1 sit in lanes 0 .. RK - 1: warp 0 reads every block's columns
             if (warp == 0) {
                 for (int i = 0; i < nb; ++i) {
-                    if (c0 + i == tail_blk) continue;
+                    if (KM == 0 && c0 + i == tail_blk) continue;
                     float v[32];
                     tmem_ld32(tmem + 32 * i, v);
                     if (lane < RK) {
@@ -406,12 +439,31 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
             }
             __syncthreads();
         }
-        if (mine && !is_tail) {
+        if (KM == 1 && mine) {
+            // per-token keys: sum over the groups of s_uj * rows (j, head) + z_uj * qsum (j, head)
+            float acc[GM];
+#pragma unroll
+            for (int hh = 0; hh < GM; ++hh) acc[hh] = 0.f;
+            if (lane < valid) {
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+                    const uint8_t *szp = R + KC + quant::tok_sz_off(lane, j, NJ);
+                    const float sk = __half2float(*reinterpret_cast<const __half *>(szp));
+                    const float zk_ = __half2float(*reinterpret_cast<const __half *>(szp + 4 * NJ));
+#pragma unroll
+                    for (int hh = 0; hh < GM; ++hh)
+                        acc[hh] = fmaf(sk, sc[(warp * RK + j * GM + hh) * SM::SC_ROW + lane],
+                                       fmaf(zk_, zk[j * GM + hh], acc[hh]));
+                }
+            }
+#pragma unroll
+            for (int hh = 0; hh < GM; ++hh) s4[hh] = acc[hh] * unscale[hh];
+        } else if (KM == 0 && mine && !is_tail) {
 #pragma unroll
             for (int hh = 0; hh < GM; ++hh)
                 s4[hh] = (sc[(warp * RK + hh) * SM::SC_ROW + lane] + sc[(warp * RK + GM + hh) * SM::SC_ROW + lane] +
                           zk[warp * GM + hh]) * unscale[hh];
-        } else if (is_tail) {
+        } else if (KM == 0 && is_tail) {
             // the open group's keys: bf16 residual rows, fp32 dot products
             float acc[GM];
 #pragma unroll
@@ -567,10 +619,10 @@ __global__ void __launch_bounds__(128, 1) decode_umma_kernel(const DecodeParams 
 
 using UmmaFn = void (*)(const DecodeParams);
 
-template <int GM>
+template <int GM, int KM>
 UmmaFn pick_umma_g(int bk, int bv) {
 #define KVQ_UCASE(BKv, BVv) \
-    if (bk == BKv && bv == BVv) return decode_umma_kernel<BKv, BVv, GM>;
+    if (bk == BKv && bv == BVv) return decode_umma_kernel<BKv, BVv, GM, KM>;
     KVQ_UCASE(2, 2) KVQ_UCASE(2, 4) KVQ_UCASE(2, 8)
     KVQ_UCASE(4, 2) KVQ_UCASE(4, 4) KVQ_UCASE(4, 8)
     KVQ_UCASE(8, 2) KVQ_UCASE(8, 4) KVQ_UCASE(8, 8)
@@ -578,39 +630,41 @@ UmmaFn pick_umma_g(int bk, int bv) {
     return nullptr;
 }
 
-UmmaFn pick_umma(int bk, int bv, int G) {
-    if (G < 1 || G > 8) return nullptr;
-    return G <= 4 ? pick_umma_g<4>(bk, bv) : pick_umma_g<8>(bk, bv);
+UmmaFn pick_umma(int bk, int bv, int G, int kmode) {
+    if (G < 1 || G > 8 || (kmode != 0 && kmode != 1)) return nullptr;
+    if (kmode == 0) return G <= 4 ? pick_umma_g<4, 0>(bk, bv) : pick_umma_g<8, 0>(bk, bv);
+    return G <= 4 ? pick_umma_g<4, 1>(bk, bv) : pick_umma_g<8, 1>(bk, bv);
 }
 
 std::mutex g_umma_mu;
-const void *g_umma_set[18] = {};
-size_t g_umma_smem[18] = {};
+const void *g_umma_set[36] = {};
+size_t g_umma_smem[36] = {};
 
 }  // namespace
 
-size_t decode_umma_smem_bytes(int bk, int bv, int G) {
-    const int rec = unit_bytes(UD, bk, bv, 0, 2);
-    return static_cast<size_t>(G <= 4 ? UmmaSmem<4>::bytes(rec) : UmmaSmem<8>::bytes(rec));
+size_t decode_umma_smem_bytes(int bk, int bv, int G, int kmode) {
+    const int rec = unit_bytes(UD, bk, bv, kmode, 2);
+    if (kmode == 0) return static_cast<size_t>(G <= 4 ? UmmaSmem<4, 0>::bytes(rec) : UmmaSmem<8, 0>::bytes(rec));
+    return static_cast<size_t>(G <= 4 ? UmmaSmem<4, 1>::bytes(rec) : UmmaSmem<8, 1>::bytes(rec));
 }
 
-cudaError_t decode_umma_occupancy(int bk, int bv, int G, int *ctas_per_sm) {
-    UmmaFn fn = pick_umma(bk, bv, G);
+cudaError_t decode_umma_occupancy(int bk, int bv, int G, int kmode, int *ctas_per_sm) {
+    UmmaFn fn = pick_umma(bk, bv, G, kmode);
     if (!fn) return cudaErrorInvalidValue;
-    const size_t smem = decode_umma_smem_bytes(bk, bv, G);
+    const size_t smem = decode_umma_smem_bytes(bk, bv, G, kmode);
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, fn, 128, smem);
 }
 
-cudaError_t launch_decode_umma(const DecodeParams &p, int bk, int bv, cudaStream_t st) {
-    UmmaFn fn = pick_umma(bk, bv, p.G);
+cudaError_t launch_decode_umma(const DecodeParams &p, int bk, int bv, int kmode, cudaStream_t st) {
+    UmmaFn fn = pick_umma(bk, bv, p.G, kmode);
     if (!fn) return cudaErrorInvalidValue;
-    const size_t smem = decode_umma_smem_bytes(bk, bv, p.G);
+    const size_t smem = decode_umma_smem_bytes(bk, bv, p.G, kmode);
     {
         std::lock_guard<std::mutex> lk(g_umma_mu);
         int slot = -1;
-        for (int k = 0; k < 18; ++k)
+        for (int k = 0; k < 36; ++k)
             if (g_umma_set[k] == reinterpret_cast<const void *>(fn) || g_umma_set[k] == nullptr) {
                 slot = k;
                 break;

@@ -873,7 +873,7 @@ static int umma_splits(kvq_handle *h, int layer, int *S_out) {
     int rc = ensure_device_info(h);
     if (rc) return rc;
     int occ = 1;
-    cudaError_t e = kvq::decode_umma_occupancy(g.bk, g.bv, h->desc.n_q_heads / h->desc.n_kv_heads, &occ);
+    cudaError_t e = kvq::decode_umma_occupancy(g.bk, g.bv, h->desc.n_q_heads / h->desc.n_kv_heads, g.kmode, &occ);
     if (e != cudaSuccess) return cuda_fail(e, "tcgen05 decode occupancy");
     const long long units = static_cast<long long>(h->desc.batch) * h->desc.n_kv_heads;
     const long long slots = static_cast<long long>(std::max(occ, 1)) * h->sm_count;
@@ -897,22 +897,22 @@ static int umma_splits(kvq_handle *h, int layer, int *S_out) {
     return KVQ_OK;
 }
 
-// kvq_decode_attn on the tcgen05 kernel (per-channel keys, head_dim 128, G <= 8).
+// kvq_decode_attn on the tcgen05 kernel (head_dim 128, G <= 8, either key mode).
 static int decode_umma(kvq_handle *h, int layer, const void *q, void *out, int out_fp32, cudaStream_t st) {
     const LayerGeom &g = h->geom[layer];
     const int G = h->desc.n_q_heads / h->desc.n_kv_heads;
-    if (g.kmode != 0 || h->desc.head_dim != 128 || G > 8)
+    if (h->desc.head_dim != 128 || G > 8)
         return fail(KVQ_EUNSUPPORTED,
-                    "the tcgen05 decode path takes per-channel keys, head_dim 128 and at most 8 query heads per "
-                    "kv head (layer %d: kmode %d, head_dim %d, %d heads per kv head)",
-                    layer, g.kmode, h->desc.head_dim, G);
+                    "the tcgen05 decode path takes head_dim 128 and at most 8 query heads per kv head (layer %d: "
+                    "head_dim %d, %d heads per kv head)",
+                    layer, h->desc.head_dim, G);
     const int L = h->len[layer];
     const int nblk = (L + 31) / 32;
     int S = 1, rc;
     if ((rc = umma_splits(h, layer, &S))) return rc;
     kvq::DecodeParams p{};
     p.rec = h->ws + g.rec_off;
-    p.res = reinterpret_cast<const uint16_t *>(h->ws + g.res_off);
+    p.res = g.res_off >= 0 ? reinterpret_cast<const uint16_t *>(h->ws + g.res_off) : nullptr;
     p.q = static_cast<const uint16_t *>(q);
     p.smax = smax_slot(h, layer, static_cast<int>(h->ver[layer]));
     if ((rc = fill_lengths(h, layer, p, 0, st))) return rc;
@@ -932,7 +932,7 @@ static int decode_umma(kvq_handle *h, int layer, const void *q, void *out, int o
     p.rec_bytes = g.rec_bytes;
     p.btab = block_table(h, layer);
     if ((rc = prepare_status(h, st))) return rc;
-    cudaError_t e = kvq::launch_decode_umma(p, g.bk, g.bv, st);
+    cudaError_t e = kvq::launch_decode_umma(p, g.bk, g.bv, g.kmode, st);
     if (e != cudaSuccess) return cuda_fail(e, "tcgen05 decode launch");
     note_write(h, st, -1);
     if (p.S > 1) {

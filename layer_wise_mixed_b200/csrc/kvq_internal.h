@@ -224,11 +224,11 @@ cudaError_t decode_occupancy(int D, int bk, int bv, int kmode, int G, long long 
                              int nstage, int nextra, int *ctas_per_sm);
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t st);
 cudaError_t launch_decode_paged(const PagedDecodeParams &p, cudaStream_t st);
-// tcgen05 variant of the per-layer decode (per-channel keys, head_dim 128, G <= 8,
+// tcgen05 variant of the per-layer decode (head_dim 128, G <= 8, either key mode,
 // decode-only; kvq_decode_umma.cu): the kernel's dynamic shared memory, CTAs per SM, launch
-size_t decode_umma_smem_bytes(int bk, int bv, int G);
-cudaError_t decode_umma_occupancy(int bk, int bv, int G, int *ctas_per_sm);
-cudaError_t launch_decode_umma(const DecodeParams &p, int bk, int bv, cudaStream_t st);
+size_t decode_umma_smem_bytes(int bk, int bv, int G, int kmode);
+cudaError_t decode_umma_occupancy(int bk, int bv, int G, int kmode, int *ctas_per_sm);
+cudaError_t launch_decode_umma(const DecodeParams &p, int bk, int bv, int kmode, cudaStream_t st);
 cudaError_t decode_paged_occupancy(int nstage, int *ctas_per_sm);
 int decode_paged_stages();
 size_t decode_paged_smem_bytes(int nstage);

@@ -1,6 +1,6 @@
 """GPU parity of the tcgen05 decode path (kvq_set_decode_path(h, KVQ_DECODE_TCGEN05))
 against the CPU oracle: both contractions of the per-layer decode on tcgen05.mma with
-tensor-memory accumulators, for per-channel keys and head_dim 128 (the flash-decoding splits merged by log-sum-exp of the "TriAxialKV per-role
+tensor-memory accumulators, for both key modes and head_dim 128 (the flash-decoding splits merged by log-sum-exp of the "TriAxialKV per-role
 mixed-precision KV quantization" page, Facts: decode path), up to 8 query heads per kv
 head.  The same T1/T2 bounds as the mma.sync path; layers outside the path's scope are
 refused without a launch."""
@@ -19,27 +19,29 @@ UMMA = (kvq.KVQ_DECODE_TCGEN05,)
 BOTH = (kvq.KVQ_DECODE_MMA_SYNC, kvq.KVQ_DECODE_TCGEN05)
 
 
+@pytest.mark.parametrize("kmode", [0, 1])
 @pytest.mark.parametrize("bk", [2, 4, 8])
 @pytest.mark.parametrize("bv", [2, 4, 8])
-def test_umma_bit_pairs(bk, bv):
-    """Every precision pair: 3 full blocks and a 1-token tail, then 9 full blocks and a
-    12-token tail (three 4-block chunks, the last one partial), forced splits."""
-    run_case(2, 2, 4, 128, [(bk, bv)], 0, [97, 203], decode_at=[97, 300], splits=(0, 1, 2, 3, 5), paths=BOTH,
-             tag=f"umma-K{bk}V{bv}")
+def test_umma_bit_pairs(bk, bv, kmode):
+    """Every precision pair and key mode: 3 full blocks and a 1-token tail, then 9 full
+    blocks and a 12-token tail (three 4-block chunks, the last one partial), forced splits."""
+    run_case(2, 2, 4, 128, [(bk, bv)], kmode, [97, 203], decode_at=[97, 300], splits=(0, 1, 2, 3, 5), paths=BOTH,
+             tag=f"umma-K{bk}V{bv}m{kmode}")
 
 
-@pytest.mark.parametrize("G", [1, 2, 3, 4, 5, 6, 7, 8])
-def test_umma_gqa(G):
-    run_case(2, 2, G, 128, [(8, 4)], 0, [150, 30, 20], decode_at=[150, 200], splits=(0, 3), paths=UMMA,
-             tag=f"umma-G{G}")
+@pytest.mark.parametrize("G,kmode", [(g, 0) for g in range(1, 9)] + [(1, 1), (2, 1), (4, 1)])
+def test_umma_gqa(G, kmode):
+    run_case(2, 2, G, 128, [(8, 4)], kmode, [150, 30, 20], decode_at=[150, 200], splits=(0, 3), paths=UMMA,
+             tag=f"umma-G{G}m{kmode}")
 
 
+@pytest.mark.parametrize("kmode", [0, 1])
 @pytest.mark.parametrize("L", [1, 2, 31, 32, 33, 64, 127, 128, 129, 131, 160, 257])
-def test_umma_lengths(L):
+def test_umma_lengths(L, kmode):
     """Tail-only units, whole groups without a tail, 4-block chunk boundaries."""
     first = max(1, L - 3)
-    run_case(2, 2, 4, 128, [(4, 2)], 0, [first] + [1] * (L - first), decode_at=[first, L], splits=(0, 1, 2),
-             paths=UMMA, tag=f"umma-L{L}")
+    run_case(2, 2, 4, 128, [(4, 2)], kmode, [first] + [1] * (L - first), decode_at=[first, L], splits=(0, 1, 2),
+             paths=UMMA, tag=f"umma-L{L}m{kmode}")
 
 
 def test_umma_llama_c2_schedule():
@@ -82,26 +84,27 @@ def test_umma_ragged_and_pools():
 EDGE = ["const", "zero_k", "zero_v", "zero_kv", "tiny", "tiny_mixed", "large", "ties", "q_big", "q_huge", "q_small"]
 
 
+@pytest.mark.parametrize("kmode", [0, 1])
 @pytest.mark.parametrize("kind", EDGE)
 @pytest.mark.parametrize("bits", [(4, 2), (8, 8), (2, 4)], ids=["K4V2", "K8V8", "K2V4"])
-def test_umma_edge(kind, bits):
+def test_umma_edge(kind, bits, kmode):
     """The quantizer's and decoder's boundary inputs (constant groups, zero tensors,
     subnormal fp16 scales, |x| near 2^14, round-half-even ties, q far outside N(0, 1))."""
     B, Hkv, G, D = 2, 2, 4, 128
     wl = workload(B, Hkv, G, D, name=f"umma-edge-{kind}")
     L = 150
-    cache = kvq.Cache(1, B, Hkv, Hkv * G, D, L, [bits], kmodes=[0])
-    K, V = inputs.edge_kv(kind, wl, 0, L, "cuda", bits=bits, kmode=0)
+    cache = kvq.Cache(1, B, Hkv, Hkv * G, D, L, [bits], kmodes=[kmode])
+    K, V = inputs.edge_kv(kind, wl, 0, L, "cuda", bits=bits, kmode=kmode)
     cache.append(0, K, V)
     q = inputs.edge_q(kind, wl, 0, L, "cuda", bits=bits)
-    _, ref = oracle.layer(bits16(K), bits16(V), bits16(q), G, bits[0], bits[1], 0)
+    _, ref = oracle.layer(bits16(K), bits16(V), bits16(q), G, bits[0], bits[1], kmode)
     kvq.kvq_set_decode_path(cache.h, kvq.KVQ_DECODE_TCGEN05)
     for S in (0, 2):
         kvq.kvq_set_num_splits(cache.h, S)
         out32 = cache.decode_attn(0, q, out_fp32=True)
         out16 = cache.decode_attn(0, q, out_fp32=False)
         torch.cuda.synchronize()
-        check_outputs(out32, out16, ref, f"{kind} K{bits[0]}V{bits[1]} splits={S}")
+        check_outputs(out32, out16, ref, f"{kind} K{bits[0]}V{bits[1]} m{kmode} splits={S}")
     assert kvq.kvq_device_status(cache.h) == 0
 
 
@@ -145,12 +148,12 @@ def test_umma_llama_c3_full_layer():
     run_case(64, 8, 4, 128, [(4, 2)], 0, [4096] + [1] * 4, decode_at=[4100], wl=wl, paths=BOTH, tag="umma-c3")
 
 
-@pytest.mark.parametrize("case", ["per-token keys", "head_dim 64"])
-def test_umma_refuses_other_layers(case):
-    """Per-token keys or head_dim 64: KVQ_EUNSUPPORTED from kvq_decode_attn on the tcgen05
-    path, and the default path still decodes."""
-    kmode, G, D = {"per-token keys": (1, 4, 128), "head_dim 64": (0, 4, 64)}[case]
-    wl = workload(1, 2, G, D, name=f"umma-refuse-{G}-{D}")
+@pytest.mark.parametrize("kmode", [0, 1])
+def test_umma_refuses_head_dim_64(kmode):
+    """head_dim 64: KVQ_EUNSUPPORTED from kvq_decode_attn on the tcgen05 path, and the
+    default path still decodes."""
+    G, D = 4, 64
+    wl = workload(1, 2, G, D, name=f"umma-refuse-{kmode}")
     cache = kvq.Cache(1, 1, 2, 2 * G, D, 64, [(4, 4)], kmodes=[kmode])
     K, V = inputs.layer_kv(wl, 0, 40, "cuda")
     cache.append(0, K[:1].contiguous(), V[:1].contiguous())
