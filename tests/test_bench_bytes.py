@@ -35,3 +35,31 @@ def test_default_schedule_mean():
     # the default workload's 128 decode steps (L = 129..256), K8V4: 24.0 MB per layer on average
     mean = sum(bench.decode_bytes(64, 8, 4, 128, L, 8, 4, 0) for L in range(129, 257)) / 128
     assert mean == pytest.approx(24.0e6, rel=2e-3)
+
+
+def test_decode_paths_entry():
+    """Per-path launch time and roofline fraction: GB/s = algorithmic bytes / time."""
+    d = bench.decode_paths_entry(18_395_136.0, 0.008, 0.032, 6558.7, "decode_split_kernel")
+    assert d["mma_sync"]["kernel"] == "decode_split_kernel"
+    assert d["mma_sync"]["avg_launch_us"] == pytest.approx(8.0)
+    assert d["mma_sync"]["hbm_gbs"] == pytest.approx(18_395_136.0 / 8e-6 / 1e9)
+    assert d["mma_sync"]["frac"] == pytest.approx(d["mma_sync"]["hbm_gbs"] / 6558.7)
+    assert d["tcgen05"]["kernel"] == "decode_umma_kernel"
+    assert d["tcgen05"]["frac"] == pytest.approx(d["mma_sync"]["frac"] / 4)
+    assert "tcgen05" not in bench.decode_paths_entry(1e6, 0.01, None, 6558.7, "decode_paged_kernel")
+
+
+def test_captured_traffic_follows_the_source_hash(tmp_path, monkeypatch):
+    """The committed traffic blocks are used only while their source hash matches, scaled
+    to the caller's algorithmic bytes."""
+    sha = bench.kernel_source_sha256()
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "decode_split_traffic.txt").write_text(
+        f"# test\nsource_sha256: {sha}\nworkload: w\nkernel: k\nL: 1\ndram_bytes: 104\nalgorithmic_bytes: 100\n\n"
+        f"source_sha256: {'0' * 64}\nworkload: v\nkernel: k\nL: 1\ndram_bytes: 200\nalgorithmic_bytes: 100\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_sha256", lambda: sha)
+    assert bench.captured_traffic("w", 1000.0) == pytest.approx(1040.0)
+    assert bench.captured_traffic("v", 1000.0) is None      # stale hash
+    assert bench.captured_traffic("x", 1000.0) is None      # no capture
