@@ -207,7 +207,8 @@ KVQ_API int kvq_set_decode_path(kvq_handle *h, int path);
  * value is capped by the number of 32-token blocks and the partial buffer size). */
 KVQ_API int kvq_set_num_splits(kvq_handle *h, int num_splits);
 
-/* The split count kvq_decode_attn would use for `layer` at its current length. */
+/* The split count kvq_decode_attn would use for `layer` at its current length, on the
+ * handle's current decode path (kvq_set_decode_path). */
 KVQ_API int kvq_get_num_splits(const kvq_handle *h, int layer, int *num_splits);
 
 /* Copy one layer's cache to host memory in canonical order (parity checks): for each

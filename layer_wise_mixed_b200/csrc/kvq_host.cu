@@ -1156,7 +1156,12 @@ int kvq_get_num_splits(const kvq_handle *hc, int layer, int *num_splits) {
         return ok();
     }
     int S = 1, nstage = 2, nextra = 0;
-    if ((rc = splits_for(h, layer, &S, &nstage, &nextra))) return rc;
+    const int G = h->desc.n_q_heads / h->desc.n_kv_heads;
+    if (h->decode_path == KVQ_DECODE_TCGEN05 && h->desc.head_dim == 128 && G <= 8) {
+        if ((rc = umma_splits(h, layer, &S))) return rc;
+    } else if ((rc = splits_for(h, layer, &S, &nstage, &nextra))) {
+        return rc;
+    }
     const int nblk = (L + 31) / 32;
     const int bps = (nblk + S - 1) / S;
     *num_splits = (nblk + bps - 1) / bps;

@@ -166,3 +166,31 @@ def test_umma_refuses_head_dim_64(kmode):
     out = cache.decode_attn(0, q, out_fp32=True)
     torch.cuda.synchronize()
     assert torch.isfinite(out).all()
+
+
+def test_umma_split_count_query():
+    """kvq_get_num_splits answers for the handle's decode path: forced counts on both paths,
+    and on the tcgen05 path the automatic count is the one its launch uses (outputs still
+    match the oracle at that count)."""
+    B, Hkv, G, D, bits = 2, 2, 4, 128, (4, 2)
+    wl = workload(B, Hkv, G, D, name="umma-splits")
+    cache = kvq.Cache(1, B, Hkv, Hkv * G, D, 300, [bits], kmodes=[0])
+    K, V = inputs.layer_kv(wl, 0, 300, "cuda")
+    cache.append(0, K, V)
+    q = inputs.step_q(wl, 0, 1, "cuda")
+    _, ref = oracle.layer(bits16(K), bits16(V), bits16(q), G, *bits, 0)
+    for path in (kvq.KVQ_DECODE_MMA_SYNC, kvq.KVQ_DECODE_TCGEN05):
+        kvq.kvq_set_decode_path(cache.h, path)
+        kvq.kvq_set_num_splits(cache.h, 3)
+        assert kvq.kvq_get_num_splits(cache.h, 0) == 3
+        kvq.kvq_set_num_splits(cache.h, 0)
+        S = kvq.kvq_get_num_splits(cache.h, 0)
+        assert 1 <= S <= 10
+        kvq.kvq_set_num_splits(cache.h, S)
+        forced = cache.decode_attn(0, q, out_fp32=True)
+        kvq.kvq_set_num_splits(cache.h, 0)
+        auto = cache.decode_attn(0, q, out_fp32=True)
+        torch.cuda.synchronize()
+        assert torch.equal(forced, auto), (path, S)   # the same split count, the same launch
+        check_outputs(auto, auto.to(torch.bfloat16), ref, f"path={path} splits={S}")
+    assert kvq.kvq_device_status(cache.h) == 0
