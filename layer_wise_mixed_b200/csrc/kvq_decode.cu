@@ -215,17 +215,19 @@ __device__ __forceinline__ void acc_init(WarpAcc<D, NT> &A) {
 }
 
 // One unit of NH 16-token halves (32-token block record, or 16-token page when NH = 1)
-// staged at R; `valid` tokens are present (TAIL: valid may be < 16 NH; per-channel
+// staged at R, of which the first NHP are processed (NHP = 1: a tail block whose tokens
+// all sit in its first half); `valid` tokens are present (TAIL: valid may be < 16 NH; per-channel
 // TAIL blocks take their keys from the bf16 residual).
 // PAIR: R holds two 16-token pages (per-token keys), one per half, each laid out
 // [K codes][K scales/zeros][V codes][V scales/zeros], instead of one 32-token record.
-template <int BK, int BV, int KM, int D, int NT, int NH, bool TAIL, bool PAIR = false>
+template <int BK, int BV, int KM, int D, int NT, int NH, bool TAIL, bool PAIR = false, int NHP = NH>
 __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R, const int valid,
                                              const BodyCtx &c) {
     constexpr int KS = D / 16;
     constexpr int NJ = D / 32;
     constexpr int NTOK = 16 * NH;        // tokens in the unit
-    constexpr int NTI = 2 * NH;          // 8-token score tiles
+    constexpr int NTI = 2 * NHP;         // 8-token score tiles processed
+    static_assert(NHP >= 1 && NHP <= NH && (NHP == NH || TAIL), "a partial unit is a tail");
     constexpr int WHK = D * BK / 64, WHV = D * BV / 64;
     constexpr int PK = 16 / BK, PV = 16 / BV;
     constexpr int KC = 2 * NH * D * BK, KSZ = (KM == 0 ? 4 * D : 2 * NH * D), VC = 2 * NH * D * BV;
@@ -280,14 +282,14 @@ __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R
         constexpr int CH = WHK < 4 ? WHK : 4;        // lane words per chunk
 #pragma unroll
         for (int k = 0; k < KS; ++k) {
-            uint32_t kw[NH][WPK];
+            uint32_t kw[NHP][WPK];
             const int w0 = (4 * k) / PK;
 #pragma unroll
             for (int x = 0; x < WPK; ++x) {
                 const int w = w0 + x;
                 const int off = (((w / CH) * 32 + lane) * CH + (w % CH)) * 4;
 #pragma unroll
-                for (int hf = 0; hf < NH; ++hf) kw[hf][x] = *reinterpret_cast<const uint32_t *>(kcode(hf) + off);
+                for (int hf = 0; hf < NHP; ++hf) kw[hf][x] = *reinterpret_cast<const uint32_t *>(kcode(hf) + off);
             }
             const uint4 aqv = c.aq_s[k * 32 + lane];
             const uint32_t ak[4] = {aqv.x, aqv.y, aqv.z, aqv.w};
@@ -406,7 +408,7 @@ __device__ __forceinline__ void process_unit(WarpAcc<D, NT> &A, const uint8_t *R
 
     // ===== O^T += V^T P'^T and the zero-point term (16-token steps) =====
 #pragma unroll
-    for (int kk = 0; kk < NH; ++kk) {
+    for (int kk = 0; kk < NHP; ++kk) {
         uint32_t vw[WHV];
         load_lane_words<WHV>(vcode(kk), lane, vw);
         uint32_t pah, pal, pbh, pbl;   // p of token pairs A (16kk+2t, +1) and B (+8, +9)
@@ -1093,7 +1095,8 @@ __global__ void __launch_bounds__(NW * 32, NT == 1 ? 4 : 3) decode_split_kernel(
             const bool patch = append_here && tail_blk == new_blk;
             if (patch)
                 patch_stage<BK, BV, KM, D>(const_cast<uint8_t *>(pipe_front(P)), (L - 1) & 31, append_scratch, lane);
-            process_unit<BK, BV, KM, D, NT, 2, true>(A, pipe_front(P), rem, c);
+            if (rem <= 16) process_unit<BK, BV, KM, D, NT, 2, true, false, 1>(A, pipe_front(P), rem, c);
+            else process_unit<BK, BV, KM, D, NT, 2, true>(A, pipe_front(P), rem, c);
             ++i;
         }
     }
