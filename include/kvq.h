@@ -55,8 +55,10 @@
  *    library never allocates device memory.  `stream` is a cudaStream_t (NULL = the
  *    legacy default stream); calls that take one are asynchronous on it.
  *  - K/V/q/out pointers must be 16-byte aligned; the workspace 256-byte aligned.
- *  - All sequences in the batch have the same length (the library tracks one L per
- *    layer).  A handle is not thread-safe: serialize calls on one handle.
+ *  - Sequences of a plan start at length 0 and stay equal under kvq_append and
+ *    kvq_append_decode; kvq_append_ragged gives them their own lengths (per-layer
+ *    plans), and the library then tracks one length per (layer, sequence).  A handle
+ *    is not thread-safe: serialize calls on one handle.
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -122,8 +124,9 @@ typedef struct kvq_handle kvq_handle;
 /* Validate a plan and create a host handle (host memory only). */
 KVQ_API int kvq_plan(const kvq_plan_desc *desc, kvq_handle **out);
 
-/* Device workspace size the plan needs: all layers' cache regions, the split
- * partials, split arrival counters and a status word. */
+/* Device workspace size the plan needs: all layers' cache regions (slabs, or block
+ * pools and block tables), the per-layer length tables, the split partials, split
+ * arrival counters, the scale maxima and a status word. */
 KVQ_API int kvq_workspace_bytes(const kvq_handle *h, size_t *bytes);
 
 /* Bind caller-owned device memory (>= kvq_workspace_bytes, 256-byte aligned) and
@@ -142,8 +145,9 @@ KVQ_API int kvq_append(kvq_handle *h, int layer, const void *K, const void *V, i
  * batches); every other entry point works per request from then on: decode attends
  * over each sequence's own tokens, kvq_append_decode appends one token to each,
  * kvq_export_layer exports each unit at its own length, kvq_truncate cuts every
- * sequence to the same length.  Plans with more than 64 requests accept only equal
- * lengths (KVQ_EUNSUPPORTED): the per-request lengths travel in the kernels' parameters.
+ * sequence to the same length.  Any batch size: up to 64 requests the per-request
+ * lengths travel in the kernels' parameters, above that in a per-layer [2][B] int32
+ * table in the workspace, written on `stream` just before the launch that reads it.
  * Errors as kvq_append, plus KVQ_EINVAL for a count outside [0, n_max]. */
 KVQ_API int kvq_append_ragged(kvq_handle *h, int layer, const void *K, const void *V, const int32_t *n_new,
                               int n_max, void *stream);
