@@ -295,6 +295,28 @@ KVQ_API int kvq_tag_distortion(int num_layers, int num_requests, int n_q_heads, 
                                int T, const uint16_t *Q, const uint16_t *K, const uint16_t *V,
                                const int32_t *tags, int num_tags, double *D2, double *D4, int64_t *counts);
 
+/* Device workspace bytes that kvq_tag_distortion_device needs at these sizes: the
+ * per-request token lists, one layer's dequantized keys and values at 2 and 4 bits
+ * (4 x num_requests x n_kv_heads x T x head_dim fp64) and the per-CTA error sums.
+ * Errors as kvq_tag_distortion_device's size checks. */
+KVQ_API int kvq_tag_distortion_workspace_bytes(int num_layers, int num_requests, int n_q_heads, int n_kv_heads,
+                                               int head_dim, int T, int num_tags, size_t *bytes);
+
+/* kvq_tag_distortion computed on the GPU: the same D_k(2), D_k(4) and counts, by the
+ * same definition, with the attention in fp64 on the device (equal to the host entry
+ * point's up to the order of the sums).  Q, K, V: device pointers, same layouts,
+ * 16-byte aligned; tags, D2, D4, counts: host pointers; workspace: caller-owned device
+ * memory of at least kvq_tag_distortion_workspace_bytes, 256-byte aligned.  Work is
+ * issued on `stream`; the call returns after the results are on the host (it
+ * synchronizes `stream`).  head_dim 64 or 128 (else KVQ_EUNSUPPORTED).  Cost
+ * O(layers x requests x n_q_heads x T^2 x head_dim), about 4 passes over each query's
+ * keys.  Errors: KVQ_EINVAL (shapes, tags out of range, null), KVQ_EALIGN,
+ * KVQ_EUNBOUND (workspace), KVQ_ECUDA. */
+KVQ_API int kvq_tag_distortion_device(int num_layers, int num_requests, int n_q_heads, int n_kv_heads,
+                                      int head_dim, int T, const void *Q, const void *K, const void *V,
+                                      const int32_t *tags, int num_tags, void *workspace, size_t workspace_bytes,
+                                      double *D2, double *D4, int64_t *counts, void *stream);
+
 /* bits[k] in {2, 4} for every tag: minimise sum_k D_{b_k}(k) subject to
  * sum_k counts[k] * bits[k] <= avg_bits * sum_k counts[k].  Tags with counts[k] == 0
  * take no part and get 4.  With P <= 22 tags present: exhaustive over all 2^P choices,

@@ -86,6 +86,8 @@ def load() -> ctypes.CDLL:
         "kvq_device_status": (I, [P, P, ctypes.POINTER(ctypes.c_uint)]),
         "kvq_tag_distortion": (I, [I, I, I, I, I, I, P, P, P, P, I, P, P, P]),
         "kvq_tag_allocate": (I, [I, P, P, P, ctypes.c_double, P, P]),
+        "kvq_tag_distortion_workspace_bytes": (I, [I, I, I, I, I, I, I, ctypes.POINTER(SZ)]),
+        "kvq_tag_distortion_device": (I, [I, I, I, I, I, I, P, P, P, P, I, P, SZ, P, P, P, P]),
         "kvq_destroy": (None, [P]),
         "kvq_last_error": (ctypes.c_char_p, []),
     }
@@ -250,6 +252,40 @@ def kvq_tag_distortion(Q, K, V, tags, num_tags: int):
     p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
     _check(load().kvq_tag_distortion(NL, R, Hq, Hkv, D, T, p(Q), p(K), p(V), p(tags), num_tags, p(D2), p(D4),
                                      p(counts)))
+    return D2, D4, counts
+
+
+def kvq_tag_distortion_workspace_bytes(NL: int, R: int, Hq: int, Hkv: int, D: int, T: int, num_tags: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load().kvq_tag_distortion_workspace_bytes(NL, R, Hq, Hkv, D, T, num_tags, ctypes.byref(n)))
+    return n.value
+
+
+def kvq_tag_distortion_device(Q, K, V, tags, num_tags: int, workspace=None, stream=None):
+    """kvq_tag_distortion on the GPU: Q, K, V CUDA tensors (bf16 or int16/uint16 holding bf16
+    bits) [NL, R, Hq, T, D] / [NL, R, Hkv, T, D]; tags host int32 [R, T].  The workspace
+    (a CUDA uint8 tensor) is allocated here when not given.  Returns (D2, D4, counts)."""
+    import numpy as np
+    import torch
+    for a in (Q, K, V):
+        if not (a.is_cuda and a.is_contiguous() and a.element_size() == 2):
+            raise ValueError("Q, K, V must be contiguous 2-byte CUDA tensors")
+    tags = np.ascontiguousarray(tags, np.int32)
+    NL, R, Hq, T, D = Q.shape
+    Hkv = K.shape[2]
+    if tuple(K.shape) != (NL, R, Hkv, T, D) or tuple(V.shape) != tuple(K.shape) or tags.shape != (R, T):
+        raise ValueError("shape mismatch")
+    need = kvq_tag_distortion_workspace_bytes(NL, R, Hq, Hkv, D, T, num_tags)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    D2 = np.zeros(num_tags, np.float64)
+    D4 = np.zeros(num_tags, np.float64)
+    counts = np.zeros(num_tags, np.int64)
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    st = _stream(stream)
+    _check(load().kvq_tag_distortion_device(NL, R, Hq, Hkv, D, T, Q.data_ptr(), K.data_ptr(), V.data_ptr(), p(tags),
+                                            num_tags, workspace.data_ptr(), workspace.numel(), p(D2), p(D4),
+                                            p(counts), st))
     return D2, D4, counts
 
 

@@ -245,3 +245,31 @@ def test_allocation_mask_meets_budget():
     ids = inputs.tag_ids(w, w.max_ctx).numpy()
     bits = tagalloc.tag_bits(w)
     assert np.array_equal(m, bits[ids])
+
+
+def test_device_distortion_host_checks():
+    """The device entry point's argument checks run on the host before any CUDA call
+    (fake device addresses are never touched)."""
+    import ctypes
+    L = kvq.load()
+    n = ctypes.c_size_t(0)
+    assert L.kvq_tag_distortion_workspace_bytes(1, 2, 8, 2, 128, 100, 5, ctypes.byref(n)) == 0
+    small = n.value
+    assert L.kvq_tag_distortion_workspace_bytes(1, 2, 8, 2, 128, 200, 5, ctypes.byref(n)) == 0
+    assert n.value > small and n.value % 256 == 0
+    # one layer's fp64 dequantized K and V at 2 and 4 bits dominate the size
+    assert n.value >= 4 * 2 * 2 * 200 * 128 * 8
+    assert L.kvq_tag_distortion_workspace_bytes(1, 2, 8, 2, 96, 200, 5, ctypes.byref(n)) == -2   # EUNSUPPORTED
+    assert L.kvq_tag_distortion_workspace_bytes(1, 2, 7, 2, 128, 200, 5, ctypes.byref(n)) == -1  # Hq % Hkv
+    tags = np.zeros((1, 4), np.int32)
+    D2, D4, cnt = np.zeros(2), np.zeros(2), np.zeros(2, np.int64)
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    fake = 1 << 20                      # 256-byte aligned, never dereferenced
+    args = lambda q, ws, nbytes, t: (1, 1, 2, 1, 64, 4, q, fake, fake, p(t), 2, ws, nbytes, p(D2), p(D4), p(cnt), None)
+    f = L.kvq_tag_distortion_device
+    assert f(*args(None, fake, 1 << 30, tags)) == -1          # null Q
+    assert f(*args(fake + 8, fake, 1 << 30, tags)) == -5      # EALIGN
+    assert f(*args(fake, None, 1 << 30, tags)) == -4          # no workspace: EUNBOUND
+    assert f(*args(fake, fake, 256, tags)) == -4              # workspace too small
+    assert f(*args(fake, fake + 16, 1 << 30, tags)) == -4     # workspace not 256-byte aligned
+    assert f(*args(fake, fake, 1 << 30, np.full((1, 4), 2, np.int32))) == -1   # tag out of range
