@@ -17,6 +17,9 @@
 //     numerator N_i with weights exp(s - m_i)); then, per (tag, b), only the terms of the
 //     tag's tokens change: O'_i = (N_i + dN_i) / (l_i + dl_i), dN and dl summed over
 //     those tokens with the same m_i.  The CTA writes its sum of squared differences.
+//     Its 16-token tiles of fp64 rows (exact and quantized) come by cp.async into two
+//     buffers, the next tile of the CTA's whole sequence of passes in flight while the
+//     current one is used.
 // Then calib_reduce_kernel takes the per-head means, the max over heads, the mean over
 // requests and the sum over layers, in a fixed order.
 #include <cuda_fp16.h>
@@ -44,7 +47,7 @@ struct CalibDims {
 
 // Workspace regions (byte offsets, 256-byte aligned).
 struct CalibLayout {
-    size_t list, off, tags, rank, gstart, ngroups, kq2, vq2, kq4, vq4, part, res, total;
+    size_t list, off, tags, rank, gstart, ngroups, kx, vx, kq2, vq2, kq4, vq4, part, res, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -65,6 +68,8 @@ CalibLayout calib_layout(const CalibDims &d) {
     L.gstart = take(static_cast<size_t>(d.R) * d.maxg * 4);          // list index of each 2-bit key group
     L.ngroups = take(static_cast<size_t>(d.R) * 4);
     const size_t arr = static_cast<size_t>(d.R) * d.Hkv * d.T * d.D * sizeof(double);   // one layer
+    L.kx = take(arr);   // exact keys and values in fp64
+    L.vx = take(arr);
     L.kq2 = take(arr);
     L.vq2 = take(arr);
     L.kq4 = take(arr);
@@ -109,11 +114,12 @@ __device__ __forceinline__ void load32(const uint16_t *src, float (&x)[32]) {
     }
 }
 
-// Thread = (token t, 32-channel group g) of one (request, kv head) of layer `lay`.
+// Thread = (token t, 32-channel group g) of one (request, kv head) of layer `lay`; it also
+// writes the exact keys and values in fp64, the form the attention kernel stages.
 __global__ void calib_token_kernel(const uint16_t *__restrict__ K, const uint16_t *__restrict__ V, int lay,
                                    CalibDims d, const int *__restrict__ tags, const int *__restrict__ rank,
-                                   const int *__restrict__ off, double *kq2, double *vq2, double *kq4,
-                                   double *vq4) {
+                                   const int *__restrict__ off, double *kx, double *vx, double *kq2, double *vq2,
+                                   double *kq4, double *vq4) {
     const int nj = d.D / 32;
     const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= static_cast<long long>(d.T) * nj) return;
@@ -126,6 +132,11 @@ __global__ void calib_token_kernel(const uint16_t *__restrict__ K, const uint16_
     double o[32];
     load32(K + src, xk);
     load32(V + src, xv);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        kx[dst + i] = static_cast<double>(xk[i]);
+        vx[dst + i] = static_cast<double>(xv[i]);
+    }
     const int k = tags[static_cast<long long>(r) * d.T + t];
     const int n = off[r * (d.ntags + 1) + k + 1] - off[r * (d.ntags + 1) + k];
     const bool leftover = rank[static_cast<long long>(r) * d.T + t] >= n / 32 * 32;
@@ -168,43 +179,19 @@ __global__ void calib_keygroup_kernel(const uint16_t *__restrict__ K, int lay, C
 
 template <int D>
 struct CalibSmem {
-    double q[kQB][D + 2];                         // rows padded: 16-byte aligned, bank-spread
-    double k[kKT][D + 2], v[kKT][D + 2];          // exact rows of the tile
-    double kh[kKT][D + 2], vh[kKT][D + 2];        // quantized rows of the tile (tag passes)
-    double pe[kQB][kKT + 2], pq[kQB][kKT + 2];    // exact / quantized weights exp(s - m_i)
+    double q[kQB][D + 2];                  // rows padded: 16-byte aligned, bank-spread
+    double t[2][4][kKT][D + 2];            // two tile buffers: exact k, exact v, quantized k, quantized v
+    double pe[kQB][kKT + 2], pq[kQB][kKT + 2];   // exact / quantized weights exp(s - m_i)
     double red[kThreads / 32];
-    int tok[kKT];
+    int tok[2][kKT];                       // token of each tile row (-1: none)
 };
 
-// Stage tile rows (8-element chunks): row `row` holds token tok (-1: zeros).
-template <int D>
-__device__ __forceinline__ void stage_bf16(double (*dst)[D + 2], const uint16_t *base, int row, int chunk, int tok) {
-    double2 *o = reinterpret_cast<double2 *>(&dst[row][8 * chunk]);
-    if (tok < 0) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) o[j] = make_double2(0.0, 0.0);
-        return;
-    }
-    const uint4 u = *reinterpret_cast<const uint4 *>(base + static_cast<long long>(tok) * D + 8 * chunk);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-        o[j] = make_double2(static_cast<double>(__uint_as_float(w[j] << 16)),
-                            static_cast<double>(__uint_as_float(w[j] & 0xffff0000u)));
+__device__ __forceinline__ void cp16(void *smem, const void *gmem) {
+    const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem) : "memory");
 }
-
-template <int D>
-__device__ __forceinline__ void stage_f64(double (*dst)[D + 2], const double *base, int row, int chunk, int tok) {
-    double2 *o = reinterpret_cast<double2 *>(&dst[row][8 * chunk]);
-    if (tok < 0) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) o[j] = make_double2(0.0, 0.0);
-        return;
-    }
-    const double2 *s = reinterpret_cast<const double2 *>(base + static_cast<long long>(tok) * D + 8 * chunk);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) o[j] = s[j];
-}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_prev() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
 // Dot products of query row qi with tile rows kp and kp + 8, in channel order.
 template <int D>
@@ -238,14 +225,23 @@ __device__ __forceinline__ double max8(double x) {
     return x;
 }
 
+// Where a CTA is in its sequence of 16-token tiles: pass 0 (row max over tokens 0..i_max),
+// pass 1 (l and N over the same tiles), then pass 2 for every (tag with a token <= i_max,
+// b): the tag's tokens in list order.
+struct TilePos {
+    int ph, k, bi, ti, nt;   // pass, tag, bit index (0: 2 bits, 1: 4 bits), tile, tiles in the pass
+};
+
 // CTA = (query block qb, query head hq, request r) of layer `lay`.  Thread t: query row
 // qi = t / 8 of the block; as a scorer it takes tile rows sub and sub + 8 (sub = t % 8),
-// as an accumulator the channels 16m + 2 sub + {0, 1}.
+// as an accumulator the channels 16m + 2 sub + {0, 1}.  Tiles are fp64 rows copied by
+// cp.async into two buffers: the next tile (of any pass) is in flight while the current
+// one is used.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    calib_attn_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K, const uint16_t *__restrict__ V,
-                      int lay, CalibDims d, double rs, const int *__restrict__ list, const int *__restrict__ off,
-                      const double *kq2, const double *vq2, const double *kq4, const double *vq4, double *part) {
+    calib_attn_kernel(const uint16_t *__restrict__ Q, int lay, CalibDims d, double rs, const int *__restrict__ list,
+                      const int *__restrict__ off, const double *kx, const double *vx, const double *kq2,
+                      const double *vq2, const double *kq4, const double *vq4, double *part) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     CalibSmem<D> &sm = *reinterpret_cast<CalibSmem<D> *>(smem_raw);
     constexpr int NM = D / 16;   // channel pairs per accumulating thread
@@ -256,147 +252,197 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i_max = min(i0 + kQB, d.T) - 1;
     const bool valid_q = i < d.T;
     const uint16_t *qbase = Q + ((static_cast<long long>(lay) * d.R + r) * d.Hq + hq) * d.T * D;
-    const long long kvo = ((static_cast<long long>(lay) * d.R + r) * d.Hkv + h) * d.T * D;
-    const uint16_t *kbase = K + kvo, *vbase = V + kvo;
-    const long long qo = (static_cast<long long>(r) * d.Hkv + h) * d.T * D;   // quantized arrays (one layer)
-
-    for (int e = tid; e < kQB * D / 8; e += kThreads) {
-        const int row = e / (D / 8), chunk = e % (D / 8);
-        stage_bf16<D>(sm.q, qbase, row, chunk, i0 + row < d.T ? i0 + row : -1);
-    }
-
-    // exact pass 1: the row max of the scores s_ij = (q_i . k_j) rs, j <= i
-    double m = -INFINITY;
-    for (int j0 = 0; j0 <= i_max; j0 += kKT) {
-        __syncthreads();
-        for (int e = tid; e < kKT * D / 8; e += kThreads) {
-            const int row = e / (D / 8), chunk = e % (D / 8);
-            stage_bf16<D>(sm.k, kbase, row, chunk, j0 + row <= i_max ? j0 + row : -1);
-        }
-        __syncthreads();
-        double s0, s1;
-        dot2<D>(sm.q, sm.k, qi, sub, s0, s1);
-        if (valid_q && j0 + sub <= i) m = fmax(m, s0 * rs);
-        if (valid_q && j0 + sub + 8 <= i) m = fmax(m, s1 * rs);
-    }
-    m = max8(m);
-
-    // exact pass 2: l_i = sum_j exp(s_ij - m_i), N_i = sum_j exp(s_ij - m_i) v_j
-    double2 N[NM];
-#pragma unroll
-    for (int mm = 0; mm < NM; ++mm) N[mm] = make_double2(0.0, 0.0);
-    double l = 0.0;
-    for (int j0 = 0; j0 <= i_max; j0 += kKT) {
-        __syncthreads();
-        for (int e = tid; e < kKT * D / 8; e += kThreads) {
-            const int row = e / (D / 8), chunk = e % (D / 8);
-            const int tok = j0 + row <= i_max ? j0 + row : -1;
-            stage_bf16<D>(sm.k, kbase, row, chunk, tok);
-            stage_bf16<D>(sm.v, vbase, row, chunk, tok);
-        }
-        __syncthreads();
-        double s0, s1;
-        dot2<D>(sm.q, sm.k, qi, sub, s0, s1);
-        const double p0 = valid_q && j0 + sub <= i ? exp(s0 * rs - m) : 0.0;
-        const double p1 = valid_q && j0 + sub + 8 <= i ? exp(s1 * rs - m) : 0.0;
-        sm.pe[qi][sub] = p0;
-        sm.pe[qi][sub + 8] = p1;
-        l += p0;
-        l += p1;
-        __syncthreads();
-#pragma unroll 4
-        for (int kk = 0; kk < kKT; ++kk) {
-            const double p = sm.pe[qi][kk];
-#pragma unroll
-            for (int mm = 0; mm < NM; ++mm) {
-                const double2 vv = *reinterpret_cast<const double2 *>(&sm.v[kk][16 * mm + 2 * sub]);
-                N[mm].x = fma(p, vv.x, N[mm].x);
-                N[mm].y = fma(p, vv.y, N[mm].y);
-            }
-        }
-    }
-    l = sum8(l);
-
-    // per (tag, b): the tag's tokens j <= i at b bits.  dN = A - B with A = sum pq vh and
-    // B = sum pe v kept apart, so a tag whose tokens quantize exactly gives 0 exactly.
+    const long long uo = (static_cast<long long>(r) * d.Hkv + h) * d.T * D;   // (request, kv head) in one layer
+    const double *kxp = kx + uo, *vxp = vx + uo;
     const int *offr = off + r * (d.ntags + 1);
     const int *listr = list + static_cast<long long>(r) * d.T;
-    for (int k = 0; k < d.ntags; ++k) {
-        const int a = offr[k], n = offr[k + 1] - a;
-        for (int bi = 0; bi < 2; ++bi) {
-            const double *kq = (bi == 0 ? kq2 : kq4) + qo;
-            const double *vq = (bi == 0 ? vq2 : vq4) + qo;
-            double2 A[NM], B[NM];
+    const int nt_exact = i_max / kKT + 1;
+
+    // tiles of tag k: its list entries <= i_max (the list is in token order)
+    auto tag_tiles = [&](int k) {
+        const int a = offr[k];
+        int lo = 0, hi = offr[k + 1] - a;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (listr[a + mid] <= i_max)
+                lo = mid + 1;
+            else
+                hi = mid;
+        }
+        return (lo + kKT - 1) / kKT;
+    };
+    auto advance = [&](TilePos &p) {   // false past the last tile
+        if (++p.ti < p.nt) return true;
+        p.ti = 0;
+        if (p.ph == 0) {
+            p.ph = 1;
+            return true;
+        }
+        if (p.ph == 1) {
+            p.ph = 2;
+            p.k = 0;
+            p.bi = 0;
+        } else if (p.bi == 0) {
+            p.bi = 1;
+            return true;
+        } else {
+            ++p.k;
+            p.bi = 0;
+        }
+        while (p.k < d.ntags && (p.nt = tag_tiles(p.k)) == 0) ++p.k;
+        return p.k < d.ntags;
+    };
+    // copies of the tile at p into buffer buf (rows without a token are zeroed), one group
+    auto issue = [&](int buf, const TilePos &p) {
+        const int narr = p.ph == 0 ? 1 : (p.ph == 1 ? 2 : 4);
+        const int a = p.ph == 2 ? offr[p.k] : 0;
+        const int n = p.ph == 2 ? offr[p.k + 1] - a : 0;
+        const int first = p.ti * kKT;
+        const double *kqp = (p.bi ? kq4 : kq2) + uo, *vqp = (p.bi ? vq4 : vq2) + uo;
+        for (int e = tid; e < kKT * (D / 2); e += kThreads) {
+            const int row = e / (D / 2), ch = e % (D / 2);
+            const int tok = p.ph == 2 ? (first + row < n ? listr[a + first + row] : -1)
+                                      : (first + row <= i_max ? first + row : -1);
+            if (ch == 0) sm.tok[buf][row] = tok;
 #pragma unroll
-            for (int mm = 0; mm < NM; ++mm) {
-                A[mm] = make_double2(0.0, 0.0);
-                B[mm] = make_double2(0.0, 0.0);
-            }
-            double dl = 0.0;
-            for (int s0i = 0; s0i < n && listr[a + s0i] <= i_max; s0i += kKT) {
-                __syncthreads();
-                for (int e = tid; e < kKT * D / 8; e += kThreads) {
-                    const int row = e / (D / 8), chunk = e % (D / 8);
-                    const int tok = s0i + row < n ? listr[a + s0i + row] : -1;
-                    if (chunk == 0) sm.tok[row] = tok;
-                    stage_bf16<D>(sm.k, kbase, row, chunk, tok);
-                    stage_bf16<D>(sm.v, vbase, row, chunk, tok);
-                    stage_f64<D>(sm.kh, kq, row, chunk, tok);
-                    stage_f64<D>(sm.vh, vq, row, chunk, tok);
-                }
-                __syncthreads();
-                double se0, se1, sq0, sq1;
-                dot2<D>(sm.q, sm.k, qi, sub, se0, se1);
-                dot2<D>(sm.q, sm.kh, qi, sub, sq0, sq1);
-                const int t0 = sm.tok[sub], t1 = sm.tok[sub + 8];
-                const bool v0 = valid_q && t0 >= 0 && t0 <= i, v1 = valid_q && t1 >= 0 && t1 <= i;
-                const double pe0 = v0 ? exp(se0 * rs - m) : 0.0, pq0 = v0 ? exp(sq0 * rs - m) : 0.0;
-                const double pe1 = v1 ? exp(se1 * rs - m) : 0.0, pq1 = v1 ? exp(sq1 * rs - m) : 0.0;
-                sm.pe[qi][sub] = pe0;
-                sm.pq[qi][sub] = pq0;
-                sm.pe[qi][sub + 8] = pe1;
-                sm.pq[qi][sub + 8] = pq1;
-                dl += pq0 - pe0;
-                dl += pq1 - pe1;
-                __syncthreads();
-#pragma unroll 2
-                for (int kk = 0; kk < kKT; ++kk) {
-                    const double pe = sm.pe[qi][kk], pq = sm.pq[qi][kk];
-#pragma unroll
-                    for (int mm = 0; mm < NM; ++mm) {
-                        const double2 vh = *reinterpret_cast<const double2 *>(&sm.vh[kk][16 * mm + 2 * sub]);
-                        const double2 vx = *reinterpret_cast<const double2 *>(&sm.v[kk][16 * mm + 2 * sub]);
-                        A[mm].x = fma(pq, vh.x, A[mm].x);
-                        A[mm].y = fma(pq, vh.y, A[mm].y);
-                        B[mm].x = fma(pe, vx.x, B[mm].x);
-                        B[mm].y = fma(pe, vx.y, B[mm].y);
-                    }
-                }
-            }
-            dl = sum8(dl);
-            double err = 0.0;
-            if (valid_q) {
-                const double lq = l + dl;
-#pragma unroll
-                for (int mm = 0; mm < NM; ++mm) {
-                    const double ex = (N[mm].x + (A[mm].x - B[mm].x)) / lq - N[mm].x / l;
-                    const double ey = (N[mm].y + (A[mm].y - B[mm].y)) / lq - N[mm].y / l;
-                    err += ex * ex;
-                    err += ey * ey;
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) err += __shfl_xor_sync(0xffffffffu, err, o);
-            __syncthreads();   // sm.red of the previous (tag, b) has been read
-            if ((tid & 31) == 0) sm.red[tid >> 5] = err;
-            __syncthreads();
-            if (tid == 0) {
-                double s = 0.0;
-                for (int w = 0; w < kThreads / 32; ++w) s += sm.red[w];
-                part[((((static_cast<long long>(lay) * d.R + r) * d.Hq + hq) * d.nqb + qb) * d.ntags + k) * 2 + bi] =
-                    s;
+            for (int x = 0; x < 4; ++x) {
+                if (x >= narr) break;
+                const double *src = x == 0 ? kxp : x == 1 ? vxp : x == 2 ? kqp : vqp;
+                double *dst = &sm.t[buf][x][row][2 * ch];
+                if (tok >= 0)
+                    cp16(dst, src + static_cast<long long>(tok) * D + 2 * ch);
+                else
+                    *reinterpret_cast<double2 *>(dst) = make_double2(0.0, 0.0);
             }
         }
+        cp_commit();
+    };
+
+    TilePos cur{0, 0, 0, 0, nt_exact};
+    issue(0, cur);
+    for (int e = tid; e < kQB * D / 8; e += kThreads) {   // query rows as fp64 (bf16 is exact)
+        const int row = e / (D / 8), chunk = e % (D / 8);
+        double2 *o = reinterpret_cast<double2 *>(&sm.q[row][8 * chunk]);
+        if (i0 + row < d.T) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(qbase + static_cast<long long>(i0 + row) * D + 8 * chunk);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                o[j] = make_double2(static_cast<double>(__uint_as_float(w[j] << 16)),
+                                    static_cast<double>(__uint_as_float(w[j] & 0xffff0000u)));
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[j] = make_double2(0.0, 0.0);
+        }
+    }
+
+    double m = -INFINITY, l = 0.0, dl = 0.0;
+    double2 N[NM], A[NM], B[NM];   // exact numerator; sum pq vh and sum pe v of the current (tag, b)
+#pragma unroll
+    for (int mm = 0; mm < NM; ++mm) N[mm] = make_double2(0.0, 0.0);
+    for (int buf = 0;; buf ^= 1) {
+        TilePos nxt = cur;
+        const bool more = advance(nxt);
+        if (more)
+            issue(buf ^ 1, nxt);
+        else
+            cp_commit();   // an empty group keeps the wait below uniform
+        cp_wait_prev();     // this tile's copies (the group before the newest) have landed
+        __syncthreads();
+        const double(*tk)[D + 2] = sm.t[buf][0];
+        if (cur.ph == 0) {   // row max of s_ij = (q_i . k_j) rs over j <= i
+            const int j0 = cur.ti * kKT;
+            double s0, s1;
+            dot2<D>(sm.q, tk, qi, sub, s0, s1);
+            if (valid_q && j0 + sub <= i) m = fmax(m, s0 * rs);
+            if (valid_q && j0 + sub + 8 <= i) m = fmax(m, s1 * rs);
+            if (cur.ti == cur.nt - 1) m = max8(m);
+        } else if (cur.ph == 1) {   // l_i and N_i with the exact weights exp(s_ij - m_i)
+            const int j0 = cur.ti * kKT;
+            double s0, s1;
+            dot2<D>(sm.q, tk, qi, sub, s0, s1);
+            const double p0 = valid_q && j0 + sub <= i ? exp(s0 * rs - m) : 0.0;
+            const double p1 = valid_q && j0 + sub + 8 <= i ? exp(s1 * rs - m) : 0.0;
+            sm.pe[qi][sub] = p0;
+            sm.pe[qi][sub + 8] = p1;
+            l += p0;
+            l += p1;
+            __syncthreads();
+#pragma unroll 4
+            for (int kk = 0; kk < kKT; ++kk) {
+                const double p = sm.pe[qi][kk];
+#pragma unroll
+                for (int mm = 0; mm < NM; ++mm) {
+                    const double2 vv = *reinterpret_cast<const double2 *>(&sm.t[buf][1][kk][16 * mm + 2 * sub]);
+                    N[mm].x = fma(p, vv.x, N[mm].x);
+                    N[mm].y = fma(p, vv.y, N[mm].y);
+                }
+            }
+            if (cur.ti == cur.nt - 1) l = sum8(l);
+        } else {   // the tag's tokens j <= i at b bits; A and B apart, so exact levels give 0 exactly
+            if (cur.ti == 0) {
+#pragma unroll
+                for (int mm = 0; mm < NM; ++mm) {
+                    A[mm] = make_double2(0.0, 0.0);
+                    B[mm] = make_double2(0.0, 0.0);
+                }
+                dl = 0.0;
+            }
+            double se0, se1, sq0, sq1;
+            dot2<D>(sm.q, tk, qi, sub, se0, se1);
+            dot2<D>(sm.q, sm.t[buf][2], qi, sub, sq0, sq1);
+            const int t0 = sm.tok[buf][sub], t1 = sm.tok[buf][sub + 8];
+            const bool v0 = valid_q && t0 >= 0 && t0 <= i, v1 = valid_q && t1 >= 0 && t1 <= i;
+            const double pe0 = v0 ? exp(se0 * rs - m) : 0.0, pq0 = v0 ? exp(sq0 * rs - m) : 0.0;
+            const double pe1 = v1 ? exp(se1 * rs - m) : 0.0, pq1 = v1 ? exp(sq1 * rs - m) : 0.0;
+            sm.pe[qi][sub] = pe0;
+            sm.pq[qi][sub] = pq0;
+            sm.pe[qi][sub + 8] = pe1;
+            sm.pq[qi][sub + 8] = pq1;
+            dl += pq0 - pe0;
+            dl += pq1 - pe1;
+            __syncthreads();
+#pragma unroll 2
+            for (int kk = 0; kk < kKT; ++kk) {
+                const double pe = sm.pe[qi][kk], pq = sm.pq[qi][kk];
+#pragma unroll
+                for (int mm = 0; mm < NM; ++mm) {
+                    const double2 vx2 = *reinterpret_cast<const double2 *>(&sm.t[buf][1][kk][16 * mm + 2 * sub]);
+                    const double2 vh = *reinterpret_cast<const double2 *>(&sm.t[buf][3][kk][16 * mm + 2 * sub]);
+                    A[mm].x = fma(pq, vh.x, A[mm].x);
+                    A[mm].y = fma(pq, vh.y, A[mm].y);
+                    B[mm].x = fma(pe, vx2.x, B[mm].x);
+                    B[mm].y = fma(pe, vx2.y, B[mm].y);
+                }
+            }
+            if (cur.ti == cur.nt - 1) {   // the pass's squared output differences, summed over the CTA
+                const double dls = sum8(dl);
+                double err = 0.0;
+                if (valid_q) {
+                    const double lq = l + dls;
+#pragma unroll
+                    for (int mm = 0; mm < NM; ++mm) {
+                        const double ex = (N[mm].x + (A[mm].x - B[mm].x)) / lq - N[mm].x / l;
+                        const double ey = (N[mm].y + (A[mm].y - B[mm].y)) / lq - N[mm].y / l;
+                        err += ex * ex;
+                        err += ey * ey;
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) err += __shfl_xor_sync(0xffffffffu, err, o);
+                if ((tid & 31) == 0) sm.red[tid >> 5] = err;
+                __syncthreads();
+                if (tid == 0) {
+                    double s = 0.0;
+                    for (int w = 0; w < kThreads / 32; ++w) s += sm.red[w];
+                    part[((((static_cast<long long>(lay) * d.R + r) * d.Hq + hq) * d.nqb + qb) * d.ntags + cur.k) * 2 +
+                         cur.bi] = s;
+                }
+            }
+        }
+        __syncthreads();   // this buffer (and sm.pe, sm.red) is free again
+        if (!more) break;
+        cur = nxt;
     }
 }
 
@@ -439,14 +485,14 @@ int check_dims(int NL, int R, int Hq, int Hkv, int D, int T, int ntags, CalibDim
 }
 
 template <int D>
-cudaError_t launch_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int lay, const CalibDims &d, double rs,
-                        const int *list, const int *off, const double *kq2, const double *vq2, const double *kq4,
+cudaError_t launch_attn(const uint16_t *Q, int lay, const CalibDims &d, double rs, const int *list, const int *off,
+                        const double *kx, const double *vx, const double *kq2, const double *vq2, const double *kq4,
                         const double *vq4, double *part, cudaStream_t st) {
     const size_t smem = sizeof(CalibSmem<D>);
     cudaError_t e = cudaFuncSetAttribute(calib_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    calib_attn_kernel<D><<<dim3(d.nqb, d.Hq, d.R), kThreads, smem, st>>>(Q, K, V, lay, d, rs, list, off, kq2, vq2,
+    calib_attn_kernel<D><<<dim3(d.nqb, d.Hq, d.R), kThreads, smem, st>>>(Q, lay, d, rs, list, off, kx, vx, kq2, vq2,
                                                                          kq4, vq4, part);
     return cudaGetLastError();
 }
@@ -515,6 +561,7 @@ int kvq_tag_distortion_device(int num_layers, int num_requests, int n_q_heads, i
     int *d_list = reinterpret_cast<int *>(ws + L.list), *d_off = reinterpret_cast<int *>(ws + L.off);
     int *d_tags = reinterpret_cast<int *>(ws + L.tags), *d_rank = reinterpret_cast<int *>(ws + L.rank);
     int *d_gstart = reinterpret_cast<int *>(ws + L.gstart), *d_ng = reinterpret_cast<int *>(ws + L.ngroups);
+    double *kx = reinterpret_cast<double *>(ws + L.kx), *vx = reinterpret_cast<double *>(ws + L.vx);
     double *kq2 = reinterpret_cast<double *>(ws + L.kq2), *vq2 = reinterpret_cast<double *>(ws + L.vq2);
     double *kq4 = reinterpret_cast<double *>(ws + L.kq4), *vq4 = reinterpret_cast<double *>(ws + L.vq4);
     double *part = reinterpret_cast<double *>(ws + L.part), *res = reinterpret_cast<double *>(ws + L.res);
@@ -534,19 +581,21 @@ int kvq_tag_distortion_device(int num_layers, int num_requests, int n_q_heads, i
 
     const uint16_t *q16 = static_cast<const uint16_t *>(Q), *k16 = static_cast<const uint16_t *>(K),
                    *v16 = static_cast<const uint16_t *>(V);
+    // a CTA writes only the (tag, b) sums of tags with a token at or before its last query
+    if ((e = cudaMemsetAsync(part, 0, L.res - L.part, st)) != cudaSuccess) return fail_cuda(e);
     const double rs = 1.0 / std::sqrt(static_cast<double>(d.D));
     const long long tok_threads = static_cast<long long>(T) * (d.D / 32);
     for (int lay = 0; lay < d.NL; ++lay) {
         calib_token_kernel<<<dim3(static_cast<unsigned>((tok_threads + 255) / 256), R * d.Hkv), 256, 0, st>>>(
-            k16, v16, lay, d, d_tags, d_rank, d_off, kq2, vq2, kq4, vq4);
+            k16, v16, lay, d, d_tags, d_rank, d_off, kx, vx, kq2, vq2, kq4, vq4);
         if ((e = cudaGetLastError()) != cudaSuccess) return fail_cuda(e);
         if (maxg_used > 0) {
             calib_keygroup_kernel<<<dim3(maxg_used, R * d.Hkv), d.D, 0, st>>>(k16, lay, d, d_list, d_gstart, d_ng,
                                                                                kq2);
             if ((e = cudaGetLastError()) != cudaSuccess) return fail_cuda(e);
         }
-        e = d.D == 128 ? launch_attn<128>(q16, k16, v16, lay, d, rs, d_list, d_off, kq2, vq2, kq4, vq4, part, st)
-                       : launch_attn<64>(q16, k16, v16, lay, d, rs, d_list, d_off, kq2, vq2, kq4, vq4, part, st);
+        e = d.D == 128 ? launch_attn<128>(q16, lay, d, rs, d_list, d_off, kx, vx, kq2, vq2, kq4, vq4, part, st)
+                       : launch_attn<64>(q16, lay, d, rs, d_list, d_off, kx, vx, kq2, vq2, kq4, vq4, part, st);
         if (e != cudaSuccess) return fail_cuda(e);
     }
     calib_reduce_kernel<<<1, 128, 0, st>>>(part, d, res);
