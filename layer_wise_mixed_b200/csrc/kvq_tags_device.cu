@@ -193,22 +193,52 @@ __device__ __forceinline__ void cp16(void *smem, const void *gmem) {
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_wait_prev() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
-// Dot products of query row qi with tile rows kp and kp + 8, in channel order.
+// Dot products of query row qi with tile rows kp and kp + 8: the even and the odd
+// channels in two chains each (channel order within a chain), then added.
 template <int D>
 __device__ __forceinline__ void dot2(const double (*q)[D + 2], const double (*k)[D + 2], int qi, int kp, double &s0,
                                      double &s1) {
-    s0 = 0.0;
-    s1 = 0.0;
+    double e0 = 0.0, o0 = 0.0, e1 = 0.0, o1 = 0.0;
 #pragma unroll 8
     for (int c = 0; c < D; c += 2) {
         const double2 a = *reinterpret_cast<const double2 *>(&q[qi][c]);
         const double2 b0 = *reinterpret_cast<const double2 *>(&k[kp][c]);
         const double2 b1 = *reinterpret_cast<const double2 *>(&k[kp + 8][c]);
-        s0 = fma(a.x, b0.x, s0);
-        s0 = fma(a.y, b0.y, s0);
-        s1 = fma(a.x, b1.x, s1);
-        s1 = fma(a.y, b1.y, s1);
+        e0 = fma(a.x, b0.x, e0);
+        o0 = fma(a.y, b0.y, o0);
+        e1 = fma(a.x, b1.x, e1);
+        o1 = fma(a.y, b1.y, o1);
     }
+    s0 = e0 + o0;
+    s1 = e1 + o1;
+}
+
+// dot2 against the exact rows k and the quantized rows kh at once (one query load per
+// channel pair); each product is summed exactly as dot2 sums it.
+template <int D>
+__device__ __forceinline__ void dot4(const double (*q)[D + 2], const double (*k)[D + 2], const double (*kh)[D + 2],
+                                     int qi, int kp, double &se0, double &se1, double &sq0, double &sq1) {
+    double e0 = 0.0, o0 = 0.0, e1 = 0.0, o1 = 0.0, f0 = 0.0, p0 = 0.0, f1 = 0.0, p1 = 0.0;
+#pragma unroll 4
+    for (int c = 0; c < D; c += 2) {
+        const double2 a = *reinterpret_cast<const double2 *>(&q[qi][c]);
+        const double2 b0 = *reinterpret_cast<const double2 *>(&k[kp][c]);
+        const double2 b1 = *reinterpret_cast<const double2 *>(&k[kp + 8][c]);
+        const double2 h0 = *reinterpret_cast<const double2 *>(&kh[kp][c]);
+        const double2 h1 = *reinterpret_cast<const double2 *>(&kh[kp + 8][c]);
+        e0 = fma(a.x, b0.x, e0);
+        o0 = fma(a.y, b0.y, o0);
+        e1 = fma(a.x, b1.x, e1);
+        o1 = fma(a.y, b1.y, o1);
+        f0 = fma(a.x, h0.x, f0);
+        p0 = fma(a.y, h0.y, p0);
+        f1 = fma(a.x, h1.x, f1);
+        p1 = fma(a.y, h1.y, p1);
+    }
+    se0 = e0 + o0;
+    se1 = e1 + o1;
+    sq0 = f0 + p0;
+    sq1 = f1 + p1;
 }
 
 __device__ __forceinline__ double sum8(double x) {   // over the 8 lanes of a query row
@@ -389,8 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 dl = 0.0;
             }
             double se0, se1, sq0, sq1;
-            dot2<D>(sm.q, tk, qi, sub, se0, se1);
-            dot2<D>(sm.q, sm.t[buf][2], qi, sub, sq0, sq1);
+            dot4<D>(sm.q, tk, sm.t[buf][2], qi, sub, se0, se1, sq0, sq1);
             const int t0 = sm.tok[buf][sub], t1 = sm.tok[buf][sub + 8];
             const bool v0 = valid_q && t0 >= 0 && t0 <= i, v1 = valid_q && t1 >= 0 && t1 <= i;
             const double pe0 = v0 ? exp(se0 * rs - m) : 0.0, pq0 = v0 ? exp(sq0 * rs - m) : 0.0;
