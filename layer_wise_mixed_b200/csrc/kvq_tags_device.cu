@@ -17,9 +17,9 @@
 //     numerator N_i with weights exp(s - m_i)); then, per (tag, b), only the terms of the
 //     tag's tokens change: O'_i = (N_i + dN_i) / (l_i + dl_i), dN and dl summed over
 //     those tokens with the same m_i.  The CTA writes its sum of squared differences.
-//     Its 16-token tiles of fp64 rows (exact and quantized) come by cp.async into two
-//     buffers, the next tile of the CTA's whole sequence of passes in flight while the
-//     current one is used.
+//     Both products run on the fp64 tensor cores (mma m8n8k4).  Its 16-token tiles of
+//     fp64 rows (exact and quantized) come by cp.async into two buffers, the next tile of
+//     the CTA's whole sequence of passes in flight while the current one is used.
 // Then calib_reduce_kernel takes the per-head means, the max over heads, the mean over
 // requests and the sum over layers, in a fixed order.
 #include <cuda_fp16.h>
@@ -179,9 +179,10 @@ __global__ void calib_keygroup_kernel(const uint16_t *__restrict__ K, int lay, C
 
 template <int D>
 struct CalibSmem {
-    double q[kQB][D + 2];                  // rows padded: 16-byte aligned, bank-spread
-    double t[2][4][kKT][D + 2];            // two tile buffers: exact k, exact v, quantized k, quantized v
-    double pe[kQB][kKT + 2], pq[kQB][kKT + 2];   // exact / quantized weights exp(s - m_i)
+    double q[kQB][D + 4];                  // rows padded: 16-byte aligned, fragment loads conflict-free
+    double t[2][4][kKT][D + 4];            // two tile buffers: exact k, exact v, quantized k, quantized v
+    double pe[kQB][kKT + 4], pq[kQB][kKT + 4];   // exact / quantized weights exp(s - m_i)
+    double mx[2][kQB], ls[2][kQB], dl[2][kQB];   // per key half: row max, sum of weights, sum of pq - pe
     double red[kThreads / 32];
     int tok[2][kKT];                       // token of each tile row (-1: none)
 };
@@ -193,66 +194,31 @@ __device__ __forceinline__ void cp16(void *smem, const void *gmem) {
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_wait_prev() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
-// Dot products of query row qi with tile rows kp and kp + 8: the even and the odd
-// channels in two chains each (channel order within a chain), then added.
-template <int D>
-__device__ __forceinline__ void dot2(const double (*q)[D + 2], const double (*k)[D + 2], int qi, int kp, double &s0,
-                                     double &s1) {
-    double e0 = 0.0, o0 = 0.0, e1 = 0.0, o1 = 0.0;
+// d += a b on the fp64 tensor cores: an 8 x 8 x 4 product per warp.  Lane l holds
+// a = A[l/4][l%4], b = B[l%4][l/4] and d = D[l/4][2(l%4)], D[l/4][2(l%4) + 1].
+__device__ __forceinline__ void dmma(double &d0, double &d1, double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};\n"
+                 : "+d"(d0), "+d"(d1)
+                 : "d"(a), "d"(b));
+}
+
+// Scores of query tile mt (rows 8mt..8mt+7) against key tile nt of rows k and of rows kh
+// (the exact and the quantized keys, one query fragment for both), channel order in
+// steps of 4: lane l gets the keys 8nt + 2(l%4) + {0, 1} of query 8mt + l/4.
+template <int D, bool TWO>
+__device__ __forceinline__ void score_tile(const double (*q)[D + 4], const double (*k)[D + 4],
+                                           const double (*kh)[D + 4], int mt, int nt, int lane, double (&se)[2],
+                                           double (&sq)[2]) {
+    se[0] = se[1] = sq[0] = sq[1] = 0.0;
+    const double *qa = &q[8 * mt + (lane >> 2)][lane & 3];
+    const double *kb = &k[8 * nt + (lane >> 2)][lane & 3];
+    const double *hb = &kh[8 * nt + (lane >> 2)][lane & 3];
 #pragma unroll 8
-    for (int c = 0; c < D; c += 2) {
-        const double2 a = *reinterpret_cast<const double2 *>(&q[qi][c]);
-        const double2 b0 = *reinterpret_cast<const double2 *>(&k[kp][c]);
-        const double2 b1 = *reinterpret_cast<const double2 *>(&k[kp + 8][c]);
-        e0 = fma(a.x, b0.x, e0);
-        o0 = fma(a.y, b0.y, o0);
-        e1 = fma(a.x, b1.x, e1);
-        o1 = fma(a.y, b1.y, o1);
+    for (int c = 0; c < D; c += 4) {
+        const double a = qa[c];
+        dmma(se[0], se[1], a, kb[c]);
+        if (TWO) dmma(sq[0], sq[1], a, hb[c]);
     }
-    s0 = e0 + o0;
-    s1 = e1 + o1;
-}
-
-// dot2 against the exact rows k and the quantized rows kh at once (one query load per
-// channel pair); each product is summed exactly as dot2 sums it.
-template <int D>
-__device__ __forceinline__ void dot4(const double (*q)[D + 2], const double (*k)[D + 2], const double (*kh)[D + 2],
-                                     int qi, int kp, double &se0, double &se1, double &sq0, double &sq1) {
-    double e0 = 0.0, o0 = 0.0, e1 = 0.0, o1 = 0.0, f0 = 0.0, p0 = 0.0, f1 = 0.0, p1 = 0.0;
-#pragma unroll 4
-    for (int c = 0; c < D; c += 2) {
-        const double2 a = *reinterpret_cast<const double2 *>(&q[qi][c]);
-        const double2 b0 = *reinterpret_cast<const double2 *>(&k[kp][c]);
-        const double2 b1 = *reinterpret_cast<const double2 *>(&k[kp + 8][c]);
-        const double2 h0 = *reinterpret_cast<const double2 *>(&kh[kp][c]);
-        const double2 h1 = *reinterpret_cast<const double2 *>(&kh[kp + 8][c]);
-        e0 = fma(a.x, b0.x, e0);
-        o0 = fma(a.y, b0.y, o0);
-        e1 = fma(a.x, b1.x, e1);
-        o1 = fma(a.y, b1.y, o1);
-        f0 = fma(a.x, h0.x, f0);
-        p0 = fma(a.y, h0.y, p0);
-        f1 = fma(a.x, h1.x, f1);
-        p1 = fma(a.y, h1.y, p1);
-    }
-    se0 = e0 + o0;
-    se1 = e1 + o1;
-    sq0 = f0 + p0;
-    sq1 = f1 + p1;
-}
-
-__device__ __forceinline__ double sum8(double x) {   // over the 8 lanes of a query row
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    x += __shfl_xor_sync(0xffffffffu, x, 2);
-    x += __shfl_xor_sync(0xffffffffu, x, 4);
-    return x;
-}
-
-__device__ __forceinline__ double max8(double x) {
-    x = fmax(x, __shfl_xor_sync(0xffffffffu, x, 1));
-    x = fmax(x, __shfl_xor_sync(0xffffffffu, x, 2));
-    x = fmax(x, __shfl_xor_sync(0xffffffffu, x, 4));
-    return x;
 }
 
 // Where a CTA is in its sequence of 16-token tiles: pass 0 (row max over tokens 0..i_max),
@@ -262,11 +228,12 @@ struct TilePos {
     int ph, k, bi, ti, nt;   // pass, tag, bit index (0: 2 bits, 1: 4 bits), tile, tiles in the pass
 };
 
-// CTA = (query block qb, query head hq, request r) of layer `lay`.  Thread t: query row
-// qi = t / 8 of the block; as a scorer it takes tile rows sub and sub + 8 (sub = t % 8),
-// as an accumulator the channels 16m + 2 sub + {0, 1}.  Tiles are fp64 rows copied by
-// cp.async into two buffers: the next tile (of any pass) is in flight while the current
-// one is used.
+// CTA = (query block qb, query head hq, request r) of layer `lay`: 8 warps, both products
+// on the fp64 tensor cores (mma m8n8k4).  Scores: warp w takes query tile mt = w % 4
+// (8 queries) and key tile w / 4 (8 of the tile's 16 keys).  Weighted values: warp w takes
+// output channels [8 NTW w, 8 NTW (w + 1)) of all 32 queries.  Tiles are fp64 rows copied
+// by cp.async into two buffers: the next tile (of any pass) is in flight while the
+// current one is used.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     calib_attn_kernel(const uint16_t *__restrict__ Q, int lay, CalibDims d, double rs, const int *__restrict__ list,
@@ -274,11 +241,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const double *vq2, const double *kq4, const double *vq4, double *part) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     CalibSmem<D> &sm = *reinterpret_cast<CalibSmem<D> *>(smem_raw);
-    constexpr int NM = D / 16;   // channel pairs per accumulating thread
-    const int tid = threadIdx.x, qi = tid >> 3, sub = tid & 7;
+    constexpr int NTW = D / 64;   // 8-channel output tiles per warp
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int mt = w & 3, nt = w >> 2;            // score tile of this warp
+    const int sq_row = 8 * mt + (lane >> 2);     // its query row in the block
+    const int key0 = 8 * nt + 2 * (lane & 3);    // its first key in the tile
     const int qb = d.nqb - 1 - static_cast<int>(blockIdx.x);   // longest rows first
     const int hq = blockIdx.y, r = blockIdx.z, h = hq / (d.Hq / d.Hkv);
-    const int i0 = qb * kQB, i = i0 + qi;
+    const int i0 = qb * kQB, i = i0 + sq_row;
     const int i_max = min(i0 + kQB, d.T) - 1;
     const bool valid_q = i < d.T;
     const uint16_t *qbase = Q + ((static_cast<long long>(lay) * d.R + r) * d.Hq + hq) * d.T * D;
@@ -355,21 +325,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         double2 *o = reinterpret_cast<double2 *>(&sm.q[row][8 * chunk]);
         if (i0 + row < d.T) {
             const uint4 u = *reinterpret_cast<const uint4 *>(qbase + static_cast<long long>(i0 + row) * D + 8 * chunk);
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                o[j] = make_double2(static_cast<double>(__uint_as_float(w[j] << 16)),
-                                    static_cast<double>(__uint_as_float(w[j] & 0xffff0000u)));
+                o[j] = make_double2(static_cast<double>(__uint_as_float(wd[j] << 16)),
+                                    static_cast<double>(__uint_as_float(wd[j] & 0xffff0000u)));
         } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j) o[j] = make_double2(0.0, 0.0);
         }
     }
 
-    double m = -INFINITY, l = 0.0, dl = 0.0;
-    double2 N[NM], A[NM], B[NM];   // exact numerator; sum pq vh and sum pe v of the current (tag, b)
+    // score side (query sq_row, keys key0, key0 + 1): row max, weight sums; value side
+    // (queries 8 m + lane / 4, channels 8 (NTW w + j) + 2 (lane % 4) + {0, 1}): N, A, B
+    double m = -INFINITY, lp = 0.0, dlp = 0.0;
+    double N[4][NTW][2], A[4][NTW][2], B[4][NTW][2];
 #pragma unroll
-    for (int mm = 0; mm < NM; ++mm) N[mm] = make_double2(0.0, 0.0);
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int j = 0; j < NTW; ++j) N[a][j][0] = N[a][j][1] = 0.0;
+
+    // weighted values of the tile: acc (+)= P V over its 16 keys, 4 per step
+    auto pv = [&](const double (*P)[kKT + 4], const double (*V)[D + 4], double (&acc)[4][NTW][2]) {
+#pragma unroll
+        for (int k4 = 0; k4 < kKT; k4 += 4) {
+            double a[4], b[NTW];
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm) a[mm] = P[8 * mm + (lane >> 2)][k4 + (lane & 3)];
+#pragma unroll
+            for (int j = 0; j < NTW; ++j) b[j] = V[k4 + (lane & 3)][8 * (NTW * w + j) + (lane >> 2)];
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm)
+#pragma unroll
+                for (int j = 0; j < NTW; ++j) dmma(acc[mm][j][0], acc[mm][j][1], a[mm], b[j]);
+        }
+    };
+
     for (int buf = 0;; buf ^= 1) {
         TilePos nxt = cur;
         const bool more = advance(nxt);
@@ -379,97 +370,92 @@ __global__ void __launch_bounds__(kThreads, 1)
             cp_commit();   // an empty group keeps the wait below uniform
         cp_wait_prev();     // this tile's copies (the group before the newest) have landed
         __syncthreads();
-        const double(*tk)[D + 2] = sm.t[buf][0];
+        const double(*tk)[D + 4] = sm.t[buf][0];
         if (cur.ph == 0) {   // row max of s_ij = (q_i . k_j) rs over j <= i
             const int j0 = cur.ti * kKT;
-            double s0, s1;
-            dot2<D>(sm.q, tk, qi, sub, s0, s1);
-            if (valid_q && j0 + sub <= i) m = fmax(m, s0 * rs);
-            if (valid_q && j0 + sub + 8 <= i) m = fmax(m, s1 * rs);
-            if (cur.ti == cur.nt - 1) m = max8(m);
-        } else if (cur.ph == 1) {   // l_i and N_i with the exact weights exp(s_ij - m_i)
-            const int j0 = cur.ti * kKT;
-            double s0, s1;
-            dot2<D>(sm.q, tk, qi, sub, s0, s1);
-            const double p0 = valid_q && j0 + sub <= i ? exp(s0 * rs - m) : 0.0;
-            const double p1 = valid_q && j0 + sub + 8 <= i ? exp(s1 * rs - m) : 0.0;
-            sm.pe[qi][sub] = p0;
-            sm.pe[qi][sub + 8] = p1;
-            l += p0;
-            l += p1;
-            __syncthreads();
-#pragma unroll 4
-            for (int kk = 0; kk < kKT; ++kk) {
-                const double p = sm.pe[qi][kk];
+            double se[2], sq[2];
+            score_tile<D, false>(sm.q, tk, tk, mt, nt, lane, se, sq);
 #pragma unroll
-                for (int mm = 0; mm < NM; ++mm) {
-                    const double2 vv = *reinterpret_cast<const double2 *>(&sm.t[buf][1][kk][16 * mm + 2 * sub]);
-                    N[mm].x = fma(p, vv.x, N[mm].x);
-                    N[mm].y = fma(p, vv.y, N[mm].y);
-                }
+            for (int v = 0; v < 2; ++v)
+                if (valid_q && j0 + key0 + v <= i) m = fmax(m, se[v] * rs);
+            if (cur.ti == cur.nt - 1) {
+                m = fmax(m, __shfl_xor_sync(0xffffffffu, m, 1));
+                m = fmax(m, __shfl_xor_sync(0xffffffffu, m, 2));
+                if ((lane & 3) == 0) sm.mx[nt][sq_row] = m;
             }
-            if (cur.ti == cur.nt - 1) l = sum8(l);
+        } else if (cur.ph == 1) {   // l_i and N_i with the exact weights exp(s_ij - m_i)
+            if (cur.ti == 0) m = fmax(sm.mx[0][sq_row], sm.mx[1][sq_row]);
+            const int j0 = cur.ti * kKT;
+            double se[2], sq[2];
+            score_tile<D, false>(sm.q, tk, tk, mt, nt, lane, se, sq);
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+                const double p = valid_q && j0 + key0 + v <= i ? exp(se[v] * rs - m) : 0.0;
+                sm.pe[sq_row][key0 + v] = p;
+                lp += p;
+            }
+            __syncthreads();
+            pv(sm.pe, sm.t[buf][1], N);
+            if (cur.ti == cur.nt - 1) {
+                lp += __shfl_xor_sync(0xffffffffu, lp, 1);
+                lp += __shfl_xor_sync(0xffffffffu, lp, 2);
+                if ((lane & 3) == 0) sm.ls[nt][sq_row] = lp;
+            }
         } else {   // the tag's tokens j <= i at b bits; A and B apart, so exact levels give 0 exactly
             if (cur.ti == 0) {
 #pragma unroll
-                for (int mm = 0; mm < NM; ++mm) {
-                    A[mm] = make_double2(0.0, 0.0);
-                    B[mm] = make_double2(0.0, 0.0);
-                }
-                dl = 0.0;
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int j = 0; j < NTW; ++j) A[a][j][0] = A[a][j][1] = B[a][j][0] = B[a][j][1] = 0.0;
+                dlp = 0.0;
             }
-            double se0, se1, sq0, sq1;
-            dot4<D>(sm.q, tk, sm.t[buf][2], qi, sub, se0, se1, sq0, sq1);
-            const int t0 = sm.tok[buf][sub], t1 = sm.tok[buf][sub + 8];
-            const bool v0 = valid_q && t0 >= 0 && t0 <= i, v1 = valid_q && t1 >= 0 && t1 <= i;
-            const double pe0 = v0 ? exp(se0 * rs - m) : 0.0, pq0 = v0 ? exp(sq0 * rs - m) : 0.0;
-            const double pe1 = v1 ? exp(se1 * rs - m) : 0.0, pq1 = v1 ? exp(sq1 * rs - m) : 0.0;
-            sm.pe[qi][sub] = pe0;
-            sm.pq[qi][sub] = pq0;
-            sm.pe[qi][sub + 8] = pe1;
-            sm.pq[qi][sub + 8] = pq1;
-            dl += pq0 - pe0;
-            dl += pq1 - pe1;
+            double se[2], sq[2];
+            score_tile<D, true>(sm.q, tk, sm.t[buf][2], mt, nt, lane, se, sq);
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+                const int tt = sm.tok[buf][key0 + v];
+                const bool ok = valid_q && tt >= 0 && tt <= i;
+                const double pe = ok ? exp(se[v] * rs - m) : 0.0, pq = ok ? exp(sq[v] * rs - m) : 0.0;
+                sm.pe[sq_row][key0 + v] = pe;
+                sm.pq[sq_row][key0 + v] = pq;
+                dlp += pq - pe;
+            }
             __syncthreads();
-#pragma unroll 2
-            for (int kk = 0; kk < kKT; ++kk) {
-                const double pe = sm.pe[qi][kk], pq = sm.pq[qi][kk];
-#pragma unroll
-                for (int mm = 0; mm < NM; ++mm) {
-                    const double2 vx2 = *reinterpret_cast<const double2 *>(&sm.t[buf][1][kk][16 * mm + 2 * sub]);
-                    const double2 vh = *reinterpret_cast<const double2 *>(&sm.t[buf][3][kk][16 * mm + 2 * sub]);
-                    A[mm].x = fma(pq, vh.x, A[mm].x);
-                    A[mm].y = fma(pq, vh.y, A[mm].y);
-                    B[mm].x = fma(pe, vx2.x, B[mm].x);
-                    B[mm].y = fma(pe, vx2.y, B[mm].y);
-                }
-            }
+            pv(sm.pq, sm.t[buf][3], A);
+            pv(sm.pe, sm.t[buf][1], B);
             if (cur.ti == cur.nt - 1) {   // the pass's squared output differences, summed over the CTA
-                const double dls = sum8(dl);
+                dlp += __shfl_xor_sync(0xffffffffu, dlp, 1);
+                dlp += __shfl_xor_sync(0xffffffffu, dlp, 2);
+                if ((lane & 3) == 0) sm.dl[nt][sq_row] = dlp;
+                __syncthreads();
                 double err = 0.0;
-                if (valid_q) {
-                    const double lq = l + dls;
 #pragma unroll
-                    for (int mm = 0; mm < NM; ++mm) {
-                        const double ex = (N[mm].x + (A[mm].x - B[mm].x)) / lq - N[mm].x / l;
-                        const double ey = (N[mm].y + (A[mm].y - B[mm].y)) / lq - N[mm].y / l;
-                        err += ex * ex;
-                        err += ey * ey;
-                    }
+                for (int mm = 0; mm < 4; ++mm) {
+                    const int row = 8 * mm + (lane >> 2);
+                    if (i0 + row >= d.T) continue;
+                    const double l = sm.ls[0][row] + sm.ls[1][row];
+                    const double lq = l + (sm.dl[0][row] + sm.dl[1][row]);
+#pragma unroll
+                    for (int j = 0; j < NTW; ++j)
+#pragma unroll
+                        for (int v = 0; v < 2; ++v) {
+                            const double e = (N[mm][j][v] + (A[mm][j][v] - B[mm][j][v])) / lq - N[mm][j][v] / l;
+                            err += e * e;
+                        }
                 }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) err += __shfl_xor_sync(0xffffffffu, err, o);
-                if ((tid & 31) == 0) sm.red[tid >> 5] = err;
+                if (lane == 0) sm.red[w] = err;
                 __syncthreads();
                 if (tid == 0) {
                     double s = 0.0;
-                    for (int w = 0; w < kThreads / 32; ++w) s += sm.red[w];
+                    for (int x = 0; x < kThreads / 32; ++x) s += sm.red[x];
                     part[((((static_cast<long long>(lay) * d.R + r) * d.Hq + hq) * d.nqb + qb) * d.ntags + cur.k) * 2 +
                          cur.bi] = s;
                 }
             }
         }
-        __syncthreads();   // this buffer (and sm.pe, sm.red) is free again
+        __syncthreads();   // this buffer (and sm.pe, sm.pq, sm.red) is free again
         if (!more) break;
         cur = nxt;
     }
