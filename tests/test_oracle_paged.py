@@ -146,3 +146,18 @@ def test_paged_layer_matches_units():
             assert np.allclose(out[b, h * G:(h + 1) * G], oracle.attention(Q[b, h * G:(h + 1) * G], Kh, Vh),
                                rtol=1e-13, atol=1e-14)
     assert off == len(img)
+
+
+@pytest.mark.parametrize("tag,L", [(2, 64), (4, 48), (4, 37)])
+def test_uniform_tags_reduce_to_uniform_layers(tag, L):
+    """All tokens INT2 (a whole number of groups) is the per-layer K2V2 cache with
+    per-channel keys; all tokens INT4 is K4V4 with per-token keys.  The paged writer and
+    the per-layer writer are separate code, so their dequantized caches must agree
+    exactly, and so must attention over them."""
+    K, V, tags = rand_seq(L, [tag] * L)
+    _, Kp, Vp = oracle.paged_unit(K, V, tags, D)
+    kmode = 0 if tag == 2 else 1
+    _, Ku, Vu = oracle.unit(K, V, D, tag, tag, kmode)
+    assert np.array_equal(Kp, Ku) and np.array_equal(Vp, Vu)
+    q = to_bf16_bits(rng.standard_normal((2, D)))
+    assert np.array_equal(oracle.attention(q, Kp, Vp), oracle.attention(q, Ku, Vu))
