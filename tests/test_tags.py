@@ -273,3 +273,24 @@ def test_device_distortion_host_checks():
     assert f(*args(fake, fake, 256, tags)) == -4              # workspace too small
     assert f(*args(fake, fake + 16, 1 << 30, tags)) == -4     # workspace not 256-byte aligned
     assert f(*args(fake, fake, 1 << 30, np.full((1, 4), 2, np.int32))) == -1   # tag out of range
+
+
+@pytest.mark.parametrize("L,bits,stride", [(64, 2, 1), (70, 2, 1), (150, 2, 2), (40, 4, 1), (90, 4, 3)])
+def test_tag_quantizer_matches_paged_writer(L, bits, stride):
+    """The distortion oracle's quantizer for one tag is the paged cache's writer for the
+    tokens of that tag (the C oracle, written separately): INT2 keys per channel over
+    consecutive groups of the tag's tokens, values per token, the last count mod 32
+    through the 4-bit path; INT4 per token.  Tokens of the tag every `stride` positions,
+    the others tagged with the other width in the paged cache and left exact here."""
+    rng = np.random.default_rng(L + bits + stride)
+    D = 128
+    K = bf16(rng.standard_normal((L, D)).astype(np.float32) * 3)
+    V = bf16(rng.standard_normal((L, D)).astype(np.float32))
+    toks = np.arange(0, L, stride)
+    ptags = np.full(L, 6 - bits, np.uint8)
+    ptags[toks] = bits
+    _, Kp, Vp = oracle.paged_unit(K, V, ptags, D)
+    Kq, Vq = otags.quantize_tag_tokens(oracle.bf16_bits_to_f32(K), oracle.bf16_bits_to_f32(V), toks, bits)
+    assert np.array_equal(Kq[toks], Kp[toks]) and np.array_equal(Vq[toks], Vp[toks])
+    rest = np.setdiff1d(np.arange(L), toks)
+    assert np.array_equal(Kq[rest], oracle.bf16_bits_to_f32(K)[rest].astype(np.float64))
