@@ -266,6 +266,11 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
         h->page4_bytes = kvq::paged_page4_bytes(D);
         h->n2_cap = static_cast<long long>(std::ceil(f2 * tokens * 1.03 / 32.0)) + d->batch;
         h->n4_main_cap = static_cast<long long>(std::ceil((1.0 - f2) * tokens * 1.03 / 16.0)) + d->batch;
+        // page tables hold int32 indices into the pools
+        if (h->n2_cap >= (1LL << 31) || h->n4_main_cap + 2LL * d->batch >= (1LL << 31)) {
+            delete h;
+            return fail(KVQ_EUNSUPPORTED, "paged plan too large: pool pages exceed int32 page-table indices");
+        }
         h->pend_base = static_cast<int>(h->n4_main_cap);
         h->n4_cap = h->n4_main_cap + 2LL * d->batch;
         h->P_cap = (d->max_ctx + 31) / 32 + (d->max_ctx + 15) / 16 + 1;

@@ -179,6 +179,11 @@ def test_paged_plan_validation(lib):
     assert paged_rc(batch=65) == kvq.KVQ_EUNSUPPORTED
     assert paged_rc(avg_bits=5.0) == kvq.KVQ_EINVAL
     assert paged_rc(avg_bits=1.5) == kvq.KVQ_EINVAL
+    # page tables hold int32 pool indices: pools past 2^31 pages are refused, not wrapped
+    assert paged_rc(batch=64, max_ctx=1 << 20, avg_bits=3.0) == kvq.KVQ_OK
+    assert paged_rc(batch=64, max_ctx=1 << 30, avg_bits=2.0) == kvq.KVQ_EUNSUPPORTED   # INT2 pool
+    assert paged_rc(batch=64, max_ctx=1 << 30, avg_bits=4.0) == kvq.KVQ_EUNSUPPORTED   # INT4 pool
+    assert "int32" in kvq.kvq_last_error()
 
 
 def test_paged_host_checks(lib):
