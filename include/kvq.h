@@ -103,7 +103,7 @@ typedef struct {
     int n_q_heads;      /* multiple of n_kv_heads; G = n_q_heads / n_kv_heads <= 8 */
     int head_dim;       /* 64 or 128 */
     int group;          /* must be 32 */
-    int max_ctx;        /* token capacity per sequence and layer */
+    int max_ctx;        /* token capacity per sequence and layer, at most 2^30 */
     const kvq_layer_cfg *layers;   /* num_layers entries, copied by kvq_plan */
     int paged;          /* 0: per-layer maps (this header's format); 1: INT2/INT4 paged */
     int page_tokens;    /* paged: 16 */

@@ -235,6 +235,7 @@ int kvq_plan(const kvq_plan_desc *d, kvq_handle **out) {
         return fail(KVQ_EINVAL, "num_layers, batch, heads and max_ctx must be positive");
     if (d->n_q_heads % d->n_kv_heads)
         return fail(KVQ_EINVAL, "n_q_heads (%d) must be a multiple of n_kv_heads (%d)", d->n_q_heads, d->n_kv_heads);
+    if (d->max_ctx > (1 << 30)) return fail(KVQ_EUNSUPPORTED, "max_ctx %d above 2^30 tokens", d->max_ctx);
     const int G = d->n_q_heads / d->n_kv_heads;
     if (G > 8) return fail(KVQ_EUNSUPPORTED, "GQA group %d > 8 not supported", G);
     if (d->group != kvq::kGroup) return fail(KVQ_EUNSUPPORTED, "group must be 32 (got %d)", d->group);

@@ -47,6 +47,7 @@ def test_plan_validation(lib):
     assert plan_rc(desc(head_dim=96)) == kvq.KVQ_EUNSUPPORTED
     assert plan_rc(desc(n_q_heads=18)) == kvq.KVQ_EUNSUPPORTED          # G = 9
     assert plan_rc(desc(batch=0)) == kvq.KVQ_EINVAL
+    assert plan_rc(desc(max_ctx=(1 << 31) - 1)) == kvq.KVQ_EUNSUPPORTED   # block counts would wrap
     assert plan_rc(desc(kmodes=[1, 0])) == kvq.KVQ_OK
     assert plan_rc(desc(kmodes=[1, 0], n_q_heads=6)) == kvq.KVQ_EUNSUPPORTED   # per-token keys, G = 3
     d = desc()
