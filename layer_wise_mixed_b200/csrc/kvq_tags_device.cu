@@ -493,6 +493,7 @@ int check_dims(int NL, int R, int Hq, int Hkv, int D, int T, int ntags, CalibDim
         return kvq::host_fail(KVQ_EINVAL, "layers, requests, heads, T and num_tags must be positive");
     if (Hq % Hkv) return kvq::host_fail(KVQ_EINVAL, "n_q_heads must be a multiple of n_kv_heads");
     if (D != 64 && D != 128) return kvq::host_fail(KVQ_EUNSUPPORTED, "head_dim must be 64 or 128 on the device path");
+    if (T > (1 << 30)) return kvq::host_fail(KVQ_EUNSUPPORTED, "T above 2^30 tokens");
     if (Hq > 65535 || R > 65535 || static_cast<long long>(R) * Hkv > 65535)
         return kvq::host_fail(KVQ_EUNSUPPORTED, "too many heads or requests for one launch");
     d = CalibDims{NL, R, Hq, Hkv, D, T, ntags, (T + kQB - 1) / kQB, T / 32 + 1};

@@ -261,6 +261,7 @@ def test_device_distortion_host_checks():
     assert n.value >= 4 * 2 * 2 * 200 * 128 * 8
     assert L.kvq_tag_distortion_workspace_bytes(1, 2, 8, 2, 96, 200, 5, ctypes.byref(n)) == -2   # EUNSUPPORTED
     assert L.kvq_tag_distortion_workspace_bytes(1, 2, 7, 2, 128, 200, 5, ctypes.byref(n)) == -1  # Hq % Hkv
+    assert L.kvq_tag_distortion_workspace_bytes(1, 1, 8, 2, 128, (1 << 31) - 1, 5, ctypes.byref(n)) == -2
     tags = np.zeros((1, 4), np.int32)
     D2, D4, cnt = np.zeros(2), np.zeros(2), np.zeros(2, np.int64)
     p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
