@@ -251,6 +251,8 @@ def test_device_distortion_host_checks():
     """The device entry point's argument checks run on the host before any CUDA call
     (fake device addresses are never touched)."""
     import ctypes
+    from layer_wise_mixed_b200 import build as kbuild
+    kbuild.build()
     L = kvq.load()
     n = ctypes.c_size_t(0)
     assert L.kvq_tag_distortion_workspace_bytes(1, 2, 8, 2, 128, 100, 5, ctypes.byref(n)) == 0
