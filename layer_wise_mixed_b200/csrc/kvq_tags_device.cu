@@ -3,8 +3,8 @@
 // routing).  The definition is the host entry point's (kvq_tag_distortion): tag k's tokens
 // at b bits and every other token exact, causal attention over the calibration prefill,
 // output MSE per query head; max over heads, mean over requests, sum over layers.  All
-// attention arithmetic is fp64 on the CUDA cores, so the results equal the host's up to
-// the order of the sums.
+// attention arithmetic is fp64 (the products on the fp64 tensor cores), so the results
+// equal the host's up to the order of the sums.
 //
 // Per layer:
 //  1. calib_token_kernel: every token's 4-bit per-token K and V (groups of 32 channels),
